@@ -1,0 +1,17 @@
+"""Oracle for TransRetrieval candidate scoring -- TEST INFRASTRUCTURE ONLY.
+
+A plain fp64 CPU restatement of the method, used to check the CUDA path.  Only the
+tests, ``__graft_entry__.smoke()`` and the bench's CPU-baseline / reference leg may
+import it; the product package never does, and shares no code with it.  The only
+module both sides use is ``datagen`` (seeded inputs, none of the method's arithmetic).
+"""
+from .transretrieval import (EPS, FlopCounter, compress_targets, flops_per_candidate_closed_form,
+                             layer_norm, prefill_user, prelu, score_candidates, topk,
+                             weighted_average, weighted_sum)
+from .pipeline import score_request, aggregate_bags
+
+__all__ = [
+    "EPS", "FlopCounter", "compress_targets", "flops_per_candidate_closed_form", "layer_norm",
+    "prefill_user", "prelu", "score_candidates", "topk", "weighted_average", "weighted_sum",
+    "score_request", "aggregate_bags",
+]
