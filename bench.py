@@ -1,0 +1,390 @@
+#!/usr/bin/env python
+"""Throughput of the TransRetrieval candidate-scoring step on B200.
+
+A step is one pass of the whole scoring path over one request of the 128D-5L workload
+(40,000 candidates, L_u = 64, 8 target fields over 4M-row tables):
+  tr_aggregate(user fields) -> tr_prefill_user -> tr_aggregate(target fields)
+  -> tr_compress_targets -> tr_score_candidates.
+``value`` is candidates scored per second over all ranks, with inputs resident in HBM;
+``e2e`` repeats the step with the request's bags copied from pinned host memory and the
+scores copied back inside the timed region.  Requests rotate over several seeded request
+sets and the embedding tables (24.6 GB) are far larger than L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank scores its own requests (weak
+scaling, no collective on the data path); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import datagen  # noqa: E402
+
+WORKLOAD = "128d5l"
+METRIC = "candidates scored/sec at 128D5L, 40k cands/request; % bf16 tensor peak"
+N_REQUEST_SETS = 4
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ algorithmic work
+
+def stack_flops_per_candidate(dims, L_u):
+    """N*(16 D^2 + 4 (L_u+1) D) + 2D (TransRetrieval §3.3 count plus own key/value and head)."""
+    return dims.n_layer * (16 * dims.D ** 2 + 4 * (L_u + 1) * dims.D) + 2 * dims.D
+
+
+def compressor_flops_per_candidate(dims):
+    c = dims.comp_dims
+    return 2 * sum(c[i] * c[i + 1] for i in range(3))
+
+
+def aggregate_bytes(bags, D, elem_bytes, out_bytes):
+    """Rows gathered + keys/weights + offsets/table ids + output rows."""
+    nnz, n_bags = bags.nnz, bags.n_bags
+    return nnz * D * elem_bytes + nnz * 8 + n_bags * 12 + 8 + n_bags * D * out_bytes
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def stop(self):
+        if not self.proc:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = [r for r in self.rows if len(r) >= 7]
+        if not rows:
+            return None
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return float("nan")
+        sm = [num(r[0]) for r in rows]
+        reasons = set()
+        for r in rows:
+            for name, v in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"), r[3:7]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.nanmedian(sm)), "sm_max_mhz": num(rows[0][1]),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU (oracle) leg
+
+def time_oracle(w, P, req, target_seconds=15.0, max_cand=None):
+    """The fp64 oracle on a bounded sample of one request: user side once, then a
+    contiguous slice of candidates.  Returns (candidates/s for the whole request
+    extrapolated from the sample, description, threads)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+
+    threads = max([t.get("num_threads", 1) for t in threadpool_info()] + [1])
+    t0 = time.perf_counter()
+    user_tokens = oracle.aggregate_bags(w, req.user, "user")
+    K, V = oracle.prefill_user(P, w.dims.n_head, user_tokens, req.domain)
+    t_user = time.perf_counter() - t0
+
+    def cand_time(n):
+        t = time.perf_counter()
+        oracle.score_request_candidates(w, P, req, np.arange(n), K, V)
+        return time.perf_counter() - t
+    n = 200
+    dt = cand_time(n)
+    per = dt / n
+    n2 = int(min(req.n_cand if max_cand is None else max_cand, max(n, target_seconds / max(per, 1e-9))))
+    if n2 > n:
+        dt = cand_time(n2)
+        n = n2
+        per = dt / n
+    total = t_user + per * req.n_cand
+    rate = req.n_cand / total
+    desc = (f"oracle (fp64 numpy) on {n} of {req.n_cand} candidates of one {w.name} request plus its user side "
+            f"({t_user:.2f} s user side, {dt:.2f} s candidates); rate = n_cand / (t_user + n_cand * t_cand/n)")
+    return rate, desc, threads, t_user + dt
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the oracle as it stands on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    w = datagen.WORKLOADS[WORKLOAD]
+    P = datagen.workload_params(w)
+    req = datagen.make_requests(w)[0]
+    # size each step to a bounded sample so W+K steps stay within a few minutes
+    budget = max(4.0, 150.0 / max(1, args.steps + args.warmup))
+    vals = []
+    for i in range(args.warmup + args.steps):
+        rate, desc, threads, secs = time_oracle(w, P, req, target_seconds=budget)
+        if i >= args.warmup:
+            vals.append(rate)
+    v = float(np.median(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "candidates/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.n_cand_per_request / v * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "128D-5L, 1 request x 40,000 candidates, L_u=64, 8 target fields, 4M-row tables",
+                   "n_cand": w.n_cand_per_request},
+        "cpu_baseline": {"value": v, "unit": "candidates/s", "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": v, "unit": "candidates/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU leg
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from transformer_candidate_scoring_b200 import api, build
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = datagen.WORKLOADS[WORKLOAD]
+    dims = w.dims
+    # distinct request sets per rank and per step (seeded)
+    sets = [datagen.make_requests(w, seed=w.seed * 1000 + rank * 100 + s) for s in range(N_REQUEST_SETS)]
+    dw = DeviceWorkload(w, device=dev, reqs=sets[0])
+    dsets = []
+    for reqs in sets:
+        dw.set_requests(reqs)
+        dsets.append((dw.user_bags, dw.target_bags, reqs))
+    stream = torch.cuda.current_stream()
+
+    def use(i):
+        ub, tb, reqs = dsets[i % N_REQUEST_SETS]
+        dw.user_bags, dw.target_bags, dw.reqs = ub, tb, reqs
+        dw.L_u = [r.L_u for r in reqs]
+        dw.domain = [r.domain for r in reqs]
+
+    stage_names = ["user_side", "target_aggregate", "compress", "score"]
+
+    def step(i, events=None):
+        use(i)
+        if events is not None:
+            events[0].record(stream)
+        dw.user_side()
+        if events is not None:
+            events[1].record(stream)
+        dw.target_aggregate()
+        if events is not None:
+            events[2].record(stream)
+        dw.compress()
+        if events is not None:
+            events[3].record(stream)
+        dw.score()
+        if events is not None:
+            events[4].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if api.sync_status() != 0:
+        raise RuntimeError("device reported an out-of-range key during warm-up")
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    launches0 = api.kernel_launches()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = api.kernel_launches() - launches0
+    clk = clocks.stop()
+    elapsed = t0.elapsed_time(t1) / 1e3
+    stage_ms = {n: float(np.mean([ev[i][k].elapsed_time(ev[i][k + 1]) for i in range(args.steps)]))
+                for k, n in enumerate(stage_names)}
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+    n_cand = dw.n_cand
+    value = n_cand * args.steps * world / elapsed
+
+    # ---- end to end: host bags in, scores out, through the same calls
+    host_sets = []
+    for ub, tb, reqs in dsets:
+        hu = [DeviceBags(*(x.cpu().pin_memory() for x in (b.offsets, b.keys, b.weights, b.bag_table))) for b in ub]
+        ht = DeviceBags(*(x.cpu().pin_memory() for x in (tb.offsets, tb.keys, tb.weights, tb.bag_table)))
+        host_sets.append((hu, ht))
+    h2d = sum(x.numel() * x.element_size() for b in host_sets[0][0] for x in (b.offsets, b.keys, b.weights, b.bag_table))
+    h2d += sum(x.numel() * x.element_size() for x in (host_sets[0][1].offsets, host_sets[0][1].keys,
+                                                        host_sets[0][1].weights, host_sets[0][1].bag_table))
+    host_scores = torch.empty(n_cand, dtype=torch.float32).pin_memory()
+    d2h = host_scores.numel() * 4
+
+    def e2e_step(i):
+        hu, ht = host_sets[i % N_REQUEST_SETS]
+        ub, tb, reqs = dsets[i % N_REQUEST_SETS]
+        for h, d in zip(hu + [ht], ub + [tb]):
+            for hs, ds in zip((h.offsets, h.keys, h.weights, h.bag_table), (d.offsets, d.keys, d.weights, d.bag_table)):
+                ds.copy_(hs, non_blocking=True)
+        step(i)
+        host_scores.copy_(dw.scores, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_elapsed = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        t = torch.tensor([e2e_elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_elapsed = float(t.item())
+    e2e_value = n_cand * args.steps * world / e2e_elapsed
+
+    # ---- rooflines of the stages
+    peaks, peak_kind = load_peaks()
+    L_u = dw.L_u[0]
+    fl_stack = stack_flops_per_candidate(dims, L_u) * n_cand
+    fl_comp = compressor_flops_per_candidate(dims) * n_cand
+    tb_host = sets[0][0].target
+    agg_bytes = aggregate_bytes(tb_host, dims.D, 2, 2)
+    stage_roof = {
+        "score": {"bound": "tensor", "achieved": fl_stack / (stage_ms["score"] / 1e3) / 1e12,
+                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"},
+        "compress": {"bound": "tensor", "achieved": fl_comp / (stage_ms["compress"] / 1e3) / 1e12,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"},
+        "target_aggregate": {"bound": "hbm", "achieved": agg_bytes / (stage_ms["target_aggregate"] / 1e3) / 1e9,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s"},
+    }
+    for r in stage_roof.values():
+        r["frac"] = r["achieved"] / r["peak"]
+        r["peak_source"] = peak_kind
+    dominant = max(("score", "compress", "target_aggregate"), key=lambda k: stage_ms[k])
+    roof = dict(stage_roof[dominant])
+    roof["kernel"] = dominant
+    roof["traffic"] = None
+
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        rate, desc, threads, secs = time_oracle(w, dw.params, sets[0][0], target_seconds=args.cpu_seconds)
+        cpu = {"value": rate, "unit": "candidates/s", "cores": threads, "kind": "oracle", "sample": desc}
+    line = {
+        "metric": METRIC, "value": value, "unit": "candidates/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "128D-5L, 1 request x 40,000 candidates per GPU, L_u=64, 8 target fields, "
+                               "16+8 tables of 4M rows (24.6 GB bf16)",
+                   "n_cand_per_gpu": n_cand, "L_u": L_u, "request_sets": N_REQUEST_SETS,
+                   "l2": "inputs larger than L2: tables 24.6 GB, uniform target keys, rotating request sets",
+                   "parallelism": f"candidate shards, {world} GPU(s), no collective"},
+        "roofline": roof,
+        "stages": {k: {"ms": stage_ms[k], **({kk: vv for kk, vv in stage_roof[k].items()} if k in stage_roof else {})}
+                   for k in stage_names},
+        "pct_bf16_peak_score_kernel": stage_roof["score"]["frac"] * 100,
+        "e2e": {"value": e2e_value, "unit": "candidates/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

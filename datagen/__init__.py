@@ -12,6 +12,7 @@ from .configs import WORKLOADS, ModelDims, Workload, scaled
 from .bags import Bags, Request, make_requests, scale_weights
 from .params import Params, make_params, workload_params
 from .tables import fill_table_device, table_rows_host, f32_to_bf16_rne
+from .stage_inputs import rand_matrix
 
 
 def user_table_id(w: Workload, t: int) -> int:
@@ -47,5 +48,5 @@ def compact_rows(w: Workload, bags: Bags, side: str):
 __all__ = [
     "WORKLOADS", "ModelDims", "Workload", "scaled", "Bags", "Request", "make_requests",
     "scale_weights", "Params", "make_params", "workload_params", "fill_table_device",
-    "table_rows_host", "f32_to_bf16_rne", "user_table_id", "target_table_id", "compact_rows",
+    "table_rows_host", "f32_to_bf16_rne", "rand_matrix", "user_table_id", "target_table_id", "compact_rows",
 ]

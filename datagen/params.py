@@ -22,7 +22,11 @@ from .tables import f32_to_bf16_rne
 Params = Dict[str, np.ndarray]
 
 
-def make_params(dims: ModelDims, seed: int) -> Params:
+def make_params(dims: ModelDims, seed: int, init: str = "paper") -> Params:
+    """``init="paper"`` is the N(0, 0.02) recipe above.  ``init="wide"`` draws matrices
+    from N(0, 1/fan_in), gains from U(0.5, 1.5), slopes from U(-0.5, 0.5) and the other
+    vectors from N(0, 0.3): attention is then far from uniform and candidates differ
+    strongly, which makes kernel-level comparisons sharper."""
     rng = np.random.default_rng(np.random.SeedSequence(seed).spawn(4)[0])
     D, H = dims.D, dims.ffn_hidden
     P: Params = {}
@@ -56,6 +60,19 @@ def make_params(dims: ModelDims, seed: int) -> Params:
             P[f"c{i}.prelu"] = 0.25 + nrm(c[i + 1])
             P[f"c{i}.ln_g"] = 1.0 + nrm(c[i + 1])
             P[f"c{i}.ln_b"] = nrm(c[i + 1])
+    if init == "wide":
+        wr = np.random.default_rng(seed + 7919)
+        for k, v in P.items():
+            if v.ndim == 2 and k != "domain_emb":
+                P[k] = wr.normal(0.0, 1.0 / np.sqrt(v.shape[0]), size=v.shape)
+            elif k.endswith("_g"):
+                P[k] = wr.uniform(0.5, 1.5, size=v.shape)
+            elif k.endswith("prelu"):
+                P[k] = wr.uniform(-0.5, 0.5, size=v.shape)
+            else:
+                P[k] = wr.normal(0.0, 0.3, size=v.shape)
+    elif init != "paper":
+        raise ValueError(init)
     for k in P:
         v = P[k].astype(np.float32)
         P[k] = f32_to_bf16_rne(v).reshape(v.shape) if dims.dtype == "bf16" else v

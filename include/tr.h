@@ -1,0 +1,203 @@
+/*
+ * tr.h -- C ABI of the TransRetrieval candidate-scoring library (libtr.so).
+ *
+ * The four calls of the scoring path, from "TransRetrieval: Scaling Up Transformer-Based
+ * Retrieval for Industrial Recommendation":
+ *   tr_aggregate         weighted-average aggregation of (key, weight) fields      (§3.2)
+ *   tr_prefill_user      user tokens + domain embedding through the N-layer Pre-LN
+ *                        Transformer, writing the per-layer user K/V cache          (§3.1, §3.4)
+ *   tr_compress_targets  3-layer MLP target compressor, F*D -> D                    (§3.3)
+ *   tr_score_candidates  single-token candidates through the same layer stack over
+ *                        the broadcast user K/V, then the linear head; candidates of
+ *                        several requests packed in one call, each isolated to its
+ *                        own request                       (§3.3, deployment section)
+ *
+ * Conventions
+ *  - Every call returns tr_status.  TR_OK is 0.  On failure, tr_last_error() returns a
+ *    thread-local message describing the first problem found.
+ *  - Arguments are validated on the host before anything is launched; an invalid call
+ *    launches nothing and writes nothing.
+ *  - Compute calls are asynchronous on the caller's CUDA stream (tr_stream is a
+ *    cudaStream_t; NULL means the legacy default stream).  Errors that only the device
+ *    can see (a key outside its table) do not stop the kernel: the offending key is
+ *    skipped and a device status word is set; tr_sync_status() reports it.
+ *  - The caller owns every input/output device buffer.  The library owns the model
+ *    handle (its repacked weights) and, per device, an internal workspace used by some
+ *    kernels; both are released by tr_model_destroy() / at process exit.
+ *  - Row-major layouts unless stated; "[a][b]" means a rows of b contiguous elements.
+ *  - dtype TR_F32 models compute in fp32 throughout.  TR_BF16 models store tables,
+ *    weights, target-field tokens and candidate tokens in bf16 and accumulate in fp32.
+ */
+#ifndef TR_H
+#define TR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int tr_status;
+#define TR_OK 0
+#define TR_ERR_INVALID_ARG 1  /* bad pointer, size, dtype or index; nothing launched        */
+#define TR_ERR_UNSUPPORTED 2  /* valid but not implemented (e.g. a model size)              */
+#define TR_ERR_CUDA 3         /* a CUDA runtime call failed; message has the CUDA error      */
+#define TR_ERR_KEY_RANGE 4    /* device saw a key >= its table's rows (that key was skipped) */
+#define TR_ERR_TIMEOUT 5      /* tr_sync_status() deadline passed before the stream drained */
+#define TR_ERR_NOMEM 6        /* device allocation for the model or workspace failed         */
+
+typedef enum { TR_F32 = 0, TR_BF16 = 1 } tr_dtype;
+
+typedef void* tr_stream; /* cudaStream_t */
+
+#define TR_MAX_TABLES 64     /* tables per tr_aggregate call            */
+#define TR_MAX_REQUESTS 64   /* requests packed in one score call      */
+#define TR_MAX_LU 256        /* user tokens per request                */
+
+/* Model sizes (TransRetrieval §4.1 xD-yL notation). */
+typedef struct {
+  int D;               /* token width; multiple of 16, <= 128                        */
+  int n_layer;         /* Transformer layers, 1..16                                  */
+  int n_head;          /* heads; d_h = D / n_head must be 16                         */
+  int ffn_hidden;      /* FFN hidden width (2*D for the paper's FLOP count)          */
+  int n_target_fields; /* F                                                          */
+  int comp_dims[4];    /* compressor F*D -> c1 -> c2 -> D; comp_dims[0] == F*D,
+                          comp_dims[3] == D                                          */
+  int n_domains;       /* domain embeddings s_d                                      */
+  tr_dtype dtype;
+} tr_model_desc;
+
+/* One layer's parameters: HOST pointers to fp32 arrays.  Linear maps are W[in][out]
+ * with y = x W + b.  For TR_BF16 models every value must be exactly representable in
+ * bf16 (it is converted without rounding checks). */
+typedef struct {
+  const float *ln1_g, *ln1_b;             /* [D]                         */
+  const float *Wq, *bq, *Wk, *bk, *Wv, *bv; /* [D][D], [D]                 */
+  const float *Wo, *bo;                   /* [D][D], [D]                  */
+  const float *ln2_g, *ln2_b;             /* [D]                          */
+  const float *W1, *b1;                   /* [D][ffn_hidden], [ffn_hidden] */
+  const float *W2, *b2;                   /* [ffn_hidden][D], [D]         */
+} tr_layer_weights;
+
+typedef struct {
+  const float* domain_emb;          /* [n_domains][D]                                */
+  const tr_layer_weights* layers;   /* host array [n_layer]                          */
+  const float *lnf_g, *lnf_b;       /* [D] final LayerNorm                           */
+  const float* w_head;              /* [D]                                           */
+  float b_head;
+  const float* comp_W[3];           /* [comp_dims[i]][comp_dims[i+1]]                */
+  const float* comp_b[3];           /* [comp_dims[i+1]]                              */
+  const float* comp_prelu[2];       /* [comp_dims[i+1]] PReLU slopes                 */
+  const float* comp_ln_g[2];        /* [comp_dims[i+1]]                              */
+  const float* comp_ln_b[2];
+} tr_model_weights;
+
+typedef struct tr_model tr_model;
+
+/* Embedding table: DEVICE pointer to [n_rows][D] values of type dtype. */
+typedef struct {
+  const void* data;
+  int64_t n_rows;
+  tr_dtype dtype;
+} tr_table;
+
+const char* tr_last_error(void);
+
+/* Copies and repacks the weights into device memory owned by the returned handle.
+ * Uses the current CUDA device.  Synchronous. */
+tr_status tr_model_create(const tr_model_desc* desc, const tr_model_weights* w, tr_model** out);
+void tr_model_destroy(tr_model* m);
+
+/*
+ * Weighted-average aggregation (TransRetrieval §3.2): for every bag b
+ *     out[b] = sum_{i in bag b} weights[i] * table[bag_table[b]][keys[i]] / sum_{i in b} weights[i]
+ * accumulated in fp32.  A bag with no keys, or whose weights sum to exactly 0, yields the
+ * zero vector.  Duplicate keys count once per occurrence.
+ *   tables     HOST array [n_tables] (<= TR_MAX_TABLES); all tables share one dtype
+ *   bag_table  DEVICE int32 [n_bags], each in [0, n_tables)  (validated on the device:
+ *              an out-of-range entry zeroes the bag and sets TR_ERR_KEY_RANGE)
+ *   offsets    DEVICE int64 [n_bags + 1], non-decreasing, offsets[0] = 0
+ *   keys       DEVICE int32 [offsets[n_bags]]; a key >= n_rows (or < 0) is skipped and
+ *              sets the device status word (TR_ERR_KEY_RANGE via tr_sync_status)
+ *   weights    DEVICE fp32  [offsets[n_bags]]
+ *   out        DEVICE [n_bags][D] of out_dtype.  For the compressor input, bag
+ *              b = c*F + f gives out viewed as [n_cand][F*D].
+ * D must be a multiple of 8 and <= 512.  n_bags = 0 is a no-op.
+ */
+tr_status tr_aggregate(const tr_table* tables, int n_tables, const int32_t* bag_table,
+                       const int64_t* offsets, const int32_t* keys, const float* weights,
+                       int64_t n_bags, int D, tr_dtype out_dtype, void* out, tr_stream stream);
+
+/*
+ * Bytes of one request's user K/V cache for L_u user tokens (0 <= L_u <= TR_MAX_LU).
+ * Layout (opaque to most callers; tests decode it):
+ *   TR_F32 model : [n_layer][2][L_u][D] fp32, K then V, row-major.
+ *   TR_BF16 model: per layer a K image then a V image, bf16, in the tensor-core operand
+ *   layout.  With Lp = L_u rounded up to 16 (rows >= L_u are zero) and 8x8 "core
+ *   matrices" of 128 contiguous bytes (8 rows of 8 consecutive elements):
+ *     K image  [Lp x D]: element (j, d) at core (d/8)*(Lp/8) + j/8, within it (j%8)*8 + d%8
+ *     V image  [D x Lp] (V transposed): element (d, j) at core (j/8)*(D/8) + d/8,
+ *              within it (d%8)*8 + j%8
+ *   each image is Lp*D*2 bytes; layer l starts at l * 2*Lp*D*2 bytes.
+ */
+size_t tr_kv_cache_bytes(const tr_model* m, int L_u);
+
+/*
+ * User side of one request (TransRetrieval §3.1 stages (3)-(4), §3.4): x = user_tokens
+ * + s_domain, then for each layer a Pre-LN attention block (every user token attends to
+ * every user token) and a Pre-LN ReLU FFN block; the layer's K = LN1(x) Wk + bk and
+ * V = LN1(x) Wv + bv are written to kv (layout above).
+ *   user_tokens DEVICE fp32 [L_u][D];  kv DEVICE buffer of tr_kv_cache_bytes(m, L_u).
+ * L_u = 0 writes nothing.
+ */
+tr_status tr_prefill_user(const tr_model* m, const float* user_tokens, int L_u, int domain,
+                          void* kv, tr_stream stream);
+
+/*
+ * Target compressor (TransRetrieval §3.3): t = W3 g2(W2 g1(W1 x + b1) + b2) + b3 with
+ * g_i(z) = LayerNorm_i(PReLU_i(z)).
+ *   x      DEVICE [n][comp_dims[0]] of the model dtype (the concatenated field tokens)
+ *   tokens DEVICE [n][D] of the model dtype.
+ */
+tr_status tr_compress_targets(const tr_model* m, const void* x, int64_t n, void* tokens,
+                              tr_stream stream);
+
+/*
+ * Score packed candidates (TransRetrieval §3.3 and deployment "Hardware-aware inference
+ * optimization").  Candidates of request r are rows req_offsets[r] .. req_offsets[r+1]-1;
+ * each runs as one token y = t + s_domain[r] through every layer: Pre-LN multi-head
+ * attention over its request's L_u cached user keys/values plus its own key/value,
+ * then the Pre-LN ReLU FFN; score = w_head . LayerNorm_f(y) + b_head.  A candidate never
+ * sees another candidate or another request's cache.
+ *   tokens      DEVICE [n][D] of the model dtype
+ *   req_offsets HOST int64 [R+1], req_offsets[0] = 0, non-decreasing, req_offsets[R] = n
+ *   kv          HOST array [R] of DEVICE pointers (caches written by tr_prefill_user)
+ *   L_u, domain HOST int32 [R]
+ *   scores      DEVICE fp32 [n]
+ * 1 <= R <= TR_MAX_REQUESTS.
+ */
+tr_status tr_score_candidates(const tr_model* m, const void* tokens, int64_t n,
+                              const int64_t* req_offsets, const void* const* kv,
+                              const int32_t* L_u, const int32_t* domain, int R, float* scores,
+                              tr_stream stream);
+
+/*
+ * Waits for `stream` (polling, up to timeout_ms; <= 0 means no limit), then reads and
+ * clears this device's status word.  Returns TR_ERR_TIMEOUT if the stream did not drain
+ * in time (the status word is left untouched), TR_ERR_KEY_RANGE if a kernel reported an
+ * out-of-range key or table index since the last call, else TR_OK.
+ */
+tr_status tr_sync_status(tr_stream stream, int timeout_ms);
+
+/* Library version, for diagnostics. */
+const char* tr_version(void);
+
+/* Number of kernels this library has launched in this process (all devices, all
+ * threads); a diagnostic for counting launches inside a timed region. */
+unsigned long long tr_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TR_H */

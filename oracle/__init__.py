@@ -8,10 +8,10 @@ module both sides use is ``datagen`` (seeded inputs, none of the method's arithm
 from .transretrieval import (EPS, FlopCounter, compress_targets, flops_per_candidate_closed_form,
                              layer_norm, prefill_user, prelu, score_candidates, topk,
                              weighted_average, weighted_sum)
-from .pipeline import score_request, aggregate_bags
+from .pipeline import aggregate_bags, score_request, score_request_candidates
 
 __all__ = [
     "EPS", "FlopCounter", "compress_targets", "flops_per_candidate_closed_form", "layer_norm",
     "prefill_user", "prelu", "score_candidates", "topk", "weighted_average", "weighted_sum",
-    "score_request", "aggregate_bags",
+    "score_request", "score_request_candidates", "aggregate_bags",
 ]

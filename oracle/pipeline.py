@@ -28,6 +28,30 @@ class RequestResult:
     scores: np.ndarray          # [n]
 
 
+def _select_candidates(req: "datagen.Request", cand: np.ndarray, F: int) -> "datagen.Bags":
+    tb = req.target
+    cand = np.asarray(cand, dtype=np.int64)
+    bag_ids = (cand[:, None] * F + np.arange(F)[None, :]).reshape(-1)
+    counts = np.diff(tb.offsets)[bag_ids]
+    off = np.zeros(len(bag_ids) + 1, dtype=np.int64)
+    np.cumsum(counts, out=off[1:])
+    starts = tb.offsets[bag_ids]
+    idx = (np.repeat(starts - off[:-1], counts) + np.arange(int(off[-1]))).astype(np.int64)
+    return datagen.Bags(off, tb.keys[idx], tb.weights[idx], tb.bag_table[bag_ids])
+
+
+def score_request_candidates(w: "datagen.Workload", P, req: "datagen.Request", cand: np.ndarray,
+                             K: np.ndarray, V: np.ndarray):
+    """Candidate side of one request given its user K/V: aggregate the selected
+    candidates' target fields, compress, score.  Returns (X, tokens, scores)."""
+    dims = w.dims
+    F = dims.n_target_fields
+    tb = _select_candidates(req, cand, F)
+    X = aggregate_bags(w, tb, "target").reshape(-1, F * dims.D)
+    tokens = compress_targets(P, X)
+    return X, tokens, score_candidates(P, dims.n_head, tokens, K, V, req.domain)
+
+
 def score_request(w: "datagen.Workload", P, req: "datagen.Request",
                   cand: np.ndarray | None = None) -> RequestResult:
     """(1) weighted-average aggregation of user and target fields, (2) target compression,
@@ -35,20 +59,9 @@ def score_request(w: "datagen.Workload", P, req: "datagen.Request",
     and reused by every candidate; then the linear head.  ``cand`` restricts the
     candidates scored (indices into the request's candidates)."""
     dims = w.dims
-    F = dims.n_target_fields
     user_tokens = aggregate_bags(w, req.user, "user")
     K, V = prefill_user(P, dims.n_head, user_tokens, req.domain)
-    tb = req.target
-    if cand is not None:
-        cand = np.asarray(cand, dtype=np.int64)
-        bag_ids = (cand[:, None] * F + np.arange(F)[None, :]).reshape(-1)
-        counts = np.diff(tb.offsets)[bag_ids]
-        off = np.zeros(len(bag_ids) + 1, dtype=np.int64)
-        np.cumsum(counts, out=off[1:])
-        idx = np.concatenate([np.arange(tb.offsets[b], tb.offsets[b + 1]) for b in bag_ids]) \
-            if len(bag_ids) else np.zeros(0, dtype=np.int64)
-        tb = datagen.Bags(off, tb.keys[idx], tb.weights[idx], tb.bag_table[bag_ids])
-    X = aggregate_bags(w, tb, "target").reshape(-1, F * dims.D)
-    tokens = compress_targets(P, X)
-    scores = score_candidates(P, dims.n_head, tokens, K, V, req.domain)
+    if cand is None:
+        cand = np.arange(req.n_cand)
+    X, tokens, scores = score_request_candidates(w, P, req, cand, K, V)
     return RequestResult(user_tokens, K, V, X, tokens, scores)

@@ -1,0 +1,56 @@
+"""The C-ABI library loads, exports every symbol include/tr.h declares, and rejects bad
+arguments on the host before touching a GPU (these calls launch nothing)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(tr_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from transformer_candidate_scoring_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_four_calls():
+    names = declared_functions()
+    for f in ("tr_aggregate", "tr_prefill_user", "tr_compress_targets", "tr_score_candidates"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_host_validation_without_gpu(lib):
+    from transformer_candidate_scoring_b200 import _lib as L
+    assert lib.tr_version().startswith(b"libtr")
+    assert lib.tr_kv_cache_bytes(None, 5) == 0
+    # n_bags == 0 is a no-op; bad table count is rejected before any launch
+    assert lib.tr_aggregate(None, 0, None, None, None, None, 0, 128, 1, None, None) == L.TR_OK
+    t = (L.Table * 1)(L.Table(0, 10, 1))
+    assert lib.tr_aggregate(t, 0, None, None, None, None, 5, 128, 1, None, None) == L.TR_ERR_INVALID_ARG
+    assert b"n_tables" in lib.tr_last_error()
+    assert lib.tr_aggregate(t, 1, None, None, None, None, 5, 128, 1, None, None) == L.TR_ERR_INVALID_ARG
+    # unsupported model sizes are refused before allocation
+    d = L.ModelDesc(96, 2, 4, 192, 8, (C.c_int * 4)(768, 384, 192, 96), 2, 1)   # d_h = 24
+    h = C.c_void_p()
+    assert lib.tr_model_create(C.byref(d), None, C.byref(h)) == L.TR_ERR_UNSUPPORTED
+    d = L.ModelDesc(64, 2, 4, 128, 8, (C.c_int * 4)(500, 256, 128, 64), 2, 1)    # comp_dims[0] != F*D
+    assert lib.tr_model_create(C.byref(d), None, C.byref(h)) == L.TR_ERR_INVALID_ARG
+    assert lib.tr_score_candidates(None, None, 0, None, None, None, None, 1, None, None) == L.TR_ERR_INVALID_ARG

@@ -1,0 +1,315 @@
+"""GPU parity: every stage of libtr against the fp64 oracle on the same seeded inputs.
+
+Inputs come from ``datagen`` only (tables, bags, stand-alone tokens); the oracle never
+reads anything the CUDA path produced.  Tolerances: fp32 models 1e-4, bf16 models 2e-2,
+as max |g - r| / max(|r|, rms(r)) (tests/common.py).
+"""
+import numpy as np
+import pytest
+import torch
+
+import datagen
+import oracle
+from common import rel_err, topk_agrees
+from kvdecode import decode_kv
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib():
+    from transformer_candidate_scoring_b200 import build
+    build.build()
+    assert torch.cuda.is_available()
+    torch.cuda.init()
+    yield
+
+
+def tr():
+    import transformer_candidate_scoring_b200 as t
+    return t
+
+
+def dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    return t.to(dtype) if dtype is not None else t
+
+
+def tdt(name):
+    return torch.bfloat16 if name == "bf16" else torch.float32
+
+
+def dims_of(name):
+    return datagen.WORKLOADS[name].dims
+
+
+# ---------------------------------------------------------------- aggregation (§3.2)
+
+def _bags(rng, n_bags, max_nf, n_rows, n_tables, empty_frac=0.1):
+    counts = rng.integers(1, max_nf + 1, size=n_bags)
+    counts[rng.random(n_bags) < empty_frac] = 0
+    off = np.zeros(n_bags + 1, np.int64)
+    np.cumsum(counts, out=off[1:])
+    keys = rng.integers(0, n_rows, size=int(off[-1])).astype(np.int32)
+    w = rng.uniform(0.1, 1.0, size=len(keys)).astype(np.float32)
+    tab = rng.integers(0, n_tables, size=n_bags).astype(np.int32)
+    return datagen.Bags(off, keys, w, tab)
+
+
+def _tables(seed, n_tables, rows, D, dt):
+    ts = []
+    for t in range(n_tables):
+        x = torch.empty(rows, D, dtype=tdt(dt), device="cuda")
+        datagen.fill_table_device(x, seed, t)
+        ts.append(x)
+    return ts
+
+
+def _oracle_agg(seed, bags, rows, D, dt):
+    tab_of_key = np.repeat(bags.bag_table.astype(np.int64), np.diff(bags.offsets))
+    out_rows = np.zeros((len(bags.keys), D))
+    for t in np.unique(tab_of_key):
+        sel = tab_of_key == t
+        out_rows[sel] = datagen.table_rows_host(seed, int(t), bags.keys[sel], D, dt)
+    return oracle.weighted_average(out_rows, bags.offsets, np.arange(len(bags.keys)), bags.weights)
+
+
+def _run_agg(tables, bags, D, out_dtype):
+    out = torch.empty(bags.n_bags, D, dtype=out_dtype, device="cuda")
+    tr().aggregate(tables, dev(bags.bag_table), dev(bags.offsets), dev(bags.keys), dev(bags.weights), out)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("dt,D", [("f32", 32), ("bf16", 64), ("bf16", 128), ("f32", 128), ("bf16", 32)])
+@pytest.mark.parametrize("out_dt", ["f32", "bf16"])
+def test_aggregate_parity(dt, D, out_dt):
+    rng = np.random.default_rng(D)
+    rows = 5000
+    tables = _tables(11, 3, rows, D, dt)
+    bags = _bags(rng, 1237, 100, rows, 3)
+    got = _run_agg(tables, bags, D, tdt(out_dt)).double().cpu().numpy()
+    ref = _oracle_agg(11, bags, rows, D, dt)
+    # fp32 accumulation error scales with the summands (table values), not with the
+    # possibly cancelling result; bf16 output adds one rounding of the result.
+    scale = float(np.abs(ref).max())
+    err = np.abs(got - ref)
+    if out_dt == "f32":
+        assert np.all(err <= 1e-6 * scale), float(err.max() / scale)
+    else:
+        assert np.all(err <= 2.0 ** -8 * np.abs(ref) + 1e-6 * scale), rel_err(got, ref)
+    empty = np.diff(bags.offsets) == 0
+    assert np.all(got[empty] == 0)
+    assert tr().sync_status() == 0
+
+
+def test_aggregate_scale_invariance_is_bitexact():
+    rng = np.random.default_rng(5)
+    tables = _tables(3, 2, 3000, 128, "bf16")
+    bags = _bags(rng, 500, 40, 3000, 2)
+    a = _run_agg(tables, bags, 128, torch.float32)
+    for c in (4.0, 0.125, 1024.0):
+        b = _run_agg(tables, datagen.scale_weights(bags, c), 128, torch.float32)
+        assert torch.equal(a, b)
+
+
+def test_aggregate_single_key_returns_row_exactly():
+    rng = np.random.default_rng(6)
+    tables = _tables(4, 1, 2000, 128, "bf16")
+    keys = rng.integers(0, 2000, size=300).astype(np.int32)
+    bags = datagen.Bags(np.arange(301, dtype=np.int64), keys, rng.uniform(0.1, 1, 300).astype(np.float32),
+                        np.zeros(300, np.int32))
+    got = _run_agg(tables, bags, 128, torch.float32)
+    assert torch.equal(got, tables[0][torch.from_numpy(keys).long().cuda()].float())
+
+
+def test_aggregate_out_of_range_key_is_skipped_and_reported():
+    rng = np.random.default_rng(7)
+    tables = _tables(5, 1, 1000, 64, "bf16")
+    bags = _bags(rng, 50, 10, 1000, 1, empty_frac=0.0)
+    bad = bags.keys.copy()
+    bad[3] = 1000           # one past the end
+    bad[7] = -5
+    got = _run_agg(tables, datagen.Bags(bags.offsets, bad, bags.weights, bags.bag_table), 64, torch.float32)
+    assert tr().sync_status() == 4
+    assert tr().sync_status() == 0          # the word is cleared by the read
+    keep = np.ones(len(bad), bool)
+    keep[[3, 7]] = False
+    cnt = np.array([keep[bags.offsets[b]:bags.offsets[b + 1]].sum() for b in range(50)])
+    off = np.zeros(51, np.int64)
+    np.cumsum(cnt, out=off[1:])
+    ref = _oracle_agg(5, datagen.Bags(off, bags.keys[keep], bags.weights[keep], bags.bag_table), 1000, 64, "bf16")
+    np.testing.assert_allclose(got.double().cpu().numpy(), ref, rtol=1e-5, atol=1e-7)
+
+
+# ---------------------------------------------------------------- prefill (§3.1, §3.4)
+
+@pytest.mark.parametrize("name,L_u,init", [("tiny", 8, "paper"), ("tiny", 1, "wide"), ("64d3l", 32, "wide"),
+                                           ("128d5l", 64, "paper"), ("128d5l", 64, "wide"),
+                                           ("128d5l", 128, "wide"), ("128d5l", 37, "wide"),
+                                           ("128d5l", 256, "wide")])
+def test_prefill_parity(name, L_u, init):
+    dims = dims_of(name)
+    P = datagen.make_params(dims, 3, init)
+    m = tr().Model(dims, P)
+    U = datagen.rand_matrix(21, (L_u, dims.D), 0.3 if init == "wide" else 0.01, "f32")
+    kv = torch.zeros(tr().kv_cache_bytes(m, L_u), dtype=torch.uint8, device="cuda")
+    tr().prefill_user(m, dev(U), L_u, 1, kv)
+    torch.cuda.synchronize()
+    dec = decode_kv(kv.cpu().numpy(), dims.dtype, dims.n_layer, L_u, dims.D)
+    K, V = oracle.prefill_user(P, dims.n_head, U, 1)
+    for l in range(dims.n_layer):
+        assert rel_err(dec[0][l], K[l]) < TOL[dims.dtype], (l, rel_err(dec[0][l], K[l]))
+        assert rel_err(dec[1][l], V[l]) < TOL[dims.dtype], (l, rel_err(dec[1][l], V[l]))
+    if dims.dtype == "bf16":
+        assert np.all(dec[2] == 0) and np.all(dec[3] == 0)     # zero padding rows
+
+
+# ---------------------------------------------------------------- compressor (§3.3)
+
+@pytest.mark.parametrize("name,n,init", [("tiny", 300, "paper"), ("64d3l", 300, "wide"), ("128d5l", 257, "paper"),
+                                         ("128d5l", 1000, "wide"), ("128d5l", 1, "wide")])
+def test_compress_parity(name, n, init):
+    dims = dims_of(name)
+    P = datagen.make_params(dims, 4, init)
+    m = tr().Model(dims, P)
+    X = datagen.rand_matrix(22, (n, dims.comp_dims[0]), 0.3 if init == "wide" else 0.01, dims.dtype)
+    out = torch.empty(n, dims.D, dtype=tdt(dims.dtype), device="cuda")
+    tr().compress_targets(m, dev(X, tdt(dims.dtype)), out)
+    torch.cuda.synchronize()
+    ref = oracle.compress_targets(P, X)
+    got = out.double().cpu().numpy()
+    assert rel_err(got, ref) < TOL[dims.dtype], rel_err(got, ref)
+
+
+# ---------------------------------------------------------------- candidate stack (§3.3)
+
+def _score_setup(name, init, L_us, n_per, seed=5, token_std=None):
+    dims = dims_of(name)
+    P = datagen.make_params(dims, seed, init)
+    m = tr().Model(dims, P)
+    std_u = 0.3 if init == "wide" else 0.01
+    std_t = token_std or (0.5 if init == "wide" else 0.3)
+    users = [datagen.rand_matrix(100 + r, (L, dims.D), std_u, "f32") for r, L in enumerate(L_us)]
+    toks = [datagen.rand_matrix(200 + r, (n, dims.D), std_t, dims.dtype) for r, n in enumerate(n_per)]
+    doms = [r % dims.n_domains for r in range(len(L_us))]
+    kvs = []
+    for r, L in enumerate(L_us):
+        kv = torch.zeros(max(tr().kv_cache_bytes(m, L), 16), dtype=torch.uint8, device="cuda")
+        if L:
+            tr().prefill_user(m, dev(users[r]), L, doms[r], kv)
+        kvs.append(kv)
+    return dims, P, m, users, toks, doms, kvs
+
+
+def _gpu_scores(m, dims, toks, kvs, L_us, doms):
+    T = dev(np.concatenate(toks), tdt(dims.dtype))
+    off = np.concatenate([[0], np.cumsum([len(t) for t in toks])])
+    s = torch.empty(int(off[-1]), dtype=torch.float32, device="cuda")
+    tr().score_candidates(m, T, off.tolist(), kvs, L_us, doms, s)
+    torch.cuda.synchronize()
+    return s.cpu().numpy().astype(np.float64), off
+
+
+def _oracle_scores(P, dims, users, toks, doms):
+    out = []
+    for U, t, d in zip(users, toks, doms):
+        K, V = oracle.prefill_user(P, dims.n_head, U, d)
+        out.append(oracle.score_candidates(P, dims.n_head, t, K, V, d))
+    return np.concatenate(out)
+
+
+@pytest.mark.parametrize("name,init,L_u,n", [("tiny", "paper", 8, 256), ("tiny", "wide", 8, 300),
+                                             ("64d3l", "wide", 32, 300), ("64d3l", "paper", 32, 129),
+                                             ("128d5l", "paper", 64, 300), ("128d5l", "wide", 64, 300),
+                                             ("128d5l", "wide", 128, 130), ("128d5l", "wide", 1, 64),
+                                             ("128d5l", "wide", 0, 50), ("128d5l", "wide", 256, 40),
+                                             ("128d5l", "wide", 64, 1)])
+def test_score_parity(name, init, L_u, n):
+    dims, P, m, users, toks, doms, kvs = _score_setup(name, init, [L_u], [n])
+    got, _ = _gpu_scores(m, dims, toks, kvs, [L_u], doms)
+    ref = _oracle_scores(P, dims, users, toks, doms)
+    e = rel_err(got, ref)
+    assert e < TOL[dims.dtype], e
+    # the candidate-dependent part alone, relative to its own spread
+    if n > 1:
+        ec = np.max(np.abs((got - got.mean()) - (ref - ref.mean()))) / ref.std()
+        assert ec < (5e-4 if dims.dtype == "f32" else 6e-2), ec
+
+
+def test_packed_requests_are_isolated_and_match_single_runs():
+    L_us = [16, 128, 0, 77, 1, 64]
+    n_per = [130, 40, 17, 256, 3, 200]
+    dims, P, m, users, toks, doms, kvs = _score_setup("128d5l", "wide", L_us, n_per)
+    packed, off = _gpu_scores(m, dims, toks, kvs, L_us, doms)
+    for r in range(len(L_us)):
+        single, _ = _gpu_scores(m, dims, [toks[r]], [kvs[r]], [L_us[r]], [doms[r]])
+        assert np.array_equal(single, packed[off[r]:off[r + 1]]), r
+    ref = _oracle_scores(P, dims, users, toks, doms)
+    for r in range(len(L_us)):
+        assert rel_err(packed[off[r]:off[r + 1]], ref[off[r]:off[r + 1]]) < TOL["bf16"]
+
+
+def test_scores_independent_of_batch_mates_bitexact():
+    dims, P, m, users, toks, doms, kvs = _score_setup("128d5l", "wide", [64], [700])
+    full, _ = _gpu_scores(m, dims, toks, kvs, [64], doms)
+    rng = np.random.default_rng(1)
+    for idx in (np.arange(0, 700, 3), rng.permutation(700)[:129], np.array([699])):
+        sub, _ = _gpu_scores(m, dims, [toks[0][idx]], kvs, [64], doms)
+        assert np.array_equal(sub, full[idx])
+
+
+# ---------------------------------------------------------------- whole request
+
+def _pipeline(name, n_cand, rows, init="paper", seed=None):
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload
+    w = datagen.scaled(datagen.WORKLOADS[name], n_cand_per_request=n_cand, rows=rows, seed=seed)
+    P = datagen.make_params(w.dims, w.seed, init)
+    dw = DeviceWorkload(w, params=P)
+    dw.step()
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    return w, P, dw
+
+
+@pytest.mark.parametrize("name,n,rows,init", [("tiny", 256, None, "paper"), ("64d3l", 1500, 20000, "paper"),
+                                              ("128d5l", 1000, 20000, "wide"), ("packed", 70, 20000, "paper")])
+def test_pipeline_end_to_end(name, n, rows, init):
+    w, P, dw = _pipeline(name, n, rows, init)
+    got = dw.scores.double().cpu().numpy()
+    for r, req in enumerate(dw.reqs):
+        ref = oracle.score_request(w, P, req).scores
+        g = got[dw.req_offsets[r]:dw.req_offsets[r + 1]]
+        assert rel_err(g, ref) < TOL[w.dims.dtype], (r, rel_err(g, ref))
+        tol_abs = TOL[w.dims.dtype] * float(np.sqrt(np.mean(ref ** 2)))
+        k = min(100, len(ref))
+        idx = np.lexsort((np.arange(len(g)), -g))[:k]
+        ok, why = topk_agrees(idx, ref, k, tol_abs)
+        assert ok, why
+
+
+@pytest.mark.parametrize("name,n_sample", [("128d5l", 96), ("packed", 48), ("large", 64)])
+def test_full_size_sampled(name, n_sample):
+    """Full BASELINE sizes (tables, candidate counts), oracle on sampled candidates."""
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload
+    w = datagen.WORKLOADS[name]
+    dw = DeviceWorkload(w)
+    dw.step()
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    got = dw.scores.double().cpu().numpy()
+    assert np.all(np.isfinite(got))
+    P = dw.params
+    rng = np.random.default_rng(0)
+    for r in range(0, len(dw.reqs), max(1, len(dw.reqs) // 3)):
+        req = dw.reqs[r]
+        cand = np.sort(rng.choice(req.n_cand, size=min(n_sample, req.n_cand), replace=False))
+        if r == 0:
+            cand = np.unique(np.concatenate([cand, [0, req.n_cand - 1]]))
+        ref = oracle.score_request(w, P, req, cand=cand).scores
+        g = got[dw.req_offsets[r] + cand]
+        assert rel_err(g, ref) < TOL["bf16"], (r, rel_err(g, ref))
+    del dw
+    torch.cuda.empty_cache()

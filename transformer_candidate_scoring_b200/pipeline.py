@@ -1,0 +1,133 @@
+"""Device-resident workload and the whole scoring step through the C ABI.
+
+One step of TransRetrieval candidate scoring (§3.1 stages (1)-(4) and the head):
+  per request: tr_aggregate(user fields) -> tr_prefill_user (K/V cache)
+  all requests packed: tr_aggregate(target fields) -> tr_compress_targets -> tr_score_candidates
+Inputs come from ``datagen`` (seeded synthetic tables and bags); tables are filled on the
+device by datagen's counter-based generator.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import List
+
+import numpy as np
+import torch
+
+import datagen
+
+from . import api
+
+
+def _dev(a: np.ndarray, device) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+@dataclass
+class DeviceBags:
+    offsets: torch.Tensor
+    keys: torch.Tensor
+    weights: torch.Tensor
+    bag_table: torch.Tensor
+
+    @staticmethod
+    def of(b: "datagen.Bags", device) -> "DeviceBags":
+        return DeviceBags(_dev(b.offsets.astype(np.int64), device), _dev(b.keys.astype(np.int32), device),
+                          _dev(b.weights.astype(np.float32), device), _dev(b.bag_table.astype(np.int32), device))
+
+
+def pack_target_bags(reqs: List["datagen.Request"]) -> "datagen.Bags":
+    offs, keys, wts, tabs = [np.zeros(1, np.int64)], [], [], []
+    base = 0
+    for r in reqs:
+        b = r.target
+        offs.append(b.offsets[1:] + base)
+        base += b.nnz
+        keys.append(b.keys)
+        wts.append(b.weights)
+        tabs.append(b.bag_table)
+    return datagen.Bags(np.concatenate(offs), np.concatenate(keys), np.concatenate(wts), np.concatenate(tabs))
+
+
+class DeviceWorkload:
+    """Tables, model, bags and activation buffers of a workload on one GPU."""
+
+    def __init__(self, w: "datagen.Workload", device="cuda", reqs=None, params=None, tables=None):
+        self.w = w
+        self.device = torch.device(device)
+        dims = w.dims
+        self.dt = api.torch_dtype(dims.dtype)
+        self.params = params if params is not None else datagen.workload_params(w)
+        self.model = api.Model(dims, self.params)
+        if tables is None:
+            tables = self.make_tables(w, self.device)
+        self.user_tables, self.target_tables = tables
+        self.reqs = reqs if reqs is not None else datagen.make_requests(w)
+        self.set_requests(self.reqs)
+
+    @staticmethod
+    def make_tables(w, device):
+        dt = api.torch_dtype(w.dims.dtype)
+        D = w.dims.D
+        ut, tt = [], []
+        for t in range(w.user_tables):
+            x = torch.empty(w.user_rows, D, dtype=dt, device=device)
+            datagen.fill_table_device(x, w.seed, datagen.user_table_id(w, t))
+            ut.append(x)
+        for t, rows in enumerate(w.target_rows):
+            x = torch.empty(rows, D, dtype=dt, device=device)
+            datagen.fill_table_device(x, w.seed, datagen.target_table_id(w, t))
+            tt.append(x)
+        return ut, tt
+
+    def set_requests(self, reqs) -> None:
+        w, dims, dev = self.w, self.w.dims, self.device
+        self.reqs = reqs
+        self.user_bags = [DeviceBags.of(r.user, dev) for r in reqs]
+        self.target_bags = DeviceBags.of(pack_target_bags(reqs), dev)
+        self.L_u = [r.L_u for r in reqs]
+        self.domain = [r.domain for r in reqs]
+        off = [0]
+        for r in reqs:
+            off.append(off[-1] + r.n_cand)
+        self.req_offsets = off
+        n = off[-1]
+        D, F = dims.D, dims.n_target_fields
+        self.user_tokens = [torch.empty(max(l, 1), D, dtype=torch.float32, device=dev) for l in self.L_u]
+        self.kv = [torch.empty(max(api.kv_cache_bytes(self.model, l), 16), dtype=torch.uint8, device=dev)
+                   for l in self.L_u]
+        self.X = torch.empty(n, F * D, dtype=self.dt, device=dev)
+        self.tokens = torch.empty(n, D, dtype=self.dt, device=dev)
+        self.scores = torch.empty(n, dtype=torch.float32, device=dev)
+
+    @property
+    def n_cand(self) -> int:
+        return self.req_offsets[-1]
+
+    # -------------------------------------------------------------- the step
+    def user_side(self, stream=None) -> None:
+        for r, b in enumerate(self.user_bags):
+            if self.L_u[r] == 0:
+                continue
+            api.aggregate(self.user_tables, b.bag_table, b.offsets, b.keys, b.weights, self.user_tokens[r],
+                          stream=stream)
+            api.prefill_user(self.model, self.user_tokens[r], self.L_u[r], self.domain[r], self.kv[r], stream=stream)
+
+    def target_aggregate(self, stream=None) -> None:
+        b = self.target_bags
+        api.aggregate(self.target_tables, b.bag_table, b.offsets, b.keys, b.weights,
+                      self.X.view(-1, self.w.dims.D), stream=stream)
+
+    def compress(self, stream=None) -> None:
+        api.compress_targets(self.model, self.X, self.tokens, stream=stream)
+
+    def score(self, stream=None) -> None:
+        api.score_candidates(self.model, self.tokens, self.req_offsets, self.kv, self.L_u, self.domain,
+                             self.scores, stream=stream)
+
+    def step(self, stream=None) -> torch.Tensor:
+        self.user_side(stream)
+        self.target_aggregate(stream)
+        self.compress(stream)
+        self.score(stream)
+        return self.scores
