@@ -76,7 +76,7 @@ tr_status workspace(size_t bytes, void** out) {
 }
 
 // tensor-core stack / compressor (defined in their own translation units)
-tr_status tc_build(tr_model* m);
+tr_status tc_build(tr_model* m, const tr_model_weights* w);
 bool tc_stack_supported(const tr_model* m);
 tr_status tc_score(const tr_model* m, const void* tokens, int64_t n, const int64_t* req_offsets,
                    const void* const* kv, const int32_t* L_u, const int32_t* domain, int R, float* scores,
@@ -179,7 +179,7 @@ tr_status tr_model_create(const tr_model_desc* desc, const tr_model_weights* w, 
   for (int i = 0; i < 3; ++i) { m->comp_W[i] = nxt(); m->comp_b[i] = nxt(); }
   for (int i = 0; i < 2; ++i) { m->comp_prelu[i] = nxt(); m->comp_ln_g[i] = nxt(); m->comp_ln_b[i] = nxt(); }
   if (desc->dtype == TR_BF16) {
-    tr_status s = tc_build(m);
+    tr_status s = tc_build(m, w);
     if (s != TR_OK) {
       tr_model_destroy(m);
       return s;
@@ -297,6 +297,8 @@ tr_status tr_sync_status(tr_stream stream, int timeout_ms) {
   TR_CUDA_TRY(cudaMemcpy(&h, ds->status, sizeof(int), cudaMemcpyDeviceToHost));
   if (h) {
     TR_CUDA_TRY(cudaMemset(ds->status, 0, sizeof(int)));
+    if (h & STATUS_KERNEL_TIMEOUT)
+      return fail(TR_ERR_TIMEOUT, "a kernel gave up waiting on an internal barrier and unwound");
     if (h & STATUS_KEY_RANGE) return fail(TR_ERR_KEY_RANGE, "a key or table index was out of range (skipped)");
   }
   return TR_OK;

@@ -41,7 +41,7 @@ void count_launch();
 
 // ---------------------------------------------------------------- device status word
 // Bits set by kernels that meet input only the device can check.
-enum : int { STATUS_KEY_RANGE = 1 };
+enum : int { STATUS_KEY_RANGE = 1, STATUS_KERNEL_TIMEOUT = 2 };
 
 // Per-device state: the status word and a grow-only workspace for multi-kernel calls.
 struct DeviceState {
