@@ -105,7 +105,9 @@ typedef struct {
 const char* tr_last_error(void);
 
 /* Copies and repacks the weights into device memory owned by the returned handle.
- * Uses the current CUDA device.  Synchronous. */
+ * Uses the current CUDA device.  Synchronous.  With the environment variable
+ * TR_FORCE_SIMT=1 at creation time, a bf16 model runs every stage on the CUDA-core
+ * (fp32 arithmetic) kernels instead of the tensor-core ones. */
 tr_status tr_model_create(const tr_model_desc* desc, const tr_model_weights* w, tr_model** out);
 void tr_model_destroy(tr_model* m);
 

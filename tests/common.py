@@ -21,6 +21,31 @@ def rel_err(got, ref, floor_frac: float = 1.0) -> float:
     return float(np.max(np.abs(g - r) / den))
 
 
+def normwise_err(got, ref) -> float:
+    """max_i |g_i - r_i| / max_i |r_i|: the max-norm relative error of the whole output."""
+    g = np.asarray(got, dtype=np.float64).reshape(-1)
+    r = np.asarray(ref, dtype=np.float64).reshape(-1)
+    if r.size == 0:
+        return 0.0
+    den = float(np.max(np.abs(r)))
+    return float(np.max(np.abs(g - r)) / (den if den > 0 else 1.0))
+
+
+def check_close(got, ref, dtype: str, what: str = "") -> dict:
+    """Parity bar for one output.
+
+    bf16: normwise error <= 2e-2 (the stated tolerance, read as the max-norm relative
+    error of the output vector) and the elementwise error, floored at the output's rms,
+    <= 5e-2.  fp32: both <= 1e-4.  Returns the measured metrics (also the elementwise
+    error with a 0.1*rms floor, for information)."""
+    tol = 2e-2 if dtype == "bf16" else 1e-4
+    tol_el = 5e-2 if dtype == "bf16" else 1e-4
+    m = {"normwise": normwise_err(got, ref), "elementwise_rms_floor": rel_err(got, ref),
+         "elementwise_0.1rms_floor": rel_err(got, ref, 0.1)}
+    assert m["normwise"] <= tol and m["elementwise_rms_floor"] <= tol_el, (what, m)
+    return m
+
+
 def topk_agrees(got_idx, ref_scores, k: int, tol_abs: float) -> tuple[bool, str]:
     """GPU top-k against oracle scores.
 

@@ -1,5 +1,6 @@
 // C ABI of libtr: argument validation, model construction, dispatch to the kernels.
 #include <stdarg.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <atomic>
@@ -83,6 +84,8 @@ tr_status tc_score(const tr_model* m, const void* tokens, int64_t n, const int64
                    cudaStream_t st);
 bool tc_comp_supported(const tr_model* m);
 tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens, cudaStream_t st);
+bool tc_prefill_supported(const tr_model* m, int L_u);
+tr_status tc_prefill(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv, cudaStream_t st);
 
 }  // namespace tr
 
@@ -178,7 +181,8 @@ tr_status tr_model_create(const tr_model_desc* desc, const tr_model_weights* w, 
   m->b_head = w->b_head;
   for (int i = 0; i < 3; ++i) { m->comp_W[i] = nxt(); m->comp_b[i] = nxt(); }
   for (int i = 0; i < 2; ++i) { m->comp_prelu[i] = nxt(); m->comp_ln_g[i] = nxt(); m->comp_ln_b[i] = nxt(); }
-  if (desc->dtype == TR_BF16) {
+  const char* force = getenv("TR_FORCE_SIMT");
+  if (desc->dtype == TR_BF16 && !(force && force[0] == '1')) {
     tr_status s = tc_build(m, w);
     if (s != TR_OK) {
       tr_model_destroy(m);
@@ -196,6 +200,7 @@ void tr_model_destroy(tr_model* m) {
   cudaSetDevice(m->device);
   if (m->f32_blob) cudaFree(m->f32_blob);
   if (m->tc_blob) cudaFree(m->tc_blob);
+  if (m->tc_comp) cudaFree(const_cast<void*>(m->tc_comp));
   cudaSetDevice(prev);
   delete m;
 }
@@ -242,6 +247,7 @@ tr_status tr_prefill_user(const tr_model* m, const float* user_tokens, int L_u, 
   if (domain < 0 || domain >= m->desc.n_domains) return fail(TR_ERR_INVALID_ARG, "domain=%d", domain);
   if (L_u == 0) return TR_OK;
   if (!user_tokens || !kv) return fail(TR_ERR_INVALID_ARG, "null device pointer");
+  if (tc_prefill_supported(m, L_u)) return tc_prefill(m, user_tokens, L_u, domain, kv, (cudaStream_t)stream);
   return simt_prefill(m, user_tokens, L_u, domain, kv, (cudaStream_t)stream);
 }
 

@@ -1,0 +1,438 @@
+// Target compressor on tcgen05 tensor cores (TransRetrieval §3.3):
+//   t = W3 g2(W2 g1(W1 x + b1) + b2) + b3,   g_i(z) = LayerNorm_i(PReLU_i(z))
+//
+// One persistent CTA per SM walks 128-row tiles and keeps each tile on chip through all
+// three layers:
+//   layer 1: x tiles arrive by TMA tensor loads (128-byte swizzle, rows past the end are
+//            zero-filled by the copy engine) together with bulk copies of the matching
+//            W1 slice, two stages deep; the [128 x c1] fp32 accumulator fills TMEM.
+//   epilogue 1: + b1, PReLU, LayerNorm over c1 (two passes over TMEM, thread = row),
+//            bf16 result written in the core-matrix layout over the now idle stage buffers.
+//   layers 2, 3: W2 / W3 slices stream through a second two-stage ring.
+//   epilogue 3: + b3, bf16, one row per thread straight to global memory.
+// Warp 0 issues copies, warp 1 issues MMAs, warps 2-5 run the epilogues.  Waits are
+// bounded as in the candidate stack kernel.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "model.cuh"
+#include "tc_common.cuh"
+
+namespace tr {
+namespace {
+
+using namespace tc;
+
+constexpr int kM = 128;
+constexpr int STAGE1 = 80 * 1024;              // x slice (16 KB) + W1 slice (<= 64 KB)
+constexpr int OFF_R1 = 0;
+constexpr int OFF_R2 = 2 * STAGE1;             // 160 KB
+constexpr int STAGE2 = 32 * 1024;
+constexpr int OFF_BAR = OFF_R2 + 2 * STAGE2;   // 224 KB
+constexpr int SMEM_BYTES = OFF_BAR + 128 + 1024;
+
+struct CompParams {
+  CUtensorMap xmap;            // x [n][c0] bf16, box {64, 128}, 128-byte swizzle
+  const uint8_t* w1;           // [c0/64] slices of W1^T [c1 x 64]
+  const uint8_t* w2;           // [c1/64] slices of W2^T [c2 x 64]
+  const uint8_t* w3;           // [c2/64] slices of W3^T [c3 x 64]
+  const float* vec;            // b1 a1 g1 be1 (c1 each), b2 a2 g2 be2 (c2 each), b3 (c3)
+  __nv_bfloat16* out;          // [n][c3]
+  int* status;
+  long long n;
+  int n_tiles, c0, c1, c2, c3;
+};
+
+struct CBars {
+  uint32_t full1[2], empty1[2], full2[2], empty2[2], r1_free, mma, epi, drain;
+};
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// K-major operand written by TMA with the 128-byte swizzle: 8-row atoms of 1024 bytes.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFF) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+
+__device__ void comp_producer(const CompParams& p, uint32_t r1, uint32_t r2, const CBars& b, volatile int* abort_flag) {
+  int s1 = 0, s2 = 0;
+  uint32_t ph1 = 0, ph2 = 0, free_phase = 0;
+  const uint32_t w1_bytes = p.c1 * 128, w2_bytes = p.c2 * 128, w3_bytes = p.c3 * 128;
+  bool ok = true;
+  bool pend1[2] = {false, false}, pend2[2] = {false, false};
+  uint32_t par1[2] = {0, 0}, par2[2] = {0, 0};
+  for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+    // the stage buffers hold the previous tile's activations until its last GEMM is done
+    if (!(ok = mbar_wait(b.r1_free, free_phase ^ 1, abort_flag))) break;
+    free_phase ^= 1;
+    for (int kc = 0; kc < p.c0 / 64 && ok; ++kc) {
+      if (!(ok = mbar_wait(b.empty1[s1], ph1 ^ 1, abort_flag))) break;
+      const uint32_t st = r1 + s1 * STAGE1;
+      mbar_arrive_expect_tx(b.full1[s1], kM * 64 * 2 + w1_bytes);
+      tma_load_2d(st, &p.xmap, kc * 64, tile * kM, b.full1[s1]);
+      bulk_g2s(st + 16384, p.w1 + (size_t)kc * w1_bytes, w1_bytes, b.full1[s1]);
+      pend1[s1] = true;
+      par1[s1] = ph1;
+      if (++s1 == 2) { s1 = 0; ph1 ^= 1; }
+    }
+    for (int j = 0; j < p.c1 / 64 + p.c2 / 64 && ok; ++j) {
+      if (!(ok = mbar_wait(b.empty2[s2], ph2 ^ 1, abort_flag))) break;
+      const bool is2 = j < p.c1 / 64;
+      const uint32_t bytes = is2 ? w2_bytes : w3_bytes;
+      const uint8_t* src = is2 ? p.w2 + (size_t)j * w2_bytes : p.w3 + (size_t)(j - p.c1 / 64) * w3_bytes;
+      mbar_arrive_expect_tx(b.full2[s2], bytes);
+      bulk_g2s(r2 + s2 * STAGE2, src, bytes, b.full2[s2]);
+      pend2[s2] = true;
+      par2[s2] = ph2;
+      if (++s2 == 2) { s2 = 0; ph2 ^= 1; }
+    }
+  }
+  if (!ok) {
+    for (int s = 0; s < 2; ++s) {
+      for (uint64_t t0 = globaltimer_ns(); pend1[s] && !mbar_try_wait(b.full1[s], par1[s]) && globaltimer_ns() - t0 < 200000000ull;) {
+      }
+      for (uint64_t t0 = globaltimer_ns(); pend2[s] && !mbar_try_wait(b.full2[s], par2[s]) && globaltimer_ns() - t0 < 200000000ull;) {
+      }
+    }
+  }
+}
+
+__device__ void comp_mma(const CompParams& p, uint32_t tmem, uint32_t r1, uint32_t r2, const CBars& b,
+                         volatile int* abort_flag) {
+  int s1 = 0, s2 = 0;
+  uint32_t ph1 = 0, ph2 = 0, epi_phase = 0;
+  bool ok = true;
+  const int n1 = std::min(p.c1, 256);
+  const uint32_t id1 = idesc_bf16(kM, n1), id2 = idesc_bf16(kM, p.c2), id3 = idesc_bf16(kM, p.c3);
+  auto wait_epi = [&]() {
+    ok = ok && mbar_wait(b.epi, epi_phase, abort_flag);
+    epi_phase ^= 1;
+    tc_fence_after();
+    return ok;
+  };
+  for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+    if (tile != (int)blockIdx.x && !wait_epi()) break;   // previous tile's last epilogue has read TMEM
+    // layer 1: [128 x c0] x [c0 x c1]
+    for (int kc = 0; kc < p.c0 / 64 && ok; ++kc) {
+      if (!(ok = mbar_wait(b.full1[s1], ph1, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t xa = r1 + s1 * STAGE1, wb = xa + 16384;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        for (int nh = 0; nh < p.c1 / n1; ++nh)
+          mma_bf16(tmem + nh * n1, sdesc_sw128(xa + kk * 32),
+                   sdesc(wb + kk * 2 * p.c1 * 16 + nh * (n1 / 8) * 128, p.c1 * 16, 128), id1,
+                   (kc > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(b.empty1[s1]);
+      if (++s1 == 2) { s1 = 0; ph1 ^= 1; }
+    }
+    if (!ok) break;
+    mma_commit(b.mma);
+    if (!wait_epi()) break;                                // h1 (bf16) in R1
+    for (int kc = 0; kc < p.c1 / 64 && ok; ++kc) {
+      if (!(ok = mbar_wait(b.full2[s2], ph2, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t wb = r2 + s2 * STAGE2;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem, sdesc(r1 + (4 * kc + kk) * 2 * kM * 16, kM * 16, 128),
+                 sdesc(wb + kk * 2 * p.c2 * 16, p.c2 * 16, 128), id2, (kc > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(b.empty2[s2]);
+      if (++s2 == 2) { s2 = 0; ph2 ^= 1; }
+    }
+    if (!ok) break;
+    mma_commit(b.mma);
+    if (!wait_epi()) break;                                // h2 (bf16) in R1
+    for (int kc = 0; kc < p.c2 / 64 && ok; ++kc) {
+      if (!(ok = mbar_wait(b.full2[s2], ph2, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t wb = r2 + s2 * STAGE2;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16(tmem + 256, sdesc(r1 + (4 * kc + kk) * 2 * kM * 16, kM * 16, 128),
+                 sdesc(wb + kk * 2 * p.c3 * 16, p.c3 * 16, 128), id3, (kc > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(b.empty2[s2]);
+      if (++s2 == 2) { s2 = 0; ph2 ^= 1; }
+    }
+    if (!ok) break;
+    mma_commit(b.r1_free);
+    mma_commit(b.mma);
+  }
+  mma_commit(b.drain);
+  for (uint64_t t0 = globaltimer_ns(); !mbar_try_wait(b.drain, 0) && globaltimer_ns() - t0 < 500000000ull;) {
+  }
+}
+
+// + bias, PReLU, LayerNorm over `cols` accumulator columns of this row -> bf16 operand in R1.
+__device__ __forceinline__ void prelu_ln_row(uint32_t tcol, int cols, const float* bias, const float* slope,
+                                             const float* g, const float* be, uint32_t dst_row) {
+  float x0 = 0.f, s1 = 0.f, s2 = 0.f;
+  for (int c = 0; c < cols; c += 64) {
+    float v[64];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) tmem_ld16(tcol + c + 16 * q, v + 16 * q);
+    tmem_wait_ld();
+    reg_fence<64>(v);
+    if (c == 0) {
+      x0 = v[0] + __ldg(bias);
+      x0 = x0 >= 0.f ? x0 : x0 * __ldg(slope);
+    }
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      float x = v[i] + __ldg(bias + c + i);
+      x = x >= 0.f ? x : x * __ldg(slope + c + i);
+      const float d = x - x0;
+      s1 += d;
+      s2 = fmaf(d, d, s2);
+    }
+  }
+  const float inv_n = 1.f / cols;
+  const float dm = s1 * inv_n;
+  const float mean = x0 + dm;
+  const float rstd = rsqrtf(fmaxf(s2 * inv_n - dm * dm, 0.f) + kLnEps);
+  for (int c = 0; c < cols; c += 64) {
+    float v[64];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) tmem_ld16(tcol + c + 16 * q, v + 16 * q);
+    tmem_wait_ld();
+    reg_fence<64>(v);
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+      float x = v[i] + __ldg(bias + c + i);
+      x = x >= 0.f ? x : x * __ldg(slope + c + i);
+      v[i] = (x - mean) * rstd * __ldg(g + c + i) + __ldg(be + c + i);
+    }
+#pragma unroll
+    for (int kc = 0; kc < 8; ++kc) st_row8(dst_row + ((c >> 3) + kc) * 2048, v + 8 * kc);
+  }
+}
+
+__device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, const CBars& b,
+                              volatile int* abort_flag) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int q = warp & 3, m = q * 32 + lane;
+  const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+  const uint32_t rowoff = (m >> 3) * 128 + (m & 7) * 16;
+  const float* v1 = p.vec;
+  const float* v2 = p.vec + 4 * p.c1;
+  const float* b3 = v2 + 4 * p.c2;
+  uint32_t mma_phase = 0;
+  bool ok = true;
+  auto wait_mma = [&]() {
+    ok = ok && mbar_wait(b.mma, mma_phase, abort_flag);
+    mma_phase ^= 1;
+    tc_fence_after();
+    return ok;
+  };
+  auto signal = [&]() {
+    tmem_wait_st();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    mbar_arrive(b.epi);
+  };
+  for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+    if (!wait_mma()) break;
+    prelu_ln_row(trow, p.c1, v1, v1 + p.c1, v1 + 2 * p.c1, v1 + 3 * p.c1, r1 + rowoff);
+    signal();
+    if (!wait_mma()) break;
+    prelu_ln_row(trow, p.c2, v2, v2 + p.c2, v2 + 2 * p.c2, v2 + 3 * p.c2, r1 + rowoff);
+    signal();
+    if (!wait_mma()) break;
+    const long long row = (long long)tile * kM + m;
+    for (int c = 0; c < p.c3; c += 16) {
+      float v[16];
+      tmem_ld16(trow + 256 + c, v);
+      tmem_wait_ld();
+      reg_fence<16>(v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] += __ldg(b3 + c + i);
+      if (row < p.n) {
+        uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.c3 + c);
+        dst[0] = make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]), pack2(v[6], v[7]));
+        dst[1] = make_uint4(pack2(v[8], v[9]), pack2(v[10], v[11]), pack2(v[12], v[13]), pack2(v[14], v[15]));
+      }
+    }
+    signal();
+  }
+}
+
+__global__ void __launch_bounds__(192, 1) compress_kernel(const __grid_constant__ CompParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t r1 = base + OFF_R1, r2 = base + OFF_R2, bar0 = base + OFF_BAR;
+  CBars b;
+  for (int s = 0; s < 2; ++s) {
+    b.full1[s] = bar0 + 8 * s;
+    b.empty1[s] = bar0 + 16 + 8 * s;
+    b.full2[s] = bar0 + 32 + 8 * s;
+    b.empty2[s] = bar0 + 48 + 8 * s;
+  }
+  b.r1_free = bar0 + 64;
+  b.mma = bar0 + 72;
+  b.epi = bar0 + 80;
+  b.drain = bar0 + 88;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_BAR + 112);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_BAR + 120);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(b.full1[s], 1);
+      mbar_init(b.empty1[s], 1);
+      mbar_init(b.full2[s], 1);
+      mbar_init(b.empty2[s], 1);
+    }
+    mbar_init(b.r1_free, 1);
+    mbar_init(b.mma, 1);
+    mbar_init(b.epi, 128);
+    mbar_init(b.drain, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.xmap)) : "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (warp == 0) {
+    if (lane == 0) comp_producer(p, r1, r2, b, abort_flag);
+  } else if (warp == 1) {
+    if (lane == 0) comp_mma(p, tmem, r1, r2, b, abort_flag);
+  } else {
+    comp_epilogue(p, tmem, r1, b, abort_flag);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, STATUS_KERNEL_TIMEOUT);
+}
+
+// W^T slice rows [0, N) x cols [k0, k0 + 64) of W [K][N] in the core-matrix layout.
+void put_slice(uint16_t* dst, const float* W, int N, int k0) {
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < 64; ++k) {
+      float f = W[(size_t)(k0 + k) * N + n];
+      uint32_t u;
+      memcpy(&u, &f, 4);
+      u = (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
+      dst[((size_t)(k / 8) * (N / 8) + n / 8) * 64 + (n % 8) * 8 + (k % 8)] = (uint16_t)u;
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool tc_comp_supported(const tr_model* m) {
+  const int* c = m->desc.comp_dims;
+  return m->desc.dtype == TR_BF16 && m->tc_comp && c[0] % 64 == 0 && c[1] % 64 == 0 && c[1] <= 512 &&
+         c[2] % 64 == 0 && c[2] <= 256 && c[3] % 16 == 0 && c[3] <= 256;
+}
+
+// Builds the compressor's weight slices; called from tc_build for bf16 models.
+tr_status tc_build_comp(tr_model* m, const tr_model_weights* w) {
+  const int* c = m->desc.comp_dims;
+  if (!(c[0] % 64 == 0 && c[1] % 64 == 0 && c[1] <= 512 && c[2] % 64 == 0 && c[2] <= 256 && c[3] % 16 == 0 &&
+        c[3] <= 256))
+    return TR_OK;
+  const size_t e1 = (size_t)c[0] * c[1], e2 = (size_t)c[1] * c[2], e3 = (size_t)c[2] * c[3];
+  std::vector<uint16_t> img(e1 + e2 + e3);
+  for (int kc = 0; kc < c[0] / 64; ++kc) put_slice(img.data() + (size_t)kc * 64 * c[1], w->comp_W[0], c[1], 64 * kc);
+  for (int kc = 0; kc < c[1] / 64; ++kc) put_slice(img.data() + e1 + (size_t)kc * 64 * c[2], w->comp_W[1], c[2], 64 * kc);
+  for (int kc = 0; kc < c[2] / 64; ++kc)
+    put_slice(img.data() + e1 + e2 + (size_t)kc * 64 * c[3], w->comp_W[2], c[3], 64 * kc);
+  std::vector<float> vec;
+  for (int i = 0; i < 2; ++i) {
+    const int n = c[i + 1];
+    vec.insert(vec.end(), w->comp_b[i], w->comp_b[i] + n);
+    vec.insert(vec.end(), w->comp_prelu[i], w->comp_prelu[i] + n);
+    vec.insert(vec.end(), w->comp_ln_g[i], w->comp_ln_g[i] + n);
+    vec.insert(vec.end(), w->comp_ln_b[i], w->comp_ln_b[i] + n);
+  }
+  vec.insert(vec.end(), w->comp_b[2], w->comp_b[2] + c[3]);
+  const size_t ib = img.size() * 2, vb = vec.size() * 4;
+  void* blob = nullptr;
+  if (cudaMalloc(&blob, ib + vb) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(TR_ERR_NOMEM, "compressor weight images: allocation failed");
+  }
+  TR_CUDA_TRY(cudaMemcpy(blob, img.data(), ib, cudaMemcpyHostToDevice));
+  TR_CUDA_TRY(cudaMemcpy((uint8_t*)blob + ib, vec.data(), vb, cudaMemcpyHostToDevice));
+  m->tc_comp = blob;
+  m->tc_comp_vec = reinterpret_cast<const float*>((uint8_t*)blob + ib);
+  return TR_OK;
+}
+
+tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens, cudaStream_t st) {
+  const int* c = m->desc.comp_dims;
+  if ((uintptr_t)x % 16 || (uintptr_t)tokens % 16) return fail(TR_ERR_INVALID_ARG, "x/tokens not 16-byte aligned");
+  auto encode = get_encode();
+  if (!encode) return fail(TR_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  DeviceState* ds = nullptr;
+  TR_TRY(device_state(&ds));
+  CompParams p;
+  memset(&p, 0, sizeof p);
+  cuuint64_t gdim[2] = {(cuuint64_t)c[0], (cuuint64_t)n};
+  cuuint64_t gstride[1] = {(cuuint64_t)c[0] * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = encode(&p.xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box, estride,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TR_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  const uint8_t* img = static_cast<const uint8_t*>(m->tc_comp);
+  p.w1 = img;
+  p.w2 = img + (size_t)c[0] * c[1] * 2;
+  p.w3 = p.w2 + (size_t)c[1] * c[2] * 2;
+  p.vec = m->tc_comp_vec;
+  p.out = static_cast<__nv_bfloat16*>(tokens);
+  p.status = ds->status;
+  p.n = n;
+  p.n_tiles = (int)((n + kM - 1) / kM);
+  p.c0 = c[0];
+  p.c1 = c[1];
+  p.c2 = c[2];
+  p.c3 = c[3];
+  static bool attr_set[64] = {};
+  int dev = 0, sms = 148;
+  TR_CUDA_TRY(cudaGetDevice(&dev));
+  TR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  if (!attr_set[dev]) {
+    TR_CUDA_TRY(cudaFuncSetAttribute(compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    attr_set[dev] = true;
+  }
+  compress_kernel<<<std::min(p.n_tiles, sms), 192, SMEM_BYTES, st>>>(p);
+  TR_LAUNCH_CHECK("compress_kernel");
+  return TR_OK;
+}
+
+}  // namespace tr

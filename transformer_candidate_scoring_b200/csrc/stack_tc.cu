@@ -47,7 +47,8 @@ constexpr int kD = 128, kH = 256, kM = 128;
 constexpr int kChunk = 16384;                 // [128 x 64] bf16 weight slice
 constexpr int kStages = 4;
 constexpr int kChunksPerLayer = 16;
-constexpr int kVecPerLayer = 5 * kD + kH;     // c1, bq, bk, bv, c2, b1
+constexpr int kVecPerLayer = 9 * kD + kH;     // c1, g1, be1, bq*qs, bk, bv, c2, g2, be2, b1
+constexpr float kQScale = 0.25f * 1.44269504088896341f;  // 1/sqrt(d_h) * log2(e)
 constexpr int kVecFinal = 2 * kD + 16;        // cf, w, b
 constexpr int kMaxLpTc = 128;
 
@@ -79,6 +80,8 @@ struct StackParams {
   int n_layer;
   int n_tiles;
   int R;
+  const float* utokens;      // user-side mode: fp32 user tokens [L_u][D]
+  uint8_t* kv_out;           // user-side mode: the request's K/V cache
   ReqInfo req[TR_MAX_REQUESTS];
 };
 
@@ -103,10 +106,11 @@ __device__ __forceinline__ TileInfo tile_info(const StackParams& p, int tile) {
 }
 
 struct Bars {
-  uint32_t full[kStages], empty[kStages], kv_full, kv_empty, mma, epi, drain;
+  uint32_t full[kStages], empty[kStages], kv_full, kv_empty, mma, epi, drain, esync;
 };
 
 // ------------------------------------------------------------------ producer (warp 0, one thread)
+template <bool PF>
 __device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, const Bars& b, volatile int* abort_flag) {
   int stage = 0;
   uint32_t phase = 0, kv_phase = 0;
@@ -120,7 +124,7 @@ __device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, co
     for (int l = 0; l < p.n_layer && ok; ++l) {
       const uint8_t* wl = p.wimg + (size_t)l * kChunksPerLayer * kChunk;
       for (int c = 0; c < kChunksPerLayer && ok; ++c) {
-        if (c == 6) {  // the request's K/V images go in between the QKV and O weights
+        if (!PF && c == 6) {  // the request's K/V images go in between the QKV and O weights
           if (!(ok = mbar_wait(b.kv_empty, kv_phase ^ 1, abort_flag))) break;
           const uint32_t bytes = 2u * t.Lp * kD * 2u;
           if (bytes) {
@@ -157,6 +161,7 @@ __device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, co
 }
 
 // ------------------------------------------------------------------ MMA issuer (warp 1, one thread)
+template <bool PF>
 __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sPH, uint32_t sKV, uint32_t ring,
                            const Bars& b, volatile int* abort_flag) {
   constexpr uint32_t ID128 = idesc_bf16(kM, 128);
@@ -199,9 +204,11 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
       chunk(sA, 4, 384, true);
       mma_commit(b.mma);
       if (!wait_epi()) break;                         // A = Q (scaled, biased)
-      ok = ok && mbar_wait(b.kv_full, kv_phase, abort_flag);
-      kv_phase ^= 1;
-      tc_fence_after();
+      if (!PF) {
+        ok = ok && mbar_wait(b.kv_full, kv_phase, abort_flag);
+        kv_phase ^= 1;
+        tc_fence_after();
+      }
       for (int g = 0; g < t.ng && ok; ++g) {
         for (int s = 0; s < t.hg; ++s) {
           const int h = g * t.hg + s;
@@ -220,7 +227,7 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
         }
       }
       if (!ok) break;
-      mma_commit(b.kv_empty);
+      if (!PF) mma_commit(b.kv_empty);
       mma_commit(b.mma);
       if (!wait_epi()) break;                         // A = attention output
       chunk(sA, 0, 0, true);                          // Y += attn Wo
@@ -244,7 +251,7 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
 }
 
 // ------------------------------------------------------------------ epilogue (warps 2-5)
-__device__ __forceinline__ void ln_rows_to_smem(float* y, uint32_t sA, int m) {
+__device__ __forceinline__ void ln_rows_to_smem(float* y, uint32_t sA, int m, const float* g, const float* be) {
   float mean = 0.f;
 #pragma unroll
   for (int i = 0; i < kD; ++i) mean += y[i];
@@ -261,7 +268,7 @@ __device__ __forceinline__ void ln_rows_to_smem(float* y, uint32_t sA, int m) {
   for (int kc = 0; kc < kD / 8; ++kc) {
     float v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = (y[kc * 8 + i] - mean) * rstd;
+    for (int i = 0; i < 8; ++i) v[i] = fmaf((y[kc * 8 + i] - mean) * rstd, __ldg(g + kc * 8 + i), __ldg(be + kc * 8 + i));
     st_row8(sA + kc * 2048 + rowoff, v);
   }
 }
@@ -273,7 +280,10 @@ __device__ __forceinline__ void load_y(uint32_t trow, float* y) {
   reg_fence<kD>(y);
 }
 
-__device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sPH, const Bars& b,
+// PF (user-side mode): the tile is the request's user tokens; each layer's K and V are
+// the tile's own, written to the K/V images in shared memory and stored to the cache.
+template <bool PF>
+__device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sPH, uint32_t sKV, const Bars& b,
                          volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int q = warp & 3;
@@ -294,12 +304,30 @@ __device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint3
     tc_fence_before();
     mbar_arrive(b.epi);
   };
+  // rendezvous of the 128 epilogue threads (bounded, like every other wait)
+  uint32_t esync_phase = 0;
+  auto epi_sync = [&]() {
+    mbar_arrive(b.esync);
+    ok = ok && mbar_wait(b.esync, esync_phase, abort_flag);
+    esync_phase ^= 1;
+    return ok;
+  };
   const float* vfin = p.vec + (size_t)p.n_layer * kVecPerLayer;
   for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
     const TileInfo t = tile_info(p, tile);
     const float* sd = p.domain_emb + (size_t)p.req[t.r].domain * kD;
     // Y = t + s_d; rows past the request's end are zero and never stored
-    {
+    if (PF) {
+      const float* src = p.utokens + (t.row0 + m) * kD;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float yv[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) yv[i] = (m < t.rows) ? __ldg(src + c * 16 + i) + __ldg(sd + c * 16 + i) : 0.f;
+        tmem_st16(trow + c * 16, yv);
+      }
+      tmem_wait_st();
+    } else {
       const uint4* src = reinterpret_cast<const uint4*>(p.tokens + (t.row0 + m) * kD);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -322,7 +350,8 @@ __device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint3
 
     for (int l = 0; l < p.n_layer && ok; ++l) {
       const float* vl = p.vec + (size_t)l * kVecPerLayer;
-      const float *c1 = vl, *bq = vl + kD, *bk = vl + 2 * kD, *bv = vl + 3 * kD, *c2 = vl + 4 * kD, *b1 = vl + 5 * kD;
+      const float *c1 = vl, *g1 = vl + kD, *be1 = vl + 2 * kD, *bq = vl + 3 * kD, *bk = vl + 4 * kD, *bv = vl + 5 * kD;
+      const float *c2 = vl + 6 * kD, *g2 = vl + 7 * kD, *be2 = vl + 8 * kD, *b1 = vl + 9 * kD;
       // ---- LN1
       if (l > 0 && !wait_mma()) break;            // FFN2 of the previous layer done
       {
@@ -330,12 +359,14 @@ __device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint3
         load_y(trow, y);
 #pragma unroll
         for (int i = 0; i < kD; ++i) y[i] += __ldg(c1 + i);
-        ln_rows_to_smem(y, sA, m);
+        ln_rows_to_smem(y, sA, m, g1, be1);
       }
       signal();
       // ---- Q, own K: the candidate's own score per head; Q to A
       if (!wait_mma()) break;
       float sself[8];
+      if (PF && threadIdx.x == 64 && l > 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      if (PF && !epi_sync()) break;               // the K/V images are free to overwrite
       for (int h = 0; h < 8; ++h) {
         float qv[16], kv[16];
         tmem_ld16(trow + 128 + 16 * h, qv);
@@ -346,12 +377,53 @@ __device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint3
         float s = 0.f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          qv[i] += __ldg(bq + 16 * h + i);
-          s = fmaf(qv[i], kv[i] + __ldg(bk + 16 * h + i), s);
+          qv[i] = fmaf(qv[i], kQScale, __ldg(bq + 16 * h + i));
+          kv[i] += __ldg(bk + 16 * h + i);
+          s = fmaf(qv[i], kv[i], s);
         }
-        sself[h] = s;
+        sself[h] = PF ? -INFINITY : s;
         st_row8(sA + (2 * h) * 2048 + rowoff, qv);
         st_row8(sA + (2 * h + 1) * 2048 + rowoff, qv + 8);
+        if (PF) {
+          // K image row m, V^T image column m (zero past L_u); the TMEM load is
+          // warp-wide, only the stores depend on the row
+          float vv[16];
+          tmem_ld16(trow + 384 + 16 * h, vv);
+          tmem_wait_ld();
+          reg_fence<16>(vv);
+          if (m < t.Lp) {
+            const bool live = m < t.L_u;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              kv[i] = live ? kv[i] : 0.f;
+              vv[i] = live ? vv[i] + __ldg(bv + 16 * h + i) : 0.f;
+            }
+            const uint32_t kb = sKV + (m >> 3) * 128 + (m & 7) * 16;
+            st_row8(kb + (2 * h) * (t.Lp / 8) * 128, kv);
+            st_row8(kb + (2 * h + 1) * (t.Lp / 8) * 128, kv + 8);
+            const uint32_t vb = sKV + t.Lp * 256 + (m >> 3) * 2048 + (m & 7) * 2;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int d = 16 * h + i;
+              const __nv_bfloat16 hv = __float2bfloat16_rn(vv[i]);
+              asm volatile("st.shared.b16 [%0], %1;" ::"r"(vb + (d >> 3) * 128 + (d & 7) * 16),
+                           "h"(*reinterpret_cast<const unsigned short*>(&hv))
+                           : "memory");
+            }
+          }
+        }
+      }
+      if (PF) {  // store this layer's K/V images to the cache with one bulk copy
+        fence_proxy_async_smem();
+        if (!epi_sync()) break;
+        if (threadIdx.x == 64) {
+          const uint32_t bytes = 2u * t.Lp * kD * 2u;
+          asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                           p.kv_out + (size_t)l * bytes),
+                       "r"(sKV), "r"(bytes)
+                       : "memory");
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
       }
       signal();
       // ---- softmax over [user keys of the request, own key], one head group at a time
@@ -426,7 +498,7 @@ __device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint3
         load_y(trow, y);
 #pragma unroll
         for (int i = 0; i < kD; ++i) y[i] += __ldg(c2 + i);
-        ln_rows_to_smem(y, sA, m);
+        ln_rows_to_smem(y, sA, m, g2, be2);
       }
       signal();
       // ---- ReLU(hidden + b1) to P/H
@@ -446,6 +518,7 @@ __device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint3
     if (!ok) break;
     // ---- head: w . LN_f(y) + b
     if (!wait_mma()) break;
+    if (PF) continue;
     float y[kD];
     load_y(trow, y);
     float mean = 0.f;
@@ -466,6 +539,7 @@ __device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint3
   }
 }
 
+template <bool PF>
 __global__ void __launch_bounds__(192, 1) stack_kernel(const __grid_constant__ StackParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -482,6 +556,7 @@ __global__ void __launch_bounds__(192, 1) stack_kernel(const __grid_constant__ S
   b.mma = b.kv_full + 16;
   b.epi = b.kv_full + 24;
   b.drain = b.kv_full + 32;
+  b.esync = b.kv_full + 40;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 112);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_BAR + 120);
 
@@ -495,6 +570,7 @@ __global__ void __launch_bounds__(192, 1) stack_kernel(const __grid_constant__ S
     mbar_init(b.mma, 1);
     mbar_init(b.epi, 128);
     mbar_init(b.drain, 1);
+    mbar_init(b.esync, 128);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -508,11 +584,12 @@ __global__ void __launch_bounds__(192, 1) stack_kernel(const __grid_constant__ S
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) producer(p, ring, sKV, b, abort_flag);
+    if (lane == 0) producer<PF>(p, ring, sKV, b, abort_flag);
   } else if (warp == 1) {
-    if (lane == 0) mma_issuer(p, tmem, sA, sPH, sKV, ring, b, abort_flag);
+    if (lane == 0) mma_issuer<PF>(p, tmem, sA, sPH, sKV, ring, b, abort_flag);
   } else {
-    epilogue(p, tmem, sA, sPH, b, abort_flag);
+    epilogue<PF>(p, tmem, sA, sPH, sKV, b, abort_flag);
+    if (PF && threadIdx.x == 64) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
@@ -546,42 +623,23 @@ bool tc_stack_supported(const tr_model* m) {
   return d.dtype == TR_BF16 && d.D == kD && d.ffn_hidden == kH && d.n_head == 8 && m->tc_stack;
 }
 
+tr_status tc_build_comp(tr_model* m, const tr_model_weights* w);
+
 tr_status tc_build(tr_model* m, const tr_model_weights* w) {
   const tr_model_desc& d = m->desc;
+  TR_TRY(tc_build_comp(m, w));
   if (!(d.dtype == TR_BF16 && d.D == kD && d.ffn_hidden == kH && d.n_head == 8)) return TR_OK;
   const int N = d.n_layer, D = kD, H = kH;
-  const double qscale = 0.25 * 1.4426950408889634;  // 1/sqrt(d_h) * log2(e)
   std::vector<uint16_t> img((size_t)N * kChunksPerLayer * kChunk / 2);
   std::vector<float> vec((size_t)N * kVecPerLayer + kVecFinal, 0.f);
   std::vector<double> c(D, 0.0);
+  auto dvec = [](const float* p, size_t n) { return std::vector<double>(p, p + n); };
   for (int l = 0; l < N; ++l) {
+    // the weights go in unchanged (exact bf16 values); LayerNorm gains/shifts, biases and
+    // the softmax scale stay fp32 and are applied by the epilogue
     const tr_layer_weights& L = w->layers[l];
-    std::vector<double> Wq(D * D), Wk(D * D), Wv(D * D), Wo(D * D), W1(D * H), W2(H * D);
-    std::vector<double> bq(D), bk(D), bv(D), b1(H);
-    for (int j = 0; j < D; ++j) {
-      bq[j] = L.bq[j];
-      bk[j] = L.bk[j];
-      bv[j] = L.bv[j];
-    }
-    for (int j = 0; j < H; ++j) b1[j] = L.b1[j];
-    for (int i = 0; i < D; ++i)
-      for (int j = 0; j < D; ++j) {
-        const double g = L.ln1_g[i], be = L.ln1_b[i];
-        Wq[i * D + j] = g * L.Wq[i * D + j] * qscale;
-        Wk[i * D + j] = g * L.Wk[i * D + j];
-        Wv[i * D + j] = g * L.Wv[i * D + j];
-        bq[j] += be * L.Wq[i * D + j];
-        bk[j] += be * L.Wk[i * D + j];
-        bv[j] += be * L.Wv[i * D + j];
-        Wo[i * D + j] = L.Wo[i * D + j];
-      }
-    for (int j = 0; j < D; ++j) bq[j] *= qscale;
-    for (int i = 0; i < D; ++i)
-      for (int j = 0; j < H; ++j) {
-        W1[i * H + j] = (double)L.ln2_g[i] * L.W1[i * H + j];
-        b1[j] += (double)L.ln2_b[i] * L.W1[i * H + j];
-      }
-    for (int i = 0; i < H * D; ++i) W2[i] = L.W2[i];
+    const auto Wq = dvec(L.Wq, D * D), Wk = dvec(L.Wk, D * D), Wv = dvec(L.Wv, D * D), Wo = dvec(L.Wo, D * D);
+    const auto W1 = dvec(L.W1, D * H), W2 = dvec(L.W2, H * D);
     uint16_t* li = img.data() + (size_t)l * kChunksPerLayer * kChunk / 2;
     const size_t ce = kChunk / 2;
     put_chunk(li + 0 * ce, Wq, D, 0, 0);
@@ -600,14 +658,18 @@ tr_status tc_build(tr_model* m, const tr_model_weights* w) {
     float* v = vec.data() + (size_t)l * kVecPerLayer;
     for (int j = 0; j < D; ++j) {
       v[j] = (float)c[j];                       // c1: biases accumulated in Y so far
-      v[D + j] = (float)bq[j];
-      v[2 * D + j] = (float)bk[j];
-      v[3 * D + j] = (float)bv[j];
+      v[D + j] = L.ln1_g[j];
+      v[2 * D + j] = L.ln1_b[j];
+      v[3 * D + j] = (float)((double)L.bq[j] * (0.25 * 1.4426950408889634));
+      v[4 * D + j] = L.bk[j];
+      v[5 * D + j] = L.bv[j];
       c[j] += L.bo[j];
-      v[4 * D + j] = (float)c[j];               // c2
+      v[6 * D + j] = (float)c[j];               // c2
+      v[7 * D + j] = L.ln2_g[j];
+      v[8 * D + j] = L.ln2_b[j];
       c[j] += L.b2[j];
     }
-    for (int j = 0; j < H; ++j) v[5 * D + j] = (float)b1[j];
+    for (int j = 0; j < H; ++j) v[9 * D + j] = L.b1[j];
   }
   float* vf = vec.data() + (size_t)N * kVecPerLayer;
   double bh = w->b_head;
@@ -630,6 +692,17 @@ tr_status tc_build(tr_model* m, const tr_model_weights* w) {
   m->tc_stack_layer_bytes = (size_t)kChunksPerLayer * kChunk;
   m->tc_vec = reinterpret_cast<const float*>((uint8_t*)m->tc_blob + img_bytes);
   m->tc_vec_layer_floats = kVecPerLayer;
+  return TR_OK;
+}
+
+tr_status set_smem_attr(int dev) {
+  static bool done[64] = {};
+  if (dev < 0 || dev >= 64) return fail(TR_ERR_UNSUPPORTED, "device %d", dev);
+  if (!done[dev]) {
+    TR_CUDA_TRY(cudaFuncSetAttribute(stack_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    TR_CUDA_TRY(cudaFuncSetAttribute(stack_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    done[dev] = true;
+  }
   return TR_OK;
 }
 
@@ -669,23 +742,46 @@ tr_status tc_score(const tr_model* m, const void* tokens, int64_t n, const int64
   if ((uintptr_t)tokens % 16) return fail(TR_ERR_INVALID_ARG, "tokens not 16-byte aligned");
   p.n_tiles = tiles;
   if (tiles == 0) return TR_OK;
-  static bool attr_set[64] = {};
   int dev = 0, sms = 148;
   TR_CUDA_TRY(cudaGetDevice(&dev));
   TR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  if (!attr_set[dev]) {
-    TR_CUDA_TRY(cudaFuncSetAttribute(stack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    attr_set[dev] = true;
-  }
+  TR_TRY(set_smem_attr(dev));
   const int grid = std::min(tiles, sms);
-  stack_kernel<<<grid, 192, SMEM_BYTES, st>>>(p);
+  stack_kernel<false><<<grid, 192, SMEM_BYTES, st>>>(p);
   TR_LAUNCH_CHECK("stack_kernel");
   return TR_OK;
 }
 
-bool tc_comp_supported(const tr_model*) { return false; }
-tr_status tc_compress(const tr_model*, const void*, int64_t, void*, cudaStream_t) {
-  return fail(TR_ERR_UNSUPPORTED, "tensor-core compressor not built");
+bool tc_prefill_supported(const tr_model* m, int L_u) { return tc_stack_supported(m) && L_u <= kMaxLpTc; }
+
+// User side of one request through the same kernel (one CTA, the user tokens as its tile).
+tr_status tc_prefill(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv, cudaStream_t st) {
+  if ((uintptr_t)kv % 16 || (uintptr_t)user_tokens % 16)
+    return fail(TR_ERR_INVALID_ARG, "user_tokens / kv not 16-byte aligned");
+  DeviceState* ds = nullptr;
+  TR_TRY(device_state(&ds));
+  StackParams p{};
+  p.wimg = static_cast<const uint8_t*>(m->tc_stack);
+  p.vec = m->tc_vec;
+  p.domain_emb = m->domain_emb;
+  p.status = ds->status;
+  p.n_layer = m->desc.n_layer;
+  p.R = 1;
+  p.n_tiles = 1;
+  p.utokens = user_tokens;
+  p.kv_out = static_cast<uint8_t*>(kv);
+  p.req[0].cand_off = 0;
+  p.req[0].n = L_u;
+  p.req[0].tile_off = 0;
+  p.req[0].L_u = L_u;
+  p.req[0].domain = domain;
+  int dev = 0;
+  TR_CUDA_TRY(cudaGetDevice(&dev));
+  TR_TRY(set_smem_attr(dev));
+  stack_kernel<true><<<1, 192, SMEM_BYTES, st>>>(p);
+  TR_LAUNCH_CHECK("stack_kernel (user side)");
+  return TR_OK;
 }
+
 
 }  // namespace tr
