@@ -185,6 +185,35 @@ tr_status tr_score_candidates(const tr_model* m, const void* tokens, int64_t n,
                               tr_stream stream);
 
 /*
+ * No-allocation variant of tr_prefill_user.  The paper has no counterpart: this entry point
+ * exists for callers that cannot call cudaMalloc when the user side runs -- code running
+ * while a CUDA stream capture is open (allocation is not a capturable operation), serving
+ * engines whose own allocator owns all device memory, and latency-critical loops that cannot
+ * afford the device-wide synchronisation a growing workspace costs.  tr_prefill_user itself
+ * allocates nothing on the tensor-core path, but its CUDA-core path grows a library-owned
+ * workspace with cudaMalloc.
+ *
+ * This call runs the CUDA-core (fp32 arithmetic) user side for any model dtype, with its
+ * scratch in one file-scope device array of TR_NOALLOC_SCRATCH_BYTES that every GPU loading
+ * the library holds until process exit.  It calls no cudaMalloc, cudaFree or allocating
+ * library routine.  Arguments and output are those of tr_prefill_user; for a TR_BF16 model the
+ * result agrees with tr_prefill_user within the bf16 tolerance, not bit for bit.
+ *   Limit: L_u * (6*D + ffn_hidden) * 4 bytes <= TR_NOALLOC_SCRATCH_BYTES (with D = 128 and
+ *          ffn_hidden = 256 that is every L_u <= TR_MAX_LU); a larger request is rejected with
+ *          TR_ERR_INVALID_ARG before anything is launched.
+ *   Sharing: every call on a device uses the same array, which keeps the last call's
+ *          contents (nothing in it has to start at zero: each call writes every element it
+ *          reads).  Calls whose kernels overlap on the GPU -- different streams, or several
+ *          host threads -- race on the array; serialise them.
+ *   Set-up: the first call on each device looks up the array's device address (and may load
+ *          the library's device code) with that device current; make that first call before
+ *          any stream capture begins.
+ */
+#define TR_NOALLOC_SCRATCH_BYTES (1u << 20)
+tr_status tr_prefill_user_noalloc(const tr_model* m, const float* user_tokens, int L_u, int domain,
+                                  void* kv, tr_stream stream);
+
+/*
  * Waits for `stream` (polling, up to timeout_ms; <= 0 means no limit), then reads and
  * clears this device's status word.  Returns TR_ERR_TIMEOUT if the stream did not drain
  * in time (the status word is left untouched), TR_ERR_KEY_RANGE if a kernel reported an

@@ -10,6 +10,7 @@ LIB_PATH = os.path.join(HERE, "libtr.so")
 TR_OK, TR_ERR_INVALID_ARG, TR_ERR_UNSUPPORTED, TR_ERR_CUDA, TR_ERR_KEY_RANGE, TR_ERR_TIMEOUT, TR_ERR_NOMEM = range(7)
 TR_F32, TR_BF16 = 0, 1
 TR_MAX_TABLES, TR_MAX_REQUESTS, TR_MAX_LU = 64, 64, 256
+TR_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 _fp = C.POINTER(C.c_float)
 
@@ -45,6 +46,7 @@ SIGNATURES = {
                                C.c_int64, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
     "tr_kv_cache_bytes": (C.c_size_t, [C.c_void_p, C.c_int]),
     "tr_prefill_user": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
+    "tr_prefill_user_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
     "tr_compress_targets": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_void_p]),
     "tr_score_candidates": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.POINTER(C.c_int64),
                                       C.POINTER(C.c_void_p), C.POINTER(C.c_int32), C.POINTER(C.c_int32),

@@ -142,6 +142,15 @@ def prefill_user(model: Model, user_tokens: torch.Tensor, L_u: int, domain: int,
     return kv
 
 
+def prefill_user_noalloc(model: Model, user_tokens: torch.Tensor, L_u: int, domain: int, kv: torch.Tensor,
+                         stream=None) -> torch.Tensor:
+    """tr_prefill_user_noalloc: the user side with no device allocation, for callers that
+    cannot allocate (open stream capture, an engine that owns all device memory)."""
+    _check(L.load().tr_prefill_user_noalloc(model.handle, _ptr(user_tokens), L_u, domain, _ptr(kv),
+                                            _stream(stream)))
+    return kv
+
+
 def compress_targets(model: Model, x: torch.Tensor, tokens: torch.Tensor, stream=None) -> torch.Tensor:
     """tr_compress_targets: x [n, F*D] -> tokens [n, D] (model dtype)."""
     _check(L.load().tr_compress_targets(model.handle, _ptr(x), x.shape[0], _ptr(tokens), _stream(stream)))

@@ -85,6 +85,8 @@ tr_status tc_score(const tr_model* m, const void* tokens, int64_t n, const int64
 bool tc_comp_supported(const tr_model* m);
 tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens, cudaStream_t st);
 bool tc_prefill_supported(const tr_model* m, int L_u);
+tr_status simt_prefill_noalloc(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv,
+                               cudaStream_t st);
 tr_status tc_prefill(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv, cudaStream_t st);
 
 }  // namespace tr
@@ -249,6 +251,15 @@ tr_status tr_prefill_user(const tr_model* m, const float* user_tokens, int L_u, 
   if (!user_tokens || !kv) return fail(TR_ERR_INVALID_ARG, "null device pointer");
   if (tc_prefill_supported(m, L_u)) return tc_prefill(m, user_tokens, L_u, domain, kv, (cudaStream_t)stream);
   return simt_prefill(m, user_tokens, L_u, domain, kv, (cudaStream_t)stream);
+}
+
+tr_status tr_prefill_user_noalloc(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv,
+                                  tr_stream stream) {
+  TR_TRY(check_model_device(m));
+  if (L_u < 0 || L_u > TR_MAX_LU) return fail(TR_ERR_INVALID_ARG, "L_u=%d (need 0..%d)", L_u, TR_MAX_LU);
+  if (domain < 0 || domain >= m->desc.n_domains) return fail(TR_ERR_INVALID_ARG, "domain=%d", domain);
+  if (L_u > 0 && (!user_tokens || !kv)) return fail(TR_ERR_INVALID_ARG, "null device pointer");
+  return simt_prefill_noalloc(m, user_tokens, L_u, domain, kv, (cudaStream_t)stream);
 }
 
 tr_status tr_compress_targets(const tr_model* m, const void* x, int64_t n, void* tokens, tr_stream stream) {

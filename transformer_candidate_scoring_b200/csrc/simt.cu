@@ -6,6 +6,7 @@
 // tiled GEMM with fused bias / ReLU / residual, row LayerNorm (optionally after PReLU),
 // one-warp-per-(row, head) attention.
 #include <algorithm>
+#include <mutex>
 
 #include "model.cuh"
 
@@ -387,6 +388,55 @@ tr_status simt_score(const tr_model* m, const void* tokens, int64_t c0, int64_t 
     }
     head_rows<<<ceil_div(M, 8), 256, 0, st>>>(y, M, D, m->lnf_g, m->lnf_b, m->w_head, m->b_head, scores + r0);
     TR_LAUNCH_CHECK("head_rows");
+  }
+  return TR_OK;
+}
+
+// ---------------------------------------------------------------- user side without allocation
+// Scratch of tr_prefill_user_noalloc: a file-scope device array (every device that loads the
+// library holds it until exit).  Host code only ever sees its host-side stand-in, so each
+// device's address is looked up once, with that device current, and passed to the kernels.
+static __device__ __align__(256) float g_noalloc_scratch[TR_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+tr_status simt_prefill_noalloc(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv,
+                               cudaStream_t st) {
+  static std::mutex mu;
+  static float* scratch_of_device[64] = {};
+  const int D = m->desc.D, H = m->desc.ffn_hidden;
+  const size_t need = (size_t)L_u * (6 * D + H) * sizeof(float);
+  if (need > TR_NOALLOC_SCRATCH_BYTES)
+    return fail(TR_ERR_INVALID_ARG,
+                "tr_prefill_user_noalloc: L_u=%d needs %zu bytes of scratch, the fixed array holds %u", L_u, need,
+                (unsigned)TR_NOALLOC_SCRATCH_BYTES);
+  if (L_u == 0) return TR_OK;
+  int dev = 0;
+  TR_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(TR_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  float* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!scratch_of_device[dev]) {
+      void* p = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess)
+        return fail(TR_ERR_CUDA, "cudaGetSymbolAddress of the no-allocation scratch failed: %s", cudaGetErrorString(e));
+      scratch_of_device[dev] = static_cast<float*>(p);
+    }
+    ws = scratch_of_device[dev];
+  }
+  float *y = ws, *a = y + L_u * D, *qkv = a + L_u * D, *o = qkv + 3 * L_u * D, *hb = o + L_u * D;
+  add_vec_rows<float><<<ceil_div((int64_t)L_u * D, 256), 256, 0, st>>>(user_tokens, y, L_u, D,
+                                                                        m->domain_emb + (int64_t)domain * D);
+  TR_LAUNCH_CHECK("add_vec_rows");
+  const int Lp = round_up16(L_u);
+  for (int l = 0; l < m->desc.n_layer; ++l) {
+    void* kv_l;
+    if (m->desc.dtype == TR_F32)
+      kv_l = (float*)kv + (size_t)l * 2 * L_u * D;
+    else
+      kv_l = (__nv_bfloat16*)kv + (size_t)l * 2 * Lp * D;
+    KvF32 self_kv{qkv + D, qkv + 2 * D, 3 * D};
+    TR_TRY(layer(m, l, y, a, qkv, o, hb, L_u, self_kv, L_u, false, kv_l, st));
   }
   return TR_OK;
 }
