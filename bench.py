@@ -3,8 +3,11 @@
 
 A step is one pass of the whole scoring path over one request of the 128D-5L workload
 (40,000 candidates, L_u = 64, 8 target fields over 4M-row tables):
-  tr_aggregate(user fields) -> tr_prefill_user -> tr_aggregate(target fields)
-  -> tr_compress_targets -> tr_score_candidates.
+  [side stream] tr_aggregate(user fields) -> tr_prefill_user
+  [main stream] tr_aggregate(target fields) -> tr_compress_targets
+  -> (join) tr_score_candidates.
+Stage times come from CUDA events on the stream each stage runs on; the user side
+overlaps the target side, so the stages do not add up to the step.
 ``value`` is candidates scored per second over all ranks, with inputs resident in HBM;
 ``e2e`` repeats the step with the request's bags copied from pinned host memory and the
 scores copied back inside the timed region.  Requests rotate over several seeded request
@@ -208,23 +211,11 @@ def run_ours(args, rank, world, local_rank):
         dw.domain = [r.domain for r in reqs]
 
     stage_names = ["user_side", "target_aggregate", "compress", "score"]
+    ev_keys = ["user0", "user1", "t0", "agg", "comp", "s0", "score"]
 
     def step(i, events=None):
         use(i)
-        if events is not None:
-            events[0].record(stream)
-        dw.user_side()
-        if events is not None:
-            events[1].record(stream)
-        dw.target_aggregate()
-        if events is not None:
-            events[2].record(stream)
-        dw.compress()
-        if events is not None:
-            events[3].record(stream)
-        dw.score()
-        if events is not None:
-            events[4].record(stream)
+        dw.step(stream, events)
 
     def barrier():
         if world > 1:
@@ -238,7 +229,7 @@ def run_ours(args, rank, world, local_rank):
 
     clocks = ClockSampler(local_rank)
     clocks.start()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    ev = [{k: torch.cuda.Event(enable_timing=True) for k in ev_keys} for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     launches0 = api.kernel_launches()
@@ -253,8 +244,10 @@ def run_ours(args, rank, world, local_rank):
     launches = api.kernel_launches() - launches0
     clk = clocks.stop()
     elapsed = t0.elapsed_time(t1) / 1e3
-    stage_ms = {n: float(np.mean([ev[i][k].elapsed_time(ev[i][k + 1]) for i in range(args.steps)]))
-                for k, n in enumerate(stage_names)}
+    spans = {"user_side": ("user0", "user1"), "target_aggregate": ("t0", "agg"), "compress": ("agg", "comp"),
+             "score": ("s0", "score")}
+    stage_ms = {n: float(np.mean([ev[i][a].elapsed_time(ev[i][b]) for i in range(args.steps)]))
+                for n, (a, b) in spans.items()}
     if world > 1:
         t = torch.tensor([elapsed], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -353,6 +346,35 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_case(args):
+    """One stage of the 128D-5L path on stand-alone seeded inputs, a few launches, no JSON:
+    the target of profiler captures (small, no tables)."""
+    import torch
+
+    from transformer_candidate_scoring_b200 import api
+
+    w = datagen.WORKLOADS[WORKLOAD]
+    dims = w.dims
+    n = args.case_n
+    m = api.Model(dims, datagen.workload_params(w))
+    U = torch.from_numpy(datagen.rand_matrix(1, (64, dims.D), 0.01, "f32")).cuda()
+    kv = torch.zeros(api.kv_cache_bytes(m, 64), dtype=torch.uint8, device="cuda")
+    X = torch.from_numpy(datagen.rand_matrix(3, (n, dims.comp_dims[0]), 0.01, "bf16")).cuda().to(torch.bfloat16)
+    T = torch.empty(n, dims.D, dtype=torch.bfloat16, device="cuda")
+    s = torch.empty(n, dtype=torch.float32, device="cuda")
+    for _ in range(args.case_reps):
+        if args.case in ("prefill", "all"):
+            api.prefill_user(m, U, 64, 1, kv)
+        if args.case in ("compress", "score", "all"):
+            api.compress_targets(m, X, T)
+        if args.case in ("score", "all"):
+            api.score_candidates(m, T, [0, n], [kv], [64], [1], s)
+    torch.cuda.synchronize()
+    if api.sync_status() != 0:
+        raise RuntimeError("device status word set")
+    print(f"case {args.case}: ok")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -361,7 +383,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--case", choices=["score", "compress", "prefill", "all"], default=None,
+                    help="run one stage on stand-alone inputs for a profiler (no timing, no JSON)")
+    ap.add_argument("--case-n", type=int, default=40000)
+    ap.add_argument("--case-reps", type=int, default=2)
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -86,11 +86,14 @@ def _run_agg(tables, bags, D, out_dtype):
 
 @pytest.mark.parametrize("dt,D", [("f32", 32), ("bf16", 64), ("bf16", 128), ("f32", 128), ("bf16", 32)])
 @pytest.mark.parametrize("out_dt", ["f32", "bf16"])
-def test_aggregate_parity(dt, D, out_dt):
-    rng = np.random.default_rng(D)
+@pytest.mark.parametrize("n_bags,max_nf", [(1237, 100), (9001, 8), (6007, 70)])
+def test_aggregate_parity(dt, D, out_dt, n_bags, max_nf):
+    """Both gather kernels: few long bags and many short ones (the pipelined kernel takes
+    >= 4096 bags), bags longer than the prefetched rows and than 32 keys, empty bags."""
+    rng = np.random.default_rng(D + n_bags)
     rows = 5000
     tables = _tables(11, 3, rows, D, dt)
-    bags = _bags(rng, 1237, 100, rows, 3)
+    bags = _bags(rng, n_bags, max_nf, rows, 3)
     got = _run_agg(tables, bags, D, tdt(out_dt)).double().cpu().numpy()
     ref = _oracle_agg(11, bags, rows, D, dt)
     # fp32 accumulation error scales with the summands (table values), not with the
@@ -132,20 +135,22 @@ def test_aggregate_single_key_returns_row_exactly():
     assert torch.all(torch.abs(got - want) <= 2.0 ** -22 * torch.abs(want))
 
 
-def test_aggregate_out_of_range_key_is_skipped_and_reported():
+@pytest.mark.parametrize("n_bags", [50, 5000])
+def test_aggregate_out_of_range_key_is_skipped_and_reported(n_bags):
     rng = np.random.default_rng(7)
     tables = _tables(5, 1, 1000, 64, "bf16")
-    bags = _bags(rng, 50, 10, 1000, 1, empty_frac=0.0)
+    bags = _bags(rng, n_bags, 10, 1000, 1, empty_frac=0.0)
     bad = bags.keys.copy()
     bad[3] = 1000           # one past the end
     bad[7] = -5
+    bad[len(bad) - 2] = 2 ** 30
     got = _run_agg(tables, datagen.Bags(bags.offsets, bad, bags.weights, bags.bag_table), 64, torch.float32)
     assert tr().sync_status() == 4
     assert tr().sync_status() == 0          # the word is cleared by the read
     keep = np.ones(len(bad), bool)
-    keep[[3, 7]] = False
-    cnt = np.array([keep[bags.offsets[b]:bags.offsets[b + 1]].sum() for b in range(50)])
-    off = np.zeros(51, np.int64)
+    keep[[3, 7, len(bad) - 2]] = False
+    cnt = np.array([keep[bags.offsets[b]:bags.offsets[b + 1]].sum() for b in range(n_bags)])
+    off = np.zeros(n_bags + 1, np.int64)
     np.cumsum(cnt, out=off[1:])
     ref = _oracle_agg(5, datagen.Bags(off, bags.keys[keep], bags.weights[keep], bags.bag_table), 1000, 64, "bf16")
     np.testing.assert_allclose(got.double().cpu().numpy(), ref, rtol=1e-5, atol=1e-7)

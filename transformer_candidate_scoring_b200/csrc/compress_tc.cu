@@ -6,12 +6,14 @@
 //   layer 1: x tiles arrive by TMA tensor loads (128-byte swizzle, rows past the end are
 //            zero-filled by the copy engine) together with bulk copies of the matching
 //            W1 slice, two stages deep; the [128 x c1] fp32 accumulator fills TMEM.
-//   epilogue 1: + b1, PReLU, LayerNorm over c1 (two passes over TMEM, thread = row),
-//            bf16 result written in the core-matrix layout over the now idle stage buffers.
+//   epilogue 1: + b1, PReLU, LayerNorm over c1 (two passes over TMEM), bf16 result written
+//            in the core-matrix layout over the now idle stage buffers.
 //   layers 2, 3: W2 / W3 slices stream through a second two-stage ring.
-//   epilogue 3: + b3, bf16, one row per thread straight to global memory.
-// Warp 0 issues copies, warp 1 issues MMAs, warps 2-5 run the epilogues.  Waits are
-// bounded as in the candidate stack kernel.
+//   epilogue 3: + b3, bf16 straight to global memory.
+// Warp 0 issues copies, warp 1 issues MMAs, warps 2-9 run the epilogues: two warps per TMEM
+// lane quadrant, each owning half of a row's columns; a row's LayerNorm statistics are merged
+// across the pair (Welford) through shared memory.  Waits are bounded as in the candidate
+// stack kernel.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <string.h>
@@ -28,18 +30,22 @@ namespace {
 using namespace tc;
 
 constexpr int kM = 128;
+// Copies of the weight slices; CTA b streams copy b % kWeightCopies.  Measured on B200, more
+// than one copy did not change the kernel time, so one copy.
+constexpr int kWeightCopies = 1;
 constexpr int STAGE1 = 80 * 1024;              // x slice (16 KB) + W1 slice (<= 64 KB)
 constexpr int OFF_R1 = 0;
 constexpr int OFF_R2 = 2 * STAGE1;             // 160 KB
 constexpr int STAGE2 = 32 * 1024;
 constexpr int OFF_BAR = OFF_R2 + 2 * STAGE2;   // 224 KB
-constexpr int SMEM_BYTES = OFF_BAR + 128 + 1024;
+constexpr int SMEM_BYTES = OFF_BAR + 160 + 1024;
 
 struct CompParams {
   CUtensorMap xmap;            // x [n][c0] bf16, box {64, 128}, 128-byte swizzle
   const uint8_t* w1;           // [c0/64] slices of W1^T [c1 x 64]
   const uint8_t* w2;           // [c1/64] slices of W2^T [c2 x 64]
   const uint8_t* w3;           // [c2/64] slices of W3^T [c3 x 64]
+  size_t wcopy_bytes;          // bytes between weight copies
   const float* vec;            // b1 a1 g1 be1 (c1 each), b2 a2 g2 be2 (c2 each), b3 (c3)
   __nv_bfloat16* out;          // [n][c3]
   int* status;
@@ -48,7 +54,7 @@ struct CompParams {
 };
 
 struct CBars {
-  uint32_t full1[2], empty1[2], full2[2], empty2[2], r1_free, mma, epi, drain;
+  uint32_t full1[2], empty1[2], full2[2], empty2[2], r1_free, mma, epi, drain, qsync[4];
 };
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
@@ -68,6 +74,7 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
 __device__ void comp_producer(const CompParams& p, uint32_t r1, uint32_t r2, const CBars& b, volatile int* abort_flag) {
   int s1 = 0, s2 = 0;
   uint32_t ph1 = 0, ph2 = 0, free_phase = 0;
+  const size_t cp = (blockIdx.x % kWeightCopies) * p.wcopy_bytes;
   const uint32_t w1_bytes = p.c1 * 128, w2_bytes = p.c2 * 128, w3_bytes = p.c3 * 128;
   bool ok = true;
   bool pend1[2] = {false, false}, pend2[2] = {false, false};
@@ -81,7 +88,7 @@ __device__ void comp_producer(const CompParams& p, uint32_t r1, uint32_t r2, con
       const uint32_t st = r1 + s1 * STAGE1;
       mbar_arrive_expect_tx(b.full1[s1], kM * 64 * 2 + w1_bytes);
       tma_load_2d(st, &p.xmap, kc * 64, tile * kM, b.full1[s1]);
-      bulk_g2s(st + 16384, p.w1 + (size_t)kc * w1_bytes, w1_bytes, b.full1[s1]);
+      bulk_g2s(st + 16384, p.w1 + cp + (size_t)kc * w1_bytes, w1_bytes, b.full1[s1]);
       pend1[s1] = true;
       par1[s1] = ph1;
       if (++s1 == 2) { s1 = 0; ph1 ^= 1; }
@@ -90,7 +97,7 @@ __device__ void comp_producer(const CompParams& p, uint32_t r1, uint32_t r2, con
       if (!(ok = mbar_wait(b.empty2[s2], ph2 ^ 1, abort_flag))) break;
       const bool is2 = j < p.c1 / 64;
       const uint32_t bytes = is2 ? w2_bytes : w3_bytes;
-      const uint8_t* src = is2 ? p.w2 + (size_t)j * w2_bytes : p.w3 + (size_t)(j - p.c1 / 64) * w3_bytes;
+      const uint8_t* src = is2 ? p.w2 + cp + (size_t)j * w2_bytes : p.w3 + cp + (size_t)(j - p.c1 / 64) * w3_bytes;
       mbar_arrive_expect_tx(b.full2[s2], bytes);
       bulk_g2s(r2 + s2 * STAGE2, src, bytes, b.full2[s2]);
       pend2[s2] = true;
@@ -174,66 +181,119 @@ __device__ void comp_mma(const CompParams& p, uint32_t tmem, uint32_t r1, uint32
   }
 }
 
-// + bias, PReLU, LayerNorm over `cols` accumulator columns of this row -> bf16 operand in R1.
-__device__ __forceinline__ void prelu_ln_row(uint32_t tcol, int cols, const float* bias, const float* slope,
-                                             const float* g, const float* be, uint32_t dst_row) {
+// Epilogue threads: two warps per TMEM lane quadrant, each owning half of a row's columns.
+struct CEpi {
+  uint32_t trow, rowoff, xbuf;
+  int m, hf, q;
+  uint32_t qbar;
+  uint32_t ph_q;
+  volatile int* abort_flag;
+  bool ok;
+  // exchange one float2 with the other half of this row (slot alternates between uses)
+  __device__ float2 swap(float2 mine, int slot) {
+    const uint32_t x = xbuf + slot * (2 * kM * 8);
+    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(x + (hf * kM + m) * 8), "f"(mine.x), "f"(mine.y)
+                 : "memory");
+    mbar_arrive(qbar);
+    ok = ok && mbar_wait(qbar, ph_q, abort_flag);
+    ph_q ^= 1;
+    float2 o;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(o.x), "=f"(o.y) : "r"(x + ((1 - hf) * kM + m) * 8)
+                 : "memory");
+    return o;
+  }
+};
+
+__device__ __forceinline__ void vec8(const float* p, float* o) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+
+// + bias, PReLU, LayerNorm over the `cols` accumulator columns of this row, of which this
+// thread owns [c0, c0 + cols/2); bf16 result into the next layer's operand in R1.
+__device__ __forceinline__ void prelu_ln_half(CEpi& e, int cols, const float* bias, const float* slope,
+                                              const float* g, const float* be, uint32_t dst_row, int slot) {
+  const int half = cols / 2, c0 = e.hf * half;
+  const uint32_t tcol = e.trow + c0;
   float x0 = 0.f, s1 = 0.f, s2 = 0.f;
-  for (int c = 0; c < cols; c += 64) {
-    float v[64];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) tmem_ld16(tcol + c + 16 * q, v + 16 * q);
+  for (int c = 0; c < half; c += 32) {
+    float v[32];
+    tmem_ld16(tcol + c, v);
+    tmem_ld16(tcol + c + 16, v + 16);
     tmem_wait_ld();
-    reg_fence<64>(v);
-    if (c == 0) {
-      x0 = v[0] + __ldg(bias);
-      x0 = x0 >= 0.f ? x0 : x0 * __ldg(slope);
-    }
+    reg_fence<32>(v);
 #pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      float x = v[i] + __ldg(bias + c + i);
-      x = x >= 0.f ? x : x * __ldg(slope + c + i);
-      const float d = x - x0;
-      s1 += d;
-      s2 = fmaf(d, d, s2);
+    for (int k = 0; k < 4; ++k) {
+      float bb[8], sl[8];
+      vec8(bias + c0 + c + 8 * k, bb);
+      vec8(slope + c0 + c + 8 * k, sl);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float x = v[8 * k + i] + bb[i];
+        x = x >= 0.f ? x : x * sl[i];
+        if (c == 0 && k == 0 && i == 0) x0 = x;
+        const float d = x - x0;
+        s1 += d;
+        s2 = fmaf(d, d, s2);
+      }
     }
   }
-  const float inv_n = 1.f / cols;
-  const float dm = s1 * inv_n;
-  const float mean = x0 + dm;
-  const float rstd = rsqrtf(fmaxf(s2 * inv_n - dm * dm, 0.f) + kLnEps);
-  for (int c = 0; c < cols; c += 64) {
-    float v[64];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) tmem_ld16(tcol + c + 16 * q, v + 16 * q);
+  // this half's mean and sum of squared deviations, merged with the other half (Welford)
+  const float inv_h = 1.f / half;
+  const float mh = x0 + s1 * inv_h;
+  const float m2h = fmaxf(s2 - s1 * s1 * inv_h, 0.f);
+  const float2 o = e.swap(make_float2(mh, m2h), slot);
+  const float dmu = mh - o.x;
+  const float mean = 0.5f * (mh + o.x);
+  const float var = (m2h + o.y + dmu * dmu * (0.25f * cols)) / cols;
+  const float rstd = rsqrtf(var + kLnEps);
+  for (int c = 0; c < half; c += 32) {
+    float v[32];
+    tmem_ld16(tcol + c, v);
+    tmem_ld16(tcol + c + 16, v + 16);
     tmem_wait_ld();
-    reg_fence<64>(v);
+    reg_fence<32>(v);
 #pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      float x = v[i] + __ldg(bias + c + i);
-      x = x >= 0.f ? x : x * __ldg(slope + c + i);
-      v[i] = (x - mean) * rstd * __ldg(g + c + i) + __ldg(be + c + i);
+    for (int k = 0; k < 4; ++k) {
+      float bb[8], sl[8], gg[8], ee[8], w[8];
+      vec8(bias + c0 + c + 8 * k, bb);
+      vec8(slope + c0 + c + 8 * k, sl);
+      vec8(g + c0 + c + 8 * k, gg);
+      vec8(be + c0 + c + 8 * k, ee);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float x = v[8 * k + i] + bb[i];
+        x = x >= 0.f ? x : x * sl[i];
+        w[i] = fmaf((x - mean) * rstd, gg[i], ee[i]);
+      }
+      st_row8(dst_row + ((c0 + c) / 8 + k) * 2048, w);
     }
-#pragma unroll
-    for (int kc = 0; kc < 8; ++kc) st_row8(dst_row + ((c >> 3) + kc) * 2048, v + 8 * kc);
   }
 }
 
 __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, const CBars& b,
                               volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q = warp & 3, m = q * 32 + lane;
-  const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-  const uint32_t rowoff = (m >> 3) * 128 + (m & 7) * 16;
+  CEpi e;
+  e.q = warp & 3;
+  e.m = e.q * 32 + lane;
+  e.hf = (warp - 2) >> 2;
+  e.trow = tmem + ((uint32_t)(e.q * 32) << 16);
+  e.rowoff = (e.m >> 3) * 128 + (e.m & 7) * 16;
+  e.xbuf = r1 + 128 * 1024;      // idle between the first layer's MMAs and the next tile's loads
+  e.qbar = b.qsync[e.q];
+  e.ph_q = 0;
+  e.abort_flag = abort_flag;
+  e.ok = true;
   const float* v1 = p.vec;
   const float* v2 = p.vec + 4 * p.c1;
   const float* b3 = v2 + 4 * p.c2;
   uint32_t mma_phase = 0;
-  bool ok = true;
   auto wait_mma = [&]() {
-    ok = ok && mbar_wait(b.mma, mma_phase, abort_flag);
+    e.ok = e.ok && mbar_wait(b.mma, mma_phase, abort_flag);
     mma_phase ^= 1;
     tc_fence_after();
-    return ok;
+    return e.ok;
   };
   auto signal = [&]() {
     tmem_wait_st();
@@ -241,22 +301,26 @@ __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, c
     tc_fence_before();
     mbar_arrive(b.epi);
   };
-  for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+  for (int tile = blockIdx.x; tile < p.n_tiles && e.ok; tile += gridDim.x) {
     if (!wait_mma()) break;
-    prelu_ln_row(trow, p.c1, v1, v1 + p.c1, v1 + 2 * p.c1, v1 + 3 * p.c1, r1 + rowoff);
+    prelu_ln_half(e, p.c1, v1, v1 + p.c1, v1 + 2 * p.c1, v1 + 3 * p.c1, r1 + e.rowoff, 0);
     signal();
     if (!wait_mma()) break;
-    prelu_ln_row(trow, p.c2, v2, v2 + p.c2, v2 + 2 * p.c2, v2 + 3 * p.c2, r1 + rowoff);
+    prelu_ln_half(e, p.c2, v2, v2 + p.c2, v2 + 2 * p.c2, v2 + 3 * p.c2, r1 + e.rowoff, 1);
     signal();
     if (!wait_mma()) break;
-    const long long row = (long long)tile * kM + m;
-    for (int c = 0; c < p.c3; c += 16) {
+    const long long row = (long long)tile * kM + e.m;
+    const int h3 = p.c3 / 2;
+    for (int c = e.hf * h3; c < (e.hf + 1) * h3; c += 16) {
       float v[16];
-      tmem_ld16(trow + 256 + c, v);
+      tmem_ld16(e.trow + 256 + c, v);
       tmem_wait_ld();
       reg_fence<16>(v);
+      float bb[16];
+      vec8(b3 + c, bb);
+      vec8(b3 + c + 8, bb + 8);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] += __ldg(b3 + c + i);
+      for (int i = 0; i < 16; ++i) v[i] += bb[i];
       if (row < p.n) {
         uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.c3 + c);
         dst[0] = make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]), pack2(v[6], v[7]));
@@ -267,7 +331,7 @@ __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, c
   }
 }
 
-__global__ void __launch_bounds__(192, 1) compress_kernel(const __grid_constant__ CompParams p) {
+__global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant__ CompParams p) {
   extern __shared__ uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_u32(smem_raw);
@@ -285,8 +349,9 @@ __global__ void __launch_bounds__(192, 1) compress_kernel(const __grid_constant_
   b.mma = bar0 + 72;
   b.epi = bar0 + 80;
   b.drain = bar0 + 88;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_BAR + 112);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_BAR + 120);
+  for (int q = 0; q < 4; ++q) b.qsync[q] = bar0 + 96 + 8 * q;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_BAR + 128);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_BAR + 136);
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(b.full1[s], 1);
@@ -296,8 +361,9 @@ __global__ void __launch_bounds__(192, 1) compress_kernel(const __grid_constant_
     }
     mbar_init(b.r1_free, 1);
     mbar_init(b.mma, 1);
-    mbar_init(b.epi, 128);
+    mbar_init(b.epi, 256);
     mbar_init(b.drain, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(b.qsync[q], 64);
     *abort_flag = 0;
     mbar_fence_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.xmap)) : "memory");
@@ -355,13 +421,13 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 bool tc_comp_supported(const tr_model* m) {
   const int* c = m->desc.comp_dims;
   return m->desc.dtype == TR_BF16 && m->tc_comp && c[0] % 64 == 0 && c[1] % 64 == 0 && c[1] <= 512 &&
-         c[2] % 64 == 0 && c[2] <= 256 && c[3] % 16 == 0 && c[3] <= 256;
+         c[2] % 64 == 0 && c[2] <= 256 && c[3] % 32 == 0 && c[3] <= 256;
 }
 
 // Builds the compressor's weight slices; called from tc_build for bf16 models.
 tr_status tc_build_comp(tr_model* m, const tr_model_weights* w) {
   const int* c = m->desc.comp_dims;
-  if (!(c[0] % 64 == 0 && c[1] % 64 == 0 && c[1] <= 512 && c[2] % 64 == 0 && c[2] <= 256 && c[3] % 16 == 0 &&
+  if (!(c[0] % 64 == 0 && c[1] % 64 == 0 && c[1] <= 512 && c[2] % 64 == 0 && c[2] <= 256 && c[3] % 32 == 0 &&
         c[3] <= 256))
     return TR_OK;
   const size_t e1 = (size_t)c[0] * c[1], e2 = (size_t)c[1] * c[2], e3 = (size_t)c[2] * c[3];
@@ -379,13 +445,15 @@ tr_status tc_build_comp(tr_model* m, const tr_model_weights* w) {
     vec.insert(vec.end(), w->comp_ln_b[i], w->comp_ln_b[i] + n);
   }
   vec.insert(vec.end(), w->comp_b[2], w->comp_b[2] + c[3]);
-  const size_t ib = img.size() * 2, vb = vec.size() * 4;
+  const size_t cb = img.size() * 2, ib = cb * kWeightCopies, vb = vec.size() * 4;
   void* blob = nullptr;
   if (cudaMalloc(&blob, ib + vb) != cudaSuccess) {
     cudaGetLastError();
     return fail(TR_ERR_NOMEM, "compressor weight images: allocation failed");
   }
-  TR_CUDA_TRY(cudaMemcpy(blob, img.data(), ib, cudaMemcpyHostToDevice));
+  for (int k = 0; k < kWeightCopies; ++k)
+    TR_CUDA_TRY(cudaMemcpy((uint8_t*)blob + k * cb, img.data(), cb, cudaMemcpyHostToDevice));
+  m->tc_comp_copy_bytes = cb;
   TR_CUDA_TRY(cudaMemcpy((uint8_t*)blob + ib, vec.data(), vb, cudaMemcpyHostToDevice));
   m->tc_comp = blob;
   m->tc_comp_vec = reinterpret_cast<const float*>((uint8_t*)blob + ib);
@@ -413,6 +481,7 @@ tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens,
   p.w1 = img;
   p.w2 = img + (size_t)c[0] * c[1] * 2;
   p.w3 = p.w2 + (size_t)c[1] * c[2] * 2;
+  p.wcopy_bytes = m->tc_comp_copy_bytes;
   p.vec = m->tc_comp_vec;
   p.out = static_cast<__nv_bfloat16*>(tokens);
   p.status = ds->status;
@@ -430,7 +499,7 @@ tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens,
     TR_CUDA_TRY(cudaFuncSetAttribute(compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
     attr_set[dev] = true;
   }
-  compress_kernel<<<std::min(p.n_tiles, sms), 192, SMEM_BYTES, st>>>(p);
+  compress_kernel<<<std::min(p.n_tiles, sms), 320, SMEM_BYTES, st>>>(p);
   TR_LAUNCH_CHECK("compress_kernel");
   return TR_OK;
 }

@@ -7,24 +7,36 @@
 // The whole N-layer stack runs with the tile on chip:
 //
 //   TMEM (512 fp32 columns x 128 lanes, lane = candidate row)
-//     [  0,128)  Y, the residual stream; the O and FFN2 GEMMs accumulate into it in place
-//     [128,256)  Q accumulator -> per-head-group scores S -> FFN hidden (first half)
-//     [256,384)  K accumulator -> attention output O       -> FFN hidden (second half)
-//     [384,512)  the candidate's own V accumulator (kept until the attention epilogue)
-//   shared memory (224 KB)
-//     A      [128 x 128] bf16  LN1 output -> Q -> attention output -> LN2 output
-//     P/H    [128 x 256] bf16  softmax numerators of one head group / ReLU(FFN hidden)
-//     KV     the request's K and V^T images of the current layer (L_u <= 128)
-//     ring   4 x 16 KB weight chunks ([128 out x 64 in] slices), streamed by the TMA engine
+//     [  0,128)  Y, the residual stream; the O and FFN2 GEMMs (and their biases)
+//                accumulate into it in place
+//     [128,256)  Q accumulator -> score buffer 0 -> FFN hidden [0,128)
+//     [256,384)  K accumulator -> score buffer 1 -> FFN hidden [128,256)
+//     [384,512)  V accumulator -> attention output O (the candidate's own V moves to
+//                registers as bf16 first)
+//   shared memory
+//     A      [128 x 128] bf16  LN1 output -> Q -> attention output -> LN2 output -> hidden[128,256)
+//     P0, P1 [128 x 128] bf16  softmax numerators of a head group (double-buffered) -> P0
+//                              holds hidden[0,128); for L_u > 64 the K/V images take P1's place
+//     KV     the request's K and V^T images of the current layer
+//     ring   4 x 20 KB: a [128 out x 64 in] weight slice plus, for the last slice of a GEMM,
+//            its [128 x 16] bias tile; streamed by the TMA engine in consumption order
+//     ones   the [128 x 16] A operand that turns a bias tile into "+ bias" in one MMA
+//     vec    LayerNorm gains/shifts of every layer and the folded head weight (<= 5 layers)
 //
-// Warp roles: warp 0 issues bulk copies (weights in consumption order, the K/V images
-// once per tile and layer), warp 1 issues tcgen05.mma from one thread, warps 2-5 are the
-// epilogue (one TMEM lane quadrant each; thread = candidate row, so LayerNorm and the
-// per-head softmax need no cross-thread reduction).  LayerNorm gains/shifts and the
-// softmax scale (1/sqrt(d_h), times log2 e for exp2) are folded into the weights when the
-// model is built; the O and FFN2 biases are carried as a per-column offset of Y that the
-// next LayerNorm adds back.  Every wait is bounded: a stalled barrier sets an error bit
-// and the kernel unwinds, releasing its tensor memory.
+// Attention runs per head group (the heads whose scores fit 128 TMEM columns).  The scores of
+// group g + 2 are computed into the buffer group g just released while the epilogue works on
+// group g + 1, so the epilogue does not wait on the tensor core between groups.
+//
+// Biases: one extra K = 16 MMA per GEMM, ones[128 x 16] x bias_tile^T, where the bias tile
+// holds the bf16 head and tail of each fp32 bias (columns 0 and 1): D += b_hi + b_lo.
+//
+// Warp roles: warp 0 issues bulk copies, warp 1 issues tcgen05.mma from one thread, warps
+// 2-9 are the epilogue: two warps per TMEM lane quadrant, each owning half of the columns
+// (64 of D, i.e. four of the eight heads).  LayerNorm statistics of a row are merged across
+// the pair (Welford merge through shared memory, synchronised per quadrant); per-head
+// softmax needs no exchange unless a head's keys are split (L_u > 64).  Every wait is
+// bounded: a stalled barrier sets an error bit and the kernel unwinds, releasing its tensor
+// memory.
 #include <math.h>
 #include <string.h>
 
@@ -45,20 +57,36 @@ using namespace tc;
 
 constexpr int kD = 128, kH = 256, kM = 128;
 constexpr int kChunk = 16384;                 // [128 x 64] bf16 weight slice
+constexpr int kBiasTile = 4096;               // [128 x 16] bf16 bias tile
+constexpr int kSlot = kChunk + kBiasTile;     // one stream item
 constexpr int kStages = 4;
 constexpr int kChunksPerLayer = 16;
-constexpr int kVecPerLayer = 9 * kD + kH;     // c1, g1, be1, bq*qs, bk, bv, c2, g2, be2, b1
-constexpr float kQScale = 0.25f * 1.44269504088896341f;  // 1/sqrt(d_h) * log2(e)
-constexpr int kVecFinal = 2 * kD + 16;        // cf, w, b
+constexpr int kVecPerLayer = 4 * kD;          // LN1 gain, LN1 shift, LN2 gain, LN2 shift
+constexpr int kVecFinal = kD + 4;             // head weight * final LN gain, folded head bias
 constexpr int kMaxLpTc = 128;
+constexpr int kMaxLayersSmemVec = 5;
+constexpr int kEpiThreads = 256;
+// Copies of the weight images in global memory; CTA b streams copy b % kWeightCopies.  All
+// CTAs stream the same weights at about the same time; measured on B200, 16 copies gave the
+// same kernel time as one (the reads are not limited by L2 slice contention), so one copy.
+constexpr int kWeightCopies = 1;
+constexpr float kQScale = 0.25f * 1.44269504088896341f;  // 1/sqrt(d_h) * log2(e)
+
+__host__ __device__ constexpr bool chunk_has_bias(int c) {
+  return c == 1 || c == 3 || c == 5 || c == 7 || c == 9 || c == 11 || c == 15;
+}
 
 constexpr int OFF_A = 0;
-constexpr int OFF_PH = OFF_A + kM * kD * 2;             // 32 KB
-constexpr int OFF_KV = OFF_PH + kM * kH * 2;            // +64 KB
-constexpr int OFF_RING = OFF_KV + 2 * kMaxLpTc * kD * 2;  // +64 KB
-constexpr int OFF_BAR = OFF_RING + kStages * kChunk;    // +64 KB
-constexpr int SMEM_BYTES = OFF_BAR + 128;
-
+constexpr int OFF_P0 = 32768;
+constexpr int OFF_P1 = 65536;                               // L_u > 64: start of the K/V images
+constexpr int OFF_KV = 98304;                               // L_u <= 64
+constexpr int OFF_RING = 131072;
+constexpr int OFF_ONES = OFF_RING + kStages * kSlot;        // 208 KB
+constexpr int OFF_X = OFF_ONES + kM * 16 * 2;               // [2 slots][2 halves][128] float2
+constexpr int OFF_VEC = OFF_X + 2 * 2 * kM * 8;
+constexpr int OFF_BAR = OFF_VEC + (kMaxLayersSmemVec * kVecPerLayer + kVecFinal) * 4;
+constexpr int SMEM_BYTES = OFF_BAR + 320;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 struct ReqInfo {
   const uint8_t* kv;
@@ -73,7 +101,8 @@ struct ReqInfo {
 struct StackParams {
   const __nv_bfloat16* tokens;
   float* scores;
-  const uint8_t* wimg;       // [n_layer][16][kChunk]
+  const uint8_t* wimg;       // kWeightCopies x [n_layer][16][kSlot]
+  size_t wcopy_bytes;        // bytes between copies
   const float* vec;          // [n_layer][kVecPerLayer] + [kVecFinal]
   const float* domain_emb;   // [n_domains][D]
   int* status;
@@ -99,19 +128,63 @@ __device__ __forceinline__ TileInfo tile_info(const StackParams& p, int tile) {
   t.rows = (int)min((long long)kM, p.req[r].cand_off + p.req[r].n - t.row0);
   t.L_u = p.req[r].L_u;
   t.Lp = (t.L_u + 15) & ~15;
-  // heads per score group: the group's scores fill at most 128 TMEM columns
+  // heads per score group: a group's scores fill at most 128 TMEM columns
   t.hg = t.Lp <= 16 ? 8 : t.Lp <= 32 ? 4 : t.Lp <= 64 ? 2 : 1;
   t.ng = t.Lp == 0 ? 0 : 8 / t.hg;
   return t;
 }
 
+// Slot s of head group g holds this head.  The first half of a group's slots are heads of
+// the first column half (0-3), the second half heads 4-7, so both epilogue halves get work.
+__device__ __forceinline__ int slot_head(int g, int s, int hg) {
+  if (hg == 1) return g;
+  const int half = hg / 2;
+  return s < half ? g * half + s : 4 + g * half + (s - half);
+}
+
 struct Bars {
-  uint32_t full[kStages], empty[kStages], kv_full, kv_empty, mma, epi, drain, esync;
+  uint32_t full[kStages], empty[kStages], kv_full, kv_empty;
+  uint32_t ev_qk, ev_s[2], ev_av, ev_o, ev_h0, ev_h1, ev_y;      // MMA -> epilogue
+  uint32_t e1, e2, e3[2], e4, e5, e6a, e6b;                      // epilogue -> MMA
+  uint32_t drain, esync, qsync[4];
 };
+
+__device__ __forceinline__ Bars make_bars(uint32_t bar0) {
+  Bars b;
+  uint32_t a = bar0;
+  auto take = [&]() { const uint32_t r = a; a += 8; return r; };
+  for (int s = 0; s < kStages; ++s) b.full[s] = take();
+  for (int s = 0; s < kStages; ++s) b.empty[s] = take();
+  b.kv_full = take();
+  b.kv_empty = take();
+  b.ev_qk = take();
+  b.ev_s[0] = take();
+  b.ev_s[1] = take();
+  b.ev_av = take();
+  b.ev_o = take();
+  b.ev_h0 = take();
+  b.ev_h1 = take();
+  b.ev_y = take();
+  b.e1 = take();
+  b.e2 = take();
+  b.e3[0] = take();
+  b.e3[1] = take();
+  b.e4 = take();
+  b.e5 = take();
+  b.e6a = take();
+  b.e6b = take();
+  b.drain = take();
+  b.esync = take();
+  for (int q = 0; q < 4; ++q) b.qsync[q] = take();
+  return b;
+}
+constexpr int kBarBytes = 8 * (2 * kStages + 2 + 8 + 8 + 2 + 4);
+static_assert(kBarBytes + 16 <= 320, "barrier area");
 
 // ------------------------------------------------------------------ producer (warp 0, one thread)
 template <bool PF>
-__device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, const Bars& b, volatile int* abort_flag) {
+__device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, const Bars& b,
+                         volatile int* abort_flag) {
   int stage = 0;
   uint32_t phase = 0, kv_phase = 0;
   bool pending[kStages] = {false, false, false, false};
@@ -122,7 +195,7 @@ __device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, co
   for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
     const TileInfo t = tile_info(p, tile);
     for (int l = 0; l < p.n_layer && ok; ++l) {
-      const uint8_t* wl = p.wimg + (size_t)l * kChunksPerLayer * kChunk;
+      const uint8_t* wl = p.wimg + (blockIdx.x % kWeightCopies) * p.wcopy_bytes + (size_t)l * kChunksPerLayer * kSlot;
       for (int c = 0; c < kChunksPerLayer && ok; ++c) {
         if (!PF && c == 6) {  // the request's K/V images go in between the QKV and O weights
           if (!(ok = mbar_wait(b.kv_empty, kv_phase ^ 1, abort_flag))) break;
@@ -138,8 +211,9 @@ __device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, co
           kv_phase ^= 1;
         }
         if (!(ok = mbar_wait(b.empty[stage], phase ^ 1, abort_flag))) break;
-        mbar_arrive_expect_tx(b.full[stage], kChunk);
-        bulk_g2s(ring + stage * kChunk, wl + (size_t)c * kChunk, kChunk, b.full[stage]);
+        const uint32_t bytes = chunk_has_bias(c) ? kSlot : kChunk;
+        mbar_arrive_expect_tx(b.full[stage], bytes);
+        bulk_g2s(ring + stage * kSlot, wl + (size_t)c * kSlot, bytes, b.full[stage]);
         pending[stage] = true;
         pend_parity[stage] = phase;
         if (++stage == kStages) {
@@ -152,39 +226,43 @@ __device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, co
   if (!ok) {  // unwinding: let the copies already issued land before the CTA exits
     for (int s = 0; s < kStages; ++s)
       if (pending[s])
-        for (uint64_t t0 = globaltimer_ns(); !mbar_try_wait(b.full[s], pend_parity[s]) && globaltimer_ns() - t0 < 200000000ull;) {
+        for (uint64_t t0 = globaltimer_ns();
+             !mbar_try_wait(b.full[s], pend_parity[s]) && globaltimer_ns() - t0 < 200000000ull;) {
         }
     if (kv_pending)
-      for (uint64_t t0 = globaltimer_ns(); !mbar_try_wait(b.kv_full, kv_pend_parity) && globaltimer_ns() - t0 < 200000000ull;) {
+      for (uint64_t t0 = globaltimer_ns();
+           !mbar_try_wait(b.kv_full, kv_pend_parity) && globaltimer_ns() - t0 < 200000000ull;) {
       }
   }
 }
 
 // ------------------------------------------------------------------ MMA issuer (warp 1, one thread)
-template <bool PF>
-__device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sPH, uint32_t sKV, uint32_t ring,
-                           const Bars& b, volatile int* abort_flag) {
+template <bool PF, int HG>
+__device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sP0, uint32_t sP1,
+                           uint32_t sKV, uint32_t ring, uint32_t sOnes, const Bars& b, volatile int* abort_flag) {
   constexpr uint32_t ID128 = idesc_bf16(kM, 128);
   constexpr uint32_t ID16 = idesc_bf16(kM, 16);
   int stage = 0;
-  uint32_t phase = 0, kv_phase = 0, epi_phase = 0;
+  uint32_t phase = 0, kv_phase = 0;
+  uint32_t ph1 = 0, ph2 = 0, ph3[2] = {0, 0}, ph4 = 0, ph5 = 0, ph6a = 0, ph6b = 0;
   bool ok = true;
-  auto wait_epi = [&]() {
-    ok = ok && mbar_wait(b.epi, epi_phase, abort_flag);
-    epi_phase ^= 1;
+  auto wait_epi = [&](uint32_t bar, uint32_t& ph) {
+    ok = ok && mbar_wait(bar, ph, abort_flag);
+    ph ^= 1;
     tc_fence_after();
     return ok;
   };
-  // one [128 x 64] weight chunk against A K-steps [ks0, ks0 + 4)
-  auto chunk = [&](uint32_t a_base, int ks0, uint32_t dcol, bool acc_first) {
+  // weight slice c against A K-steps [ks0, ks0 + 4); the slice's bias tile, if any, last
+  auto chunk = [&](int c, uint32_t a_base, int ks0, uint32_t dcol, bool acc_first) {
     if (!ok) return;
     if (!(ok = mbar_wait(b.full[stage], phase, abort_flag))) return;
     tc_fence_after();
-    const uint32_t w = ring + stage * kChunk;
+    const uint32_t w = ring + stage * kSlot;
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tmem + dcol, sdesc(a_base + (ks0 + kk) * 4096, 2048, 128), sdesc(w + kk * 4096, 2048, 128), ID128,
                (kk > 0 || acc_first) ? 1u : 0u);
+    if (chunk_has_bias(c)) mma_bf16(tmem + dcol, sdesc(sOnes, 2048, 128), sdesc(w + kChunk, 2048, 128), ID128, 1u);
     mma_commit(b.empty[stage]);
     if (++stage == kStages) {
       stage = 0;
@@ -194,54 +272,74 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
   for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
     const TileInfo t = tile_info(p, tile);
     const uint32_t idS = idesc_bf16(kM, t.Lp > 0 ? t.Lp : 16);
+    // scores of head group g into TMEM buffer g % 2
+    auto issue_S = [&](int g) {
+      const int buf = g & 1;
+      for (int s = 0; s < HG; ++s) {
+        const int h = slot_head(g, s, HG);
+        mma_bf16(tmem + 128 + 128 * buf + s * t.Lp, sdesc(sA + h * 4096, 2048, 128),
+                 sdesc(sKV + 2 * h * (t.Lp / 8) * 128, (t.Lp / 8) * 128, 128), idS, 0u);
+      }
+      mma_commit(b.ev_s[buf]);
+    };
+    // O[:, head] += P_head V_head for the heads of group g
+    auto issue_AV = [&](int g) {
+      const uint32_t pbase = (HG >= 2 && (g & 1)) ? sP1 : sP0;
+      for (int s = 0; s < HG; ++s) {
+        const int h = slot_head(g, s, HG);
+        const uint32_t pb = pbase + s * t.Lp * 256;
+        const uint32_t vb = sKV + t.Lp * 256;
+        for (int kk = 0; kk < t.Lp / 16; ++kk)
+          mma_bf16(tmem + 384 + 16 * h, sdesc(pb + kk * 4096, 2048, 128),
+                   sdesc(vb + (32 * kk + 2 * h) * 128, 2048, 128), ID16, kk > 0 ? 1u : 0u);
+      }
+    };
     for (int l = 0; l < p.n_layer && ok; ++l) {
-      if (!wait_epi()) break;                         // A = LN1(y)
-      chunk(sA, 0, 128, false);                       // Q
-      chunk(sA, 4, 128, true);
-      chunk(sA, 0, 256, false);                       // K (own)
-      chunk(sA, 4, 256, true);
-      chunk(sA, 0, 384, false);                       // V (own)
-      chunk(sA, 4, 384, true);
-      mma_commit(b.mma);
-      if (!wait_epi()) break;                         // A = Q (scaled, biased)
+      if (!wait_epi(b.e1, ph1)) break;                // A = LN1(y)
+      chunk(0, sA, 0, 128, false);                    // Q + bq
+      chunk(1, sA, 4, 128, true);
+      chunk(2, sA, 0, 256, false);                    // own K + bk
+      chunk(3, sA, 4, 256, true);
+      chunk(4, sA, 0, 384, false);                    // own V + bv
+      chunk(5, sA, 4, 384, true);
+      mma_commit(b.ev_qk);
+      if (!wait_epi(b.e2, ph2)) break;                // A = Q (scaled); own V in registers
       if (!PF) {
         ok = ok && mbar_wait(b.kv_full, kv_phase, abort_flag);
         kv_phase ^= 1;
         tc_fence_after();
       }
+      if (ok && t.ng > 0) issue_S(0);
+      if (ok && HG >= 2 && t.ng > 1) issue_S(1);
       for (int g = 0; g < t.ng && ok; ++g) {
-        for (int s = 0; s < t.hg; ++s) {
-          const int h = g * t.hg + s;
-          mma_bf16(tmem + 128 + s * t.Lp, sdesc(sA + h * 4096, 2048, 128),
-                   sdesc(sKV + 2 * h * (t.Lp / 8) * 128, (t.Lp / 8) * 128, 128), idS, 0u);
-        }
-        mma_commit(b.mma);
-        if (!wait_epi()) break;                       // P of this head group in P/H
-        for (int s = 0; s < t.hg; ++s) {
-          const int h = g * t.hg + s;
-          const uint32_t pb = sPH + s * t.Lp * 256;
-          const uint32_t vb = sKV + t.Lp * 256;
-          for (int kk = 0; kk < t.Lp / 16; ++kk)
-            mma_bf16(tmem + 256 + 16 * h, sdesc(pb + kk * 4096, 2048, 128),
-                     sdesc(vb + (32 * kk + 2 * h) * 128, 2048, 128), ID16, kk > 0 ? 1u : 0u);
-        }
+        if (!wait_epi(b.e3[g & 1], ph3[g & 1])) break;   // P of group g written, its scores read
+        issue_AV(g);
+        // two P buffers: group g + 2 reuses g's score buffer; one P buffer (L_u > 64):
+        // group g + 1 is issued after group g's AV, so its P is free once its scores land
+        if (HG >= 2 && g + 2 < t.ng) issue_S(g + 2);
+        if (HG == 1 && g + 1 < t.ng) issue_S(g + 1);
       }
       if (!ok) break;
       if (!PF) mma_commit(b.kv_empty);
-      mma_commit(b.mma);
-      if (!wait_epi()) break;                         // A = attention output
-      chunk(sA, 0, 0, true);                          // Y += attn Wo
-      chunk(sA, 4, 0, true);
-      mma_commit(b.mma);
-      if (!wait_epi()) break;                         // A = LN2(y)
-      chunk(sA, 0, 128, false);                       // hidden[:, 0:128]
-      chunk(sA, 4, 128, true);
-      chunk(sA, 0, 256, false);                       // hidden[:, 128:256]
-      chunk(sA, 4, 256, true);
-      mma_commit(b.mma);
-      if (!wait_epi()) break;                         // P/H = ReLU(hidden)
-      for (int q = 0; q < 4; ++q) chunk(sPH, 4 * q, 0, true);  // Y += H W2
-      mma_commit(b.mma);
+      mma_commit(b.ev_av);
+      if (!wait_epi(b.e4, ph4)) break;                // A = attention output
+      chunk(6, sA, 0, 0, true);                       // Y += attn Wo + bo
+      chunk(7, sA, 4, 0, true);
+      mma_commit(b.ev_o);
+      if (!wait_epi(b.e5, ph5)) break;                // A = LN2(y)
+      chunk(8, sA, 0, 128, false);                    // hidden[0,128) + b1
+      chunk(9, sA, 4, 128, true);
+      mma_commit(b.ev_h0);
+      chunk(10, sA, 0, 256, false);                   // hidden[128,256) + b1
+      chunk(11, sA, 4, 256, true);
+      mma_commit(b.ev_h1);
+      if (!wait_epi(b.e6a, ph6a)) break;              // P0 = ReLU(hidden[0,128))
+      chunk(12, sP0, 0, 0, true);                     // Y += H W2, first half of K
+      chunk(13, sP0, 4, 0, true);
+      if (!wait_epi(b.e6b, ph6b)) break;              // A = ReLU(hidden[128,256))
+      chunk(14, sA, 0, 0, true);                      // second half of K, + b2
+      chunk(15, sA, 4, 0, true);
+      mma_commit(b.ev_y);
     }
   }
   // drain every MMA still in flight before the tensor memory is released
@@ -250,315 +348,422 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
   }
 }
 
-// ------------------------------------------------------------------ epilogue (warps 2-5)
-__device__ __forceinline__ void ln_rows_to_smem(float* y, uint32_t sA, int m, const float* g, const float* be) {
-  float mean = 0.f;
-#pragma unroll
-  for (int i = 0; i < kD; ++i) mean += y[i];
-  mean *= (1.f / kD);
-  float var = 0.f;
-#pragma unroll
-  for (int i = 0; i < kD; ++i) {
-    const float d = y[i] - mean;
-    var = fmaf(d, d, var);
-  }
-  const float rstd = rsqrtf(var * (1.f / kD) + kLnEps);
-  const uint32_t rowoff = (m >> 3) * 128 + (m & 7) * 16;
-#pragma unroll
-  for (int kc = 0; kc < kD / 8; ++kc) {
-    float v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = fmaf((y[kc * 8 + i] - mean) * rstd, __ldg(g + kc * 8 + i), __ldg(be + kc * 8 + i));
-    st_row8(sA + kc * 2048 + rowoff, v);
-  }
-}
+// ------------------------------------------------------------------ epilogue (warps 2-9)
+struct Epi {
+  uint32_t trow;        // TMEM address of this row, column 0
+  uint32_t rowoff;      // byte offset of this row inside a 128-row core-matrix operand
+  int m, hf, q;         // row, column half (0: columns 0-63 / heads 0-3), lane quadrant
+  uint32_t sA, sP0, sP1, sKV, sX;
+  const float* vec;     // LayerNorm vectors (shared memory copy when it fits)
+  Bars b;
+  volatile int* abort_flag;
+  bool ok;
+  uint32_t ph_qk, ph_s[2], ph_av, ph_o, ph_h0, ph_h1, ph_y, ph_sync, ph_q;
 
-__device__ __forceinline__ void load_y(uint32_t trow, float* y) {
-#pragma unroll
-  for (int c = 0; c < 8; ++c) tmem_ld16(trow + c * 16, y + c * 16);
-  tmem_wait_ld();
-  reg_fence<kD>(y);
-}
-
-// PF (user-side mode): the tile is the request's user tokens; each layer's K and V are
-// the tile's own, written to the K/V images in shared memory and stored to the cache.
-template <bool PF>
-__device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sPH, uint32_t sKV, const Bars& b,
-                         volatile int* abort_flag) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q = warp & 3;
-  const int m = q * 32 + lane;
-  const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-  const uint32_t rowoff = (m >> 3) * 128 + (m & 7) * 16;
-  uint32_t mma_phase = 0;
-  bool ok = true;
-  auto wait_mma = [&]() {
-    ok = ok && mbar_wait(b.mma, mma_phase, abort_flag);
-    mma_phase ^= 1;
+  __device__ bool wait(uint32_t bar, uint32_t& ph) {
+    ok = ok && mbar_wait(bar, ph, abort_flag);
+    ph ^= 1;
     tc_fence_after();
     return ok;
-  };
-  auto signal = [&]() {
+  }
+  __device__ void signal(uint32_t bar) {
     tmem_wait_st();
     fence_proxy_async_smem();
     tc_fence_before();
-    mbar_arrive(b.epi);
-  };
-  // rendezvous of the 128 epilogue threads (bounded, like every other wait)
-  uint32_t esync_phase = 0;
-  auto epi_sync = [&]() {
+    mbar_arrive(bar);
+  }
+  // rendezvous of the 256 epilogue threads (bounded)
+  __device__ bool sync() {
     mbar_arrive(b.esync);
-    ok = ok && mbar_wait(b.esync, esync_phase, abort_flag);
-    esync_phase ^= 1;
+    ok = ok && mbar_wait(b.esync, ph_sync, abort_flag);
+    ph_sync ^= 1;
     return ok;
-  };
-  const float* vfin = p.vec + (size_t)p.n_layer * kVecPerLayer;
-  for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-    const TileInfo t = tile_info(p, tile);
-    const float* sd = p.domain_emb + (size_t)p.req[t.r].domain * kD;
-    // Y = t + s_d; rows past the request's end are zero and never stored
-    if (PF) {
-      const float* src = p.utokens + (t.row0 + m) * kD;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float yv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) yv[i] = (m < t.rows) ? __ldg(src + c * 16 + i) + __ldg(sd + c * 16 + i) : 0.f;
-        tmem_st16(trow + c * 16, yv);
-      }
-      tmem_wait_st();
-    } else {
-      const uint4* src = reinterpret_cast<const uint4*>(p.tokens + (t.row0 + m) * kD);
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float yv[16];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const uint4 u = (m < t.rows) ? __ldg(src + 2 * c + hh) : make_uint4(0, 0, 0, 0);
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int col = c * 16 + hh * 8 + 2 * i;
-            yv[hh * 8 + 2 * i] = (m < t.rows) ? __uint_as_float(w[i] << 16) + __ldg(sd + col) : 0.f;
-            yv[hh * 8 + 2 * i + 1] = (m < t.rows) ? __uint_as_float(w[i] & 0xFFFF0000u) + __ldg(sd + col + 1) : 0.f;
-          }
-        }
-        tmem_st16(trow + c * 16, yv);
-      }
-      tmem_wait_st();
-    }
+  }
+  // exchange one float2 with the other column half of this row through exchange slot
+  // `slot`; consecutive exchanges inside one phase must alternate slots
+  __device__ float2 swap(float2 mine, int slot) {
+    const uint32_t x = sX + slot * (2 * kM * 8);
+    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(x + (hf * kM + m) * 8), "f"(mine.x), "f"(mine.y)
+                 : "memory");
+    mbar_arrive(b.qsync[q]);
+    ok = ok && mbar_wait(b.qsync[q], ph_q, abort_flag);
+    ph_q ^= 1;
+    float2 o;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(o.x), "=f"(o.y) : "r"(x + ((1 - hf) * kM + m) * 8)
+                 : "memory");
+    return o;
+  }
+};
 
-    for (int l = 0; l < p.n_layer && ok; ++l) {
-      const float* vl = p.vec + (size_t)l * kVecPerLayer;
-      const float *c1 = vl, *g1 = vl + kD, *be1 = vl + 2 * kD, *bq = vl + 3 * kD, *bk = vl + 4 * kD, *bv = vl + 5 * kD;
-      const float *c2 = vl + 6 * kD, *g2 = vl + 7 * kD, *be2 = vl + 8 * kD, *b1 = vl + 9 * kD;
-      // ---- LN1
-      if (l > 0 && !wait_mma()) break;            // FFN2 of the previous layer done
-      {
-        float y[kD];
-        load_y(trow, y);
+// Compiler-only barrier: keeps the loads of the next step from being hoisted above it, so
+// that per-column vectors are not all held in registers at once.
+__device__ __forceinline__ void step_barrier() { asm volatile("" ::: "memory"); }
+
+__device__ __forceinline__ void load64(uint32_t taddr, float* v) {
 #pragma unroll
-        for (int i = 0; i < kD; ++i) y[i] += __ldg(c1 + i);
-        ln_rows_to_smem(y, sA, m, g1, be1);
-      }
-      signal();
-      // ---- Q, own K: the candidate's own score per head; Q to A
-      if (!wait_mma()) break;
-      float sself[8];
-      if (PF && threadIdx.x == 64 && l > 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-      if (PF && !epi_sync()) break;               // the K/V images are free to overwrite
-      for (int h = 0; h < 8; ++h) {
-        float qv[16], kv[16];
-        tmem_ld16(trow + 128 + 16 * h, qv);
-        tmem_ld16(trow + 256 + 16 * h, kv);
-        tmem_wait_ld();
-        reg_fence<16>(qv);
-        reg_fence<16>(kv);
-        float s = 0.f;
+  for (int c = 0; c < 4; ++c) tmem_ld16(taddr + c * 16, v + c * 16);
+  tmem_wait_ld();
+  reg_fence<64>(v);
+}
+
+// Row mean / rstd of a 128-wide row held as two 64-column halves (Welford merge).
+__device__ __forceinline__ float2 row_stats(Epi& e, const float* y) {
+  float mean = 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          qv[i] = fmaf(qv[i], kQScale, __ldg(bq + 16 * h + i));
-          kv[i] += __ldg(bk + 16 * h + i);
-          s = fmaf(qv[i], kv[i], s);
-        }
-        sself[h] = PF ? -INFINITY : s;
-        st_row8(sA + (2 * h) * 2048 + rowoff, qv);
-        st_row8(sA + (2 * h + 1) * 2048 + rowoff, qv + 8);
-        if (PF) {
-          // K image row m, V^T image column m (zero past L_u); the TMEM load is
-          // warp-wide, only the stores depend on the row
-          float vv[16];
-          tmem_ld16(trow + 384 + 16 * h, vv);
-          tmem_wait_ld();
-          reg_fence<16>(vv);
-          if (m < t.Lp) {
-            const bool live = m < t.L_u;
+  for (int i = 0; i < 64; ++i) mean += y[i];
+  mean *= (1.f / 64);
+  float m2 = 0.f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              kv[i] = live ? kv[i] : 0.f;
-              vv[i] = live ? vv[i] + __ldg(bv + 16 * h + i) : 0.f;
-            }
-            const uint32_t kb = sKV + (m >> 3) * 128 + (m & 7) * 16;
-            st_row8(kb + (2 * h) * (t.Lp / 8) * 128, kv);
-            st_row8(kb + (2 * h + 1) * (t.Lp / 8) * 128, kv + 8);
-            const uint32_t vb = sKV + t.Lp * 256 + (m >> 3) * 2048 + (m & 7) * 2;
+  for (int i = 0; i < 64; ++i) m2 = fmaf(y[i] - mean, y[i] - mean, m2);
+  const float2 o = e.swap(make_float2(mean, m2), 0);
+  const float d = mean - o.x;
+  const float mu = 0.5f * (mean + o.x);
+  const float var = (m2 + o.y + d * d * 32.f) * (1.f / kD);
+  return make_float2(mu, rsqrtf(var + kLnEps));
+}
+
+// LayerNorm of this thread's 64 columns -> bf16 into the A operand.
+__device__ __forceinline__ void ln_to_A(Epi& e, const float* y, const float* gamma, const float* beta) {
+  const float2 st = row_stats(e, y);
+  const float4* g4 = reinterpret_cast<const float4*>(gamma + 64 * e.hf);
+  const float4* b4 = reinterpret_cast<const float4*>(beta + 64 * e.hf);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int d = 16 * h + i;
-              const __nv_bfloat16 hv = __float2bfloat16_rn(vv[i]);
-              asm volatile("st.shared.b16 [%0], %1;" ::"r"(vb + (d >> 3) * 128 + (d & 7) * 16),
-                           "h"(*reinterpret_cast<const unsigned short*>(&hv))
-                           : "memory");
-            }
-          }
-        }
-      }
-      if (PF) {  // store this layer's K/V images to the cache with one bulk copy
-        fence_proxy_async_smem();
-        if (!epi_sync()) break;
-        if (threadIdx.x == 64) {
-          const uint32_t bytes = 2u * t.Lp * kD * 2u;
-          asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
-                           p.kv_out + (size_t)l * bytes),
-                       "r"(sKV), "r"(bytes)
-                       : "memory");
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-        }
-      }
-      signal();
-      // ---- softmax over [user keys of the request, own key], one head group at a time
-      float pself[8], linv[8];
+  for (int kc = 0; kc < 8; ++kc) {
+    const float4 ga = g4[2 * kc], gb = g4[2 * kc + 1];
+    const float4 ba = b4[2 * kc], bb = b4[2 * kc + 1];
+    const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+    const float bbv[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+    float v[8];
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        pself[h] = 1.f;
-        linv[h] = 1.f;
-      }
-      for (int g = 0; g < t.ng && ok; ++g) {
-        if (!wait_mma()) break;
-        for (int s = 0; s < t.hg; ++s) {
-          const int h = g * t.hg + s;
-          // two passes over the head's scores in TMEM: the row max, then exp2 / sum / P
-          const uint32_t scol = trow + 128 + s * t.Lp;
-          float mx = sself[h];
-          for (int c = 0; c < t.Lp / 16; ++c) {
-            float sv[16];
-            tmem_ld16(scol + c * 16, sv);
-            tmem_wait_ld();
-            reg_fence<16>(sv);
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              if (c * 16 + i < t.L_u) mx = fmaxf(mx, sv[i]);
-          }
-          float sum = 0.f;
-          const uint32_t pb = sPH + s * t.Lp * 256 + rowoff;
-          for (int c = 0; c < t.Lp / 16; ++c) {
-            float sv[16];
-            tmem_ld16(scol + c * 16, sv);
-            tmem_wait_ld();
-            reg_fence<16>(sv);
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float e = (c * 16 + i < t.L_u) ? ex2(sv[i] - mx) : 0.f;
-              sv[i] = e;
-              sum += e;
-            }
-            st_row8(pb + (2 * c) * 2048, sv);
-            st_row8(pb + (2 * c + 1) * 2048, sv + 8);
-          }
-          pself[h] = ex2(sself[h] - mx);
-          linv[h] = 1.f / (sum + pself[h]);
-        }
-        signal();
-      }
-      if (!ok) break;
-      // ---- attention output = (sum_j p_j v_j + p_self v_self) / l, to A
-      if (!wait_mma()) break;
-      for (int h = 0; h < 8; ++h) {
-        float o[16], v[16];
-        tmem_ld16(trow + 256 + 16 * h, o);
-        tmem_ld16(trow + 384 + 16 * h, v);
-        tmem_wait_ld();
-        reg_fence<16>(o);
-        reg_fence<16>(v);
-        const float ps = pself[h], li = linv[h];
-        const bool has_users = t.ng > 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float vs = v[i] + __ldg(bv + 16 * h + i);
-          o[i] = ((has_users ? o[i] : 0.f) + ps * vs) * li;
-        }
-        st_row8(sA + (2 * h) * 2048 + rowoff, o);
-        st_row8(sA + (2 * h + 1) * 2048 + rowoff, o + 8);
-      }
-      signal();
-      // ---- LN2
-      if (!wait_mma()) break;                     // Y += attn Wo done
-      {
-        float y[kD];
-        load_y(trow, y);
-#pragma unroll
-        for (int i = 0; i < kD; ++i) y[i] += __ldg(c2 + i);
-        ln_rows_to_smem(y, sA, m, g2, be2);
-      }
-      signal();
-      // ---- ReLU(hidden + b1) to P/H
-      if (!wait_mma()) break;
-      for (int c = 0; c < kH / 16; ++c) {
-        float hv[16];
-        tmem_ld16(trow + 128 + 16 * c, hv);
-        tmem_wait_ld();
-        reg_fence<16>(hv);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) hv[i] = fmaxf(hv[i] + __ldg(b1 + 16 * c + i), 0.f);
-        st_row8(sPH + (2 * c) * 2048 + rowoff, hv);
-        st_row8(sPH + (2 * c + 1) * 2048 + rowoff, hv + 8);
-      }
-      signal();
-    }
-    if (!ok) break;
-    // ---- head: w . LN_f(y) + b
-    if (!wait_mma()) break;
-    if (PF) continue;
-    float y[kD];
-    load_y(trow, y);
-    float mean = 0.f;
-#pragma unroll
-    for (int i = 0; i < kD; ++i) {
-      y[i] += __ldg(vfin + i);
-      mean += y[i];
-    }
-    mean *= (1.f / kD);
-    float var = 0.f;
-#pragma unroll
-    for (int i = 0; i < kD; ++i) var = fmaf(y[i] - mean, y[i] - mean, var);
-    const float rstd = rsqrtf(var * (1.f / kD) + kLnEps);
-    float acc = 0.f;
-#pragma unroll
-    for (int i = 0; i < kD; ++i) acc = fmaf((y[i] - mean) * rstd, __ldg(vfin + kD + i), acc);
-    if (m < t.rows) p.scores[t.row0 + m] = acc + __ldg(vfin + 2 * kD);
+    for (int i = 0; i < 8; ++i) v[i] = fmaf((y[kc * 8 + i] - st.x) * st.y, gg[i], bbv[i]);
+    st_row8(e.sA + (8 * e.hf + kc) * 2048 + e.rowoff, v);
+    step_barrier();
   }
 }
 
-template <bool PF>
-__global__ void __launch_bounds__(192, 1) stack_kernel(const __grid_constant__ StackParams p) {
+// ReLU of 64 accumulator columns -> bf16 into an operand (its K-chunks kc0 .. kc0 + 7).
+__device__ __forceinline__ void relu_to(Epi& e, uint32_t tcol, uint32_t dst, int kc0) {
+  float v[64];
+  load64(tcol, v);
+#pragma unroll
+  for (int kc = 0; kc < 8; ++kc) {
+    float w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w[i] = fmaxf(v[kc * 8 + i], 0.f);
+    st_row8(dst + (kc0 + kc) * 2048 + e.rowoff, w);
+  }
+}
+
+template <bool PF, int HG>
+__device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t, Epi& e) {
+  constexpr int NG = 8 / HG;
+  constexpr int SV = HG == 8 ? 16 : HG == 4 ? 32 : 64;   // keys one thread holds for one head
+  const int hf = e.hf, m = e.m;
+  const uint32_t ycol = e.trow + 64 * hf;
+  const float* sd = p.domain_emb + (size_t)p.req[t.r].domain * kD + 64 * hf;
+  // ---- Y = t + s_d (rows past the request's end are zero and never stored)
+  {
+    float y[64];
+    const float4* sd4 = reinterpret_cast<const float4*>(sd);
+    const bool live = m < t.rows;
+    if (PF) {
+      const float4* src = reinterpret_cast<const float4*>(p.utokens + (t.row0 + m) * kD + 64 * hf);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const float4 u = live ? __ldg(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 d = __ldg(sd4 + c);
+        y[4 * c] = live ? u.x + d.x : 0.f;
+        y[4 * c + 1] = live ? u.y + d.y : 0.f;
+        y[4 * c + 2] = live ? u.z + d.z : 0.f;
+        y[4 * c + 3] = live ? u.w + d.w : 0.f;
+        step_barrier();
+      }
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(p.tokens + (t.row0 + m) * kD + 64 * hf);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 u = live ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+        const float4 da = __ldg(sd4 + 2 * c), db = __ldg(sd4 + 2 * c + 1);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        const float d[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          y[c * 8 + 2 * i] = live ? __uint_as_float(w[i] << 16) + d[2 * i] : 0.f;
+          y[c * 8 + 2 * i + 1] = live ? __uint_as_float(w[i] & 0xFFFF0000u) + d[2 * i + 1] : 0.f;
+        }
+        step_barrier();
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_st16(ycol + 16 * c, y + 16 * c);
+    tmem_wait_st();
+  }
+
+  for (int l = 0; l < p.n_layer; ++l) {
+    const float* vl = e.vec + (size_t)l * kVecPerLayer;
+    // ---- LN1 -> A
+    if (l > 0 && !e.wait(e.b.ev_y, e.ph_y)) return;
+    {
+      float y[64];
+      load64(ycol, y);
+      ln_to_A(e, y, vl, vl + kD);
+    }
+    e.signal(e.b.e1);
+    // ---- Q (scaled) -> A; own score per head; own V -> registers; user side: K/V images
+    if (!e.wait(e.b.ev_qk, e.ph_qk)) return;
+    if (PF) {
+      if (threadIdx.x == 64 && l > 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      if (!e.sync()) return;                       // the K/V images are free to overwrite
+    }
+    float sself[4];
+    uint32_t vself[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int h = 4 * hf + j;
+      float qv[16], kv[16], vv[16];
+      tmem_ld16(e.trow + 128 + 16 * h, qv);
+      tmem_ld16(e.trow + 256 + 16 * h, kv);
+      tmem_ld16(e.trow + 384 + 16 * h, vv);
+      tmem_wait_ld();
+      reg_fence<16>(qv);
+      reg_fence<16>(kv);
+      reg_fence<16>(vv);
+      float s = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        qv[i] *= kQScale;
+        s = fmaf(qv[i], kv[i], s);
+      }
+      sself[j] = PF ? -INFINITY : s;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) vself[j][i] = pack2(vv[2 * i], vv[2 * i + 1]);
+      st_row8(e.sA + (2 * h) * 2048 + e.rowoff, qv);
+      st_row8(e.sA + (2 * h + 1) * 2048 + e.rowoff, qv + 8);
+      if (PF && m < t.Lp) {
+        // K image row m, V^T image column m (zero past L_u)
+        const bool live = m < t.L_u;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          kv[i] = live ? kv[i] : 0.f;
+          vv[i] = live ? vv[i] : 0.f;
+        }
+        const uint32_t kb = e.sKV + (m >> 3) * 128 + (m & 7) * 16;
+        st_row8(kb + (2 * h) * (t.Lp / 8) * 128, kv);
+        st_row8(kb + (2 * h + 1) * (t.Lp / 8) * 128, kv + 8);
+        const uint32_t vb = e.sKV + t.Lp * 256 + (m >> 3) * 2048 + (m & 7) * 2;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int d = 16 * h + i;
+          const __nv_bfloat16 hv = __float2bfloat16_rn(vv[i]);
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(vb + (d >> 3) * 128 + (d & 7) * 16),
+                       "h"(*reinterpret_cast<const unsigned short*>(&hv))
+                       : "memory");
+        }
+      }
+    }
+    if (PF) {  // store this layer's K/V images to the cache with one bulk copy
+      fence_proxy_async_smem();
+      if (!e.sync()) return;
+      if (threadIdx.x == 64) {
+        const uint32_t bytes = 2u * t.Lp * kD * 2u;
+        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(p.kv_out + (size_t)l * bytes),
+                     "r"(e.sKV), "r"(bytes)
+                     : "memory");
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
+    }
+    e.signal(e.b.e2);
+    // ---- softmax over [user keys of the request, own key], one head group at a time
+    float pself[4] = {1.f, 1.f, 1.f, 1.f}, linv[4] = {1.f, 1.f, 1.f, 1.f};
+    if constexpr (HG >= 2) {
+#pragma unroll
+      for (int g = 0; g < NG; ++g) {
+        if (g >= t.ng) break;
+        if (!e.wait(e.b.ev_s[g & 1], e.ph_s[g & 1])) return;
+        const uint32_t sbuf = e.trow + 128 + 128 * (g & 1);
+        const uint32_t pbuf = (g & 1) ? e.sP1 : e.sP0;
+#pragma unroll
+        for (int j = 0; j < HG / 2; ++j) {
+          const int jj = g * (HG / 2) + j;          // this half's head index (0..3)
+          const int slot = hf * (HG / 2) + j;
+          float sv[SV];
+#pragma unroll
+          for (int c = 0; c < SV / 16; ++c)
+            if (c < t.Lp / 16) tmem_ld16(sbuf + slot * t.Lp + 16 * c, sv + 16 * c);
+          tmem_wait_ld();
+          reg_fence<SV>(sv);
+          float mx = sself[jj];
+#pragma unroll
+          for (int i = 0; i < SV; ++i)
+            if (i < t.L_u) mx = fmaxf(mx, sv[i]);
+          float sum = 0.f;
+#pragma unroll
+          for (int i = 0; i < SV; ++i) {
+            const float ev = (i < t.L_u) ? ex2(sv[i] - mx) : 0.f;
+            sv[i] = ev;
+            sum += ev;
+          }
+          const uint32_t pb = pbuf + slot * t.Lp * 256 + e.rowoff;
+#pragma unroll
+          for (int jc = 0; jc < SV / 8; ++jc)
+            if (jc < t.Lp / 8) st_row8(pb + jc * 2048, sv + 8 * jc);
+          pself[jj] = ex2(sself[jj] - mx);
+          linv[jj] = 1.f / (sum + pself[jj]);
+        }
+        e.signal(e.b.e3[g & 1]);
+      }
+    } else {
+      // L_u > 64: one head per group, its keys split between the two column halves
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        if (!e.wait(e.b.ev_s[g & 1], e.ph_s[g & 1])) return;
+        const uint32_t sbuf = e.trow + 128 + 128 * (g & 1);
+        const int k0 = 64 * hf;
+        const int nk = min(64, t.Lp - k0);       // > 0: Lp >= 80
+        float sv[64];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c < nk / 16) tmem_ld16(sbuf + k0 + 16 * c, sv + 16 * c);
+        tmem_wait_ld();
+        reg_fence<64>(sv);
+        const bool owner = (g >> 2) == hf;       // this half owns head g (and its own score)
+        float mx = owner ? sself[g & 3] : -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (i < nk && k0 + i < t.L_u) mx = fmaxf(mx, sv[i]);
+        mx = fmaxf(mx, e.swap(make_float2(mx, 0.f), 0).x);
+        float sum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float ev = (i < nk && k0 + i < t.L_u) ? ex2(sv[i] - mx) : 0.f;
+          sv[i] = ev;
+          sum += ev;
+        }
+        const uint32_t pb = e.sP0 + e.rowoff + (k0 / 8) * 2048;
+#pragma unroll
+        for (int jc = 0; jc < 8; ++jc)
+          if (jc < nk / 8) st_row8(pb + jc * 2048, sv + 8 * jc);
+        const float ps = owner ? ex2(sself[g & 3] - mx) : 0.f;
+        const float tot = sum + ps + e.swap(make_float2(sum + ps, 0.f), 1).x;
+        if (owner) {
+          pself[g & 3] = ps;
+          linv[g & 3] = 1.f / tot;
+        }
+        e.signal(e.b.e3[g & 1]);
+      }
+    }
+    // ---- attention output = (sum_j p_j v_j + p_self v_self) / l  -> A
+    if (!e.wait(e.b.ev_av, e.ph_av)) return;
+    const bool has_users = t.ng > 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int h = 4 * hf + j;
+      float o[16];
+      tmem_ld16(e.trow + 384 + 16 * h, o);
+      tmem_wait_ld();
+      reg_fence<16>(o);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t w = vself[j][i];
+        const float v0 = __uint_as_float(w << 16), v1 = __uint_as_float(w & 0xFFFF0000u);
+        o[2 * i] = ((has_users ? o[2 * i] : 0.f) + pself[j] * v0) * linv[j];
+        o[2 * i + 1] = ((has_users ? o[2 * i + 1] : 0.f) + pself[j] * v1) * linv[j];
+      }
+      st_row8(e.sA + (2 * h) * 2048 + e.rowoff, o);
+      st_row8(e.sA + (2 * h + 1) * 2048 + e.rowoff, o + 8);
+    }
+    e.signal(e.b.e4);
+    // ---- LN2 -> A
+    if (!e.wait(e.b.ev_o, e.ph_o)) return;
+    {
+      float y[64];
+      load64(ycol, y);
+      ln_to_A(e, y, vl + 2 * kD, vl + 3 * kD);
+    }
+    e.signal(e.b.e5);
+    // ---- ReLU(hidden) -> P0 (first half of the hidden units) and A (second half)
+    if (!e.wait(e.b.ev_h0, e.ph_h0)) return;
+    relu_to(e, e.trow + 128 + 64 * hf, e.sP0, 8 * hf);
+    e.signal(e.b.e6a);
+    if (!e.wait(e.b.ev_h1, e.ph_h1)) return;
+    relu_to(e, e.trow + 256 + 64 * hf, e.sA, 8 * hf);
+    e.signal(e.b.e6b);
+  }
+  // ---- head: w . LN_f(y) + b
+  if (!e.wait(e.b.ev_y, e.ph_y)) return;
+  if (PF) return;
+  float y[64];
+  load64(ycol, y);
+  const float2 st = row_stats(e, y);
+  const float* vf = e.vec + (size_t)p.n_layer * kVecPerLayer;
+  const float4* w4 = reinterpret_cast<const float4*>(vf + 64 * hf);
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float4 w = w4[i];
+    acc = fmaf((y[4 * i] - st.x) * st.y, w.x, acc);
+    acc = fmaf((y[4 * i + 1] - st.x) * st.y, w.y, acc);
+    acc = fmaf((y[4 * i + 2] - st.x) * st.y, w.z, acc);
+    acc = fmaf((y[4 * i + 3] - st.x) * st.y, w.w, acc);
+    step_barrier();
+  }
+  const float tot = acc + e.swap(make_float2(acc, 0.f), 1).x;
+  if (hf == 0 && m < t.rows) p.scores[t.row0 + m] = tot + vf[kD];
+}
+
+template <bool PF, int HG>
+__device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sP0, uint32_t sP1, uint32_t sKV,
+                         uint32_t sX, uint32_t sOnes, float* svec, const Bars& b, volatile int* abort_flag) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Epi e;
+  e.q = warp & 3;
+  e.m = e.q * 32 + lane;
+  e.hf = (warp - 2) >> 2;
+  e.trow = tmem + ((uint32_t)(e.q * 32) << 16);
+  e.rowoff = (e.m >> 3) * 128 + (e.m & 7) * 16;
+  e.sA = sA;
+  e.sP0 = sP0;
+  e.sP1 = sP1;
+  e.sKV = sKV;
+  e.sX = sX;
+  e.b = b;
+  e.abort_flag = abort_flag;
+  e.ok = true;
+  e.ph_qk = e.ph_s[0] = e.ph_s[1] = e.ph_av = e.ph_o = e.ph_h0 = e.ph_h1 = e.ph_y = e.ph_sync = e.ph_q = 0;
+  // the constant ones tile: columns 0 and 1 of every row are 1 (bias head and tail)
+  if (e.hf == 0) {
+    const float one2[8] = {1.f, 1.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, zero[8] = {};
+    st_row8(sOnes + e.rowoff, one2);
+    st_row8(sOnes + 2048 + e.rowoff, zero);
+  }
+  // LayerNorm vectors and the head weight: a shared-memory copy when they fit
+  const int nvec = p.n_layer * kVecPerLayer + kVecFinal;
+  if (p.n_layer <= kMaxLayersSmemVec) {
+    const int tid = threadIdx.x - 64;
+    for (int i = tid; i < nvec; i += kEpiThreads) svec[i] = __ldg(p.vec + i);
+    if (!e.sync()) return;
+    e.vec = svec;
+  } else {
+    e.vec = p.vec;
+  }
+  for (int tile = blockIdx.x; tile < p.n_tiles && e.ok; tile += gridDim.x) {
+    const TileInfo t = tile_info(p, tile);
+    epi_tile<PF, HG>(p, t, e);   // the host launches one kernel per head-group size
+  }
+}
+
+template <bool PF, int HG>
+__global__ void __launch_bounds__(64 + kEpiThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base = smem_u32(smem);
-  const uint32_t sA = base + OFF_A, sPH = base + OFF_PH, sKV = base + OFF_KV, ring = base + OFF_RING;
-  const uint32_t bar0 = base + OFF_BAR;
-  Bars b;
-  for (int s = 0; s < kStages; ++s) {
-    b.full[s] = bar0 + 8 * s;
-    b.empty[s] = bar0 + 8 * (kStages + s);
-  }
-  b.kv_full = bar0 + 8 * (2 * kStages);
-  b.kv_empty = b.kv_full + 8;
-  b.mma = b.kv_full + 16;
-  b.epi = b.kv_full + 24;
-  b.drain = b.kv_full + 32;
-  b.esync = b.kv_full + 40;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 112);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_BAR + 120);
+  const uint32_t sA = base + OFF_A, sP0 = base + OFF_P0, sP1 = base + OFF_P1, ring = base + OFF_RING;
+  const uint32_t sKV = base + (HG == 1 ? OFF_P1 : OFF_KV);
+  const uint32_t sOnes = base + OFF_ONES, sX = base + OFF_X;
+  float* svec = reinterpret_cast<float*>(smem + OFF_VEC);
+  const Bars b = make_bars(base + OFF_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + kBarBytes);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_BAR + kBarBytes + 8);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -567,10 +772,10 @@ __global__ void __launch_bounds__(192, 1) stack_kernel(const __grid_constant__ S
     }
     mbar_init(b.kv_full, 1);
     mbar_init(b.kv_empty, 1);
-    mbar_init(b.mma, 1);
-    mbar_init(b.epi, 128);
-    mbar_init(b.drain, 1);
-    mbar_init(b.esync, 128);
+    for (uint32_t a : {b.ev_qk, b.ev_s[0], b.ev_s[1], b.ev_av, b.ev_o, b.ev_h0, b.ev_h1, b.ev_y, b.drain})
+      mbar_init(a, 1);
+    for (uint32_t a : {b.e1, b.e2, b.e3[0], b.e3[1], b.e4, b.e5, b.e6a, b.e6b, b.esync}) mbar_init(a, kEpiThreads);
+    for (int q = 0; q < 4; ++q) mbar_init(b.qsync[q], 64);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -586,9 +791,9 @@ __global__ void __launch_bounds__(192, 1) stack_kernel(const __grid_constant__ S
   if (warp == 0) {
     if (lane == 0) producer<PF>(p, ring, sKV, b, abort_flag);
   } else if (warp == 1) {
-    if (lane == 0) mma_issuer<PF>(p, tmem, sA, sPH, sKV, ring, b, abort_flag);
+    if (lane == 0) mma_issuer<PF, HG>(p, tmem, sA, sP0, sP1, sKV, ring, sOnes, b, abort_flag);
   } else {
-    epilogue<PF>(p, tmem, sA, sPH, sKV, b, abort_flag);
+    epilogue<PF, HG>(p, tmem, sA, sP0, sP1, sKV, sX, sOnes, svec, b, abort_flag);
     if (PF && threadIdx.x == 64) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
   tc_fence_before();
@@ -600,20 +805,37 @@ __global__ void __launch_bounds__(192, 1) stack_kernel(const __grid_constant__ S
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, STATUS_KERNEL_TIMEOUT);
 }
 
-// ------------------------------------------------------------------ host: weight folding and images
+// ------------------------------------------------------------------ host: operand images
+
+uint16_t bf16_bits(float f) {
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  u = (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;  // round to nearest even
+  return (uint16_t)u;
+}
+float bf16_value(uint16_t h) {
+  const uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
 
 // W^T slice [n0, n0+128) x [k0, k0+64) of W [K][N] (row-major, W[k][n]) in core-matrix layout.
-void put_chunk(uint16_t* dst, const std::vector<double>& W, int N, int n0, int k0) {
+void put_chunk(uint16_t* dst, const float* W, int N, int n0, int k0) {
   for (int n = 0; n < 128; ++n)
-    for (int k = 0; k < 64; ++k) {
-      const double v = W[(size_t)(k0 + k) * N + (n0 + n)];
-      const size_t off = ((size_t)(k / 8) * 16 + n / 8) * 64 + (n % 8) * 8 + (k % 8);
-      const float f = (float)v;
-      uint32_t u;
-      memcpy(&u, &f, 4);
-      u = (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;  // round to nearest even
-      dst[off] = (uint16_t)u;
-    }
+    for (int k = 0; k < 64; ++k)
+      dst[((size_t)(k / 8) * 16 + n / 8) * 64 + (n % 8) * 8 + (k % 8)] = bf16_bits(W[(size_t)(k0 + k) * N + n0 + n]);
+}
+
+// Bias tile [128 x 16]: column 0 the bf16 nearest to b[n0+n], column 1 the bf16 of the rest.
+void put_bias(uint16_t* dst, const float* bias, int n0) {
+  for (int n = 0; n < 128; ++n) {
+    const float v = bias[n0 + n];
+    const uint16_t hi = bf16_bits(v);
+    const uint16_t lo = bf16_bits(v - bf16_value(hi));
+    for (int k = 0; k < 16; ++k)
+      dst[((size_t)(k / 8) * 16 + n / 8) * 64 + (n % 8) * 8 + (k % 8)] = k == 0 ? hi : k == 1 ? lo : 0;
+  }
 }
 
 }  // namespace
@@ -630,79 +852,90 @@ tr_status tc_build(tr_model* m, const tr_model_weights* w) {
   TR_TRY(tc_build_comp(m, w));
   if (!(d.dtype == TR_BF16 && d.D == kD && d.ffn_hidden == kH && d.n_head == 8)) return TR_OK;
   const int N = d.n_layer, D = kD, H = kH;
-  std::vector<uint16_t> img((size_t)N * kChunksPerLayer * kChunk / 2);
+  const size_t se = kSlot / 2;  // elements per stream slot
+  std::vector<uint16_t> img((size_t)N * kChunksPerLayer * se, 0);
   std::vector<float> vec((size_t)N * kVecPerLayer + kVecFinal, 0.f);
-  std::vector<double> c(D, 0.0);
-  auto dvec = [](const float* p, size_t n) { return std::vector<double>(p, p + n); };
   for (int l = 0; l < N; ++l) {
-    // the weights go in unchanged (exact bf16 values); LayerNorm gains/shifts, biases and
-    // the softmax scale stay fp32 and are applied by the epilogue
+    // weights go in unchanged (exact bf16 values); LayerNorm gains/shifts stay fp32 in the
+    // epilogue; biases become bias tiles next to the last slice of their GEMM
     const tr_layer_weights& L = w->layers[l];
-    const auto Wq = dvec(L.Wq, D * D), Wk = dvec(L.Wk, D * D), Wv = dvec(L.Wv, D * D), Wo = dvec(L.Wo, D * D);
-    const auto W1 = dvec(L.W1, D * H), W2 = dvec(L.W2, H * D);
-    uint16_t* li = img.data() + (size_t)l * kChunksPerLayer * kChunk / 2;
-    const size_t ce = kChunk / 2;
-    put_chunk(li + 0 * ce, Wq, D, 0, 0);
-    put_chunk(li + 1 * ce, Wq, D, 0, 64);
-    put_chunk(li + 2 * ce, Wk, D, 0, 0);
-    put_chunk(li + 3 * ce, Wk, D, 0, 64);
-    put_chunk(li + 4 * ce, Wv, D, 0, 0);
-    put_chunk(li + 5 * ce, Wv, D, 0, 64);
-    put_chunk(li + 6 * ce, Wo, D, 0, 0);
-    put_chunk(li + 7 * ce, Wo, D, 0, 64);
-    put_chunk(li + 8 * ce, W1, H, 0, 0);
-    put_chunk(li + 9 * ce, W1, H, 0, 64);
-    put_chunk(li + 10 * ce, W1, H, 128, 0);
-    put_chunk(li + 11 * ce, W1, H, 128, 64);
-    for (int q = 0; q < 4; ++q) put_chunk(li + (12 + q) * ce, W2, D, 0, 64 * q);
+    uint16_t* li = img.data() + (size_t)l * kChunksPerLayer * se;
+    auto slot = [&](int c) { return li + (size_t)c * se; };
+    auto bias = [&](int c) { return li + (size_t)c * se + kChunk / 2; };
+    put_chunk(slot(0), L.Wq, D, 0, 0);
+    put_chunk(slot(1), L.Wq, D, 0, 64);
+    put_bias(bias(1), L.bq, 0);
+    put_chunk(slot(2), L.Wk, D, 0, 0);
+    put_chunk(slot(3), L.Wk, D, 0, 64);
+    put_bias(bias(3), L.bk, 0);
+    put_chunk(slot(4), L.Wv, D, 0, 0);
+    put_chunk(slot(5), L.Wv, D, 0, 64);
+    put_bias(bias(5), L.bv, 0);
+    put_chunk(slot(6), L.Wo, D, 0, 0);
+    put_chunk(slot(7), L.Wo, D, 0, 64);
+    put_bias(bias(7), L.bo, 0);
+    put_chunk(slot(8), L.W1, H, 0, 0);
+    put_chunk(slot(9), L.W1, H, 0, 64);
+    put_bias(bias(9), L.b1, 0);
+    put_chunk(slot(10), L.W1, H, 128, 0);
+    put_chunk(slot(11), L.W1, H, 128, 64);
+    put_bias(bias(11), L.b1, 128);
+    for (int q = 0; q < 4; ++q) put_chunk(slot(12 + q), L.W2, D, 0, 64 * q);
+    put_bias(bias(15), L.b2, 0);
     float* v = vec.data() + (size_t)l * kVecPerLayer;
     for (int j = 0; j < D; ++j) {
-      v[j] = (float)c[j];                       // c1: biases accumulated in Y so far
-      v[D + j] = L.ln1_g[j];
-      v[2 * D + j] = L.ln1_b[j];
-      v[3 * D + j] = (float)((double)L.bq[j] * (0.25 * 1.4426950408889634));
-      v[4 * D + j] = L.bk[j];
-      v[5 * D + j] = L.bv[j];
-      c[j] += L.bo[j];
-      v[6 * D + j] = (float)c[j];               // c2
-      v[7 * D + j] = L.ln2_g[j];
-      v[8 * D + j] = L.ln2_b[j];
-      c[j] += L.b2[j];
+      v[j] = L.ln1_g[j];
+      v[D + j] = L.ln1_b[j];
+      v[2 * D + j] = L.ln2_g[j];
+      v[3 * D + j] = L.ln2_b[j];
     }
-    for (int j = 0; j < H; ++j) v[9 * D + j] = L.b1[j];
   }
   float* vf = vec.data() + (size_t)N * kVecPerLayer;
   double bh = w->b_head;
   for (int j = 0; j < D; ++j) {
-    vf[j] = (float)c[j];
-    vf[D + j] = (float)((double)w->w_head[j] * w->lnf_g[j]);
+    vf[j] = (float)((double)w->w_head[j] * w->lnf_g[j]);
     bh += (double)w->w_head[j] * w->lnf_b[j];
   }
-  vf[2 * D] = (float)bh;
-  const size_t img_bytes = img.size() * 2, vec_bytes = vec.size() * 4;
+  vf[D] = (float)bh;
+  const size_t copy_bytes = img.size() * 2, vec_bytes = vec.size() * 4;
+  const size_t img_bytes = copy_bytes * kWeightCopies;
   const size_t total = img_bytes + ((vec_bytes + 255) & ~size_t(255));
   if (cudaMalloc(&m->tc_blob, total) != cudaSuccess) {
     cudaGetLastError();
     return fail(TR_ERR_NOMEM, "tensor-core weight images: allocation of %zu bytes failed", total);
   }
   m->tc_bytes = total;
-  TR_CUDA_TRY(cudaMemcpy(m->tc_blob, img.data(), img_bytes, cudaMemcpyHostToDevice));
+  for (int k = 0; k < kWeightCopies; ++k)
+    TR_CUDA_TRY(cudaMemcpy((uint8_t*)m->tc_blob + k * copy_bytes, img.data(), copy_bytes, cudaMemcpyHostToDevice));
   TR_CUDA_TRY(cudaMemcpy((uint8_t*)m->tc_blob + img_bytes, vec.data(), vec_bytes, cudaMemcpyHostToDevice));
   m->tc_stack = m->tc_blob;
-  m->tc_stack_layer_bytes = (size_t)kChunksPerLayer * kChunk;
+  m->tc_stack_copy_bytes = copy_bytes;
+  m->tc_stack_layer_bytes = (size_t)kChunksPerLayer * kSlot;
   m->tc_vec = reinterpret_cast<const float*>((uint8_t*)m->tc_blob + img_bytes);
   m->tc_vec_layer_floats = kVecPerLayer;
   return TR_OK;
 }
 
-tr_status set_smem_attr(int dev) {
-  static bool done[64] = {};
+int hg_of(int L_u) {
+  const int Lp = (L_u + 15) & ~15;
+  return Lp <= 16 ? 8 : Lp <= 32 ? 4 : Lp <= 64 ? 2 : 1;
+}
+
+template <bool PF>
+tr_status launch_stack(int hg, int grid, const StackParams& p, cudaStream_t st) {
+  static bool done[64][4] = {};
+  int dev = 0;
+  TR_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return fail(TR_ERR_UNSUPPORTED, "device %d", dev);
-  if (!done[dev]) {
-    TR_CUDA_TRY(cudaFuncSetAttribute(stack_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    TR_CUDA_TRY(cudaFuncSetAttribute(stack_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    done[dev] = true;
+  const int hi = hg == 8 ? 0 : hg == 4 ? 1 : hg == 2 ? 2 : 3;
+  void (*k)(StackParams) = hg == 8 ? stack_kernel<PF, 8> : hg == 4 ? stack_kernel<PF, 4>
+                         : hg == 2 ? stack_kernel<PF, 2> : stack_kernel<PF, 1>;
+  if (!done[dev][hi]) {
+    TR_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
+    done[dev][hi] = true;
   }
+  k<<<grid, 64 + kEpiThreads, SMEM_BYTES, st>>>(p);
+  TR_LAUNCH_CHECK(PF ? "stack_kernel (user side)" : "stack_kernel");
   return TR_OK;
 }
 
@@ -718,37 +951,42 @@ tr_status tc_score(const tr_model* m, const void* tokens, int64_t n, const int64
   }
   DeviceState* ds = nullptr;
   TR_TRY(device_state(&ds));
-  StackParams p{};
-  p.tokens = static_cast<const __nv_bfloat16*>(tokens);
-  p.scores = scores;
-  p.wimg = static_cast<const uint8_t*>(m->tc_stack);
-  p.vec = m->tc_vec;
-  p.domain_emb = m->domain_emb;
-  p.status = ds->status;
-  p.n_layer = m->desc.n_layer;
-  p.R = R;
-  int tiles = 0;
-  for (int r = 0; r < R; ++r) {
-    const int64_t nr = req_offsets[r + 1] - req_offsets[r];
-    p.req[r].kv = static_cast<const uint8_t*>(kv[r]);
-    p.req[r].cand_off = req_offsets[r];
-    p.req[r].n = nr;
-    p.req[r].tile_off = tiles;
-    p.req[r].L_u = L_u[r];
-    p.req[r].domain = domain[r];
-    if ((uintptr_t)kv[r] % 16 && L_u[r] > 0 && nr > 0) return fail(TR_ERR_INVALID_ARG, "kv[%d] is not 16-byte aligned", r);
-    tiles += (int)((nr + kM - 1) / kM);
-  }
   if ((uintptr_t)tokens % 16) return fail(TR_ERR_INVALID_ARG, "tokens not 16-byte aligned");
-  p.n_tiles = tiles;
-  if (tiles == 0) return TR_OK;
-  int dev = 0, sms = 148;
+  for (int r = 0; r < R; ++r)
+    if ((uintptr_t)kv[r] % 16 && L_u[r] > 0 && req_offsets[r + 1] > req_offsets[r])
+      return fail(TR_ERR_INVALID_ARG, "kv[%d] is not 16-byte aligned", r);
+  int sms = 148, dev = 0;
   TR_CUDA_TRY(cudaGetDevice(&dev));
   TR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  TR_TRY(set_smem_attr(dev));
-  const int grid = std::min(tiles, sms);
-  stack_kernel<false><<<grid, 192, SMEM_BYTES, st>>>(p);
-  TR_LAUNCH_CHECK("stack_kernel");
+  // one launch per head-group size (requests of one class share the kernel's code path)
+  for (int hg : {2, 1, 4, 8}) {
+    StackParams p{};
+    p.tokens = static_cast<const __nv_bfloat16*>(tokens);
+    p.scores = scores;
+    p.wimg = static_cast<const uint8_t*>(m->tc_stack);
+    p.wcopy_bytes = m->tc_stack_copy_bytes;
+    p.vec = m->tc_vec;
+    p.domain_emb = m->domain_emb;
+    p.status = ds->status;
+    p.n_layer = m->desc.n_layer;
+    int tiles = 0, k = 0;
+    for (int r = 0; r < R; ++r) {
+      const int64_t nr = req_offsets[r + 1] - req_offsets[r];
+      if (hg_of(L_u[r]) != hg || nr == 0) continue;
+      p.req[k].kv = static_cast<const uint8_t*>(kv[r]);
+      p.req[k].cand_off = req_offsets[r];
+      p.req[k].n = nr;
+      p.req[k].tile_off = tiles;
+      p.req[k].L_u = L_u[r];
+      p.req[k].domain = domain[r];
+      tiles += (int)((nr + kM - 1) / kM);
+      ++k;
+    }
+    if (tiles == 0) continue;
+    p.R = k;
+    p.n_tiles = tiles;
+    TR_TRY(launch_stack<false>(hg, std::min(tiles, sms), p, st));
+  }
   return TR_OK;
 }
 
@@ -762,6 +1000,7 @@ tr_status tc_prefill(const tr_model* m, const float* user_tokens, int L_u, int d
   TR_TRY(device_state(&ds));
   StackParams p{};
   p.wimg = static_cast<const uint8_t*>(m->tc_stack);
+  p.wcopy_bytes = m->tc_stack_copy_bytes;
   p.vec = m->tc_vec;
   p.domain_emb = m->domain_emb;
   p.status = ds->status;
@@ -775,13 +1014,7 @@ tr_status tc_prefill(const tr_model* m, const float* user_tokens, int L_u, int d
   p.req[0].tile_off = 0;
   p.req[0].L_u = L_u;
   p.req[0].domain = domain;
-  int dev = 0;
-  TR_CUDA_TRY(cudaGetDevice(&dev));
-  TR_TRY(set_smem_attr(dev));
-  stack_kernel<true><<<1, 192, SMEM_BYTES, st>>>(p);
-  TR_LAUNCH_CHECK("stack_kernel (user side)");
-  return TR_OK;
+  return launch_stack<true>(hg_of(L_u), 1, p, st);
 }
-
 
 }  // namespace tr

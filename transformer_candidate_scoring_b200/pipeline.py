@@ -125,9 +125,37 @@ class DeviceWorkload:
         api.score_candidates(self.model, self.tokens, self.req_offsets, self.kv, self.L_u, self.domain,
                              self.scores, stream=stream)
 
-    def step(self, stream=None) -> torch.Tensor:
-        self.user_side(stream)
-        self.target_aggregate(stream)
-        self.compress(stream)
-        self.score(stream)
+    def step(self, stream=None, events=None) -> torch.Tensor:
+        """One request batch.  The user side (aggregation + prefill, one CTA per request)
+        runs on a side stream concurrently with the target aggregation and compression; the
+        scoring waits for both.  ``events``: optional dict of CUDA events recorded at stage
+        boundaries (keys user0, user1 on the side stream; t0, agg, comp, s0, score on the main)."""
+        main = stream if stream is not None else torch.cuda.current_stream(self.device)
+        if not hasattr(self, "_side"):
+            self._side = torch.cuda.Stream(self.device)
+        side = self._side
+        fork = torch.cuda.Event()
+        fork.record(main)
+        side.wait_event(fork)
+        if events:
+            events["user0"].record(side)
+        self.user_side(side)
+        if events:
+            events["user1"].record(side)
+        join = torch.cuda.Event()
+        join.record(side)
+        if events:
+            events["t0"].record(main)
+        self.target_aggregate(main)
+        if events:
+            events["agg"].record(main)
+        self.compress(main)
+        if events:
+            events["comp"].record(main)
+        main.wait_event(join)
+        if events:
+            events["s0"].record(main)
+        self.score(main)
+        if events:
+            events["score"].record(main)
         return self.scores
