@@ -188,15 +188,16 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
-    from transformer_candidate_scoring_b200 import api, build
+    from transformer_candidate_scoring_b200 import api
     from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload
+    from transformer_candidate_scoring_b200.shard import max_over_ranks, rank_seed
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = datagen.WORKLOADS[WORKLOAD]
     dims = w.dims
     # distinct request sets per rank and per step (seeded)
-    sets = [datagen.make_requests(w, seed=w.seed * 1000 + rank * 100 + s) for s in range(N_REQUEST_SETS)]
+    sets = [datagen.make_requests(w, seed=rank_seed(w.seed, rank, s)) for s in range(N_REQUEST_SETS)]
     dw = DeviceWorkload(w, device=dev, reqs=sets[0])
     dsets = []
     for reqs in sets:
@@ -248,10 +249,7 @@ def run_ours(args, rank, world, local_rank):
              "score": ("s0", "score")}
     stage_ms = {n: float(np.mean([ev[i][a].elapsed_time(ev[i][b]) for i in range(args.steps)]))
                 for n, (a, b) in spans.items()}
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(elapsed)
     n_cand = dw.n_cand
     value = n_cand * args.steps * world / elapsed
 
@@ -289,10 +287,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     e2e_elapsed = e0.elapsed_time(e1) / 1e3
-    if world > 1:
-        t = torch.tensor([e2e_elapsed], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_elapsed = float(t.item())
+    e2e_elapsed = max_over_ranks(e2e_elapsed)
     e2e_value = n_cand * args.steps * world / e2e_elapsed
 
     # ---- rooflines of the stages

@@ -18,8 +18,8 @@
 //     P0, P1 [128 x 128] bf16  softmax numerators of a head group (double-buffered) -> P0
 //                              holds hidden[0,128); for L_u > 64 the K/V images take P1's place
 //     KV     the request's K and V^T images of the current layer
-//     ring   4 x 20 KB: a [128 out x 64 in] weight slice plus, for the last slice of a GEMM,
-//            its [128 x 16] bias tile; streamed by the TMA engine in consumption order
+//     ring   2 x 36 KB: a [128 out x 128 in] weight block plus its [128 x 16] bias tile;
+//            streamed by the TMA engine in consumption order
 //     ones   the [128 x 16] A operand that turns a bias tile into "+ bias" in one MMA
 //     vec    LayerNorm gains/shifts of every layer and the folded head weight (<= 5 layers)
 //
@@ -30,8 +30,9 @@
 // Biases: one extra K = 16 MMA per GEMM, ones[128 x 16] x bias_tile^T, where the bias tile
 // holds the bf16 head and tail of each fp32 bias (columns 0 and 1): D += b_hi + b_lo.
 //
-// Warp roles: warp 0 issues bulk copies, warp 1 issues tcgen05.mma from one thread, warps
-// 2-9 are the epilogue: two warps per TMEM lane quadrant, each owning half of the columns
+// Warp roles: warp 0 issues bulk copies, warp 1 issues tcgen05.mma from one thread (warps 2
+// and 3 only complete that warpgroup and hand their registers over), warps 4-11 are the
+// epilogue: two warps per TMEM lane quadrant, each owning half of the columns
 // (64 of D, i.e. four of the eight heads).  LayerNorm statistics of a row are merged across
 // the pair (Welford merge through shared memory, synchronised per quadrant); per-head
 // softmax needs no exchange unless a head's keys are split (L_u > 64).  Every wait is
@@ -56,32 +57,43 @@ namespace {
 using namespace tc;
 
 constexpr int kD = 128, kH = 256, kM = 128;
-constexpr int kChunk = 16384;                 // [128 x 64] bf16 weight slice
+constexpr int kChunk = 16384;                 // [128 out x 64 in] bf16 weight slice
 constexpr int kBiasTile = 4096;               // [128 x 16] bf16 bias tile
-constexpr int kSlot = kChunk + kBiasTile;     // one stream item
-constexpr int kStages = 4;
-constexpr int kChunksPerLayer = 16;
+// One stream item: a [128 out x 128 in] weight block (two slices) plus its bias tile.  On
+// B200 a bulk copy costs about the same time per copy from 16 to 64 KB (a few hundred
+// cycles each, copies of one SM largely serialised), so items are as large as the ring
+// allows.
+constexpr int kSlot = 2 * kChunk + kBiasTile;
+constexpr int kStages = 2;
+constexpr int kItemsPerLayer = 8;
 constexpr int kVecPerLayer = 4 * kD;          // LN1 gain, LN1 shift, LN2 gain, LN2 shift
 constexpr int kVecFinal = kD + 4;             // head weight * final LN gain, folded head bias
 constexpr int kMaxLpTc = 128;
 constexpr int kMaxLayersSmemVec = 5;
 constexpr int kEpiThreads = 256;
+// Warps 0-3 (one warpgroup): bulk-copy producer, MMA issuer, two idle warps; warps 4-11:
+// the epilogue.  The control warpgroup gives registers to the epilogue (setmaxnreg), so
+// the epilogue runs without spills: 4 x 32 x kCtlRegs + 8 x 32 x kEpiRegs <= 384 x 168.
+constexpr int kThreads = 128 + kEpiThreads;
+constexpr int kEpiThread0 = 128;
+constexpr int kCtlRegs = 104, kEpiRegs = 200;
+static_assert(4 * 32 * kCtlRegs + 8 * 32 * kEpiRegs <= kThreads * 168, "register split exceeds the launch");
 // Copies of the weight images in global memory; CTA b streams copy b % kWeightCopies.  All
 // CTAs stream the same weights at about the same time; measured on B200, 16 copies gave the
 // same kernel time as one (the reads are not limited by L2 slice contention), so one copy.
 constexpr int kWeightCopies = 1;
 constexpr float kQScale = 0.25f * 1.44269504088896341f;  // 1/sqrt(d_h) * log2(e)
 
-__host__ __device__ constexpr bool chunk_has_bias(int c) {
-  return c == 1 || c == 3 || c == 5 || c == 7 || c == 9 || c == 11 || c == 15;
-}
+// Items: Wq, Wk, Wv, Wo, W1 (output columns 0-127), W1 (128-255), W2 (input rows 0-127),
+// W2 (rows 128-255); every item but the first half of W2 carries its GEMM's bias tile.
+__host__ __device__ constexpr bool item_has_bias(int j) { return j != 6; }
 
 constexpr int OFF_A = 0;
 constexpr int OFF_P0 = 32768;
 constexpr int OFF_P1 = 65536;                               // L_u > 64: start of the K/V images
 constexpr int OFF_KV = 98304;                               // L_u <= 64
 constexpr int OFF_RING = 131072;
-constexpr int OFF_ONES = OFF_RING + kStages * kSlot;        // 208 KB
+constexpr int OFF_ONES = OFF_RING + kStages * kSlot;        // 200 KB
 constexpr int OFF_X = OFF_ONES + kM * 16 * 2;               // [2 slots][2 halves][128] float2
 constexpr int OFF_VEC = OFF_X + 2 * 2 * kM * 8;
 constexpr int OFF_BAR = OFF_VEC + (kMaxLayersSmemVec * kVecPerLayer + kVecFinal) * 4;
@@ -142,43 +154,37 @@ __device__ __forceinline__ int slot_head(int g, int s, int hg) {
   return s < half ? g * half + s : 4 + g * half + (s - half);
 }
 
+// The CTA's mbarriers, 8 bytes apart from one base address (offsets are compile-time, so
+// the issuing threads hold one register for all of them).
 struct Bars {
-  uint32_t full[kStages], empty[kStages], kv_full, kv_empty;
-  uint32_t ev_qk, ev_s[2], ev_av, ev_o, ev_h0, ev_h1, ev_y;      // MMA -> epilogue
-  uint32_t e1, e2, e3[2], e4, e5, e6a, e6b;                      // epilogue -> MMA
-  uint32_t drain, esync, qsync[4];
+  uint32_t base;
+  __device__ __forceinline__ uint32_t at(int i) const { return base + 8u * (uint32_t)i; }
+  __device__ __forceinline__ uint32_t full(int s) const { return at(s); }
+  __device__ __forceinline__ uint32_t empty(int s) const { return at(kStages + s); }
+  __device__ __forceinline__ uint32_t kv_full() const { return at(2 * kStages); }
+  __device__ __forceinline__ uint32_t kv_empty() const { return at(2 * kStages + 1); }
+  // MMA -> epilogue
+  __device__ __forceinline__ uint32_t ev_qk() const { return at(2 * kStages + 2); }
+  __device__ __forceinline__ uint32_t ev_s(int i) const { return at(2 * kStages + 3 + i); }
+  __device__ __forceinline__ uint32_t ev_av() const { return at(2 * kStages + 5); }
+  __device__ __forceinline__ uint32_t ev_o() const { return at(2 * kStages + 6); }
+  __device__ __forceinline__ uint32_t ev_h0() const { return at(2 * kStages + 7); }
+  __device__ __forceinline__ uint32_t ev_h1() const { return at(2 * kStages + 8); }
+  __device__ __forceinline__ uint32_t ev_y() const { return at(2 * kStages + 9); }
+  // epilogue -> MMA
+  __device__ __forceinline__ uint32_t e1() const { return at(2 * kStages + 10); }
+  __device__ __forceinline__ uint32_t e2() const { return at(2 * kStages + 11); }
+  __device__ __forceinline__ uint32_t e3(int i) const { return at(2 * kStages + 12 + i); }
+  __device__ __forceinline__ uint32_t e4() const { return at(2 * kStages + 14); }
+  __device__ __forceinline__ uint32_t e5() const { return at(2 * kStages + 15); }
+  __device__ __forceinline__ uint32_t e6a() const { return at(2 * kStages + 16); }
+  __device__ __forceinline__ uint32_t e6b() const { return at(2 * kStages + 17); }
+  __device__ __forceinline__ uint32_t drain() const { return at(2 * kStages + 18); }
+  __device__ __forceinline__ uint32_t esync() const { return at(2 * kStages + 19); }
+  __device__ __forceinline__ uint32_t qsync(int q) const { return at(2 * kStages + 20 + q); }
 };
-
-__device__ __forceinline__ Bars make_bars(uint32_t bar0) {
-  Bars b;
-  uint32_t a = bar0;
-  auto take = [&]() { const uint32_t r = a; a += 8; return r; };
-  for (int s = 0; s < kStages; ++s) b.full[s] = take();
-  for (int s = 0; s < kStages; ++s) b.empty[s] = take();
-  b.kv_full = take();
-  b.kv_empty = take();
-  b.ev_qk = take();
-  b.ev_s[0] = take();
-  b.ev_s[1] = take();
-  b.ev_av = take();
-  b.ev_o = take();
-  b.ev_h0 = take();
-  b.ev_h1 = take();
-  b.ev_y = take();
-  b.e1 = take();
-  b.e2 = take();
-  b.e3[0] = take();
-  b.e3[1] = take();
-  b.e4 = take();
-  b.e5 = take();
-  b.e6a = take();
-  b.e6b = take();
-  b.drain = take();
-  b.esync = take();
-  for (int q = 0; q < 4; ++q) b.qsync[q] = take();
-  return b;
-}
-constexpr int kBarBytes = 8 * (2 * kStages + 2 + 8 + 8 + 2 + 4);
+constexpr int kNumBars = 2 * kStages + 24;
+constexpr int kBarBytes = 8 * kNumBars;
 static_assert(kBarBytes + 16 <= 320, "barrier area");
 
 // ------------------------------------------------------------------ producer (warp 0, one thread)
@@ -187,35 +193,34 @@ __device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, co
                          volatile int* abort_flag) {
   int stage = 0;
   uint32_t phase = 0, kv_phase = 0;
-  bool pending[kStages] = {false, false, false, false};
-  uint32_t pend_parity[kStages] = {0, 0, 0, 0};
+  uint32_t pending = 0, pend_parity = 0;       // bit s: slot s has a copy in flight / its parity
   bool kv_pending = false;
   uint32_t kv_pend_parity = 0;
   bool ok = true;
   for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
     const TileInfo t = tile_info(p, tile);
     for (int l = 0; l < p.n_layer && ok; ++l) {
-      const uint8_t* wl = p.wimg + (blockIdx.x % kWeightCopies) * p.wcopy_bytes + (size_t)l * kChunksPerLayer * kSlot;
-      for (int c = 0; c < kChunksPerLayer && ok; ++c) {
-        if (!PF && c == 6) {  // the request's K/V images go in between the QKV and O weights
-          if (!(ok = mbar_wait(b.kv_empty, kv_phase ^ 1, abort_flag))) break;
+      const uint8_t* wl = p.wimg + (blockIdx.x % kWeightCopies) * p.wcopy_bytes + (size_t)l * kItemsPerLayer * kSlot;
+      for (int j = 0; j < kItemsPerLayer && ok; ++j) {
+        if (!PF && j == 3) {  // the request's K/V images go in between the QKV and O weights
+          if (!(ok = mbar_wait(b.kv_empty(), kv_phase ^ 1, abort_flag))) break;
           const uint32_t bytes = 2u * t.Lp * kD * 2u;
           if (bytes) {
-            mbar_arrive_expect_tx(b.kv_full, bytes);
-            bulk_g2s(kvbuf, p.req[t.r].kv + (size_t)l * bytes, bytes, b.kv_full);
+            mbar_arrive_expect_tx(b.kv_full(), bytes);
+            bulk_g2s(kvbuf, p.req[t.r].kv + (size_t)l * bytes, bytes, b.kv_full());
             kv_pending = true;
             kv_pend_parity = kv_phase;
           } else {
-            mbar_arrive(b.kv_full);
+            mbar_arrive(b.kv_full());
           }
           kv_phase ^= 1;
         }
-        if (!(ok = mbar_wait(b.empty[stage], phase ^ 1, abort_flag))) break;
-        const uint32_t bytes = chunk_has_bias(c) ? kSlot : kChunk;
-        mbar_arrive_expect_tx(b.full[stage], bytes);
-        bulk_g2s(ring + stage * kSlot, wl + (size_t)c * kSlot, bytes, b.full[stage]);
-        pending[stage] = true;
-        pend_parity[stage] = phase;
+        if (!(ok = mbar_wait(b.empty(stage), phase ^ 1, abort_flag))) break;
+        const uint32_t bytes = item_has_bias(j) ? kSlot : 2 * kChunk;
+        mbar_arrive_expect_tx(b.full(stage), bytes);
+        bulk_g2s(ring + stage * kSlot, wl + (size_t)j * kSlot, bytes, b.full(stage));
+        pending |= 1u << stage;
+        pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == kStages) {
           stage = 0;
           phase ^= 1;
@@ -225,13 +230,13 @@ __device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, co
   }
   if (!ok) {  // unwinding: let the copies already issued land before the CTA exits
     for (int s = 0; s < kStages; ++s)
-      if (pending[s])
+      if ((pending >> s) & 1u)
         for (uint64_t t0 = globaltimer_ns();
-             !mbar_try_wait(b.full[s], pend_parity[s]) && globaltimer_ns() - t0 < 200000000ull;) {
+             !mbar_try_wait(b.full(s), (pend_parity >> s) & 1u) && globaltimer_ns() - t0 < 200000000ull;) {
         }
     if (kv_pending)
       for (uint64_t t0 = globaltimer_ns();
-           !mbar_try_wait(b.kv_full, kv_pend_parity) && globaltimer_ns() - t0 < 200000000ull;) {
+           !mbar_try_wait(b.kv_full(), kv_pend_parity) && globaltimer_ns() - t0 < 200000000ull;) {
       }
   }
 }
@@ -244,7 +249,7 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
   constexpr uint32_t ID16 = idesc_bf16(kM, 16);
   int stage = 0;
   uint32_t phase = 0, kv_phase = 0;
-  uint32_t ph1 = 0, ph2 = 0, ph3[2] = {0, 0}, ph4 = 0, ph5 = 0, ph6a = 0, ph6b = 0;
+  uint32_t ph1 = 0, ph2 = 0, ph3a = 0, ph3b = 0, ph4 = 0, ph5 = 0, ph6a = 0, ph6b = 0;
   bool ok = true;
   auto wait_epi = [&](uint32_t bar, uint32_t& ph) {
     ok = ok && mbar_wait(bar, ph, abort_flag);
@@ -252,18 +257,18 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
     tc_fence_after();
     return ok;
   };
-  // weight slice c against A K-steps [ks0, ks0 + 4); the slice's bias tile, if any, last
-  auto chunk = [&](int c, uint32_t a_base, int ks0, uint32_t dcol, bool acc_first) {
+  // weight block j against the 128-wide K of operand A; the block's bias tile, if any, last
+  auto item = [&](int j, uint32_t a_base, uint32_t dcol, bool acc_first) {
     if (!ok) return;
-    if (!(ok = mbar_wait(b.full[stage], phase, abort_flag))) return;
+    if (!(ok = mbar_wait(b.full(stage), phase, abort_flag))) return;
     tc_fence_after();
     const uint32_t w = ring + stage * kSlot;
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tmem + dcol, sdesc(a_base + (ks0 + kk) * 4096, 2048, 128), sdesc(w + kk * 4096, 2048, 128), ID128,
+    for (int kk = 0; kk < 8; ++kk)
+      mma_bf16(tmem + dcol, sdesc(a_base + kk * 4096, 2048, 128), sdesc(w + kk * 4096, 2048, 128), ID128,
                (kk > 0 || acc_first) ? 1u : 0u);
-    if (chunk_has_bias(c)) mma_bf16(tmem + dcol, sdesc(sOnes, 2048, 128), sdesc(w + kChunk, 2048, 128), ID128, 1u);
-    mma_commit(b.empty[stage]);
+    if (item_has_bias(j)) mma_bf16(tmem + dcol, sdesc(sOnes, 2048, 128), sdesc(w + 2 * kChunk, 2048, 128), ID128, 1u);
+    mma_commit(b.empty(stage));
     if (++stage == kStages) {
       stage = 0;
       phase ^= 1;
@@ -280,7 +285,7 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
         mma_bf16(tmem + 128 + 128 * buf + s * t.Lp, sdesc(sA + h * 4096, 2048, 128),
                  sdesc(sKV + 2 * h * (t.Lp / 8) * 128, (t.Lp / 8) * 128, 128), idS, 0u);
       }
-      mma_commit(b.ev_s[buf]);
+      mma_commit(b.ev_s(buf));
     };
     // O[:, head] += P_head V_head for the heads of group g
     auto issue_AV = [&](int g) {
@@ -295,24 +300,23 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
       }
     };
     for (int l = 0; l < p.n_layer && ok; ++l) {
-      if (!wait_epi(b.e1, ph1)) break;                // A = LN1(y)
-      chunk(0, sA, 0, 128, false);                    // Q + bq
-      chunk(1, sA, 4, 128, true);
-      chunk(2, sA, 0, 256, false);                    // own K + bk
-      chunk(3, sA, 4, 256, true);
-      chunk(4, sA, 0, 384, false);                    // own V + bv
-      chunk(5, sA, 4, 384, true);
-      mma_commit(b.ev_qk);
-      if (!wait_epi(b.e2, ph2)) break;                // A = Q (scaled); own V in registers
+      // opaque per layer: keeps descriptor arithmetic from being hoisted into registers
+      asm volatile("" : "+r"(sA), "+r"(sP0), "+r"(sP1), "+r"(sKV), "+r"(ring), "+r"(sOnes), "+r"(tmem));
+      if (!wait_epi(b.e1(), ph1)) break;                // A = LN1(y)
+      item(0, sA, 128, false);                        // Q + bq
+      item(1, sA, 256, false);                        // own K + bk
+      item(2, sA, 384, false);                        // own V + bv
+      mma_commit(b.ev_qk());
+      if (!wait_epi(b.e2(), ph2)) break;                // A = Q (scaled); own V in registers
       if (!PF) {
-        ok = ok && mbar_wait(b.kv_full, kv_phase, abort_flag);
+        ok = ok && mbar_wait(b.kv_full(), kv_phase, abort_flag);
         kv_phase ^= 1;
         tc_fence_after();
       }
       if (ok && t.ng > 0) issue_S(0);
       if (ok && HG >= 2 && t.ng > 1) issue_S(1);
       for (int g = 0; g < t.ng && ok; ++g) {
-        if (!wait_epi(b.e3[g & 1], ph3[g & 1])) break;   // P of group g written, its scores read
+        if (!((g & 1) ? wait_epi(b.e3(1), ph3b) : wait_epi(b.e3(0), ph3a))) break;   // P of group g written, its scores read
         issue_AV(g);
         // two P buffers: group g + 2 reuses g's score buffer; one P buffer (L_u > 64):
         // group g + 1 is issued after group g's AV, so its P is free once its scores land
@@ -320,31 +324,26 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
         if (HG == 1 && g + 1 < t.ng) issue_S(g + 1);
       }
       if (!ok) break;
-      if (!PF) mma_commit(b.kv_empty);
-      mma_commit(b.ev_av);
-      if (!wait_epi(b.e4, ph4)) break;                // A = attention output
-      chunk(6, sA, 0, 0, true);                       // Y += attn Wo + bo
-      chunk(7, sA, 4, 0, true);
-      mma_commit(b.ev_o);
-      if (!wait_epi(b.e5, ph5)) break;                // A = LN2(y)
-      chunk(8, sA, 0, 128, false);                    // hidden[0,128) + b1
-      chunk(9, sA, 4, 128, true);
-      mma_commit(b.ev_h0);
-      chunk(10, sA, 0, 256, false);                   // hidden[128,256) + b1
-      chunk(11, sA, 4, 256, true);
-      mma_commit(b.ev_h1);
-      if (!wait_epi(b.e6a, ph6a)) break;              // P0 = ReLU(hidden[0,128))
-      chunk(12, sP0, 0, 0, true);                     // Y += H W2, first half of K
-      chunk(13, sP0, 4, 0, true);
-      if (!wait_epi(b.e6b, ph6b)) break;              // A = ReLU(hidden[128,256))
-      chunk(14, sA, 0, 0, true);                      // second half of K, + b2
-      chunk(15, sA, 4, 0, true);
-      mma_commit(b.ev_y);
+      if (!PF) mma_commit(b.kv_empty());
+      mma_commit(b.ev_av());
+      if (!wait_epi(b.e4(), ph4)) break;                // A = attention output
+      item(3, sA, 0, true);                           // Y += attn Wo + bo
+      mma_commit(b.ev_o());
+      if (!wait_epi(b.e5(), ph5)) break;                // A = LN2(y)
+      item(4, sA, 128, false);                        // hidden[0,128) + b1
+      mma_commit(b.ev_h0());
+      item(5, sA, 256, false);                        // hidden[128,256) + b1
+      mma_commit(b.ev_h1());
+      if (!wait_epi(b.e6a(), ph6a)) break;              // P0 = ReLU(hidden[0,128))
+      item(6, sP0, 0, true);                          // Y += H W2, first half of K
+      if (!wait_epi(b.e6b(), ph6b)) break;              // A = ReLU(hidden[128,256))
+      item(7, sA, 0, true);                           // second half of K, + b2
+      mma_commit(b.ev_y());
     }
   }
   // drain every MMA still in flight before the tensor memory is released
-  mma_commit(b.drain);
-  for (uint64_t t0 = globaltimer_ns(); !mbar_try_wait(b.drain, 0) && globaltimer_ns() - t0 < 500000000ull;) {
+  mma_commit(b.drain());
+  for (uint64_t t0 = globaltimer_ns(); !mbar_try_wait(b.drain(), 0) && globaltimer_ns() - t0 < 500000000ull;) {
   }
 }
 
@@ -374,8 +373,8 @@ struct Epi {
   }
   // rendezvous of the 256 epilogue threads (bounded)
   __device__ bool sync() {
-    mbar_arrive(b.esync);
-    ok = ok && mbar_wait(b.esync, ph_sync, abort_flag);
+    mbar_arrive(b.esync());
+    ok = ok && mbar_wait(b.esync(), ph_sync, abort_flag);
     ph_sync ^= 1;
     return ok;
   }
@@ -385,8 +384,8 @@ struct Epi {
     const uint32_t x = sX + slot * (2 * kM * 8);
     asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(x + (hf * kM + m) * 8), "f"(mine.x), "f"(mine.y)
                  : "memory");
-    mbar_arrive(b.qsync[q]);
-    ok = ok && mbar_wait(b.qsync[q], ph_q, abort_flag);
+    mbar_arrive(b.qsync(q));
+    ok = ok && mbar_wait(b.qsync(q), ph_q, abort_flag);
     ph_q ^= 1;
     float2 o;
     asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(o.x), "=f"(o.y) : "r"(x + ((1 - hf) * kM + m) * 8)
@@ -408,13 +407,16 @@ __device__ __forceinline__ void load64(uint32_t taddr, float* v) {
 
 // Row mean / rstd of a 128-wide row held as two 64-column halves (Welford merge).
 __device__ __forceinline__ float2 row_stats(Epi& e, const float* y) {
-  float mean = 0.f;
+  // four independent partial sums per pass: short dependency chains
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int i = 0; i < 64; ++i) mean += y[i];
-  mean *= (1.f / 64);
-  float m2 = 0.f;
+  for (int i = 0; i < 64; ++i) a[i & 3] += y[i];
+  const float mean = ((a[0] + a[1]) + (a[2] + a[3])) * (1.f / 64);
 #pragma unroll
-  for (int i = 0; i < 64; ++i) m2 = fmaf(y[i] - mean, y[i] - mean, m2);
+  for (int i = 0; i < 4; ++i) a[i] = 0.f;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) a[i & 3] = fmaf(y[i] - mean, y[i] - mean, a[i & 3]);
+  const float m2 = (a[0] + a[1]) + (a[2] + a[3]);
   const float2 o = e.swap(make_float2(mean, m2), 0);
   const float d = mean - o.x;
   const float mu = 0.5f * (mean + o.x);
@@ -502,17 +504,17 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
   for (int l = 0; l < p.n_layer; ++l) {
     const float* vl = e.vec + (size_t)l * kVecPerLayer;
     // ---- LN1 -> A
-    if (l > 0 && !e.wait(e.b.ev_y, e.ph_y)) return;
+    if (l > 0 && !e.wait(e.b.ev_y(), e.ph_y)) return;
     {
       float y[64];
       load64(ycol, y);
       ln_to_A(e, y, vl, vl + kD);
     }
-    e.signal(e.b.e1);
+    e.signal(e.b.e1());
     // ---- Q (scaled) -> A; own score per head; own V -> registers; user side: K/V images
-    if (!e.wait(e.b.ev_qk, e.ph_qk)) return;
+    if (!e.wait(e.b.ev_qk(), e.ph_qk)) return;
     if (PF) {
-      if (threadIdx.x == 64 && l > 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      if (threadIdx.x == kEpiThread0 && l > 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       if (!e.sync()) return;                       // the K/V images are free to overwrite
     }
     float sself[4];
@@ -564,7 +566,7 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
     if (PF) {  // store this layer's K/V images to the cache with one bulk copy
       fence_proxy_async_smem();
       if (!e.sync()) return;
-      if (threadIdx.x == 64) {
+      if (threadIdx.x == kEpiThread0) {
         const uint32_t bytes = 2u * t.Lp * kD * 2u;
         asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(p.kv_out + (size_t)l * bytes),
                      "r"(e.sKV), "r"(bytes)
@@ -572,14 +574,14 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
       }
     }
-    e.signal(e.b.e2);
+    e.signal(e.b.e2());
     // ---- softmax over [user keys of the request, own key], one head group at a time
     float pself[4] = {1.f, 1.f, 1.f, 1.f}, linv[4] = {1.f, 1.f, 1.f, 1.f};
     if constexpr (HG >= 2) {
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
         if (g >= t.ng) break;
-        if (!e.wait(e.b.ev_s[g & 1], e.ph_s[g & 1])) return;
+        if (!e.wait(e.b.ev_s(g & 1), e.ph_s[g & 1])) return;
         const uint32_t sbuf = e.trow + 128 + 128 * (g & 1);
         const uint32_t pbuf = (g & 1) ? e.sP1 : e.sP0;
 #pragma unroll
@@ -592,17 +594,20 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
             if (c < t.Lp / 16) tmem_ld16(sbuf + slot * t.Lp + 16 * c, sv + 16 * c);
           tmem_wait_ld();
           reg_fence<SV>(sv);
-          float mx = sself[jj];
+          // max and sum with four independent chains each
+          float m4[4] = {sself[jj], -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int i = 0; i < SV; ++i)
-            if (i < t.L_u) mx = fmaxf(mx, sv[i]);
-          float sum = 0.f;
+            if (i < t.L_u) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
+          const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int i = 0; i < SV; ++i) {
             const float ev = (i < t.L_u) ? ex2(sv[i] - mx) : 0.f;
             sv[i] = ev;
-            sum += ev;
+            s4[i & 3] += ev;
           }
+          const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
           const uint32_t pb = pbuf + slot * t.Lp * 256 + e.rowoff;
 #pragma unroll
           for (int jc = 0; jc < SV / 8; ++jc)
@@ -610,13 +615,13 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
           pself[jj] = ex2(sself[jj] - mx);
           linv[jj] = 1.f / (sum + pself[jj]);
         }
-        e.signal(e.b.e3[g & 1]);
+        e.signal(e.b.e3(g & 1));
       }
     } else {
       // L_u > 64: one head per group, its keys split between the two column halves
 #pragma unroll
       for (int g = 0; g < 8; ++g) {
-        if (!e.wait(e.b.ev_s[g & 1], e.ph_s[g & 1])) return;
+        if (!e.wait(e.b.ev_s(g & 1), e.ph_s[g & 1])) return;
         const uint32_t sbuf = e.trow + 128 + 128 * (g & 1);
         const int k0 = 64 * hf;
         const int nk = min(64, t.Lp - k0);       // > 0: Lp >= 80
@@ -627,18 +632,20 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
         tmem_wait_ld();
         reg_fence<64>(sv);
         const bool owner = (g >> 2) == hf;       // this half owns head g (and its own score)
-        float mx = owner ? sself[g & 3] : -INFINITY;
+        float m4[4] = {owner ? sself[g & 3] : -INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int i = 0; i < 64; ++i)
-          if (i < nk && k0 + i < t.L_u) mx = fmaxf(mx, sv[i]);
+          if (i < nk && k0 + i < t.L_u) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
+        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         mx = fmaxf(mx, e.swap(make_float2(mx, 0.f), 0).x);
-        float sum = 0.f;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           const float ev = (i < nk && k0 + i < t.L_u) ? ex2(sv[i] - mx) : 0.f;
           sv[i] = ev;
-          sum += ev;
+          s4[i & 3] += ev;
         }
+        const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
         const uint32_t pb = e.sP0 + e.rowoff + (k0 / 8) * 2048;
 #pragma unroll
         for (int jc = 0; jc < 8; ++jc)
@@ -649,11 +656,11 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
           pself[g & 3] = ps;
           linv[g & 3] = 1.f / tot;
         }
-        e.signal(e.b.e3[g & 1]);
+        e.signal(e.b.e3(g & 1));
       }
     }
     // ---- attention output = (sum_j p_j v_j + p_self v_self) / l  -> A
-    if (!e.wait(e.b.ev_av, e.ph_av)) return;
+    if (!e.wait(e.b.ev_av(), e.ph_av)) return;
     const bool has_users = t.ng > 0;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -672,41 +679,42 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
       st_row8(e.sA + (2 * h) * 2048 + e.rowoff, o);
       st_row8(e.sA + (2 * h + 1) * 2048 + e.rowoff, o + 8);
     }
-    e.signal(e.b.e4);
+    e.signal(e.b.e4());
     // ---- LN2 -> A
-    if (!e.wait(e.b.ev_o, e.ph_o)) return;
+    if (!e.wait(e.b.ev_o(), e.ph_o)) return;
     {
       float y[64];
       load64(ycol, y);
       ln_to_A(e, y, vl + 2 * kD, vl + 3 * kD);
     }
-    e.signal(e.b.e5);
+    e.signal(e.b.e5());
     // ---- ReLU(hidden) -> P0 (first half of the hidden units) and A (second half)
-    if (!e.wait(e.b.ev_h0, e.ph_h0)) return;
+    if (!e.wait(e.b.ev_h0(), e.ph_h0)) return;
     relu_to(e, e.trow + 128 + 64 * hf, e.sP0, 8 * hf);
-    e.signal(e.b.e6a);
-    if (!e.wait(e.b.ev_h1, e.ph_h1)) return;
+    e.signal(e.b.e6a());
+    if (!e.wait(e.b.ev_h1(), e.ph_h1)) return;
     relu_to(e, e.trow + 256 + 64 * hf, e.sA, 8 * hf);
-    e.signal(e.b.e6b);
+    e.signal(e.b.e6b());
   }
   // ---- head: w . LN_f(y) + b
-  if (!e.wait(e.b.ev_y, e.ph_y)) return;
+  if (!e.wait(e.b.ev_y(), e.ph_y)) return;
   if (PF) return;
   float y[64];
   load64(ycol, y);
   const float2 st = row_stats(e, y);
   const float* vf = e.vec + (size_t)p.n_layer * kVecPerLayer;
   const float4* w4 = reinterpret_cast<const float4*>(vf + 64 * hf);
-  float acc = 0.f;
+  float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const float4 w = w4[i];
-    acc = fmaf((y[4 * i] - st.x) * st.y, w.x, acc);
-    acc = fmaf((y[4 * i + 1] - st.x) * st.y, w.y, acc);
-    acc = fmaf((y[4 * i + 2] - st.x) * st.y, w.z, acc);
-    acc = fmaf((y[4 * i + 3] - st.x) * st.y, w.w, acc);
+    a4[0] = fmaf((y[4 * i] - st.x) * st.y, w.x, a4[0]);
+    a4[1] = fmaf((y[4 * i + 1] - st.x) * st.y, w.y, a4[1]);
+    a4[2] = fmaf((y[4 * i + 2] - st.x) * st.y, w.z, a4[2]);
+    a4[3] = fmaf((y[4 * i + 3] - st.x) * st.y, w.w, a4[3]);
     step_barrier();
   }
+  const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
   const float tot = acc + e.swap(make_float2(acc, 0.f), 1).x;
   if (hf == 0 && m < t.rows) p.scores[t.row0 + m] = tot + vf[kD];
 }
@@ -718,7 +726,7 @@ __device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint3
   Epi e;
   e.q = warp & 3;
   e.m = e.q * 32 + lane;
-  e.hf = (warp - 2) >> 2;
+  e.hf = (warp - 4) >> 2;
   e.trow = tmem + ((uint32_t)(e.q * 32) << 16);
   e.rowoff = (e.m >> 3) * 128 + (e.m & 7) * 16;
   e.sA = sA;
@@ -739,7 +747,7 @@ __device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint3
   // LayerNorm vectors and the head weight: a shared-memory copy when they fit
   const int nvec = p.n_layer * kVecPerLayer + kVecFinal;
   if (p.n_layer <= kMaxLayersSmemVec) {
-    const int tid = threadIdx.x - 64;
+    const int tid = threadIdx.x - kEpiThread0;
     for (int i = tid; i < nvec; i += kEpiThreads) svec[i] = __ldg(p.vec + i);
     if (!e.sync()) return;
     e.vec = svec;
@@ -753,7 +761,7 @@ __device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint3
 }
 
 template <bool PF, int HG>
-__global__ void __launch_bounds__(64 + kEpiThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
+__global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base = smem_u32(smem);
@@ -761,21 +769,21 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1) stack_kernel(const __grid
   const uint32_t sKV = base + (HG == 1 ? OFF_P1 : OFF_KV);
   const uint32_t sOnes = base + OFF_ONES, sX = base + OFF_X;
   float* svec = reinterpret_cast<float*>(smem + OFF_VEC);
-  const Bars b = make_bars(base + OFF_BAR);
+  const Bars b{base + OFF_BAR};
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + kBarBytes);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_BAR + kBarBytes + 8);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(b.full[s], 1);
-      mbar_init(b.empty[s], 1);
+      mbar_init(b.full(s), 1);
+      mbar_init(b.empty(s), 1);
     }
-    mbar_init(b.kv_full, 1);
-    mbar_init(b.kv_empty, 1);
-    for (uint32_t a : {b.ev_qk, b.ev_s[0], b.ev_s[1], b.ev_av, b.ev_o, b.ev_h0, b.ev_h1, b.ev_y, b.drain})
+    mbar_init(b.kv_full(), 1);
+    mbar_init(b.kv_empty(), 1);
+    for (uint32_t a : {b.ev_qk(), b.ev_s(0), b.ev_s(1), b.ev_av(), b.ev_o(), b.ev_h0(), b.ev_h1(), b.ev_y(), b.drain()})
       mbar_init(a, 1);
-    for (uint32_t a : {b.e1, b.e2, b.e3[0], b.e3[1], b.e4, b.e5, b.e6a, b.e6b, b.esync}) mbar_init(a, kEpiThreads);
-    for (int q = 0; q < 4; ++q) mbar_init(b.qsync[q], 64);
+    for (uint32_t a : {b.e1(), b.e2(), b.e3(0), b.e3(1), b.e4(), b.e5(), b.e6a(), b.e6b(), b.esync()}) mbar_init(a, kEpiThreads);
+    for (int q = 0; q < 4; ++q) mbar_init(b.qsync(q), 64);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -788,13 +796,14 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1) stack_kernel(const __grid
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    if (lane == 0) producer<PF>(p, ring, sKV, b, abort_flag);
-  } else if (warp == 1) {
-    if (lane == 0) mma_issuer<PF, HG>(p, tmem, sA, sP0, sP1, sKV, ring, sOnes, b, abort_flag);
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
+    if (warp == 0 && lane == 0) producer<PF>(p, ring, sKV, b, abort_flag);
+    if (warp == 1 && lane == 0) mma_issuer<PF, HG>(p, tmem, sA, sP0, sP1, sKV, ring, sOnes, b, abort_flag);
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
     epilogue<PF, HG>(p, tmem, sA, sP0, sP1, sKV, sX, sOnes, svec, b, abort_flag);
-    if (PF && threadIdx.x == 64) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (PF && threadIdx.x == kEpiThread0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
@@ -853,35 +862,30 @@ tr_status tc_build(tr_model* m, const tr_model_weights* w) {
   if (!(d.dtype == TR_BF16 && d.D == kD && d.ffn_hidden == kH && d.n_head == 8)) return TR_OK;
   const int N = d.n_layer, D = kD, H = kH;
   const size_t se = kSlot / 2;  // elements per stream slot
-  std::vector<uint16_t> img((size_t)N * kChunksPerLayer * se, 0);
+  std::vector<uint16_t> img((size_t)N * kItemsPerLayer * se, 0);
   std::vector<float> vec((size_t)N * kVecPerLayer + kVecFinal, 0.f);
   for (int l = 0; l < N; ++l) {
     // weights go in unchanged (exact bf16 values); LayerNorm gains/shifts stay fp32 in the
     // epilogue; biases become bias tiles next to the last slice of their GEMM
     const tr_layer_weights& L = w->layers[l];
-    uint16_t* li = img.data() + (size_t)l * kChunksPerLayer * se;
-    auto slot = [&](int c) { return li + (size_t)c * se; };
-    auto bias = [&](int c) { return li + (size_t)c * se + kChunk / 2; };
-    put_chunk(slot(0), L.Wq, D, 0, 0);
-    put_chunk(slot(1), L.Wq, D, 0, 64);
-    put_bias(bias(1), L.bq, 0);
-    put_chunk(slot(2), L.Wk, D, 0, 0);
-    put_chunk(slot(3), L.Wk, D, 0, 64);
-    put_bias(bias(3), L.bk, 0);
-    put_chunk(slot(4), L.Wv, D, 0, 0);
-    put_chunk(slot(5), L.Wv, D, 0, 64);
-    put_bias(bias(5), L.bv, 0);
-    put_chunk(slot(6), L.Wo, D, 0, 0);
-    put_chunk(slot(7), L.Wo, D, 0, 64);
-    put_bias(bias(7), L.bo, 0);
-    put_chunk(slot(8), L.W1, H, 0, 0);
-    put_chunk(slot(9), L.W1, H, 0, 64);
-    put_bias(bias(9), L.b1, 0);
-    put_chunk(slot(10), L.W1, H, 128, 0);
-    put_chunk(slot(11), L.W1, H, 128, 64);
-    put_bias(bias(11), L.b1, 128);
-    for (int q = 0; q < 4; ++q) put_chunk(slot(12 + q), L.W2, D, 0, 64 * q);
-    put_bias(bias(15), L.b2, 0);
+    uint16_t* li = img.data() + (size_t)l * kItemsPerLayer * se;
+    // item j: slice (K 0-63) | slice (K 64-127) | bias tile
+    auto half = [&](int j, int h) { return li + (size_t)j * se + (size_t)h * (kChunk / 2); };
+    auto bias = [&](int j) { return li + (size_t)j * se + kChunk; };
+    const float* Wn[4] = {L.Wq, L.Wk, L.Wv, L.Wo};
+    const float* bn[4] = {L.bq, L.bk, L.bv, L.bo};
+    for (int j = 0; j < 4; ++j) {
+      put_chunk(half(j, 0), Wn[j], D, 0, 0);
+      put_chunk(half(j, 1), Wn[j], D, 0, 64);
+      put_bias(bias(j), bn[j], 0);
+    }
+    for (int j = 0; j < 2; ++j) {   // W1, output columns 128 j .. 128 j + 127
+      put_chunk(half(4 + j, 0), L.W1, H, 128 * j, 0);
+      put_chunk(half(4 + j, 1), L.W1, H, 128 * j, 64);
+      put_bias(bias(4 + j), L.b1, 128 * j);
+    }
+    for (int q = 0; q < 4; ++q) put_chunk(half(6 + q / 2, q % 2), L.W2, D, 0, 64 * q);
+    put_bias(bias(7), L.b2, 0);
     float* v = vec.data() + (size_t)l * kVecPerLayer;
     for (int j = 0; j < D; ++j) {
       v[j] = L.ln1_g[j];
@@ -910,7 +914,7 @@ tr_status tc_build(tr_model* m, const tr_model_weights* w) {
   TR_CUDA_TRY(cudaMemcpy((uint8_t*)m->tc_blob + img_bytes, vec.data(), vec_bytes, cudaMemcpyHostToDevice));
   m->tc_stack = m->tc_blob;
   m->tc_stack_copy_bytes = copy_bytes;
-  m->tc_stack_layer_bytes = (size_t)kChunksPerLayer * kSlot;
+  m->tc_stack_layer_bytes = (size_t)kItemsPerLayer * kSlot;
   m->tc_vec = reinterpret_cast<const float*>((uint8_t*)m->tc_blob + img_bytes);
   m->tc_vec_layer_floats = kVecPerLayer;
   return TR_OK;
@@ -934,7 +938,7 @@ tr_status launch_stack(int hg, int grid, const StackParams& p, cudaStream_t st) 
     TR_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
     done[dev][hi] = true;
   }
-  k<<<grid, 64 + kEpiThreads, SMEM_BYTES, st>>>(p);
+  k<<<grid, kThreads, SMEM_BYTES, st>>>(p);
   TR_LAUNCH_CHECK(PF ? "stack_kernel (user side)" : "stack_kernel");
   return TR_OK;
 }
