@@ -50,6 +50,29 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def profiled_traffic(kernel: str):
+    """DRAM bytes per launch of ``kernel`` from the committed ncu summary under profiles/,
+    or None when there is none or the kernel's sources changed since it was captured."""
+    import glob
+    import hashlib
+    import re
+
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        text = open(path).read()
+        m = re.search(r"kernel: (\S+)\ntraffic_bytes_per_launch: (\d+)\nsources: ([^\n]+)\nsources_sha256: ([0-9a-f]+)", text)
+        if not m or m.group(1) != kernel:
+            continue
+        h = hashlib.sha256()
+        try:
+            for f in m.group(3).split():
+                with open(os.path.join(ROOT, f), "rb") as fh:
+                    h.update(fh.read())
+        except OSError:
+            return None
+        return int(m.group(2)) if h.hexdigest() == m.group(4) else None
+    return None
+
+
 # ------------------------------------------------------------------ algorithmic work
 
 def stack_flops_per_candidate(dims, L_u):
@@ -311,7 +334,7 @@ def run_ours(args, rank, world, local_rank):
     dominant = max(("score", "compress", "target_aggregate"), key=lambda k: stage_ms[k])
     roof = dict(stage_roof[dominant])
     roof["kernel"] = dominant
-    roof["traffic"] = None
+    roof["traffic"] = profiled_traffic("stack_kernel") if dominant == "score" else None
 
     if rank != 0:
         return

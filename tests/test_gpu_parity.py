@@ -88,8 +88,9 @@ def _run_agg(tables, bags, D, out_dtype):
 @pytest.mark.parametrize("out_dt", ["f32", "bf16"])
 @pytest.mark.parametrize("n_bags,max_nf", [(1237, 100), (9001, 8), (6007, 70)])
 def test_aggregate_parity(dt, D, out_dt, n_bags, max_nf):
-    """Both gather kernels: few long bags and many short ones (the pipelined kernel takes
-    >= 4096 bags), bags longer than the prefetched rows and than 32 keys, empty bags."""
+    """Few long bags and many short ones: bags longer than the rows a lane group keeps in
+    flight and than one key chunk, empty bags, and 1 to 8 bags per warp (D and dtype set
+    the lanes per row)."""
     rng = np.random.default_rng(D + n_bags)
     rows = 5000
     tables = _tables(11, 3, rows, D, dt)

@@ -74,91 +74,136 @@ __device__ __forceinline__ void store_out<__nv_bfloat16, 4>(__nv_bfloat16* dst, 
 }
 
 // LPR lanes per row, CI 16-byte column blocks per lane (D = LPR * CI * NV).
+//
+// Each group of LPR lanes owns one bag at a time (a warp works on 32 / LPR bags at once)
+// and keeps up to UNROLL row loads in flight, so a warp has several bags' rows in flight
+// and needs no cross-lane reduction of the row sums.  A bag costs three dependent memory
+// round trips (table id and offsets -> keys and weights -> rows); the group hides two of
+// them behind the previous bag: the next bag's table id and offsets are requested when a
+// bag starts, and its first LPR keys and weights once the current rows are in flight.
+// Loop trip counts are the warp's maximum, so every shuffle is warp-uniform.
 template <typename T, typename O, int LPR, int CI>
-__global__ void __launch_bounds__(256) wavg_kernel(TableSet tabs, int n_tables,
-                                                   const int32_t* __restrict__ bag_table,
-                                                   const int64_t* __restrict__ offsets,
-                                                   const int32_t* __restrict__ keys,
-                                                   const float* __restrict__ weights, int64_t n_bags,
-                                                   O* __restrict__ out, int* status) {
+__global__ void __launch_bounds__(256, 4) wavg_kernel(TableSet tabs, int n_tables,
+                                                      const int32_t* __restrict__ bag_table,
+                                                      const int64_t* __restrict__ offsets,
+                                                      const int32_t* __restrict__ keys,
+                                                      const float* __restrict__ weights, int64_t n_bags,
+                                                      O* __restrict__ out, int* status) {
   constexpr int NV = Vec16<T>::N;
   constexpr int D = LPR * CI * NV;
-  constexpr int RPS = 32 / LPR;   // rows per warp step
-  constexpr int UNROLL = 4;
+  constexpr int G = 32 / LPR;                 // bags per warp
+  constexpr int UNROLL = LPR < 8 ? LPR : 8;   // rows in flight per lane group
   const int lane = threadIdx.x & 31;
-  const int sub = lane / LPR;
+  const int grp = lane / LPR;
   const int cl = lane % LPR;
   const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5) * G;
+  bool bad = false;
 
-  for (int64_t b = warp; b < n_bags; b += nwarps) {
-    const int tbl = __ldg(bag_table + b);
-    const int64_t s0 = __ldg(offsets + b), s1 = __ldg(offsets + b + 1);
+  // the first bag's header and first key chunk
+  int tbl_n = 0;
+  int64_t s0_n = 0, s1_n = 0;
+  int k_n = -1;
+  float v_n = 0.f;
+  {
+    const int64_t b = warp * G + grp;
+    if (b < n_bags) {
+      tbl_n = __ldg(bag_table + b);
+      s0_n = __ldg(offsets + b);
+      s1_n = __ldg(offsets + b + 1);
+      if (cl < s1_n - s0_n) {
+        k_n = __ldg(keys + s0_n + cl);
+        v_n = __ldg(weights + s0_n + cl);
+      }
+    }
+  }
+  for (int64_t it = warp * G; it < n_bags; it += stride) {
+    const int64_t b = it + grp;
+    const bool live_bag = b < n_bags;
+    const int tbl = tbl_n;
+    const int64_t s0 = s0_n, s1 = s1_n;
+    int k = k_n;
+    float v = v_n;
+    const int64_t b2 = b + stride;
+    const bool has_next = b2 < n_bags;
+    if (has_next) {
+      tbl_n = __ldg(bag_table + b2);
+      s0_n = __ldg(offsets + b2);
+      s1_n = __ldg(offsets + b2 + 1);
+    }
+    bool next_keys = false;   // the next bag's first key chunk requested yet
+    auto fetch_next_keys = [&]() {
+      next_keys = true;
+      k_n = -1;
+      v_n = 0.f;
+      if (cl < s1_n - s0_n) {
+        k_n = __ldg(keys + s0_n + cl);
+        v_n = __ldg(weights + s0_n + cl);
+      }
+    };
+    const bool bad_table = live_bag && (tbl < 0 || tbl >= n_tables);
+    bad |= bad_table;
+    const int n = (live_bag && !bad_table) ? (int)(s1 - s0) : 0;
+    const int n_max = __reduce_max_sync(0xffffffffu, n);   // the warp's longest bag
+    const T* table = static_cast<const T*>(tabs.ptr[n > 0 ? tbl : 0]);
+    const int64_t nrows = n > 0 ? tabs.rows[tbl] : 0;
     float acc[CI][NV];
 #pragma unroll
     for (int c = 0; c < CI; ++c)
 #pragma unroll
       for (int i = 0; i < NV; ++i) acc[c][i] = 0.f;
     float wsum = 0.f;
-    bool bad = false;
-    if (tbl < 0 || tbl >= n_tables) {
-      bad = true;
-    } else {
-      const T* table = static_cast<const T*>(tabs.ptr[tbl]);
-      const int64_t nrows = tabs.rows[tbl];
-      for (int64_t base = s0; base < s1; base += 32) {
-        const int cnt = (int)(s1 - base < 32 ? s1 - base : 32);
-        int k = -1;
-        float v = 0.f;
-        if (lane < cnt) {
-          k = __ldg(keys + base + lane);
-          v = __ldg(weights + base + lane);
-          if (k < 0 || (int64_t)k >= nrows) {
-            bad = true;
-            k = -1;
-            v = 0.f;
-          }
-        }
-        wsum += v;
-        for (int j0 = 0; j0 < cnt; j0 += RPS * UNROLL) {
-          uint4 raw[UNROLL][CI];
-          float wv[UNROLL];
-#pragma unroll
-          for (int u = 0; u < UNROLL; ++u) {
-            const int j = j0 + u * RPS + sub;
-            const int kk = __shfl_sync(0xffffffffu, k, j & 31);
-            wv[u] = __shfl_sync(0xffffffffu, v, j & 31);
-            const bool live = (j < cnt) && kk >= 0;
-            if (!live) wv[u] = 0.f;
-            const uint4* row = reinterpret_cast<const uint4*>(table + (int64_t)(live ? kk : 0) * D);
-#pragma unroll
-            for (int c = 0; c < CI; ++c)
-              raw[u][c] = live ? ld_stream(row + c * LPR + cl) : make_uint4(0, 0, 0, 0);
-          }
-#pragma unroll
-          for (int u = 0; u < UNROLL; ++u)
-#pragma unroll
-            for (int c = 0; c < CI; ++c) {
-              float f[NV];
-              Vec16<T>::unpack(raw[u][c], f);
-#pragma unroll
-              for (int i = 0; i < NV; ++i) acc[c][i] = fmaf(wv[u], f[i], acc[c][i]);
-            }
+    for (int base = 0; base < n_max; base += LPR) {
+      const int cnt = n - base;                     // keys of this bag in the chunk (may be <= 0)
+      if (base != 0) {                              // chunks after the prefetched one
+        k = -1;
+        v = 0.f;
+        if (cl < cnt) {
+          k = __ldg(keys + s0 + base + cl);
+          v = __ldg(weights + s0 + base + cl);
         }
       }
+      if (cl >= cnt) {
+        k = -1;
+        v = 0.f;
+      } else if (k < 0 || (int64_t)k >= nrows) {
+        bad = true;
+        k = -1;
+        v = 0.f;
+      }
+      wsum += v;
+      const int cnt_max = n_max - base < LPR ? n_max - base : LPR;   // warp-uniform
+      for (int j0 = 0; j0 < cnt_max; j0 += UNROLL) {
+        uint4 raw[UNROLL][CI];
+        float wv[UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+          const int j = j0 + u;
+          const int kk = __shfl_sync(0xffffffffu, k, j % LPR, LPR);
+          wv[u] = __shfl_sync(0xffffffffu, v, j % LPR, LPR);
+          const bool live = j < cnt && kk >= 0;
+          if (!live) wv[u] = 0.f;
+          const uint4* row = reinterpret_cast<const uint4*>(table + (int64_t)(live ? kk : 0) * D);
+#pragma unroll
+          for (int c = 0; c < CI; ++c)
+            raw[u][c] = live ? ld_stream(row + c * LPR + cl) : make_uint4(0, 0, 0, 0);
+        }
+        if (has_next && !next_keys) fetch_next_keys();   // overlaps these rows
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u)
+#pragma unroll
+          for (int c = 0; c < CI; ++c) {
+            float f[NV];
+            Vec16<T>::unpack(raw[u][c], f);
+#pragma unroll
+            for (int i = 0; i < NV; ++i) acc[c][i] = fmaf(wv[u], f[i], acc[c][i]);
+          }
+      }
     }
-    // combine the RPS row-groups and the weight sum across the warp
+    if (has_next && !next_keys) fetch_next_keys();   // empty or rejected bag
 #pragma unroll
-    for (int off = LPR; off < 32; off <<= 1)
-#pragma unroll
-      for (int c = 0; c < CI; ++c)
-#pragma unroll
-        for (int i = 0; i < NV; ++i) acc[c][i] += __shfl_xor_sync(0xffffffffu, acc[c][i], off);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
-    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, STATUS_KEY_RANGE);
-    const bool bad_table = (tbl < 0 || tbl >= n_tables);
-    if (sub == 0) {
+    for (int off = LPR / 2; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+    if (live_bag) {
 #pragma unroll
       for (int c = 0; c < CI; ++c) {
         float r[NV];
@@ -168,6 +213,7 @@ __global__ void __launch_bounds__(256) wavg_kernel(TableSet tabs, int n_tables,
       }
     }
   }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, STATUS_KEY_RANGE);
 }
 
 template <typename T, typename O>
@@ -179,8 +225,12 @@ tr_status dispatch(const TableSet& ts, int n_tables, const int32_t* bag_table, c
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t blocks_needed = (n_bags + 7) / 8;
-  const int grid = (int)std::min<int64_t>(blocks_needed, (int64_t)sms * 8);
+  // 8 warps per block, 32 / LPR bags per warp at a time; 4 blocks per SM are resident and
+  // the grid is 32 blocks per SM, so that blocks started late (an SM held by a concurrent
+  // kernel) take a small share of the work
+  const int64_t bags_per_block = 8 * (32 / (vecs < 32 ? vecs : 32));
+  const int64_t blocks_needed = (n_bags + bags_per_block - 1) / bags_per_block;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, (int64_t)sms * 32));
 #define TR_WAVG(LPR, CI)                                                                               \
   wavg_kernel<T, O, LPR, CI><<<grid, 256, 0, st>>>(ts, n_tables, bag_table, offsets, keys, weights, \
                                                    n_bags, out, status)

@@ -105,13 +105,22 @@ class DeviceWorkload:
         return self.req_offsets[-1]
 
     # -------------------------------------------------------------- the step
-    def user_side(self, stream=None) -> None:
+    def user_aggregate(self, stream=None) -> None:
         for r, b in enumerate(self.user_bags):
             if self.L_u[r] == 0:
                 continue
             api.aggregate(self.user_tables, b.bag_table, b.offsets, b.keys, b.weights, self.user_tokens[r],
                           stream=stream)
+
+    def user_prefill(self, stream=None) -> None:
+        for r in range(len(self.user_bags)):
+            if self.L_u[r] == 0:
+                continue
             api.prefill_user(self.model, self.user_tokens[r], self.L_u[r], self.domain[r], self.kv[r], stream=stream)
+
+    def user_side(self, stream=None) -> None:
+        self.user_aggregate(stream)
+        self.user_prefill(stream)
 
     def target_aggregate(self, stream=None) -> None:
         b = self.target_bags
@@ -126,20 +135,26 @@ class DeviceWorkload:
                              self.scores, stream=stream)
 
     def step(self, stream=None, events=None) -> torch.Tensor:
-        """One request batch.  The user side (aggregation + prefill, one CTA per request)
-        runs on a side stream concurrently with the target aggregation and compression; the
-        scoring waits for both.  ``events``: optional dict of CUDA events recorded at stage
-        boundaries (keys user0, user1 on the side stream; t0, agg, comp, s0, score on the main)."""
+        """One request batch.  The user aggregation (a few small launches) runs first on the
+        caller's stream; then the user prefill (one CTA per request, which needs a whole SM)
+        runs on a high-priority side stream while the target aggregation and compression run
+        on the caller's stream.  Both become ready together, so the prefill CTAs are placed
+        before the gather fills the SMs, and the prefill ends before the compressor needs
+        every SM.  The scoring waits for both.  ``events``: optional dict of CUDA events
+        recorded at stage boundaries (keys user0, user1 on the side stream; t0, agg, comp, s0,
+        score on the main)."""
         main = stream if stream is not None else torch.cuda.current_stream(self.device)
         if not hasattr(self, "_side"):
-            self._side = torch.cuda.Stream(self.device)
+            lo, hi = torch.cuda.Stream.priority_range()
+            self._side = torch.cuda.Stream(self.device, priority=hi)
         side = self._side
+        if events:
+            events["user0"].record(main)
+        self.user_aggregate(main)
         fork = torch.cuda.Event()
         fork.record(main)
         side.wait_event(fork)
-        if events:
-            events["user0"].record(side)
-        self.user_side(side)
+        self.user_prefill(side)
         if events:
             events["user1"].record(side)
         join = torch.cuda.Event()
