@@ -9,23 +9,22 @@
 //   TMEM (512 fp32 columns x 128 lanes, lane = candidate row)
 //     [  0,128)  Y, the residual stream; the O and FFN2 GEMMs (and their biases)
 //                accumulate into it in place
-//     [128,256)  Q accumulator -> score buffer 0 -> FFN hidden [0,128)
-//     [256,384)  K accumulator -> score buffer 1 -> FFN hidden [128,256)
+//     [128,256)  Q accumulator -> score buffer 0 (softmax numerators written over the scores
+//                as bf16, the A operand of P V) -> FFN hidden [0,128)
+//     [256,384)  K accumulator -> score buffer 1 (same) -> FFN hidden [128,256)
 //     [384,512)  V accumulator -> attention output O (the candidate's own V moves to
-//                registers as bf16 first)
+//                registers as bf16 first) -> ReLU(hidden) as bf16, the A operand of W2
 //   shared memory
-//     A      [128 x 128] bf16  LN1 output -> Q -> attention output -> LN2 output -> hidden[128,256)
-//     P0, P1 [128 x 128] bf16  softmax numerators of a head group (double-buffered) -> P0
-//                              holds hidden[0,128); for L_u > 64 the K/V images take P1's place
-//     KV     the request's K and V^T images of the current layer
-//     ring   2 x 36 KB: a [128 out x 128 in] weight block plus its [128 x 16] bias tile;
+//     A      [128 x 128] bf16  LN1 output -> Q -> attention output -> LN2 output
+//     KV     the request's K and V^T images of the current layer (up to 64 KB)
+//     ring   3 x 36 KB: a [128 out x 128 in] weight block plus its [128 x 16] bias tile;
 //            streamed by the TMA engine in consumption order
 //     ones   the [128 x 16] A operand that turns a bias tile into "+ bias" in one MMA
 //     vec    LayerNorm gains/shifts of every layer and the folded head weight (<= 5 layers)
 //
 // Attention runs per head group (the heads whose scores fit 128 TMEM columns).  The scores of
-// group g + 2 are computed into the buffer group g just released while the epilogue works on
-// group g + 1, so the epilogue does not wait on the tensor core between groups.
+// group g + 2 are computed into the buffer group g used, once group g's P V products have
+// completed, while the epilogue works on group g + 1.
 //
 // Biases: one extra K = 16 MMA per GEMM, ones[128 x 16] x bias_tile^T, where the bias tile
 // holds the bf16 head and tail of each fp32 bias (columns 0 and 1): D += b_hi + b_lo.
@@ -64,7 +63,7 @@ constexpr int kBiasTile = 4096;               // [128 x 16] bf16 bias tile
 // cycles each, copies of one SM largely serialised), so items are as large as the ring
 // allows.
 constexpr int kSlot = 2 * kChunk + kBiasTile;
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kItemsPerLayer = 8;
 constexpr int kVecPerLayer = 4 * kD;          // LN1 gain, LN1 shift, LN2 gain, LN2 shift
 constexpr int kVecFinal = kD + 4;             // head weight * final LN gain, folded head bias
@@ -89,11 +88,9 @@ constexpr float kQScale = 0.25f * 1.44269504088896341f;  // 1/sqrt(d_h) * log2(e
 __host__ __device__ constexpr bool item_has_bias(int j) { return j != 6; }
 
 constexpr int OFF_A = 0;
-constexpr int OFF_P0 = 32768;
-constexpr int OFF_P1 = 65536;                               // L_u > 64: start of the K/V images
-constexpr int OFF_KV = 98304;                               // L_u <= 64
-constexpr int OFF_RING = 131072;
-constexpr int OFF_ONES = OFF_RING + kStages * kSlot;        // 200 KB
+constexpr int OFF_KV = 32768;                               // 2 x L_p x 128 bf16, L_p <= 128
+constexpr int OFF_RING = 98304;
+constexpr int OFF_ONES = OFF_RING + kStages * kSlot;        // 204 KB
 constexpr int OFF_X = OFF_ONES + kM * 16 * 2;               // [2 slots][2 halves][128] float2
 constexpr int OFF_VEC = OFF_X + 2 * 2 * kM * 8;
 constexpr int OFF_BAR = OFF_VEC + (kMaxLayersSmemVec * kVecPerLayer + kVecFinal) * 4;
@@ -182,8 +179,10 @@ struct Bars {
   __device__ __forceinline__ uint32_t drain() const { return at(2 * kStages + 18); }
   __device__ __forceinline__ uint32_t esync() const { return at(2 * kStages + 19); }
   __device__ __forceinline__ uint32_t qsync(int q) const { return at(2 * kStages + 20 + q); }
+  // MMA -> MMA: the P V products that read score buffer i have completed
+  __device__ __forceinline__ uint32_t av_done(int i) const { return at(2 * kStages + 24 + i); }
 };
-constexpr int kNumBars = 2 * kStages + 24;
+constexpr int kNumBars = 2 * kStages + 26;
 constexpr int kBarBytes = 8 * kNumBars;
 static_assert(kBarBytes + 16 <= 320, "barrier area");
 
@@ -243,13 +242,14 @@ __device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, co
 
 // ------------------------------------------------------------------ MMA issuer (warp 1, one thread)
 template <bool PF, int HG>
-__device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sP0, uint32_t sP1,
-                           uint32_t sKV, uint32_t ring, uint32_t sOnes, const Bars& b, volatile int* abort_flag) {
+__device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sKV, uint32_t ring,
+                           uint32_t sOnes, const Bars& b, volatile int* abort_flag) {
   constexpr uint32_t ID128 = idesc_bf16(kM, 128);
   constexpr uint32_t ID16 = idesc_bf16(kM, 16);
   int stage = 0;
   uint32_t phase = 0, kv_phase = 0;
   uint32_t ph1 = 0, ph2 = 0, ph3a = 0, ph3b = 0, ph4 = 0, ph5 = 0, ph6a = 0, ph6b = 0;
+  uint32_t av_pend = 0, av_ph = 0;   // bit i: a P V commit on buffer i not yet waited for / its parity
   bool ok = true;
   auto wait_epi = [&](uint32_t bar, uint32_t& ph) {
     ok = ok && mbar_wait(bar, ph, abort_flag);
@@ -257,16 +257,21 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
     tc_fence_after();
     return ok;
   };
-  // weight block j against the 128-wide K of operand A; the block's bias tile, if any, last
-  auto item = [&](int j, uint32_t a_base, uint32_t dcol, bool acc_first) {
+  // weight block j against the 128-wide K of operand A (shared memory at a_base, or tensor
+  // memory columns a_col .. a_col + 63 when A_TMEM); the block's bias tile, if any, last
+  auto item = [&](int j, uint32_t a_base, uint32_t dcol, bool acc_first, bool a_tmem) {
     if (!ok) return;
     if (!(ok = mbar_wait(b.full(stage), phase, abort_flag))) return;
     tc_fence_after();
     const uint32_t w = ring + stage * kSlot;
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      mma_bf16(tmem + dcol, sdesc(a_base + kk * 4096, 2048, 128), sdesc(w + kk * 4096, 2048, 128), ID128,
-               (kk > 0 || acc_first) ? 1u : 0u);
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t acc = (kk > 0 || acc_first) ? 1u : 0u;
+      if (a_tmem)
+        mma_bf16_ta(tmem + dcol, tmem + a_base + kk * 8, sdesc(w + kk * 4096, 2048, 128), ID128, acc);
+      else
+        mma_bf16(tmem + dcol, sdesc(a_base + kk * 4096, 2048, 128), sdesc(w + kk * 4096, 2048, 128), ID128, acc);
+    }
     if (item_has_bias(j)) mma_bf16(tmem + dcol, sdesc(sOnes, 2048, 128), sdesc(w + 2 * kChunk, 2048, 128), ID128, 1u);
     mma_commit(b.empty(stage));
     if (++stage == kStages) {
@@ -277,9 +282,20 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
   for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
     const TileInfo t = tile_info(p, tile);
     const uint32_t idS = idesc_bf16(kM, t.Lp > 0 ? t.Lp : 16);
+    // P V of the last group that used a score buffer must be complete before new scores
+    // overwrite its numerators
+    auto av_wait = [&](int buf) {
+      if (!((av_pend >> buf) & 1u)) return;
+      ok = ok && mbar_wait(b.av_done(buf), (av_ph >> buf) & 1u, abort_flag);
+      av_ph ^= 1u << buf;
+      av_pend &= ~(1u << buf);
+      tc_fence_after();
+    };
     // scores of head group g into TMEM buffer g % 2
     auto issue_S = [&](int g) {
       const int buf = g & 1;
+      av_wait(buf);
+      if (!ok) return;
       for (int s = 0; s < HG; ++s) {
         const int h = slot_head(g, s, HG);
         mma_bf16(tmem + 128 + 128 * buf + s * t.Lp, sdesc(sA + h * 4096, 2048, 128),
@@ -287,25 +303,28 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
       }
       mma_commit(b.ev_s(buf));
     };
-    // O[:, head] += P_head V_head for the heads of group g
+    // O[:, head] += P_head V_head for the heads of group g; P is read from tensor memory
+    // (slot s's numerators over the first half of its score columns)
     auto issue_AV = [&](int g) {
-      const uint32_t pbase = (HG >= 2 && (g & 1)) ? sP1 : sP0;
+      const int buf = g & 1;
       for (int s = 0; s < HG; ++s) {
         const int h = slot_head(g, s, HG);
-        const uint32_t pb = pbase + s * t.Lp * 256;
+        const uint32_t pcol = 128 + 128 * buf + s * t.Lp;
         const uint32_t vb = sKV + t.Lp * 256;
         for (int kk = 0; kk < t.Lp / 16; ++kk)
-          mma_bf16(tmem + 384 + 16 * h, sdesc(pb + kk * 4096, 2048, 128),
-                   sdesc(vb + (32 * kk + 2 * h) * 128, 2048, 128), ID16, kk > 0 ? 1u : 0u);
+          mma_bf16_ta(tmem + 384 + 16 * h, tmem + pcol + kk * 8, sdesc(vb + (32 * kk + 2 * h) * 128, 2048, 128),
+                      ID16, kk > 0 ? 1u : 0u);
       }
+      mma_commit(b.av_done(buf));
+      av_pend |= 1u << buf;
     };
     for (int l = 0; l < p.n_layer && ok; ++l) {
       // opaque per layer: keeps descriptor arithmetic from being hoisted into registers
-      asm volatile("" : "+r"(sA), "+r"(sP0), "+r"(sP1), "+r"(sKV), "+r"(ring), "+r"(sOnes), "+r"(tmem));
+      asm volatile("" : "+r"(sA), "+r"(sKV), "+r"(ring), "+r"(sOnes), "+r"(tmem));
       if (!wait_epi(b.e1(), ph1)) break;                // A = LN1(y)
-      item(0, sA, 128, false);                        // Q + bq
-      item(1, sA, 256, false);                        // own K + bk
-      item(2, sA, 384, false);                        // own V + bv
+      item(0, sA, 128, false, false);                 // Q + bq
+      item(1, sA, 256, false, false);                 // own K + bk
+      item(2, sA, 384, false, false);                 // own V + bv
       mma_commit(b.ev_qk());
       if (!wait_epi(b.e2(), ph2)) break;                // A = Q (scaled); own V in registers
       if (!PF) {
@@ -323,21 +342,23 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
         if (HG >= 2 && g + 2 < t.ng) issue_S(g + 2);
         if (HG == 1 && g + 1 < t.ng) issue_S(g + 1);
       }
+      av_wait(0);
+      av_wait(1);
       if (!ok) break;
       if (!PF) mma_commit(b.kv_empty());
       mma_commit(b.ev_av());
       if (!wait_epi(b.e4(), ph4)) break;                // A = attention output
-      item(3, sA, 0, true);                           // Y += attn Wo + bo
+      item(3, sA, 0, true, false);                    // Y += attn Wo + bo
       mma_commit(b.ev_o());
       if (!wait_epi(b.e5(), ph5)) break;                // A = LN2(y)
-      item(4, sA, 128, false);                        // hidden[0,128) + b1
+      item(4, sA, 128, false, false);                 // hidden[0,128) + b1
       mma_commit(b.ev_h0());
-      item(5, sA, 256, false);                        // hidden[128,256) + b1
+      item(5, sA, 256, false, false);                 // hidden[128,256) + b1
       mma_commit(b.ev_h1());
-      if (!wait_epi(b.e6a(), ph6a)) break;              // P0 = ReLU(hidden[0,128))
-      item(6, sP0, 0, true);                          // Y += H W2, first half of K
-      if (!wait_epi(b.e6b(), ph6b)) break;              // A = ReLU(hidden[128,256))
-      item(7, sA, 0, true);                           // second half of K, + b2
+      if (!wait_epi(b.e6a(), ph6a)) break;              // TMEM [384,448) = ReLU(hidden[0,128))
+      item(6, 384, 0, true, true);                    // Y += H W2, first half of K
+      if (!wait_epi(b.e6b(), ph6b)) break;              // TMEM [448,512) = ReLU(hidden[128,256))
+      item(7, 448, 0, true, true);                    // second half of K, + b2
       mma_commit(b.ev_y());
     }
   }
@@ -352,7 +373,7 @@ struct Epi {
   uint32_t trow;        // TMEM address of this row, column 0
   uint32_t rowoff;      // byte offset of this row inside a 128-row core-matrix operand
   int m, hf, q;         // row, column half (0: columns 0-63 / heads 0-3), lane quadrant
-  uint32_t sA, sP0, sP1, sKV, sX;
+  uint32_t sA, sKV, sX;
   const float* vec;     // LayerNorm vectors (shared memory copy when it fits)
   Bars b;
   volatile int* abort_flag;
@@ -443,17 +464,14 @@ __device__ __forceinline__ void ln_to_A(Epi& e, const float* y, const float* gam
   }
 }
 
-// ReLU of 64 accumulator columns -> bf16 into an operand (its K-chunks kc0 .. kc0 + 7).
-__device__ __forceinline__ void relu_to(Epi& e, uint32_t tcol, uint32_t dst, int kc0) {
+// ReLU of 64 accumulator columns -> bf16 pairs in 32 TMEM columns (an A operand row).
+__device__ __forceinline__ void relu_to_tmem(uint32_t tcol, uint32_t dcol) {
   float v[64];
   load64(tcol, v);
 #pragma unroll
-  for (int kc = 0; kc < 8; ++kc) {
-    float w[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = fmaxf(v[kc * 8 + i], 0.f);
-    st_row8(dst + (kc0 + kc) * 2048 + e.rowoff, w);
-  }
+  for (int i = 0; i < 64; ++i) v[i] = fmaxf(v[i], 0.f);
+  tmem_st_bf16x32(dcol, v);
+  tmem_st_bf16x32(dcol + 16, v + 32);
 }
 
 template <bool PF, int HG>
@@ -578,40 +596,56 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
     // ---- softmax over [user keys of the request, own key], one head group at a time
     float pself[4] = {1.f, 1.f, 1.f, 1.f}, linv[4] = {1.f, 1.f, 1.f, 1.f};
     if constexpr (HG >= 2) {
+      const int nb = t.Lp / 16;                   // 16-key blocks holding keys (>= 1)
+      const int tail = t.L_u - 16 * (nb - 1);     // keys in the last block (1..16)
 #pragma unroll
       for (int g = 0; g < NG; ++g) {
         if (g >= t.ng) break;
         if (!e.wait(e.b.ev_s(g & 1), e.ph_s[g & 1])) return;
         const uint32_t sbuf = e.trow + 128 + 128 * (g & 1);
-        const uint32_t pbuf = (g & 1) ? e.sP1 : e.sP0;
 #pragma unroll
         for (int j = 0; j < HG / 2; ++j) {
           const int jj = g * (HG / 2) + j;          // this half's head index (0..3)
           const int slot = hf * (HG / 2) + j;
           float sv[SV];
 #pragma unroll
-          for (int c = 0; c < SV / 16; ++c)
-            if (c < t.Lp / 16) tmem_ld16(sbuf + slot * t.Lp + 16 * c, sv + 16 * c);
+          for (int c = 0; c < SV / 16; ++c) {
+            if (c < nb) {
+              tmem_ld16(sbuf + slot * t.Lp + 16 * c, sv + 16 * c);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) sv[16 * c + i] = -INFINITY;
+            }
+          }
           tmem_wait_ld();
           reg_fence<SV>(sv);
+          // padding keys (L_u not a multiple of 16) -> -inf, so the loops below need no masks
+          if (tail < 16) {
+#pragma unroll
+            for (int i = 0; i < SV; ++i) sv[i] = i < t.L_u ? sv[i] : -INFINITY;
+          }
           // max and sum with four independent chains each
           float m4[4] = {sself[jj], -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int i = 0; i < SV; ++i)
-            if (i < t.L_u) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
+          for (int i = 0; i < SV; ++i) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
           const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
           float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int i = 0; i < SV; ++i) {
-            const float ev = (i < t.L_u) ? ex2(sv[i] - mx) : 0.f;
+            const float ev = ex2(sv[i] - mx);
             sv[i] = ev;
             s4[i & 3] += ev;
           }
           const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-          const uint32_t pb = pbuf + slot * t.Lp * 256 + e.rowoff;
+          // numerators as bf16 over the first half of this slot's own score columns (the
+          // P V products read only the first L_p / 2 of them)
+          const uint32_t pcol = sbuf + slot * t.Lp;
+          if constexpr (SV == 16) {
+            tmem_st_bf16x16(pcol, sv);
+          } else {
 #pragma unroll
-          for (int jc = 0; jc < SV / 8; ++jc)
-            if (jc < t.Lp / 8) st_row8(pb + jc * 2048, sv + 8 * jc);
+            for (int c = 0; c < SV / 32; ++c) tmem_st_bf16x32(pcol + 16 * c, sv + 32 * c);
+          }
           pself[jj] = ex2(sself[jj] - mx);
           linv[jj] = 1.f / (sum + pself[jj]);
         }
@@ -646,10 +680,10 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
           s4[i & 3] += ev;
         }
         const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-        const uint32_t pb = e.sP0 + e.rowoff + (k0 / 8) * 2048;
-#pragma unroll
-        for (int jc = 0; jc < 8; ++jc)
-          if (jc < nk / 8) st_row8(pb + jc * 2048, sv + 8 * jc);
+        // keys 64 hf .. as bf16 from column 32 hf of the buffer: over this half's own scores
+        // (hf = 0) or the first half's, which both halves have read before the max exchange
+        tmem_st_bf16x32(sbuf + 32 * hf, sv);
+        tmem_st_bf16x32(sbuf + 32 * hf + 16, sv + 32);
         const float ps = owner ? ex2(sself[g & 3] - mx) : 0.f;
         const float tot = sum + ps + e.swap(make_float2(sum + ps, 0.f), 1).x;
         if (owner) {
@@ -690,10 +724,10 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
     e.signal(e.b.e5());
     // ---- ReLU(hidden) -> P0 (first half of the hidden units) and A (second half)
     if (!e.wait(e.b.ev_h0(), e.ph_h0)) return;
-    relu_to(e, e.trow + 128 + 64 * hf, e.sP0, 8 * hf);
+    relu_to_tmem(e.trow + 128 + 64 * hf, e.trow + 384 + 32 * hf);
     e.signal(e.b.e6a());
     if (!e.wait(e.b.ev_h1(), e.ph_h1)) return;
-    relu_to(e, e.trow + 256 + 64 * hf, e.sA, 8 * hf);
+    relu_to_tmem(e.trow + 256 + 64 * hf, e.trow + 448 + 32 * hf);
     e.signal(e.b.e6b());
   }
   // ---- head: w . LN_f(y) + b
@@ -720,7 +754,7 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
 }
 
 template <bool PF, int HG>
-__device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sP0, uint32_t sP1, uint32_t sKV,
+__device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sKV,
                          uint32_t sX, uint32_t sOnes, float* svec, const Bars& b, volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Epi e;
@@ -730,8 +764,6 @@ __device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint3
   e.trow = tmem + ((uint32_t)(e.q * 32) << 16);
   e.rowoff = (e.m >> 3) * 128 + (e.m & 7) * 16;
   e.sA = sA;
-  e.sP0 = sP0;
-  e.sP1 = sP1;
   e.sKV = sKV;
   e.sX = sX;
   e.b = b;
@@ -765,8 +797,7 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base = smem_u32(smem);
-  const uint32_t sA = base + OFF_A, sP0 = base + OFF_P0, sP1 = base + OFF_P1, ring = base + OFF_RING;
-  const uint32_t sKV = base + (HG == 1 ? OFF_P1 : OFF_KV);
+  const uint32_t sA = base + OFF_A, sKV = base + OFF_KV, ring = base + OFF_RING;
   const uint32_t sOnes = base + OFF_ONES, sX = base + OFF_X;
   float* svec = reinterpret_cast<float*>(smem + OFF_VEC);
   const Bars b{base + OFF_BAR};
@@ -780,7 +811,8 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
     }
     mbar_init(b.kv_full(), 1);
     mbar_init(b.kv_empty(), 1);
-    for (uint32_t a : {b.ev_qk(), b.ev_s(0), b.ev_s(1), b.ev_av(), b.ev_o(), b.ev_h0(), b.ev_h1(), b.ev_y(), b.drain()})
+    for (uint32_t a : {b.ev_qk(), b.ev_s(0), b.ev_s(1), b.ev_av(), b.ev_o(), b.ev_h0(), b.ev_h1(), b.ev_y(), b.drain(),
+                       b.av_done(0), b.av_done(1)})
       mbar_init(a, 1);
     for (uint32_t a : {b.e1(), b.e2(), b.e3(0), b.e3(1), b.e4(), b.e5(), b.e6a(), b.e6b(), b.esync()}) mbar_init(a, kEpiThreads);
     for (int q = 0; q < 4; ++q) mbar_init(b.qsync(q), 64);
@@ -799,10 +831,10 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
     if (warp == 0 && lane == 0) producer<PF>(p, ring, sKV, b, abort_flag);
-    if (warp == 1 && lane == 0) mma_issuer<PF, HG>(p, tmem, sA, sP0, sP1, sKV, ring, sOnes, b, abort_flag);
+    if (warp == 1 && lane == 0) mma_issuer<PF, HG>(p, tmem, sA, sKV, ring, sOnes, b, abort_flag);
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
-    epilogue<PF, HG>(p, tmem, sA, sP0, sP1, sKV, sX, sOnes, svec, b, abort_flag);
+    epilogue<PF, HG>(p, tmem, sA, sKV, sX, sOnes, svec, b, abort_flag);
     if (PF && threadIdx.x == kEpiThread0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
   tc_fence_before();
