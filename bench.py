@@ -212,7 +212,7 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
 
     from transformer_candidate_scoring_b200 import api
-    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, HostFeed
     from transformer_candidate_scoring_b200.shard import max_over_ranks, rank_seed
 
     torch.cuda.set_device(local_rank)
@@ -276,36 +276,25 @@ def run_ours(args, rank, world, local_rank):
     n_cand = dw.n_cand
     value = n_cand * args.steps * world / elapsed
 
-    # ---- end to end: host bags in, scores out, through the same calls
-    host_sets = []
+    # ---- end to end: host bags in, scores out, through the package's host feed (the bags
+    # of batch i + 1 are copied while batch i computes)
+    host_batches = []
     for ub, tb, reqs in dsets:
         hu = [DeviceBags(*(x.cpu().pin_memory() for x in (b.offsets, b.keys, b.weights, b.bag_table))) for b in ub]
         ht = DeviceBags(*(x.cpu().pin_memory() for x in (tb.offsets, tb.keys, tb.weights, tb.bag_table)))
-        host_sets.append((hu, ht))
-    h2d = sum(x.numel() * x.element_size() for b in host_sets[0][0] for x in (b.offsets, b.keys, b.weights, b.bag_table))
-    h2d += sum(x.numel() * x.element_size() for x in (host_sets[0][1].offsets, host_sets[0][1].keys,
-                                                        host_sets[0][1].weights, host_sets[0][1].bag_table))
-    host_scores = torch.empty(n_cand, dtype=torch.float32).pin_memory()
-    d2h = host_scores.numel() * 4
+        host_batches.append((hu, ht, reqs))
+    feed = HostFeed(dw, host_batches)
+    h2d = float(np.mean(feed.h2d_bytes))
+    host_scores = [torch.empty(n_cand, dtype=torch.float32).pin_memory() for _ in range(2)]
+    d2h = n_cand * 4
 
-    def e2e_step(i):
-        hu, ht = host_sets[i % N_REQUEST_SETS]
-        ub, tb, reqs = dsets[i % N_REQUEST_SETS]
-        for h, d in zip(hu + [ht], ub + [tb]):
-            for hs, ds in zip((h.offsets, h.keys, h.weights, h.bag_table), (d.offsets, d.keys, d.weights, d.bag_table)):
-                ds.copy_(hs, non_blocking=True)
-        step(i)
-        host_scores.copy_(dw.scores, non_blocking=True)
-
-    for i in range(args.warmup):
-        e2e_step(i)
+    feed.run(0, args.warmup, host_scores, stream)
     torch.cuda.synchronize()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(args.steps):
-        e2e_step(i)
+    feed.run(args.warmup, args.steps, host_scores, stream)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()

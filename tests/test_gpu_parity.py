@@ -325,3 +325,30 @@ def test_full_size_sampled(name, n_sample):
         print(r, check_close(g, ref, "bf16", f"request {r}"))
     del dw
     torch.cuda.empty_cache()
+
+
+def test_host_feed_matches_device_resident_steps():
+    """Bags fed from pinned host memory with the copy of batch i + 1 overlapping batch i
+    (two device slots) give bit-identical scores to the device-resident steps."""
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, HostFeed, pack_target_bags
+    w = datagen.scaled(datagen.WORKLOADS["128d5l"], n_cand_per_request=500, rows=20000)
+    sets = [datagen.make_requests(w, seed=900 + k) for k in range(3)]
+    dw = DeviceWorkload(w, reqs=sets[0])
+    ref = []
+    for reqs in sets:
+        dw.set_requests(reqs)
+        dw.step()
+        ref.append(dw.scores.clone())
+    dw.set_requests(sets[0])
+
+    def pinned(b):
+        return DeviceBags(*(x.pin_memory() for x in (b.offsets, b.keys, b.weights, b.bag_table)))
+    batches = [([pinned(DeviceBags.of(r.user, "cpu")) for r in reqs], pinned(DeviceBags.of(pack_target_bags(reqs), "cpu")),
+                reqs) for reqs in sets]
+    feed = HostFeed(dw, batches)
+    out = [torch.empty(dw.n_cand, dtype=torch.float32).pin_memory() for _ in range(7)]
+    feed.run(0, 7, out)
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    for i in range(7):
+        assert torch.equal(out[i], ref[i % 3].cpu()), i

@@ -104,6 +104,14 @@ class DeviceWorkload:
     def n_cand(self) -> int:
         return self.req_offsets[-1]
 
+    def use_bags(self, user_bags, target_bags, reqs) -> None:
+        """Point the next step at other device bags of requests with the same L_u and
+        candidate counts as the current ones (no reallocation of activations)."""
+        if [r.L_u for r in reqs] != self.L_u or [r.n_cand for r in reqs] != [r.n_cand for r in self.reqs]:
+            raise ValueError("use_bags: requests differ in L_u or candidate count; call set_requests")
+        self.user_bags, self.target_bags, self.reqs = list(user_bags), target_bags, reqs
+        self.domain = [r.domain for r in reqs]
+
     # -------------------------------------------------------------- the step
     def user_aggregate(self, stream=None) -> None:
         for r, b in enumerate(self.user_bags):
@@ -174,3 +182,76 @@ class DeviceWorkload:
         if events:
             events["score"].record(main)
         return self.scores
+
+
+def _bag_tensors(b: DeviceBags):
+    return (b.offsets, b.keys, b.weights, b.bag_table)
+
+
+class HostFeed:
+    """Request batches whose bags sit in pinned host memory, scored back to back (the
+    serving case).  The bags of batch i + 1 are copied to the device on a copy stream while
+    batch i computes (two device slots, guarded by events); each batch's scores are copied
+    back to a pinned host buffer on the compute stream.
+
+    ``batches``: list of (user bags per request, target bags, requests), every bag tensor in
+    pinned host memory; all batches have the requests' L_u and candidate counts of ``dw``.
+    """
+
+    def __init__(self, dw: DeviceWorkload, batches):
+        self.dw = dw
+        self.batches = batches
+        dev = dw.device
+        n_req = len(batches[0][0])
+        self.slots = []
+        for _ in range(2):   # device buffers with the largest size any batch needs
+            def alloc(pick):
+                return DeviceBags(*(torch.empty(max(int(getattr(pick(bt), f).numel()) for bt in batches),
+                                                dtype=getattr(pick(batches[0]), f).dtype, device=dev)
+                                    for f in ("offsets", "keys", "weights", "bag_table")))
+            users = [alloc(lambda bt, r=r: bt[0][r]) for r in range(n_req)]
+            target = alloc(lambda bt: bt[1])
+            self.slots.append((users, target))
+        self.copy_stream = torch.cuda.Stream(dev)
+        self.ready = [torch.cuda.Event() for _ in range(2)]
+        self.free = [torch.cuda.Event() for _ in range(2)]
+        self.h2d_bytes = [sum(x.numel() * x.element_size() for b in bt[0] + [bt[1]] for x in _bag_tensors(b))
+                          for bt in batches]
+
+    def _views(self, i):
+        """Device views of slot i % 2 sized for batch i."""
+        users, target = self.slots[i % 2]
+        hu, ht, _ = self.batches[i % len(self.batches)]
+
+        def fit(dst, src):
+            return DeviceBags(*(d[:s.numel()] for d, s in zip(_bag_tensors(dst), _bag_tensors(src))))
+        return [fit(d, h) for d, h in zip(users, hu)], fit(target, ht)
+
+    def _copy_in(self, i):
+        hu, ht, _ = self.batches[i % len(self.batches)]
+        du, dt = self._views(i)
+        cs = self.copy_stream
+        cs.wait_event(self.free[i % 2])            # batch i - 2 is done with this slot
+        with torch.cuda.stream(cs):
+            for d, h in zip(du + [dt], hu + [ht]):
+                for dx, hx in zip(_bag_tensors(d), _bag_tensors(h)):
+                    dx.copy_(hx, non_blocking=True)
+        self.ready[i % 2].record(cs)
+
+    def run(self, first: int, count: int, host_scores, stream=None) -> None:
+        """Score batches first .. first + count - 1 (batch i uses host batch i mod len);
+        the scores of batch i land in ``host_scores[i % len(host_scores)]`` (pinned)."""
+        main = stream if stream is not None else torch.cuda.current_stream(self.dw.device)
+        start = torch.cuda.Event()
+        start.record(main)
+        self.copy_stream.wait_event(start)         # copies begin after work already on main
+        self._copy_in(first)
+        for i in range(first, first + count):
+            if i + 1 < first + count:
+                self._copy_in(i + 1)
+            main.wait_event(self.ready[i % 2])
+            du, dt = self._views(i)
+            self.dw.use_bags(du, dt, self.batches[i % len(self.batches)][2])
+            self.dw.step(main)
+            self.free[i % 2].record(main)
+            host_scores[i % len(host_scores)].copy_(self.dw.scores, non_blocking=True)
