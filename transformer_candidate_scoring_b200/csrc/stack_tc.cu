@@ -334,13 +334,24 @@ __device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uin
       }
       if (ok && t.ng > 0) issue_S(0);
       if (ok && HG >= 2 && t.ng > 1) issue_S(1);
-      for (int g = 0; g < t.ng && ok; ++g) {
-        if (!((g & 1) ? wait_epi(b.e3(1), ph3b) : wait_epi(b.e3(0), ph3a))) break;   // P of group g written, its scores read
-        issue_AV(g);
-        // two P buffers: group g + 2 reuses g's score buffer; one P buffer (L_u > 64):
-        // group g + 1 is issued after group g's AV, so its P is free once its scores land
-        if (HG >= 2 && g + 2 < t.ng) issue_S(g + 2);
-        if (HG == 1 && g + 1 < t.ng) issue_S(g + 1);
+      if constexpr (HG >= 2) {
+        // rounds of gpr groups (the epilogue's GPR); two score buffers are in flight, so
+        // after round g0 the scores of groups g0 + 2 .. g0 + 1 + gpr are issued
+        constexpr int gpr = 1;
+        for (int g0 = 0; g0 < t.ng && ok; g0 += gpr) {
+          const bool odd = (g0 / gpr) & 1;
+          if (!(odd ? wait_epi(b.e3(1), ph3b) : wait_epi(b.e3(0), ph3a))) break;   // round's numerators written
+          for (int gi = 0; gi < gpr; ++gi) issue_AV(g0 + gi);
+          for (int gi = 0; gi < gpr; ++gi)
+            if (g0 + 2 + gi < t.ng) issue_S(g0 + 2 + gi);
+        }
+      } else {
+        for (int g = 0; g < t.ng && ok; ++g) {
+          if (!((g & 1) ? wait_epi(b.e3(1), ph3b) : wait_epi(b.e3(0), ph3a))) break;   // P of group g written
+          issue_AV(g);
+          // group g + 1 goes to the other score buffer once the P V that last read it is done
+          if (g + 1 < t.ng) issue_S(g + 1);
+        }
       }
       av_wait(0);
       av_wait(1);
@@ -596,60 +607,84 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t
     // ---- softmax over [user keys of the request, own key], one head group at a time
     float pself[4] = {1.f, 1.f, 1.f, 1.f}, linv[4] = {1.f, 1.f, 1.f, 1.f};
     if constexpr (HG >= 2) {
+      // One score group per round: while the epilogue works on group g + 1 the tensor core
+      // multiplies group g's numerators by V and computes group g + 2's scores into the
+      // buffer group g used.  (Two groups per round measured no faster: it loses that
+      // overlap.)  Rounds signal e3(0) and e3(1) in turn, so the MMA thread's wait on one
+      // never sees it complete twice.
+      constexpr int GPR = 1;
       const int nb = t.Lp / 16;                   // 16-key blocks holding keys (>= 1)
       const int tail = t.L_u - 16 * (nb - 1);     // keys in the last block (1..16)
 #pragma unroll
-      for (int g = 0; g < NG; ++g) {
-        if (g >= t.ng) break;
-        if (!e.wait(e.b.ev_s(g & 1), e.ph_s[g & 1])) return;
-        const uint32_t sbuf = e.trow + 128 + 128 * (g & 1);
+      for (int g0 = 0; g0 < NG; g0 += GPR) {
+        if (g0 >= t.ng) break;
 #pragma unroll
-        for (int j = 0; j < HG / 2; ++j) {
-          const int jj = g * (HG / 2) + j;          // this half's head index (0..3)
-          const int slot = hf * (HG / 2) + j;
-          float sv[SV];
+        for (int gi = 0; gi < GPR; ++gi)
+          if (!e.wait(e.b.ev_s((g0 + gi) & 1), e.ph_s[(g0 + gi) & 1])) return;
 #pragma unroll
-          for (int c = 0; c < SV / 16; ++c) {
-            if (c < nb) {
-              tmem_ld16(sbuf + slot * t.Lp + 16 * c, sv + 16 * c);
+        for (int gi = 0; gi < GPR; ++gi) {
+          const int g = g0 + gi;
+          const uint32_t sbuf = e.trow + 128 + 128 * (g & 1);
+#pragma unroll
+          for (int j = 0; j < HG / 2; ++j) {
+            const int jj = g * (HG / 2) + j;        // this half's head index (0..3)
+            const int slot = hf * (HG / 2) + j;
+            float sv[SV];
+#pragma unroll
+            for (int c = 0; c < SV / 16; ++c) {
+              if (c < nb) {
+                tmem_ld16(sbuf + slot * t.Lp + 16 * c, sv + 16 * c);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) sv[16 * c + i] = -INFINITY;
+              }
+            }
+            tmem_wait_ld();
+            reg_fence<SV>(sv);
+            // padding keys (L_u not a multiple of 16) -> -inf, so the loops below need no masks
+            if (tail < 16) {
+#pragma unroll
+              for (int i = 0; i < SV; ++i) sv[i] = i < t.L_u ? sv[i] : -INFINITY;
+            }
+            // max: four chains of three-input maxima
+            float m4[4] = {sself[jj], -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int i = 0; i < SV; i += 8) {
+              m4[0] = max3(m4[0], sv[i], sv[i + 1]);
+              m4[1] = max3(m4[1], sv[i + 2], sv[i + 3]);
+              m4[2] = max3(m4[2], sv[i + 4], sv[i + 5]);
+              m4[3] = max3(m4[3], sv[i + 6], sv[i + 7]);
+            }
+            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            // exponentials; the subtraction and the running sums on packed pairs
+            const uint64_t neg = f32x2(-mx, -mx);
+            uint64_t acc[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
+#pragma unroll
+            for (int i = 0; i < SV; i += 2) {
+              float x0, x1;
+              f32x2_split(add_f32x2(f32x2(sv[i], sv[i + 1]), neg), x0, x1);
+              sv[i] = ex2(x0);
+              sv[i + 1] = ex2(x1);
+              acc[(i >> 1) & 1] = add_f32x2(acc[(i >> 1) & 1], f32x2(sv[i], sv[i + 1]));
+            }
+            float a0, a1, b0, b1;
+            f32x2_split(acc[0], a0, a1);
+            f32x2_split(acc[1], b0, b1);
+            const float sum = (a0 + a1) + (b0 + b1);
+            // numerators as bf16 over the first half of this slot's own score columns (the
+            // P V products read only the first L_p / 2 of them)
+            const uint32_t pcol = sbuf + slot * t.Lp;
+            if constexpr (SV == 16) {
+              tmem_st_bf16x16(pcol, sv);
             } else {
 #pragma unroll
-              for (int i = 0; i < 16; ++i) sv[16 * c + i] = -INFINITY;
+              for (int c = 0; c < SV / 32; ++c) tmem_st_bf16x32(pcol + 16 * c, sv + 32 * c);
             }
+            pself[jj] = ex2(sself[jj] - mx);
+            linv[jj] = 1.f / (sum + pself[jj]);
           }
-          tmem_wait_ld();
-          reg_fence<SV>(sv);
-          // padding keys (L_u not a multiple of 16) -> -inf, so the loops below need no masks
-          if (tail < 16) {
-#pragma unroll
-            for (int i = 0; i < SV; ++i) sv[i] = i < t.L_u ? sv[i] : -INFINITY;
-          }
-          // max and sum with four independent chains each
-          float m4[4] = {sself[jj], -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int i = 0; i < SV; ++i) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
-          const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-          float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int i = 0; i < SV; ++i) {
-            const float ev = ex2(sv[i] - mx);
-            sv[i] = ev;
-            s4[i & 3] += ev;
-          }
-          const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-          // numerators as bf16 over the first half of this slot's own score columns (the
-          // P V products read only the first L_p / 2 of them)
-          const uint32_t pcol = sbuf + slot * t.Lp;
-          if constexpr (SV == 16) {
-            tmem_st_bf16x16(pcol, sv);
-          } else {
-#pragma unroll
-            for (int c = 0; c < SV / 32; ++c) tmem_st_bf16x32(pcol + 16 * c, sv + 32 * c);
-          }
-          pself[jj] = ex2(sself[jj] - mx);
-          linv[jj] = 1.f / (sum + pself[jj]);
         }
-        e.signal(e.b.e3(g & 1));
+        e.signal(e.b.e3((g0 / GPR) & 1));
       }
     } else {
       // L_u > 64: one head per group, its keys split between the two column halves
