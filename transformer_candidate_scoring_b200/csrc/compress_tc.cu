@@ -38,7 +38,12 @@ constexpr int OFF_R1 = 0;
 constexpr int OFF_R2 = 2 * STAGE1;             // 160 KB
 constexpr int STAGE2 = 32 * 1024;
 constexpr int OFF_BAR = OFF_R2 + 2 * STAGE2;   // 224 KB
-constexpr int SMEM_BYTES = OFF_BAR + 160 + 1024;
+constexpr int OFF_B3 = OFF_BAR + 256;           // the last layer's bias (c3 <= 256 floats)
+constexpr int SMEM_BYTES = OFF_B3 + 1024 + 1024;
+// The per-column vectors of the layer whose epilogue runs are staged in shared memory at
+// R1 + 132 KB (8 KB): that part of the second x/W1 stage is idle from the end of a tile's
+// first GEMM until the next tile's loads, which wait for its last GEMM.
+constexpr int OFF_VEC = OFF_R1 + 132 * 1024;
 
 struct CompParams {
   CUtensorMap xmap;            // x [n][c0] bf16, box {64, 128}, 128-byte swizzle
@@ -54,7 +59,7 @@ struct CompParams {
 };
 
 struct CBars {
-  uint32_t full1[2], empty1[2], full2[2], empty2[2], r1_free, mma, epi, drain, qsync[4];
+  uint32_t full1[2], empty1[2], full2[2], empty2[2], r1_free, mma, epi, drain, qsync[4], vsync;
 };
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
@@ -204,8 +209,9 @@ struct CEpi {
   }
 };
 
+// eight consecutive floats of a vector staged in shared memory
 __device__ __forceinline__ void vec8(const float* p, float* o) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p)), b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
   o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
 }
 
@@ -271,8 +277,8 @@ __device__ __forceinline__ void prelu_ln_half(CEpi& e, int cols, const float* bi
   }
 }
 
-__device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, const CBars& b,
-                              volatile int* abort_flag) {
+__device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, const CBars& b, float* svec,
+                              float* sb3, volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   CEpi e;
   e.q = warp & 3;
@@ -288,7 +294,16 @@ __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, c
   const float* v1 = p.vec;
   const float* v2 = p.vec + 4 * p.c1;
   const float* b3 = v2 + 4 * p.c2;
-  uint32_t mma_phase = 0;
+  const int et = threadIdx.x - 64;                 // 0 .. 255
+  for (int i = et; i < p.c3; i += 256) sb3[i] = __ldg(b3 + i);   // visible after the first vsync
+  uint32_t mma_phase = 0, vph = 0;
+  // rendezvous of the 256 epilogue threads after a vector staging (bounded)
+  auto vbar = [&]() {
+    mbar_arrive(b.vsync);
+    e.ok = e.ok && mbar_wait(b.vsync, vph, abort_flag);
+    vph ^= 1;
+    return e.ok;
+  };
   auto wait_mma = [&]() {
     e.ok = e.ok && mbar_wait(b.mma, mma_phase, abort_flag);
     mma_phase ^= 1;
@@ -302,11 +317,26 @@ __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, c
     mbar_arrive(b.epi);
   };
   for (int tile = blockIdx.x; tile < p.n_tiles && e.ok; tile += gridDim.x) {
+    // layer 1's vectors (4 c1 floats) are read into registers while its GEMM runs and
+    // stored once it is done
+    float4 r1v[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      if (et + 256 * k < p.c1) r1v[k] = __ldg(reinterpret_cast<const float4*>(v1) + et + 256 * k);
     if (!wait_mma()) break;
-    prelu_ln_half(e, p.c1, v1, v1 + p.c1, v1 + 2 * p.c1, v1 + 3 * p.c1, r1 + e.rowoff, 0);
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      if (et + 256 * k < p.c1) reinterpret_cast<float4*>(svec)[et + 256 * k] = r1v[k];
+    if (!vbar()) break;
+    prelu_ln_half(e, p.c1, svec, svec + p.c1, svec + 2 * p.c1, svec + 3 * p.c1, r1 + e.rowoff, 0);
     signal();
+    // layer 2's: every thread has finished reading layer 1's once the layer-2 GEMM is done
+    float4 r2v;
+    if (et < p.c2) r2v = __ldg(reinterpret_cast<const float4*>(v2) + et);
     if (!wait_mma()) break;
-    prelu_ln_half(e, p.c2, v2, v2 + p.c2, v2 + 2 * p.c2, v2 + 3 * p.c2, r1 + e.rowoff, 1);
+    if (et < p.c2) reinterpret_cast<float4*>(svec)[et] = r2v;
+    if (!vbar()) break;
+    prelu_ln_half(e, p.c2, svec, svec + p.c2, svec + 2 * p.c2, svec + 3 * p.c2, r1 + e.rowoff, 1);
     signal();
     if (!wait_mma()) break;
     const long long row = (long long)tile * kM + e.m;
@@ -317,8 +347,8 @@ __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, c
       tmem_wait_ld();
       reg_fence<16>(v);
       float bb[16];
-      vec8(b3 + c, bb);
-      vec8(b3 + c + 8, bb + 8);
+      vec8(sb3 + c, bb);
+      vec8(sb3 + c + 8, bb + 8);
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] += bb[i];
       if (row < p.n) {
@@ -350,6 +380,7 @@ __global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant_
   b.epi = bar0 + 80;
   b.drain = bar0 + 88;
   for (int q = 0; q < 4; ++q) b.qsync[q] = bar0 + 96 + 8 * q;
+  b.vsync = bar0 + 144;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_BAR + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_BAR + 136);
   if (threadIdx.x == 0) {
@@ -364,6 +395,7 @@ __global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant_
     mbar_init(b.epi, 256);
     mbar_init(b.drain, 1);
     for (int q = 0; q < 4; ++q) mbar_init(b.qsync[q], 64);
+    mbar_init(b.vsync, 256);
     *abort_flag = 0;
     mbar_fence_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.xmap)) : "memory");
@@ -381,7 +413,8 @@ __global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant_
   } else if (warp == 1) {
     if (lane == 0) comp_mma(p, tmem, r1, r2, b, abort_flag);
   } else {
-    comp_epilogue(p, tmem, r1, b, abort_flag);
+    comp_epilogue(p, tmem, r1, b, reinterpret_cast<float*>(gbase + OFF_VEC), reinterpret_cast<float*>(gbase + OFF_B3),
+                  abort_flag);
   }
   tc_fence_before();
   __syncthreads();
