@@ -276,6 +276,20 @@ def run_ours(args, rank, world, local_rank):
     n_cand = dw.n_cand
     value = n_cand * args.steps * world / elapsed
 
+    # ---- per-request top-k of the scores (the selection step after scoring; timed on its
+    # own, it is not one of the step's stages)
+    TOPK = 2000
+    dw.select(TOPK, stream)
+    torch.cuda.synchronize()
+    k0 = torch.cuda.Event(enable_timing=True)
+    k1 = torch.cuda.Event(enable_timing=True)
+    k0.record(stream)
+    for _ in range(args.steps):
+        dw.select(TOPK, stream)
+    k1.record(stream)
+    torch.cuda.synchronize()
+    topk_ms = k0.elapsed_time(k1) / args.steps
+
     # ---- end to end: host bags in, scores out, through the package's host feed (the bags
     # of batch i + 1 are copied while batch i computes)
     host_batches = []
@@ -344,6 +358,7 @@ def run_ours(args, rank, world, local_rank):
         "stages": {k: {"ms": stage_ms[k], **({kk: vv for kk, vv in stage_roof[k].items()} if k in stage_roof else {})}
                    for k in stage_names},
         "pct_bf16_peak_score_kernel": stage_roof["score"]["frac"] * 100,
+        "topk": {"k": TOPK, "ms": topk_ms, "note": "tr_topk over the step's scores, timed separately"},
         "e2e": {"value": e2e_value, "unit": "candidates/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": int(launches),

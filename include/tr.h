@@ -185,6 +185,24 @@ tr_status tr_score_candidates(const tr_model* m, const void* tokens, int64_t n,
                               tr_stream stream);
 
 /*
+ * Per-request top-k of the scores (the selection step of GPU retrieval, TransRetrieval
+ * deployment section "Hardware-aware inference optimization": a request's scored candidates
+ * are reduced to the best k on the GPU).
+ *   scores      DEVICE fp32 [n], candidates grouped by request as in tr_score_candidates
+ *   req_offsets HOST int64 [R+1], req_offsets[0] = 0, non-decreasing, req_offsets[R] = n
+ *   k           1 .. TR_MAX_TOPK
+ *   out_idx     DEVICE int64 [R][k]: for request r, candidate indices within the request
+ *               (0-based) by descending score; equal scores by lower index; a request with
+ *               fewer than k candidates is padded with -1
+ *   out_score   DEVICE fp32 [R][k] or NULL: the selected scores (padding -inf)
+ * NaN scores rank below every other score.  The selected set and its order are unique, so
+ * the result does not depend on the launch or on other requests.  1 <= R <= TR_MAX_REQUESTS.
+ */
+#define TR_MAX_TOPK 4096
+tr_status tr_topk(const float* scores, int64_t n, const int64_t* req_offsets, int R, int k, int64_t* out_idx,
+                  float* out_score, tr_stream stream);
+
+/*
  * No-allocation variant of tr_prefill_user.  The paper has no counterpart: this entry point
  * exists for callers that cannot call cudaMalloc when the user side runs -- code running
  * while a CUDA stream capture is open (allocation is not a capturable operation), serving

@@ -54,3 +54,16 @@ def test_host_validation_without_gpu(lib):
     d = L.ModelDesc(64, 2, 4, 128, 8, (C.c_int * 4)(500, 256, 128, 64), 2, 1)    # comp_dims[0] != F*D
     assert lib.tr_model_create(C.byref(d), None, C.byref(h)) == L.TR_ERR_INVALID_ARG
     assert lib.tr_score_candidates(None, None, 0, None, None, None, None, 1, None, None) == L.TR_ERR_INVALID_ARG
+
+
+def test_topk_host_validation_without_gpu(lib):
+    from transformer_candidate_scoring_b200 import _lib as L
+    off = (C.c_int64 * 3)(0, 5, 9)
+    assert lib.tr_topk(None, 9, off, 2, 0, None, None, None) == L.TR_ERR_INVALID_ARG          # k = 0
+    assert lib.tr_topk(None, 9, off, 2, L.TR_MAX_TOPK + 1, None, None, None) == L.TR_ERR_INVALID_ARG
+    assert lib.tr_topk(None, 9, off, 0, 5, None, None, None) == L.TR_ERR_INVALID_ARG          # R = 0
+    assert lib.tr_topk(None, 8, off, 2, 5, None, None, None) == L.TR_ERR_INVALID_ARG          # offsets != n
+    bad = (C.c_int64 * 3)(0, 6, 5)
+    assert lib.tr_topk(None, 5, bad, 2, 5, None, None, None) == L.TR_ERR_INVALID_ARG          # decreasing
+    assert lib.tr_topk(None, 9, off, 2, 5, None, None, None) == L.TR_ERR_INVALID_ARG          # null outputs
+    assert b"null" in lib.tr_last_error()

@@ -6,7 +6,7 @@ driver.  There is no CPU fallback: every call raises if libtr.so is missing.
 """
 from . import api
 from .api import (Model, TrError, aggregate, compress_targets, kv_cache_bytes, prefill_user,
-                  prefill_user_noalloc, score_candidates, sync_status)
+                  prefill_user_noalloc, score_candidates, sync_status, topk)
 
 __all__ = ["api", "Model", "TrError", "aggregate", "compress_targets", "kv_cache_bytes",
-           "prefill_user", "prefill_user_noalloc", "score_candidates", "sync_status"]
+           "prefill_user", "prefill_user_noalloc", "score_candidates", "sync_status", "topk"]

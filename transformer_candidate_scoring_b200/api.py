@@ -170,6 +170,20 @@ def score_candidates(model: Model, tokens: torch.Tensor, req_offsets: Sequence[i
     return scores
 
 
+def topk(scores: torch.Tensor, req_offsets: Sequence[int], k: int, out_idx: torch.Tensor = None,
+         out_score: torch.Tensor = None, stream=None):
+    """tr_topk: per-request top-k; returns (out_idx int64 [R, k], out_score fp32 [R, k])."""
+    R = len(req_offsets) - 1
+    off = (C.c_int64 * (R + 1))(*[int(x) for x in req_offsets])
+    if out_idx is None:
+        out_idx = torch.empty(R, k, dtype=torch.int64, device=scores.device)
+    if out_score is None:
+        out_score = torch.empty(R, k, dtype=torch.float32, device=scores.device)
+    _check(L.load().tr_topk(_ptr(scores), int(req_offsets[-1]), off, R, int(k), _ptr(out_idx), _ptr(out_score),
+                            _stream(stream)))
+    return out_idx, out_score
+
+
 def sync_status(stream=None, timeout_ms: int = 10_000) -> int:
     """tr_sync_status; returns the status code (does not raise)."""
     return int(L.load().tr_sync_status(_stream(stream), timeout_ms))

@@ -297,6 +297,22 @@ tr_status tr_score_candidates(const tr_model* m, const void* tokens, int64_t n, 
   return TR_OK;
 }
 
+tr_status tr_topk(const float* scores, int64_t n, const int64_t* req_offsets, int R, int k, int64_t* out_idx,
+                  float* out_score, tr_stream stream) {
+  if (R < 1 || R > TR_MAX_REQUESTS) return fail(TR_ERR_INVALID_ARG, "R=%d (need 1..%d)", R, TR_MAX_REQUESTS);
+  if (k < 1 || k > TR_MAX_TOPK) return fail(TR_ERR_INVALID_ARG, "k=%d (need 1..%d)", k, TR_MAX_TOPK);
+  if (!req_offsets) return fail(TR_ERR_INVALID_ARG, "null req_offsets");
+  if (n < 0 || req_offsets[0] != 0 || req_offsets[R] != n)
+    return fail(TR_ERR_INVALID_ARG, "req_offsets must run from 0 to n=%lld", (long long)n);
+  for (int r = 0; r < R; ++r) {
+    if (req_offsets[r + 1] < req_offsets[r]) return fail(TR_ERR_INVALID_ARG, "req_offsets decrease at %d", r);
+    if (req_offsets[r + 1] - req_offsets[r] >= (int64_t)1 << 31)
+      return fail(TR_ERR_UNSUPPORTED, "request %d has 2^31 or more candidates", r);
+  }
+  if (!out_idx || (n > 0 && !scores)) return fail(TR_ERR_INVALID_ARG, "null device pointer");
+  return launch_topk(scores, req_offsets, R, k, out_idx, out_score, (cudaStream_t)stream);
+}
+
 tr_status tr_sync_status(tr_stream stream, int timeout_ms) {
   const cudaStream_t st = (cudaStream_t)stream;
   const auto t0 = std::chrono::steady_clock::now();

@@ -142,6 +142,14 @@ class DeviceWorkload:
         api.score_candidates(self.model, self.tokens, self.req_offsets, self.kv, self.L_u, self.domain,
                              self.scores, stream=stream)
 
+    def select(self, k: int, stream=None):
+        """Per-request top-k of the last step's scores (tr_topk): (indices within each
+        request [R, k] int64, scores [R, k] fp32), padded with -1 / -inf."""
+        if not hasattr(self, "_sel") or self._sel[0].shape != (len(self.reqs), k):
+            self._sel = (torch.empty(len(self.reqs), k, dtype=torch.int64, device=self.device),
+                         torch.empty(len(self.reqs), k, dtype=torch.float32, device=self.device))
+        return api.topk(self.scores, self.req_offsets, k, self._sel[0], self._sel[1], stream=stream)
+
     def step(self, stream=None, events=None) -> torch.Tensor:
         """One request batch.  The user aggregation (a few small launches) runs first on the
         caller's stream; then the user prefill (one CTA per request, which needs a whole SM)
