@@ -132,6 +132,26 @@ tr_status tr_aggregate(const tr_table* tables, int n_tables, const int32_t* bag_
                        int64_t n_bags, int D, tr_dtype out_dtype, void* out, tr_stream stream);
 
 /*
+ * Aggregator variants of tr_aggregate (TransRetrieval §3.2 names them as the alternatives
+ * weighted average replaces; they are here for that comparison).  Same arguments and layout
+ * as tr_aggregate plus `mode`:
+ *   TR_AGG_MEAN  sum_i v_i h(k_i) / sum_i v_i   (tr_aggregate; zero when sum_i v_i = 0)
+ *   TR_AGG_SUM   sum_i v_i h(k_i)               (the weighted sum of §3.2's profiling paragraph)
+ *   TR_AGG_MAX   max_i h(k_i) element-wise     (max pooling; weights unused; empty bag -> 0)
+ * optionally OR-ed with
+ *   TR_AGG_POST_LN  LayerNorm over the D columns of each token, without gain or shift, eps 1e-5
+ *                   (post-aggregation LayerNorm).
+ * Any other value is rejected with TR_ERR_INVALID_ARG.
+ */
+#define TR_AGG_MEAN 0
+#define TR_AGG_SUM 1
+#define TR_AGG_MAX 2
+#define TR_AGG_POST_LN 0x100
+tr_status tr_aggregate_ex(const tr_table* tables, int n_tables, const int32_t* bag_table, const int64_t* offsets,
+                          const int32_t* keys, const float* weights, int64_t n_bags, int D, tr_dtype out_dtype,
+                          int mode, void* out, tr_stream stream);
+
+/*
  * Bytes of one request's user K/V cache for L_u user tokens (0 <= L_u <= TR_MAX_LU).
  * Layout (opaque to most callers; tests decode it):
  *   TR_F32 model : [n_layer][2][L_u][D] fp32, K then V, row-major.

@@ -96,6 +96,36 @@ def weighted_sum(rows, offsets, keys, weights) -> np.ndarray:
     return out
 
 
+def max_pool(rows, offsets, keys) -> np.ndarray:
+    """Element-wise maximum of a bag's embedding rows: the max-pooling aggregator §3.2
+    rejects (extreme-value bias).  Weights do not enter; an empty bag gives zeros."""
+    rows = np.asarray(rows, dtype=np.float64)
+    offsets = np.asarray(offsets, dtype=np.int64)
+    out = np.zeros((len(offsets) - 1, rows.shape[1]))
+    for b in range(len(offsets) - 1):
+        s, e = offsets[b], offsets[b + 1]
+        if e > s:
+            out[b] = rows[np.asarray(keys[s:e], dtype=np.int64)].max(axis=0)
+    return out
+
+
+def aggregate(rows, offsets, keys, weights, mode: str = "mean", post_ln: bool = False) -> np.ndarray:
+    """One token per bag with the aggregator `mode` ("mean": weighted average, §3.2;
+    "sum": weighted sum; "max": max pooling), optionally followed by the post-aggregation
+    LayerNorm §3.2 compares against (no affine parameters, eps as everywhere else)."""
+    if mode == "mean":
+        o = weighted_average(rows, offsets, keys, weights)
+    elif mode == "sum":
+        o = weighted_sum(rows, offsets, keys, weights)
+    elif mode == "max":
+        o = max_pool(rows, offsets, keys)
+    else:
+        raise ValueError(mode)
+    if post_ln:
+        o = layer_norm(o, np.ones(o.shape[1]), np.zeros(o.shape[1]))
+    return o
+
+
 # ------------------------------------------------------------------ building blocks
 
 def layer_norm(x: np.ndarray, g: np.ndarray, b: np.ndarray) -> np.ndarray:

@@ -67,3 +67,14 @@ def test_topk_host_validation_without_gpu(lib):
     assert lib.tr_topk(None, 5, bad, 2, 5, None, None, None) == L.TR_ERR_INVALID_ARG          # decreasing
     assert lib.tr_topk(None, 9, off, 2, 5, None, None, None) == L.TR_ERR_INVALID_ARG          # null outputs
     assert b"null" in lib.tr_last_error()
+
+
+def test_aggregate_ex_mode_validation_without_gpu(lib):
+    from transformer_candidate_scoring_b200 import _lib as L
+    t = (L.Table * 1)(L.Table(16, 10, 1))
+    # unknown modes are rejected before anything else is looked at; n_bags == 0 is a no-op
+    for bad in (3, 7, -1, 0x200, 0x100 | 5):
+        assert lib.tr_aggregate_ex(t, 1, None, None, None, None, 5, 128, 1, bad, None, None) == L.TR_ERR_INVALID_ARG
+        assert b"mode" in lib.tr_last_error()
+    for ok in (0, 1, 2, 0x100, 0x101, 0x102):
+        assert lib.tr_aggregate_ex(t, 1, None, None, None, None, 0, 128, 1, ok, None, None) == L.TR_OK

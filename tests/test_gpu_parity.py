@@ -110,6 +110,44 @@ def test_aggregate_parity(dt, D, out_dt, n_bags, max_nf):
     assert tr().sync_status() == 0
 
 
+def _oracle_agg_mode(seed, bags, rows, D, dt, mode, post_ln):
+    tab_of_key = np.repeat(bags.bag_table.astype(np.int64), np.diff(bags.offsets))
+    out_rows = np.zeros((len(bags.keys), D))
+    for t in np.unique(tab_of_key):
+        sel = tab_of_key == t
+        out_rows[sel] = datagen.table_rows_host(seed, int(t), bags.keys[sel], D, dt)
+    return oracle.aggregate(out_rows, bags.offsets, np.arange(len(bags.keys)), bags.weights, mode, post_ln)
+
+
+@pytest.mark.parametrize("mode", ["mean", "sum", "max"])
+@pytest.mark.parametrize("post_ln", [False, True])
+@pytest.mark.parametrize("dt,D", [("bf16", 128), ("f32", 64), ("bf16", 32)])
+def test_aggregate_variants_parity(mode, post_ln, dt, D):
+    """The §3.2 alternatives (weighted sum, max pooling, post-aggregation LayerNorm) against
+    the oracle; max pooling without LayerNorm is exact."""
+    rng = np.random.default_rng(D + len(mode) + post_ln)
+    rows = 3000
+    tables = _tables(12, 2, rows, D, dt)
+    bags = _bags(rng, 2500, 40, rows, 2)
+    out = torch.empty(bags.n_bags, D, dtype=torch.float32, device="cuda")
+    tr().aggregate(tables, dev(bags.bag_table), dev(bags.offsets), dev(bags.keys), dev(bags.weights), out,
+                   mode=mode, post_ln=post_ln)
+    torch.cuda.synchronize()
+    got = out.double().cpu().numpy()
+    ref = _oracle_agg_mode(12, bags, rows, D, dt, mode, post_ln)
+    empty = np.diff(bags.offsets) == 0
+    assert np.all(got[empty] == 0)
+    if mode == "max" and not post_ln:
+        assert np.array_equal(got, ref)
+    elif post_ln:
+        # LayerNorm output is O(1); fp32 accumulation and normalisation
+        np.testing.assert_allclose(got, ref, rtol=0, atol=2e-4)
+    else:
+        scale = float(np.abs(ref).max())
+        assert np.all(np.abs(got - ref) <= 2e-6 * scale), float(np.abs(got - ref).max() / scale)
+    assert tr().sync_status() == 0
+
+
 def test_aggregate_scale_invariance_is_bitexact():
     rng = np.random.default_rng(5)
     tables = _tables(3, 2, 3000, 128, "bf16")

@@ -375,3 +375,61 @@ def test_compressor_flops():
 def test_topk_order_and_ties():
     s = np.array([0.5, 0.9, 0.5, -1.0, 0.9, 0.1])
     assert T.topk(s, 4).tolist() == [1, 4, 0, 2]
+
+
+# ---------------------------------------------------------------- aggregator variants (§3.2)
+
+def test_max_pool_pins():
+    rng = np.random.default_rng(21)
+    rows = rng.standard_normal((50, 6))
+    off = np.array([0, 1, 4, 4, 9])
+    keys = rng.integers(0, 50, 9)
+    got = T.max_pool(rows, off, keys)
+    # single-key bag returns its row; empty bag zeros; element-wise maximum by plain loops
+    assert np.array_equal(got[0], rows[keys[0]])
+    assert np.array_equal(got[2], np.zeros(6))
+    for b, (s, e) in enumerate(zip(off[:-1], off[1:])):
+        if e == s:
+            continue
+        for d in range(6):
+            m = -np.inf
+            for i in range(s, e):
+                m = max(m, rows[keys[i], d])
+            assert got[b, d] == m
+    # permutation of a bag's keys does not matter; duplicating a key does not either
+    perm = keys.copy()
+    perm[1:4] = perm[1:4][::-1]
+    assert np.array_equal(T.max_pool(rows, off, perm), got)
+    # the extreme-value bias §3.2 names: the maximum is >= the weighted average (positive weights)
+    w = rng.uniform(0.1, 1, 9)
+    avg = T.weighted_average(rows, off, keys, w)
+    ne = np.diff(off) > 0
+    assert np.all(got[ne] >= avg[ne] - 1e-12)
+
+
+def test_aggregate_modes_and_post_layernorm():
+    import torch
+    rng = np.random.default_rng(22)
+    rows = rng.standard_normal((40, 8))
+    off = np.array([0, 3, 7, 12])
+    keys = rng.integers(0, 40, 12)
+    w = rng.uniform(0.1, 1, 12)
+    assert np.array_equal(T.aggregate(rows, off, keys, w, "mean"), T.weighted_average(rows, off, keys, w))
+    assert np.array_equal(T.aggregate(rows, off, keys, w, "sum"), T.weighted_sum(rows, off, keys, w))
+    assert np.array_equal(T.aggregate(rows, off, keys, w, "max"), T.max_pool(rows, off, keys))
+    for mode in ("mean", "sum", "max"):
+        base = T.aggregate(rows, off, keys, w, mode)
+        ln = T.aggregate(rows, off, keys, w, mode, post_ln=True)
+        ref = torch.nn.functional.layer_norm(torch.from_numpy(base), (8,), eps=T.EPS).numpy()
+        np.testing.assert_allclose(ln, ref, rtol=1e-12, atol=1e-12)
+    # LayerNorm erases the per-field magnitude: scaling all weights of the weighted sum leaves
+    # the normalised token unchanged up to the eps inside the square root
+    s1 = T.aggregate(rows, off, keys, w, "sum", post_ln=True)
+    s2 = T.aggregate(rows, off, keys, 7.0 * w, "sum", post_ln=True)
+    np.testing.assert_allclose(s1, s2, rtol=0, atol=1e-4)
+    assert np.abs(s1 - s2).max() > 0
+    try:
+        T.aggregate(rows, off, keys, w, "median")
+        assert False
+    except ValueError:
+        pass

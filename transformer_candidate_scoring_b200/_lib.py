@@ -45,6 +45,8 @@ SIGNATURES = {
     "tr_model_destroy": (None, [C.c_void_p]),
     "tr_aggregate": (C.c_int, [C.POINTER(Table), C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
                                C.c_int64, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
+    "tr_aggregate_ex": (C.c_int, [C.POINTER(Table), C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p,
+                               C.c_int64, C.c_int, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
     "tr_kv_cache_bytes": (C.c_size_t, [C.c_void_p, C.c_int]),
     "tr_prefill_user": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),
     "tr_prefill_user_noalloc": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p]),

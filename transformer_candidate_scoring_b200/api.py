@@ -117,17 +117,28 @@ class Model:
             pass
 
 
+AGG_MODES = {"mean": 0, "sum": 1, "max": 2}
+AGG_POST_LN = 0x100
+
+
 def aggregate(tables: Sequence[torch.Tensor], bag_table: torch.Tensor, offsets: torch.Tensor,
-              keys: torch.Tensor, weights: torch.Tensor, out: torch.Tensor, stream=None) -> torch.Tensor:
-    """tr_aggregate: weighted average of each bag into out [n_bags, D]."""
+              keys: torch.Tensor, weights: torch.Tensor, out: torch.Tensor, stream=None, mode: str = "mean",
+              post_ln: bool = False) -> torch.Tensor:
+    """tr_aggregate (mode "mean", no LayerNorm) or tr_aggregate_ex: one token per bag into
+    out [n_bags, D]."""
     n = len(tables)
     arr = (L.Table * max(n, 1))()
     for i, t in enumerate(tables):
         arr[i] = L.Table(t.data_ptr(), t.shape[0], dtype_code(t.dtype))
     D = out.shape[-1]
     n_bags = offsets.numel() - 1
-    _check(L.load().tr_aggregate(arr, n, _ptr(bag_table), _ptr(offsets), _ptr(keys), _ptr(weights),
-                                 n_bags, D, dtype_code(out.dtype), _ptr(out), _stream(stream)))
+    if mode == "mean" and not post_ln:
+        _check(L.load().tr_aggregate(arr, n, _ptr(bag_table), _ptr(offsets), _ptr(keys), _ptr(weights),
+                                     n_bags, D, dtype_code(out.dtype), _ptr(out), _stream(stream)))
+    else:
+        code = AGG_MODES[mode] | (AGG_POST_LN if post_ln else 0)
+        _check(L.load().tr_aggregate_ex(arr, n, _ptr(bag_table), _ptr(offsets), _ptr(keys), _ptr(weights),
+                                        n_bags, D, dtype_code(out.dtype), code, _ptr(out), _stream(stream)))
     return out
 
 

@@ -82,13 +82,15 @@ __device__ __forceinline__ void store_out<__nv_bfloat16, 4>(__nv_bfloat16* dst, 
 // them behind the previous bag: the next bag's table id and offsets are requested when a
 // bag starts, and its first LPR keys and weights once the current rows are in flight.
 // Loop trip counts are the warp's maximum, so every shuffle is warp-uniform.
-template <typename T, typename O, int LPR, int CI>
+// VAR = false compiles the plain weighted average (TR_AGG_MEAN without LayerNorm) only;
+// VAR = true reads the aggregator and the LayerNorm flag from `mode`.
+template <typename T, typename O, int LPR, int CI, bool VAR>
 __global__ void __launch_bounds__(256, 4) wavg_kernel(TableSet tabs, int n_tables,
                                                       const int32_t* __restrict__ bag_table,
                                                       const int64_t* __restrict__ offsets,
                                                       const int32_t* __restrict__ keys,
                                                       const float* __restrict__ weights, int64_t n_bags,
-                                                      O* __restrict__ out, int* status) {
+                                                      int mode, O* __restrict__ out, int* status) {
   constexpr int NV = Vec16<T>::N;
   constexpr int D = LPR * CI * NV;
   constexpr int G = 32 / LPR;                 // bags per warp
@@ -98,6 +100,8 @@ __global__ void __launch_bounds__(256, 4) wavg_kernel(TableSet tabs, int n_table
   const int cl = lane % LPR;
   const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t stride = (int64_t)gridDim.x * (blockDim.x >> 5) * G;
+  const int agg = VAR ? mode & 0xFF : TR_AGG_MEAN;   // TR_AGG_MEAN / TR_AGG_SUM / TR_AGG_MAX
+  const bool is_max = VAR && agg == TR_AGG_MAX, post_ln = VAR && (mode & TR_AGG_POST_LN) != 0;
   bool bad = false;
 
   // the first bag's header and first key chunk
@@ -151,7 +155,7 @@ __global__ void __launch_bounds__(256, 4) wavg_kernel(TableSet tabs, int n_table
 #pragma unroll
     for (int c = 0; c < CI; ++c)
 #pragma unroll
-      for (int i = 0; i < NV; ++i) acc[c][i] = 0.f;
+      for (int i = 0; i < NV; ++i) acc[c][i] = is_max ? -INFINITY : 0.f;
     float wsum = 0.f;
     for (int base = 0; base < n_max; base += LPR) {
       const int cnt = n - base;                     // keys of this bag in the chunk (may be <= 0)
@@ -176,12 +180,14 @@ __global__ void __launch_bounds__(256, 4) wavg_kernel(TableSet tabs, int n_table
       for (int j0 = 0; j0 < cnt_max; j0 += UNROLL) {
         uint4 raw[UNROLL][CI];
         float wv[UNROLL];
+        bool lv[UNROLL];
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
           const int j = j0 + u;
           const int kk = __shfl_sync(0xffffffffu, k, j % LPR, LPR);
           wv[u] = __shfl_sync(0xffffffffu, v, j % LPR, LPR);
           const bool live = j < cnt && kk >= 0;
+          lv[u] = live;
           if (!live) wv[u] = 0.f;
           const uint4* row = reinterpret_cast<const uint4*>(table + (int64_t)(live ? kk : 0) * D);
 #pragma unroll
@@ -189,28 +195,70 @@ __global__ void __launch_bounds__(256, 4) wavg_kernel(TableSet tabs, int n_table
             raw[u][c] = live ? ld_stream(row + c * LPR + cl) : make_uint4(0, 0, 0, 0);
         }
         if (has_next && !next_keys) fetch_next_keys();   // overlaps these rows
+        if (is_max) {
 #pragma unroll
-        for (int u = 0; u < UNROLL; ++u)
+          for (int u = 0; u < UNROLL; ++u)
 #pragma unroll
-          for (int c = 0; c < CI; ++c) {
-            float f[NV];
-            Vec16<T>::unpack(raw[u][c], f);
+            for (int c = 0; c < CI; ++c) {
+              float f[NV];
+              Vec16<T>::unpack(raw[u][c], f);
 #pragma unroll
-            for (int i = 0; i < NV; ++i) acc[c][i] = fmaf(wv[u], f[i], acc[c][i]);
-          }
+              for (int i = 0; i < NV; ++i) acc[c][i] = lv[u] ? fmaxf(acc[c][i], f[i]) : acc[c][i];
+            }
+        } else {
+#pragma unroll
+          for (int u = 0; u < UNROLL; ++u)
+#pragma unroll
+            for (int c = 0; c < CI; ++c) {
+              float f[NV];
+              Vec16<T>::unpack(raw[u][c], f);
+#pragma unroll
+              for (int i = 0; i < NV; ++i) acc[c][i] = fmaf(wv[u], f[i], acc[c][i]);
+            }
+        }
       }
     }
     if (has_next && !next_keys) fetch_next_keys();   // empty or rejected bag
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+    // this lane's columns of the token: mean divides by the weight sum (zero when it is zero),
+    // sum keeps the accumulation, max gives zero for a bag without rows
+    float r[CI][NV];
+#pragma unroll
+    for (int c = 0; c < CI; ++c)
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const float a = acc[c][i];
+        r[c][i] = bad_table                ? 0.f
+                  : agg == TR_AGG_MEAN     ? (wsum != 0.f ? a / wsum : 0.f)
+                  : is_max                 ? (a == -INFINITY ? 0.f : a)
+                                           : a;
+      }
+    if (post_ln) {   // LayerNorm over the D columns, held by the LPR lanes of this group
+      float s = 0.f;
+#pragma unroll
+      for (int c = 0; c < CI; ++c)
+#pragma unroll
+        for (int i = 0; i < NV; ++i) s += r[c][i];
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      const float mean = s * (1.f / D);
+      float q = 0.f;
+#pragma unroll
+      for (int c = 0; c < CI; ++c)
+#pragma unroll
+        for (int i = 0; i < NV; ++i) q = fmaf(r[c][i] - mean, r[c][i] - mean, q);
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
+      const float rstd = rsqrtf(q * (1.f / D) + kLnEps);
+#pragma unroll
+      for (int c = 0; c < CI; ++c)
+#pragma unroll
+        for (int i = 0; i < NV; ++i) r[c][i] = (r[c][i] - mean) * rstd;
+    }
     if (live_bag) {
 #pragma unroll
-      for (int c = 0; c < CI; ++c) {
-        float r[NV];
-#pragma unroll
-        for (int i = 0; i < NV; ++i) r[i] = (wsum != 0.f && !bad_table) ? acc[c][i] / wsum : 0.f;
-        store_out<O, NV>(out + b * D + (c * LPR + cl) * NV, r);
-      }
+      for (int c = 0; c < CI; ++c) store_out<O, NV>(out + b * D + (c * LPR + cl) * NV, r[c]);
     }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, STATUS_KEY_RANGE);
@@ -218,8 +266,8 @@ __global__ void __launch_bounds__(256, 4) wavg_kernel(TableSet tabs, int n_table
 
 template <typename T, typename O>
 tr_status dispatch(const TableSet& ts, int n_tables, const int32_t* bag_table, const int64_t* offsets,
-                   const int32_t* keys, const float* weights, int64_t n_bags, int D, O* out, int* status,
-                   cudaStream_t st) {
+                   const int32_t* keys, const float* weights, int64_t n_bags, int D, int mode, O* out,
+                   int* status, cudaStream_t st) {
   constexpr int NV = Vec16<T>::N;
   const int vecs = D / NV;
   int dev = 0, sms = 148;
@@ -231,9 +279,13 @@ tr_status dispatch(const TableSet& ts, int n_tables, const int32_t* bag_table, c
   const int64_t bags_per_block = 8 * (32 / (vecs < 32 ? vecs : 32));
   const int64_t blocks_needed = (n_bags + bags_per_block - 1) / bags_per_block;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, (int64_t)sms * 32));
-#define TR_WAVG(LPR, CI)                                                                               \
-  wavg_kernel<T, O, LPR, CI><<<grid, 256, 0, st>>>(ts, n_tables, bag_table, offsets, keys, weights, \
-                                                   n_bags, out, status)
+#define TR_WAVG(LPR, CI)                                                                                     \
+  if (mode == TR_AGG_MEAN)                                                                                 \
+    wavg_kernel<T, O, LPR, CI, false><<<grid, 256, 0, st>>>(ts, n_tables, bag_table, offsets, keys, weights, \
+                                                            n_bags, mode, out, status);                      \
+  else                                                                                                     \
+    wavg_kernel<T, O, LPR, CI, true><<<grid, 256, 0, st>>>(ts, n_tables, bag_table, offsets, keys, weights,  \
+                                                           n_bags, mode, out, status)
   switch (vecs) {
     case 1: TR_WAVG(1, 1); break;
     case 2: TR_WAVG(2, 1); break;
@@ -254,7 +306,7 @@ tr_status dispatch(const TableSet& ts, int n_tables, const int32_t* bag_table, c
 
 tr_status launch_aggregate(const tr_table* tables, int n_tables, const int32_t* bag_table,
                            const int64_t* offsets, const int32_t* keys, const float* weights,
-                           int64_t n_bags, int D, tr_dtype out_dtype, void* out, cudaStream_t st) {
+                           int64_t n_bags, int D, tr_dtype out_dtype, int mode, void* out, cudaStream_t st) {
   DeviceState* ds = nullptr;
   TR_TRY(device_state(&ds));
   TableSet ts = {};
@@ -264,15 +316,15 @@ tr_status launch_aggregate(const tr_table* tables, int n_tables, const int32_t* 
   }
   const tr_dtype tdt = tables[0].dtype;
   if (tdt == TR_BF16 && out_dtype == TR_BF16)
-    return dispatch<__nv_bfloat16, __nv_bfloat16>(ts, n_tables, bag_table, offsets, keys, weights, n_bags, D,
+    return dispatch<__nv_bfloat16, __nv_bfloat16>(ts, n_tables, bag_table, offsets, keys, weights, n_bags, D, mode,
                                                   static_cast<__nv_bfloat16*>(out), ds->status, st);
   if (tdt == TR_BF16 && out_dtype == TR_F32)
-    return dispatch<__nv_bfloat16, float>(ts, n_tables, bag_table, offsets, keys, weights, n_bags, D,
+    return dispatch<__nv_bfloat16, float>(ts, n_tables, bag_table, offsets, keys, weights, n_bags, D, mode,
                                           static_cast<float*>(out), ds->status, st);
   if (tdt == TR_F32 && out_dtype == TR_F32)
-    return dispatch<float, float>(ts, n_tables, bag_table, offsets, keys, weights, n_bags, D,
+    return dispatch<float, float>(ts, n_tables, bag_table, offsets, keys, weights, n_bags, D, mode,
                                   static_cast<float*>(out), ds->status, st);
-  return dispatch<float, __nv_bfloat16>(ts, n_tables, bag_table, offsets, keys, weights, n_bags, D,
+  return dispatch<float, __nv_bfloat16>(ts, n_tables, bag_table, offsets, keys, weights, n_bags, D, mode,
                                         static_cast<__nv_bfloat16*>(out), ds->status, st);
 }
 

@@ -218,6 +218,16 @@ static tr_status check_model_device(const tr_model* m) {
 tr_status tr_aggregate(const tr_table* tables, int n_tables, const int32_t* bag_table, const int64_t* offsets,
                        const int32_t* keys, const float* weights, int64_t n_bags, int D, tr_dtype out_dtype,
                        void* out, tr_stream stream) {
+  return tr_aggregate_ex(tables, n_tables, bag_table, offsets, keys, weights, n_bags, D, out_dtype, TR_AGG_MEAN,
+                         out, stream);
+}
+
+tr_status tr_aggregate_ex(const tr_table* tables, int n_tables, const int32_t* bag_table, const int64_t* offsets,
+                          const int32_t* keys, const float* weights, int64_t n_bags, int D, tr_dtype out_dtype,
+                          int mode, void* out, tr_stream stream) {
+  const int agg = mode & ~TR_AGG_POST_LN;
+  if (agg != TR_AGG_MEAN && agg != TR_AGG_SUM && agg != TR_AGG_MAX)
+    return fail(TR_ERR_INVALID_ARG, "aggregation mode %d", mode);
   if (n_bags < 0) return fail(TR_ERR_INVALID_ARG, "n_bags=%lld", (long long)n_bags);
   if (n_bags == 0) return TR_OK;
   if (!tables || n_tables <= 0 || n_tables > TR_MAX_TABLES)
@@ -231,7 +241,7 @@ tr_status tr_aggregate(const tr_table* tables, int n_tables, const int32_t* bag_
     if ((uintptr_t)tables[i].data % 16) return fail(TR_ERR_INVALID_ARG, "table %d is not 16-byte aligned", i);
   }
   if ((uintptr_t)out % 16) return fail(TR_ERR_INVALID_ARG, "out is not 16-byte aligned");
-  return launch_aggregate(tables, n_tables, bag_table, offsets, keys, weights, n_bags, D, out_dtype, out,
+  return launch_aggregate(tables, n_tables, bag_table, offsets, keys, weights, n_bags, D, out_dtype, mode, out,
                           (cudaStream_t)stream);
 }
 

@@ -48,5 +48,5 @@ tr_status launch_topk(const float* scores, const int64_t* req_offsets, int R, in
                       float* out_score, cudaStream_t st);
 tr_status launch_aggregate(const tr_table* tables, int n_tables, const int32_t* bag_table,
                            const int64_t* offsets, const int32_t* keys, const float* weights,
-                           int64_t n_bags, int D, tr_dtype out_dtype, void* out, cudaStream_t st);
+                           int64_t n_bags, int D, tr_dtype out_dtype, int mode, void* out, cudaStream_t st);
 }  // namespace tr

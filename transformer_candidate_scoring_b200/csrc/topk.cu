@@ -19,6 +19,7 @@ namespace {
 
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
+constexpr int kUnroll = 8;   // score loads in flight per thread
 
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f);
@@ -36,8 +37,7 @@ struct TopkParams {
 
 __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ TopkParams p) {
   __shared__ uint32_t hist[kWarps][256];
-  __shared__ uint32_t tot[256];
-  __shared__ uint32_t s_prefix, s_krem, s_sel_gt, s_warp_eq[kWarps], s_eq_base;
+  __shared__ uint32_t s_prefix, s_krem, s_sel_gt, s_warp_eq[kWarps], s_eq_base, s_eq_total;
   extern __shared__ unsigned long long sel[];              // [k_pow2] composite sort keys
   const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long long b0 = p.off[r], n = p.off[r + 1] - p.off[r];
@@ -51,26 +51,45 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ 
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < kWarps * 256; i += kThreads) (&hist[0][0])[i] = 0u;
       __syncthreads();
-      for (long long i = tid; i < n; i += kThreads) {
-        const uint32_t key = order_key(__ldg(sc + i));
-        if ((key & mask) == prefix) atomicAdd(&hist[warp][(key >> shift) & 0xFFu], 1u);
+      // eight loads in flight per thread (the pass is bound by load latency, not atomics)
+      for (long long i0 = 0; i0 < n; i0 += (long long)kThreads * kUnroll) {
+        uint32_t key[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const long long i = i0 + (long long)u * kThreads + tid;
+          key[u] = i < n ? order_key(__ldg(sc + i)) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const long long i = i0 + (long long)u * kThreads + tid;
+          if (i < n && (key[u] & mask) == prefix) atomicAdd(&hist[warp][(key[u] >> shift) & 0xFFu], 1u);
+        }
+      }
+      __syncthreads();
+      // bin totals from the top digit down, as an inclusive scan over 256 threads: thread t
+      // holds digit 255 - t, and the digit whose running count first reaches krem wins
+      __shared__ uint32_t s_wsum[8];
+      uint32_t cnt = 0, incl = 0;
+      if (tid < 256) {
+        const int d = 255 - tid;
+        for (int w = 0; w < kWarps; ++w) cnt += hist[w][d];
+        incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (lane == 31) s_wsum[warp] = incl;
       }
       __syncthreads();
       if (tid < 256) {
-        uint32_t s = 0;
-        for (int w = 0; w < kWarps; ++w) s += hist[w][tid];
-        tot[tid] = s;
-      }
-      __syncthreads();
-      if (tid == 0) {   // from the top digit down: the digit holding the krem-th largest
-        uint32_t above = 0;
-        int d = 255;
-        for (; d > 0; --d) {
-          if (above + tot[d] >= krem) break;
-          above += tot[d];
+        for (int w = 0; w < warp; ++w) incl += s_wsum[w];
+        const uint32_t excl = incl - cnt;
+        if (excl < krem && krem <= incl) {
+          s_prefix = prefix | ((uint32_t)(255 - tid) << shift);
+          s_krem = krem - excl;
+          s_eq_total = cnt;   // after the last pass: how many scores equal the threshold
         }
-        s_prefix = prefix | ((uint32_t)d << shift);
-        s_krem = krem - above;
       }
       __syncthreads();
       prefix = s_prefix;
@@ -86,35 +105,64 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ 
     s_eq_base = 0;
   }
   __syncthreads();
-  // ---- collect in index order (chunks of kThreads); ties ranked by a block scan
+  // ---- collect.  When every score equal to the threshold is kept (always, unless ties
+  // straddle the k-th place) one unordered pass suffices; otherwise the equal scores are
+  // ranked by index with a block scan, chunk by chunk in index order.
   const int n_gt = all ? 0 : take - (int)krem;   // slots [0, n_gt) for keys above thr
-  for (long long c0 = 0; c0 < n; c0 += kThreads) {
-    const long long i = c0 + tid;
-    uint32_t key = 0;
-    bool gt = false, eq = false;
-    if (i < n) {
-      key = order_key(__ldg(sc + i));
-      gt = all || key > thr;
-      eq = !all && key == thr;
+  const bool keep_all_eq = all || s_eq_total == krem;
+  for (long long g0 = 0; keep_all_eq && g0 < n; g0 += (long long)kThreads * kUnroll) {
+    uint32_t keys[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long i = g0 + (long long)u * kThreads + tid;
+      keys[u] = i < n ? order_key(__ldg(sc + i)) : 0u;
     }
-    if (gt) {
-      const uint32_t slot = atomicAdd(&s_sel_gt, 1u);
-      sel[slot] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)i);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long i = g0 + (long long)u * kThreads + tid;
+      const bool in = i < n && (all || keys[u] >= thr);
+      const unsigned bal = __ballot_sync(0xffffffffu, in);
+      uint32_t base = 0;
+      if (lane == 0 && bal) base = atomicAdd(&s_sel_gt, (uint32_t)__popc(bal));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (in) sel[base + __popc(bal & ((1u << lane) - 1u))] = ((unsigned long long)keys[u] << 32) | (0xFFFFFFFFu - (uint32_t)i);
     }
-    const unsigned bal = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) s_warp_eq[warp] = __popc(bal);
-    __syncthreads();
-    uint32_t before = s_eq_base;
-    for (int w = 0; w < warp; ++w) before += s_warp_eq[w];
-    before += __popc(bal & ((1u << lane) - 1u));
-    if (eq && before < krem) sel[n_gt + before] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)i);
-    __syncthreads();
-    if (tid == 0) {
-      uint32_t s = 0;
-      for (int w = 0; w < kWarps; ++w) s += s_warp_eq[w];
-      s_eq_base += s;
+  }
+  for (long long g0 = 0; !keep_all_eq && g0 < n; g0 += (long long)kThreads * kUnroll) {
+    uint32_t keys[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {   // the loads of eight chunks first
+      const long long i = g0 + (long long)u * kThreads + tid;
+      keys[u] = i < n ? order_key(__ldg(sc + i)) : 0u;
     }
-    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {   // then the chunks in index order
+      const long long c0 = g0 + (long long)u * kThreads;
+      if (c0 >= n) break;
+      const long long i = c0 + tid;
+      const uint32_t key = keys[u];
+      const bool gt = i < n && (all || key > thr);
+      const bool eq = i < n && !all && key == thr;
+      const unsigned bal_gt = __ballot_sync(0xffffffffu, gt);   // one slot reservation per warp
+      uint32_t base = 0;
+      if (lane == 0 && bal_gt) base = atomicAdd(&s_sel_gt, (uint32_t)__popc(bal_gt));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (gt) sel[base + __popc(bal_gt & ((1u << lane) - 1u))] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)i);
+      const unsigned bal = __ballot_sync(0xffffffffu, eq);
+      if (lane == 0) s_warp_eq[warp] = __popc(bal);
+      __syncthreads();
+      uint32_t before = s_eq_base;
+      for (int w = 0; w < warp; ++w) before += s_warp_eq[w];
+      before += __popc(bal & ((1u << lane) - 1u));
+      if (eq && before < krem) sel[n_gt + before] = ((unsigned long long)key << 32) | (0xFFFFFFFFu - (uint32_t)i);
+      __syncthreads();
+      if (tid == 0) {
+        uint32_t t = 0;
+        for (int w = 0; w < kWarps; ++w) t += s_warp_eq[w];
+        s_eq_base += t;
+      }
+      __syncthreads();
+    }
   }
   // pad to the sort size with the smallest composite key
   for (int i = take + tid; i < p.k_pow2; i += kThreads) sel[i] = 0ull;
