@@ -397,6 +397,41 @@ def run_case(args):
     print(f"case {args.case}: ok")
 
 
+def run_bulk(args):
+    """Near-line bulk compression (the index-build path): --case-n items of the 128D-5L
+    workload's target side (8 fields over the 4M-row target tables, uniform keys),
+    aggregated and compressed in chunks of 256K items; prints one JSON line with items/s.
+    Not the headline: the step above is."""
+    import torch
+
+    from transformer_candidate_scoring_b200 import api
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, compress_corpus
+
+    w = datagen.WORKLOADS[WORKLOAD]
+    dims = w.dims
+    n = args.case_n
+    tables = DeviceWorkload.make_tables(w.with_(user_tables=0), torch.device("cuda"))
+    model = api.Model(dims, datagen.workload_params(w))
+    bags = DeviceBags.of(datagen.make_target_bags(np.random.default_rng(w.seed + 77), w, n), "cuda")
+    out = torch.empty(n, dims.D, dtype=torch.bfloat16, device="cuda")
+    F = dims.n_target_fields
+    compress_corpus(model, tables[1], bags, n, F, out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(1, args.case_reps)
+    e0.record()
+    for _ in range(reps):
+        compress_corpus(model, tables[1], bags, n, F, out)
+    e1.record()
+    torch.cuda.synchronize()
+    if api.sync_status() != 0:
+        raise RuntimeError("device status word set")
+    sec = e0.elapsed_time(e1) / 1e3 / reps
+    print(json.dumps({"case": "bulk_compression", "items": n, "items_per_s": n / sec, "ms": sec * 1e3,
+                      "workload": "128D-5L target side, 8 fields, 4M-row tables, chunks of 262144 items"}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -405,11 +440,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--case", choices=["score", "compress", "prefill", "all"], default=None,
+    ap.add_argument("--case", choices=["score", "compress", "prefill", "all", "bulk"], default=None,
                     help="run one stage on stand-alone inputs for a profiler (no timing, no JSON)")
     ap.add_argument("--case-n", type=int, default=40000)
     ap.add_argument("--case-reps", type=int, default=2)
     args = ap.parse_args()
+    if args.case == "bulk":
+        run_bulk(args)
+        return
     if args.case:
         run_case(args)
         return

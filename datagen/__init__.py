@@ -9,7 +9,7 @@ from __future__ import annotations
 import numpy as np
 
 from .configs import WORKLOADS, ModelDims, Workload, scaled
-from .bags import Bags, Request, make_requests, scale_weights
+from .bags import Bags, Request, make_requests, make_target_bags, scale_weights
 from .params import Params, make_params, workload_params
 from .tables import fill_table_device, table_rows_host, f32_to_bf16_rne
 from .stage_inputs import rand_matrix
@@ -46,7 +46,7 @@ def compact_rows(w: Workload, bags: Bags, side: str):
 
 
 __all__ = [
-    "WORKLOADS", "ModelDims", "Workload", "scaled", "Bags", "Request", "make_requests",
+    "WORKLOADS", "ModelDims", "Workload", "scaled", "Bags", "Request", "make_requests", "make_target_bags",
     "scale_weights", "Params", "make_params", "workload_params", "fill_table_device",
     "table_rows_host", "f32_to_bf16_rne", "rand_matrix", "user_table_id", "target_table_id", "compact_rows",
 ]

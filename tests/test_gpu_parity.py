@@ -390,3 +390,41 @@ def test_host_feed_matches_device_resident_steps():
     assert tr().sync_status() == 0
     for i in range(7):
         assert torch.equal(out[i], ref[i % 3].cpu()), i
+
+
+def test_compress_corpus_chunked_equals_one_pass_and_oracle():
+    """Near-line bulk compression in chunks (with a ragged last chunk) gives the same bits
+    as one aggregate + compress pass over all items, and matches the oracle on a sample."""
+    from transformer_candidate_scoring_b200 import api
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, compress_corpus
+    w = datagen.scaled(datagen.WORKLOADS["128d5l"], n_cand_per_request=64, rows=20000)
+    dw = DeviceWorkload(w)
+    n_items = 5000
+    bags = datagen.make_target_bags(np.random.default_rng(4), w, n_items)
+    db = DeviceBags.of(bags, "cuda")
+    F, D = w.dims.n_target_fields, w.dims.D
+    out = torch.empty(n_items, D, dtype=torch.bfloat16, device="cuda")
+    compress_corpus(dw.model, dw.target_tables, db, n_items, F, out, chunk=1536)
+    X = torch.empty(n_items, F * D, dtype=torch.bfloat16, device="cuda")
+    api.aggregate(dw.target_tables, db.bag_table, db.offsets, db.keys, db.weights, X.view(-1, D))
+    ref_gpu = torch.empty(n_items, D, dtype=torch.bfloat16, device="cuda")
+    api.compress_targets(dw.model, X, ref_gpu)
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    assert torch.equal(out, ref_gpu)
+    # oracle on a sample of items (including the last, ragged chunk)
+    idx = np.array([0, 1, 1535, 1536, 3071, 4607, 4999])
+    rows = []
+    for i in idx:
+        sub = datagen.Bags(bags.offsets[i * F:(i + 1) * F + 1] - bags.offsets[i * F],
+                           bags.keys[bags.offsets[i * F]:bags.offsets[(i + 1) * F]],
+                           bags.weights[bags.offsets[i * F]:bags.offsets[(i + 1) * F]], bags.bag_table[i * F:(i + 1) * F])
+        toks = []
+        for f in range(F):
+            k = sub.keys[sub.offsets[f]:sub.offsets[f + 1]]
+            r = datagen.table_rows_host(w.seed, datagen.target_table_id(w, int(sub.bag_table[f])), k, D, "bf16")
+            toks.append(oracle.weighted_average(r, np.array([0, len(k)]), np.arange(len(k)),
+                                                sub.weights[sub.offsets[f]:sub.offsets[f + 1]])[0])
+        rows.append(np.concatenate(toks))
+    ref = oracle.compress_targets(dw.params, np.stack(rows))
+    check_close(out[torch.from_numpy(idx).cuda()].double().cpu().numpy(), ref, "bf16", "corpus sample")

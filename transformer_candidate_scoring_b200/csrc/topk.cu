@@ -62,7 +62,18 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ 
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
           const long long i = i0 + (long long)u * kThreads + tid;
-          if (i < n && (key[u] & mask) == prefix) atomicAdd(&hist[warp][(key[u] >> shift) & 0xFFu], 1u);
+          const bool hit = i < n && (key[u] & mask) == prefix;
+          const uint32_t digit = (key[u] >> shift) & 0xFFu;
+          // a request's scores share their high bits, so a warp's hits often fall in one
+          // bin: then one lane adds them all instead of 32 serialised atomics
+          const unsigned bal = __ballot_sync(0xffffffffu, hit);
+          if (!bal) continue;
+          const uint32_t d0 = __shfl_sync(0xffffffffu, digit, __ffs(bal) - 1);
+          if (__all_sync(0xffffffffu, !hit || digit == d0)) {
+            if (lane == 0) atomicAdd(&hist[warp][d0], (uint32_t)__popc(bal));
+          } else if (hit) {
+            atomicAdd(&hist[warp][digit], 1u);
+          }
         }
       }
       __syncthreads();

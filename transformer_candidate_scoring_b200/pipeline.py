@@ -263,3 +263,23 @@ class HostFeed:
             self.dw.step(main)
             self.free[i % 2].record(main)
             host_scores[i % len(host_scores)].copy_(self.dw.scores, non_blocking=True)
+
+
+def compress_corpus(model, target_tables, bags: DeviceBags, n_items: int, n_fields: int, out: torch.Tensor,
+                    chunk: int = 1 << 18, stream=None) -> torch.Tensor:
+    """Near-line index build (TransRetrieval §3.3: the compressed target token is also the
+    item's index vector, computed off the request path): every item of a corpus, its
+    ``n_fields`` target-field bags aggregated (tr_aggregate) and compressed
+    (tr_compress_targets) into ``out`` [n_items, D], ``chunk`` items at a time through one
+    [chunk, F*D] buffer.  ``bags`` holds the corpus's bags on the device, item i's fields at
+    bags i*F .. i*F+F-1 (CSR offsets into the full key/weight arrays)."""
+    D = out.shape[1]
+    X = torch.empty(min(chunk, max(n_items, 1)), n_fields * D, dtype=out.dtype, device=out.device)
+    for c0 in range(0, n_items, chunk):
+        c1 = min(n_items, c0 + chunk)
+        m = c1 - c0
+        b0, b1 = c0 * n_fields, c1 * n_fields
+        api.aggregate(target_tables, bags.bag_table[b0:b1], bags.offsets[b0:b1 + 1], bags.keys, bags.weights,
+                      X[:m].view(-1, D), stream=stream)
+        api.compress_targets(model, X[:m], out[c0:c1], stream=stream)
+    return out
