@@ -428,3 +428,21 @@ def test_compress_corpus_chunked_equals_one_pass_and_oracle():
         rows.append(np.concatenate(toks))
     ref = oracle.compress_targets(dw.params, np.stack(rows))
     check_close(out[torch.from_numpy(idx).cuda()].double().cpu().numpy(), ref, "bf16", "corpus sample")
+
+
+def test_captured_step_replays_bit_identical():
+    """A step captured into a CUDA graph and replayed gives the eager step's scores bit for
+    bit (same kernels, same inputs)."""
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload
+    w = datagen.scaled(datagen.WORKLOADS["packed"], n_cand_per_request=300, rows=20000)
+    dw = DeviceWorkload(w)
+    dw.step()
+    torch.cuda.synchronize()
+    ref = dw.scores.clone()
+    dw.scores.zero_()
+    g = dw.capture_step(torch.cuda.Stream())
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    assert torch.equal(dw.scores, ref)

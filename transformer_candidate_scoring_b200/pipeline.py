@@ -150,6 +150,16 @@ class DeviceWorkload:
                          torch.empty(len(self.reqs), k, dtype=torch.float32, device=self.device))
         return api.topk(self.scores, self.req_offsets, k, self._sel[0], self._sel[1], stream=stream)
 
+    def capture_step(self, stream=None) -> "torch.cuda.CUDAGraph":
+        """One step with the current bags, captured into a CUDA graph (replay it to run the
+        step again without host launch overhead; the bags, caches and activations it reads
+        and writes are the ones bound now).  Run an eager step first: the library sets up
+        per-device state on first use, which capture does not allow."""
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            self.step()
+        return g
+
     def step(self, stream=None, events=None) -> torch.Tensor:
         """One request batch.  The user aggregation (a few small launches) runs first on the
         caller's stream; then the user prefill (one CTA per request, which needs a whole SM)
