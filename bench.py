@@ -468,6 +468,48 @@ def run_bulk(args):
           flush=True)
 
 
+def run_uncompressed(args):
+    """The cost target compression removes (§3.3): --case-n candidates of one 128D-5L request
+    scored as L_t = 8 uncompressed field tokens and as one compressed token, both on the
+    CUDA-core path (the only path that takes L_t > 1), plus the tensor-core single-token path
+    for reference; prints one JSON line with the times and the FLOP ratio."""
+    import torch
+
+    from transformer_candidate_scoring_b200 import api
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload
+
+    w = datagen.scaled(datagen.WORKLOADS[WORKLOAD], n_cand_per_request=args.case_n, rows=200_000)
+    dims = w.dims
+    dw = DeviceWorkload(w)
+    dw.step()
+    torch.cuda.synchronize()
+    F, D, n = dims.n_target_fields, dims.D, dw.n_cand
+    X = dw.X.view(n, F, D)
+    s = torch.empty(n, dtype=torch.float32, device="cuda")
+    args_kv = (dw.req_offsets, dw.kv, dw.L_u, dw.domain, s)
+
+    def timed(fn, reps=3):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+    t8 = timed(lambda: api.score_candidates_uncompressed(dw.model, X, F, *args_kv))
+    t1 = timed(lambda: api.score_candidates_uncompressed(dw.model, dw.tokens, 1, *args_kv))
+    ttc = timed(lambda: api.score_candidates(dw.model, dw.tokens, *args_kv))
+    L_u = dw.L_u[0]
+    f8 = dims.n_layer * (16 * F * D * D + 4 * F * (L_u + F) * D) + 2 * D * F
+    f1 = stack_flops_per_candidate(dims, L_u)
+    print(json.dumps({"case": "uncompressed_targets", "candidates": n, "L_t": F, "L_u": L_u,
+                      "ms_L_t_8_cuda_cores": t8, "ms_L_t_1_cuda_cores": t1, "ms_L_t_1_tensor_cores": ttc,
+                      "time_saving_cuda_cores": 1 - t1 / t8, "flops_per_candidate_L_t_8": f8,
+                      "flops_per_candidate_L_t_1": f1, "flop_saving": 1 - f1 / f8}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -476,13 +518,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--case", choices=["score", "compress", "prefill", "all", "bulk"], default=None,
+    ap.add_argument("--case", choices=["score", "compress", "prefill", "all", "bulk", "uncompressed"], default=None,
                     help="run one stage on stand-alone inputs for a profiler (no timing, no JSON)")
     ap.add_argument("--case-n", type=int, default=40000)
     ap.add_argument("--case-reps", type=int, default=2)
     args = ap.parse_args()
     if args.case == "bulk":
         run_bulk(args)
+        return
+    if args.case == "uncompressed":
+        run_uncompressed(args)
         return
     if args.case:
         run_case(args)

@@ -205,6 +205,23 @@ tr_status tr_score_candidates(const tr_model* m, const void* tokens, int64_t n,
                               tr_stream stream);
 
 /*
+ * The uncompressed-target variant (TransRetrieval §3.3 compares against it): each candidate
+ * is L_t target tokens instead of one compressed token.  Every token runs through the same
+ * layer stack, attending to its request's L_u cached user keys/values and to the keys/values
+ * of its own candidate's L_t tokens (never another candidate's); the candidate's score is the
+ * mean over its tokens of w_head . LayerNorm_f(y_t) + b_head.  With L_t = 1 this is
+ * tr_score_candidates.  It runs on the CUDA-core path (fp32 arithmetic, any model dtype): it
+ * exists to measure the per-candidate cost that target compression removes, not for serving.
+ *   tokens      DEVICE [n][L_t][D] of the model dtype (candidate c's tokens are rows c*L_t ..)
+ *   L_t         1 .. TR_MAX_LT
+ *   req_offsets, kv, L_u, domain, R, scores: as tr_score_candidates (n counts candidates).
+ */
+#define TR_MAX_LT 16
+tr_status tr_score_candidates_uncompressed(const tr_model* m, const void* tokens, int64_t n, int L_t,
+                                           const int64_t* req_offsets, const void* const* kv, const int32_t* L_u,
+                                           const int32_t* domain, int R, float* scores, tr_stream stream);
+
+/*
  * Per-request top-k of the scores (the selection step of GPU retrieval, TransRetrieval
  * deployment section "Hardware-aware inference optimization": a request's scored candidates
  * are reduced to the best k on the GPU).

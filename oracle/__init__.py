@@ -6,12 +6,12 @@ import it; the product package never does, and shares no code with it.  The only
 module both sides use is ``datagen`` (seeded inputs, none of the method's arithmetic).
 """
 from .transretrieval import (EPS, FlopCounter, compress_targets, flops_per_candidate_closed_form,
-                             layer_norm, prefill_user, prelu, score_candidates, topk,
+                             layer_norm, prefill_user, prelu, score_candidates, score_candidates_uncompressed, topk,
                              weighted_average, weighted_sum, max_pool, aggregate)
 from .pipeline import aggregate_bags, score_request, score_request_candidates
 
 __all__ = [
     "EPS", "FlopCounter", "compress_targets", "flops_per_candidate_closed_form", "layer_norm",
-    "prefill_user", "prelu", "score_candidates", "topk", "weighted_average", "weighted_sum", "max_pool", "aggregate",
+    "prefill_user", "prelu", "score_candidates", "score_candidates_uncompressed", "topk", "weighted_average", "weighted_sum", "max_pool", "aggregate",
     "score_request", "score_request_candidates", "aggregate_bags",
 ]

@@ -245,6 +245,41 @@ def score_candidates(P, n_head: int, tokens: np.ndarray, K: np.ndarray, V: np.nd
     return (_mm(z, _p(P, "w_head")[:, None]) + _p(P, "b_head"))[:, 0]
 
 
+def score_candidates_uncompressed(P, n_head: int, tokens: np.ndarray, K: np.ndarray, V: np.ndarray,
+                                  domain: int) -> np.ndarray:
+    """The uncompressed-target alternative §3.3 measures compression against: a candidate is
+    L_t target tokens (tokens: [n, L_t, D]).  Each token attends to the request's L_u cached
+    user keys/values and to the keys/values of its own candidate's L_t tokens, as the tokens
+    of [user tokens..., candidate tokens] do when user tokens cannot see the candidate;
+    candidates never see each other.  The score is the mean over the candidate's tokens of
+    w . LayerNorm_f(y_t) + b (the pages give no head for this variant; reading).  With
+    L_t = 1 this is score_candidates.  Returns [n]."""
+    t = np.asarray(tokens, dtype=np.float64)
+    n, L_t, D = t.shape
+    y = t.reshape(n * L_t, D) + _p(P, "domain_emb")[domain]
+    dh = D // n_head
+    L_u = K.shape[1]
+    for l in range(K.shape[0]):
+        q, k, v = _qkv(P, l, y)
+        qh, kh, vh = (_split_heads(x, n_head).reshape(n, L_t, n_head, dh) for x in (q, k, v))
+        Ku = _split_heads(np.asarray(K[l], dtype=np.float64), n_head)
+        Vu = _split_heads(np.asarray(V[l], dtype=np.float64), n_head)
+        s_user = np.einsum("cthd,lhd->cthl", qh, Ku)
+        s_own = np.einsum("cthd,cshd->cths", qh, kh)                   # own candidate's tokens
+        _count(2 * n * L_t * (L_u + L_t) * D)
+        sc = np.concatenate([s_user, s_own], axis=-1) / np.sqrt(dh)     # [n, L_t, H, L_u + L_t]
+        sc = sc - sc.max(axis=-1, keepdims=True)
+        p = np.exp(sc)
+        p = p / p.sum(axis=-1, keepdims=True)
+        o = np.einsum("cthl,lhd->cthd", p[..., :L_u], Vu) + np.einsum("cths,cshd->cthd", p[..., L_u:], vh)
+        _count(2 * n * L_t * (L_u + L_t) * D)
+        y = y + _mm(o.reshape(n * L_t, D), _p(P, f"l{l}.Wo")) + _p(P, f"l{l}.bo")
+        y = y + _ffn(P, l, y)
+    z = layer_norm(y, _p(P, "lnf_g"), _p(P, "lnf_b"))
+    per_token = (_mm(z, _p(P, "w_head")[:, None]) + _p(P, "b_head"))[:, 0]
+    return per_token.reshape(n, L_t).mean(axis=1)
+
+
 def topk(scores: np.ndarray, k: int) -> np.ndarray:
     """Indices of the k largest scores, descending; equal scores by lower index first."""
     s = np.asarray(scores, dtype=np.float64)

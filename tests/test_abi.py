@@ -78,3 +78,10 @@ def test_aggregate_ex_mode_validation_without_gpu(lib):
         assert b"mode" in lib.tr_last_error()
     for ok in (0, 1, 2, 0x100, 0x101, 0x102):
         assert lib.tr_aggregate_ex(t, 1, None, None, None, None, 0, 128, 1, ok, None, None) == L.TR_OK
+
+
+def test_uncompressed_host_validation_without_gpu(lib):
+    from transformer_candidate_scoring_b200 import _lib as L
+    # a null model handle is refused before anything else
+    assert lib.tr_score_candidates_uncompressed(None, None, 0, 8, None, None, None, None, 1, None,
+                                                None) == L.TR_ERR_INVALID_ARG

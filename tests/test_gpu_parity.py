@@ -446,3 +446,39 @@ def test_captured_step_replays_bit_identical():
     torch.cuda.synchronize()
     assert tr().sync_status() == 0
     assert torch.equal(dw.scores, ref)
+
+
+@pytest.mark.parametrize("name,init,L_t,L_us,n_per", [
+    ("tiny", "wide", 4, [8, 3], [37, 20]),
+    ("tiny", "paper", 8, [8], [50]),
+    ("64d3l", "wide", 8, [32, 0], [40, 9]),
+    ("128d5l", "wide", 8, [64], [60]),
+])
+def test_uncompressed_targets_parity(name, init, L_t, L_us, n_per):
+    """Candidates of L_t target tokens (the variant target compression replaces) against the
+    oracle, packed requests included."""
+    dims, P, m, users, _, doms, kvs = _score_setup(name, init, L_us, n_per)
+    std = 0.5 if init == "wide" else 0.3
+    toks = [datagen.rand_matrix(300 + r, (n, L_t, dims.D), std, dims.dtype) for r, n in enumerate(n_per)]
+    T = dev(np.concatenate(toks), tdt(dims.dtype))
+    off = np.concatenate([[0], np.cumsum(n_per)]).tolist()
+    s = torch.empty(off[-1], dtype=torch.float32, device="cuda")
+    tr().api.score_candidates_uncompressed(m, T, L_t, off, kvs, L_us, doms, s)
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    got = s.cpu().numpy().astype(np.float64)
+    for r, (U, t, d) in enumerate(zip(users, toks, doms)):
+        K, V = oracle.prefill_user(P, dims.n_head, U, d)
+        ref = oracle.score_candidates_uncompressed(P, dims.n_head, t, K, V, d)
+        check_close(got[off[r]:off[r + 1]], ref, dims.dtype, f"request {r}")
+
+
+def test_uncompressed_with_one_token_equals_single_token_path_fp32():
+    """L_t = 1 on the fp32 model runs the same CUDA-core code as tr_score_candidates: bit-equal."""
+    dims, P, m, users, toks, doms, kvs = _score_setup("tiny", "wide", [8, 5], [40, 17])
+    a, off = _gpu_scores(m, dims, toks, kvs, [8, 5], doms)
+    T = dev(np.concatenate(toks), tdt(dims.dtype))
+    s = torch.empty(int(off[-1]), dtype=torch.float32, device="cuda")
+    tr().api.score_candidates_uncompressed(m, T, 1, off.tolist(), kvs, [8, 5], doms, s)
+    torch.cuda.synchronize()
+    assert np.array_equal(s.cpu().numpy().astype(np.float64), a)

@@ -433,3 +433,73 @@ def test_aggregate_modes_and_post_layernorm():
         assert False
     except ValueError:
         pass
+
+
+# ---------------------------------------------------------------- uncompressed targets (§3.3)
+
+def _torch_full_sequence_scores_multi(P, dims, user_tokens, tokens, domain):
+    """Brute force for candidates of L_t tokens: each candidate's tokens run as the tail of
+    [users..., candidate tokens] through PyTorch's encoder layers, users masked from the
+    candidate's tokens; score = mean over the candidate's tokens of the head."""
+    D, H, N = dims.D, dims.n_head, dims.n_layer
+    s = np.asarray(P["domain_emb"], np.float64)[domain]
+    n, L_t, _ = tokens.shape
+    L_u = len(user_tokens)
+    seq = np.concatenate([np.broadcast_to(user_tokens + s, (n, L_u, D)), tokens + s], axis=1)
+    x = torch.from_numpy(np.ascontiguousarray(seq))
+    mask = torch.zeros(L_u + L_t, L_u + L_t, dtype=torch.bool)
+    mask[:L_u, L_u:] = True
+    with torch.no_grad():
+        for l in range(N):
+            x = torch_layer(P, l, D, H)(x, src_mask=mask)
+        z = _ln(P["lnf_g"], P["lnf_b"])(x[:, L_u:])
+    per = (z.numpy() @ np.asarray(P["w_head"], np.float64)) + float(np.asarray(P["b_head"]))
+    return per.mean(axis=1)
+
+
+@pytest.mark.parametrize("L_t", [1, 3, 8])
+def test_uncompressed_scores_equal_full_sequence_forward(L_t):
+    dims = _dims(D=32, N=2, H=2)
+    P = _wide_params(dims, 5)
+    rng = _rng(40 + L_t)
+    users = rng.normal(size=(6, dims.D))
+    K, V = T.prefill_user(P, dims.n_head, users, 1)
+    toks = rng.normal(size=(5, L_t, dims.D))
+    got = T.score_candidates_uncompressed(P, dims.n_head, toks, K, V, 1)
+    ref = _torch_full_sequence_scores_multi(P, dims, users, toks, 1)
+    np.testing.assert_allclose(got, ref, rtol=1e-9, atol=1e-10)
+
+
+def test_uncompressed_reduces_to_single_token_and_is_permutation_invariant():
+    dims = _dims(D=32, N=2, H=2)
+    P = _wide_params(dims, 6)
+    rng = _rng(50)
+    users = rng.normal(size=(7, dims.D))
+    K, V = T.prefill_user(P, dims.n_head, users, 0)
+    one = rng.normal(size=(9, dims.D))
+    np.testing.assert_allclose(T.score_candidates_uncompressed(P, dims.n_head, one[:, None, :], K, V, 0),
+                               T.score_candidates(P, dims.n_head, one, K, V, 0), rtol=1e-12, atol=1e-12)
+    toks = rng.normal(size=(4, 5, dims.D))
+    a = T.score_candidates_uncompressed(P, dims.n_head, toks, K, V, 0)
+    b = T.score_candidates_uncompressed(P, dims.n_head, toks[:, ::-1], K, V, 0)   # own tokens reversed
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+    c = T.score_candidates_uncompressed(P, dims.n_head, toks[[2]], K, V, 0)        # batch-mates do not matter
+    np.testing.assert_allclose(c, a[[2]], rtol=1e-12, atol=1e-12)
+
+
+def test_uncompressed_flops_and_the_compression_saving():
+    """Instrumented FLOPs of the L_t-token stack = N (16 L_t D^2 + 4 L_t (L_u + L_t) D) + 2 D L_t,
+    and at the 128D-5L backbone (L_t = 8 fields, L_u = 64) compression to one token saves
+    about 85 % of the per-candidate FLOPs (§3.3 and the summary's claim)."""
+    D, N, L_u, L_t = 32, 2, 8, 4
+    dims = _dims(D=D, N=N, H=2)
+    P = datagen.make_params(dims, 0)
+    rng = _rng(60)
+    K = rng.normal(size=(N, L_u, D))
+    V = rng.normal(size=(N, L_u, D))
+    with T.FlopCounter() as fc:
+        T.score_candidates_uncompressed(P, dims.n_head, rng.normal(size=(3, L_t, D)), K, V, 0)
+    assert fc.flops == 3 * (N * (16 * L_t * D * D + 4 * L_t * (L_u + L_t) * D) + 2 * D * L_t)
+    full = T.flops_per_candidate_closed_form(128, 5, 64, L_t=8, self_term=False, head=False)
+    comp = T.flops_per_candidate_closed_form(128, 5, 64, L_t=1, self_term=False, head=False)
+    assert 0.85 <= 1 - comp / full <= 0.90

@@ -12,6 +12,7 @@ TR_F32, TR_BF16 = 0, 1
 TR_MAX_TABLES, TR_MAX_REQUESTS, TR_MAX_LU = 64, 64, 256
 TR_NOALLOC_SCRATCH_BYTES = 1 << 20
 TR_MAX_TOPK = 4096
+TR_MAX_LT = 16
 
 _fp = C.POINTER(C.c_float)
 
@@ -54,6 +55,9 @@ SIGNATURES = {
     "tr_score_candidates": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.POINTER(C.c_int64),
                                       C.POINTER(C.c_void_p), C.POINTER(C.c_int32), C.POINTER(C.c_int32),
                                       C.c_int, C.c_void_p, C.c_void_p]),
+    "tr_score_candidates_uncompressed": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int64, C.c_int, C.POINTER(C.c_int64),
+                                                   C.POINTER(C.c_void_p), C.POINTER(C.c_int32), C.POINTER(C.c_int32),
+                                                   C.c_int, C.c_void_p, C.c_void_p]),
     "tr_topk": (C.c_int, [C.c_void_p, C.c_int64, C.POINTER(C.c_int64), C.c_int, C.c_int, C.c_void_p, C.c_void_p,
                           C.c_void_p]),
     "tr_sync_status": (C.c_int, [C.c_void_p, C.c_int]),

@@ -181,6 +181,21 @@ def score_candidates(model: Model, tokens: torch.Tensor, req_offsets: Sequence[i
     return scores
 
 
+def score_candidates_uncompressed(model: Model, tokens: torch.Tensor, L_t: int, req_offsets: Sequence[int],
+                                  kv: Sequence[torch.Tensor], L_u: Sequence[int], domain: Sequence[int],
+                                  scores: torch.Tensor, stream=None) -> torch.Tensor:
+    """tr_score_candidates_uncompressed: candidates of L_t target tokens each (tokens
+    [n, L_t, D] or [n*L_t, D]); scores [n] fp32."""
+    R = len(L_u)
+    off = (C.c_int64 * (R + 1))(*[int(x) for x in req_offsets])
+    kvp = (C.c_void_p * R)(*[(k.data_ptr() if k is not None and k.numel() else 0) for k in kv])
+    lu = (C.c_int32 * R)(*[int(x) for x in L_u])
+    dm = (C.c_int32 * R)(*[int(x) for x in domain])
+    _check(L.load().tr_score_candidates_uncompressed(model.handle, _ptr(tokens), int(req_offsets[-1]), int(L_t), off,
+                                                     kvp, lu, dm, R, _ptr(scores), _stream(stream)))
+    return scores
+
+
 def topk(scores: torch.Tensor, req_offsets: Sequence[int], k: int, out_idx: torch.Tensor = None,
          out_score: torch.Tensor = None, stream=None):
     """tr_topk: per-request top-k; returns (out_idx int64 [R, k], out_score fp32 [R, k])."""

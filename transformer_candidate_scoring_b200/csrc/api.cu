@@ -307,6 +307,30 @@ tr_status tr_score_candidates(const tr_model* m, const void* tokens, int64_t n, 
   return TR_OK;
 }
 
+tr_status tr_score_candidates_uncompressed(const tr_model* m, const void* tokens, int64_t n, int L_t,
+                                           const int64_t* req_offsets, const void* const* kv, const int32_t* L_u,
+                                           const int32_t* domain, int R, float* scores, tr_stream stream) {
+  TR_TRY(check_model_device(m));
+  if (L_t < 1 || L_t > TR_MAX_LT) return fail(TR_ERR_INVALID_ARG, "L_t=%d (need 1..%d)", L_t, TR_MAX_LT);
+  if (R < 1 || R > TR_MAX_REQUESTS) return fail(TR_ERR_INVALID_ARG, "R=%d (need 1..%d)", R, TR_MAX_REQUESTS);
+  if (!req_offsets || !kv || !L_u || !domain) return fail(TR_ERR_INVALID_ARG, "null host array");
+  if (n < 0 || req_offsets[0] != 0 || req_offsets[R] != n)
+    return fail(TR_ERR_INVALID_ARG, "req_offsets must run from 0 to n=%lld", (long long)n);
+  for (int r = 0; r < R; ++r) {
+    if (req_offsets[r + 1] < req_offsets[r]) return fail(TR_ERR_INVALID_ARG, "req_offsets decrease at %d", r);
+    if (L_u[r] < 0 || L_u[r] > TR_MAX_LU) return fail(TR_ERR_INVALID_ARG, "L_u[%d]=%d", r, L_u[r]);
+    if (domain[r] < 0 || domain[r] >= m->desc.n_domains) return fail(TR_ERR_INVALID_ARG, "domain[%d]=%d", r, domain[r]);
+    if (L_u[r] > 0 && req_offsets[r + 1] > req_offsets[r] && !kv[r])
+      return fail(TR_ERR_INVALID_ARG, "kv[%d] is null", r);
+  }
+  if (n == 0) return TR_OK;
+  if (!tokens || !scores) return fail(TR_ERR_INVALID_ARG, "null device pointer");
+  const cudaStream_t st = (cudaStream_t)stream;
+  for (int r = 0; r < R; ++r)
+    TR_TRY(simt_score_lt(m, tokens, req_offsets[r], req_offsets[r + 1], L_t, kv[r], L_u[r], domain[r], scores, st));
+  return TR_OK;
+}
+
 tr_status tr_topk(const float* scores, int64_t n, const int64_t* req_offsets, int R, int k, int64_t* out_idx,
                   float* out_score, tr_stream stream) {
   if (R < 1 || R > TR_MAX_REQUESTS) return fail(TR_ERR_INVALID_ARG, "R=%d (need 1..%d)", R, TR_MAX_REQUESTS);

@@ -145,12 +145,14 @@ struct KvBf16Image {
   }
 };
 
-// One warp per (row, head): softmax over the L_u user keys (+ the row's own key when
-// kself != nullptr) of q.k / sqrt(d_h), then the weighted sum of values.
+// One warp per (row, head): softmax over the L_u user keys plus the keys of the row's own
+// candidate (Lt rows: rows (row / Lt) * Lt .. + Lt - 1, i.e. the row itself when Lt = 1,
+// none when Lt = 0) of q.k / sqrt(d_h), then the weighted sum of values.
+constexpr int kMaxLt = 16;
 template <typename KV>
 __global__ void attention_rows(const float* __restrict__ q, int ldq, const float* __restrict__ kself,
                                const float* __restrict__ vself, int ldself, KV kv, int L_u, int M, int H,
-                               float* __restrict__ o, int ldo) {
+                               float* __restrict__ o, int ldo, int Lt) {
   const int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (w >= (int64_t)M * H) return;
@@ -174,15 +176,21 @@ __global__ void attention_rows(const float* __restrict__ q, int ldq, const float
       mx = fmaxf(mx, s[t]);
     }
   }
-  float sself = -INFINITY;
-  if (kself) {
-    float a = 0.f;
+  const int64_t g0 = Lt > 0 ? (int64_t)(row / Lt) * Lt : 0;   // first row of this candidate
+  float sself[kMaxLt];
 #pragma unroll
-    for (int d = 0; d < kDHead; ++d) a = fmaf(qv[d], kself[(int64_t)row * ldself + h * kDHead + d], a);
-    sself = a * scale;
+  for (int t = 0; t < kMaxLt; ++t) {
+    sself[t] = -INFINITY;
+    if (t < Lt) {
+      float a = 0.f;
+#pragma unroll
+      for (int d = 0; d < kDHead; ++d) a = fmaf(qv[d], kself[(g0 + t) * ldself + h * kDHead + d], a);
+      sself[t] = a * scale;
+    }
   }
   for (int off = 16; off; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-  mx = fmaxf(mx, sself);
+#pragma unroll
+  for (int t = 0; t < kMaxLt; ++t) mx = fmaxf(mx, sself[t]);
   float acc[kDHead] = {};
   float sum = 0.f;
 #pragma unroll
@@ -200,11 +208,14 @@ __global__ void attention_rows(const float* __restrict__ q, int ldq, const float
 #pragma unroll
     for (int d = 0; d < kDHead; ++d) acc[d] += __shfl_xor_sync(0xffffffffu, acc[d], off);
   }
-  if (kself) {
-    const float p = __expf(sself - mx);
-    sum += p;
 #pragma unroll
-    for (int d = 0; d < kDHead; ++d) acc[d] = fmaf(p, vself[(int64_t)row * ldself + h * kDHead + d], acc[d]);
+  for (int t = 0; t < kMaxLt; ++t) {
+    if (t < Lt) {
+      const float p = __expf(sself[t] - mx);
+      sum += p;
+#pragma unroll
+      for (int d = 0; d < kDHead; ++d) acc[d] = fmaf(p, vself[(g0 + t) * ldself + h * kDHead + d], acc[d]);
+    }
   }
   if (lane < kDHead) {
     float r = 0.f;
@@ -274,7 +285,7 @@ __global__ void convert_rows(const float* __restrict__ X, TO* __restrict__ Y, in
 // One Pre-LN layer over M rows held in y (fp32 [M][D]); attention reads `kv`.
 template <typename KV>
 tr_status layer(const tr_model* m, int l, float* y, float* a, float* qkv, float* o, float* hbuf, int M, KV kv,
-                int L_u, bool self_term, void* kv_out, cudaStream_t st) {
+                int L_u, int lt, void* kv_out, cudaStream_t st) {
   const int D = m->desc.D, H = m->desc.ffn_hidden, NH = m->desc.n_head;
   const tr_layer_dev& L = m->layers[l];
   TR_TRY(layernorm<float>(y, D, a, D, M, D, nullptr, L.ln1_g, L.ln1_b, st));
@@ -289,9 +300,8 @@ tr_status layer(const tr_model* m, int l, float* y, float* a, float* qkv, float*
     TR_LAUNCH_CHECK("kv_write");
   }
   const int64_t warps = (int64_t)M * NH;
-  attention_rows<KV><<<ceil_div(warps, 8), 256, 0, st>>>(qkv, 3 * D, self_term ? qkv + D : nullptr,
-                                                          self_term ? qkv + 2 * D : nullptr, 3 * D, kv, L_u, M,
-                                                          NH, o, D);
+  attention_rows<KV><<<ceil_div(warps, 8), 256, 0, st>>>(qkv, 3 * D, qkv + D, qkv + 2 * D, 3 * D, kv, L_u, M, NH, o,
+                                                          D, lt);
   TR_LAUNCH_CHECK("attention_rows");
   TR_TRY(gemm<float>(o, D, L.Wo, D, L.bo, y, D, M, D, D, EPI_ACCUM, st));
   TR_TRY(layernorm<float>(y, D, a, D, M, D, nullptr, L.ln2_g, L.ln2_b, st));
@@ -321,7 +331,7 @@ tr_status simt_prefill(const tr_model* m, const float* user_tokens, int L_u, int
       kv_l = (__nv_bfloat16*)kv + (size_t)l * 2 * Lp * D;
     // attention among the users reads their fp32 K/V straight from the qkv buffer
     KvF32 self_kv{qkv + D, qkv + 2 * D, 3 * D};
-    TR_TRY(layer(m, l, y, a, qkv, o, hb, L_u, self_kv, L_u, false, kv_l, st));
+    TR_TRY(layer(m, l, y, a, qkv, o, hb, L_u, self_kv, L_u, 0, kv_l, st));
   }
   return TR_OK;
 }
@@ -355,20 +365,35 @@ tr_status simt_compress(const tr_model* m, const void* x, int64_t n, void* token
   return TR_OK;
 }
 
-tr_status simt_score(const tr_model* m, const void* tokens, int64_t c0, int64_t c1, const void* kv, int L_u,
-                     int domain, float* scores, cudaStream_t st) {
+// Mean of each group of lt consecutive per-token scores (one candidate's tokens).
+__global__ void group_mean(const float* __restrict__ x, int64_t n, int lt, float* __restrict__ out) {
+  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= n) return;
+  float s = 0.f;
+  for (int t = 0; t < lt; ++t) s += x[c * lt + t];
+  out[c] = s / lt;
+}
+
+// Candidates c0 .. c1-1, each of lt tokens (rows c*lt .. c*lt+lt-1 of `tokens`): every
+// token runs through the layers attending to the request's users and to its own
+// candidate's lt tokens; the candidate's score is the mean of its tokens' head outputs
+// (for lt = 1 the plain single-token score).
+tr_status simt_score_lt(const tr_model* m, const void* tokens, int64_t c0, int64_t c1, int lt, const void* kv,
+                        int L_u, int domain, float* scores, cudaStream_t st) {
   const int D = m->desc.D, H = m->desc.ffn_hidden;
-  const int64_t chunk = 16384;
+  const int64_t chunk = std::max<int64_t>(1, 16384 / lt);     // candidates per pass
   const int64_t n = c1 - c0;
   if (n <= 0) return TR_OK;
-  const int64_t rows = std::min<int64_t>(n, chunk);
+  const int64_t rows = std::min<int64_t>(n, chunk) * lt;
   float* ws = nullptr;
-  TR_TRY(workspace((size_t)rows * (6 * D + H) * sizeof(float), (void**)&ws));
+  TR_TRY(workspace((size_t)rows * (6 * D + H + 1) * sizeof(float), (void**)&ws));
   float *y = ws, *a = y + rows * D, *qkv = a + rows * D, *o = qkv + 3 * rows * D, *hb = o + rows * D;
+  float* tok_scores = hb + rows * H;
   const int Lp = round_up16(L_u);
-  for (int64_t r0 = c0; r0 < c1; r0 += chunk) {
-    const int M = (int)std::min<int64_t>(chunk, c1 - r0);
-    const int64_t cnt = (int64_t)M * D;
+  for (int64_t q0 = c0; q0 < c1; q0 += chunk) {
+    const int64_t nc = std::min<int64_t>(chunk, c1 - q0);
+    const int M = (int)(nc * lt);
+    const int64_t r0 = q0 * lt, cnt = (int64_t)M * D;
     if (m->desc.dtype == TR_F32)
       add_vec_rows<float><<<ceil_div(cnt, 256), 256, 0, st>>>((const float*)tokens + r0 * D, y, M, D,
                                                               m->domain_emb + (int64_t)domain * D);
@@ -379,17 +404,27 @@ tr_status simt_score(const tr_model* m, const void* tokens, int64_t c0, int64_t 
     for (int l = 0; l < m->desc.n_layer; ++l) {
       if (m->desc.dtype == TR_F32) {
         const float* base = (const float*)kv + (size_t)l * 2 * L_u * D;
-        TR_TRY(layer(m, l, y, a, qkv, o, hb, M, KvF32{base, base + (size_t)L_u * D, D}, L_u, true, nullptr, st));
+        TR_TRY(layer(m, l, y, a, qkv, o, hb, M, KvF32{base, base + (size_t)L_u * D, D}, L_u, lt, nullptr, st));
       } else {
         const __nv_bfloat16* base = (const __nv_bfloat16*)kv + (size_t)l * 2 * Lp * D;
-        TR_TRY(layer(m, l, y, a, qkv, o, hb, M, KvBf16Image{base, base + (size_t)Lp * D, Lp, D}, L_u, true, nullptr,
+        TR_TRY(layer(m, l, y, a, qkv, o, hb, M, KvBf16Image{base, base + (size_t)Lp * D, Lp, D}, L_u, lt, nullptr,
                      st));
       }
     }
-    head_rows<<<ceil_div(M, 8), 256, 0, st>>>(y, M, D, m->lnf_g, m->lnf_b, m->w_head, m->b_head, scores + r0);
+    float* dst = lt == 1 ? scores + q0 : tok_scores;
+    head_rows<<<ceil_div(M, 8), 256, 0, st>>>(y, M, D, m->lnf_g, m->lnf_b, m->w_head, m->b_head, dst);
     TR_LAUNCH_CHECK("head_rows");
+    if (lt > 1) {
+      group_mean<<<ceil_div(nc, 256), 256, 0, st>>>(tok_scores, nc, lt, scores + q0);
+      TR_LAUNCH_CHECK("group_mean");
+    }
   }
   return TR_OK;
+}
+
+tr_status simt_score(const tr_model* m, const void* tokens, int64_t c0, int64_t c1, const void* kv, int L_u,
+                     int domain, float* scores, cudaStream_t st) {
+  return simt_score_lt(m, tokens, c0, c1, 1, kv, L_u, domain, scores, st);
 }
 
 // ---------------------------------------------------------------- user side without allocation
@@ -436,7 +471,7 @@ tr_status simt_prefill_noalloc(const tr_model* m, const float* user_tokens, int 
     else
       kv_l = (__nv_bfloat16*)kv + (size_t)l * 2 * Lp * D;
     KvF32 self_kv{qkv + D, qkv + 2 * D, 3 * D};
-    TR_TRY(layer(m, l, y, a, qkv, o, hb, L_u, self_kv, L_u, false, kv_l, st));
+    TR_TRY(layer(m, l, y, a, qkv, o, hb, L_u, self_kv, L_u, 0, kv_l, st));
   }
   return TR_OK;
 }

@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ 
   const float* sc = p.scores + b0;
   const int k = p.k;
   const int take = (int)(n < k ? n : k);
+  const int n32 = (int)n;
 
   // ---- radix select: the key of the take-th largest score and how many equal to it to keep
   uint32_t prefix = 0, mask = 0, krem = (uint32_t)take;
@@ -51,29 +52,18 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ 
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < kWarps * 256; i += kThreads) (&hist[0][0])[i] = 0u;
       __syncthreads();
-      // eight loads in flight per thread (the pass is bound by load latency, not atomics)
-      for (long long i0 = 0; i0 < n; i0 += (long long)kThreads * kUnroll) {
+      // eight loads in flight per thread; 32-bit indices (a request has < 2^31 candidates)
+      for (int i0 = 0; i0 < n32; i0 += kThreads * kUnroll) {
         uint32_t key[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-          const long long i = i0 + (long long)u * kThreads + tid;
-          key[u] = i < n ? order_key(__ldg(sc + i)) : 0u;
+          const int i = i0 + u * kThreads + tid;
+          key[u] = i < n32 ? order_key(__ldg(sc + i)) : 0u;
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-          const long long i = i0 + (long long)u * kThreads + tid;
-          const bool hit = i < n && (key[u] & mask) == prefix;
-          const uint32_t digit = (key[u] >> shift) & 0xFFu;
-          // a request's scores share their high bits, so a warp's hits often fall in one
-          // bin: then one lane adds them all instead of 32 serialised atomics
-          const unsigned bal = __ballot_sync(0xffffffffu, hit);
-          if (!bal) continue;
-          const uint32_t d0 = __shfl_sync(0xffffffffu, digit, __ffs(bal) - 1);
-          if (__all_sync(0xffffffffu, !hit || digit == d0)) {
-            if (lane == 0) atomicAdd(&hist[warp][d0], (uint32_t)__popc(bal));
-          } else if (hit) {
-            atomicAdd(&hist[warp][digit], 1u);
-          }
+          const int i = i0 + u * kThreads + tid;
+          if (i < n32 && (key[u] & mask) == prefix) atomicAdd(&hist[warp][(key[u] >> shift) & 0xFFu], 1u);
         }
       }
       __syncthreads();
@@ -121,17 +111,17 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(const __grid_constant__ 
   // ranked by index with a block scan, chunk by chunk in index order.
   const int n_gt = all ? 0 : take - (int)krem;   // slots [0, n_gt) for keys above thr
   const bool keep_all_eq = all || s_eq_total == krem;
-  for (long long g0 = 0; keep_all_eq && g0 < n; g0 += (long long)kThreads * kUnroll) {
+  for (int g0 = 0; keep_all_eq && g0 < n32; g0 += kThreads * kUnroll) {
     uint32_t keys[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const long long i = g0 + (long long)u * kThreads + tid;
-      keys[u] = i < n ? order_key(__ldg(sc + i)) : 0u;
+      const int i = g0 + u * kThreads + tid;
+      keys[u] = i < n32 ? order_key(__ldg(sc + i)) : 0u;
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const long long i = g0 + (long long)u * kThreads + tid;
-      const bool in = i < n && (all || keys[u] >= thr);
+      const int i = g0 + u * kThreads + tid;
+      const bool in = i < n32 && (all || keys[u] >= thr);
       const unsigned bal = __ballot_sync(0xffffffffu, in);
       uint32_t base = 0;
       if (lane == 0 && bal) base = atomicAdd(&s_sel_gt, (uint32_t)__popc(bal));
