@@ -30,9 +30,6 @@ namespace {
 using namespace tc;
 
 constexpr int kM = 128;
-// Copies of the weight slices; CTA b streams copy b % kWeightCopies.  Measured on B200, more
-// than one copy did not change the kernel time, so one copy.
-constexpr int kWeightCopies = 1;
 constexpr int STAGE1 = 80 * 1024;              // x slice (16 KB) + W1 slice (<= 64 KB)
 constexpr int OFF_R1 = 0;
 constexpr int OFF_R2 = 2 * STAGE1;             // 160 KB
@@ -50,7 +47,6 @@ struct CompParams {
   const uint8_t* w1;           // [c0/64] slices of W1^T [c1 x 64]
   const uint8_t* w2;           // [c1/64] slices of W2^T [c2 x 64]
   const uint8_t* w3;           // [c2/64] slices of W3^T [c3 x 64]
-  size_t wcopy_bytes;          // bytes between weight copies
   const float* vec;            // b1 a1 g1 be1 (c1 each), b2 a2 g2 be2 (c2 each), b3 (c3)
   __nv_bfloat16* out;          // [n][c3]
   int* status;
@@ -79,7 +75,6 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
 __device__ void comp_producer(const CompParams& p, uint32_t r1, uint32_t r2, const CBars& b, volatile int* abort_flag) {
   int s1 = 0, s2 = 0;
   uint32_t ph1 = 0, ph2 = 0, free_phase = 0;
-  const size_t cp = (blockIdx.x % kWeightCopies) * p.wcopy_bytes;
   const uint32_t w1_bytes = p.c1 * 128, w2_bytes = p.c2 * 128, w3_bytes = p.c3 * 128;
   bool ok = true;
   bool pend1[2] = {false, false}, pend2[2] = {false, false};
@@ -93,7 +88,7 @@ __device__ void comp_producer(const CompParams& p, uint32_t r1, uint32_t r2, con
       const uint32_t st = r1 + s1 * STAGE1;
       mbar_arrive_expect_tx(b.full1[s1], kM * 64 * 2 + w1_bytes);
       tma_load_2d(st, &p.xmap, kc * 64, tile * kM, b.full1[s1]);
-      bulk_g2s(st + 16384, p.w1 + cp + (size_t)kc * w1_bytes, w1_bytes, b.full1[s1]);
+      bulk_g2s(st + 16384, p.w1 + (size_t)kc * w1_bytes, w1_bytes, b.full1[s1]);
       pend1[s1] = true;
       par1[s1] = ph1;
       if (++s1 == 2) { s1 = 0; ph1 ^= 1; }
@@ -102,7 +97,7 @@ __device__ void comp_producer(const CompParams& p, uint32_t r1, uint32_t r2, con
       if (!(ok = mbar_wait(b.empty2[s2], ph2 ^ 1, abort_flag))) break;
       const bool is2 = j < p.c1 / 64;
       const uint32_t bytes = is2 ? w2_bytes : w3_bytes;
-      const uint8_t* src = is2 ? p.w2 + cp + (size_t)j * w2_bytes : p.w3 + cp + (size_t)(j - p.c1 / 64) * w3_bytes;
+      const uint8_t* src = is2 ? p.w2 + (size_t)j * w2_bytes : p.w3 + (size_t)(j - p.c1 / 64) * w3_bytes;
       mbar_arrive_expect_tx(b.full2[s2], bytes);
       bulk_g2s(r2 + s2 * STAGE2, src, bytes, b.full2[s2]);
       pend2[s2] = true;
@@ -478,15 +473,13 @@ tr_status tc_build_comp(tr_model* m, const tr_model_weights* w) {
     vec.insert(vec.end(), w->comp_ln_b[i], w->comp_ln_b[i] + n);
   }
   vec.insert(vec.end(), w->comp_b[2], w->comp_b[2] + c[3]);
-  const size_t cb = img.size() * 2, ib = cb * kWeightCopies, vb = vec.size() * 4;
+  const size_t ib = img.size() * 2, vb = vec.size() * 4;
   void* blob = nullptr;
   if (cudaMalloc(&blob, ib + vb) != cudaSuccess) {
     cudaGetLastError();
     return fail(TR_ERR_NOMEM, "compressor weight images: allocation failed");
   }
-  for (int k = 0; k < kWeightCopies; ++k)
-    TR_CUDA_TRY(cudaMemcpy((uint8_t*)blob + k * cb, img.data(), cb, cudaMemcpyHostToDevice));
-  m->tc_comp_copy_bytes = cb;
+  TR_CUDA_TRY(cudaMemcpy(blob, img.data(), ib, cudaMemcpyHostToDevice));
   TR_CUDA_TRY(cudaMemcpy((uint8_t*)blob + ib, vec.data(), vb, cudaMemcpyHostToDevice));
   m->tc_comp = blob;
   m->tc_comp_vec = reinterpret_cast<const float*>((uint8_t*)blob + ib);
@@ -514,7 +507,6 @@ tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens,
   p.w1 = img;
   p.w2 = img + (size_t)c[0] * c[1] * 2;
   p.w3 = p.w2 + (size_t)c[1] * c[2] * 2;
-  p.wcopy_bytes = m->tc_comp_copy_bytes;
   p.vec = m->tc_comp_vec;
   p.out = static_cast<__nv_bfloat16*>(tokens);
   p.status = ds->status;

@@ -29,8 +29,6 @@ struct tr_model {
   size_t tc_bytes = 0;
   const void* tc_stack = nullptr;       // per-layer weight images of the candidate stack
   size_t tc_stack_layer_bytes = 0;
-  size_t tc_stack_copy_bytes = 0;       // bytes between the stack's weight-image copies
-  size_t tc_comp_copy_bytes = 0;        // bytes between the compressor's weight-image copies
   const float* tc_vec = nullptr;        // folded bias / gain vectors of the candidate stack
   size_t tc_vec_layer_floats = 0;
   const void* tc_comp = nullptr;        // compressor operand images

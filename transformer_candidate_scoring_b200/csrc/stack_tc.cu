@@ -77,10 +77,6 @@ constexpr int kThreads = 128 + kEpiThreads;
 constexpr int kEpiThread0 = 128;
 constexpr int kCtlRegs = 104, kEpiRegs = 200;
 static_assert(4 * 32 * kCtlRegs + 8 * 32 * kEpiRegs <= kThreads * 168, "register split exceeds the launch");
-// Copies of the weight images in global memory; CTA b streams copy b % kWeightCopies.  All
-// CTAs stream the same weights at about the same time; measured on B200, 16 copies gave the
-// same kernel time as one (the reads are not limited by L2 slice contention), so one copy.
-constexpr int kWeightCopies = 1;
 constexpr float kQScale = 0.25f * 1.44269504088896341f;  // 1/sqrt(d_h) * log2(e)
 
 // Items: Wq, Wk, Wv, Wo, W1 (output columns 0-127), W1 (128-255), W2 (input rows 0-127),
@@ -110,8 +106,7 @@ struct ReqInfo {
 struct StackParams {
   const __nv_bfloat16* tokens;
   float* scores;
-  const uint8_t* wimg;       // kWeightCopies x [n_layer][16][kSlot]
-  size_t wcopy_bytes;        // bytes between copies
+  const uint8_t* wimg;       // [n_layer][kItemsPerLayer][kSlot]
   const float* vec;          // [n_layer][kVecPerLayer] + [kVecFinal]
   const float* domain_emb;   // [n_domains][D]
   int* status;
@@ -199,7 +194,7 @@ __device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, co
   for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
     const TileInfo t = tile_info(p, tile);
     for (int l = 0; l < p.n_layer && ok; ++l) {
-      const uint8_t* wl = p.wimg + (blockIdx.x % kWeightCopies) * p.wcopy_bytes + (size_t)l * kItemsPerLayer * kSlot;
+      const uint8_t* wl = p.wimg + (size_t)l * kItemsPerLayer * kSlot;
       for (int j = 0; j < kItemsPerLayer && ok; ++j) {
         if (!PF && j == 3) {  // the request's K/V images go in between the QKV and O weights
           if (!(ok = mbar_wait(b.kv_empty(), kv_phase ^ 1, abort_flag))) break;
@@ -968,19 +963,16 @@ tr_status tc_build(tr_model* m, const tr_model_weights* w) {
     bh += (double)w->w_head[j] * w->lnf_b[j];
   }
   vf[D] = (float)bh;
-  const size_t copy_bytes = img.size() * 2, vec_bytes = vec.size() * 4;
-  const size_t img_bytes = copy_bytes * kWeightCopies;
+  const size_t img_bytes = img.size() * 2, vec_bytes = vec.size() * 4;
   const size_t total = img_bytes + ((vec_bytes + 255) & ~size_t(255));
   if (cudaMalloc(&m->tc_blob, total) != cudaSuccess) {
     cudaGetLastError();
     return fail(TR_ERR_NOMEM, "tensor-core weight images: allocation of %zu bytes failed", total);
   }
   m->tc_bytes = total;
-  for (int k = 0; k < kWeightCopies; ++k)
-    TR_CUDA_TRY(cudaMemcpy((uint8_t*)m->tc_blob + k * copy_bytes, img.data(), copy_bytes, cudaMemcpyHostToDevice));
+  TR_CUDA_TRY(cudaMemcpy(m->tc_blob, img.data(), img_bytes, cudaMemcpyHostToDevice));
   TR_CUDA_TRY(cudaMemcpy((uint8_t*)m->tc_blob + img_bytes, vec.data(), vec_bytes, cudaMemcpyHostToDevice));
   m->tc_stack = m->tc_blob;
-  m->tc_stack_copy_bytes = copy_bytes;
   m->tc_stack_layer_bytes = (size_t)kItemsPerLayer * kSlot;
   m->tc_vec = reinterpret_cast<const float*>((uint8_t*)m->tc_blob + img_bytes);
   m->tc_vec_layer_floats = kVecPerLayer;
@@ -1035,7 +1027,6 @@ tr_status tc_score(const tr_model* m, const void* tokens, int64_t n, const int64
     p.tokens = static_cast<const __nv_bfloat16*>(tokens);
     p.scores = scores;
     p.wimg = static_cast<const uint8_t*>(m->tc_stack);
-    p.wcopy_bytes = m->tc_stack_copy_bytes;
     p.vec = m->tc_vec;
     p.domain_emb = m->domain_emb;
     p.status = ds->status;
@@ -1071,7 +1062,6 @@ tr_status tc_prefill(const tr_model* m, const float* user_tokens, int L_u, int d
   TR_TRY(device_state(&ds));
   StackParams p{};
   p.wimg = static_cast<const uint8_t*>(m->tc_stack);
-  p.wcopy_bytes = m->tc_stack_copy_bytes;
   p.vec = m->tc_vec;
   p.domain_emb = m->domain_emb;
   p.status = ds->status;
