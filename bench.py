@@ -178,6 +178,15 @@ def time_oracle(w, P, req, target_seconds=15.0, max_cand=None):
     return rate, desc, threads, t_user + dt
 
 
+def bench_config(n_cand: int, L_u: int, world: int) -> dict:
+    """The workload both arms report."""
+    return {"workload": "128D-5L, 1 request x 40,000 candidates per GPU, L_u=64, 8 target fields, "
+                        "16+8 tables of 4M rows (24.6 GB bf16)",
+            "n_cand_per_gpu": n_cand, "L_u": L_u, "request_sets": N_REQUEST_SETS,
+            "l2": "inputs larger than L2: tables 24.6 GB, uniform target keys, rotating request sets",
+            "parallelism": f"candidate shards, {world} GPU(s), no collective"}
+
+
 def run_reference(args, rank, world):
     """Reference arm: the oracle as it stands on the host cores (rank 0 only)."""
     if rank != 0:
@@ -197,8 +206,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": v, "unit": "candidates/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.n_cand_per_request / v * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "128D-5L, 1 request x 40,000 candidates, L_u=64, 8 target fields, 4M-row tables",
-                   "n_cand": w.n_cand_per_request},
+        "config": bench_config(w.n_cand_per_request, 64, 1),
         "cpu_baseline": {"value": v, "unit": "candidates/s", "cores": threads, "kind": "oracle", "sample": desc},
         "e2e": {"value": v, "unit": "candidates/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -383,11 +391,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "candidates/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "128D-5L, 1 request x 40,000 candidates per GPU, L_u=64, 8 target fields, "
-                               "16+8 tables of 4M rows (24.6 GB bf16)",
-                   "n_cand_per_gpu": n_cand, "L_u": L_u, "request_sets": N_REQUEST_SETS,
-                   "l2": "inputs larger than L2: tables 24.6 GB, uniform target keys, rotating request sets",
-                   "parallelism": f"candidate shards, {world} GPU(s), no collective"},
+        "config": bench_config(n_cand, L_u, world),
         "roofline": roof,
         "stages": {k: {"ms": stage_ms[k], **({kk: vv for kk, vv in stage_roof[k].items()} if k in stage_roof else {})}
                    for k in stage_names},
