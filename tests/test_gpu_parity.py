@@ -390,6 +390,15 @@ def test_host_feed_matches_device_resident_steps():
     assert tr().sync_status() == 0
     for i in range(7):
         assert torch.equal(out[i], ref[i % 3].cpu()), i
+    # the same through replayed graphs (one per device slot and host batch)
+    feed.capture()
+    for o in out:
+        o.zero_()
+    feed.run(0, 7, out)
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    for i in range(7):
+        assert torch.equal(out[i], ref[i % 3].cpu()), ("graph", i)
 
 
 def test_compress_corpus_chunked_equals_one_pass_and_oracle():

@@ -256,10 +256,22 @@ class HostFeed:
                     dx.copy_(hx, non_blocking=True)
         self.ready[i % 2].record(cs)
 
+    def capture(self) -> None:
+        """Capture one CUDA graph per (device slot, host batch) pair, so that run() replays
+        the step instead of launching its kernels one by one.  Call it after one run(): the
+        library sets up per-device state on first use, which capture does not allow."""
+        self.graphs = {}
+        n = len(self.batches)
+        for i in range(2 * n if n % 2 else n):       # every (slot, batch) pair occurs
+            du, dt = self._views(i)
+            self.dw.use_bags(du, dt, self.batches[i % n][2])
+            self.graphs[(i % 2, i % n)] = self.dw.capture_step(torch.cuda.Stream(self.dw.device))
+
     def run(self, first: int, count: int, host_scores, stream=None) -> None:
         """Score batches first .. first + count - 1 (batch i uses host batch i mod len);
         the scores of batch i land in ``host_scores[i % len(host_scores)]`` (pinned)."""
         main = stream if stream is not None else torch.cuda.current_stream(self.dw.device)
+        graphs = getattr(self, "graphs", None)
         start = torch.cuda.Event()
         start.record(main)
         self.copy_stream.wait_event(start)         # copies begin after work already on main
@@ -268,9 +280,13 @@ class HostFeed:
             if i + 1 < first + count:
                 self._copy_in(i + 1)
             main.wait_event(self.ready[i % 2])
-            du, dt = self._views(i)
-            self.dw.use_bags(du, dt, self.batches[i % len(self.batches)][2])
-            self.dw.step(main)
+            if graphs is not None:
+                with torch.cuda.stream(main):
+                    graphs[(i % 2, i % len(self.batches))].replay()
+            else:
+                du, dt = self._views(i)
+                self.dw.use_bags(du, dt, self.batches[i % len(self.batches)][2])
+                self.dw.step(main)
             self.free[i % 2].record(main)
             host_scores[i % len(host_scores)].copy_(self.dw.scores, non_blocking=True)
 
