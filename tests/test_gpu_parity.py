@@ -342,7 +342,7 @@ def test_pipeline_end_to_end(name, n, rows, init):
 
 @pytest.mark.parametrize("name,n_sample", [("128d5l", 96), ("packed", 48), ("large", 64)])
 def test_full_size_sampled(name, n_sample):
-    """Full BASELINE sizes (tables, candidate counts), oracle on sampled candidates."""
+    """The full workload sizes (tables, candidate counts), oracle on sampled candidates."""
     from transformer_candidate_scoring_b200.pipeline import DeviceWorkload
     w = datagen.WORKLOADS[name]
     dw = DeviceWorkload(w)
