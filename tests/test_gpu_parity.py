@@ -148,6 +148,27 @@ def test_aggregate_variants_parity(mode, post_ln, dt, D):
     assert tr().sync_status() == 0
 
 
+def test_aggregate_variants_skip_and_report_out_of_range_keys():
+    rng = np.random.default_rng(17)
+    tables = _tables(5, 1, 1000, 64, "bf16")
+    bags = _bags(rng, 300, 10, 1000, 1, empty_frac=0.0)
+    bad = bags.keys.copy()
+    bad[[2, 50]] = [1000, -3]
+    keep = np.ones(len(bad), bool)
+    keep[[2, 50]] = False
+    cnt = np.array([keep[bags.offsets[b]:bags.offsets[b + 1]].sum() for b in range(300)])
+    off = np.zeros(301, np.int64)
+    np.cumsum(cnt, out=off[1:])
+    clean = datagen.Bags(off, bags.keys[keep], bags.weights[keep], bags.bag_table)
+    for mode in ("sum", "max"):
+        out = torch.empty(300, 64, dtype=torch.float32, device="cuda")
+        tr().aggregate(tables, dev(bags.bag_table), dev(bags.offsets), dev(bad), dev(bags.weights), out, mode=mode)
+        torch.cuda.synchronize()
+        assert tr().sync_status() == 4, mode
+        ref = _oracle_agg_mode(5, clean, 1000, 64, "bf16", mode, False)
+        np.testing.assert_allclose(out.double().cpu().numpy(), ref, rtol=1e-5, atol=1e-7)
+
+
 def test_aggregate_scale_invariance_is_bitexact():
     rng = np.random.default_rng(5)
     tables = _tables(3, 2, 3000, 128, "bf16")

@@ -86,3 +86,20 @@ def test_topk_of_pipeline_scores_full_size():
     ref = oracle.score_request(w, dw.params, dw.reqs[0], cand=np.concatenate([top, rest])).scores
     tol = 2e-2 * float(np.max(np.abs(ref)))
     assert ref[:50].min() >= ref[50:].max() - tol
+
+
+def test_topk_all_equal_scores_take_lowest_indices():
+    """Every score equal: the threshold ties straddle the k-th place, so the index-ordered
+    ranking decides (lowest indices first)."""
+    off = [0, 10000, 10003]
+    scores = np.full(off[-1], 1.5, np.float32)
+    got_i, got_v = _run(scores, off, 100)
+    assert got_i[0].tolist() == list(range(100))
+    assert got_i[1].tolist() == [0, 1, 2] + [-1] * 97
+    assert np.all(got_v[0] == 1.5)
+
+
+def test_topk_empty_requests():
+    off = [0, 0, 0]
+    got_i, got_v = _run(np.zeros(1, np.float32)[:0], off, 5)
+    assert np.all(got_i == -1) and np.all(np.isneginf(got_v))
