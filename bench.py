@@ -8,12 +8,15 @@ A step is one pass of the whole scoring path over one request of the 128D-5L wor
   -> (join) tr_score_candidates.
 Stage times come from CUDA events on the stream each stage runs on; the user side
 overlaps the target side, so the stages do not add up to the step.
-``value`` is candidates scored per second over all ranks, with inputs resident in HBM;
-``e2e`` repeats the step with the request's bags copied from pinned host memory and the
-scores copied back inside the timed region.  Requests rotate over several seeded request
-sets and the embedding tables (24.6 GB) are far larger than L2.
+``value`` is candidates scored per second over all ranks, with inputs resident in HBM, the
+steps replayed from CUDA graphs; ``e2e`` repeats the step with the request's bags copied
+from pinned host memory (overlapped with the previous batch) and the scores copied back
+inside the timed region.  Requests rotate over several seeded request sets and the
+embedding tables (24.6 GB) are far larger than L2.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py --case bulk|uncompressed [--case-n N]      side measurements (JSON line)
+  python bench.py --case score|compress|prefill|all          one stage, for a profiler
 
 Multi-GPU: one process per GPU (torchrun); every rank scores its own requests (weak
 scaling, no collective on the data path); times are the max over ranks.
