@@ -422,6 +422,132 @@ def test_host_feed_matches_device_resident_steps():
         assert torch.equal(out[i], ref[i % 3].cpu()), ("graph", i)
 
 
+def _serial_reference(w, sets):
+    """Scores of each request set through DeviceWorkload.step, one after the other."""
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload
+    dw = DeviceWorkload(w, reqs=sets[0])
+    ref = []
+    for reqs in sets:
+        dw.set_requests(reqs)
+        dw.step()
+        ref.append(dw.scores.clone())
+    torch.cuda.synchronize()
+    dw.set_requests(sets[0])
+    return dw, ref
+
+
+@pytest.mark.parametrize("n_sms", [6, 148])
+def test_overlapped_steps_match_serial_steps(n_sms):
+    """Consecutive requests overlapped over two slots (the score split at the last partial
+    wave, the next request's aggregation beside it) give each request the scores of a
+    serial step, bit for bit, eagerly and from one captured graph.  n_sms = 6 forces a
+    split at this size (16 tiles: 12 + 4); at 148 there is a single wave and no split."""
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload, Overlapped, score_split
+    w = datagen.scaled(datagen.WORKLOADS["128d5l"], n_cand_per_request=2000, rows=20000)
+    sets = [datagen.make_requests(w, seed=700 + k) for k in range(3)]
+    dw, ref = _serial_reference(w, sets)
+    dw2 = DeviceWorkload(w, reqs=sets[0], params=dw.params, tables=(dw.user_tables, dw.target_tables))
+    ov = Overlapped([dw, dw2])
+    ov.n_sms = n_sms
+    assert (score_split(dw.req_offsets, n_sms) == 1536) == (n_sms == 6)
+    n_batch = 7
+    out = [torch.zeros(dw.n_cand, dtype=torch.float32, device="cuda") for _ in range(n_batch)]
+
+    def bind(i, slot, main):
+        slot.use_bags(*_set_bags(dw, sets, i))
+
+    def scored(i, slot, back):
+        with torch.cuda.stream(back):
+            out[i].copy_(slot.scores)
+
+    ov.run(0, n_batch, bind=bind, scored=scored)
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    for i in range(n_batch):
+        assert torch.equal(out[i], ref[i % 3]), ("eager", i)
+    for o in out:
+        o.zero_()
+    g = ov.capture(0, n_batch, bind=bind, scored=scored)
+    assert ov.launches_per_step == (6 if n_sms == 6 else 5)
+    g.replay()
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    for i in range(n_batch):
+        assert torch.equal(out[i], ref[i % 3]), ("graph", i)
+
+
+_SET_BAGS = {}
+
+
+def _set_bags(dw, sets, i):
+    """Device bags of request set i % len(sets) (uploaded once per set)."""
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, pack_target_bags
+    reqs = sets[i % len(sets)]
+    key = (id(dw), i % len(sets))
+    if key not in _SET_BAGS:
+        _SET_BAGS[key] = ([DeviceBags.of(r.user, dw.device) for r in reqs],
+                          DeviceBags.of(pack_target_bags(reqs), dw.device), reqs)
+    return _SET_BAGS[key]
+
+
+def test_overlapped_packed_requests_split_inside_a_request():
+    """Packed batches of 16 requests with different L_u: the score split falls inside a
+    request (score_range gives each piece the request's cache), scores match serial steps."""
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload, Overlapped, score_split
+    w = datagen.scaled(datagen.WORKLOADS["packed"], n_cand_per_request=300, rows=20000)
+    sets = [datagen.make_requests(w, seed=800 + k) for k in range(2)]
+    dw, ref = _serial_reference(w, sets)
+    dw.set_requests(sets[0])
+    dw2 = DeviceWorkload(w, reqs=sets[1], params=dw.params, tables=(dw.user_tables, dw.target_tables))
+    ov = Overlapped([dw, dw2])
+    ov.n_sms = 10                                  # 48 tiles -> 40 + 8, cut inside request 13
+    cut = score_split(dw.req_offsets, ov.n_sms)
+    assert cut is not None and cut not in dw.req_offsets
+    out = [torch.zeros(dw.n_cand, dtype=torch.float32, device="cuda") for _ in range(5)]
+
+    def scored(i, slot, back):
+        with torch.cuda.stream(back):
+            out[i].copy_(slot.scores)
+
+    ov.run(0, 5, scored=scored)
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    for i in range(5):
+        assert torch.equal(out[i], ref[i % 2]), i
+
+
+def test_host_feed_overlapped_matches_serial_steps():
+    """Host-fed batches through the overlapped slots (bags copied during the previous batch,
+    scores copied back after the last score launch), eager and as one captured graph."""
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, HostFeed, Overlapped, pack_target_bags
+    w = datagen.scaled(datagen.WORKLOADS["128d5l"], n_cand_per_request=1000, rows=20000)
+    sets = [datagen.make_requests(w, seed=950 + k) for k in range(3)]
+    dw, ref = _serial_reference(w, sets)
+    dw2 = DeviceWorkload(w, reqs=sets[0], params=dw.params, tables=(dw.user_tables, dw.target_tables))
+    ov = Overlapped([dw, dw2])
+    ov.n_sms = 5                                   # 8 tiles -> 5 + 3
+
+    def pinned(b):
+        return DeviceBags(*(x.pin_memory() for x in (b.offsets, b.keys, b.weights, b.bag_table)))
+    batches = [([pinned(DeviceBags.of(r.user, "cpu")) for r in reqs], pinned(DeviceBags.of(pack_target_bags(reqs), "cpu")),
+                reqs) for reqs in sets]
+    feed = HostFeed(dw, batches)
+    out = [torch.empty(dw.n_cand, dtype=torch.float32).pin_memory() for _ in range(7)]
+    feed.run_overlapped(ov, 0, 7, out)
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    for i in range(7):
+        assert torch.equal(out[i], ref[i % 3].cpu()), ("eager", i)
+    for o in out:
+        o.zero_()
+    g = feed.capture_overlapped(ov, 0, 7, out)
+    g.replay()
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    for i in range(7):
+        assert torch.equal(out[i], ref[i % 3].cpu()), ("graph", i)
+
+
 def test_compress_corpus_chunked_equals_one_pass_and_oracle():
     """Near-line bulk compression in chunks (with a ragged last chunk) gives the same bits
     as one aggregate + compress pass over all items, and matches the oracle on a sample."""

@@ -1,0 +1,306 @@
+"""Host-side scheduling logic of the pipeline (no GPU): where the score call is split so
+that the next request can start beside the score kernel's last partial wave."""
+import itertools
+
+import numpy as np
+import pytest
+
+from transformer_candidate_scoring_b200.pipeline import SCORE_TILE, score_split
+
+
+def _tiles(off):
+    return [-(-(off[r + 1] - off[r]) // SCORE_TILE) for r in range(len(off) - 1)]
+
+
+def _tile_index(off, c):
+    """Number of tiles that lie wholly before packed candidate c (c on a tile boundary)."""
+    t = 0
+    for r in range(len(off) - 1):
+        if c >= off[r + 1]:
+            t += -(-(off[r + 1] - off[r]) // SCORE_TILE)
+        elif c > off[r]:
+            assert (c - off[r]) % SCORE_TILE == 0, "split not on a tile boundary of its request"
+            t += (c - off[r]) // SCORE_TILE
+    return t
+
+
+def test_single_request_of_the_128d5l_workload():
+    # 40,000 candidates = 313 tiles = 2 full waves of 148 + 17: the split is after 296 tiles
+    assert score_split([0, 40000], 148) == 296 * 128
+
+
+@pytest.mark.parametrize("off,n_sms", [([0, 148 * 128], 148), ([0, 100], 148), ([0, 147 * 128 + 5], 148),
+                                       ([0, 0], 148), ([0, 40000], 0), ([0, 300, 300, 900], 8)])
+def test_no_split_without_a_partial_wave(off, n_sms):
+    # an exact number of waves, a single wave, no candidates or no SM count: nothing to split
+    # (the last case: 3 + 0 + 5 = 8 tiles, one wave of 8)
+    assert score_split(off, n_sms) is None
+
+
+def test_split_at_a_request_boundary_and_inside_a_request():
+    off = [300 * i for i in range(17)]             # 16 requests of 3 tiles (the last one ragged)
+    assert score_split(off, 7) == 4200             # 48 = 42 + 6: after request 13
+    assert score_split(off, 10) == 3900 + 128      # 48 = 40 + 8: one tile into request 13
+
+
+def test_split_properties_over_random_batches():
+    rng = np.random.default_rng(3)
+    for _ in range(400):
+        R = int(rng.integers(1, 12))
+        sizes = rng.integers(0, 2000, size=R)
+        sizes[rng.random(R) < 0.2] = 0             # some empty requests
+        off = [0] + list(itertools.accumulate(int(x) for x in sizes))
+        n_sms = int(rng.integers(1, 40))
+        T = sum(_tiles(off))
+        cut = score_split(off, n_sms)
+        if T <= n_sms or T % n_sms == 0:
+            assert cut is None
+            continue
+        assert cut is not None and 0 < cut < off[-1]
+        a = _tile_index(off, cut)
+        assert a == T - T % n_sms                  # the full waves before the cut
+        assert a % n_sms == 0
+
+
+# ---------------------------------------------------------------- stream-order race check
+#
+# Overlapped and HostFeed.run_overlapped issue work on several CUDA streams ordered only by
+# events.  The fakes below stand in for torch's streams, events and buffers and record, for
+# every launch and copy, the stream it went to and the buffers it reads and writes.  The
+# check then requires every pair of conflicting accesses (one of them a write) to be
+# ordered on the device in the order the host issued them: by stream order, or through a
+# chain of event records and waits.
+
+class _Log:
+    def __init__(self):
+        self.ops = []                    # (stream, index on stream, reads, writes, label)
+        self.waits = []                  # (waiting stream, index on it, recording stream, count)
+
+
+class _Stream:
+    _n = 0
+
+    def __init__(self, log, *a, **k):
+        self.log, self.n_ops = log, 0
+        _Stream._n += 1
+        self.id = _Stream._n
+
+    def wait_event(self, ev):
+        if ev.at is None:                # never recorded: no dependency (as in torch)
+            return
+        self.log.waits.append((self, self.n_ops, ev.at[0], ev.at[1]))
+
+    def launch(self, reads, writes, label):
+        self.log.ops.append((self, self.n_ops, tuple(reads), tuple(writes), label))
+        self.n_ops += 1
+
+
+class _Event:
+    def __init__(self, *a, **k):
+        self.at = None
+
+    def record(self, stream):
+        self.at = (stream, stream.n_ops)   # covers the stream's first n_ops operations
+
+
+class _Cuda:
+    def __init__(self, log):
+        self.log = log
+        self.cur = [_Stream(log)]
+
+        def make_stream(*a, **k):
+            return _Stream(log)
+        make_stream.priority_range = lambda: (0, -1)
+        self.Stream = make_stream
+
+    def Event(self, *a, **k):
+        return _Event()
+
+    def current_stream(self, *a):
+        return self.cur[-1]
+
+    def stream(self, s):
+        cuda = self
+
+        class _Ctx:
+            def __enter__(self):
+                cuda.cur.append(s)
+
+            def __exit__(self, *exc):
+                cuda.cur.pop()
+        return _Ctx()
+
+    def get_device_properties(self, dev):
+        class _P:
+            multi_processor_count = 148
+        return _P()
+
+
+class _Buf:
+    def __init__(self, cuda, name, n=1):
+        self.cuda, self.name, self.n = cuda, name, n
+        self.dtype = "i64"
+
+    def numel(self):
+        return self.n
+
+    def element_size(self):
+        return 4
+
+    def __getitem__(self, sl):
+        return self
+
+    def copy_(self, src, non_blocking=False):
+        self.cuda.current_stream().launch([src.name], [self.name], f"copy {src.name} -> {self.name}")
+        return self
+
+
+class _Torch:
+    def __init__(self, log):
+        self.cuda = _Cuda(log)
+        self._k = 0
+
+    def empty(self, n, dtype=None, device=None):
+        self._k += 1
+        return _Buf(self.cuda, f"dev{self._k}", n)
+
+
+class _Slot:
+    """DeviceWorkload stand-in: each stage reads and writes the named buffers."""
+
+    def __init__(self, cuda, name, n_cand):
+        self.cuda, self.name, self.device = cuda, name, "cpu"
+        self.req_offsets = [0, n_cand]
+        self.scores = _Buf(cuda, f"{name}.scores")
+        self.ub = self.tb = None
+
+    @property
+    def n_cand(self):
+        return self.req_offsets[-1]
+
+    def use_bags(self, ub, tb, reqs):
+        self.ub, self.tb = ub, tb
+
+    def _bags(self, bags):
+        return [x.name for b in bags for x in (b.offsets, b.keys, b.weights, b.bag_table)]
+
+    def user_aggregate(self, s):
+        s.launch(self._bags(self.ub), [f"{self.name}.user_tokens"], f"{self.name} user_aggregate")
+
+    def user_prefill(self, s):
+        s.launch([f"{self.name}.user_tokens"], [f"{self.name}.kv"], f"{self.name} prefill")
+
+    def target_aggregate(self, s):
+        s.launch(self._bags([self.tb]), [f"{self.name}.X"], f"{self.name} target_aggregate")
+
+    def compress(self, s):
+        s.launch([f"{self.name}.X"], [f"{self.name}.tokens"], f"{self.name} compress")
+
+    def score(self, s):
+        s.launch([f"{self.name}.tokens", f"{self.name}.kv"], [f"{self.name}.scores"], f"{self.name} score")
+
+    def score_range(self, c0, c1, s):
+        s.launch([f"{self.name}.tokens", f"{self.name}.kv"], [f"{self.name}.scores"], f"{self.name} score[{c0}:{c1})")
+
+
+def _races(log):
+    """Pairs of conflicting accesses that the device may run out of issue order."""
+    ops = log.ops
+    node = {(o[0].id, o[1]): k for k, o in enumerate(ops)}
+    # happens-before: op k precedes every later op of its stream, and every op after a wait
+    # that covers it
+    succ = {k: set() for k in range(len(ops))}
+    by_stream = {}
+    for k, o in enumerate(ops):
+        by_stream.setdefault(o[0].id, []).append(k)
+    for ks in by_stream.values():
+        for a, b in zip(ks, ks[1:]):
+            succ[a].add(b)
+    for s, idx, rs, count in log.waits:
+        if count == 0:
+            continue
+        src = node[(rs.id, count - 1)]
+        nxt = [k for k in by_stream.get(s.id, []) if ops[k][1] >= idx]
+        if nxt:
+            succ[src].add(nxt[0])
+
+    def reach(a):
+        seen, todo = set(), [a]
+        while todo:
+            for b in succ[todo.pop()]:
+                if b not in seen:
+                    seen.add(b)
+                    todo.append(b)
+        return seen
+
+    after = [reach(k) for k in range(len(ops))]
+    bad = []
+    for a in range(len(ops)):
+        for b in range(a + 1, len(ops)):
+            ra, wa, rb, wb = set(ops[a][2]), set(ops[a][3]), set(ops[b][2]), set(ops[b][3])
+            if (wa & (rb | wb)) or (ra & wb):
+                if b not in after[a]:
+                    bad.append((ops[a][4], ops[b][4]))
+    return bad
+
+
+@pytest.fixture
+def fake_cuda(monkeypatch):
+    from transformer_candidate_scoring_b200 import pipeline
+    log = _Log()
+    fake = _Torch(log)
+    monkeypatch.setattr(pipeline, "torch", fake)
+    return pipeline, fake, log
+
+
+def test_race_check_detects_a_missing_wait(fake_cuda):
+    # the checker itself: a consumer on another stream without the wait is a race
+    pipeline, fake, log = fake_cuda
+    a, b = fake.cuda.Stream(), fake.cuda.Stream()
+    a.launch([], ["x"], "produce")
+    b.launch(["x"], [], "consume")
+    assert _races(log) == [("produce", "consume")]
+    ev = fake.cuda.Event()
+    ev.record(a)
+    b.wait_event(ev)
+    b.launch(["x"], [], "consume again")
+    assert ("produce", "consume again") not in _races(log)
+
+
+@pytest.mark.parametrize("n_cand,count", [(40000, 6), (1000, 5)])
+def test_overlapped_steps_have_no_stream_races(fake_cuda, n_cand, count):
+    pipeline, fake, log = fake_cuda
+    slots = [_Slot(fake.cuda, f"slot{k}", n_cand) for k in range(2)]
+    resident = [([], _Bags(fake.cuda, f"set{k}")) for k in range(3)]   # read-only device bags
+
+    def bind(i, dw, main):
+        dw.use_bags(*resident[i % 3], None)
+
+    def scored(i, dw, back):
+        with fake.cuda.stream(back):
+            out = _Buf(fake.cuda, f"out{i}")
+            out.copy_(dw.scores)
+
+    ov = pipeline.Overlapped(slots)
+    ov.run(0, count, fake.cuda.current_stream(), bind=bind, scored=scored)
+    assert len(log.ops) > 5 * count
+    assert _races(log) == []
+
+
+def _Bags(cuda, name):
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags
+    return DeviceBags(*(_Buf(cuda, f"{name}.{f}") for f in ("offsets", "keys", "weights", "bag_table")))
+
+
+def test_host_feed_overlapped_has_no_stream_races(fake_cuda):
+    pipeline, fake, log = fake_cuda
+    slots = [_Slot(fake.cuda, f"slot{k}", 40000) for k in range(2)]
+    batches = [([_Bags(fake.cuda, f"host{k}.user")], _Bags(fake.cuda, f"host{k}.target"), None) for k in range(3)]
+    feed = pipeline.HostFeed(slots[0], batches)
+    ov = pipeline.Overlapped(slots)
+    host_scores = [_Buf(fake.cuda, f"host_scores{k}") for k in range(2)]
+    feed.run_overlapped(ov, 0, 7, host_scores, fake.cuda.current_stream())
+    labels = [o[4] for o in log.ops]
+    assert sum(l.startswith("copy host") for l in labels) == 7 * 8      # 2 bags x 4 arrays per batch
+    assert sum("-> host_scores" in l for l in labels) == 7
+    assert _races(log) == []

@@ -142,6 +142,24 @@ class DeviceWorkload:
         api.score_candidates(self.model, self.tokens, self.req_offsets, self.kv, self.L_u, self.domain,
                              self.scores, stream=stream)
 
+    def score_range(self, c0: int, c1: int, stream=None) -> None:
+        """tr_score_candidates over the packed candidates [c0, c1) only: each request's share
+        of the range keeps its K/V cache, L_u and domain.  A candidate's score depends on
+        its own token and its request's cache alone, so scoring a batch in two ranges gives
+        the same scores as one call."""
+        off, kv, lu, dm = [0], [], [], []
+        for r in range(len(self.L_u)):
+            lo, hi = max(self.req_offsets[r], c0), min(self.req_offsets[r + 1], c1)
+            if hi <= lo:
+                continue
+            off.append(off[-1] + hi - lo)
+            kv.append(self.kv[r])
+            lu.append(self.L_u[r])
+            dm.append(self.domain[r])
+        if len(off) > 1:
+            api.score_candidates(self.model, self.tokens[c0:c1], off, kv, lu, dm, self.scores[c0:c1],
+                                 stream=stream)
+
     def select(self, k: int, stream=None):
         """Per-request top-k of the last step's scores (tr_topk): (indices within each
         request [R, k] int64, scores [R, k] fp32), padded with -1 / -inf."""
@@ -200,6 +218,122 @@ class DeviceWorkload:
         if events:
             events["score"].record(main)
         return self.scores
+
+
+SCORE_TILE = 128   # candidates per tile of the tensor-core score kernel
+
+
+def score_split(req_offsets, n_sms: int, tile: int = SCORE_TILE):
+    """The packed candidate index at which the score kernel's last, partial wave of tiles
+    begins, or None when it has none.  The kernel cuts every request into tiles of
+    ``tile`` candidates, in request order, and runs one persistent CTA per SM that takes
+    tiles b, b + n_sms, b + 2 n_sms, ...; with T tiles and T mod n_sms = t > 0 (and more
+    than one wave), the last t tiles form a wave of their own on t SMs while the other SMs
+    wait.  The split index lies on a tile boundary of its request."""
+    tiles = [-(-(req_offsets[r + 1] - req_offsets[r]) // tile) for r in range(len(req_offsets) - 1)]
+    T = sum(tiles)
+    if n_sms <= 0 or T <= n_sms or T % n_sms == 0:
+        return None
+    cut = T - T % n_sms
+    acc = 0
+    for r, t in enumerate(tiles):
+        if acc + t == cut:
+            return req_offsets[r + 1]
+        if acc + t > cut:
+            return req_offsets[r] + (cut - acc) * tile
+        acc += t
+    return None
+
+
+class Overlapped:
+    """Request batches scored back to back, consecutive batches overlapped on the device.
+
+    The step of one batch runs as in DeviceWorkload.step (user side on a high-priority
+    stream beside the target aggregation and compression), but its scoring is issued on a
+    third stream in two launches: the tiles of the score kernel's full waves, then the last
+    partial wave (score_split).  The next batch's aggregation waits only for the first of
+    the two, so it fills the SMs that the partial wave leaves idle.  Batches alternate
+    between two DeviceWorkload slots (activations, caches and scores), so no batch
+    overwrites buffers that the previous one still reads: slot i % 2 is reused by batch
+    i + 2 only after batch i + 1's full waves, which follow batch i's whole score on the
+    same stream.  Scores are identical to those of DeviceWorkload.step.
+    """
+
+    def __init__(self, slots: List[DeviceWorkload]):
+        if len(slots) != 2:
+            raise ValueError("Overlapped needs two DeviceWorkload slots")
+        self.slots = slots
+        dev = slots[0].device
+        _, hi = torch.cuda.Stream.priority_range()
+        self.user = torch.cuda.Stream(dev, priority=hi)
+        self.back = torch.cuda.Stream(dev)
+        self.n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        self.launches_per_step = None
+
+    def run(self, first: int, count: int, stream=None, bind=None, fronted=None, scored=None) -> None:
+        """Batches first .. first + count - 1 on ``stream`` (the caller's), which waits for
+        all of them at the end.  Hooks, each given (i, slot, stream):
+          bind(i, dw, main)     before batch i's first launch (point ``dw`` at its bags);
+          fronted(i, dw, main)  after its target aggregation (its bags are no longer read);
+          scored(i, dw, back)   after its last score launch (its scores are final)."""
+        main = stream if stream is not None else torch.cuda.current_stream(self.slots[0].device)
+        start = torch.cuda.Event()
+        start.record(main)
+        self.back.wait_event(start)
+        self.user.wait_event(start)
+        prev_full = None
+        last = None
+        for i in range(first, first + count):
+            dw = self.slots[i % 2]
+            if prev_full is not None:
+                main.wait_event(prev_full)
+            if bind is not None:
+                bind(i, dw, main)
+            dw.user_aggregate(main)
+            fork = torch.cuda.Event()
+            fork.record(main)
+            self.user.wait_event(fork)
+            dw.user_prefill(self.user)
+            join = torch.cuda.Event()
+            join.record(self.user)
+            dw.target_aggregate(main)
+            if fronted is not None:
+                fronted(i, dw, main)
+            dw.compress(main)
+            comp = torch.cuda.Event()
+            comp.record(main)
+            self.back.wait_event(comp)
+            self.back.wait_event(join)
+            n = dw.n_cand
+            cut = score_split(dw.req_offsets, self.n_sms)
+            full = torch.cuda.Event()
+            if cut is None:
+                dw.score(self.back)
+                full.record(self.back)
+            else:
+                dw.score_range(0, cut, self.back)
+                full.record(self.back)
+                dw.score_range(cut, n, self.back)
+            if scored is not None:
+                scored(i, dw, self.back)
+            prev_full = full
+            last = torch.cuda.Event()
+            last.record(self.back)
+        if last is not None:
+            main.wait_event(last)
+
+    def capture(self, first: int, count: int, **hooks) -> "torch.cuda.CUDAGraph":
+        """run(first, count, ...) captured into one CUDA graph (replay it to run the same
+        batches again; the overlap holds between the captured batches, not across replays).
+        Run the slots eagerly once first: the library sets up per-device state on first
+        use, which capture does not allow."""
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(self.slots[0].device)
+        l0 = api.kernel_launches()
+        with torch.cuda.graph(g, stream=cap):
+            self.run(first, count, cap, **hooks)
+        self.launches_per_step = (api.kernel_launches() - l0) / max(count, 1)
+        return g
 
 
 def _bag_tensors(b: DeviceBags):
@@ -289,6 +423,45 @@ class HostFeed:
                 self.dw.step(main)
             self.free[i % 2].record(main)
             host_scores[i % len(host_scores)].copy_(self.dw.scores, non_blocking=True)
+
+    def run_overlapped(self, ov: "Overlapped", first: int, count: int, host_scores, stream=None) -> None:
+        """run() through an Overlapped pair of slots (``ov.slots[0]`` is ``self.dw`` or one
+        like it): batch i computes in slot i % 2 from bag slot i % 2, batch i + 1's bags are
+        copied while batch i computes, a bag slot is refilled once the batch before has
+        finished its target aggregation, and each batch's scores are copied to the host on
+        the stream that scored them, right after its last score launch."""
+        main = stream if stream is not None else torch.cuda.current_stream(self.dw.device)
+        self.ready = [torch.cuda.Event() for _ in range(2)]   # fresh: no wait on an earlier run
+        self.free = [torch.cuda.Event() for _ in range(2)]
+        start = torch.cuda.Event()
+        start.record(main)
+        self.copy_stream.wait_event(start)
+        self._copy_in(first)
+        end = first + count
+
+        def bind(i, dw, m):
+            if i + 1 < end:
+                self._copy_in(i + 1)
+            m.wait_event(self.ready[i % 2])
+            du, dt = self._views(i)
+            dw.use_bags(du, dt, self.batches[i % len(self.batches)][2])
+
+        def fronted(i, dw, m):
+            self.free[i % 2].record(m)
+
+        def scored(i, dw, back):
+            with torch.cuda.stream(back):
+                host_scores[i % len(host_scores)].copy_(dw.scores, non_blocking=True)
+
+        ov.run(first, count, main, bind=bind, fronted=fronted, scored=scored)
+
+    def capture_overlapped(self, ov: "Overlapped", first: int, count: int, host_scores) -> "torch.cuda.CUDAGraph":
+        """run_overlapped(...) captured into one CUDA graph, host copies included."""
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(self.dw.device)
+        with torch.cuda.graph(g, stream=cap):
+            self.run_overlapped(ov, first, count, host_scores, cap)
+        return g
 
 
 def compress_corpus(model, target_tables, bags: DeviceBags, n_items: int, n_fields: int, out: torch.Tensor,
