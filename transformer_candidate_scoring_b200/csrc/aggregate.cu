@@ -1,14 +1,16 @@
 // Weighted-average aggregation of (key, weight) bags (TransRetrieval §3.2):
 //   out[b] = sum_i v_i h(k_i) / sum_i v_i
 //
-// HBM-bound gather.  One warp owns one bag at a time (grid-stride over bags).  A table
-// row is split into 16-byte vectors; `LPR` lanes cover one row, so a warp reads
-// 32/LPR rows per step (two 256-byte rows for D = 128 bf16).  Keys and weights of up to
-// 32 entries are fetched with one coalesced load each and broadcast by shuffle; row
-// loads of four steps are issued before any is consumed, so each lane keeps several
-// 16-byte reads in flight.  Accumulation is fp32; the division by the weight sum is a
-// correctly rounded IEEE divide, so scaling all weights of a bag by 2^k leaves the
-// result bit-identical.
+// HBM-bound gather.  A table row is split into 16-byte vectors and `LPR` lanes cover one
+// row (16 lanes for a 256-byte row, D = 128 bf16).  Two kernels share the arithmetic:
+//  - wavg_kernel, for many bags: each group of LPR lanes owns one bag at a time (a warp
+//    works on 32 / LPR bags), with several rows in flight per group;
+//  - wavg_split_kernel, for few bags (fewer than one resident round of blocks): one block
+//    per bag, its 256 / LPR lane groups share the bag's rows and their partial sums meet
+//    in shared memory, so a long bag costs one round of row loads instead of many.
+// Keys and weights are fetched LPR at a time and broadcast by shuffle.  Accumulation is
+// fp32; the division by the weight sum is a correctly rounded IEEE divide, so scaling all
+// weights of a bag by 2^k leaves the result bit-identical.
 #include <algorithm>
 
 #include "model.cuh"
@@ -71,6 +73,97 @@ __device__ __forceinline__ void store_out<__nv_bfloat16, 8>(__nv_bfloat16* dst, 
 template <>
 __device__ __forceinline__ void store_out<__nv_bfloat16, 4>(__nv_bfloat16* dst, const float* v) {
   *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]));
+}
+
+// The bag's token from its fp32 accumulation (this lane's CI x NV columns, column
+// (c * LPR + lane) * NV + i) and its weight sum: the mean divides by the weight sum (zero
+// when it is zero), the sum keeps the accumulation, the max gives zero for a bag without
+// rows; then the optional LayerNorm over the D columns that the LPR lanes of the group
+// hold.  Every lane of the warp calls it (the LayerNorm reductions are shuffles).
+template <int LPR, int CI, int NV>
+__device__ __forceinline__ void finish_bag(float (&r)[CI][NV], const float (&acc)[CI][NV], float wsum,
+                                           bool bad_table, int agg, bool is_max, bool post_ln) {
+  constexpr int D = LPR * CI * NV;
+#pragma unroll
+  for (int c = 0; c < CI; ++c)
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const float a = acc[c][i];
+      r[c][i] = bad_table                ? 0.f
+                : agg == TR_AGG_MEAN     ? (wsum != 0.f ? a / wsum : 0.f)
+                : is_max                 ? (a == -INFINITY ? 0.f : a)
+                                         : a;
+    }
+  if (post_ln) {
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < CI; ++c)
+#pragma unroll
+      for (int i = 0; i < NV; ++i) s += r[c][i];
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    const float mean = s * (1.f / D);
+    float q = 0.f;
+#pragma unroll
+    for (int c = 0; c < CI; ++c)
+#pragma unroll
+      for (int i = 0; i < NV; ++i) q = fmaf(r[c][i] - mean, r[c][i] - mean, q);
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
+    const float rstd = rsqrtf(q * (1.f / D) + kLnEps);
+#pragma unroll
+    for (int c = 0; c < CI; ++c)
+#pragma unroll
+      for (int i = 0; i < NV; ++i) r[c][i] = (r[c][i] - mean) * rstd;
+  }
+}
+
+// Up to UNROLL rows of one chunk of LPR keys into the group's accumulator: the keys and
+// weights sit one per lane of the group (k < 0 for none), rows j0 .. j0 + UNROLL - 1 of the
+// chunk are loaded before any is consumed, and `between()` runs while they are in flight.
+// cnt: the group's keys in this chunk.
+template <typename T, int LPR, int CI, int UNROLL, typename Between>
+__device__ __forceinline__ void gather_rows(float (&acc)[CI][Vec16<T>::N], const T* table, int k, float v, int cnt,
+                                            int j0, int cl, bool is_max, Between&& between) {
+  constexpr int NV = Vec16<T>::N;
+  constexpr int D = LPR * CI * NV;
+  uint4 raw[UNROLL][CI];
+  float wv[UNROLL];
+  bool lv[UNROLL];
+#pragma unroll
+  for (int u = 0; u < UNROLL; ++u) {
+    const int j = j0 + u;
+    const int kk = __shfl_sync(0xffffffffu, k, j % LPR, LPR);
+    wv[u] = __shfl_sync(0xffffffffu, v, j % LPR, LPR);
+    const bool live = j < cnt && kk >= 0;
+    lv[u] = live;
+    if (!live) wv[u] = 0.f;
+    const uint4* row = reinterpret_cast<const uint4*>(table + (int64_t)(live ? kk : 0) * D);
+#pragma unroll
+    for (int c = 0; c < CI; ++c) raw[u][c] = live ? ld_stream(row + c * LPR + cl) : make_uint4(0, 0, 0, 0);
+  }
+  between();
+  if (is_max) {
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u)
+#pragma unroll
+      for (int c = 0; c < CI; ++c) {
+        float f[NV];
+        Vec16<T>::unpack(raw[u][c], f);
+#pragma unroll
+        for (int i = 0; i < NV; ++i) acc[c][i] = lv[u] ? fmaxf(acc[c][i], f[i]) : acc[c][i];
+      }
+  } else {
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u)
+#pragma unroll
+      for (int c = 0; c < CI; ++c) {
+        float f[NV];
+        Vec16<T>::unpack(raw[u][c], f);
+#pragma unroll
+        for (int i = 0; i < NV; ++i) acc[c][i] = fmaf(wv[u], f[i], acc[c][i]);
+      }
+  }
 }
 
 // LPR lanes per row, CI 16-byte column blocks per lane (D = LPR * CI * NV).
@@ -177,89 +270,119 @@ __global__ void __launch_bounds__(256, 4) wavg_kernel(TableSet tabs, int n_table
       }
       wsum += v;
       const int cnt_max = n_max - base < LPR ? n_max - base : LPR;   // warp-uniform
-      for (int j0 = 0; j0 < cnt_max; j0 += UNROLL) {
-        uint4 raw[UNROLL][CI];
-        float wv[UNROLL];
-        bool lv[UNROLL];
-#pragma unroll
-        for (int u = 0; u < UNROLL; ++u) {
-          const int j = j0 + u;
-          const int kk = __shfl_sync(0xffffffffu, k, j % LPR, LPR);
-          wv[u] = __shfl_sync(0xffffffffu, v, j % LPR, LPR);
-          const bool live = j < cnt && kk >= 0;
-          lv[u] = live;
-          if (!live) wv[u] = 0.f;
-          const uint4* row = reinterpret_cast<const uint4*>(table + (int64_t)(live ? kk : 0) * D);
-#pragma unroll
-          for (int c = 0; c < CI; ++c)
-            raw[u][c] = live ? ld_stream(row + c * LPR + cl) : make_uint4(0, 0, 0, 0);
-        }
-        if (has_next && !next_keys) fetch_next_keys();   // overlaps these rows
-        if (is_max) {
-#pragma unroll
-          for (int u = 0; u < UNROLL; ++u)
-#pragma unroll
-            for (int c = 0; c < CI; ++c) {
-              float f[NV];
-              Vec16<T>::unpack(raw[u][c], f);
-#pragma unroll
-              for (int i = 0; i < NV; ++i) acc[c][i] = lv[u] ? fmaxf(acc[c][i], f[i]) : acc[c][i];
-            }
-        } else {
-#pragma unroll
-          for (int u = 0; u < UNROLL; ++u)
-#pragma unroll
-            for (int c = 0; c < CI; ++c) {
-              float f[NV];
-              Vec16<T>::unpack(raw[u][c], f);
-#pragma unroll
-              for (int i = 0; i < NV; ++i) acc[c][i] = fmaf(wv[u], f[i], acc[c][i]);
-            }
-        }
-      }
+      for (int j0 = 0; j0 < cnt_max; j0 += UNROLL)
+        gather_rows<T, LPR, CI, UNROLL>(acc, table, k, v, cnt, j0, cl, is_max, [&]() {
+          if (has_next && !next_keys) fetch_next_keys();   // overlaps these rows
+        });
     }
     if (has_next && !next_keys) fetch_next_keys();   // empty or rejected bag
 #pragma unroll
     for (int off = LPR / 2; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
-    // this lane's columns of the token: mean divides by the weight sum (zero when it is zero),
-    // sum keeps the accumulation, max gives zero for a bag without rows
     float r[CI][NV];
-#pragma unroll
-    for (int c = 0; c < CI; ++c)
-#pragma unroll
-      for (int i = 0; i < NV; ++i) {
-        const float a = acc[c][i];
-        r[c][i] = bad_table                ? 0.f
-                  : agg == TR_AGG_MEAN     ? (wsum != 0.f ? a / wsum : 0.f)
-                  : is_max                 ? (a == -INFINITY ? 0.f : a)
-                                           : a;
-      }
-    if (post_ln) {   // LayerNorm over the D columns, held by the LPR lanes of this group
-      float s = 0.f;
-#pragma unroll
-      for (int c = 0; c < CI; ++c)
-#pragma unroll
-        for (int i = 0; i < NV; ++i) s += r[c][i];
-#pragma unroll
-      for (int off = LPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-      const float mean = s * (1.f / D);
-      float q = 0.f;
-#pragma unroll
-      for (int c = 0; c < CI; ++c)
-#pragma unroll
-        for (int i = 0; i < NV; ++i) q = fmaf(r[c][i] - mean, r[c][i] - mean, q);
-#pragma unroll
-      for (int off = LPR / 2; off > 0; off >>= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
-      const float rstd = rsqrtf(q * (1.f / D) + kLnEps);
-#pragma unroll
-      for (int c = 0; c < CI; ++c)
-#pragma unroll
-        for (int i = 0; i < NV; ++i) r[c][i] = (r[c][i] - mean) * rstd;
-    }
+    finish_bag<LPR, CI, NV>(r, acc, wsum, bad_table, agg, is_max, post_ln);
     if (live_bag) {
 #pragma unroll
       for (int c = 0; c < CI; ++c) store_out<O, NV>(out + b * D + (c * LPR + cl) * NV, r[c]);
     }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, STATUS_KEY_RANGE);
+}
+
+// Few bags: one block (256 threads) per bag, grid-stride over bags.  The block's
+// NG = 256 / LPR lane groups share the bag: group g takes entries g, g + NG, g + 2 NG, ...
+// (each lane of a group fetches one key and weight of the group's next LPR entries, so a
+// chunk of the block reads NG * LPR = 256 consecutive entries), gathers their rows with
+// up to UNROLL in flight, and leaves its partial sum (or max) and weight sum in shared
+// memory.  Warp 0 combines the NG partials in group order and finishes the bag as
+// wavg_kernel does.  A bag of n rows takes about n / (NG * UNROLL) rounds of row loads
+// instead of n / UNROLL.
+template <typename T, typename O, int LPR, int CI, bool VAR>
+__global__ void __launch_bounds__(256, 4) wavg_split_kernel(TableSet tabs, int n_tables,
+                                                            const int32_t* __restrict__ bag_table,
+                                                            const int64_t* __restrict__ offsets,
+                                                            const int32_t* __restrict__ keys,
+                                                            const float* __restrict__ weights, int64_t n_bags,
+                                                            int mode, O* __restrict__ out, int* status) {
+  constexpr int NV = Vec16<T>::N;
+  constexpr int D = LPR * CI * NV;
+  constexpr int NG = 256 / LPR;
+  constexpr int UNROLL = LPR < 8 ? LPR : 8;
+  __shared__ float part[NG][D];               // 256 * CI * NV floats: at most 32 KB
+  __shared__ float part_w[NG];
+  const int lane = threadIdx.x & 31;
+  const int grp = threadIdx.x / LPR;
+  const int cl = threadIdx.x % LPR;
+  const int agg = VAR ? mode & 0xFF : TR_AGG_MEAN;
+  const bool is_max = VAR && agg == TR_AGG_MAX, post_ln = VAR && (mode & TR_AGG_POST_LN) != 0;
+  bool bad = false;
+  for (int64_t b = blockIdx.x; b < n_bags; b += gridDim.x) {   // block-uniform
+    const int tbl = __ldg(bag_table + b);
+    const int64_t s0 = __ldg(offsets + b), s1 = __ldg(offsets + b + 1);
+    const bool bad_table = tbl < 0 || tbl >= n_tables;
+    bad |= bad_table;
+    const int n = bad_table ? 0 : (int)(s1 - s0);
+    const int mine = n > grp ? (n - grp + NG - 1) / NG : 0;          // this group's entries
+    const int mine_max = __reduce_max_sync(0xffffffffu, mine);
+    const T* table = static_cast<const T*>(tabs.ptr[n > 0 ? tbl : 0]);
+    const int64_t nrows = n > 0 ? tabs.rows[tbl] : 0;
+    float acc[CI][NV];
+#pragma unroll
+    for (int c = 0; c < CI; ++c)
+#pragma unroll
+      for (int i = 0; i < NV; ++i) acc[c][i] = is_max ? -INFINITY : 0.f;
+    float wsum = 0.f;
+    for (int base = 0; base < mine_max; base += LPR) {
+      const int cnt = mine - base;
+      int k = -1;
+      float v = 0.f;
+      if (cl < cnt) {
+        const int64_t e = s0 + grp + (int64_t)NG * (base + cl);
+        k = __ldg(keys + e);
+        v = __ldg(weights + e);
+        if (k < 0 || (int64_t)k >= nrows) {
+          bad = true;
+          k = -1;
+          v = 0.f;
+        }
+      }
+      wsum += v;
+      const int cnt_max = mine_max - base < LPR ? mine_max - base : LPR;   // warp-uniform
+      for (int j0 = 0; j0 < cnt_max; j0 += UNROLL)
+        gather_rows<T, LPR, CI, UNROLL>(acc, table, k, v, cnt, j0, cl, is_max, []() {});
+    }
+#pragma unroll
+    for (int off = LPR / 2; off > 0; off >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+#pragma unroll
+    for (int c = 0; c < CI; ++c)
+#pragma unroll
+      for (int i = 0; i < NV; ++i) part[grp][(c * LPR + cl) * NV + i] = acc[c][i];
+    if (cl == 0) part_w[grp] = wsum;
+    __syncthreads();
+    if (threadIdx.x < 32) {   // warp 0: every group in it combines the same columns; group 0 stores
+      float tot[CI][NV];
+#pragma unroll
+      for (int c = 0; c < CI; ++c)
+#pragma unroll
+        for (int i = 0; i < NV; ++i) tot[c][i] = is_max ? -INFINITY : 0.f;
+      float ws = 0.f;
+      for (int g = 0; g < NG; ++g) {
+#pragma unroll
+        for (int c = 0; c < CI; ++c)
+#pragma unroll
+          for (int i = 0; i < NV; ++i) {
+            const float x = part[g][(c * LPR + cl) * NV + i];
+            tot[c][i] = is_max ? fmaxf(tot[c][i], x) : tot[c][i] + x;
+          }
+        ws += part_w[g];
+      }
+      float r[CI][NV];
+      finish_bag<LPR, CI, NV>(r, tot, ws, bad_table, agg, is_max, post_ln);
+      if (grp == 0) {
+#pragma unroll
+        for (int c = 0; c < CI; ++c) store_out<O, NV>(out + b * D + (c * LPR + cl) * NV, r[c]);
+      }
+    }
+    __syncthreads();          // the partials are rewritten by the next bag
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(status, STATUS_KEY_RANGE);
 }
@@ -279,13 +402,16 @@ tr_status dispatch(const TableSet& ts, int n_tables, const int32_t* bag_table, c
   const int64_t bags_per_block = 8 * (32 / (vecs < 32 ? vecs : 32));
   const int64_t blocks_needed = (n_bags + bags_per_block - 1) / bags_per_block;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, (int64_t)sms * 32));
-#define TR_WAVG(LPR, CI)                                                                                     \
-  if (mode == TR_AGG_MEAN)                                                                                 \
-    wavg_kernel<T, O, LPR, CI, false><<<grid, 256, 0, st>>>(ts, n_tables, bag_table, offsets, keys, weights, \
-                                                            n_bags, mode, out, status);                      \
-  else                                                                                                     \
-    wavg_kernel<T, O, LPR, CI, true><<<grid, 256, 0, st>>>(ts, n_tables, bag_table, offsets, keys, weights,  \
-                                                           n_bags, mode, out, status)
+  // few bags (one resident round of one-bag blocks, 4 per SM): a block per bag
+  const bool split = n_bags <= (int64_t)sms * 4;
+  const int grid_split = (int)std::max<int64_t>(1, n_bags);
+#define TR_WAVG_K(K, G, LPR, CI, VAR) \
+  K<T, O, LPR, CI, VAR><<<G, 256, 0, st>>>(ts, n_tables, bag_table, offsets, keys, weights, n_bags, mode, out, status)
+#define TR_WAVG(LPR, CI)                                                                \
+  if (split && mode == TR_AGG_MEAN) TR_WAVG_K(wavg_split_kernel, grid_split, LPR, CI, false); \
+  else if (split) TR_WAVG_K(wavg_split_kernel, grid_split, LPR, CI, true);                    \
+  else if (mode == TR_AGG_MEAN) TR_WAVG_K(wavg_kernel, grid, LPR, CI, false);                 \
+  else TR_WAVG_K(wavg_kernel, grid, LPR, CI, true)
   switch (vecs) {
     case 1: TR_WAVG(1, 1); break;
     case 2: TR_WAVG(2, 1); break;
@@ -298,7 +424,8 @@ tr_status dispatch(const TableSet& ts, int n_tables, const int32_t* bag_table, c
     default: return fail(TR_ERR_UNSUPPORTED, "tr_aggregate: D=%d gives %d vectors per row (need 1..32 as a power of two, 64 or 128)", D, vecs);
   }
 #undef TR_WAVG
-  TR_LAUNCH_CHECK("wavg_kernel");
+#undef TR_WAVG_K
+  TR_LAUNCH_CHECK(split ? "wavg_split_kernel" : "wavg_kernel");
   return TR_OK;
 }
 
