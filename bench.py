@@ -379,13 +379,20 @@ def run_ours(args, rank, world, local_rank):
 
     feed.run_overlapped(ov, 0, args.warmup, host_scores, stream)
     torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    feed.run_overlapped(ov, args.warmup, args.steps, host_scores, stream)   # eager launches
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_eager_ms = max_over_ranks(e0.elapsed_time(e1) / 1e3) / args.steps * 1e3
     # the same launch mode as the timed value: one graph of the K steps, host copies inside
     g_e2e = feed.capture_overlapped(ov, args.warmup, args.steps, host_scores)
     g_e2e.replay()
     torch.cuda.synchronize()
     barrier()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     g_e2e.replay()
     e1.record(stream)
@@ -394,6 +401,14 @@ def run_ours(args, rank, world, local_rank):
     e2e_elapsed = e0.elapsed_time(e1) / 1e3
     e2e_elapsed = max_over_ranks(e2e_elapsed)
     e2e_value = n_cand * args.steps * world / e2e_elapsed
+    # the same host traffic with no compute: the copy-bound floor of the e2e step
+    feed.copies_only(0, args.warmup, host_scores, dw.scores, stream)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    feed.copies_only(args.warmup, args.steps, host_scores, dw.scores, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    copy_ms = max_over_ranks(e0.elapsed_time(e1) / 1e3) / args.steps * 1e3
 
     # ---- rooflines of the stages
     peaks, peak_kind = load_peaks()
@@ -435,7 +450,10 @@ def run_ours(args, rank, world, local_rank):
         "pct_bf16_peak_score_kernel": stage_roof["score"]["frac"] * 100,
         "topk": {"k": TOPK, "ms": topk_ms, "note": "tr_topk over the step's scores, timed separately"},
         "e2e": {"value": e2e_value, "unit": "candidates/s", "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h)},
+                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_elapsed / args.steps * 1e3,
+                "eager_ms_per_step": e2e_eager_ms,
+                "copies_only_ms_per_step": copy_ms,
+                "h2d_gbs_copies_only": h2d / (copy_ms / 1e3) / 1e9},
         "gpu_launches": int(launches),
         "launch": {"graphs": bool(use_graphs), "e2e_graphs": bool(use_graphs),
                    "overlap": "request i+1's aggregation runs beside request i's last partial wave of score tiles",

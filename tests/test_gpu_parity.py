@@ -86,11 +86,13 @@ def _run_agg(tables, bags, D, out_dtype):
 
 @pytest.mark.parametrize("dt,D", [("f32", 32), ("bf16", 64), ("bf16", 128), ("f32", 128), ("bf16", 32)])
 @pytest.mark.parametrize("out_dt", ["f32", "bf16"])
-@pytest.mark.parametrize("n_bags,max_nf", [(1237, 100), (9001, 8), (6007, 70)])
+@pytest.mark.parametrize("n_bags,max_nf", [(1237, 100), (9001, 8), (6007, 70), (300, 400), (37, 3000), (500, 8)])
 def test_aggregate_parity(dt, D, out_dt, n_bags, max_nf):
     """Few long bags and many short ones: bags longer than the rows a lane group keeps in
     flight and than one key chunk, empty bags, and 1 to 8 bags per warp (D and dtype set
-    the lanes per row)."""
+    the lanes per row).  Calls of at most 4 bags per SM take the block-per-bag kernel
+    (300, 37 and 500 bags here), bags of up to 3000 rows spanning several key chunks of
+    every lane group."""
     rng = np.random.default_rng(D + n_bags)
     rows = 5000
     tables = _tables(11, 3, rows, D, dt)
@@ -122,13 +124,15 @@ def _oracle_agg_mode(seed, bags, rows, D, dt, mode, post_ln):
 @pytest.mark.parametrize("mode", ["mean", "sum", "max"])
 @pytest.mark.parametrize("post_ln", [False, True])
 @pytest.mark.parametrize("dt,D", [("bf16", 128), ("f32", 64), ("bf16", 32)])
-def test_aggregate_variants_parity(mode, post_ln, dt, D):
+@pytest.mark.parametrize("n_bags,max_nf", [(2500, 40), (200, 600)])
+def test_aggregate_variants_parity(mode, post_ln, dt, D, n_bags, max_nf):
     """The §3.2 alternatives (weighted sum, max pooling, post-aggregation LayerNorm) against
-    the oracle; max pooling without LayerNorm is exact."""
-    rng = np.random.default_rng(D + len(mode) + post_ln)
+    the oracle, through both kernels (200 bags: block per bag); max pooling without
+    LayerNorm is exact."""
+    rng = np.random.default_rng(D + len(mode) + post_ln + n_bags)
     rows = 3000
     tables = _tables(12, 2, rows, D, dt)
-    bags = _bags(rng, 2500, 40, rows, 2)
+    bags = _bags(rng, n_bags, max_nf, rows, 2)
     out = torch.empty(bags.n_bags, D, dtype=torch.float32, device="cuda")
     tr().aggregate(tables, dev(bags.bag_table), dev(bags.offsets), dev(bags.keys), dev(bags.weights), out,
                    mode=mode, post_ln=post_ln)
@@ -438,10 +442,11 @@ def _serial_reference(w, sets):
 
 @pytest.mark.parametrize("n_sms", [6, 148])
 def test_overlapped_steps_match_serial_steps(n_sms):
-    """Consecutive requests overlapped over two slots (the score split at the last partial
-    wave, the next request's aggregation beside it) give each request the scores of a
-    serial step, bit for bit, eagerly and from one captured graph.  n_sms = 6 forces a
-    split at this size (16 tiles: 12 + 4); at 148 there is a single wave and no split."""
+    """Consecutive requests overlapped over two slots (compression and scoring split at
+    their last partial wave, whose tail runs beside the next request's aggregation) give
+    each request the scores of a serial step, bit for bit, eagerly and from one captured
+    graph.  n_sms = 6 forces a split at this size (16 tiles: 12 + 4); at 148 there is a
+    single wave and no split."""
     from transformer_candidate_scoring_b200.pipeline import DeviceWorkload, Overlapped, score_split
     w = datagen.scaled(datagen.WORKLOADS["128d5l"], n_cand_per_request=2000, rows=20000)
     sets = [datagen.make_requests(w, seed=700 + k) for k in range(3)]
@@ -468,7 +473,7 @@ def test_overlapped_steps_match_serial_steps(n_sms):
     for o in out:
         o.zero_()
     g = ov.capture(0, n_batch, bind=bind, scored=scored)
-    assert ov.launches_per_step == (6 if n_sms == 6 else 5)
+    assert ov.launches_per_step == (7 if n_sms == 6 else 5)   # compress and score each in two parts
     g.replay()
     torch.cuda.synchronize()
     assert tr().sync_status() == 0

@@ -196,6 +196,9 @@ class _Slot:
     def compress(self, s):
         s.launch([f"{self.name}.X"], [f"{self.name}.tokens"], f"{self.name} compress")
 
+    def compress_range(self, c0, c1, s):
+        s.launch([f"{self.name}.X"], [f"{self.name}.tokens"], f"{self.name} compress[{c0}:{c1})")
+
     def score(self, s):
         s.launch([f"{self.name}.tokens", f"{self.name}.kv"], [f"{self.name}.scores"], f"{self.name} score")
 

@@ -138,6 +138,11 @@ class DeviceWorkload:
     def compress(self, stream=None) -> None:
         api.compress_targets(self.model, self.X, self.tokens, stream=stream)
 
+    def compress_range(self, c0: int, c1: int, stream=None) -> None:
+        """tr_compress_targets over the packed candidates [c0, c1) only (rows are independent)."""
+        if c1 > c0:
+            api.compress_targets(self.model, self.X[c0:c1], self.tokens[c0:c1], stream=stream)
+
     def score(self, stream=None) -> None:
         api.score_candidates(self.model, self.tokens, self.req_offsets, self.kv, self.L_u, self.domain,
                              self.scores, stream=stream)
@@ -248,15 +253,22 @@ def score_split(req_offsets, n_sms: int, tile: int = SCORE_TILE):
 class Overlapped:
     """Request batches scored back to back, consecutive batches overlapped on the device.
 
-    The step of one batch runs as in DeviceWorkload.step (user side on a high-priority
-    stream beside the target aggregation and compression), but its scoring is issued on a
-    third stream in two launches: the tiles of the score kernel's full waves, then the last
-    partial wave (score_split).  The next batch's aggregation waits only for the first of
-    the two, so it fills the SMs that the partial wave leaves idle.  Batches alternate
-    between two DeviceWorkload slots (activations, caches and scores), so no batch
-    overwrites buffers that the previous one still reads: slot i % 2 is reused by batch
-    i + 2 only after batch i + 1's full waves, which follow batch i's whole score on the
-    same stream.  Scores are identical to those of DeviceWorkload.step.
+    The compressor and the score kernel both cut the batch into 128-candidate tiles and
+    run one persistent CTA per SM, so a batch whose tile count is not a multiple of the SM
+    count ends each of them with a partial wave that leaves most SMs idle.  Here a batch
+    is cut at score_split into a head (the full waves) and a tail:
+      main stream  user aggregation -> target aggregation -> compress(head)
+      user stream  (high priority) user prefill
+      back stream  (high priority) score(head) | compress(tail) -> score(tail)
+    The next batch's user and target aggregation wait only for score(head), so the tail's
+    compression and scoring (one partial wave of each, on a few SMs) run beside the next
+    batch's gather.  The back stream's priority places the tail's CTAs, which need whole
+    SMs, before the gather's many small blocks fill them.
+
+    Batches alternate between two DeviceWorkload slots (activations, caches and scores),
+    so no batch overwrites buffers that the previous one still reads: slot i % 2 is reused
+    by batch i + 2 only after batch i + 1's score(head), which follows batch i's tail on
+    the back stream.  Scores are identical to those of DeviceWorkload.step.
     """
 
     def __init__(self, slots: List[DeviceWorkload]):
@@ -266,7 +278,7 @@ class Overlapped:
         dev = slots[0].device
         _, hi = torch.cuda.Stream.priority_range()
         self.user = torch.cuda.Stream(dev, priority=hi)
-        self.back = torch.cuda.Stream(dev)
+        self.back = torch.cuda.Stream(dev, priority=hi)
         self.n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
         self.launches_per_step = None
 
@@ -275,7 +287,8 @@ class Overlapped:
         all of them at the end.  Hooks, each given (i, slot, stream):
           bind(i, dw, main)     before batch i's first launch (point ``dw`` at its bags);
           fronted(i, dw, main)  after its target aggregation (its bags are no longer read);
-          scored(i, dw, back)   after its last score launch (its scores are final)."""
+          scored(i, dw, back)   after its last score launch (its scores are final).
+        ``first``/``count`` only name the batches for the hooks and pick slot i % 2."""
         main = stream if stream is not None else torch.cuda.current_stream(self.slots[0].device)
         start = torch.cuda.Event()
         start.record(main)
@@ -299,13 +312,14 @@ class Overlapped:
             dw.target_aggregate(main)
             if fronted is not None:
                 fronted(i, dw, main)
-            dw.compress(main)
+            n = dw.n_cand
+            cut = score_split(dw.req_offsets, self.n_sms)
+            head = n if cut is None else cut
+            dw.compress_range(0, head, main)
             comp = torch.cuda.Event()
             comp.record(main)
             self.back.wait_event(comp)
             self.back.wait_event(join)
-            n = dw.n_cand
-            cut = score_split(dw.req_offsets, self.n_sms)
             full = torch.cuda.Event()
             if cut is None:
                 dw.score(self.back)
@@ -313,6 +327,7 @@ class Overlapped:
             else:
                 dw.score_range(0, cut, self.back)
                 full.record(self.back)
+                dw.compress_range(cut, n, self.back)
                 dw.score_range(cut, n, self.back)
             if scored is not None:
                 scored(i, dw, self.back)
@@ -454,6 +469,20 @@ class HostFeed:
                 host_scores[i % len(host_scores)].copy_(dw.scores, non_blocking=True)
 
         ov.run(first, count, main, bind=bind, fronted=fronted, scored=scored)
+
+    def copies_only(self, first: int, count: int, host_scores, scores, stream=None) -> None:
+        """The host traffic of run() alone, on ``stream``: each batch's bags in (the same
+        copies into the same slots) and ``scores`` [n] back out, with no compute.  Timing it
+        gives the copy-bound floor of the host-fed step."""
+        main = stream if stream is not None else torch.cuda.current_stream(self.dw.device)
+        with torch.cuda.stream(main):
+            for i in range(first, first + count):
+                hu, ht, _ = self.batches[i % len(self.batches)]
+                du, dt = self._views(i)
+                for d, h in zip(du + [dt], hu + [ht]):
+                    for dx, hx in zip(_bag_tensors(d), _bag_tensors(h)):
+                        dx.copy_(hx, non_blocking=True)
+                host_scores[i % len(host_scores)].copy_(scores, non_blocking=True)
 
     def capture_overlapped(self, ov: "Overlapped", first: int, count: int, host_scores) -> "torch.cuda.CUDAGraph":
         """run_overlapped(...) captured into one CUDA graph, host copies included."""
