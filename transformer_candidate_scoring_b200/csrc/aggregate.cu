@@ -9,8 +9,8 @@
 //    per bag, its 256 / LPR lane groups share the bag's rows and their partial sums meet
 //    in shared memory, so a long bag costs one round of row loads instead of many.
 // Keys and weights are fetched LPR at a time and broadcast by shuffle.  Accumulation is
-// fp32; the division by the weight sum is a correctly rounded IEEE divide, so scaling all
-// weights of a bag by 2^k leaves the result bit-identical.
+// fp32 (packed fp32x2 FMAs); the mean multiplies by a correctly rounded reciprocal of the
+// weight sum, so scaling all weights of a bag by 2^k leaves the result bit-identical.
 #include <algorithm>
 
 #include "model.cuh"
@@ -42,6 +42,15 @@ template <> struct Vec16<__nv_bfloat16> {
     }
   }
 };
+
+// a0 += w * x0, a1 += w * x1 as one packed fp32x2 FMA (each lane rounded as fmaf)
+__device__ __forceinline__ void fma2(float& a0, float& a1, float w, float x0, float x1) {
+  asm("{\n\t.reg .b64 a, x, w;\n\t"
+      "mov.b64 a, {%0, %1};\n\tmov.b64 x, {%3, %4};\n\tmov.b64 w, {%2, %2};\n\t"
+      "fma.rn.f32x2 a, w, x, a;\n\tmov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(w), "f"(x0), "f"(x1));
+}
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 r;
@@ -84,13 +93,17 @@ template <int LPR, int CI, int NV>
 __device__ __forceinline__ void finish_bag(float (&r)[CI][NV], const float (&acc)[CI][NV], float wsum,
                                            bool bad_table, int agg, bool is_max, bool post_ln) {
   constexpr int D = LPR * CI * NV;
+  // the mean multiplies by one correctly rounded reciprocal of the weight sum (one IEEE
+  // divide per bag, not per column); scaling every weight by 2^k scales the sum and the
+  // reciprocal exactly, so the token stays bit-identical
+  const float inv = wsum != 0.f ? 1.f / wsum : 0.f;
 #pragma unroll
   for (int c = 0; c < CI; ++c)
 #pragma unroll
     for (int i = 0; i < NV; ++i) {
       const float a = acc[c][i];
       r[c][i] = bad_table                ? 0.f
-                : agg == TR_AGG_MEAN     ? (wsum != 0.f ? a / wsum : 0.f)
+                : agg == TR_AGG_MEAN     ? a * inv
                 : is_max                 ? (a == -INFINITY ? 0.f : a)
                                          : a;
     }
@@ -161,7 +174,7 @@ __device__ __forceinline__ void gather_rows(float (&acc)[CI][Vec16<T>::N], const
         float f[NV];
         Vec16<T>::unpack(raw[u][c], f);
 #pragma unroll
-        for (int i = 0; i < NV; ++i) acc[c][i] = fmaf(wv[u], f[i], acc[c][i]);
+        for (int i = 0; i < NV; i += 2) fma2(acc[c][i], acc[c][i + 1], wv[u], f[i], f[i + 1]);
       }
   }
 }
