@@ -187,13 +187,13 @@ def test_aggregate_single_key_returns_row_exactly():
     rng = np.random.default_rng(6)
     tables = _tables(4, 1, 2000, 128, "bf16")
     keys = rng.integers(0, 2000, size=300).astype(np.int32)
-    # v * h / v is exact in binary floating point when v is a power of two
+    # (v * h) * (1 / v) is exact in binary floating point when v is a power of two
     w = (2.0 ** rng.integers(-6, 6, size=300)).astype(np.float32)
     bags = datagen.Bags(np.arange(301, dtype=np.int64), keys, w, np.zeros(300, np.int32))
     got = _run_agg(tables, bags, 128, torch.float32)
     want = tables[0][torch.from_numpy(keys).long().cuda()].float()
     assert torch.equal(got, want)
-    # any other weight: within one rounding of the product and one of the quotient
+    # any other weight: within the roundings of v * h, of 1 / v and of their product (3 half-ulps)
     bags = datagen.Bags(bags.offsets, keys, rng.uniform(0.1, 1, 300).astype(np.float32), bags.bag_table)
     got = _run_agg(tables, bags, 128, torch.float32)
     assert torch.all(torch.abs(got - want) <= 2.0 ** -22 * torch.abs(want))
