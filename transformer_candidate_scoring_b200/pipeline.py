@@ -234,7 +234,11 @@ def score_split(req_offsets, n_sms: int, tile: int = SCORE_TILE):
     ``tile`` candidates, in request order, and runs one persistent CTA per SM that takes
     tiles b, b + n_sms, b + 2 n_sms, ...; with T tiles and T mod n_sms = t > 0 (and more
     than one wave), the last t tiles form a wave of their own on t SMs while the other SMs
-    wait.  The split index lies on a tile boundary of its request."""
+    wait.  The split index lies on a tile boundary of its request.  The score kernel runs
+    one launch per class of requests with the same heads per score group (L_u up to 16,
+    32, 64, 128), so for a batch that mixes classes the cut is a good guess rather than
+    the exact wave boundary; either way both parts are valid batches and the scores do not
+    change."""
     tiles = [-(-(req_offsets[r + 1] - req_offsets[r]) // tile) for r in range(len(req_offsets) - 1)]
     T = sum(tiles)
     if n_sms <= 0 or T <= n_sms or T % n_sms == 0:
