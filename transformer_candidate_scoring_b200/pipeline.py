@@ -261,18 +261,18 @@ class Overlapped:
     run one persistent CTA per SM, so a batch whose tile count is not a multiple of the SM
     count ends each of them with a partial wave that leaves most SMs idle.  Here a batch
     is cut at score_split into a head (the full waves) and a tail:
-      main stream  user aggregation -> target aggregation -> compress(head)
-      user stream  (high priority) user prefill
-      back stream  (high priority) score(head) | compress(tail) -> score(tail)
-    The next batch's user and target aggregation wait only for score(head), so the tail's
-    compression and scoring (one partial wave of each, on a few SMs) run beside the next
-    batch's gather.  The back stream's priority places the tail's CTAs, which need whole
-    SMs, before the gather's many small blocks fill them.
+      main stream  user aggregation -> target aggregation -> compress(head) -> score(head)
+      user stream  (high priority) user prefill, joined before score(head)
+      back stream  (high priority) compress(tail) -> score(tail), after score(head)
+    The next batch follows score(head) on the main stream, so the tail's compression and
+    scoring (one partial wave of each, on a few SMs) run beside the next batch's gather.
+    The back stream's priority places the tail's CTAs, which need whole SMs, before the
+    gather's many small blocks fill them.
 
-    Batches alternate between two DeviceWorkload slots (activations, caches and scores),
-    so no batch overwrites buffers that the previous one still reads: slot i % 2 is reused
-    by batch i + 2 only after batch i + 1's score(head), which follows batch i's tail on
-    the back stream.  Scores are identical to those of DeviceWorkload.step.
+    Batches alternate between two DeviceWorkload slots (activations, caches and scores);
+    batch i + 2 reuses slot i % 2 only after batch i's tail has finished (an event the main
+    stream waits for, long satisfied by then).  Scores are identical to those of
+    DeviceWorkload.step.
     """
 
     def __init__(self, slots: List[DeviceWorkload]):
@@ -291,19 +291,18 @@ class Overlapped:
         all of them at the end.  Hooks, each given (i, slot, stream):
           bind(i, dw, main)     before batch i's first launch (point ``dw`` at its bags);
           fronted(i, dw, main)  after its target aggregation (its bags are no longer read);
-          scored(i, dw, back)   after its last score launch (its scores are final).
+          scored(i, dw, s)      after its last score launch, on that launch's stream.
         ``first``/``count`` only name the batches for the hooks and pick slot i % 2."""
         main = stream if stream is not None else torch.cuda.current_stream(self.slots[0].device)
         start = torch.cuda.Event()
         start.record(main)
         self.back.wait_event(start)
         self.user.wait_event(start)
-        prev_full = None
-        last = None
+        tails = {}                                  # batch -> event: its tail launches are done
         for i in range(first, first + count):
             dw = self.slots[i % 2]
-            if prev_full is not None:
-                main.wait_event(prev_full)
+            if i - 2 in tails:                      # the slot's previous batch has finished
+                main.wait_event(tails.pop(i - 2))
             if bind is not None:
                 bind(i, dw, main)
             dw.user_aggregate(main)
@@ -320,26 +319,24 @@ class Overlapped:
             cut = score_split(dw.req_offsets, self.n_sms)
             head = n if cut is None else cut
             dw.compress_range(0, head, main)
-            comp = torch.cuda.Event()
-            comp.record(main)
-            self.back.wait_event(comp)
-            self.back.wait_event(join)
-            full = torch.cuda.Event()
+            main.wait_event(join)
             if cut is None:
-                dw.score(self.back)
-                full.record(self.back)
-            else:
-                dw.score_range(0, cut, self.back)
-                full.record(self.back)
-                dw.compress_range(cut, n, self.back)
-                dw.score_range(cut, n, self.back)
+                dw.score(main)
+                if scored is not None:
+                    scored(i, dw, main)
+                continue
+            dw.score_range(0, cut, main)
+            full = torch.cuda.Event()
+            full.record(main)
+            self.back.wait_event(full)
+            dw.compress_range(cut, n, self.back)
+            dw.score_range(cut, n, self.back)
             if scored is not None:
                 scored(i, dw, self.back)
-            prev_full = full
-            last = torch.cuda.Event()
-            last.record(self.back)
-        if last is not None:
-            main.wait_event(last)
+            tails[i] = torch.cuda.Event()
+            tails[i].record(self.back)
+        for ev in tails.values():
+            main.wait_event(ev)
 
     def capture(self, first: int, count: int, **hooks) -> "torch.cuda.CUDAGraph":
         """run(first, count, ...) captured into one CUDA graph (replay it to run the same
