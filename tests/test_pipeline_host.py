@@ -307,3 +307,63 @@ def test_host_feed_overlapped_has_no_stream_races(fake_cuda):
     assert sum(l.startswith("copy host") for l in labels) == 7 * 8      # 2 bags x 4 arrays per batch
     assert sum("-> host_scores" in l for l in labels) == 7
     assert _races(log) == []
+
+
+# ---------------------------------------------------------------- range calls (host marshalling)
+
+def _range_workload(sizes, L_u, D=4):
+    """A DeviceWorkload's request bookkeeping on CPU tensors (no model, no GPU)."""
+    import torch
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload
+    dw = object.__new__(DeviceWorkload)
+    off = [0]
+    for n in sizes:
+        off.append(off[-1] + n)
+    dw.req_offsets = off
+    dw.L_u = list(L_u)
+    dw.domain = [r % 3 for r in range(len(sizes))]
+    dw.kv = [torch.full((16,), r, dtype=torch.uint8) for r in range(len(sizes))]
+    dw.model = "model"
+    n = off[-1]
+    dw.tokens = torch.arange(n * D, dtype=torch.float32).view(n, D)
+    dw.X = torch.arange(n * 2 * D, dtype=torch.float32).view(n, 2 * D)
+    dw.scores = torch.zeros(n)
+    return dw
+
+
+def test_score_range_slices_requests_and_keeps_their_caches(monkeypatch):
+    from transformer_candidate_scoring_b200 import pipeline
+    calls = []
+    monkeypatch.setattr(pipeline.api, "score_candidates",
+                        lambda model, tokens, off, kv, lu, dm, scores, stream=None:
+                        calls.append((tokens, list(off), [int(k[0]) for k in kv], list(lu), list(dm), scores)))
+    dw = _range_workload([300, 0, 500, 200], [64, 10, 128, 32])
+    cut = 300 + 128                               # one tile into request 2
+    dw.score_range(0, cut, "s")
+    dw.score_range(cut, dw.n_cand, "s")
+    (t0, off0, kv0, lu0, dm0, s0), (t1, off1, kv1, lu1, dm1, s1) = calls
+    # head: request 0 whole, the empty request 1 dropped, the first 128 of request 2
+    assert off0 == [0, 300, 428] and kv0 == [0, 2] and lu0 == [64, 128] and dm0 == [0, 2]
+    # tail: the rest of request 2 and request 3, offsets rebased to the range
+    assert off1 == [0, 372, 572] and kv1 == [2, 3] and lu1 == [128, 32] and dm1 == [2, 0]
+    # the token and score views start at the cut and cover the range
+    assert t0.shape[0] == cut and t1.shape[0] == dw.n_cand - cut
+    assert t1.data_ptr() == dw.tokens[cut:].data_ptr() and s1.data_ptr() == dw.scores[cut:].data_ptr()
+    # a range with no candidates makes no call
+    dw.score_range(300, 300, "s")
+    assert len(calls) == 2
+
+
+def test_compress_range_passes_row_views(monkeypatch):
+    from transformer_candidate_scoring_b200 import pipeline
+    calls = []
+    monkeypatch.setattr(pipeline.api, "compress_targets",
+                        lambda model, x, tokens, stream=None: calls.append((x, tokens)))
+    dw = _range_workload([300, 500], [64, 64])
+    dw.compress_range(0, 512, None)
+    dw.compress_range(512, 800, None)
+    dw.compress_range(800, 800, None)           # empty: no call
+    assert len(calls) == 2
+    (x0, t0), (x1, t1) = calls
+    assert x0.shape[0] == 512 and x1.shape[0] == 288
+    assert x1.data_ptr() == dw.X[512:].data_ptr() and t1.data_ptr() == dw.tokens[512:].data_ptr()
