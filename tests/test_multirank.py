@@ -11,7 +11,8 @@ import pytest
 import torch.multiprocessing as mp
 
 import datagen
-from transformer_candidate_scoring_b200.shard import local_requests, max_over_ranks, rank_seed, shard_bounds
+from transformer_candidate_scoring_b200.shard import (local_requests, max_over_ranks, merge_topk, rank_seed,
+                                                      shard_bounds, split_request)
 
 
 class _R:
@@ -125,3 +126,79 @@ def test_gloo_two_ranks_shard_equals_single_process():
     assert main[0], "sharded oracle scores differ from the single-process scores"
     assert main[1], "ranks drew identical requests"
     assert main[2] == 2.5 and other[2] == 2.5
+
+
+@pytest.mark.parametrize("n,world,tile", [(40000, 8, 128), (40000, 1, 128), (100, 4, 128), (0, 2, 128),
+                                          (1000, 3, 7), (129, 2, 128)])
+def test_split_request_partition(n, world, tile):
+    c = split_request(n, world, tile)
+    assert len(c) == world + 1 and c[0] == 0 and c[-1] == n
+    assert all(c[i] <= c[i + 1] for i in range(world))
+    assert all(x % tile == 0 for x in c[:-1])
+    tiles = [-(-(c[i + 1] - c[i]) // tile) for i in range(world)]
+    assert max(tiles) - min(tiles) <= 1
+
+
+def _local_topk(scores, lo, hi, k):
+    """This rank's top-k over candidates [lo, hi) as tr_topk returns it: descending, equal
+    scores by lower index, padded with -1 / -inf; indices offset to the whole request."""
+    import torch
+
+    import oracle
+    sel = oracle.topk(scores[lo:hi], k) if hi > lo else np.zeros(0, np.int64)
+    idx = np.full(k, -1, np.int64)
+    sc = np.full(k, -np.inf, np.float32)
+    idx[:len(sel)] = sel + lo
+    sc[:len(sel)] = scores[lo:hi][sel]
+    return torch.from_numpy(idx), torch.from_numpy(sc)
+
+
+def _topk_worker(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        def select(s, kk):          # the oracle's top-k on the gathered scores (test stand-in for tr_topk)
+            return torch.from_numpy(oracle.topk(s.numpy(), kk))
+        results = []
+        rng = np.random.default_rng(5)
+        for n, k, levels in [(1000, 100, 7), (1000, 37, 0), (150, 200, 5), (3, 5, 0), (257, 256, 2)]:
+            # few distinct values make ties, many across the ranks' boundary
+            raw = rng.integers(0, levels, size=n) if levels else rng.normal(size=n)
+            scores = raw.astype(np.float32)
+            c = split_request(n, world)
+            li, ls = _local_topk(scores, c[rank], c[rank + 1], k)
+            idx, sc = merge_topk(li, ls, k, select=select)
+            want = oracle.topk(scores, k)
+            ok = (np.array_equal(idx.numpy()[:len(want)], want)
+                  and np.array_equal(sc.numpy()[:len(want)], scores[want])
+                  and np.all(idx.numpy()[len(want):] == -1) and np.all(sc.numpy()[len(want):] == -np.inf))
+            results.append((n, k, bool(ok)))
+        q.put((rank, results))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gloo_two_ranks_merged_topk_equals_whole_request():
+    """One request split over two ranks: the merged local top-k lists equal the top-k of
+    the whole request, ties (by lower index) and padding included."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_topk_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=240)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    out = dict(q.get(timeout=5) for _ in range(2))
+    for rank in (0, 1):
+        assert all(ok for _, _, ok in out[rank]), out[rank]

@@ -65,3 +65,68 @@ def max_over_ranks(x: float, group=None) -> float:
     t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
     return float(t.item())
+
+
+# ------------------------------------------------------------------ one request over ranks
+#
+# A request too large for one GPU's time budget can be split: every rank recomputes the
+# request's user side (cheaper than sending the K/V cache) and scores a contiguous slice of
+# its candidates, then the ranks exchange their local top-k in one all-gather and each
+# selects the request's top-k from the world x k gathered pairs.  The local top-k of each
+# slice holds every candidate of that slice that can reach the global top-k, so the merge
+# is exact.
+
+
+def split_request(n_cand: int, world: int, tile: int = 128) -> List[int]:
+    """Boundaries c[0] = 0 <= c[1] <= ... <= c[world] = n_cand: rank r scores candidates
+    [c[r], c[r+1]) of one request.  Cuts fall on multiples of ``tile`` (the score kernel's
+    tile), and the ranks' tile counts differ by at most one."""
+    if world < 1:
+        raise ValueError("world must be >= 1")
+    if n_cand < 0 or tile < 1:
+        raise ValueError("n_cand must be >= 0 and tile >= 1")
+    T = -(-n_cand // tile)
+    return [min(n_cand, tile * (T * r // world)) for r in range(world)] + [n_cand]
+
+
+def merge_topk(local_idx, local_scores, k: int, group=None, select=None):
+    """The top-k of one request whose candidates are split over the ranks of ``group``.
+
+    local_idx [k] int64 / local_scores [k] fp32: this rank's top-k over its slice as
+    tr_topk gives it (descending, equal scores by lower index, padded with -1 / -inf), the
+    indices already offset to the whole request.  One collective gathers every rank's
+    pairs, packed into one int64 tensor of 2k entries; then ``select(scores, k)`` returns
+    the positions of the k best of the world * k gathered scores (default: tr_topk on the
+    device).  Rank r's slice precedes rank r + 1's, and each list is ordered, so equal
+    scores resolve to the lower candidate index as in a single tr_topk over the request.
+    Padding entries compete with NaN scores (below every other score); only a request
+    with NaN scores and fewer than k other candidates can see padding win a tie.
+    Returns (idx [k] int64, scores [k] fp32), identical on every rank."""
+    import torch
+    import torch.distributed as dist
+
+    if select is None:
+        from . import api
+
+        def select(s, kk):
+            pos, _ = api.topk(s, [0, s.numel()], kk)
+            return pos[0]
+    world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
+    if local_idx.numel() != k or local_scores.numel() != k:
+        raise ValueError("local_idx and local_scores must hold k entries")
+    nan = torch.full_like(local_scores, float("nan"))
+    s = torch.where(local_idx >= 0, local_scores, nan)          # padding ranks last
+    packed = torch.cat([local_idx.to(torch.int64), s.view(torch.int32).to(torch.int64)])
+    parts = [torch.empty_like(packed) for _ in range(world)]
+    if world > 1:
+        dist.all_gather(parts, packed, group=group)
+    else:
+        parts = [packed]
+    allp = torch.stack(parts).view(world, 2, k)
+    all_idx = allp[:, 0, :].reshape(-1)
+    all_scores = allp[:, 1, :].reshape(-1).to(torch.int32).view(torch.float32)
+    pos = select(all_scores, k)
+    idx = all_idx[pos]
+    sc = all_scores[pos]
+    sc = torch.where(idx >= 0, sc, torch.full_like(sc, float("-inf")))
+    return idx, sc
