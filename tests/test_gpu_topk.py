@@ -103,3 +103,34 @@ def test_topk_empty_requests():
     off = [0, 0, 0]
     got_i, got_v = _run(np.zeros(1, np.float32)[:0], off, 5)
     assert np.all(got_i == -1) and np.all(np.isneginf(got_v))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("n,k,levels,cuts", [(40000, 2000, 50, [0, 19968, 40000]), (1000, 300, 4, [0, 384, 640, 1000]),
+                                             (300, 500, 0, [0, 0, 300])])
+def test_split_request_topk_merge_on_device(n, k, levels, cuts):
+    """A request's candidates in slices (emulated ranks on one GPU): tr_topk per slice,
+    indices offset, packed, then merged with tr_topk as the selection; equal to tr_topk
+    over the whole request, ties and padding included."""
+    import torch
+
+    from transformer_candidate_scoring_b200 import api
+    from transformer_candidate_scoring_b200.shard import merge_gathered, pack_topk
+    rng = np.random.default_rng(n + k)
+    raw = rng.integers(0, levels, size=n) if levels else rng.normal(size=n)
+    scores = torch.from_numpy(raw.astype(np.float32)).cuda()
+    parts = []
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        idx = torch.full((k,), -1, dtype=torch.int64, device="cuda")
+        sc = torch.full((k,), float("-inf"), dtype=torch.float32, device="cuda")
+        if hi > lo:
+            pi, ps = api.topk(scores[lo:hi].contiguous(), [0, hi - lo], k)
+            idx = torch.where(pi[0] >= 0, pi[0] + lo, pi[0])
+            sc = ps[0]
+        parts.append(pack_topk(idx, sc, k))
+    got_idx, got_sc = merge_gathered(parts, k)
+    want_idx, want_sc = api.topk(scores, [0, n], k)
+    torch.cuda.synchronize()
+    assert api.sync_status() == 0
+    assert torch.equal(got_idx, want_idx[0]), (got_idx[:10], want_idx[0][:10])
+    assert torch.equal(got_sc, want_sc[0])

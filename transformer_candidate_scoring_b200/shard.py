@@ -89,44 +89,58 @@ def split_request(n_cand: int, world: int, tile: int = 128) -> List[int]:
     return [min(n_cand, tile * (T * r // world)) for r in range(world)] + [n_cand]
 
 
-def merge_topk(local_idx, local_scores, k: int, group=None, select=None):
-    """The top-k of one request whose candidates are split over the ranks of ``group``.
-
-    local_idx [k] int64 / local_scores [k] fp32: this rank's top-k over its slice as
-    tr_topk gives it (descending, equal scores by lower index, padded with -1 / -inf), the
-    indices already offset to the whole request.  One collective gathers every rank's
-    pairs, packed into one int64 tensor of 2k entries; then ``select(scores, k)`` returns
-    the positions of the k best of the world * k gathered scores (default: tr_topk on the
-    device).  Rank r's slice precedes rank r + 1's, and each list is ordered, so equal
-    scores resolve to the lower candidate index as in a single tr_topk over the request.
-    Padding entries compete with NaN scores (below every other score); only a request
-    with NaN scores and fewer than k other candidates can see padding win a tie.
-    Returns (idx [k] int64, scores [k] fp32), identical on every rank."""
+def pack_topk(local_idx, local_scores, k: int):
+    """One rank's top-k as the all-gather sends it: [2k] int64, the k indices then the k
+    scores' fp32 bits, padding (index -1) turned into NaN scores so it ranks last."""
     import torch
-    import torch.distributed as dist
+
+    if local_idx.numel() != k or local_scores.numel() != k:
+        raise ValueError("local_idx and local_scores must hold k entries")
+    s = torch.where(local_idx >= 0, local_scores, torch.full_like(local_scores, float("nan")))
+    return torch.cat([local_idx.to(torch.int64), s.contiguous().view(torch.int32).to(torch.int64)])
+
+
+def merge_gathered(parts, k: int, select=None):
+    """The request's top-k from every rank's packed list, in rank order: (idx [k] int64,
+    scores [k] fp32), padded with -1 / -inf.  ``select(scores, k)`` returns the positions
+    of the k best gathered scores (default: tr_topk on the device)."""
+    import torch
 
     if select is None:
         from . import api
 
-        def select(s, kk):
-            pos, _ = api.topk(s, [0, s.numel()], kk)
+        def select(sc, kk):
+            pos, _ = api.topk(sc, [0, sc.numel()], kk)
             return pos[0]
-    world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
-    if local_idx.numel() != k or local_scores.numel() != k:
-        raise ValueError("local_idx and local_scores must hold k entries")
-    nan = torch.full_like(local_scores, float("nan"))
-    s = torch.where(local_idx >= 0, local_scores, nan)          # padding ranks last
-    packed = torch.cat([local_idx.to(torch.int64), s.view(torch.int32).to(torch.int64)])
-    parts = [torch.empty_like(packed) for _ in range(world)]
-    if world > 1:
-        dist.all_gather(parts, packed, group=group)
-    else:
-        parts = [packed]
+    world = len(parts)
     allp = torch.stack(parts).view(world, 2, k)
     all_idx = allp[:, 0, :].reshape(-1)
     all_scores = allp[:, 1, :].reshape(-1).to(torch.int32).view(torch.float32)
     pos = select(all_scores, k)
     idx = all_idx[pos]
     sc = all_scores[pos]
-    sc = torch.where(idx >= 0, sc, torch.full_like(sc, float("-inf")))
-    return idx, sc
+    return idx, torch.where(idx >= 0, sc, torch.full_like(sc, float("-inf")))
+
+
+def merge_topk(local_idx, local_scores, k: int, group=None, select=None):
+    """The top-k of one request whose candidates are split over the ranks of ``group``.
+
+    local_idx [k] int64 / local_scores [k] fp32: this rank's top-k over its slice as
+    tr_topk gives it (descending, equal scores by lower index, padded with -1 / -inf), the
+    indices already offset to the whole request.  One collective gathers every rank's
+    pairs (pack_topk: one int64 tensor of 2k entries); then every rank selects the k best
+    of the world * k gathered pairs (merge_gathered).  Rank r's slice precedes rank
+    r + 1's and each list is ordered, so equal scores resolve to the lower candidate index
+    as in a single tr_topk over the request.  Padding competes as NaN (below every other
+    score): only a request with NaN scores and fewer than k other candidates can see
+    padding win a tie.  Returns (idx [k] int64, scores [k] fp32), identical on every rank."""
+    import torch
+    import torch.distributed as dist
+
+    packed = pack_topk(local_idx, local_scores, k)
+    world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
+    parts = [packed]
+    if world > 1:
+        parts = [torch.empty_like(packed) for _ in range(world)]
+        dist.all_gather(parts, packed, group=group)
+    return merge_gathered(parts, k, select)
