@@ -114,8 +114,10 @@ void tr_model_destroy(tr_model* m);
 /*
  * Weighted-average aggregation (TransRetrieval §3.2): for every bag b
  *     out[b] = sum_{i in bag b} weights[i] * table[bag_table[b]][keys[i]] / sum_{i in b} weights[i]
- * accumulated in fp32.  A bag with no keys, or whose weights sum to exactly 0, yields the
- * zero vector.  Duplicate keys count once per occurrence.
+ * accumulated in fp32; the division is a multiplication by the correctly rounded fp32
+ * reciprocal of the weight sum, so scaling every weight of a bag by a power of two leaves
+ * the result bit-identical.  A bag with no keys, or whose weights sum to exactly 0, yields
+ * the zero vector.  Duplicate keys count once per occurrence.
  *   tables     HOST array [n_tables] (<= TR_MAX_TABLES); all tables share one dtype
  *   bag_table  DEVICE int32 [n_bags], each in [0, n_tables)  (validated on the device:
  *              an out-of-range entry zeroes the bag and sets TR_ERR_KEY_RANGE)
