@@ -293,7 +293,7 @@ def run_ours(args, rank, world, local_rank):
     graphs = []
     for s_i in range(N_REQUEST_SETS):
         use(s_i)
-        graphs.append(dw.capture_step(torch.cuda.Stream()))
+        graphs.append(dw.capture_step())
     for i in range(args.warmup):
         graphs[i % N_REQUEST_SETS].replay()
     torch.cuda.synchronize()

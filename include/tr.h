@@ -22,8 +22,14 @@
  *    can see (a key outside its table) do not stop the kernel: the offending key is
  *    skipped and a device status word is set; tr_sync_status() reports it.
  *  - The caller owns every input/output device buffer.  The library owns the model
- *    handle (its repacked weights) and, per device, an internal workspace used by some
- *    kernels; both are released by tr_model_destroy() / at process exit.
+ *    handle (its repacked weights, released by tr_model_destroy()), a status word per
+ *    device, and scratch for the calls that run as a sequence of CUDA-core kernels (fp32
+ *    models, user sides or score calls with more than 128 user tokens, the uncompressed-
+ *    target variant): one buffer per (device, stream), kept until process exit.  Calls on
+ *    different streams never share scratch; calls on one stream are ordered by it.  A call
+ *    that needs more scratch than its stream's buffer holds synchronises that stream and
+ *    reallocates it, so the first such call on a stream must not be made while the stream
+ *    is being captured into a CUDA graph.  The tensor-core paths use no scratch.
  *  - Row-major layouts unless stated; "[a][b]" means a rows of b contiguous elements.
  *  - dtype TR_F32 models compute in fp32 throughout.  TR_BF16 models store tables,
  *    weights, target-field tokens and candidate tokens in bf16 and accumulate in fp32.

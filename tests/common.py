@@ -1,7 +1,21 @@
 """Shared test helpers: error metrics and top-k agreement (no method arithmetic)."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
+
+# The stated bar: max relative error 2e-2 for bf16 models, 1e-4 for fp32.  It applies to
+# the scores, element by element (relative error floored at the output's rms, so that
+# values near zero do not make it ill-conditioned), and to the whole score vector in
+# max-norm.
+TOL_SCORE = {"bf16": 2e-2, "f32": 1e-4}
+# Intermediate outputs of the bf16 path (the per-layer K/V images of the user side, the
+# compressed target tokens) are stored in bf16 after several bf16-operand GEMMs.  Their
+# normwise error is held to the score bar; elementwise they get this named, separate bound
+# (the measured maxima are listed with the parity readings in the design notes).
+TOL_INTERMEDIATE_EL_BF16 = 5e-2
 
 
 def rel_err(got, ref, floor_frac: float = 1.0) -> float:
@@ -31,19 +45,39 @@ def normwise_err(got, ref) -> float:
     return float(np.max(np.abs(g - r)) / (den if den > 0 else 1.0))
 
 
-def check_close(got, ref, dtype: str, what: str = "") -> dict:
+def _log(entry: dict) -> None:
+    path = os.environ.get("TR_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(entry) + "\n")
+
+
+def check_close(got, ref, dtype: str, what: str = "", kind: str = "score") -> dict:
     """Parity bar for one output.
 
-    bf16: normwise error <= 2e-2 (the stated tolerance, read as the max-norm relative
-    error of the output vector) and the elementwise error, floored at the output's rms,
-    <= 5e-2.  fp32: both <= 1e-4.  Returns the measured metrics (also the elementwise
-    error with a 0.1*rms floor, for information)."""
-    tol = 2e-2 if dtype == "bf16" else 1e-4
-    tol_el = 5e-2 if dtype == "bf16" else 1e-4
+    kind="score" (the scores of a request): elementwise error with the rms floor and the
+    normwise error both <= 2e-2 for bf16, <= 1e-4 for fp32.
+    kind="intermediate" (K/V images, compressed tokens): normwise <= the same bar,
+    elementwise <= TOL_INTERMEDIATE_EL_BF16 for bf16 (1e-4 for fp32).
+    Returns the measured metrics (also the elementwise error with a 0.1*rms floor, for
+    information); with TR_PARITY_LOG set, appends them to that file as one JSON line."""
+    if kind not in ("score", "intermediate"):
+        raise ValueError(kind)
+    tol = TOL_SCORE[dtype]
+    tol_el = TOL_INTERMEDIATE_EL_BF16 if (kind == "intermediate" and dtype == "bf16") else tol
     m = {"normwise": normwise_err(got, ref), "elementwise_rms_floor": rel_err(got, ref),
          "elementwise_0.1rms_floor": rel_err(got, ref, 0.1)}
-    assert m["normwise"] <= tol and m["elementwise_rms_floor"] <= tol_el, (what, m)
+    _log({"test": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], "what": what, "kind": kind,
+          "dtype": dtype, "n": int(np.asarray(ref).size), **m})
+    assert m["normwise"] <= tol and m["elementwise_rms_floor"] <= tol_el, (what, kind, m)
     return m
+
+
+def score_topk_tol(ref_scores, dtype: str) -> float:
+    """Absolute score band for top-k agreement: the stated relative bar times the rms of the
+    oracle's scores (the same floor as the elementwise score metric)."""
+    r = np.asarray(ref_scores, dtype=np.float64)
+    return TOL_SCORE[dtype] * float(np.sqrt(np.mean(r * r))) if r.size else 0.0
 
 
 def topk_agrees(got_idx, ref_scores, k: int, tol_abs: float) -> tuple[bool, str]:

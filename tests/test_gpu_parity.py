@@ -1,9 +1,11 @@
 """GPU parity: every stage of libtr against the fp64 oracle on the same seeded inputs.
 
 Inputs come from ``datagen`` only (tables, bags, stand-alone tokens); the oracle never
-reads anything the CUDA path produced.  Tolerances (tests/common.py, check_close): fp32
-models 1e-4; bf16 models 2e-2 as the max-norm relative error of each output, with the
-elementwise error floored at the output's rms bounded by 5e-2.
+reads anything the CUDA path produced.  Tolerances (tests/common.py, check_close): scores
+within 1e-4 (fp32 models) or 2e-2 (bf16 models), both element by element (relative error
+floored at the scores' rms) and in max-norm; intermediate bf16 outputs (K/V images,
+compressed tokens) are held to the same max-norm bar and to a separate, named elementwise
+bound.
 """
 import numpy as np
 import pytest
@@ -11,7 +13,7 @@ import torch
 
 import datagen
 import oracle
-from common import check_close, normwise_err, rel_err, topk_agrees
+from common import check_close, normwise_err, rel_err, score_topk_tol, topk_agrees
 from kvdecode import decode_kv
 
 pytestmark = pytest.mark.gpu
@@ -237,8 +239,8 @@ def test_prefill_parity(name, L_u, init):
     dec = decode_kv(kv.cpu().numpy(), dims.dtype, dims.n_layer, L_u, dims.D)
     K, V = oracle.prefill_user(P, dims.n_head, U, 1)
     for l in range(dims.n_layer):
-        check_close(dec[0][l], K[l], dims.dtype, f"K layer {l}")
-        check_close(dec[1][l], V[l], dims.dtype, f"V layer {l}")
+        check_close(dec[0][l], K[l], dims.dtype, f"K layer {l}", kind="intermediate")
+        check_close(dec[1][l], V[l], dims.dtype, f"V layer {l}", kind="intermediate")
     if dims.dtype == "bf16":
         assert np.all(dec[2] == 0) and np.all(dec[3] == 0)     # zero padding rows
 
@@ -257,7 +259,7 @@ def test_compress_parity(name, n, init):
     torch.cuda.synchronize()
     ref = oracle.compress_targets(P, X)
     got = out.double().cpu().numpy()
-    check_close(got, ref, dims.dtype, "tokens")
+    check_close(got, ref, dims.dtype, "tokens", kind="intermediate")
 
 
 # ---------------------------------------------------------------- candidate stack (§3.3)
@@ -358,7 +360,7 @@ def test_pipeline_end_to_end(name, n, rows, init):
         ref = oracle.score_request(w, P, req).scores
         g = got[dw.req_offsets[r]:dw.req_offsets[r + 1]]
         print(r, check_close(g, ref, w.dims.dtype, f"request {r}"))
-        tol_abs = TOL[w.dims.dtype] * float(np.max(np.abs(ref)))
+        tol_abs = score_topk_tol(ref, w.dims.dtype)
         k = min(100, len(ref))
         idx = np.lexsort((np.arange(len(g)), -g))[:k]
         ok, why = topk_agrees(idx, ref, k, tol_abs)
@@ -440,15 +442,16 @@ def _serial_reference(w, sets):
     return dw, ref
 
 
-@pytest.mark.parametrize("n_sms", [6, 148])
-def test_overlapped_steps_match_serial_steps(n_sms):
+@pytest.mark.parametrize("name,n_sms", [("128d5l", 6), ("128d5l", 148), ("64d3l", 6), ("tiny", 6)])
+def test_overlapped_steps_match_serial_steps(name, n_sms):
     """Consecutive requests overlapped over two slots (compression and scoring split at
     their last partial wave, whose tail runs beside the next request's aggregation) give
     each request the scores of a serial step, bit for bit, eagerly and from one captured
     graph.  n_sms = 6 forces a split at this size (16 tiles: 12 + 4); at 148 there is a
-    single wave and no split."""
+    single wave and no split.  The fp32 model runs every stage on the CUDA-core kernels,
+    whose scratch is per stream: the user, main and tail streams run them concurrently."""
     from transformer_candidate_scoring_b200.pipeline import DeviceWorkload, Overlapped, score_split
-    w = datagen.scaled(datagen.WORKLOADS["128d5l"], n_cand_per_request=2000, rows=20000)
+    w = datagen.scaled(datagen.WORKLOADS[name], n_cand_per_request=2000, rows=20000)
     sets = [datagen.make_requests(w, seed=700 + k) for k in range(3)]
     dw, ref = _serial_reference(w, sets)
     dw2 = DeviceWorkload(w, reqs=sets[0], params=dw.params, tables=(dw.user_tables, dw.target_tables))
@@ -473,7 +476,10 @@ def test_overlapped_steps_match_serial_steps(n_sms):
     for o in out:
         o.zero_()
     g = ov.capture(0, n_batch, bind=bind, scored=scored)
-    assert ov.launches_per_step == (7 if n_sms == 6 else 5)   # compress and score each in two parts
+    if name == "128d5l":
+        assert ov.launches_per_step == (7 if n_sms == 6 else 5)   # compress and score each in two parts
+    for o in out:
+        o.zero_()
     g.replay()
     torch.cuda.synchronize()
     assert tr().sync_status() == 0
@@ -543,9 +549,9 @@ def test_host_feed_overlapped_matches_serial_steps():
     assert tr().sync_status() == 0
     for i in range(7):
         assert torch.equal(out[i], ref[i % 3].cpu()), ("eager", i)
+    g = feed.capture_overlapped(ov, 0, 7, out)
     for o in out:
         o.zero_()
-    g = feed.capture_overlapped(ov, 0, 7, out)
     g.replay()
     torch.cuda.synchronize()
     assert tr().sync_status() == 0
@@ -588,7 +594,8 @@ def test_compress_corpus_chunked_equals_one_pass_and_oracle():
                                                 sub.weights[sub.offsets[f]:sub.offsets[f + 1]])[0])
         rows.append(np.concatenate(toks))
     ref = oracle.compress_targets(dw.params, np.stack(rows))
-    check_close(out[torch.from_numpy(idx).cuda()].double().cpu().numpy(), ref, "bf16", "corpus sample")
+    check_close(out[torch.from_numpy(idx).cuda()].double().cpu().numpy(), ref, "bf16", "corpus sample",
+                kind="intermediate")
 
 
 def test_captured_step_replays_bit_identical():
@@ -600,8 +607,8 @@ def test_captured_step_replays_bit_identical():
     dw.step()
     torch.cuda.synchronize()
     ref = dw.scores.clone()
+    g = dw.capture_step()
     dw.scores.zero_()
-    g = dw.capture_step(torch.cuda.Stream())
     g.replay()
     g.replay()
     torch.cuda.synchronize()

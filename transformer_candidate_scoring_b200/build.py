@@ -1,28 +1,39 @@
-"""Builds libtr.so in-tree with nvcc for sm_100a."""
+"""Builds libtr.so in-tree with nvcc for sm_100a.
+
+Every ``csrc/*.cu`` is compiled to its own object under ``_build/`` (in parallel, and only
+when it or a header changed), then the objects are linked into ``libtr.so``.
+"""
 from __future__ import annotations
 
 import glob
 import os
 import subprocess
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtr.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
+OBJ_DIR = os.path.join(os.path.dirname(HERE), "_build")
 
-NVCC_FLAGS = [
-    "-gencode", "arch=compute_100a,code=sm_100a",
-    "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
-    "--expt-relaxed-constexpr",
-]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+NVCC_FLAGS = [*ARCH, "-lineinfo", "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr"]
 
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
+def _headers():
+    return sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "tr.h")]
+
+
 def _inputs():
-    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "tr.h")]
+    return sources() + _headers()
+
+
+def _obj(src: str) -> str:
+    return os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + ".o")
 
 
 def is_stale() -> bool:
@@ -36,9 +47,25 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     if not force and not is_stale():
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
-    cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-o", LIB + ".tmp", *sources()]
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    newest_header = max(os.path.getmtime(h) for h in _headers())
+
+    def compile_one(src):
+        obj = _obj(src)
+        if (not force and os.path.exists(obj) and not extra
+                and os.path.getmtime(obj) > max(os.path.getmtime(src), newest_header)):
+            return
+        cmd = [nvcc, *NVCC_FLAGS, *extra, "-I", INCLUDE, "-c", "-o", obj + ".tmp", src]
+        if verbose:
+            print(" ".join(cmd), flush=True)
+        subprocess.run(cmd, check=True)
+        os.replace(obj + ".tmp", obj)
+
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        list(ex.map(compile_one, sources()))
+    cmd = [nvcc, *ARCH, "-shared", "-o", LIB + ".tmp", *[_obj(s) for s in sources()]]
     if verbose:
-        print(" ".join(cmd))
+        print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
     os.replace(LIB + ".tmp", LIB)
     return LIB

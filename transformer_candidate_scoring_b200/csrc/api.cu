@@ -54,25 +54,56 @@ tr_status device_state(DeviceState** out) {
   return TR_OK;
 }
 
-tr_status workspace(size_t bytes, void** out) {
-  DeviceState* s = nullptr;
-  TR_TRY(device_state(&s));
+namespace {
+struct StreamScratch {
+  int dev;
+  cudaStream_t stream;
+  void* ptr;
+  size_t bytes;
+};
+std::vector<StreamScratch> g_scratch;   // guarded by g_dev_mu
+std::vector<std::pair<int, const void*>> g_attr_done;
+}  // namespace
+
+tr_status workspace(size_t bytes, cudaStream_t st, void** out) {
+  int dev = 0;
+  TR_CUDA_TRY(cudaGetDevice(&dev));
   std::lock_guard<std::mutex> lk(g_dev_mu);
-  if (s->workspace_bytes < bytes) {
-    if (s->workspace) {
-      TR_CUDA_TRY(cudaDeviceSynchronize());
-      TR_CUDA_TRY(cudaFree(s->workspace));
-      s->workspace = nullptr;
-      s->workspace_bytes = 0;
+  StreamScratch* s = nullptr;
+  for (auto& e : g_scratch)
+    if (e.dev == dev && e.stream == st) s = &e;
+  if (!s) {
+    g_scratch.push_back({dev, st, nullptr, 0});
+    s = &g_scratch.back();
+  }
+  if (s->bytes < bytes) {
+    if (s->ptr) {
+      // earlier work on this stream may still read the old buffer
+      TR_CUDA_TRY(cudaStreamSynchronize(st));
+      TR_CUDA_TRY(cudaFree(s->ptr));
+      s->ptr = nullptr;
+      s->bytes = 0;
     }
-    size_t want = bytes + bytes / 4;
-    if (cudaMalloc(&s->workspace, want) != cudaSuccess) {
+    const size_t want = bytes + bytes / 4;
+    if (cudaMalloc(&s->ptr, want) != cudaSuccess) {
       cudaGetLastError();
+      s->ptr = nullptr;
       return fail(TR_ERR_NOMEM, "workspace allocation of %zu bytes failed", want);
     }
-    s->workspace_bytes = want;
+    s->bytes = want;
   }
-  *out = s->workspace;
+  *out = s->ptr;
+  return TR_OK;
+}
+
+tr_status ensure_smem_attr(const void* kernel, int bytes) {
+  int dev = 0;
+  TR_CUDA_TRY(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  for (auto& e : g_attr_done)
+    if (e.first == dev && e.second == kernel) return TR_OK;
+  TR_CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  g_attr_done.push_back({dev, kernel});
   return TR_OK;
 }
 

@@ -43,14 +43,17 @@ void count_launch();
 // Bits set by kernels that meet input only the device can check.
 enum : int { STATUS_KEY_RANGE = 1, STATUS_KERNEL_TIMEOUT = 2 };
 
-// Per-device state: the status word and a grow-only workspace for multi-kernel calls.
+// Per-device state: the status word.
 struct DeviceState {
   int* status = nullptr;       // device int
-  void* workspace = nullptr;   // device scratch
-  size_t workspace_bytes = 0;
 };
 tr_status device_state(DeviceState** out);                 // of the current device
-tr_status workspace(size_t bytes, void** out);             // grows the current device's workspace
+// Scratch of the multi-kernel (CUDA-core) calls: one grow-only buffer per (device, stream),
+// so that calls on different streams never share scratch.  Growing it synchronises the
+// stream and reallocates.
+tr_status workspace(size_t bytes, cudaStream_t st, void** out);
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel), under a lock.
+tr_status ensure_smem_attr(const void* kernel, int bytes);
 
 // ---------------------------------------------------------------- numeric helpers
 __device__ __forceinline__ float to_f32(float x) { return x; }

@@ -516,14 +516,10 @@ tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens,
   p.c1 = c[1];
   p.c2 = c[2];
   p.c3 = c[3];
-  static bool attr_set[64] = {};
   int dev = 0, sms = 148;
   TR_CUDA_TRY(cudaGetDevice(&dev));
   TR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  if (!attr_set[dev]) {
-    TR_CUDA_TRY(cudaFuncSetAttribute(compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    attr_set[dev] = true;
-  }
+  TR_TRY(ensure_smem_attr((const void*)compress_kernel, SMEM_BYTES));
   compress_kernel<<<std::min(p.n_tiles, sms), 320, SMEM_BYTES, st>>>(p);
   TR_LAUNCH_CHECK("compress_kernel");
   return TR_OK;

@@ -317,7 +317,7 @@ tr_status simt_prefill(const tr_model* m, const float* user_tokens, int L_u, int
   const int D = m->desc.D, H = m->desc.ffn_hidden;
   if (L_u == 0) return TR_OK;
   float* ws = nullptr;
-  TR_TRY(workspace((size_t)L_u * (6 * D + H) * sizeof(float), (void**)&ws));
+  TR_TRY(workspace((size_t)L_u * (6 * D + H) * sizeof(float), st, (void**)&ws));
   float *y = ws, *a = y + L_u * D, *qkv = a + L_u * D, *o = qkv + 3 * L_u * D, *hb = o + L_u * D;
   add_vec_rows<float><<<ceil_div((int64_t)L_u * D, 256), 256, 0, st>>>(user_tokens, y, L_u, D,
                                                                         m->domain_emb + (int64_t)domain * D);
@@ -341,7 +341,7 @@ tr_status simt_compress(const tr_model* m, const void* x, int64_t n, void* token
   const int64_t chunk = 16384;
   float* ws = nullptr;
   const int64_t rows = std::min<int64_t>(n, chunk);
-  TR_TRY(workspace((size_t)rows * (c[1] + c[2] + c[3]) * sizeof(float), (void**)&ws));
+  TR_TRY(workspace((size_t)rows * (c[1] + c[2] + c[3]) * sizeof(float), st, (void**)&ws));
   float *h1 = ws, *h2 = h1 + rows * c[1], *t = h2 + rows * c[2];
   for (int64_t r0 = 0; r0 < n; r0 += chunk) {
     const int M = (int)std::min<int64_t>(chunk, n - r0);
@@ -386,7 +386,7 @@ tr_status simt_score_lt(const tr_model* m, const void* tokens, int64_t c0, int64
   if (n <= 0) return TR_OK;
   const int64_t rows = std::min<int64_t>(n, chunk) * lt;
   float* ws = nullptr;
-  TR_TRY(workspace((size_t)rows * (6 * D + H + 1) * sizeof(float), (void**)&ws));
+  TR_TRY(workspace((size_t)rows * (6 * D + H + 1) * sizeof(float), st, (void**)&ws));
   float *y = ws, *a = y + rows * D, *qkv = a + rows * D, *o = qkv + 3 * rows * D, *hb = o + rows * D;
   float* tok_scores = hb + rows * H;
   const int Lp = round_up16(L_u);

@@ -986,17 +986,9 @@ int hg_of(int L_u) {
 
 template <bool PF>
 tr_status launch_stack(int hg, int grid, const StackParams& p, cudaStream_t st) {
-  static bool done[64][4] = {};
-  int dev = 0;
-  TR_CUDA_TRY(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return fail(TR_ERR_UNSUPPORTED, "device %d", dev);
-  const int hi = hg == 8 ? 0 : hg == 4 ? 1 : hg == 2 ? 2 : 3;
   void (*k)(StackParams) = hg == 8 ? stack_kernel<PF, 8> : hg == 4 ? stack_kernel<PF, 4>
                          : hg == 2 ? stack_kernel<PF, 2> : stack_kernel<PF, 1>;
-  if (!done[dev][hi]) {
-    TR_CUDA_TRY(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES));
-    done[dev][hi] = true;
-  }
+  TR_TRY(ensure_smem_attr((const void*)k, SMEM_BYTES));
   k<<<grid, kThreads, SMEM_BYTES, st>>>(p);
   TR_LAUNCH_CHECK(PF ? "stack_kernel (user side)" : "stack_kernel");
   return TR_OK;

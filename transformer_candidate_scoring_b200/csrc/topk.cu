@@ -213,14 +213,7 @@ tr_status launch_topk(const float* scores, const int64_t* req_offsets, int R, in
   p.k_pow2 = kp;
   for (int r = 0; r <= R; ++r) p.off[r] = req_offsets[r];
   const size_t smem = (size_t)kp * sizeof(unsigned long long);
-  static bool attr_set[64] = {};
-  int dev = 0;
-  TR_CUDA_TRY(cudaGetDevice(&dev));
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    TR_CUDA_TRY(cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)(TR_MAX_TOPK * sizeof(unsigned long long))));
-    attr_set[dev] = true;
-  }
+  TR_TRY(ensure_smem_attr((const void*)topk_kernel, (int)(TR_MAX_TOPK * sizeof(unsigned long long))));
   topk_kernel<<<R, kThreads, smem, st>>>(p);
   TR_LAUNCH_CHECK("topk_kernel");
   return TR_OK;

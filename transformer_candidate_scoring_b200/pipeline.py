@@ -173,13 +173,22 @@ class DeviceWorkload:
                          torch.empty(len(self.reqs), k, dtype=torch.float32, device=self.device))
         return api.topk(self.scores, self.req_offsets, k, self._sel[0], self._sel[1], stream=stream)
 
+    def capture_stream(self) -> "torch.cuda.Stream":
+        """The stream this workload captures graphs on (created once)."""
+        if not hasattr(self, "_cap"):
+            self._cap = torch.cuda.Stream(self.device)
+        return self._cap
+
     def capture_step(self, stream=None) -> "torch.cuda.CUDAGraph":
         """One step with the current bags, captured into a CUDA graph (replay it to run the
         step again without host launch overhead; the bags, caches and activations it reads
-        and writes are the ones bound now).  Run an eager step first: the library sets up
-        per-device state on first use, which capture does not allow."""
+        and writes are the ones bound now).  The first capture on a stream runs the step
+        once eagerly on it: the library sets up per-device state and, for its CUDA-core
+        kernels, per-stream scratch on first use, which a capture does not allow."""
+        cap = stream if stream is not None else self.capture_stream()
+        warm_up_stream(cap, lambda: self.step(cap))
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
+        with torch.cuda.graph(g, stream=cap):
             self.step()
         return g
 
@@ -223,6 +232,20 @@ class DeviceWorkload:
         if events:
             events["score"].record(main)
         return self.scores
+
+
+_WARM_STREAMS = set()
+
+
+def warm_up_stream(stream, run) -> None:
+    """Runs ``run()`` eagerly once per stream (then waits for it), before the first capture
+    on that stream."""
+    key = (stream.device.index, int(stream.cuda_stream))
+    if key in _WARM_STREAMS:
+        return
+    run()
+    stream.synchronize()
+    _WARM_STREAMS.add(key)
 
 
 SCORE_TILE = 128   # candidates per tile of the tensor-core score kernel
@@ -283,6 +306,7 @@ class Overlapped:
         _, hi = torch.cuda.Stream.priority_range()
         self.user = torch.cuda.Stream(dev, priority=hi)
         self.back = torch.cuda.Stream(dev, priority=hi)
+        self.cap = torch.cuda.Stream(dev)
         self.n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
         self.launches_per_step = None
 
@@ -341,10 +365,12 @@ class Overlapped:
     def capture(self, first: int, count: int, **hooks) -> "torch.cuda.CUDAGraph":
         """run(first, count, ...) captured into one CUDA graph (replay it to run the same
         batches again; the overlap holds between the captured batches, not across replays).
-        Run the slots eagerly once first: the library sets up per-device state on first
-        use, which capture does not allow."""
+        The first capture runs the batches once eagerly on the capture stream: the library
+        sets up per-device state and per-stream scratch on first use, which capture does
+        not allow."""
         g = torch.cuda.CUDAGraph()
-        cap = torch.cuda.Stream(self.slots[0].device)
+        cap = self.cap
+        warm_up_stream(cap, lambda: self.run(first, count, cap, **hooks))
         l0 = api.kernel_launches()
         with torch.cuda.graph(g, stream=cap):
             self.run(first, count, cap, **hooks)
@@ -408,14 +434,14 @@ class HostFeed:
 
     def capture(self) -> None:
         """Capture one CUDA graph per (device slot, host batch) pair, so that run() replays
-        the step instead of launching its kernels one by one.  Call it after one run(): the
-        library sets up per-device state on first use, which capture does not allow."""
+        the step instead of launching its kernels one by one (on the workload's capture
+        stream; see DeviceWorkload.capture_step)."""
         self.graphs = {}
         n = len(self.batches)
         for i in range(2 * n if n % 2 else n):       # every (slot, batch) pair occurs
             du, dt = self._views(i)
             self.dw.use_bags(du, dt, self.batches[i % n][2])
-            self.graphs[(i % 2, i % n)] = self.dw.capture_step(torch.cuda.Stream(self.dw.device))
+            self.graphs[(i % 2, i % n)] = self.dw.capture_step()
 
     def run(self, first: int, count: int, host_scores, stream=None) -> None:
         """Score batches first .. first + count - 1 (batch i uses host batch i mod len);
@@ -486,9 +512,11 @@ class HostFeed:
                 host_scores[i % len(host_scores)].copy_(scores, non_blocking=True)
 
     def capture_overlapped(self, ov: "Overlapped", first: int, count: int, host_scores) -> "torch.cuda.CUDAGraph":
-        """run_overlapped(...) captured into one CUDA graph, host copies included."""
+        """run_overlapped(...) captured into one CUDA graph, host copies included (on
+        ``ov``'s capture stream, warmed as in Overlapped.capture)."""
         g = torch.cuda.CUDAGraph()
-        cap = torch.cuda.Stream(self.dw.device)
+        cap = ov.cap
+        warm_up_stream(cap, lambda: self.run_overlapped(ov, first, count, host_scores, cap))
         with torch.cuda.graph(g, stream=cap):
             self.run_overlapped(ov, first, count, host_scores, cap)
         return g
