@@ -184,6 +184,17 @@ def time_oracle(w, P, req, target_seconds=15.0, max_cand=None):
     return rate, desc, threads, t_user + dt
 
 
+def oracle_rates(w, P, req, seconds_all=15.0, seconds_one=6.0):
+    """The oracle's candidates/s on one request with every host thread its BLAS uses and
+    with one thread, plus the host's core counts."""
+    from threadpoolctl import threadpool_limits
+    rate, desc, threads, _ = time_oracle(w, P, req, target_seconds=seconds_all)
+    with threadpool_limits(limits=1):
+        rate1, _, _, _ = time_oracle(w, P, req, target_seconds=seconds_one)
+    return {"value": rate, "unit": "candidates/s", "cores": threads, "kind": "oracle", "sample": desc,
+            "one_thread": rate1, "nproc": os.cpu_count(), "affinity": len(os.sched_getaffinity(0))}
+
+
 def bench_config(n_cand: int, L_u: int, world: int) -> dict:
     """The workload both arms report."""
     return {"workload": "128D-5L, 1 request x 40,000 candidates per GPU, L_u=64, 8 target fields, "
@@ -200,17 +211,22 @@ def run_reference(args, rank, world):
     w = datagen.WORKLOADS[WORKLOAD]
     P = datagen.workload_params(w)
     req = datagen.make_requests(w)[0]
-    # size each step to a bounded sample so W+K steps stay within a few minutes
-    budget = max(4.0, 150.0 / max(1, args.steps + args.warmup))
-    vals = []
+    # each step is a bounded sample of the request (its user side and a slice of its
+    # candidates), sized so that the W + K steps stay within a few minutes; ms_per_step is
+    # the time one such step took
+    budget = max(2.0, 150.0 / max(1, args.steps + args.warmup))
+    vals, secs_all = [], []
     for i in range(args.warmup + args.steps):
         rate, desc, threads, secs = time_oracle(w, P, req, target_seconds=budget)
         if i >= args.warmup:
             vals.append(rate)
+            secs_all.append(secs)
     v = float(np.median(vals))
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "candidates/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.n_cand_per_request / v * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": float(np.mean(secs_all)) * 1e3,
+        "step": "one bounded sample of the request per step (its user side plus a slice of its candidates); "
+                "value = the request's candidates / (user side + per-candidate time x candidates)",
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": bench_config(w.n_cand_per_request, 64, 1),
         "cpu_baseline": {"value": v, "unit": "candidates/s", "cores": threads, "kind": "oracle", "sample": desc},
@@ -221,12 +237,136 @@ def run_reference(args, rank, world):
 
 # ------------------------------------------------------------------ GPU leg
 
+STAGE_SPANS = {"user_side": ("user0", "user1"), "target_aggregate": ("t0", "agg"), "compress": ("agg", "comp"),
+               "score": ("s0", "score")}
+EV_KEYS = ["user0", "user1", "t0", "agg", "comp", "s0", "score"]
+
+
+def stage_rooflines(dims, reqs, stage_ms, peaks, peak_kind):
+    """Achieved rate and fraction of the measured peak of the three bulk stages of one step."""
+    n_cand = sum(r.n_cand for r in reqs)
+    fl_stack = sum(stack_flops_per_candidate(dims, r.L_u) * r.n_cand for r in reqs)
+    fl_comp = compressor_flops_per_candidate(dims) * n_cand
+    eb = 2 if dims.dtype == "bf16" else 4
+    agg_bytes = sum(aggregate_bytes(r.target, dims.D, eb, eb) for r in reqs)
+    roof = {
+        "score": {"bound": "tensor", "achieved": fl_stack / (stage_ms["score"] / 1e3) / 1e12,
+                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"},
+        "compress": {"bound": "tensor", "achieved": fl_comp / (stage_ms["compress"] / 1e3) / 1e12,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"},
+        "target_aggregate": {"bound": "hbm", "achieved": agg_bytes / (stage_ms["target_aggregate"] / 1e3) / 1e9,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s"},
+    }
+    for r in roof.values():
+        r["frac"] = r["achieved"] / r["peak"]
+        r["peak_source"] = peak_kind
+    return roof
+
+
+def measure_side(name, w, params, tables, reqs, dev, steps, warmup, peaks, peak_kind, cpu_seconds):
+    """One of the other workloads on the same GPU (every stage through the C calls): stage
+    times from eager steps, the step from one CUDA graph per step replayed back to back, and
+    the overlapped stream of requests (one graph); the oracle's rate on the same request."""
+    import torch
+
+    from transformer_candidate_scoring_b200 import api
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload, Overlapped
+
+    stream = torch.cuda.current_stream()
+    dw = DeviceWorkload(w, device=dev, reqs=reqs, params=params, tables=tables)
+    for _ in range(warmup):
+        dw.step(stream)
+    torch.cuda.synchronize()
+    ev = [{k: torch.cuda.Event(enable_timing=True) for k in EV_KEYS} for _ in range(steps)]
+    for i in range(steps):
+        dw.step(stream, ev[i])
+    torch.cuda.synchronize()
+    stage_ms = {n: float(np.mean([ev[i][a].elapsed_time(ev[i][b]) for i in range(steps)]))
+                for n, (a, b) in STAGE_SPANS.items()}
+    g = dw.capture_step()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    serial_ms = e0.elapsed_time(e1) / steps
+    del g
+    dw2 = DeviceWorkload(w, device=dev, reqs=reqs, params=params, tables=tables)
+    ov = Overlapped([dw, dw2])
+    ov.run(0, warmup, stream)
+    torch.cuda.synchronize()
+    g = ov.capture(0, steps)
+    g.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ov_ms = e0.elapsed_time(e1) / steps
+    del g
+    if api.sync_status() != 0:
+        raise RuntimeError(f"device status word set during the {name} measurement")
+    n_cand = dw.n_cand
+    out = {"workload": w.name, "candidates_per_step": n_cand, "requests": len(reqs),
+           "L_u": [r.L_u for r in reqs] if len(reqs) > 1 else reqs[0].L_u,
+           "value": n_cand / (ov_ms / 1e3), "unit": "candidates/s", "ms_per_step": ov_ms,
+           "serial_graph_ms_per_step": serial_ms,
+           "stages": {k: {"ms": v} for k, v in stage_ms.items()}}
+    for k, r in stage_rooflines(w.dims, reqs, stage_ms, peaks, peak_kind).items():
+        out["stages"][k].update(r)
+    if cpu_seconds > 0:
+        out["cpu_baseline"] = oracle_rates(w, params, reqs[0], cpu_seconds, cpu_seconds / 2)
+    del dw, dw2, ov
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_side_configs(args, dev, main_dw, peaks, peak_kind):
+    """The 64D-3L, packed 16 x 4,096 and 52M-row large-corpus workloads (the other
+    single-GPU configurations the headline is reported beside)."""
+    import torch
+
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload
+
+    res = {}
+    cpu_s = 0.0 if args.no_cpu_baseline else 6.0
+    steps, warm = max(3, min(args.steps, 10)), 3
+    # 64D-3L: its own tables (16 of 1M rows x 64) and parameters
+    w = datagen.WORKLOADS["64d3l"]
+    res["64d3l"] = measure_side("64d3l", w, datagen.workload_params(w), DeviceWorkload.make_tables(w, dev),
+                                datagen.make_requests(w), dev, steps, warm, peaks, peak_kind, cpu_s)
+    torch.cuda.empty_cache()
+    # packed: 16 requests of the 128D-5L model, L_u ~ U{16..128}, 4,096 candidates each (the
+    # headline workload's tables and parameters; the request shapes are the packed recipe's)
+    w = datagen.WORKLOADS["packed"]
+    tables = (main_dw.user_tables, main_dw.target_tables)
+    res["packed"] = measure_side("packed", w, main_dw.params, tables, datagen.make_requests(w), dev, steps, warm,
+                                 peaks, peak_kind, cpu_s)
+    res["packed"]["tables"] = "the 128D-5L workload's tables and parameters"
+    # large corpus: target field 0 reads one 52M-row table (uniform keys); the other tables
+    # are the headline workload's
+    w = datagen.WORKLOADS["large"]
+    big = torch.empty(w.target_rows[0], w.dims.D, dtype=torch.bfloat16, device=dev)
+    datagen.fill_table_device(big, w.seed, datagen.target_table_id(w, 0))
+    tables = (main_dw.user_tables, [big] + list(main_dw.target_tables[1:]))
+    res["large"] = measure_side("large", w, main_dw.params, tables, datagen.make_requests(w), dev,
+                                max(3, steps // 2), 2, peaks, peak_kind, cpu_s)
+    res["large"]["tables"] = "one 52M x 128 bf16 table (13.3 GB) for field 0 plus the 128D-5L workload's tables"
+    del big
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
     from transformer_candidate_scoring_b200 import api
-    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, HostFeed, Overlapped
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, HostFeed, Overlapped, score_split
     from transformer_candidate_scoring_b200.shard import max_over_ranks, rank_seed
 
     torch.cuda.set_device(local_rank)
@@ -369,7 +509,7 @@ def run_ours(args, rank, world, local_rank):
     # of batch i + 1 are copied while batch i computes)
     host_batches = []
     for ub, tb, reqs in dsets:
-        hu = [DeviceBags(*(x.cpu().pin_memory() for x in (b.offsets, b.keys, b.weights, b.bag_table))) for b in ub]
+        hu = DeviceBags(*(x.cpu().pin_memory() for x in (ub.offsets, ub.keys, ub.weights, ub.bag_table)))
         ht = DeviceBags(*(x.cpu().pin_memory() for x in (tb.offsets, tb.keys, tb.weights, tb.bag_table)))
         host_batches.append((hu, ht, reqs))
     feed = HostFeed(dw, host_batches)
@@ -413,32 +553,38 @@ def run_ours(args, rank, world, local_rank):
     # ---- rooflines of the stages
     peaks, peak_kind = load_peaks()
     L_u = dw.L_u[0]
-    fl_stack = stack_flops_per_candidate(dims, L_u) * n_cand
-    fl_comp = compressor_flops_per_candidate(dims) * n_cand
-    tb_host = sets[0][0].target
-    agg_bytes = aggregate_bytes(tb_host, dims.D, 2, 2)
-    stage_roof = {
-        "score": {"bound": "tensor", "achieved": fl_stack / (stage_ms["score"] / 1e3) / 1e12,
-                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"},
-        "compress": {"bound": "tensor", "achieved": fl_comp / (stage_ms["compress"] / 1e3) / 1e12,
-                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"},
-        "target_aggregate": {"bound": "hbm", "achieved": agg_bytes / (stage_ms["target_aggregate"] / 1e3) / 1e9,
-                             "peak": peaks["hbm_gbs"], "unit": "GB/s"},
-    }
-    for r in stage_roof.values():
-        r["frac"] = r["achieved"] / r["peak"]
-        r["peak_source"] = peak_kind
+    stage_roof = stage_rooflines(dims, sets[0], stage_ms, peaks, peak_kind)
     dominant = max(("score", "compress", "target_aggregate"), key=lambda k: stage_ms[k])
     roof = dict(stage_roof[dominant])
     roof["kernel"] = dominant
     roof["traffic"] = profiled_traffic("stack_kernel") if dominant == "score" else None
+    # the score kernel over its full rounds alone (the candidates before score_split: every
+    # CTA busy until the end), eager launches timed with events on the launching stream
+    cut = score_split(dw.req_offsets, torch.cuda.get_device_properties(dev).multi_processor_count)
+    full_round = None
+    if cut is not None:
+        use(0)
+        dw.step(stream)
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dw.score_range(0, cut, stream)
+        f0.record(stream)
+        for _ in range(args.steps):
+            dw.score_range(0, cut, stream)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        fr_ms = f0.elapsed_time(f1) / args.steps
+        fr_ach = stack_flops_per_candidate(dims, L_u) * cut / (fr_ms / 1e3) / 1e12
+        full_round = {"candidates": cut, "ms": fr_ms, "achieved": fr_ach, "unit": "TFLOP/s",
+                      "peak": peaks["bf16_tflops"], "frac": fr_ach / peaks["bf16_tflops"], "peak_source": peak_kind}
+    roof_score_full = full_round
+    side = None if (args.no_side_configs or world > 1) else run_side_configs(args, dev, dw, peaks, peak_kind)
 
     if rank != 0:
         return
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        rate, desc, threads, secs = time_oracle(w, dw.params, sets[0][0], target_seconds=args.cpu_seconds)
-        cpu = {"value": rate, "unit": "candidates/s", "cores": threads, "kind": "oracle", "sample": desc}
+        cpu = oracle_rates(w, dw.params, sets[0][0], args.cpu_seconds, args.cpu_seconds / 2)
     line = {
         "metric": METRIC, "value": value, "unit": "candidates/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed / args.steps * 1e3, "higher_is_better": True,
@@ -448,6 +594,8 @@ def run_ours(args, rank, world, local_rank):
         "stages": {k: {"ms": stage_ms[k], **({kk: vv for kk, vv in stage_roof[k].items()} if k in stage_roof else {})}
                    for k in stage_names},
         "pct_bf16_peak_score_kernel": stage_roof["score"]["frac"] * 100,
+        "score_full_rounds": roof_score_full,
+        "configs": side,
         "topk": {"k": TOPK, "ms": topk_ms, "note": "tr_topk over the step's scores, timed separately"},
         "e2e": {"value": e2e_value, "unit": "candidates/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_elapsed / args.steps * 1e3,
@@ -480,7 +628,7 @@ def run_case(args):
     U = torch.from_numpy(datagen.rand_matrix(1, (64, dims.D), 0.01, "f32")).cuda()
     kv = torch.zeros(api.kv_cache_bytes(m, 64), dtype=torch.uint8, device="cuda")
     X = torch.from_numpy(datagen.rand_matrix(3, (n, dims.comp_dims[0]), 0.01, "bf16")).cuda().to(torch.bfloat16)
-    T = torch.empty(n, dims.D, dtype=torch.bfloat16, device="cuda")
+    T = torch.empty(n, dims.D, dtype=torch.float32, device="cuda")
     s = torch.empty(n, dtype=torch.float32, device="cuda")
     for _ in range(args.case_reps):
         if args.case in ("prefill", "all"):
@@ -511,7 +659,7 @@ def run_bulk(args):
     tables = DeviceWorkload.make_tables(w.with_(user_tables=0), torch.device("cuda"))
     model = api.Model(dims, datagen.workload_params(w))
     bags = DeviceBags.of(datagen.make_target_bags(np.random.default_rng(w.seed + 77), w, n), "cuda")
-    out = torch.empty(n, dims.D, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(n, dims.D, dtype=torch.float32, device="cuda")
     F = dims.n_target_fields
     compress_corpus(model, tables[1], bags, n, F, out)
     torch.cuda.synchronize()
@@ -579,6 +727,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-side-configs", action="store_true", help="skip the 64D-3L, packed and large workloads")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", choices=["score", "compress", "prefill", "all", "bulk", "uncompressed"], default=None,
                     help="run one stage on stand-alone inputs for a profiler (no timing, no JSON)")

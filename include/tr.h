@@ -32,7 +32,12 @@
  *    is being captured into a CUDA graph.  The tensor-core paths use no scratch.
  *  - Row-major layouts unless stated; "[a][b]" means a rows of b contiguous elements.
  *  - dtype TR_F32 models compute in fp32 throughout.  TR_BF16 models store tables,
- *    weights, target-field tokens and candidate tokens in bf16 and accumulate in fp32.
+ *    weights and target-field tokens in bf16; the compressed candidate tokens are fp32 for
+ *    every model.  The tensor-core kernels of a TR_BF16 model multiply fp16 operands (the
+ *    bf16 weights converted exactly, activations rounded to fp16's 11-bit significand),
+ *    except the compressor's first layer, which multiplies the bf16 field tokens by bf16
+ *    weights; every product accumulates in fp32.  A TR_BF16 model whose LayerNorm gains
+ *    and weights could push an fp16 operand out of range runs on the CUDA-core kernels.
  */
 #ifndef TR_H
 #define TR_H
@@ -163,7 +168,7 @@ tr_status tr_aggregate_ex(const tr_table* tables, int n_tables, const int32_t* b
  * Bytes of one request's user K/V cache for L_u user tokens (0 <= L_u <= TR_MAX_LU).
  * Layout (opaque to most callers; tests decode it):
  *   TR_F32 model : [n_layer][2][L_u][D] fp32, K then V, row-major.
- *   TR_BF16 model: per layer a K image then a V image, bf16, in the tensor-core operand
+ *   TR_BF16 model: per layer a K image then a V image, fp16, in the tensor-core operand
  *   layout.  With Lp = L_u rounded up to 16 (rows >= L_u are zero) and 8x8 "core
  *   matrices" of 128 contiguous bytes (8 rows of 8 consecutive elements):
  *     K image  [Lp x D]: element (j, d) at core (d/8)*(Lp/8) + j/8, within it (j%8)*8 + d%8
@@ -185,10 +190,22 @@ tr_status tr_prefill_user(const tr_model* m, const float* user_tokens, int L_u, 
                           void* kv, tr_stream stream);
 
 /*
+ * The user sides of R requests in one call: tr_prefill_user for every request r, run as one
+ * launch of one tensor-core CTA per request when the model and every L_u (<= 128) allow it,
+ * else one call after the other.  Requests with L_u[r] = 0 write nothing.
+ *   user_tokens HOST array [R] of DEVICE fp32 [L_u[r]][D]
+ *   L_u, domain HOST int32 [R]
+ *   kv          HOST array [R] of DEVICE buffers of tr_kv_cache_bytes(m, L_u[r]) bytes
+ * 1 <= R <= TR_MAX_REQUESTS.  Every argument is validated before anything is launched.
+ */
+tr_status tr_prefill_users(const tr_model* m, const float* const* user_tokens, const int32_t* L_u,
+                           const int32_t* domain, void* const* kv, int R, tr_stream stream);
+
+/*
  * Target compressor (TransRetrieval §3.3): t = W3 g2(W2 g1(W1 x + b1) + b2) + b3 with
  * g_i(z) = LayerNorm_i(PReLU_i(z)).
  *   x      DEVICE [n][comp_dims[0]] of the model dtype (the concatenated field tokens)
- *   tokens DEVICE [n][D] of the model dtype.
+ *   tokens DEVICE fp32 [n][D].
  */
 tr_status tr_compress_targets(const tr_model* m, const void* x, int64_t n, void* tokens,
                               tr_stream stream);
@@ -200,7 +217,7 @@ tr_status tr_compress_targets(const tr_model* m, const void* x, int64_t n, void*
  * attention over its request's L_u cached user keys/values plus its own key/value,
  * then the Pre-LN ReLU FFN; score = w_head . LayerNorm_f(y) + b_head.  A candidate never
  * sees another candidate or another request's cache.
- *   tokens      DEVICE [n][D] of the model dtype
+ *   tokens      DEVICE fp32 [n][D] (as tr_compress_targets writes them)
  *   req_offsets HOST int64 [R+1], req_offsets[0] = 0, non-decreasing, req_offsets[R] = n
  *   kv          HOST array [R] of DEVICE pointers (caches written by tr_prefill_user)
  *   L_u, domain HOST int32 [R]

@@ -3,13 +3,13 @@ import numpy as np
 
 
 def decode_kv(raw: np.ndarray, dtype: str, n_layer: int, L_u: int, D: int):
-    """raw: uint8 bytes of the cache -> (K, V) float64 [n_layer, L_u, D]."""
+    """raw: uint8 bytes of the cache -> (K, V) float64 [n_layer, L_u, D] (fp32 model: fp32
+    rows; bf16 model: fp16 core-matrix images)."""
     if dtype == "f32":
         a = raw[: n_layer * 2 * L_u * D * 4].view(np.float32).reshape(n_layer, 2, L_u, D).astype(np.float64)
         return a[:, 0], a[:, 1]
     Lp = (L_u + 15) // 16 * 16
-    u16 = raw[: n_layer * 2 * Lp * D * 2].view(np.uint16).reshape(n_layer, 2, Lp * D)
-    f = (u16.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    f = raw[: n_layer * 2 * Lp * D * 2].view(np.float16).reshape(n_layer, 2, Lp * D).astype(np.float64)
     K = np.zeros((n_layer, Lp, D))
     V = np.zeros((n_layer, Lp, D))
     j = np.arange(Lp)[:, None]

@@ -254,7 +254,7 @@ def test_compress_parity(name, n, init):
     P = datagen.make_params(dims, 4, init)
     m = tr().Model(dims, P)
     X = datagen.rand_matrix(22, (n, dims.comp_dims[0]), 0.3 if init == "wide" else 0.01, dims.dtype)
-    out = torch.empty(n, dims.D, dtype=tdt(dims.dtype), device="cuda")
+    out = torch.empty(n, dims.D, dtype=torch.float32, device="cuda")
     tr().compress_targets(m, dev(X, tdt(dims.dtype)), out)
     torch.cuda.synchronize()
     ref = oracle.compress_targets(P, X)
@@ -283,7 +283,7 @@ def _score_setup(name, init, L_us, n_per, seed=5, token_std=None):
 
 
 def _gpu_scores(m, dims, toks, kvs, L_us, doms):
-    T = dev(np.concatenate(toks), tdt(dims.dtype))
+    T = dev(np.concatenate(toks), torch.float32)
     off = np.concatenate([[0], np.cumsum([len(t) for t in toks])])
     s = torch.empty(int(off[-1]), dtype=torch.float32, device="cuda")
     tr().score_candidates(m, T, off.tolist(), kvs, L_us, doms, s)
@@ -395,7 +395,7 @@ def test_full_size_sampled(name, n_sample):
 def test_host_feed_matches_device_resident_steps():
     """Bags fed from pinned host memory with the copy of batch i + 1 overlapping batch i
     (two device slots) give bit-identical scores to the device-resident steps."""
-    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, HostFeed, pack_target_bags
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, HostFeed, pack_target_bags, pack_user_bags
     w = datagen.scaled(datagen.WORKLOADS["128d5l"], n_cand_per_request=500, rows=20000)
     sets = [datagen.make_requests(w, seed=900 + k) for k in range(3)]
     dw = DeviceWorkload(w, reqs=sets[0])
@@ -408,7 +408,7 @@ def test_host_feed_matches_device_resident_steps():
 
     def pinned(b):
         return DeviceBags(*(x.pin_memory() for x in (b.offsets, b.keys, b.weights, b.bag_table)))
-    batches = [([pinned(DeviceBags.of(r.user, "cpu")) for r in reqs], pinned(DeviceBags.of(pack_target_bags(reqs), "cpu")),
+    batches = [(pinned(DeviceBags.of(pack_user_bags(reqs), "cpu")), pinned(DeviceBags.of(pack_target_bags(reqs), "cpu")),
                 reqs) for reqs in sets]
     feed = HostFeed(dw, batches)
     out = [torch.empty(dw.n_cand, dtype=torch.float32).pin_memory() for _ in range(7)]
@@ -447,8 +447,8 @@ def test_overlapped_steps_match_serial_steps(name, n_sms):
     """Consecutive requests overlapped over two slots (compression and scoring split at
     their last partial wave, whose tail runs beside the next request's aggregation) give
     each request the scores of a serial step, bit for bit, eagerly and from one captured
-    graph.  n_sms = 6 forces a split at this size (16 tiles: 12 + 4); at 148 there is a
-    single wave and no split.  The fp32 model runs every stage on the CUDA-core kernels,
+    graph.  n_sms = 6 forces a split at this size (16 tiles = 8 units of two: 6 + 2); at 148
+    there is a single round and no split.  The fp32 model runs every stage on the CUDA-core kernels,
     whose scratch is per stream: the user, main and tail streams run them concurrently."""
     from transformer_candidate_scoring_b200.pipeline import DeviceWorkload, Overlapped, score_split
     w = datagen.scaled(datagen.WORKLOADS[name], n_cand_per_request=2000, rows=20000)
@@ -492,11 +492,11 @@ _SET_BAGS = {}
 
 def _set_bags(dw, sets, i):
     """Device bags of request set i % len(sets) (uploaded once per set)."""
-    from transformer_candidate_scoring_b200.pipeline import DeviceBags, pack_target_bags
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, pack_target_bags, pack_user_bags
     reqs = sets[i % len(sets)]
     key = (id(dw), i % len(sets))
     if key not in _SET_BAGS:
-        _SET_BAGS[key] = ([DeviceBags.of(r.user, dw.device) for r in reqs],
+        _SET_BAGS[key] = (DeviceBags.of(pack_user_bags(reqs), dw.device),
                           DeviceBags.of(pack_target_bags(reqs), dw.device), reqs)
     return _SET_BAGS[key]
 
@@ -511,7 +511,7 @@ def test_overlapped_packed_requests_split_inside_a_request():
     dw.set_requests(sets[0])
     dw2 = DeviceWorkload(w, reqs=sets[1], params=dw.params, tables=(dw.user_tables, dw.target_tables))
     ov = Overlapped([dw, dw2])
-    ov.n_sms = 10                                  # 48 tiles -> 40 + 8, cut inside request 13
+    ov.n_sms = 9                                   # 32 units -> 27 + 5, cut one unit into request 13
     cut = score_split(dw.req_offsets, ov.n_sms)
     assert cut is not None and cut not in dw.req_offsets
     out = [torch.zeros(dw.n_cand, dtype=torch.float32, device="cuda") for _ in range(5)]
@@ -530,17 +530,17 @@ def test_overlapped_packed_requests_split_inside_a_request():
 def test_host_feed_overlapped_matches_serial_steps():
     """Host-fed batches through the overlapped slots (bags copied during the previous batch,
     scores copied back after the last score launch), eager and as one captured graph."""
-    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, HostFeed, Overlapped, pack_target_bags
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, HostFeed, Overlapped, pack_target_bags, pack_user_bags
     w = datagen.scaled(datagen.WORKLOADS["128d5l"], n_cand_per_request=1000, rows=20000)
     sets = [datagen.make_requests(w, seed=950 + k) for k in range(3)]
     dw, ref = _serial_reference(w, sets)
     dw2 = DeviceWorkload(w, reqs=sets[0], params=dw.params, tables=(dw.user_tables, dw.target_tables))
     ov = Overlapped([dw, dw2])
-    ov.n_sms = 5                                   # 8 tiles -> 5 + 3
+    ov.n_sms = 3                                   # 4 units -> 3 + 1
 
     def pinned(b):
         return DeviceBags(*(x.pin_memory() for x in (b.offsets, b.keys, b.weights, b.bag_table)))
-    batches = [([pinned(DeviceBags.of(r.user, "cpu")) for r in reqs], pinned(DeviceBags.of(pack_target_bags(reqs), "cpu")),
+    batches = [(pinned(DeviceBags.of(pack_user_bags(reqs), "cpu")), pinned(DeviceBags.of(pack_target_bags(reqs), "cpu")),
                 reqs) for reqs in sets]
     feed = HostFeed(dw, batches)
     out = [torch.empty(dw.n_cand, dtype=torch.float32).pin_memory() for _ in range(7)]
@@ -570,11 +570,11 @@ def test_compress_corpus_chunked_equals_one_pass_and_oracle():
     bags = datagen.make_target_bags(np.random.default_rng(4), w, n_items)
     db = DeviceBags.of(bags, "cuda")
     F, D = w.dims.n_target_fields, w.dims.D
-    out = torch.empty(n_items, D, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty(n_items, D, dtype=torch.float32, device="cuda")
     compress_corpus(dw.model, dw.target_tables, db, n_items, F, out, chunk=1536)
     X = torch.empty(n_items, F * D, dtype=torch.bfloat16, device="cuda")
     api.aggregate(dw.target_tables, db.bag_table, db.offsets, db.keys, db.weights, X.view(-1, D))
-    ref_gpu = torch.empty(n_items, D, dtype=torch.bfloat16, device="cuda")
+    ref_gpu = torch.empty(n_items, D, dtype=torch.float32, device="cuda")
     api.compress_targets(dw.model, X, ref_gpu)
     torch.cuda.synchronize()
     assert tr().sync_status() == 0

@@ -1,46 +1,52 @@
 """Host-side scheduling logic of the pipeline (no GPU): where the score call is split so
-that the next request can start beside the score kernel's last partial wave."""
+that the next request can start beside the score kernel's last partial round of units
+(two 128-candidate tiles of one request per CTA)."""
 import itertools
 
 import numpy as np
 import pytest
 
-from transformer_candidate_scoring_b200.pipeline import SCORE_TILE, score_split
+from transformer_candidate_scoring_b200.pipeline import SCORE_TILE, SCORE_UNIT, score_split
+
+PER = SCORE_TILE * SCORE_UNIT
 
 
-def _tiles(off):
-    return [-(-(off[r + 1] - off[r]) // SCORE_TILE) for r in range(len(off) - 1)]
+def _units(off):
+    return [-(-(off[r + 1] - off[r]) // PER) for r in range(len(off) - 1)]
 
 
-def _tile_index(off, c):
-    """Number of tiles that lie wholly before packed candidate c (c on a tile boundary)."""
+def _unit_index(off, c):
+    """Number of units that lie wholly before packed candidate c (c on a unit boundary)."""
     t = 0
     for r in range(len(off) - 1):
         if c >= off[r + 1]:
-            t += -(-(off[r + 1] - off[r]) // SCORE_TILE)
+            t += -(-(off[r + 1] - off[r]) // PER)
         elif c > off[r]:
-            assert (c - off[r]) % SCORE_TILE == 0, "split not on a tile boundary of its request"
-            t += (c - off[r]) // SCORE_TILE
+            assert (c - off[r]) % PER == 0, "split not on a unit boundary of its request"
+            t += (c - off[r]) // PER
     return t
 
 
 def test_single_request_of_the_128d5l_workload():
-    # 40,000 candidates = 313 tiles = 2 full waves of 148 + 17: the split is after 296 tiles
+    # 40,000 candidates = 313 tiles = 157 units = one full round of 148 + 9: the split is
+    # after 148 units (296 tiles)
     assert score_split([0, 40000], 148) == 296 * 128
 
 
-@pytest.mark.parametrize("off,n_sms", [([0, 148 * 128], 148), ([0, 100], 148), ([0, 147 * 128 + 5], 148),
-                                       ([0, 0], 148), ([0, 40000], 0), ([0, 300, 300, 900], 8)])
-def test_no_split_without_a_partial_wave(off, n_sms):
-    # an exact number of waves, a single wave, no candidates or no SM count: nothing to split
-    # (the last case: 3 + 0 + 5 = 8 tiles, one wave of 8)
+@pytest.mark.parametrize("off,n_sms", [([0, 296 * 128], 148), ([0, 100], 148), ([0, 295 * 128 + 5], 148),
+                                       ([0, 0], 148), ([0, 40000], 0), ([0, 300, 300, 900], 5)])
+def test_no_split_without_a_partial_round(off, n_sms):
+    # an exact number of rounds, a single round, no candidates or no SM count: nothing to
+    # split (the last case: 2 + 0 + 3 = 5 units, one round of 5)
     assert score_split(off, n_sms) is None
 
 
 def test_split_at_a_request_boundary_and_inside_a_request():
-    off = [300 * i for i in range(17)]             # 16 requests of 3 tiles (the last one ragged)
-    assert score_split(off, 7) == 4200             # 48 = 42 + 6: after request 13
-    assert score_split(off, 10) == 3900 + 128      # 48 = 40 + 8: one tile into request 13
+    off = [300 * i for i in range(17)]             # 16 requests of 2 units (3 tiles; the last unit short)
+    assert score_split(off, 7) == 4200             # 32 = 28 + 4: after request 13
+    assert score_split(off, 10) == 4500            # 32 = 30 + 2: after request 14
+    off = [1000 * i for i in range(4)]             # 3 requests of 4 units
+    assert score_split(off, 5) == 2000 + 2 * PER   # 12 = 10 + 2: two units into request 2
 
 
 def test_split_properties_over_random_batches():
@@ -51,14 +57,14 @@ def test_split_properties_over_random_batches():
         sizes[rng.random(R) < 0.2] = 0             # some empty requests
         off = [0] + list(itertools.accumulate(int(x) for x in sizes))
         n_sms = int(rng.integers(1, 40))
-        T = sum(_tiles(off))
+        U = sum(_units(off))
         cut = score_split(off, n_sms)
-        if T <= n_sms or T % n_sms == 0:
+        if U <= n_sms or U % n_sms == 0:
             assert cut is None
             continue
         assert cut is not None and 0 < cut < off[-1]
-        a = _tile_index(off, cut)
-        assert a == T - T % n_sms                  # the full waves before the cut
+        a = _unit_index(off, cut)
+        assert a == U - U % n_sms                  # the full rounds before the cut
         assert a % n_sms == 0
 
 
@@ -185,7 +191,7 @@ class _Slot:
         return [x.name for b in bags for x in (b.offsets, b.keys, b.weights, b.bag_table)]
 
     def user_aggregate(self, s):
-        s.launch(self._bags(self.ub), [f"{self.name}.user_tokens"], f"{self.name} user_aggregate")
+        s.launch(self._bags([self.ub]), [f"{self.name}.user_tokens"], f"{self.name} user_aggregate")
 
     def user_prefill(self, s):
         s.launch([f"{self.name}.user_tokens"], [f"{self.name}.kv"], f"{self.name} prefill")
@@ -274,7 +280,7 @@ def test_race_check_detects_a_missing_wait(fake_cuda):
 def test_overlapped_steps_have_no_stream_races(fake_cuda, n_cand, count):
     pipeline, fake, log = fake_cuda
     slots = [_Slot(fake.cuda, f"slot{k}", n_cand) for k in range(2)]
-    resident = [([], _Bags(fake.cuda, f"set{k}")) for k in range(3)]   # read-only device bags
+    resident = [(_Bags(fake.cuda, f"set{k}.user"), _Bags(fake.cuda, f"set{k}")) for k in range(3)]   # read-only
 
     def bind(i, dw, main):
         dw.use_bags(*resident[i % 3], None)
@@ -298,7 +304,7 @@ def _Bags(cuda, name):
 def test_host_feed_overlapped_has_no_stream_races(fake_cuda):
     pipeline, fake, log = fake_cuda
     slots = [_Slot(fake.cuda, f"slot{k}", 40000) for k in range(2)]
-    batches = [([_Bags(fake.cuda, f"host{k}.user")], _Bags(fake.cuda, f"host{k}.target"), None) for k in range(3)]
+    batches = [(_Bags(fake.cuda, f"host{k}.user"), _Bags(fake.cuda, f"host{k}.target"), None) for k in range(3)]
     feed = pipeline.HostFeed(slots[0], batches)
     ov = pipeline.Overlapped(slots)
     host_scores = [_Buf(fake.cuda, f"host_scores{k}") for k in range(2)]

@@ -153,6 +153,21 @@ def prefill_user(model: Model, user_tokens: torch.Tensor, L_u: int, domain: int,
     return kv
 
 
+def prefill_users(model: Model, user_tokens: Sequence[torch.Tensor], L_u: Sequence[int], domain: Sequence[int],
+                  kv: Sequence[torch.Tensor], stream=None) -> None:
+    """tr_prefill_users: the user sides of R requests in one call (fp32 user tokens [L_u, D]
+    of each request -> its K/V cache)."""
+    R = len(L_u)
+    ut = (C.c_void_p * R)(*[(t.data_ptr() if int(l) else 0) for t, l in zip(user_tokens, L_u)])
+    kvp = (C.c_void_p * R)(*[(k.data_ptr() if int(l) else 0) for k, l in zip(kv, L_u)])
+    lu = (C.c_int32 * R)(*[int(x) for x in L_u])
+    dm = (C.c_int32 * R)(*[int(x) for x in domain])
+    for t in list(user_tokens) + list(kv):
+        if not t.is_cuda:
+            raise ValueError("expected CUDA tensors")
+    _check(L.load().tr_prefill_users(model.handle, ut, lu, dm, kvp, R, _stream(stream)))
+
+
 def prefill_user_noalloc(model: Model, user_tokens: torch.Tensor, L_u: int, domain: int, kv: torch.Tensor,
                          stream=None) -> torch.Tensor:
     """tr_prefill_user_noalloc: the user side with no device allocation, for callers that
@@ -163,14 +178,18 @@ def prefill_user_noalloc(model: Model, user_tokens: torch.Tensor, L_u: int, doma
 
 
 def compress_targets(model: Model, x: torch.Tensor, tokens: torch.Tensor, stream=None) -> torch.Tensor:
-    """tr_compress_targets: x [n, F*D] -> tokens [n, D] (model dtype)."""
+    """tr_compress_targets: x [n, F*D] (model dtype) -> tokens [n, D] fp32."""
+    if tokens.dtype != torch.float32:
+        raise ValueError("compressed tokens are fp32")
     _check(L.load().tr_compress_targets(model.handle, _ptr(x), x.shape[0], _ptr(tokens), _stream(stream)))
     return tokens
 
 
 def score_candidates(model: Model, tokens: torch.Tensor, req_offsets: Sequence[int], kv: Sequence[torch.Tensor],
                      L_u: Sequence[int], domain: Sequence[int], scores: torch.Tensor, stream=None) -> torch.Tensor:
-    """tr_score_candidates over packed requests; scores [n] fp32."""
+    """tr_score_candidates over packed requests: tokens [n, D] fp32; scores [n] fp32."""
+    if tokens.dtype != torch.float32:
+        raise ValueError("candidate tokens are fp32")
     R = len(L_u)
     off = (C.c_int64 * (R + 1))(*[int(x) for x in req_offsets])
     kvp = (C.c_void_p * R)(*[(k.data_ptr() if k is not None and k.numel() else 0) for k in kv])

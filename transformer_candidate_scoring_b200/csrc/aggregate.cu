@@ -190,8 +190,8 @@ __device__ __forceinline__ void gather_rows(float (&acc)[CI][Vec16<T>::N], const
 // Loop trip counts are the warp's maximum, so every shuffle is warp-uniform.
 // VAR = false compiles the plain weighted average (TR_AGG_MEAN without LayerNorm) only;
 // VAR = true reads the aggregator and the LayerNorm flag from `mode`.
-template <typename T, typename O, int LPR, int CI, bool VAR>
-__global__ void __launch_bounds__(256, 4) wavg_kernel(TableSet tabs, int n_tables,
+template <typename T, typename O, int LPR, int CI, bool VAR, int MINB>
+__global__ void __launch_bounds__(256, MINB) wavg_kernel(TableSet tabs, int n_tables,
                                                       const int32_t* __restrict__ bag_table,
                                                       const int64_t* __restrict__ offsets,
                                                       const int32_t* __restrict__ keys,
@@ -409,31 +409,38 @@ tr_status dispatch(const TableSet& ts, int n_tables, const int32_t* bag_table, c
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // 8 warps per block, 32 / LPR bags per warp at a time; 4 blocks per SM are resident and
-  // the grid is 32 blocks per SM, so that blocks started late (an SM held by a concurrent
-  // kernel) take a small share of the work
-  const int64_t bags_per_block = 8 * (32 / (vecs < 32 ? vecs : 32));
-  const int64_t blocks_needed = (n_bags + bags_per_block - 1) / bags_per_block;
-  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, (int64_t)sms * 32));
+  // 8 warps per block, 32 / LPR bags per warp at a time.  With one 16-byte vector per lane
+  // (CI = 1) 4 blocks per SM are resident and the grid is 32 blocks per SM, so that blocks
+  // started late (an SM held by a concurrent kernel) take a small share of the work.  Rows
+  // of 16 vectors (a 256-byte bf16 row of D = 128) go to 8 lanes with two vectors each: half
+  // the lanes per row and twice the bags per warp halve the per-bag instructions of the
+  // group (headers, key chunks, the weight-sum reduction and the finish); that needs more
+  // registers, so 2 blocks per SM are resident and the grid is 16 blocks per SM.
+  auto grid_of = [&](int lpr, int per_sm) {
+    const int64_t bags_per_block = 8 * (32 / lpr);
+    const int64_t blocks_needed = (n_bags + bags_per_block - 1) / bags_per_block;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(blocks_needed, (int64_t)sms * per_sm));
+  };
   // few bags (one resident round of one-bag blocks, 4 per SM): a block per bag
   const bool split = n_bags <= (int64_t)sms * 4;
   const int grid_split = (int)std::max<int64_t>(1, n_bags);
-#define TR_WAVG_K(K, G, LPR, CI, VAR) \
-  K<T, O, LPR, CI, VAR><<<G, 256, 0, st>>>(ts, n_tables, bag_table, offsets, keys, weights, n_bags, mode, out, status)
-#define TR_WAVG(LPR, CI)                                                                \
-  if (split && mode == TR_AGG_MEAN) TR_WAVG_K(wavg_split_kernel, grid_split, LPR, CI, false); \
-  else if (split) TR_WAVG_K(wavg_split_kernel, grid_split, LPR, CI, true);                    \
-  else if (mode == TR_AGG_MEAN) TR_WAVG_K(wavg_kernel, grid, LPR, CI, false);                 \
-  else TR_WAVG_K(wavg_kernel, grid, LPR, CI, true)
+#define TR_WAVG_K(K, G, LPR, CI, VAR, ...) \
+  K<T, O, LPR, CI, VAR, ##__VA_ARGS__><<<G, 256, 0, st>>>(ts, n_tables, bag_table, offsets, keys, weights, n_bags, mode, out, status)
+#define TR_WAVG(LPR, CI, MINB, PER_SM, SLPR, SCI)                                                     \
+  if (split && mode == TR_AGG_MEAN) TR_WAVG_K(wavg_split_kernel, grid_split, SLPR, SCI, false);            \
+  else if (split) TR_WAVG_K(wavg_split_kernel, grid_split, SLPR, SCI, true);                               \
+  else if (mode == TR_AGG_MEAN) TR_WAVG_K(wavg_kernel, grid_of(LPR, PER_SM), LPR, CI, false, MINB);        \
+  else TR_WAVG_K(wavg_kernel, grid_of(LPR, PER_SM), LPR, CI, true, MINB)
+  // (the block-per-bag kernel keeps one vector per lane and 16-lane groups)
   switch (vecs) {
-    case 1: TR_WAVG(1, 1); break;
-    case 2: TR_WAVG(2, 1); break;
-    case 4: TR_WAVG(4, 1); break;
-    case 8: TR_WAVG(8, 1); break;
-    case 16: TR_WAVG(16, 1); break;
-    case 32: TR_WAVG(32, 1); break;
-    case 64: TR_WAVG(32, 2); break;
-    case 128: TR_WAVG(32, 4); break;
+    case 1: TR_WAVG(1, 1, 4, 32, 1, 1); break;
+    case 2: TR_WAVG(2, 1, 4, 32, 2, 1); break;
+    case 4: TR_WAVG(4, 1, 4, 32, 4, 1); break;
+    case 8: TR_WAVG(8, 1, 4, 32, 8, 1); break;
+    case 16: TR_WAVG(8, 2, 2, 16, 16, 1); break;
+    case 32: TR_WAVG(32, 1, 4, 32, 32, 1); break;
+    case 64: TR_WAVG(32, 2, 4, 32, 32, 2); break;
+    case 128: TR_WAVG(32, 4, 4, 32, 32, 4); break;
     default: return fail(TR_ERR_UNSUPPORTED, "tr_aggregate: D=%d gives %d vectors per row (need 1..32 as a power of two, 64 or 128)", D, vecs);
   }
 #undef TR_WAVG

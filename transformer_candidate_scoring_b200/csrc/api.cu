@@ -119,6 +119,8 @@ bool tc_prefill_supported(const tr_model* m, int L_u);
 tr_status simt_prefill_noalloc(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv,
                                cudaStream_t st);
 tr_status tc_prefill(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv, cudaStream_t st);
+tr_status tc_prefill_batch(const tr_model* m, const float* const* user_tokens, const int32_t* L_u,
+                           const int32_t* domain, void* const* kv, int R, cudaStream_t st);
 
 }  // namespace tr
 
@@ -294,6 +296,25 @@ tr_status tr_prefill_user(const tr_model* m, const float* user_tokens, int L_u, 
   return simt_prefill(m, user_tokens, L_u, domain, kv, (cudaStream_t)stream);
 }
 
+tr_status tr_prefill_users(const tr_model* m, const float* const* user_tokens, const int32_t* L_u,
+                           const int32_t* domain, void* const* kv, int R, tr_stream stream) {
+  TR_TRY(check_model_device(m));
+  if (R < 1 || R > TR_MAX_REQUESTS) return fail(TR_ERR_INVALID_ARG, "R=%d (need 1..%d)", R, TR_MAX_REQUESTS);
+  if (!user_tokens || !L_u || !domain || !kv) return fail(TR_ERR_INVALID_ARG, "null host array");
+  bool batch = true;
+  for (int r = 0; r < R; ++r) {
+    if (L_u[r] < 0 || L_u[r] > TR_MAX_LU) return fail(TR_ERR_INVALID_ARG, "L_u[%d]=%d (need 0..%d)", r, L_u[r], TR_MAX_LU);
+    if (domain[r] < 0 || domain[r] >= m->desc.n_domains) return fail(TR_ERR_INVALID_ARG, "domain[%d]=%d", r, domain[r]);
+    if (L_u[r] > 0 && (!user_tokens[r] || !kv[r])) return fail(TR_ERR_INVALID_ARG, "request %d: null device pointer", r);
+    batch = batch && (L_u[r] == 0 || tc_prefill_supported(m, L_u[r]));
+  }
+  const cudaStream_t st = (cudaStream_t)stream;
+  if (batch) return tc_prefill_batch(m, user_tokens, L_u, domain, kv, R, st);
+  for (int r = 0; r < R; ++r)
+    if (L_u[r] > 0) TR_TRY(tr_prefill_user(m, user_tokens[r], L_u[r], domain[r], kv[r], stream));
+  return TR_OK;
+}
+
 tr_status tr_prefill_user_noalloc(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv,
                                   tr_stream stream) {
   TR_TRY(check_model_device(m));
@@ -358,7 +379,8 @@ tr_status tr_score_candidates_uncompressed(const tr_model* m, const void* tokens
   if (!tokens || !scores) return fail(TR_ERR_INVALID_ARG, "null device pointer");
   const cudaStream_t st = (cudaStream_t)stream;
   for (int r = 0; r < R; ++r)
-    TR_TRY(simt_score_lt(m, tokens, req_offsets[r], req_offsets[r + 1], L_t, kv[r], L_u[r], domain[r], scores, st));
+    TR_TRY(simt_score_lt(m, tokens, m->desc.dtype == TR_F32, req_offsets[r], req_offsets[r + 1], L_t, kv[r], L_u[r],
+                         domain[r], scores, st));
   return TR_OK;
 }
 

@@ -6,16 +6,20 @@
 //   layer 1: x tiles arrive by TMA tensor loads (128-byte swizzle, rows past the end are
 //            zero-filled by the copy engine) together with bulk copies of the matching
 //            W1 slice, two stages deep; the [128 x c1] fp32 accumulator fills TMEM.
-//   epilogue 1: + b1, PReLU, LayerNorm over c1 (two passes over TMEM), bf16 result written
+//   epilogue 1: + b1, PReLU, LayerNorm over c1 (two passes over TMEM), fp16 result written
 //            in the core-matrix layout over the now idle stage buffers.
-//   layers 2, 3: W2 / W3 slices stream through a second two-stage ring.
-//   epilogue 3: + b3, bf16 straight to global memory.
+//   layers 2, 3: W2 / W3 slices (fp16) stream through a second two-stage ring; the hidden
+//            activations and these weights are fp16 operands (x and W1 stay bf16, x's
+//            storage type), which rounds them 8x more finely than bf16 at the same rate.
+//   epilogue 3: + b3, fp32 tokens straight to global memory.
 // Warp 0 issues copies, warp 1 issues MMAs, warps 2-9 run the epilogues: two warps per TMEM
 // lane quadrant, each owning half of a row's columns; a row's LayerNorm statistics are merged
 // across the pair (Welford) through shared memory.  Waits are bounded as in the candidate
 // stack kernel.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <math.h>
 #include <string.h>
 
 #include <algorithm>
@@ -48,7 +52,7 @@ struct CompParams {
   const uint8_t* w2;           // [c1/64] slices of W2^T [c2 x 64]
   const uint8_t* w3;           // [c2/64] slices of W3^T [c3 x 64]
   const float* vec;            // b1 a1 g1 be1 (c1 each), b2 a2 g2 be2 (c2 each), b3 (c3)
-  __nv_bfloat16* out;          // [n][c3]
+  float* out;                  // [n][c3]
   int* status;
   long long n;
   int n_tiles, c0, c1, c2, c3;
@@ -64,6 +68,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
           dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+
+// fp16 x fp16 -> fp32, both operands K-major
+constexpr uint32_t idesc_f16c(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t pack_h2c(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 // K-major operand written by TMA with the 128-byte swizzle: 8-row atoms of 1024 bytes.
@@ -121,7 +135,8 @@ __device__ void comp_mma(const CompParams& p, uint32_t tmem, uint32_t r1, uint32
   uint32_t ph1 = 0, ph2 = 0, epi_phase = 0;
   bool ok = true;
   const int n1 = std::min(p.c1, 256);
-  const uint32_t id1 = idesc_bf16(kM, n1), id2 = idesc_bf16(kM, p.c2), id3 = idesc_bf16(kM, p.c3);
+  // layer 1 multiplies bf16 x by bf16 W1; layers 2 and 3 fp16 activations by fp16 weights
+  const uint32_t id1 = idesc_bf16(kM, n1), id2 = idesc_f16c(kM, p.c2), id3 = idesc_f16c(kM, p.c3);
   auto wait_epi = [&]() {
     ok = ok && mbar_wait(b.epi, epi_phase, abort_flag);
     epi_phase ^= 1;
@@ -211,7 +226,7 @@ __device__ __forceinline__ void vec8(const float* p, float* o) {
 }
 
 // + bias, PReLU, LayerNorm over the `cols` accumulator columns of this row, of which this
-// thread owns [c0, c0 + cols/2); bf16 result into the next layer's operand in R1.
+// thread owns [c0, c0 + cols/2); fp16 result into the next layer's operand in R1.
 __device__ __forceinline__ void prelu_ln_half(CEpi& e, int cols, const float* bias, const float* slope,
                                               const float* g, const float* be, uint32_t dst_row, int slot) {
   const int half = cols / 2, c0 = e.hf * half;
@@ -267,7 +282,8 @@ __device__ __forceinline__ void prelu_ln_half(CEpi& e, int cols, const float* bi
         x = x >= 0.f ? x : x * sl[i];
         w[i] = fmaf((x - mean) * rstd, gg[i], ee[i]);
       }
-      st_row8(dst_row + ((c0 + c) / 8 + k) * 2048, w);
+      st_shared_v4(dst_row + ((c0 + c) / 8 + k) * 2048, pack_h2c(w[0], w[1]), pack_h2c(w[2], w[3]),
+                   pack_h2c(w[4], w[5]), pack_h2c(w[6], w[7]));
     }
   }
 }
@@ -347,9 +363,9 @@ __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, c
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] += bb[i];
       if (row < p.n) {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + row * p.c3 + c);
-        dst[0] = make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]), pack2(v[6], v[7]));
-        dst[1] = make_uint4(pack2(v[8], v[9]), pack2(v[10], v[11]), pack2(v[12], v[13]), pack2(v[14], v[15]));
+        float4* dst = reinterpret_cast<float4*>(p.out + row * p.c3 + c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
       }
     }
     signal();
@@ -420,16 +436,40 @@ __global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant_
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, STATUS_KERNEL_TIMEOUT);
 }
 
-// W^T slice rows [0, N) x cols [k0, k0 + 64) of W [K][N] in the core-matrix layout.
-void put_slice(uint16_t* dst, const float* W, int N, int k0) {
+// W^T slice rows [0, N) x cols [k0, k0 + 64) of W [K][N] in the core-matrix layout, as bf16
+// (f16 = false) or fp16.
+void put_slice(uint16_t* dst, const float* W, int N, int k0, bool f16) {
   for (int n = 0; n < N; ++n)
     for (int k = 0; k < 64; ++k) {
       float f = W[(size_t)(k0 + k) * N + n];
-      uint32_t u;
-      memcpy(&u, &f, 4);
-      u = (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
-      dst[((size_t)(k / 8) * (N / 8) + n / 8) * 64 + (n % 8) * 8 + (k % 8)] = (uint16_t)u;
+      uint16_t h;
+      if (f16) {
+        const __half hv = __float2half_rn(f);
+        memcpy(&h, &hv, 2);
+      } else {
+        uint32_t u;
+        memcpy(&u, &f, 4);
+        h = (uint16_t)((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
+      }
+      dst[((size_t)(k / 8) * (N / 8) + n / 8) * 64 + (n % 8) * 8 + (k % 8)] = h;
     }
+}
+
+// Whether the fp16 operands of layers 2 and 3 stay far inside fp16's range: they are
+// LayerNorm outputs (|value| <= max|gain| sqrt(width) + max|shift|) and the weights.
+bool comp_fp16_safe(const tr_model_desc& d, const tr_model_weights* w) {
+  const int* c = d.comp_dims;
+  const double limit = 16384.0;
+  for (int i = 0; i < 2; ++i) {
+    double g = 0, b = 0, wm = 0;
+    for (int j = 0; j < c[i + 1]; ++j) {
+      g = std::max(g, (double)fabsf(w->comp_ln_g[i][j]));
+      b = std::max(b, (double)fabsf(w->comp_ln_b[i][j]));
+    }
+    for (size_t j = 0; j < (size_t)c[i + 1] * c[i + 2]; ++j) wm = std::max(wm, (double)fabsf(w->comp_W[i + 1][j]));
+    if (!(g * sqrt((double)c[i + 1]) + b < limit && wm < limit)) return false;
+  }
+  return true;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
@@ -458,12 +498,15 @@ tr_status tc_build_comp(tr_model* m, const tr_model_weights* w) {
   if (!(c[0] % 64 == 0 && c[1] % 64 == 0 && c[1] <= 512 && c[2] % 64 == 0 && c[2] <= 256 && c[3] % 32 == 0 &&
         c[3] <= 256))
     return TR_OK;
+  if (!comp_fp16_safe(m->desc, w)) return TR_OK;   // the CUDA-core path serves this model
   const size_t e1 = (size_t)c[0] * c[1], e2 = (size_t)c[1] * c[2], e3 = (size_t)c[2] * c[3];
   std::vector<uint16_t> img(e1 + e2 + e3);
-  for (int kc = 0; kc < c[0] / 64; ++kc) put_slice(img.data() + (size_t)kc * 64 * c[1], w->comp_W[0], c[1], 64 * kc);
-  for (int kc = 0; kc < c[1] / 64; ++kc) put_slice(img.data() + e1 + (size_t)kc * 64 * c[2], w->comp_W[1], c[2], 64 * kc);
+  for (int kc = 0; kc < c[0] / 64; ++kc)
+    put_slice(img.data() + (size_t)kc * 64 * c[1], w->comp_W[0], c[1], 64 * kc, false);
+  for (int kc = 0; kc < c[1] / 64; ++kc)
+    put_slice(img.data() + e1 + (size_t)kc * 64 * c[2], w->comp_W[1], c[2], 64 * kc, true);
   for (int kc = 0; kc < c[2] / 64; ++kc)
-    put_slice(img.data() + e1 + e2 + (size_t)kc * 64 * c[3], w->comp_W[2], c[3], 64 * kc);
+    put_slice(img.data() + e1 + e2 + (size_t)kc * 64 * c[3], w->comp_W[2], c[3], 64 * kc, true);
   std::vector<float> vec;
   for (int i = 0; i < 2; ++i) {
     const int n = c[i + 1];
@@ -508,7 +551,7 @@ tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens,
   p.w2 = img + (size_t)c[0] * c[1] * 2;
   p.w3 = p.w2 + (size_t)c[1] * c[2] * 2;
   p.vec = m->tc_comp_vec;
-  p.out = static_cast<__nv_bfloat16*>(tokens);
+  p.out = static_cast<float*>(tokens);
   p.status = ds->status;
   p.n = n;
   p.n_tiles = (int)((n + kM - 1) / kM);

@@ -41,9 +41,9 @@ tr_status simt_prefill(const tr_model* m, const float* user_tokens, int L_u, int
                        cudaStream_t st);
 tr_status simt_compress(const tr_model* m, const void* x, int64_t n, void* tokens, cudaStream_t st);
 tr_status simt_score(const tr_model* m, const void* tokens, int64_t c0, int64_t c1, const void* kv,
-                     int L_u, int domain, float* scores, cudaStream_t st);
-tr_status simt_score_lt(const tr_model* m, const void* tokens, int64_t c0, int64_t c1, int lt, const void* kv,
-                        int L_u, int domain, float* scores, cudaStream_t st);
+                     int L_u, int domain, float* scores, cudaStream_t st);   // fp32 tokens
+tr_status simt_score_lt(const tr_model* m, const void* tokens, bool tokens_f32, int64_t c0, int64_t c1, int lt,
+                        const void* kv, int L_u, int domain, float* scores, cudaStream_t st);
 tr_status launch_topk(const float* scores, const int64_t* req_offsets, int R, int k, int64_t* out_idx,
                       float* out_score, cudaStream_t st);
 tr_status launch_aggregate(const tr_table* tables, int n_tables, const int32_t* bag_table,

@@ -5,6 +5,8 @@
 // take.  Stages run as a short sequence of plain kernels over an fp32 workspace:
 // tiled GEMM with fused bias / ReLU / residual, row LayerNorm (optionally after PReLU),
 // one-warp-per-(row, head) attention.
+#include <cuda_fp16.h>
+
 #include <algorithm>
 #include <mutex>
 
@@ -133,15 +135,15 @@ struct KvF32 {
   __device__ float k(int j, int d) const { return K[(int64_t)j * ld + d]; }
   __device__ float v(int j, int d) const { return V[(int64_t)j * ld + d]; }
 };
-struct KvBf16Image {
-  const __nv_bfloat16* K;  // [Lp x D] core-matrix image
-  const __nv_bfloat16* V;  // [D x Lp] core-matrix image
+struct KvF16Image {
+  const __half* K;  // [Lp x D] core-matrix image
+  const __half* V;  // [D x Lp] core-matrix image
   int Lp, D;
   __device__ float k(int j, int d) const {
-    return __bfloat162float(K[((d >> 3) * (Lp >> 3) + (j >> 3)) * 64 + (j & 7) * 8 + (d & 7)]);
+    return __half2float(K[((d >> 3) * (Lp >> 3) + (j >> 3)) * 64 + (j & 7) * 8 + (d & 7)]);
   }
   __device__ float v(int j, int d) const {
-    return __bfloat162float(V[((j >> 3) * (D >> 3) + (d >> 3)) * 64 + (d & 7) * 8 + (j & 7)]);
+    return __half2float(V[((j >> 3) * (D >> 3) + (d >> 3)) * 64 + (d & 7) * 8 + (j & 7)]);
   }
 };
 
@@ -235,8 +237,7 @@ __global__ void kv_write_f32(const float* __restrict__ qkv, int L_u, int D, floa
   cache_l[i] = qkv[(int64_t)j * 3 * D + (1 + which) * D + d];
 }
 
-__global__ void kv_write_bf16(const float* __restrict__ qkv, int L_u, int Lp, int D,
-                              __nv_bfloat16* __restrict__ cache_l) {
+__global__ void kv_write_f16(const float* __restrict__ qkv, int L_u, int Lp, int D, __half* __restrict__ cache_l) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= 2 * Lp * D) return;
   const bool isv = i >= Lp * D;
@@ -251,7 +252,7 @@ __global__ void kv_write_bf16(const float* __restrict__ qkv, int L_u, int Lp, in
     d = (core % (D >> 3)) * 8 + (within >> 3);
   }
   const float v = (j < L_u) ? qkv[(int64_t)j * 3 * D + (isv ? 2 : 1) * D + d] : 0.f;
-  cache_l[i] = __float2bfloat16_rn(v);
+  cache_l[i] = __float2half_rn(v);
 }
 
 // score = w . LayerNorm_f(y) + b; one warp per row.
@@ -295,7 +296,7 @@ tr_status layer(const tr_model* m, int l, float* y, float* a, float* qkv, float*
       kv_write_f32<<<ceil_div(2 * M * D, 256), 256, 0, st>>>(qkv, M, D, (float*)kv_out);
     } else {
       const int Lp = round_up16(M);
-      kv_write_bf16<<<ceil_div(2 * Lp * D, 256), 256, 0, st>>>(qkv, M, Lp, D, (__nv_bfloat16*)kv_out);
+      kv_write_f16<<<ceil_div(2 * Lp * D, 256), 256, 0, st>>>(qkv, M, Lp, D, (__half*)kv_out);
     }
     TR_LAUNCH_CHECK("kv_write");
   }
@@ -328,7 +329,7 @@ tr_status simt_prefill(const tr_model* m, const float* user_tokens, int L_u, int
     if (m->desc.dtype == TR_F32)
       kv_l = (float*)kv + (size_t)l * 2 * L_u * D;
     else
-      kv_l = (__nv_bfloat16*)kv + (size_t)l * 2 * Lp * D;
+      kv_l = (__half*)kv + (size_t)l * 2 * Lp * D;
     // attention among the users reads their fp32 K/V straight from the qkv buffer
     KvF32 self_kv{qkv + D, qkv + 2 * D, 3 * D};
     TR_TRY(layer(m, l, y, a, qkv, o, hb, L_u, self_kv, L_u, 0, kv_l, st));
@@ -356,10 +357,7 @@ tr_status simt_compress(const tr_model* m, const void* x, int64_t n, void* token
     TR_TRY(layernorm<float>(h2, c[2], h2, c[2], M, c[2], m->comp_prelu[1], m->comp_ln_g[1], m->comp_ln_b[1], st));
     TR_TRY(gemm<float>(h2, c[2], m->comp_W[2], c[3], m->comp_b[2], t, c[3], M, c[3], c[2], EPI_NONE, st));
     const int64_t cnt = (int64_t)M * c[3];
-    if (m->desc.dtype == TR_F32)
-      convert_rows<float><<<ceil_div(cnt, 256), 256, 0, st>>>(t, (float*)tokens + r0 * c[3], cnt);
-    else
-      convert_rows<__nv_bfloat16><<<ceil_div(cnt, 256), 256, 0, st>>>(t, (__nv_bfloat16*)tokens + r0 * c[3], cnt);
+    convert_rows<float><<<ceil_div(cnt, 256), 256, 0, st>>>(t, (float*)tokens + r0 * c[3], cnt);
     TR_LAUNCH_CHECK("convert_rows");
   }
   return TR_OK;
@@ -378,8 +376,8 @@ __global__ void group_mean(const float* __restrict__ x, int64_t n, int lt, float
 // token runs through the layers attending to the request's users and to its own
 // candidate's lt tokens; the candidate's score is the mean of its tokens' head outputs
 // (for lt = 1 the plain single-token score).
-tr_status simt_score_lt(const tr_model* m, const void* tokens, int64_t c0, int64_t c1, int lt, const void* kv,
-                        int L_u, int domain, float* scores, cudaStream_t st) {
+tr_status simt_score_lt(const tr_model* m, const void* tokens, bool tokens_f32, int64_t c0, int64_t c1, int lt,
+                        const void* kv, int L_u, int domain, float* scores, cudaStream_t st) {
   const int D = m->desc.D, H = m->desc.ffn_hidden;
   const int64_t chunk = std::max<int64_t>(1, 16384 / lt);     // candidates per pass
   const int64_t n = c1 - c0;
@@ -394,7 +392,7 @@ tr_status simt_score_lt(const tr_model* m, const void* tokens, int64_t c0, int64
     const int64_t nc = std::min<int64_t>(chunk, c1 - q0);
     const int M = (int)(nc * lt);
     const int64_t r0 = q0 * lt, cnt = (int64_t)M * D;
-    if (m->desc.dtype == TR_F32)
+    if (tokens_f32)
       add_vec_rows<float><<<ceil_div(cnt, 256), 256, 0, st>>>((const float*)tokens + r0 * D, y, M, D,
                                                               m->domain_emb + (int64_t)domain * D);
     else
@@ -406,8 +404,8 @@ tr_status simt_score_lt(const tr_model* m, const void* tokens, int64_t c0, int64
         const float* base = (const float*)kv + (size_t)l * 2 * L_u * D;
         TR_TRY(layer(m, l, y, a, qkv, o, hb, M, KvF32{base, base + (size_t)L_u * D, D}, L_u, lt, nullptr, st));
       } else {
-        const __nv_bfloat16* base = (const __nv_bfloat16*)kv + (size_t)l * 2 * Lp * D;
-        TR_TRY(layer(m, l, y, a, qkv, o, hb, M, KvBf16Image{base, base + (size_t)Lp * D, Lp, D}, L_u, lt, nullptr,
+        const __half* base = (const __half*)kv + (size_t)l * 2 * Lp * D;
+        TR_TRY(layer(m, l, y, a, qkv, o, hb, M, KvF16Image{base, base + (size_t)Lp * D, Lp, D}, L_u, lt, nullptr,
                      st));
       }
     }
@@ -424,7 +422,7 @@ tr_status simt_score_lt(const tr_model* m, const void* tokens, int64_t c0, int64
 
 tr_status simt_score(const tr_model* m, const void* tokens, int64_t c0, int64_t c1, const void* kv, int L_u,
                      int domain, float* scores, cudaStream_t st) {
-  return simt_score_lt(m, tokens, c0, c1, 1, kv, L_u, domain, scores, st);
+  return simt_score_lt(m, tokens, true, c0, c1, 1, kv, L_u, domain, scores, st);
 }
 
 // ---------------------------------------------------------------- user side without allocation
@@ -469,7 +467,7 @@ tr_status simt_prefill_noalloc(const tr_model* m, const float* user_tokens, int 
     if (m->desc.dtype == TR_F32)
       kv_l = (float*)kv + (size_t)l * 2 * L_u * D;
     else
-      kv_l = (__nv_bfloat16*)kv + (size_t)l * 2 * Lp * D;
+      kv_l = (__half*)kv + (size_t)l * 2 * Lp * D;
     KvF32 self_kv{qkv + D, qkv + 2 * D, 3 * D};
     TR_TRY(layer(m, l, y, a, qkv, o, hb, L_u, self_kv, L_u, 0, kv_l, st));
   }

@@ -1,42 +1,46 @@
-// Fused candidate stack on tcgen05 tensor cores (TransRetrieval §3.3, deployment section
-// "Hardware-aware inference optimization").
+// Fused Transformer stack on tcgen05 tensor cores (TransRetrieval §3.3, §3.4, deployment
+// section "Hardware-aware inference optimization"), for D = 64 and D = 128 (d_h = 16, FFN
+// hidden 2D).  One kernel serves both sides of a request:
+//   score mode  candidate tiles: every row attends to its request's cached user K/V plus its
+//               own key/value; final LayerNorm and the linear head give the score;
+//   user mode   the request's user tokens as one tile, attending to each other; each layer's
+//               K/V images are written to the request's cache (one bulk store per layer).
 //
-// One persistent CTA per SM walks 128-candidate tiles; a tile never mixes requests, so
-// every row of a tile attends to the same user K/V (the paper's "expand" broadcast: the
-// request's cache is staged once per tile and layer, never replicated per candidate).
-// The whole N-layer stack runs with the tile on chip:
+// Two 128-row tiles ("slots") are in flight per CTA, so that one slot's LayerNorm, softmax
+// and hand-offs run while the tensor core works on the other slot's products.  Each slot
+// owns 256 TMEM columns, four epilogue warps (one thread per tile row, the whole row) and an
+// MMA-issuing thread; the two slots of a CTA take two consecutive tiles of one request (a
+// "unit") and share its K/V images and every weight item of the stream.
 //
-//   TMEM (512 fp32 columns x 128 lanes, lane = candidate row)
-//     [  0,128)  Y, the residual stream; the O and FFN2 GEMMs (and their biases)
-//                accumulate into it in place
-//     [128,256)  Q accumulator -> score buffer 0 (softmax numerators written over the scores
-//                as bf16, the A operand of P V) -> FFN hidden [0,128)
-//     [256,384)  K accumulator -> score buffer 1 (same) -> FFN hidden [128,256)
-//     [384,512)  V accumulator -> attention output O (the candidate's own V moves to
-//                registers as bf16 first) -> ReLU(hidden) as bf16, the A operand of W2
+//   TMEM (per slot, 256 fp32 columns, lane = tile row)
+//     [0, D)        Y, the residual stream; the O and FFN2 products (and their biases)
+//                   accumulate into it in place
+//     [D, D + 128)  work area W, in turn: own K, own V, Q (each read out by the epilogue),
+//                   the scores of one head group (numerators written back over them as
+//                   fp16, the A operand of P V, whose result lands beside them), the FFN
+//                   hidden units (a 128-wide half at a time; ReLU written back as fp16, the
+//                   A operand of W2)
 //   shared memory
-//     A      [128 x 128] bf16  LN1 output -> Q -> attention output -> LN2 output
-//     KV     the request's K and V^T images of the current layer (up to 64 KB)
-//     ring   3 x 36 KB: a [128 out x 128 in] weight block plus its [128 x 16] bias tile;
-//            streamed by the TMA engine in consumption order
+//     A      per slot [128 x D] fp16: LN1 output -> Q -> attention output -> LN2 output
+//     KV     the unit's K and V^T images of the current layer (score mode: loaded by bulk
+//            copy; user mode: written by the epilogue, then stored to the cache)
+//     ring   weight items in consumption order (K, V, Q, O, W1, W2 per layer), each
+//            consumed by both slots before its buffer is refilled
 //     ones   the [128 x 16] A operand that turns a bias tile into "+ bias" in one MMA
-//     vec    LayerNorm gains/shifts of every layer and the folded head weight (<= 5 layers)
+//     vec    LayerNorm gains/shifts of every layer and the folded head weight
 //
-// Attention runs per head group (the heads whose scores fit 128 TMEM columns).  The scores of
-// group g + 2 are computed into the buffer group g used, once group g's P V products have
-// completed, while the epilogue works on group g + 1.
+// Operands are fp16 (the weights are bf16 values, converted exactly; activations are
+// rounded to fp16, whose 11-bit significand keeps the error of the five-layer stack a few
+// times below that of bf16 operands at the same tensor-core rate); accumulation, LayerNorm
+// and softmax are fp32.  A model whose parameters could push an fp16 operand out of range
+// is not built for this kernel (it runs on the CUDA-core path).
 //
-// Biases: one extra K = 16 MMA per GEMM, ones[128 x 16] x bias_tile^T, where the bias tile
-// holds the bf16 head and tail of each fp32 bias (columns 0 and 1): D += b_hi + b_lo.
-//
-// Warp roles: warp 0 issues bulk copies, warp 1 issues tcgen05.mma from one thread (warps 2
-// and 3 only complete that warpgroup and hand their registers over), warps 4-11 are the
-// epilogue: two warps per TMEM lane quadrant, each owning half of the columns
-// (64 of D, i.e. four of the eight heads).  LayerNorm statistics of a row are merged across
-// the pair (Welford merge through shared memory, synchronised per quadrant); per-head
-// softmax needs no exchange unless a head's keys are split (L_u > 64).  Every wait is
-// bounded: a stalled barrier sets an error bit and the kernel unwinds, releasing its tensor
-// memory.
+// Warp roles: warp 0 streams weight items, warp 3 streams K/V images (and owns the TMEM
+// allocation), warps 1 and 2 issue the MMAs of slot 0 and slot 1, warps 4-7 and 8-11 are the
+// epilogues of slot 0 and slot 1.  Every epilogue/MMA hand-off of a slot is a strict
+// alternation on two mbarriers.  Every wait is bounded: a stalled barrier sets an error bit
+// and the kernel unwinds, releasing its tensor memory.
+#include <cuda_fp16.h>
 #include <math.h>
 #include <string.h>
 
@@ -55,803 +59,807 @@ namespace {
 
 using namespace tc;
 
-constexpr int kD = 128, kH = 256, kM = 128;
-constexpr int kChunk = 16384;                 // [128 out x 64 in] bf16 weight slice
-constexpr int kBiasTile = 4096;               // [128 x 16] bf16 bias tile
-// One stream item: a [128 out x 128 in] weight block (two slices) plus its bias tile.  On
-// B200 a bulk copy costs about the same time per copy from 16 to 64 KB (a few hundred
-// cycles each, copies of one SM largely serialised), so items are as large as the ring
-// allows.
-constexpr int kSlot = 2 * kChunk + kBiasTile;
-constexpr int kStages = 3;
-constexpr int kItemsPerLayer = 8;
-constexpr int kVecPerLayer = 4 * kD;          // LN1 gain, LN1 shift, LN2 gain, LN2 shift
-constexpr int kVecFinal = kD + 4;             // head weight * final LN gain, folded head bias
-constexpr int kMaxLpTc = 128;
-constexpr int kMaxLayersSmemVec = 5;
-constexpr int kEpiThreads = 256;
-// Warps 0-3 (one warpgroup): bulk-copy producer, MMA issuer, two idle warps; warps 4-11:
-// the epilogue.  The control warpgroup gives registers to the epilogue (setmaxnreg), so
-// the epilogue runs without spills: 4 x 32 x kCtlRegs + 8 x 32 x kEpiRegs <= 384 x 168.
-constexpr int kThreads = 128 + kEpiThreads;
-constexpr int kEpiThread0 = 128;
-constexpr int kCtlRegs = 104, kEpiRegs = 200;
+constexpr int kM = 128;
+constexpr int kSlotCols = 256;
+constexpr int kWork = 128;
+constexpr int kSlotThreads = 128;                    // epilogue threads per slot
+constexpr int kThreads = 128 + 2 * kSlotThreads;     // control warpgroup + two epilogue warpgroups
+constexpr int kCtlRegs = 56, kEpiRegs = 224;
 static_assert(4 * 32 * kCtlRegs + 8 * 32 * kEpiRegs <= kThreads * 168, "register split exceeds the launch");
-constexpr float kQScale = 0.25f * 1.44269504088896341f;  // 1/sqrt(d_h) * log2(e)
+constexpr int kMaxStages = 4;
+constexpr int kMaxLp = 128;
+constexpr float kL2E = 1.44269504088896341f;
+constexpr int kSmemLimit = 232448;
 
-// Items: Wq, Wk, Wv, Wo, W1 (output columns 0-127), W1 (128-255), W2 (input rows 0-127),
-// W2 (rows 128-255); every item but the first half of W2 carries its GEMM's bias tile.
-__host__ __device__ constexpr bool item_has_bias(int j) { return j != 6; }
+// fp16 x fp16 -> fp32, both operands K-major
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
 
-constexpr int OFF_A = 0;
-constexpr int OFF_KV = 32768;                               // 2 x L_p x 128 bf16, L_p <= 128
-constexpr int OFF_RING = 98304;
-constexpr int OFF_ONES = OFF_RING + kStages * kSlot;        // 204 KB
-constexpr int OFF_X = OFF_ONES + kM * 16 * 2;               // [2 slots][2 halves][128] float2
-constexpr int OFF_VEC = OFF_X + 2 * 2 * kM * 8;
-constexpr int OFF_BAR = OFF_VEC + (kMaxLayersSmemVec * kVecPerLayer + kVecFinal) * 4;
-constexpr int SMEM_BYTES = OFF_BAR + 320;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+// One GEMM of the weight stream: its B operand [N x K] (core-matrix layout, K-major) at
+// byte `off` of weight item `item`, and its [N x 16] bias tile at byte `bias` (-1: none).
+struct Piece {
+  int item, off, N, K, bias;
+};
+enum { P_K = 0, P_V = 1, P_Q = 2, P_O = 3, P_W1A = 4, P_W2A = 5, P_W1B = 6, P_W2B = 7 };
+
+template <int D>
+struct Cfg;
+// D = 128: one item per GEMM: K, V, Q, O, W1 (hidden 0-127), W2 (hidden 0-127, no bias),
+// W1 (hidden 128-255), W2 (hidden 128-255, + b2).  32 KB of weights + a 4 KB bias tile.
+template <>
+struct Cfg<128> {
+  static constexpr int kNH = 8, kItems = 8, kPieces = 8, kItemBytes = 36864, kFfnHalves = 2;
+  __host__ __device__ static constexpr Piece piece(int p) { return Piece{p, 0, 128, 128, p == P_W2A ? -1 : 32768}; }
+  __host__ __device__ static constexpr int item_bytes(int j) { return j == P_W2A ? 32768 : 36864; }
+};
+// D = 64: two items per layer: [K | V | Q | O] (8 KB + a 2 KB bias tile each) and
+// [W1 (N = 128) + bias | W2 (K = 128) + bias].
+template <>
+struct Cfg<64> {
+  static constexpr int kNH = 4, kItems = 2, kPieces = 6, kItemBytes = 40960, kFfnHalves = 1;
+  __host__ __device__ static constexpr Piece piece(int p) {
+    return p < 4 ? Piece{0, p * 10240, 64, 64, p * 10240 + 8192}
+                 : (p == P_W1A ? Piece{1, 0, 128, 64, 16384} : Piece{1, 20480, 64, 128, 36864});
+  }
+  __host__ __device__ static constexpr int item_bytes(int j) { return j == 0 ? 40960 : 38912; }
+};
+
+template <int D>
+constexpr int vec_per_layer() { return 4 * D; }   // LN1 gain, LN1 shift, LN2 gain, LN2 shift
+
+// Head groups of one launch: a head's scores take SW work-area columns (SW = 32, 64 or 128,
+// at least the launch's longest padded user sequence), a group is the HG heads that fit.
+template <int D, int SW>
+struct Groups {
+  static constexpr int HG = kWork / SW;
+  static constexpr int NG = Cfg<D>::kNH / HG;
+  static_assert(SW == 32 || SW == 64 || SW == 128, "head slot width");
+};
 
 struct ReqInfo {
-  const uint8_t* kv;
+  const uint8_t* kv;          // score mode: the request's K/V images; user mode: the cache to write
+  const float* utokens;       // user mode: fp32 user tokens [L_u][D]
   long long cand_off;
-  long long n;
-  int tile_off;
+  long long n;                // candidates (score mode) / user tokens (user mode)
+  int unit_off;
   int L_u;
   int domain;
   int pad;
 };
 
 struct StackParams {
-  const __nv_bfloat16* tokens;
+  const float* tokens;        // score mode: fp32 candidate tokens [n][D]
   float* scores;
-  const uint8_t* wimg;       // [n_layer][kItemsPerLayer][kSlot]
-  const float* vec;          // [n_layer][kVecPerLayer] + [kVecFinal]
-  const float* domain_emb;   // [n_domains][D]
+  const uint8_t* wimg;        // [n_layer][kItems][kItemBytes]
+  const float* vec;           // [n_layer][4 D] + [D + 4]
+  const float* domain_emb;    // fp32 [n_domains][D]
   int* status;
-  int n_layer;
-  int n_tiles;
-  int R;
-  const float* utokens;      // user-side mode: fp32 user tokens [L_u][D]
-  uint8_t* kv_out;           // user-side mode: the request's K/V cache
+  int n_layer, n_units, R, pair;
+  int off_kv, off_ring, off_ones, off_vec, off_bar, stages;
   ReqInfo req[TR_MAX_REQUESTS];
 };
 
-struct TileInfo {
-  int r, rows, L_u, Lp, hg, ng;
+struct Tile {
+  bool active;
+  int r, rows, L_u, Lp, dom;
   long long row0;
 };
 
-__device__ __forceinline__ TileInfo tile_info(const StackParams& p, int tile) {
+template <int D>
+__device__ __forceinline__ Tile tile_of(const StackParams& p, int u, int slot) {
   int r = 0;
-  while (r + 1 < p.R && tile >= p.req[r + 1].tile_off) ++r;
-  TileInfo t;
+  while (r + 1 < p.R && u >= p.req[r + 1].unit_off) ++r;
+  Tile t;
   t.r = r;
-  t.row0 = p.req[r].cand_off + (long long)(tile - p.req[r].tile_off) * kM;
-  t.rows = (int)min((long long)kM, p.req[r].cand_off + p.req[r].n - t.row0);
+  const long long local = (long long)(u - p.req[r].unit_off) * (p.pair ? 2 : 1) + slot;
+  t.row0 = p.req[r].cand_off + local * kM;
+  const long long end = p.req[r].cand_off + p.req[r].n;
+  t.active = (slot == 0 || p.pair) && t.row0 < end;
+  t.rows = t.active ? (int)min((long long)kM, end - t.row0) : 0;
   t.L_u = p.req[r].L_u;
   t.Lp = (t.L_u + 15) & ~15;
-  // heads per score group: a group's scores fill at most 128 TMEM columns
-  t.hg = t.Lp <= 16 ? 8 : t.Lp <= 32 ? 4 : t.Lp <= 64 ? 2 : 1;
-  t.ng = t.Lp == 0 ? 0 : 8 / t.hg;
+  t.dom = p.req[r].domain;
   return t;
 }
 
-// Slot s of head group g holds this head.  The first half of a group's slots are heads of
-// the first column half (0-3), the second half heads 4-7, so both epilogue halves get work.
-__device__ __forceinline__ int slot_head(int g, int s, int hg) {
-  if (hg == 1) return g;
-  const int half = hg / 2;
-  return s < half ? g * half + s : 4 + g * half + (s - half);
-}
-
-// The CTA's mbarriers, 8 bytes apart from one base address (offsets are compile-time, so
-// the issuing threads hold one register for all of them).
+// The CTA's mbarriers, 8 bytes apart.
 struct Bars {
   uint32_t base;
   __device__ __forceinline__ uint32_t at(int i) const { return base + 8u * (uint32_t)i; }
   __device__ __forceinline__ uint32_t full(int s) const { return at(s); }
-  __device__ __forceinline__ uint32_t empty(int s) const { return at(kStages + s); }
-  __device__ __forceinline__ uint32_t kv_full() const { return at(2 * kStages); }
-  __device__ __forceinline__ uint32_t kv_empty() const { return at(2 * kStages + 1); }
-  // MMA -> epilogue
-  __device__ __forceinline__ uint32_t ev_qk() const { return at(2 * kStages + 2); }
-  __device__ __forceinline__ uint32_t ev_s(int i) const { return at(2 * kStages + 3 + i); }
-  __device__ __forceinline__ uint32_t ev_av() const { return at(2 * kStages + 5); }
-  __device__ __forceinline__ uint32_t ev_o() const { return at(2 * kStages + 6); }
-  __device__ __forceinline__ uint32_t ev_h0() const { return at(2 * kStages + 7); }
-  __device__ __forceinline__ uint32_t ev_h1() const { return at(2 * kStages + 8); }
-  __device__ __forceinline__ uint32_t ev_y() const { return at(2 * kStages + 9); }
-  // epilogue -> MMA
-  __device__ __forceinline__ uint32_t e1() const { return at(2 * kStages + 10); }
-  __device__ __forceinline__ uint32_t e2() const { return at(2 * kStages + 11); }
-  __device__ __forceinline__ uint32_t e3(int i) const { return at(2 * kStages + 12 + i); }
-  __device__ __forceinline__ uint32_t e4() const { return at(2 * kStages + 14); }
-  __device__ __forceinline__ uint32_t e5() const { return at(2 * kStages + 15); }
-  __device__ __forceinline__ uint32_t e6a() const { return at(2 * kStages + 16); }
-  __device__ __forceinline__ uint32_t e6b() const { return at(2 * kStages + 17); }
-  __device__ __forceinline__ uint32_t drain() const { return at(2 * kStages + 18); }
-  __device__ __forceinline__ uint32_t esync() const { return at(2 * kStages + 19); }
-  __device__ __forceinline__ uint32_t qsync(int q) const { return at(2 * kStages + 20 + q); }
-  // MMA -> MMA: the P V products that read score buffer i have completed
-  __device__ __forceinline__ uint32_t av_done(int i) const { return at(2 * kStages + 24 + i); }
+  __device__ __forceinline__ uint32_t empty(int s) const { return at(kMaxStages + s); }
+  __device__ __forceinline__ uint32_t kv_full() const { return at(2 * kMaxStages); }
+  __device__ __forceinline__ uint32_t kv_empty(int slot) const { return at(2 * kMaxStages + 1 + slot); }
+  __device__ __forceinline__ uint32_t e2m(int slot) const { return at(2 * kMaxStages + 3 + slot); }
+  __device__ __forceinline__ uint32_t m2e(int slot) const { return at(2 * kMaxStages + 5 + slot); }
+  __device__ __forceinline__ uint32_t mm(int slot) const { return at(2 * kMaxStages + 7 + slot); }
+  __device__ __forceinline__ uint32_t drain(int slot) const { return at(2 * kMaxStages + 9 + slot); }
 };
-constexpr int kNumBars = 2 * kStages + 26;
-constexpr int kBarBytes = 8 * kNumBars;
-static_assert(kBarBytes + 16 <= 320, "barrier area");
+constexpr int kNumBars = 2 * kMaxStages + 11;
+constexpr int kBarArea = 8 * kNumBars + 32;   // + TMEM address and abort flag
 
-// ------------------------------------------------------------------ producer (warp 0, one thread)
-template <bool PF>
-__device__ void producer(const StackParams& p, uint32_t ring, uint32_t kvbuf, const Bars& b,
-                         volatile int* abort_flag) {
+// ------------------------------------------------------------------ small helpers
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float h_lo(uint32_t w) { return __low2float(*reinterpret_cast<const __half2*>(&w)); }
+__device__ __forceinline__ float h_hi(uint32_t w) { return __high2float(*reinterpret_cast<const __half2*>(&w)); }
+// eight fp32 values -> one 16-byte row of a core matrix (fp16)
+__device__ __forceinline__ void st_row8h(uint32_t addr, const float* v) {
+  st_shared_v4(addr, pack_h2(v[0], v[1]), pack_h2(v[2], v[3]), pack_h2(v[4], v[5]), pack_h2(v[6], v[7]));
+}
+__device__ __forceinline__ void ld8(const float* p, float* o) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  tmem_ld16(taddr, v);
+  tmem_ld16(taddr + 16, v + 16);
+}
+__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+// Compiler-only barrier: keeps later loads from being hoisted above it.
+__device__ __forceinline__ void step_barrier() { asm volatile("" ::: "memory"); }
+
+// Bounded wait of one thread for its own bulk copies in flight, used while unwinding.
+__device__ __forceinline__ void settle(uint32_t bar, uint32_t parity) {
+  for (uint64_t t0 = globaltimer_ns(); !mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < 200000000ull;) {
+  }
+}
+
+// ------------------------------------------------------------------ producers
+// Weight items in consumption order, for every unit and layer of this CTA (warp 0, one thread).
+template <int D>
+__device__ void weight_producer(const StackParams& p, uint32_t ring, const Bars& b, volatile int* abort_flag) {
+  using C = Cfg<D>;
   int stage = 0;
-  uint32_t phase = 0, kv_phase = 0;
-  uint32_t pending = 0, pend_parity = 0;       // bit s: slot s has a copy in flight / its parity
-  bool kv_pending = false;
-  uint32_t kv_pend_parity = 0;
+  uint32_t phase = 0, pending = 0, pend_par = 0;
   bool ok = true;
-  for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-    const TileInfo t = tile_info(p, tile);
-    for (int l = 0; l < p.n_layer && ok; ++l) {
-      const uint8_t* wl = p.wimg + (size_t)l * kItemsPerLayer * kSlot;
-      for (int j = 0; j < kItemsPerLayer && ok; ++j) {
-        if (!PF && j == 3) {  // the request's K/V images go in between the QKV and O weights
-          if (!(ok = mbar_wait(b.kv_empty(), kv_phase ^ 1, abort_flag))) break;
-          const uint32_t bytes = 2u * t.Lp * kD * 2u;
-          if (bytes) {
-            mbar_arrive_expect_tx(b.kv_full(), bytes);
-            bulk_g2s(kvbuf, p.req[t.r].kv + (size_t)l * bytes, bytes, b.kv_full());
-            kv_pending = true;
-            kv_pend_parity = kv_phase;
-          } else {
-            mbar_arrive(b.kv_full());
-          }
-          kv_phase ^= 1;
-        }
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x)
+    for (int l = 0; l < p.n_layer && ok; ++l)
+      for (int j = 0; j < C::kItems && ok; ++j) {
         if (!(ok = mbar_wait(b.empty(stage), phase ^ 1, abort_flag))) break;
-        const uint32_t bytes = item_has_bias(j) ? kSlot : 2 * kChunk;
+        const uint32_t bytes = C::item_bytes(j);
         mbar_arrive_expect_tx(b.full(stage), bytes);
-        bulk_g2s(ring + stage * kSlot, wl + (size_t)j * kSlot, bytes, b.full(stage));
+        bulk_g2s(ring + stage * C::kItemBytes, p.wimg + ((size_t)l * C::kItems + j) * C::kItemBytes, bytes,
+                 b.full(stage));
         pending |= 1u << stage;
-        pend_parity = (pend_parity & ~(1u << stage)) | (phase << stage);
-        if (++stage == kStages) {
+        pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == p.stages) {
           stage = 0;
           phase ^= 1;
         }
       }
-    }
-  }
-  if (!ok) {  // unwinding: let the copies already issued land before the CTA exits
-    for (int s = 0; s < kStages; ++s)
-      if ((pending >> s) & 1u)
-        for (uint64_t t0 = globaltimer_ns();
-             !mbar_try_wait(b.full(s), (pend_parity >> s) & 1u) && globaltimer_ns() - t0 < 200000000ull;) {
-        }
-    if (kv_pending)
-      for (uint64_t t0 = globaltimer_ns();
-           !mbar_try_wait(b.kv_full(), kv_pend_parity) && globaltimer_ns() - t0 < 200000000ull;) {
-      }
-  }
+  if (!ok)
+    for (int s = 0; s < p.stages; ++s)
+      if ((pending >> s) & 1u) settle(b.full(s), (pend_par >> s) & 1u);
 }
 
-// ------------------------------------------------------------------ MMA issuer (warp 1, one thread)
-template <bool PF, int HG>
-__device__ void mma_issuer(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sKV, uint32_t ring,
+// The unit's K/V images of each layer (score mode; warp 3, one thread).  A layer's images are
+// loaded once every active slot has finished the previous layer's attention.
+template <int D>
+__device__ void kv_producer(const StackParams& p, uint32_t sKV, const Bars& b, volatile int* abort_flag) {
+  uint32_t ph0 = 0, ph1 = 0;
+  bool ok = true, pending = false;
+  uint32_t pend_par = 0, kv_phase = 0;
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    const Tile t0 = tile_of<D>(p, u, 0), t1 = tile_of<D>(p, u, 1);
+    const uint32_t bytes = 2u * t0.Lp * D * 2u;
+    for (int l = 0; l < p.n_layer && ok; ++l) {
+      if (!(ok = mbar_wait(b.kv_empty(0), ph0 ^ 1, abort_flag))) break;
+      ph0 ^= 1;
+      if (t1.active) {
+        if (!(ok = mbar_wait(b.kv_empty(1), ph1 ^ 1, abort_flag))) break;
+        ph1 ^= 1;
+      }
+      if (bytes) {
+        mbar_arrive_expect_tx(b.kv_full(), bytes);
+        bulk_g2s(sKV, p.req[t0.r].kv + (size_t)l * bytes, bytes, b.kv_full());
+        pending = true;
+        pend_par = kv_phase;
+      } else {
+        mbar_arrive(b.kv_full());
+      }
+      kv_phase ^= 1;
+    }
+  }
+  if (!ok && pending) settle(b.kv_full(), pend_par);
+}
+
+// ------------------------------------------------------------------ MMA issuer (one thread per slot)
+template <int D, int SW, bool UM>
+__device__ void mma_issuer(const StackParams& p, int slot, uint32_t tmem, uint32_t sA, uint32_t sKV, uint32_t ring,
                            uint32_t sOnes, const Bars& b, volatile int* abort_flag) {
-  constexpr uint32_t ID128 = idesc_bf16(kM, 128);
-  constexpr uint32_t ID16 = idesc_bf16(kM, 16);
+  using C = Cfg<D>;
+  constexpr uint32_t ID16 = idesc_f16(kM, 16);
+  const uint32_t tY = tmem + kSlotCols * slot, tW = tY + D;
+  const uint32_t e2m = b.e2m(slot), m2e = b.m2e(slot);
   int stage = 0;
-  uint32_t phase = 0, kv_phase = 0;
-  uint32_t ph1 = 0, ph2 = 0, ph3a = 0, ph3b = 0, ph4 = 0, ph5 = 0, ph6a = 0, ph6b = 0;
-  uint32_t av_pend = 0, av_ph = 0;   // bit i: a P V commit on buffer i not yet waited for / its parity
-  bool ok = true;
-  auto wait_epi = [&](uint32_t bar, uint32_t& ph) {
-    ok = ok && mbar_wait(bar, ph, abort_flag);
-    ph ^= 1;
+  uint32_t phase = 0, ph_e = 0, ph_kv = 0, ph_mm = 0;
+  bool ok = true, store_pending = false;
+  auto wait_e = [&]() {
+    ok = ok && mbar_wait(e2m, ph_e, abort_flag);
+    ph_e ^= 1;
     tc_fence_after();
     return ok;
   };
-  // weight block j against the 128-wide K of operand A (shared memory at a_base, or tensor
-  // memory columns a_col .. a_col + 63 when A_TMEM); the block's bias tile, if any, last
-  auto item = [&](int j, uint32_t a_base, uint32_t dcol, bool acc_first, bool a_tmem) {
-    if (!ok) return;
-    if (!(ok = mbar_wait(b.full(stage), phase, abort_flag))) return;
-    tc_fence_after();
-    const uint32_t w = ring + stage * kSlot;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t acc = (kk > 0 || acc_first) ? 1u : 0u;
-      if (a_tmem)
-        mma_bf16_ta(tmem + dcol, tmem + a_base + kk * 8, sdesc(w + kk * 4096, 2048, 128), ID128, acc);
-      else
-        mma_bf16(tmem + dcol, sdesc(a_base + kk * 4096, 2048, 128), sdesc(w + kk * 4096, 2048, 128), ID128, acc);
-    }
-    if (item_has_bias(j)) mma_bf16(tmem + dcol, sdesc(sOnes, 2048, 128), sdesc(w + 2 * kChunk, 2048, 128), ID128, 1u);
-    mma_commit(b.empty(stage));
-    if (++stage == kStages) {
+  auto advance = [&]() {
+    if (++stage == p.stages) {
       stage = 0;
       phase ^= 1;
     }
   };
-  for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-    const TileInfo t = tile_info(p, tile);
-    const uint32_t idS = idesc_bf16(kM, t.Lp > 0 ? t.Lp : 16);
-    // P V of the last group that used a score buffer must be complete before new scores
-    // overwrite its numerators
-    auto av_wait = [&](int buf) {
-      if (!((av_pend >> buf) & 1u)) return;
-      ok = ok && mbar_wait(b.av_done(buf), (av_ph >> buf) & 1u, abort_flag);
-      av_ph ^= 1u << buf;
-      av_pend &= ~(1u << buf);
+  // D[dcol..] (+)= A x B^T (+ bias) for weight piece pi; A in shared memory (a = operand
+  // base) or, for the FFN's second product, in tensor memory (a = column)
+  auto piece = [&](int pi, uint32_t dcol, bool acc, bool a_tmem, uint32_t a) {
+    const Piece pc = C::piece(pi);
+    const bool first = pi == 0 || C::piece(pi - 1).item != pc.item;
+    const bool last = pi == C::kPieces - 1 || C::piece(pi + 1).item != pc.item;
+    if (!ok) return;
+    if (first) {
+      if (!(ok = mbar_wait(b.full(stage), phase, abort_flag))) return;
       tc_fence_after();
-    };
-    // scores of head group g into TMEM buffer g % 2
-    auto issue_S = [&](int g) {
-      const int buf = g & 1;
-      av_wait(buf);
-      if (!ok) return;
-      for (int s = 0; s < HG; ++s) {
-        const int h = slot_head(g, s, HG);
-        mma_bf16(tmem + 128 + 128 * buf + s * t.Lp, sdesc(sA + h * 4096, 2048, 128),
-                 sdesc(sKV + 2 * h * (t.Lp / 8) * 128, (t.Lp / 8) * 128, 128), idS, 0u);
+    }
+    const uint32_t item = ring + stage * C::kItemBytes;
+    const uint32_t id = idesc_f16(kM, pc.N);
+#pragma unroll 1
+    for (int kk = 0; kk < pc.K / 16; ++kk) {
+      const uint64_t bd = sdesc(item + pc.off + kk * pc.N * 32, pc.N * 16, 128);
+      const uint32_t accf = (kk > 0 || acc) ? 1u : 0u;
+      if (a_tmem)
+        mma_bf16_ta(dcol, a + kk * 8, bd, id, accf);
+      else
+        mma_bf16(dcol, sdesc(a + kk * 4096, 2048, 128), bd, id, accf);
+    }
+    if (pc.bias >= 0) mma_bf16(dcol, sdesc(sOnes, 2048, 128), sdesc(item + pc.bias, pc.N * 16, 128), id, 1u);
+    if (last) {
+      mma_commit(b.empty(stage));
+      advance();
+    }
+  };
+  for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+    const Tile t = tile_of<D>(p, u, slot);
+    if (!t.active) {
+      // the other slot works alone on this unit: release its weight items as they arrive
+      for (int l = 0; l < p.n_layer && ok; ++l) {
+        for (int j = 0; j < C::kItems && ok; ++j) {
+          if (!(ok = mbar_wait(b.full(stage), phase, abort_flag))) break;
+          mbar_arrive(b.empty(stage));
+          advance();
+        }
+        ph_kv ^= 1;
       }
-      mma_commit(b.ev_s(buf));
-    };
-    // O[:, head] += P_head V_head for the heads of group g; P is read from tensor memory
-    // (slot s's numerators over the first half of its score columns)
-    auto issue_AV = [&](int g) {
-      const int buf = g & 1;
-      for (int s = 0; s < HG; ++s) {
-        const int h = slot_head(g, s, HG);
-        const uint32_t pcol = 128 + 128 * buf + s * t.Lp;
-        const uint32_t vb = sKV + t.Lp * 256;
-        for (int kk = 0; kk < t.Lp / 16; ++kk)
-          mma_bf16_ta(tmem + 384 + 16 * h, tmem + pcol + kk * 8, sdesc(vb + (32 * kk + 2 * h) * 128, 2048, 128),
-                      ID16, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(b.av_done(buf));
-      av_pend |= 1u << buf;
-    };
+      continue;
+    }
+    const uint32_t idS = idesc_f16(kM, t.Lp > 0 ? t.Lp : 16);
+    const uint32_t vimg = sKV + (uint32_t)t.Lp * D * 2;
     for (int l = 0; l < p.n_layer && ok; ++l) {
       // opaque per layer: keeps descriptor arithmetic from being hoisted into registers
-      asm volatile("" : "+r"(sA), "+r"(sKV), "+r"(ring), "+r"(sOnes), "+r"(tmem));
-      if (!wait_epi(b.e1(), ph1)) break;                // A = LN1(y)
-      item(0, sA, 128, false, false);                 // Q + bq
-      item(1, sA, 256, false, false);                 // own K + bk
-      item(2, sA, 384, false, false);                 // own V + bv
-      mma_commit(b.ev_qk());
-      if (!wait_epi(b.e2(), ph2)) break;                // A = Q (scaled); own V in registers
-      if (!PF) {
-        ok = ok && mbar_wait(b.kv_full(), kv_phase, abort_flag);
-        kv_phase ^= 1;
+      asm volatile("" : "+r"(sA), "+r"(sKV), "+r"(ring), "+r"(sOnes));
+      if (!wait_e()) break;                            // A = LN1(y)
+      piece(P_K, tW, false, false, sA);
+      if (UM && store_pending) {                       // the last layer's images have left shared memory
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        store_pending = false;
+      }
+      mma_commit(m2e);
+      if (!wait_e()) break;                            // own K read (user mode: K image written)
+      piece(P_V, tW, false, false, sA);
+      mma_commit(m2e);
+      if (!wait_e()) break;                            // own V read (user mode: V image written)
+      piece(P_Q, tW, false, false, sA);
+      mma_commit(m2e);
+      if (!wait_e()) break;                            // A = Q (score mode without users: attention output)
+      if constexpr (UM) {
+        const uint32_t bytes = 2u * t.Lp * D * 2u;
+        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                         p.req[t.r].kv + (size_t)l * bytes),
+                     "r"(sKV), "r"(bytes)
+                     : "memory");
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        store_pending = true;
+      } else {
+        ok = ok && mbar_wait(b.kv_full(), ph_kv, abort_flag);
+        ph_kv ^= 1;
         tc_fence_after();
       }
-      if (ok && t.ng > 0) issue_S(0);
-      if (ok && HG >= 2 && t.ng > 1) issue_S(1);
-      if constexpr (HG >= 2) {
-        // rounds of gpr groups (the epilogue's GPR); two score buffers are in flight, so
-        // after round g0 the scores of groups g0 + 2 .. g0 + 1 + gpr are issued
-        constexpr int gpr = 1;
-        for (int g0 = 0; g0 < t.ng && ok; g0 += gpr) {
-          const bool odd = (g0 / gpr) & 1;
-          if (!(odd ? wait_epi(b.e3(1), ph3b) : wait_epi(b.e3(0), ph3a))) break;   // round's numerators written
-          for (int gi = 0; gi < gpr; ++gi) issue_AV(g0 + gi);
-          for (int gi = 0; gi < gpr; ++gi)
-            if (g0 + 2 + gi < t.ng) issue_S(g0 + 2 + gi);
+      constexpr int HG = Groups<D, SW>::HG;
+      const int ng = t.Lp > 0 ? Groups<D, SW>::NG : 0;
+      for (int g = 0; g < ng && ok; ++g) {
+        for (int i = 0; i < HG; ++i) {                 // scores of the group's heads
+          const int h = g * HG + i;
+          mma_bf16(tW + i * SW, sdesc(sA + h * 4096, 2048, 128),
+                   sdesc(sKV + 2 * h * (t.Lp / 8) * 128, (t.Lp / 8) * 128, 128), idS, 0u);
         }
-      } else {
-        for (int g = 0; g < t.ng && ok; ++g) {
-          if (!((g & 1) ? wait_epi(b.e3(1), ph3b) : wait_epi(b.e3(0), ph3a))) break;   // P of group g written
-          issue_AV(g);
-          // group g + 1 goes to the other score buffer once the P V that last read it is done
-          if (g + 1 < t.ng) issue_S(g + 1);
+        mma_commit(m2e);
+        if (!wait_e()) break;                          // numerators written
+        for (int i = 0; i < HG; ++i) {                 // P V beside each head's numerators
+          const int h = g * HG + i;
+          const uint32_t pc = tW + i * SW;
+          for (int kk = 0; kk < t.Lp / 16; ++kk)
+            mma_bf16_ta(pc + SW / 2, pc + kk * 8, sdesc(vimg + (2 * kk * (D / 8) + 2 * h) * 128, (D / 8) * 128, 128),
+                        ID16, kk > 0 ? 1u : 0u);
         }
+        if (!UM && g == ng - 1) mma_commit(b.kv_empty(slot));
+        mma_commit(m2e);
+        if (!wait_e()) break;                          // attention output of the group in A
       }
-      av_wait(0);
-      av_wait(1);
       if (!ok) break;
-      if (!PF) mma_commit(b.kv_empty());
-      mma_commit(b.ev_av());
-      if (!wait_epi(b.e4(), ph4)) break;                // A = attention output
-      item(3, sA, 0, true, false);                    // Y += attn Wo + bo
-      mma_commit(b.ev_o());
-      if (!wait_epi(b.e5(), ph5)) break;                // A = LN2(y)
-      item(4, sA, 128, false, false);                 // hidden[0,128) + b1
-      mma_commit(b.ev_h0());
-      item(5, sA, 256, false, false);                 // hidden[128,256) + b1
-      mma_commit(b.ev_h1());
-      if (!wait_epi(b.e6a(), ph6a)) break;              // TMEM [384,448) = ReLU(hidden[0,128))
-      item(6, 384, 0, true, true);                    // Y += H W2, first half of K
-      if (!wait_epi(b.e6b(), ph6b)) break;              // TMEM [448,512) = ReLU(hidden[128,256))
-      item(7, 448, 0, true, true);                    // second half of K, + b2
-      mma_commit(b.ev_y());
+      if (!UM && ng == 0) mbar_arrive(b.kv_empty(slot));   // no product read the images
+      piece(P_O, tY, true, false, sA);                // Y += attn Wo + bo
+      mma_commit(m2e);
+      if (!wait_e()) break;                            // A = LN2(y)
+      piece(P_W1A, tW, false, false, sA);              // hidden (first half) + b1
+      mma_commit(m2e);
+      if (!wait_e()) break;                            // ReLU as fp16 in W[0, 64)
+      piece(P_W2A, tY, true, true, tW);                // Y += relu W2 (first half of K)
+      if constexpr (C::kFfnHalves == 2) {
+        // the second half of the hidden units overwrites W: the first W2 product must be done
+        mma_commit(b.mm(slot));
+        ok = ok && mbar_wait(b.mm(slot), ph_mm, abort_flag);
+        ph_mm ^= 1;
+        tc_fence_after();
+        piece(P_W1B, tW, false, false, sA);
+        mma_commit(m2e);
+        if (!wait_e()) break;
+        piece(P_W2B, tY, true, true, tW);              // + b2
+      }
+      mma_commit(m2e);
     }
   }
+  if (UM && store_pending) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   // drain every MMA still in flight before the tensor memory is released
-  mma_commit(b.drain());
-  for (uint64_t t0 = globaltimer_ns(); !mbar_try_wait(b.drain(), 0) && globaltimer_ns() - t0 < 500000000ull;) {
+  mma_commit(b.drain(slot));
+  for (uint64_t t0 = globaltimer_ns(); !mbar_try_wait(b.drain(slot), 0) && globaltimer_ns() - t0 < 500000000ull;) {
   }
 }
 
-// ------------------------------------------------------------------ epilogue (warps 2-9)
+// ------------------------------------------------------------------ epilogue (one thread per row)
 struct Epi {
-  uint32_t trow;        // TMEM address of this row, column 0
-  uint32_t rowoff;      // byte offset of this row inside a 128-row core-matrix operand
-  int m, hf, q;         // row, column half (0: columns 0-63 / heads 0-3), lane quadrant
-  uint32_t sA, sKV, sX;
-  const float* vec;     // LayerNorm vectors (shared memory copy when it fits)
-  Bars b;
+  uint32_t tY, tW;            // TMEM address of this row: residual, work area
+  uint32_t sA, rowoff, sKV;
+  int m;
+  uint32_t e2m, m2e, ph;
+  const float* vec;
   volatile int* abort_flag;
   bool ok;
-  uint32_t ph_qk, ph_s[2], ph_av, ph_o, ph_h0, ph_h1, ph_y, ph_sync, ph_q;
-
-  __device__ bool wait(uint32_t bar, uint32_t& ph) {
-    ok = ok && mbar_wait(bar, ph, abort_flag);
+  __device__ __forceinline__ bool wait() {
+    ok = ok && mbar_wait(m2e, ph, abort_flag);
     ph ^= 1;
     tc_fence_after();
     return ok;
   }
-  __device__ void signal(uint32_t bar) {
+  __device__ __forceinline__ void signal() {
     tmem_wait_st();
     fence_proxy_async_smem();
     tc_fence_before();
-    mbar_arrive(bar);
-  }
-  // rendezvous of the 256 epilogue threads (bounded)
-  __device__ bool sync() {
-    mbar_arrive(b.esync());
-    ok = ok && mbar_wait(b.esync(), ph_sync, abort_flag);
-    ph_sync ^= 1;
-    return ok;
-  }
-  // exchange one float2 with the other column half of this row through exchange slot
-  // `slot`; consecutive exchanges inside one phase must alternate slots
-  __device__ float2 swap(float2 mine, int slot) {
-    const uint32_t x = sX + slot * (2 * kM * 8);
-    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(x + (hf * kM + m) * 8), "f"(mine.x), "f"(mine.y)
-                 : "memory");
-    mbar_arrive(b.qsync(q));
-    ok = ok && mbar_wait(b.qsync(q), ph_q, abort_flag);
-    ph_q ^= 1;
-    float2 o;
-    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(o.x), "=f"(o.y) : "r"(x + ((1 - hf) * kM + m) * 8)
-                 : "memory");
-    return o;
+    mbar_arrive(e2m);
   }
 };
 
-// Compiler-only barrier: keeps the loads of the next step from being hoisted above it, so
-// that per-column vectors are not all held in registers at once.
-__device__ __forceinline__ void step_barrier() { asm volatile("" ::: "memory"); }
-
-__device__ __forceinline__ void load64(uint32_t taddr, float* v) {
+template <int D>
+__device__ __forceinline__ void load_row(uint32_t taddr, float* y) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) tmem_ld16(taddr + c * 16, v + c * 16);
+  for (int c = 0; c < D / 32; ++c) tmem_ld32(taddr + 32 * c, y + 32 * c);
   tmem_wait_ld();
-  reg_fence<64>(v);
+  reg_fence<D>(y);
 }
 
-// Row mean / rstd of a 128-wide row held as two 64-column halves (Welford merge).
-__device__ __forceinline__ float2 row_stats(Epi& e, const float* y) {
-  // four independent partial sums per pass: short dependency chains
+// Row mean and 1/sqrt(var + eps) (two passes over the registers).
+template <int D>
+__device__ __forceinline__ float2 row_stats(const float* y) {
   float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int i = 0; i < 64; ++i) a[i & 3] += y[i];
-  const float mean = ((a[0] + a[1]) + (a[2] + a[3])) * (1.f / 64);
+  for (int i = 0; i < D; ++i) a[i & 3] += y[i];
+  const float mean = ((a[0] + a[1]) + (a[2] + a[3])) * (1.f / D);
 #pragma unroll
   for (int i = 0; i < 4; ++i) a[i] = 0.f;
 #pragma unroll
-  for (int i = 0; i < 64; ++i) a[i & 3] = fmaf(y[i] - mean, y[i] - mean, a[i & 3]);
-  const float m2 = (a[0] + a[1]) + (a[2] + a[3]);
-  const float2 o = e.swap(make_float2(mean, m2), 0);
-  const float d = mean - o.x;
-  const float mu = 0.5f * (mean + o.x);
-  const float var = (m2 + o.y + d * d * 32.f) * (1.f / kD);
-  return make_float2(mu, rsqrtf(var + kLnEps));
+  for (int i = 0; i < D; ++i) {
+    const float d = y[i] - mean;
+    a[i & 3] = fmaf(d, d, a[i & 3]);
+  }
+  return make_float2(mean, rsqrtf(((a[0] + a[1]) + (a[2] + a[3])) * (1.f / D) + kLnEps));
 }
 
-// LayerNorm of this thread's 64 columns -> bf16 into the A operand.
-__device__ __forceinline__ void ln_to_A(Epi& e, const float* y, const float* gamma, const float* beta) {
-  const float2 st = row_stats(e, y);
-  const float4* g4 = reinterpret_cast<const float4*>(gamma + 64 * e.hf);
-  const float4* b4 = reinterpret_cast<const float4*>(beta + 64 * e.hf);
+// LayerNorm of the row -> fp16 A operand row.
+template <int D>
+__device__ __forceinline__ void ln_to_A(const Epi& e, const float* y, const float* g, const float* b) {
+  const float2 st = row_stats<D>(y);
 #pragma unroll
-  for (int kc = 0; kc < 8; ++kc) {
-    const float4 ga = g4[2 * kc], gb = g4[2 * kc + 1];
-    const float4 ba = b4[2 * kc], bb = b4[2 * kc + 1];
-    const float gg[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-    const float bbv[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
-    float v[8];
+  for (int kc = 0; kc < D / 8; ++kc) {
+    float gg[8], bb[8], v[8];
+    ld8(g + 8 * kc, gg);
+    ld8(b + 8 * kc, bb);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = fmaf((y[kc * 8 + i] - st.x) * st.y, gg[i], bbv[i]);
-    st_row8(e.sA + (8 * e.hf + kc) * 2048 + e.rowoff, v);
+    for (int i = 0; i < 8; ++i) v[i] = fmaf((y[8 * kc + i] - st.x) * st.y, gg[i], bb[i]);
+    st_row8h(e.sA + kc * 2048 + e.rowoff, v);
     step_barrier();
   }
 }
 
-// ReLU of 64 accumulator columns -> bf16 pairs in 32 TMEM columns (an A operand row).
-__device__ __forceinline__ void relu_to_tmem(uint32_t tcol, uint32_t dcol) {
-  float v[64];
-  load64(tcol, v);
+// 128 columns of the work area -> ReLU -> fp16 pairs in its first 64 columns (in place: every
+// value is read before the first store).
+__device__ __forceinline__ void relu_in_place(uint32_t tW) {
+  float h[128];
 #pragma unroll
-  for (int i = 0; i < 64; ++i) v[i] = fmaxf(v[i], 0.f);
-  tmem_st_bf16x32(dcol, v);
-  tmem_st_bf16x32(dcol + 16, v + 32);
+  for (int c = 0; c < 4; ++c) tmem_ld32(tW + 32 * c, h + 32 * c);
+  tmem_wait_ld();
+  reg_fence<128>(h);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t r[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = pack_h2(fmaxf(h[32 * c + 2 * i], 0.f), fmaxf(h[32 * c + 2 * i + 1], 0.f));
+    tmem_st16u(tW + 16 * c, r);
+  }
 }
 
-template <bool PF, int HG>
-__device__ __forceinline__ void epi_tile(const StackParams& p, const TileInfo& t, Epi& e) {
-  constexpr int NG = 8 / HG;
-  constexpr int SV = HG == 8 ? 16 : HG == 4 ? 32 : 64;   // keys one thread holds for one head
-  const int hf = e.hf, m = e.m;
-  const uint32_t ycol = e.trow + 64 * hf;
-  const float* sd = p.domain_emb + (size_t)p.req[t.r].domain * kD + 64 * hf;
-  // ---- Y = t + s_d (rows past the request's end are zero and never stored)
-  {
-    float y[64];
-    const float4* sd4 = reinterpret_cast<const float4*>(sd);
-    const bool live = m < t.rows;
-    if (PF) {
-      const float4* src = reinterpret_cast<const float4*>(p.utokens + (t.row0 + m) * kD + 64 * hf);
+// Softmax of one head's row over its Lp key columns at `base` (keys >= L_u masked) together
+// with the own key's score `sself` (-inf when there is none): numerators as fp16 pairs over
+// the first Lp/2 columns; returns (own numerator, 1 / sum).
+template <int SW>
+__device__ __forceinline__ float2 softmax_head(uint32_t base, int Lp, int L_u, float sself) {
+  const int nb = Lp / 16;
+  if constexpr (SW <= 64) {
+    float sv[SW];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const float4 u = live ? __ldg(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 d = __ldg(sd4 + c);
-        y[4 * c] = live ? u.x + d.x : 0.f;
-        y[4 * c + 1] = live ? u.y + d.y : 0.f;
-        y[4 * c + 2] = live ? u.z + d.z : 0.f;
-        y[4 * c + 3] = live ? u.w + d.w : 0.f;
-        step_barrier();
-      }
-    } else {
-      const uint4* src = reinterpret_cast<const uint4*>(p.tokens + (t.row0 + m) * kD + 64 * hf);
+    for (int c = 0; c < SW / 16; ++c)
+      if (c < nb) tmem_ld16(base + 16 * c, sv + 16 * c);
+    tmem_wait_ld();
+    reg_fence<SW>(sv);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 u = live ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
-        const float4 da = __ldg(sd4 + 2 * c), db = __ldg(sd4 + 2 * c + 1);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-        const float d[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+    for (int i = 0; i < SW; ++i)
+      if (i >= L_u) sv[i] = -INFINITY;
+    float m4[4] = {sself, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          y[c * 8 + 2 * i] = live ? __uint_as_float(w[i] << 16) + d[2 * i] : 0.f;
-          y[c * 8 + 2 * i + 1] = live ? __uint_as_float(w[i] & 0xFFFF0000u) + d[2 * i + 1] : 0.f;
+    for (int i = 0; i < SW; i += 8) {
+      m4[0] = max3(m4[0], sv[i], sv[i + 1]);
+      m4[1] = max3(m4[1], sv[i + 2], sv[i + 3]);
+      m4[2] = max3(m4[2], sv[i + 4], sv[i + 5]);
+      m4[3] = max3(m4[3], sv[i + 6], sv[i + 7]);
+    }
+    const float nm = -fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * kL2E;
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int c = 0; c < SW / 16; ++c)
+      if (c < nb) {
+        uint32_t r[8];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          sv[16 * c + i] = ex2(fmaf(sv[16 * c + i], kL2E, nm));
+          s4[i & 3] += sv[16 * c + i];
         }
-        step_barrier();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) r[i] = pack_h2(sv[16 * c + 2 * i], sv[16 * c + 2 * i + 1]);
+        tmem_st8u(base + 8 * c, r);
       }
-    }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_st16(ycol + 16 * c, y + 16 * c);
-    tmem_wait_st();
-  }
-
-  for (int l = 0; l < p.n_layer; ++l) {
-    const float* vl = e.vec + (size_t)l * kVecPerLayer;
-    // ---- LN1 -> A
-    if (l > 0 && !e.wait(e.b.ev_y(), e.ph_y)) return;
-    {
-      float y[64];
-      load64(ycol, y);
-      ln_to_A(e, y, vl, vl + kD);
-    }
-    e.signal(e.b.e1());
-    // ---- Q (scaled) -> A; own score per head; own V -> registers; user side: K/V images
-    if (!e.wait(e.b.ev_qk(), e.ph_qk)) return;
-    if (PF) {
-      if (threadIdx.x == kEpiThread0 && l > 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-      if (!e.sync()) return;                       // the K/V images are free to overwrite
-    }
-    float sself[4];
-    uint32_t vself[4][8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int h = 4 * hf + j;
-      float qv[16], kv[16], vv[16];
-      tmem_ld16(e.trow + 128 + 16 * h, qv);
-      tmem_ld16(e.trow + 256 + 16 * h, kv);
-      tmem_ld16(e.trow + 384 + 16 * h, vv);
+    const float ps = ex2(fmaf(sself, kL2E, nm));
+    return make_float2(ps, 1.f / (((s4[0] + s4[1]) + (s4[2] + s4[3])) + ps));
+  } else {
+    // two passes over 16-key chunks: the maximum, then the numerators (chunk c's numerators
+    // land in columns 8c .. 8c + 7, which only chunks up to c have occupied)
+    float mx = sself;
+#pragma unroll 1
+    for (int c = 0; c < nb; ++c) {
+      float v[16];
+      tmem_ld16(base + 16 * c, v);
       tmem_wait_ld();
-      reg_fence<16>(qv);
-      reg_fence<16>(kv);
-      reg_fence<16>(vv);
-      float s = 0.f;
+      reg_fence<16>(v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (16 * c + i < L_u) mx = fmaxf(mx, v[i]);
+    }
+    const float nm = -mx * kL2E;
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 1
+    for (int c = 0; c < nb; ++c) {
+      float v[16];
+      tmem_ld16(base + 16 * c, v);
+      tmem_wait_ld();
+      reg_fence<16>(v);
+      uint32_t r[8];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        qv[i] *= kQScale;
-        s = fmaf(qv[i], kv[i], s);
+        v[i] = 16 * c + i < L_u ? ex2(fmaf(v[i], kL2E, nm)) : 0.f;
+        s4[i & 3] += v[i];
       }
-      sself[j] = PF ? -INFINITY : s;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) vself[j][i] = pack2(vv[2 * i], vv[2 * i + 1]);
-      st_row8(e.sA + (2 * h) * 2048 + e.rowoff, qv);
-      st_row8(e.sA + (2 * h + 1) * 2048 + e.rowoff, qv + 8);
-      if (PF && m < t.Lp) {
-        // K image row m, V^T image column m (zero past L_u)
-        const bool live = m < t.L_u;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          kv[i] = live ? kv[i] : 0.f;
-          vv[i] = live ? vv[i] : 0.f;
-        }
-        const uint32_t kb = e.sKV + (m >> 3) * 128 + (m & 7) * 16;
-        st_row8(kb + (2 * h) * (t.Lp / 8) * 128, kv);
-        st_row8(kb + (2 * h + 1) * (t.Lp / 8) * 128, kv + 8);
-        const uint32_t vb = e.sKV + t.Lp * 256 + (m >> 3) * 2048 + (m & 7) * 2;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int d = 16 * h + i;
-          const __nv_bfloat16 hv = __float2bfloat16_rn(vv[i]);
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(vb + (d >> 3) * 128 + (d & 7) * 16),
-                       "h"(*reinterpret_cast<const unsigned short*>(&hv))
-                       : "memory");
-        }
-      }
+      for (int i = 0; i < 8; ++i) r[i] = pack_h2(v[2 * i], v[2 * i + 1]);
+      tmem_st8u(base + 8 * c, r);
     }
-    if (PF) {  // store this layer's K/V images to the cache with one bulk copy
-      fence_proxy_async_smem();
-      if (!e.sync()) return;
-      if (threadIdx.x == kEpiThread0) {
-        const uint32_t bytes = 2u * t.Lp * kD * 2u;
-        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(p.kv_out + (size_t)l * bytes),
-                     "r"(e.sKV), "r"(bytes)
-                     : "memory");
-        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-      }
+    const float ps = ex2(fmaf(sself, kL2E, nm));
+    return make_float2(ps, 1.f / (((s4[0] + s4[1]) + (s4[2] + s4[3])) + ps));
+  }
+}
+
+template <int D, int SW, bool UM>
+__device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Epi& e) {
+  constexpr int NH = Cfg<D>::kNH;
+  const int m = e.m;
+  const bool live = m < t.rows;
+  // ---- Y = token + s_d (rows past the tile's end are zero and never stored)
+  {
+    float y[D];
+    const float4* sd4 = reinterpret_cast<const float4*>(p.domain_emb + (size_t)t.dom * D);
+    const float4* src = reinterpret_cast<const float4*>(
+        UM ? p.req[t.r].utokens + (size_t)m * D : p.tokens + (size_t)(t.row0 + m) * D);
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) {
+      const float4 u = live ? __ldg(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 d = __ldg(sd4 + c);
+      y[4 * c] = live ? u.x + d.x : 0.f;
+      y[4 * c + 1] = live ? u.y + d.y : 0.f;
+      y[4 * c + 2] = live ? u.z + d.z : 0.f;
+      y[4 * c + 3] = live ? u.w + d.w : 0.f;
     }
-    e.signal(e.b.e2());
-    // ---- softmax over [user keys of the request, own key], one head group at a time
-    float pself[4] = {1.f, 1.f, 1.f, 1.f}, linv[4] = {1.f, 1.f, 1.f, 1.f};
-    if constexpr (HG >= 2) {
-      // One score group per round: while the epilogue works on group g + 1 the tensor core
-      // multiplies group g's numerators by V and computes group g + 2's scores into the
-      // buffer group g used.  (Two groups per round measured no faster: it loses that
-      // overlap.)  Rounds signal e3(0) and e3(1) in turn, so the MMA thread's wait on one
-      // never sees it complete twice.
-      constexpr int GPR = 1;
-      const int nb = t.Lp / 16;                   // 16-key blocks holding keys (>= 1)
-      const int tail = t.L_u - 16 * (nb - 1);     // keys in the last block (1..16)
 #pragma unroll
-      for (int g0 = 0; g0 < NG; g0 += GPR) {
-        if (g0 >= t.ng) break;
+    for (int c = 0; c < D / 16; ++c) tmem_st16(e.tY + 16 * c, y + 16 * c);
+    tmem_wait_st();
+  }
+  // (Y is re-read from tensor memory at the top of every layer, so that no register copy of
+  // it stays live through the layer)
+  for (int l = 0; l < p.n_layer; ++l) {
+    const float* vl = e.vec + (size_t)l * vec_per_layer<D>();
+    if (l > 0 && !e.wait()) return;                // the previous layer's FFN product is in Y
+    {
+      float y[D];
+      load_row<D>(e.tY, y);
+      ln_to_A<D>(e, y, vl, vl + D);
+    }
+    e.signal();
+    // ---- own K and V (user mode: this row of the layer's K and V^T images), read in two
+    // halves of D/2 columns
+    uint32_t kreg[UM ? 1 : D / 2], vreg[UM ? 1 : D / 2];
 #pragma unroll
-        for (int gi = 0; gi < GPR; ++gi)
-          if (!e.wait(e.b.ev_s((g0 + gi) & 1), e.ph_s[(g0 + gi) & 1])) return;
+    for (int pass = 0; pass < 2; ++pass) {
+      if (!e.wait()) return;
 #pragma unroll
-        for (int gi = 0; gi < GPR; ++gi) {
-          const int g = g0 + gi;
-          const uint32_t sbuf = e.trow + 128 + 128 * (g & 1);
+      for (int hb = 0; hb < 2; ++hb) {
+        float x[D / 2];
 #pragma unroll
-          for (int j = 0; j < HG / 2; ++j) {
-            const int jj = g * (HG / 2) + j;        // this half's head index (0..3)
-            const int slot = hf * (HG / 2) + j;
-            float sv[SV];
+        for (int c = 0; c < D / 64; ++c) tmem_ld32(e.tW + D / 2 * hb + 32 * c, x + 32 * c);
+        tmem_wait_ld();
+        reg_fence<D / 2>(x);
+        if constexpr (UM) {
+          if (m < t.Lp) {
+            const bool real = m < t.L_u;
+            if (pass == 0) {   // K image [Lp x D]: row m, eight columns per core-matrix row
 #pragma unroll
-            for (int c = 0; c < SV / 16; ++c) {
-              if (c < nb) {
-                tmem_ld16(sbuf + slot * t.Lp + 16 * c, sv + 16 * c);
-              } else {
+              for (int j = 0; j < D / 16; ++j) {
+                const int cc = D / 16 * hb + j;
+                float v[8];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) sv[16 * c + i] = -INFINITY;
+                for (int i = 0; i < 8; ++i) v[i] = real ? x[8 * j + i] : 0.f;
+                st_row8h(e.sKV + (cc * (t.Lp / 8) + (m >> 3)) * 128 + (m & 7) * 16, v);
+              }
+            } else {           // V^T image [D x Lp]: column m
+              const uint32_t vb = e.sKV + t.Lp * D * 2 + (m >> 3) * (D / 8) * 128 + (m & 7) * 2;
+#pragma unroll
+              for (int i = 0; i < D / 2; ++i) {
+                const int d = D / 2 * hb + i;
+                const __half hv = __float2half_rn(real ? x[i] : 0.f);
+                asm volatile("st.shared.b16 [%0], %1;" ::"r"(vb + (d >> 3) * 128 + (d & 7) * 16),
+                             "h"(*reinterpret_cast<const unsigned short*>(&hv))
+                             : "memory");
               }
             }
-            tmem_wait_ld();
-            reg_fence<SV>(sv);
-            // padding keys (L_u not a multiple of 16) -> -inf, so the loops below need no masks
-            if (tail < 16) {
+          }
+        } else {
 #pragma unroll
-              for (int i = 0; i < SV; ++i) sv[i] = i < t.L_u ? sv[i] : -INFINITY;
-            }
-            // max: four chains of three-input maxima
-            float m4[4] = {sself[jj], -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int i = 0; i < SV; i += 8) {
-              m4[0] = max3(m4[0], sv[i], sv[i + 1]);
-              m4[1] = max3(m4[1], sv[i + 2], sv[i + 3]);
-              m4[2] = max3(m4[2], sv[i + 4], sv[i + 5]);
-              m4[3] = max3(m4[3], sv[i + 6], sv[i + 7]);
-            }
-            const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            // exponentials; the subtraction and the running sums on packed pairs
-            const uint64_t neg = f32x2(-mx, -mx);
-            uint64_t acc[2] = {f32x2(0.f, 0.f), f32x2(0.f, 0.f)};
-#pragma unroll
-            for (int i = 0; i < SV; i += 2) {
-              float x0, x1;
-              f32x2_split(add_f32x2(f32x2(sv[i], sv[i + 1]), neg), x0, x1);
-              sv[i] = ex2(x0);
-              sv[i + 1] = ex2(x1);
-              acc[(i >> 1) & 1] = add_f32x2(acc[(i >> 1) & 1], f32x2(sv[i], sv[i + 1]));
-            }
-            float a0, a1, b0, b1;
-            f32x2_split(acc[0], a0, a1);
-            f32x2_split(acc[1], b0, b1);
-            const float sum = (a0 + a1) + (b0 + b1);
-            // numerators as bf16 over the first half of this slot's own score columns (the
-            // P V products read only the first L_p / 2 of them)
-            const uint32_t pcol = sbuf + slot * t.Lp;
-            if constexpr (SV == 16) {
-              tmem_st_bf16x16(pcol, sv);
-            } else {
-#pragma unroll
-              for (int c = 0; c < SV / 32; ++c) tmem_st_bf16x32(pcol + 16 * c, sv + 32 * c);
-            }
-            pself[jj] = ex2(sself[jj] - mx);
-            linv[jj] = 1.f / (sum + pself[jj]);
+          for (int i = 0; i < D / 4; ++i) {
+            if (pass == 0)
+              kreg[D / 4 * hb + i] = pack_h2(x[2 * i], x[2 * i + 1]);
+            else
+              vreg[D / 4 * hb + i] = pack_h2(x[2 * i], x[2 * i + 1]);
           }
         }
-        e.signal(e.b.e3((g0 / GPR) & 1));
       }
-    } else {
-      // L_u > 64: one head per group, its keys split between the two column halves
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        if (!e.wait(e.b.ev_s(g & 1), e.ph_s[g & 1])) return;
-        const uint32_t sbuf = e.trow + 128 + 128 * (g & 1);
-        const int k0 = 64 * hf;
-        const int nk = min(64, t.Lp - k0);       // > 0: Lp >= 80
-        float sv[64];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          if (c < nk / 16) tmem_ld16(sbuf + k0 + 16 * c, sv + 16 * c);
-        tmem_wait_ld();
-        reg_fence<64>(sv);
-        const bool owner = (g >> 2) == hf;       // this half owns head g (and its own score)
-        float m4[4] = {owner ? sself[g & 3] : -INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (i < nk && k0 + i < t.L_u) m4[i & 3] = fmaxf(m4[i & 3], sv[i]);
-        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        mx = fmaxf(mx, e.swap(make_float2(mx, 0.f), 0).x);
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float ev = (i < nk && k0 + i < t.L_u) ? ex2(sv[i] - mx) : 0.f;
-          sv[i] = ev;
-          s4[i & 3] += ev;
-        }
-        const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-        // keys 64 hf .. as bf16 from column 32 hf of the buffer: over this half's own scores
-        // (hf = 0) or the first half's, which both halves have read before the max exchange
-        tmem_st_bf16x32(sbuf + 32 * hf, sv);
-        tmem_st_bf16x32(sbuf + 32 * hf + 16, sv + 32);
-        const float ps = owner ? ex2(sself[g & 3] - mx) : 0.f;
-        const float tot = sum + ps + e.swap(make_float2(sum + ps, 0.f), 1).x;
-        if (owner) {
-          pself[g & 3] = ps;
-          linv[g & 3] = 1.f / tot;
-        }
-        e.signal(e.b.e3(g & 1));
-      }
+      e.signal();
     }
-    // ---- attention output = (sum_j p_j v_j + p_self v_self) / l  -> A
-    if (!e.wait(e.b.ev_av(), e.ph_av)) return;
-    const bool has_users = t.ng > 0;
+    // ---- Q (pre-scaled by 1/sqrt(d_h) through its weights) -> A; own score per head
+    float sself[NH];
+    if (!e.wait()) return;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int h = 4 * hf + j;
-      float o[16];
-      tmem_ld16(e.trow + 384 + 16 * h, o);
+    for (int hc = 0; hc < D / 32; ++hc) {
+      float q[32];
+      tmem_ld32(e.tW + 32 * hc, q);
       tmem_wait_ld();
-      reg_fence<16>(o);
+      reg_fence<32>(q);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t w = vself[j][i];
-        const float v0 = __uint_as_float(w << 16), v1 = __uint_as_float(w & 0xFFFF0000u);
-        o[2 * i] = ((has_users ? o[2 * i] : 0.f) + pself[j] * v0) * linv[j];
-        o[2 * i + 1] = ((has_users ? o[2 * i + 1] : 0.f) + pself[j] * v1) * linv[j];
+      for (int j = 0; j < 2; ++j) {
+        const int h = 2 * hc + j;
+        if constexpr (UM) {
+          sself[h] = -INFINITY;
+        } else {
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            s0 = fmaf(q[16 * j + 2 * i], h_lo(kreg[8 * h + i]), s0);
+            s1 = fmaf(q[16 * j + 2 * i + 1], h_hi(kreg[8 * h + i]), s1);
+          }
+          sself[h] = s0 + s1;
+        }
+        if (UM || t.Lp > 0) {
+          st_row8h(e.sA + (2 * h) * 2048 + e.rowoff, q + 16 * j);
+          st_row8h(e.sA + (2 * h + 1) * 2048 + e.rowoff, q + 16 * j + 8);
+        } else {             // no user keys: the attention output is the own value
+          float o[16];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            o[2 * i] = h_lo(vreg[8 * h + i]);
+            o[2 * i + 1] = h_hi(vreg[8 * h + i]);
+          }
+          st_row8h(e.sA + (2 * h) * 2048 + e.rowoff, o);
+          st_row8h(e.sA + (2 * h + 1) * 2048 + e.rowoff, o + 8);
+        }
       }
-      st_row8(e.sA + (2 * h) * 2048 + e.rowoff, o);
-      st_row8(e.sA + (2 * h + 1) * 2048 + e.rowoff, o + 8);
     }
-    e.signal(e.b.e4());
+    e.signal();
+    // ---- attention, one head group at a time
+    constexpr int HG = Groups<D, SW>::HG;
+    if (t.Lp > 0) {
+#pragma unroll
+      for (int g = 0; g < Groups<D, SW>::NG; ++g) {
+        float ps[HG], li[HG];
+        if (!e.wait()) return;                     // scores of group g
+        // one head after the other (not interleaved by the compiler: that would hold several
+        // heads' scores in registers at once)
+#pragma unroll 1
+        for (int i = 0; i < HG; ++i) {
+          float ss = sself[g * HG];
+#pragma unroll
+          for (int k = 1; k < HG; ++k)
+            if (i == k) ss = sself[g * HG + k];
+          const float2 r = softmax_head<SW>(e.tW + i * SW, t.Lp, t.L_u, ss);
+#pragma unroll
+          for (int k = 0; k < HG; ++k)
+            if (i == k) {
+              ps[k] = r.x;
+              li[k] = r.y;
+            }
+        }
+        e.signal();
+        if (!e.wait()) return;                     // P V of group g
+#pragma unroll
+        for (int i = 0; i < HG; ++i) {
+          const int h = g * HG + i;
+          float o[16];
+          tmem_ld16(e.tW + i * SW + SW / 2, o);
+          tmem_wait_ld();
+          reg_fence<16>(o);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if constexpr (UM) {
+              o[2 * j] *= li[i];
+              o[2 * j + 1] *= li[i];
+            } else {
+              o[2 * j] = fmaf(ps[i], h_lo(vreg[8 * h + j]), o[2 * j]) * li[i];
+              o[2 * j + 1] = fmaf(ps[i], h_hi(vreg[8 * h + j]), o[2 * j + 1]) * li[i];
+            }
+          }
+          st_row8h(e.sA + (2 * h) * 2048 + e.rowoff, o);
+          st_row8h(e.sA + (2 * h + 1) * 2048 + e.rowoff, o + 8);
+        }
+        e.signal();
+      }
+    }
     // ---- LN2 -> A
-    if (!e.wait(e.b.ev_o(), e.ph_o)) return;
+    if (!e.wait()) return;                         // Y += attn Wo + bo
     {
-      float y[64];
-      load64(ycol, y);
-      ln_to_A(e, y, vl + 2 * kD, vl + 3 * kD);
+      float y[D];
+      load_row<D>(e.tY, y);
+      ln_to_A<D>(e, y, vl + 2 * D, vl + 3 * D);
     }
-    e.signal(e.b.e5());
-    // ---- ReLU(hidden) -> P0 (first half of the hidden units) and A (second half)
-    if (!e.wait(e.b.ev_h0(), e.ph_h0)) return;
-    relu_to_tmem(e.trow + 128 + 64 * hf, e.trow + 384 + 32 * hf);
-    e.signal(e.b.e6a());
-    if (!e.wait(e.b.ev_h1(), e.ph_h1)) return;
-    relu_to_tmem(e.trow + 256 + 64 * hf, e.trow + 448 + 32 * hf);
-    e.signal(e.b.e6b());
+    e.signal();
+    // ---- ReLU(hidden) -> fp16 A operand in the work area, a 128-unit half at a time
+#pragma unroll
+    for (int half = 0; half < Cfg<D>::kFfnHalves; ++half) {
+      if (!e.wait()) return;
+      relu_in_place(e.tW);
+      e.signal();
+    }
   }
-  // ---- head: w . LN_f(y) + b
-  if (!e.wait(e.b.ev_y(), e.ph_y)) return;
-  if (PF) return;
-  float y[64];
-  load64(ycol, y);
-  const float2 st = row_stats(e, y);
-  const float* vf = e.vec + (size_t)p.n_layer * kVecPerLayer;
-  const float4* w4 = reinterpret_cast<const float4*>(vf + 64 * hf);
+  // ---- head: w . LN_f(y) + b (w folded with the final LayerNorm's gain)
+  if (!e.wait()) return;
+  if (UM) return;
+  float y[D];
+  load_row<D>(e.tY, y);
+  const float2 st = row_stats<D>(y);
+  const float* vf = e.vec + (size_t)p.n_layer * vec_per_layer<D>();
   float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float4 w = w4[i];
-    a4[0] = fmaf((y[4 * i] - st.x) * st.y, w.x, a4[0]);
-    a4[1] = fmaf((y[4 * i + 1] - st.x) * st.y, w.y, a4[1]);
-    a4[2] = fmaf((y[4 * i + 2] - st.x) * st.y, w.z, a4[2]);
-    a4[3] = fmaf((y[4 * i + 3] - st.x) * st.y, w.w, a4[3]);
-    step_barrier();
+  for (int c = 0; c < D / 8; ++c) {
+    float w[8];
+    ld8(vf + 8 * c, w);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a4[i & 3] = fmaf((y[8 * c + i] - st.x) * st.y, w[i], a4[i & 3]);
   }
-  const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-  const float tot = acc + e.swap(make_float2(acc, 0.f), 1).x;
-  if (hf == 0 && m < t.rows) p.scores[t.row0 + m] = tot + vf[kD];
+  if (live) p.scores[t.row0 + m] = ((a4[0] + a4[1]) + (a4[2] + a4[3])) + vf[D];
 }
 
-template <bool PF, int HG>
-__device__ void epilogue(const StackParams& p, uint32_t tmem, uint32_t sA, uint32_t sKV,
-                         uint32_t sX, uint32_t sOnes, float* svec, const Bars& b, volatile int* abort_flag) {
+template <int D, int SW, bool UM>
+__device__ void epilogue(const StackParams& p, int slot, uint32_t tmem, uint32_t sA, uint32_t sKV, uint32_t sOnes,
+                         const float* vec, const Bars& b, volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Epi e;
-  e.q = warp & 3;
-  e.m = e.q * 32 + lane;
-  e.hf = (warp - 4) >> 2;
-  e.trow = tmem + ((uint32_t)(e.q * 32) << 16);
-  e.rowoff = (e.m >> 3) * 128 + (e.m & 7) * 16;
+  e.m = (warp & 3) * 32 + lane;
+  e.tY = tmem + ((uint32_t)((warp & 3) * 32) << 16) + kSlotCols * slot;
+  e.tW = e.tY + D;
   e.sA = sA;
+  e.rowoff = (e.m >> 3) * 128 + (e.m & 7) * 16;
   e.sKV = sKV;
-  e.sX = sX;
-  e.b = b;
+  e.e2m = b.e2m(slot);
+  e.m2e = b.m2e(slot);
+  e.ph = 0;
+  e.vec = vec;
   e.abort_flag = abort_flag;
   e.ok = true;
-  e.ph_qk = e.ph_s[0] = e.ph_s[1] = e.ph_av = e.ph_o = e.ph_h0 = e.ph_h1 = e.ph_y = e.ph_sync = e.ph_q = 0;
-  // the constant ones tile: columns 0 and 1 of every row are 1 (bias head and tail)
-  if (e.hf == 0) {
-    const float one2[8] = {1.f, 1.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, zero[8] = {};
-    st_row8(sOnes + e.rowoff, one2);
-    st_row8(sOnes + 2048 + e.rowoff, zero);
-  }
-  // LayerNorm vectors and the head weight: a shared-memory copy when they fit
-  const int nvec = p.n_layer * kVecPerLayer + kVecFinal;
-  if (p.n_layer <= kMaxLayersSmemVec) {
-    const int tid = threadIdx.x - kEpiThread0;
-    for (int i = tid; i < nvec; i += kEpiThreads) svec[i] = __ldg(p.vec + i);
-    if (!e.sync()) return;
-    e.vec = svec;
-  } else {
-    e.vec = p.vec;
-  }
-  for (int tile = blockIdx.x; tile < p.n_tiles && e.ok; tile += gridDim.x) {
-    const TileInfo t = tile_info(p, tile);
-    epi_tile<PF, HG>(p, t, e);   // the host launches one kernel per head-group size
+  for (int u = blockIdx.x; u < p.n_units && e.ok; u += gridDim.x) {
+    const Tile t = tile_of<D>(p, u, slot);
+    if (t.active) epi_tile<D, SW, UM>(p, t, e);
   }
 }
 
-template <bool PF, int HG>
+template <int D, int SW, bool UM>
 __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base = smem_u32(smem);
-  const uint32_t sA = base + OFF_A, sKV = base + OFF_KV, ring = base + OFF_RING;
-  const uint32_t sOnes = base + OFF_ONES, sX = base + OFF_X;
-  float* svec = reinterpret_cast<float*>(smem + OFF_VEC);
-  const Bars b{base + OFF_BAR};
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + kBarBytes);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_BAR + kBarBytes + 8);
+  const uint32_t sA0 = base, sKV = base + p.off_kv, ring = base + p.off_ring, sOnes = base + p.off_ones;
+  const Bars b{base + p.off_bar};
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + p.off_bar + 8 * kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + p.off_bar + 8 * kNumBars + 8);
+  const float* vec = p.off_vec >= 0 ? reinterpret_cast<const float*>(smem + p.off_vec) : p.vec;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < kMaxStages; ++s) {
       mbar_init(b.full(s), 1);
-      mbar_init(b.empty(s), 1);
+      mbar_init(b.empty(s), p.pair ? 2 : 1);
     }
     mbar_init(b.kv_full(), 1);
-    mbar_init(b.kv_empty(), 1);
-    for (uint32_t a : {b.ev_qk(), b.ev_s(0), b.ev_s(1), b.ev_av(), b.ev_o(), b.ev_h0(), b.ev_h1(), b.ev_y(), b.drain(),
-                       b.av_done(0), b.av_done(1)})
-      mbar_init(a, 1);
-    for (uint32_t a : {b.e1(), b.e2(), b.e3(0), b.e3(1), b.e4(), b.e5(), b.e6a(), b.e6b(), b.esync()}) mbar_init(a, kEpiThreads);
-    for (int q = 0; q < 4; ++q) mbar_init(b.qsync(q), 64);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(b.kv_empty(s), 1);
+      mbar_init(b.e2m(s), kSlotThreads);
+      mbar_init(b.m2e(s), 1);
+      mbar_init(b.mm(s), 1);
+      mbar_init(b.drain(s), 1);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 1) {
+  if (warp == 3) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
+  }
+  // constant operands: the ones tile (columns 0 and 1 of every row are 1) and the vectors
+  if (threadIdx.x >= 128) {
+    const int t = threadIdx.x - 128;
+    if (t < kM) {
+      const float one2[8] = {1.f, 1.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, zero[8] = {};
+      const uint32_t ro = (t >> 3) * 128 + (t & 7) * 16;
+      st_row8h(sOnes + ro, one2);
+      st_row8h(sOnes + 2048 + ro, zero);
+    }
+    if (p.off_vec >= 0) {
+      const int nvec = p.n_layer * vec_per_layer<D>() + D + 4;
+      float* sv = reinterpret_cast<float*>(smem + p.off_vec);
+      for (int i = t; i < nvec; i += 2 * kSlotThreads) sv[i] = __ldg(p.vec + i);
+    }
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -860,16 +868,21 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
-    if (warp == 0 && lane == 0) producer<PF>(p, ring, sKV, b, abort_flag);
-    if (warp == 1 && lane == 0) mma_issuer<PF, HG>(p, tmem, sA, sKV, ring, sOnes, b, abort_flag);
+    if (lane == 0) {
+      if (warp == 0) weight_producer<D>(p, ring, b, abort_flag);
+      if (warp == 1) mma_issuer<D, SW, UM>(p, 0, tmem, sA0, sKV, ring, sOnes, b, abort_flag);
+      if (warp == 2 && p.pair) mma_issuer<D, SW, UM>(p, 1, tmem, sA0 + kM * D * 2, sKV, ring, sOnes, b, abort_flag);
+      if (warp == 3 && !UM) kv_producer<D>(p, sKV, b, abort_flag);
+    }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
-    epilogue<PF, HG>(p, tmem, sA, sKV, sX, sOnes, svec, b, abort_flag);
-    if (PF && threadIdx.x == kEpiThread0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    const int slot = (warp - 4) >> 2;
+    if (slot == 0 || p.pair)
+      epilogue<D, SW, UM>(p, slot, tmem, sA0 + slot * kM * D * 2, sKV, sOnes, vec, b, abort_flag);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 3) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -878,77 +891,118 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
 
 // ------------------------------------------------------------------ host: operand images
 
-uint16_t bf16_bits(float f) {
-  uint32_t u;
-  memcpy(&u, &f, 4);
-  u = (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;  // round to nearest even
-  return (uint16_t)u;
+uint16_t f16_bits(float f) {
+  const __half h = __float2half_rn(f);
+  uint16_t u;
+  memcpy(&u, &h, 2);
+  return u;
 }
-float bf16_value(uint16_t h) {
-  const uint32_t u = (uint32_t)h << 16;
-  float f;
-  memcpy(&f, &u, 4);
-  return f;
-}
-
-// W^T slice [n0, n0+128) x [k0, k0+64) of W [K][N] (row-major, W[k][n]) in core-matrix layout.
-void put_chunk(uint16_t* dst, const float* W, int N, int n0, int k0) {
-  for (int n = 0; n < 128; ++n)
-    for (int k = 0; k < 64; ++k)
-      dst[((size_t)(k / 8) * 16 + n / 8) * 64 + (n % 8) * 8 + (k % 8)] = bf16_bits(W[(size_t)(k0 + k) * N + n0 + n]);
+float f16_value(uint16_t u) {
+  __half h;
+  memcpy(&h, &u, 2);
+  return __half2float(h);
 }
 
-// Bias tile [128 x 16]: column 0 the bf16 nearest to b[n0+n], column 1 the bf16 of the rest.
-void put_bias(uint16_t* dst, const float* bias, int n0) {
-  for (int n = 0; n < 128; ++n) {
-    const float v = bias[n0 + n];
-    const uint16_t hi = bf16_bits(v);
-    const uint16_t lo = bf16_bits(v - bf16_value(hi));
+// B operand [N x K] of the product x W (W [K_total][ld] row-major, columns n0.., rows k0..),
+// scaled by `scale`, in the core-matrix layout, fp16.
+void put_B(uint16_t* dst, const float* W, int ld, int n0, int k0, int N, int K, float scale) {
+  for (int n = 0; n < N; ++n)
+    for (int k = 0; k < K; ++k)
+      dst[((size_t)(k / 8) * (N / 8) + n / 8) * 64 + (n % 8) * 8 + (k % 8)] =
+          f16_bits(W[(size_t)(k0 + k) * ld + n0 + n] * scale);
+}
+// Bias tile [N x 16]: column 0 the fp16 nearest to b[n0+n] * scale, column 1 the fp16 of the rest.
+void put_bias(uint16_t* dst, const float* bias, int n0, int N, float scale) {
+  for (int n = 0; n < N; ++n) {
+    const float v = bias[n0 + n] * scale;
+    const uint16_t hi = f16_bits(v);
+    const uint16_t lo = f16_bits(v - f16_value(hi));
     for (int k = 0; k < 16; ++k)
-      dst[((size_t)(k / 8) * 16 + n / 8) * 64 + (n % 8) * 8 + (k % 8)] = k == 0 ? hi : k == 1 ? lo : 0;
+      dst[((size_t)(k / 8) * (N / 8) + n / 8) * 64 + (n % 8) * 8 + (k % 8)] = k == 0 ? hi : k == 1 ? lo : 0;
   }
+}
+
+template <int D>
+void build_layer_items(uint8_t* li, const tr_layer_weights& L) {
+  using C = Cfg<D>;
+  const int H = 2 * D;
+  // Q's weights and bias carry 1/sqrt(d_h) = 1/4 (exact in floating point)
+  const float* Wn[4] = {L.Wk, L.Wv, L.Wq, L.Wo};
+  const float* bn[4] = {L.bk, L.bv, L.bq, L.bo};
+  const float sc[4] = {1.f, 1.f, 0.25f, 1.f};
+  auto at = [&](int pi, int off) {
+    const Piece pc = C::piece(pi);
+    return reinterpret_cast<uint16_t*>(li + (size_t)pc.item * C::kItemBytes + off);
+  };
+  for (int j = 0; j < 4; ++j) {
+    const Piece pc = C::piece(j);
+    put_B(at(j, pc.off), Wn[j], D, 0, 0, D, D, sc[j]);
+    put_bias(at(j, pc.bias), bn[j], 0, D, sc[j]);
+  }
+  for (int hf = 0; hf < C::kFfnHalves; ++hf) {
+    const int p1 = hf == 0 ? P_W1A : P_W1B, p2 = hf == 0 ? P_W2A : P_W2B;
+    const Piece a = C::piece(p1), b = C::piece(p2);
+    put_B(at(p1, a.off), L.W1, H, 128 * hf, 0, 128, D, 1.f);            // hidden units 128 hf ..
+    put_bias(at(p1, a.bias), L.b1, 128 * hf, 128, 1.f);
+    put_B(at(p2, b.off), L.W2, D, 0, 128 * hf, D, 128, 1.f);            // rows 128 hf .. of W2
+    if (b.bias >= 0) put_bias(at(p2, b.bias), L.b2, 0, D, 1.f);
+  }
+}
+
+// Whether every fp16 operand of the stack stays far inside fp16's range: LayerNorm outputs
+// are bounded by max|gain| sqrt(D) + max|shift|, a product's outputs by that bound times the
+// largest column sum of |W| plus max|bias|, the attention output by the bound of V, ReLU by
+// the bound of its input.
+bool fp16_operands_safe(const tr_model_desc& d, const tr_model_weights* w) {
+  const int D = d.D, H = d.ffn_hidden;
+  auto amax = [](const float* p, size_t n) {
+    double m = 0;
+    for (size_t i = 0; i < n; ++i) m = std::max(m, (double)fabsf(p[i]));
+    return m;
+  };
+  auto colsum = [](const float* W, int K, int N) {
+    double m = 0;
+    for (int n = 0; n < N; ++n) {
+      double s = 0;
+      for (int k = 0; k < K; ++k) s += fabs((double)W[(size_t)k * N + n]);
+      m = std::max(m, s);
+    }
+    return m;
+  };
+  const double limit = 16384.0;
+  for (int l = 0; l < d.n_layer; ++l) {
+    const tr_layer_weights& L = w->layers[l];
+    const double b1 = amax(L.ln1_g, D) * sqrt((double)D) + amax(L.ln1_b, D);
+    const double b2 = amax(L.ln2_g, D) * sqrt((double)D) + amax(L.ln2_b, D);
+    const double q = b1 * colsum(L.Wq, D, D) + amax(L.bq, D);
+    const double k = b1 * colsum(L.Wk, D, D) + amax(L.bk, D);
+    const double v = b1 * colsum(L.Wv, D, D) + amax(L.bv, D);
+    const double h = b2 * colsum(L.W1, D, H) + amax(L.b1, H);
+    if (!(b1 < limit && b2 < limit && q < limit && k < limit && v < limit && h < limit)) return false;
+    const double wmax = std::max({amax(L.Wq, (size_t)D * D), amax(L.Wk, (size_t)D * D), amax(L.Wv, (size_t)D * D),
+                                  amax(L.Wo, (size_t)D * D), amax(L.W1, (size_t)D * H), amax(L.W2, (size_t)H * D)});
+    if (!(wmax < limit)) return false;
+  }
+  return true;
 }
 
 }  // namespace
 
-bool tc_stack_supported(const tr_model* m) {
-  const tr_model_desc& d = m->desc;
-  return d.dtype == TR_BF16 && d.D == kD && d.ffn_hidden == kH && d.n_head == 8 && m->tc_stack;
-}
+bool tc_stack_supported(const tr_model* m) { return m->tc_stack != nullptr; }
 
 tr_status tc_build_comp(tr_model* m, const tr_model_weights* w);
 
-tr_status tc_build(tr_model* m, const tr_model_weights* w) {
+template <int D>
+tr_status build_stack_images(tr_model* m, const tr_model_weights* w) {
+  using C = Cfg<D>;
   const tr_model_desc& d = m->desc;
-  TR_TRY(tc_build_comp(m, w));
-  if (!(d.dtype == TR_BF16 && d.D == kD && d.ffn_hidden == kH && d.n_head == 8)) return TR_OK;
-  const int N = d.n_layer, D = kD, H = kH;
-  const size_t se = kSlot / 2;  // elements per stream slot
-  std::vector<uint16_t> img((size_t)N * kItemsPerLayer * se, 0);
-  std::vector<float> vec((size_t)N * kVecPerLayer + kVecFinal, 0.f);
+  const int N = d.n_layer;
+  std::vector<uint8_t> img((size_t)N * C::kItems * C::kItemBytes, 0);
+  std::vector<float> vec((size_t)N * vec_per_layer<D>() + D + 4, 0.f);
   for (int l = 0; l < N; ++l) {
-    // weights go in unchanged (exact bf16 values); LayerNorm gains/shifts stay fp32 in the
-    // epilogue; biases become bias tiles next to the last slice of their GEMM
+    build_layer_items<D>(img.data() + (size_t)l * C::kItems * C::kItemBytes, w->layers[l]);
     const tr_layer_weights& L = w->layers[l];
-    uint16_t* li = img.data() + (size_t)l * kItemsPerLayer * se;
-    // item j: slice (K 0-63) | slice (K 64-127) | bias tile
-    auto half = [&](int j, int h) { return li + (size_t)j * se + (size_t)h * (kChunk / 2); };
-    auto bias = [&](int j) { return li + (size_t)j * se + kChunk; };
-    const float* Wn[4] = {L.Wq, L.Wk, L.Wv, L.Wo};
-    const float* bn[4] = {L.bq, L.bk, L.bv, L.bo};
-    for (int j = 0; j < 4; ++j) {
-      put_chunk(half(j, 0), Wn[j], D, 0, 0);
-      put_chunk(half(j, 1), Wn[j], D, 0, 64);
-      put_bias(bias(j), bn[j], 0);
-    }
-    for (int j = 0; j < 2; ++j) {   // W1, output columns 128 j .. 128 j + 127
-      put_chunk(half(4 + j, 0), L.W1, H, 128 * j, 0);
-      put_chunk(half(4 + j, 1), L.W1, H, 128 * j, 64);
-      put_bias(bias(4 + j), L.b1, 128 * j);
-    }
-    for (int q = 0; q < 4; ++q) put_chunk(half(6 + q / 2, q % 2), L.W2, D, 0, 64 * q);
-    put_bias(bias(7), L.b2, 0);
-    float* v = vec.data() + (size_t)l * kVecPerLayer;
+    float* v = vec.data() + (size_t)l * vec_per_layer<D>();
     for (int j = 0; j < D; ++j) {
       v[j] = L.ln1_g[j];
       v[D + j] = L.ln1_b[j];
@@ -956,14 +1010,14 @@ tr_status tc_build(tr_model* m, const tr_model_weights* w) {
       v[3 * D + j] = L.ln2_b[j];
     }
   }
-  float* vf = vec.data() + (size_t)N * kVecPerLayer;
+  float* vf = vec.data() + (size_t)N * vec_per_layer<D>();
   double bh = w->b_head;
   for (int j = 0; j < D; ++j) {
     vf[j] = (float)((double)w->w_head[j] * w->lnf_g[j]);
     bh += (double)w->w_head[j] * w->lnf_b[j];
   }
   vf[D] = (float)bh;
-  const size_t img_bytes = img.size() * 2, vec_bytes = vec.size() * 4;
+  const size_t img_bytes = img.size(), vec_bytes = vec.size() * 4;
   const size_t total = img_bytes + ((vec_bytes + 255) & ~size_t(255));
   if (cudaMalloc(&m->tc_blob, total) != cudaSuccess) {
     cudaGetLastError();
@@ -973,83 +1027,132 @@ tr_status tc_build(tr_model* m, const tr_model_weights* w) {
   TR_CUDA_TRY(cudaMemcpy(m->tc_blob, img.data(), img_bytes, cudaMemcpyHostToDevice));
   TR_CUDA_TRY(cudaMemcpy((uint8_t*)m->tc_blob + img_bytes, vec.data(), vec_bytes, cudaMemcpyHostToDevice));
   m->tc_stack = m->tc_blob;
-  m->tc_stack_layer_bytes = (size_t)kItemsPerLayer * kSlot;
+  m->tc_stack_layer_bytes = (size_t)C::kItems * C::kItemBytes;
   m->tc_vec = reinterpret_cast<const float*>((uint8_t*)m->tc_blob + img_bytes);
-  m->tc_vec_layer_floats = kVecPerLayer;
+  m->tc_vec_layer_floats = vec_per_layer<D>();
   return TR_OK;
 }
 
-int hg_of(int L_u) {
-  const int Lp = (L_u + 15) & ~15;
-  return Lp <= 16 ? 8 : Lp <= 32 ? 4 : Lp <= 64 ? 2 : 1;
+tr_status tc_build(tr_model* m, const tr_model_weights* w) {
+  const tr_model_desc& d = m->desc;
+  TR_TRY(tc_build_comp(m, w));
+  if (!(d.dtype == TR_BF16 && (d.D == 64 || d.D == 128) && d.ffn_hidden == 2 * d.D && d.n_head * 16 == d.D))
+    return TR_OK;
+  if (!fp16_operands_safe(d, w)) return TR_OK;    // the CUDA-core path serves this model
+  return d.D == 128 ? build_stack_images<128>(m, w) : build_stack_images<64>(m, w);
 }
 
-template <bool PF>
-tr_status launch_stack(int hg, int grid, const StackParams& p, cudaStream_t st) {
-  void (*k)(StackParams) = hg == 8 ? stack_kernel<PF, 8> : hg == 4 ? stack_kernel<PF, 4>
-                         : hg == 2 ? stack_kernel<PF, 2> : stack_kernel<PF, 1>;
-  TR_TRY(ensure_smem_attr((const void*)k, SMEM_BYTES));
-  k<<<grid, kThreads, SMEM_BYTES, st>>>(p);
-  TR_LAUNCH_CHECK(PF ? "stack_kernel (user side)" : "stack_kernel");
+namespace {
+
+// Shared-memory layout of one launch; false when it does not fit.
+template <int D>
+bool plan_smem(StackParams& p, int n_layer, int lp_max, bool pair, int& smem_bytes) {
+  const int a_bytes = (pair ? 2 : 1) * kM * D * 2;
+  p.off_kv = a_bytes;
+  const int kv_bytes = 2 * lp_max * D * 2;
+  p.off_ones = p.off_kv + ((kv_bytes + 1023) & ~1023);
+  p.off_ring = p.off_ones + kM * 16 * 2;
+  const int vec_bytes = (n_layer * vec_per_layer<D>() + D + 4) * 4;
+  const int fixed = p.off_ring + kBarArea;
+  int stages = std::min(kMaxStages, (kSmemLimit - fixed - vec_bytes) / Cfg<D>::kItemBytes);
+  bool vec_in_smem = true;
+  if (stages < 2) {
+    vec_in_smem = false;
+    stages = std::min(kMaxStages, (kSmemLimit - fixed) / Cfg<D>::kItemBytes);
+  }
+  if (stages < 2) return false;
+  p.stages = stages;
+  int off = p.off_ring + stages * Cfg<D>::kItemBytes;
+  if (vec_in_smem) {
+    p.off_vec = off;
+    off += (vec_bytes + 15) & ~15;
+  } else {
+    p.off_vec = -1;
+  }
+  p.off_bar = off;
+  smem_bytes = off + kBarArea;
+  return smem_bytes <= kSmemLimit;
+}
+
+template <int D, int SW, bool UM>
+tr_status launch(int grid, const StackParams& p, int smem, cudaStream_t st) {
+  auto k = stack_kernel<D, SW, UM>;
+  TR_TRY(ensure_smem_attr((const void*)k, kSmemLimit));
+  k<<<grid, kThreads, smem, st>>>(p);
+  TR_LAUNCH_CHECK(UM ? "stack_kernel (user side)" : "stack_kernel");
   return TR_OK;
 }
+
+template <int D>
+tr_status score_launch(const tr_model* m, const void* tokens, const int64_t* req_offsets, const void* const* kv,
+                       const int32_t* L_u, const int32_t* domain, int R, float* scores, cudaStream_t st) {
+  DeviceState* ds = nullptr;
+  TR_TRY(device_state(&ds));
+  StackParams p{};
+  p.tokens = static_cast<const float*>(tokens);
+  p.scores = scores;
+  p.wimg = static_cast<const uint8_t*>(m->tc_stack);
+  p.vec = m->tc_vec;
+  p.domain_emb = m->domain_emb;
+  p.status = ds->status;
+  p.n_layer = m->desc.n_layer;
+  p.pair = 1;
+  int units = 0, k = 0, lp_max = 0;
+  for (int r = 0; r < R; ++r) {
+    const int64_t nr = req_offsets[r + 1] - req_offsets[r];
+    if (nr == 0) continue;
+    p.req[k].kv = static_cast<const uint8_t*>(kv[r]);
+    p.req[k].cand_off = req_offsets[r];
+    p.req[k].n = nr;
+    p.req[k].unit_off = units;
+    p.req[k].L_u = L_u[r];
+    p.req[k].domain = domain[r];
+    lp_max = std::max(lp_max, round_up16(L_u[r]));
+    units += (int)((nr + 2 * kM - 1) / (2 * kM));
+    ++k;
+  }
+  if (units == 0) return TR_OK;
+  p.R = k;
+  p.n_units = units;
+  int smem = 0;
+  const int sw = lp_max <= 32 ? 32 : lp_max <= 64 ? 64 : kMaxLp;   // head slot width of this launch
+  if (!plan_smem<D>(p, p.n_layer, sw, true, smem))
+    return fail(TR_ERR_UNSUPPORTED, "stack kernel: %d layers do not fit shared memory", p.n_layer);
+  int sms = 148, dev = 0;
+  TR_CUDA_TRY(cudaGetDevice(&dev));
+  TR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const int grid = std::min(units, sms);
+  return sw == 32 ? launch<D, 32, false>(grid, p, smem, st)
+       : sw == 64 ? launch<D, 64, false>(grid, p, smem, st)
+                  : launch<D, kMaxLp, false>(grid, p, smem, st);
+}
+
+}  // namespace
 
 tr_status tc_score(const tr_model* m, const void* tokens, int64_t n, const int64_t* req_offsets,
                    const void* const* kv, const int32_t* L_u, const int32_t* domain, int R, float* scores,
                    cudaStream_t st) {
   bool fits = true;
-  for (int r = 0; r < R; ++r) fits = fits && L_u[r] <= kMaxLpTc;
+  for (int r = 0; r < R; ++r) fits = fits && L_u[r] <= kMaxLp;
   if (!fits) {  // long user sequences: CUDA-core path
     for (int r = 0; r < R; ++r)
       TR_TRY(simt_score(m, tokens, req_offsets[r], req_offsets[r + 1], kv[r], L_u[r], domain[r], scores, st));
     return TR_OK;
   }
-  DeviceState* ds = nullptr;
-  TR_TRY(device_state(&ds));
   if ((uintptr_t)tokens % 16) return fail(TR_ERR_INVALID_ARG, "tokens not 16-byte aligned");
   for (int r = 0; r < R; ++r)
     if ((uintptr_t)kv[r] % 16 && L_u[r] > 0 && req_offsets[r + 1] > req_offsets[r])
       return fail(TR_ERR_INVALID_ARG, "kv[%d] is not 16-byte aligned", r);
-  int sms = 148, dev = 0;
-  TR_CUDA_TRY(cudaGetDevice(&dev));
-  TR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  // one launch per head-group size (requests of one class share the kernel's code path)
-  for (int hg : {2, 1, 4, 8}) {
-    StackParams p{};
-    p.tokens = static_cast<const __nv_bfloat16*>(tokens);
-    p.scores = scores;
-    p.wimg = static_cast<const uint8_t*>(m->tc_stack);
-    p.vec = m->tc_vec;
-    p.domain_emb = m->domain_emb;
-    p.status = ds->status;
-    p.n_layer = m->desc.n_layer;
-    int tiles = 0, k = 0;
-    for (int r = 0; r < R; ++r) {
-      const int64_t nr = req_offsets[r + 1] - req_offsets[r];
-      if (hg_of(L_u[r]) != hg || nr == 0) continue;
-      p.req[k].kv = static_cast<const uint8_t*>(kv[r]);
-      p.req[k].cand_off = req_offsets[r];
-      p.req[k].n = nr;
-      p.req[k].tile_off = tiles;
-      p.req[k].L_u = L_u[r];
-      p.req[k].domain = domain[r];
-      tiles += (int)((nr + kM - 1) / kM);
-      ++k;
-    }
-    if (tiles == 0) continue;
-    p.R = k;
-    p.n_tiles = tiles;
-    TR_TRY(launch_stack<false>(hg, std::min(tiles, sms), p, st));
-  }
-  return TR_OK;
+  return m->desc.D == 128 ? score_launch<128>(m, tokens, req_offsets, kv, L_u, domain, R, scores, st)
+                          : score_launch<64>(m, tokens, req_offsets, kv, L_u, domain, R, scores, st);
 }
 
-bool tc_prefill_supported(const tr_model* m, int L_u) { return tc_stack_supported(m) && L_u <= kMaxLpTc; }
+bool tc_prefill_supported(const tr_model* m, int L_u) { return tc_stack_supported(m) && L_u <= kMaxLp; }
 
-// User side of one request through the same kernel (one CTA, the user tokens as its tile).
-tr_status tc_prefill(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv, cudaStream_t st) {
-  if ((uintptr_t)kv % 16 || (uintptr_t)user_tokens % 16)
-    return fail(TR_ERR_INVALID_ARG, "user_tokens / kv not 16-byte aligned");
+// User sides of R requests through the same kernel: one CTA per request (with L_u > 0), the
+// request's user tokens as its tile.
+tr_status tc_prefill_batch(const tr_model* m, const float* const* user_tokens, const int32_t* L_u,
+                           const int32_t* domain, void* const* kv, int R, cudaStream_t st) {
   DeviceState* ds = nullptr;
   TR_TRY(device_state(&ds));
   StackParams p{};
@@ -1058,16 +1161,36 @@ tr_status tc_prefill(const tr_model* m, const float* user_tokens, int L_u, int d
   p.domain_emb = m->domain_emb;
   p.status = ds->status;
   p.n_layer = m->desc.n_layer;
-  p.R = 1;
-  p.n_tiles = 1;
-  p.utokens = user_tokens;
-  p.kv_out = static_cast<uint8_t*>(kv);
-  p.req[0].cand_off = 0;
-  p.req[0].n = L_u;
-  p.req[0].tile_off = 0;
-  p.req[0].L_u = L_u;
-  p.req[0].domain = domain;
-  return launch_stack<true>(hg_of(L_u), 1, p, st);
+  p.pair = 0;
+  int k = 0;
+  for (int r = 0; r < R; ++r) {
+    if (L_u[r] == 0) continue;
+    if ((uintptr_t)kv[r] % 16 || (uintptr_t)user_tokens[r] % 16)
+      return fail(TR_ERR_INVALID_ARG, "request %d: user_tokens / kv not 16-byte aligned", r);
+    p.req[k].kv = static_cast<const uint8_t*>(kv[r]);
+    p.req[k].utokens = user_tokens[r];
+    p.req[k].cand_off = 0;
+    p.req[k].n = L_u[r];
+    p.req[k].unit_off = k;
+    p.req[k].L_u = L_u[r];
+    p.req[k].domain = domain[r];
+    ++k;
+  }
+  if (k == 0) return TR_OK;
+  p.R = k;
+  p.n_units = k;
+  int smem = 0;
+  const bool fit = m->desc.D == 128 ? plan_smem<128>(p, p.n_layer, kMaxLp, false, smem)
+                                    : plan_smem<64>(p, p.n_layer, kMaxLp, false, smem);
+  if (!fit) return fail(TR_ERR_UNSUPPORTED, "stack kernel: %d layers do not fit shared memory", p.n_layer);
+  return m->desc.D == 128 ? launch<128, kMaxLp, true>(k, p, smem, st) : launch<64, kMaxLp, true>(k, p, smem, st);
+}
+
+// User side of one request (one CTA).
+tr_status tc_prefill(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv, cudaStream_t st) {
+  const int32_t lu = L_u, dm = domain;
+  void* kvp = kv;
+  return tc_prefill_batch(m, &user_tokens, &lu, &dm, &kvp, 1, st);
 }
 
 }  // namespace tr

@@ -36,17 +36,27 @@ class DeviceBags:
                           _dev(b.weights.astype(np.float32), device), _dev(b.bag_table.astype(np.int32), device))
 
 
-def pack_target_bags(reqs: List["datagen.Request"]) -> "datagen.Bags":
+def _pack(bag_sets) -> "datagen.Bags":
     offs, keys, wts, tabs = [np.zeros(1, np.int64)], [], [], []
     base = 0
-    for r in reqs:
-        b = r.target
+    for b in bag_sets:
         offs.append(b.offsets[1:] + base)
         base += b.nnz
         keys.append(b.keys)
         wts.append(b.weights)
         tabs.append(b.bag_table)
     return datagen.Bags(np.concatenate(offs), np.concatenate(keys), np.concatenate(wts), np.concatenate(tabs))
+
+
+def pack_target_bags(reqs: List["datagen.Request"]) -> "datagen.Bags":
+    """Every request's target bags, one after the other (candidate order)."""
+    return _pack([r.target for r in reqs])
+
+
+def pack_user_bags(reqs: List["datagen.Request"]) -> "datagen.Bags":
+    """Every request's user-field bags, one after the other (request r's fields follow those
+    of requests 0 .. r-1)."""
+    return _pack([r.user for r in reqs])
 
 
 class DeviceWorkload:
@@ -83,7 +93,7 @@ class DeviceWorkload:
     def set_requests(self, reqs) -> None:
         w, dims, dev = self.w, self.w.dims, self.device
         self.reqs = reqs
-        self.user_bags = [DeviceBags.of(r.user, dev) for r in reqs]
+        self.user_bags = DeviceBags.of(pack_user_bags(reqs), dev)
         self.target_bags = DeviceBags.of(pack_target_bags(reqs), dev)
         self.L_u = [r.L_u for r in reqs]
         self.domain = [r.domain for r in reqs]
@@ -93,11 +103,16 @@ class DeviceWorkload:
         self.req_offsets = off
         n = off[-1]
         D, F = dims.D, dims.n_target_fields
-        self.user_tokens = [torch.empty(max(l, 1), D, dtype=torch.float32, device=dev) for l in self.L_u]
+        # every request's user tokens in one buffer (one aggregation call fills them all)
+        uoff = np.concatenate([[0], np.cumsum(self.L_u)]).astype(int)
+        self.user_tokens_all = torch.empty(max(int(uoff[-1]), 1), D, dtype=torch.float32, device=dev)
+        self.user_tokens = [self.user_tokens_all[uoff[r]:uoff[r] + max(l, 1)] if l else self.user_tokens_all[:1]
+                            for r, l in enumerate(self.L_u)]
+        self.n_user = int(uoff[-1])
         self.kv = [torch.empty(max(api.kv_cache_bytes(self.model, l), 16), dtype=torch.uint8, device=dev)
                    for l in self.L_u]
         self.X = torch.empty(n, F * D, dtype=self.dt, device=dev)
-        self.tokens = torch.empty(n, D, dtype=self.dt, device=dev)
+        self.tokens = torch.empty(n, D, dtype=torch.float32, device=dev)     # compressed tokens (fp32)
         self.scores = torch.empty(n, dtype=torch.float32, device=dev)
 
     @property
@@ -109,22 +124,21 @@ class DeviceWorkload:
         candidate counts as the current ones (no reallocation of activations)."""
         if [r.L_u for r in reqs] != self.L_u or [r.n_cand for r in reqs] != [r.n_cand for r in self.reqs]:
             raise ValueError("use_bags: requests differ in L_u or candidate count; call set_requests")
-        self.user_bags, self.target_bags, self.reqs = list(user_bags), target_bags, reqs
+        self.user_bags, self.target_bags, self.reqs = user_bags, target_bags, reqs
         self.domain = [r.domain for r in reqs]
 
     # -------------------------------------------------------------- the step
     def user_aggregate(self, stream=None) -> None:
-        for r, b in enumerate(self.user_bags):
-            if self.L_u[r] == 0:
-                continue
-            api.aggregate(self.user_tables, b.bag_table, b.offsets, b.keys, b.weights, self.user_tokens[r],
-                          stream=stream)
+        """Every request's user fields in one tr_aggregate call."""
+        if self.n_user:
+            b = self.user_bags
+            api.aggregate(self.user_tables, b.bag_table, b.offsets, b.keys, b.weights,
+                          self.user_tokens_all[:self.n_user], stream=stream)
 
     def user_prefill(self, stream=None) -> None:
-        for r in range(len(self.user_bags)):
-            if self.L_u[r] == 0:
-                continue
-            api.prefill_user(self.model, self.user_tokens[r], self.L_u[r], self.domain[r], self.kv[r], stream=stream)
+        """Every request's user side in one tr_prefill_users call."""
+        if self.n_user:
+            api.prefill_users(self.model, self.user_tokens, self.L_u, self.domain, self.kv, stream=stream)
 
     def user_side(self, stream=None) -> None:
         self.user_aggregate(stream)
@@ -249,41 +263,42 @@ def warm_up_stream(stream, run) -> None:
 
 
 SCORE_TILE = 128   # candidates per tile of the tensor-core score kernel
+SCORE_UNIT = 2     # tiles of one request that a CTA of the score kernel holds at a time
 
 
-def score_split(req_offsets, n_sms: int, tile: int = SCORE_TILE):
-    """The packed candidate index at which the score kernel's last, partial wave of tiles
-    begins, or None when it has none.  The kernel cuts every request into tiles of
-    ``tile`` candidates, in request order, and runs one persistent CTA per SM that takes
-    tiles b, b + n_sms, b + 2 n_sms, ...; with T tiles and T mod n_sms = t > 0 (and more
-    than one wave), the last t tiles form a wave of their own on t SMs while the other SMs
-    wait.  The split index lies on a tile boundary of its request.  The score kernel runs
-    one launch per class of requests with the same heads per score group (L_u up to 16,
-    32, 64, 128), so for a batch that mixes classes the cut is a good guess rather than
-    the exact wave boundary; either way both parts are valid batches and the scores do not
-    change."""
-    tiles = [-(-(req_offsets[r + 1] - req_offsets[r]) // tile) for r in range(len(req_offsets) - 1)]
-    T = sum(tiles)
-    if n_sms <= 0 or T <= n_sms or T % n_sms == 0:
+def score_split(req_offsets, n_sms: int, tile: int = SCORE_TILE, unit: int = SCORE_UNIT):
+    """The packed candidate index at which the score kernel's last, partial round of work
+    begins, or None when it has none.  The kernel cuts every request into tiles of ``tile``
+    candidates and groups a request's tiles into units of ``unit`` consecutive tiles (its last
+    unit may be shorter), in request order; one persistent CTA per SM takes units b,
+    b + n_sms, b + 2 n_sms, ...  With U units and U mod n_sms = u > 0 (and more than one
+    round), the last u units form a round of their own on u SMs while the other SMs wait.
+    The split index lies on a unit boundary of its request.  Both parts are valid batches
+    and the scores do not change."""
+    per = tile * unit
+    units = [-(-(req_offsets[r + 1] - req_offsets[r]) // per) for r in range(len(req_offsets) - 1)]
+    U = sum(units)
+    if n_sms <= 0 or U <= n_sms or U % n_sms == 0:
         return None
-    cut = T - T % n_sms
+    cut = U - U % n_sms
     acc = 0
-    for r, t in enumerate(tiles):
-        if acc + t == cut:
+    for r, u in enumerate(units):
+        if acc + u == cut:
             return req_offsets[r + 1]
-        if acc + t > cut:
-            return req_offsets[r] + (cut - acc) * tile
-        acc += t
+        if acc + u > cut:
+            return req_offsets[r] + (cut - acc) * per
+        acc += u
     return None
 
 
 class Overlapped:
     """Request batches scored back to back, consecutive batches overlapped on the device.
 
-    The compressor and the score kernel both cut the batch into 128-candidate tiles and
-    run one persistent CTA per SM, so a batch whose tile count is not a multiple of the SM
-    count ends each of them with a partial wave that leaves most SMs idle.  Here a batch
-    is cut at score_split into a head (the full waves) and a tail:
+    The compressor and the score kernel both run one persistent CTA per SM over the batch
+    (the compressor one 128-candidate tile at a time, the score kernel two), so a batch whose
+    work is not a multiple of the SM count ends each of them with a partial round that leaves
+    most SMs idle.  Here a batch is cut at score_split into a head (the full rounds of the
+    score kernel) and a tail:
       main stream  user aggregation -> target aggregation -> compress(head) -> score(head)
       user stream  (high priority) user prefill, joined before score(head)
       back stream  (high priority) compress(tail) -> score(tail), after score(head)
@@ -388,28 +403,26 @@ class HostFeed:
     batch i computes (two device slots, guarded by events); each batch's scores are copied
     back to a pinned host buffer on the compute stream.
 
-    ``batches``: list of (user bags per request, target bags, requests), every bag tensor in
-    pinned host memory; all batches have the requests' L_u and candidate counts of ``dw``.
+    ``batches``: list of (user bags, target bags, requests) -- each the requests' bags packed
+    as pack_user_bags / pack_target_bags do, every tensor in pinned host memory; all batches
+    have the requests' L_u and candidate counts of ``dw``.
     """
 
     def __init__(self, dw: DeviceWorkload, batches):
         self.dw = dw
         self.batches = batches
         dev = dw.device
-        n_req = len(batches[0][0])
         self.slots = []
         for _ in range(2):   # device buffers with the largest size any batch needs
             def alloc(pick):
                 return DeviceBags(*(torch.empty(max(int(getattr(pick(bt), f).numel()) for bt in batches),
                                                 dtype=getattr(pick(batches[0]), f).dtype, device=dev)
                                     for f in ("offsets", "keys", "weights", "bag_table")))
-            users = [alloc(lambda bt, r=r: bt[0][r]) for r in range(n_req)]
-            target = alloc(lambda bt: bt[1])
-            self.slots.append((users, target))
+            self.slots.append((alloc(lambda bt: bt[0]), alloc(lambda bt: bt[1])))
         self.copy_stream = torch.cuda.Stream(dev)
         self.ready = [torch.cuda.Event() for _ in range(2)]
         self.free = [torch.cuda.Event() for _ in range(2)]
-        self.h2d_bytes = [sum(x.numel() * x.element_size() for b in bt[0] + [bt[1]] for x in _bag_tensors(b))
+        self.h2d_bytes = [sum(x.numel() * x.element_size() for b in (bt[0], bt[1]) for x in _bag_tensors(b))
                           for bt in batches]
 
     def _views(self, i):
@@ -419,7 +432,7 @@ class HostFeed:
 
         def fit(dst, src):
             return DeviceBags(*(d[:s.numel()] for d, s in zip(_bag_tensors(dst), _bag_tensors(src))))
-        return [fit(d, h) for d, h in zip(users, hu)], fit(target, ht)
+        return fit(users, hu), fit(target, ht)
 
     def _copy_in(self, i):
         hu, ht, _ = self.batches[i % len(self.batches)]
@@ -427,7 +440,7 @@ class HostFeed:
         cs = self.copy_stream
         cs.wait_event(self.free[i % 2])            # batch i - 2 is done with this slot
         with torch.cuda.stream(cs):
-            for d, h in zip(du + [dt], hu + [ht]):
+            for d, h in ((du, hu), (dt, ht)):
                 for dx, hx in zip(_bag_tensors(d), _bag_tensors(h)):
                     dx.copy_(hx, non_blocking=True)
         self.ready[i % 2].record(cs)
@@ -506,7 +519,7 @@ class HostFeed:
             for i in range(first, first + count):
                 hu, ht, _ = self.batches[i % len(self.batches)]
                 du, dt = self._views(i)
-                for d, h in zip(du + [dt], hu + [ht]):
+                for d, h in ((du, hu), (dt, ht)):
                     for dx, hx in zip(_bag_tensors(d), _bag_tensors(h)):
                         dx.copy_(hx, non_blocking=True)
                 host_scores[i % len(host_scores)].copy_(scores, non_blocking=True)
@@ -527,11 +540,12 @@ def compress_corpus(model, target_tables, bags: DeviceBags, n_items: int, n_fiel
     """Near-line index build (TransRetrieval §3.3: the compressed target token is also the
     item's index vector, computed off the request path): every item of a corpus, its
     ``n_fields`` target-field bags aggregated (tr_aggregate) and compressed
-    (tr_compress_targets) into ``out`` [n_items, D], ``chunk`` items at a time through one
-    [chunk, F*D] buffer.  ``bags`` holds the corpus's bags on the device, item i's fields at
-    bags i*F .. i*F+F-1 (CSR offsets into the full key/weight arrays)."""
+    (tr_compress_targets) into ``out`` [n_items, D] fp32, ``chunk`` items at a time through one
+    [chunk, F*D] buffer of the model's dtype.  ``bags`` holds the corpus's bags on the device,
+    item i's fields at bags i*F .. i*F+F-1 (CSR offsets into the full key/weight arrays)."""
     D = out.shape[1]
-    X = torch.empty(min(chunk, max(n_items, 1)), n_fields * D, dtype=out.dtype, device=out.device)
+    X = torch.empty(min(chunk, max(n_items, 1)), n_fields * D, dtype=api.torch_dtype(model.dims.dtype),
+                    device=out.device)
     for c0 in range(0, n_items, chunk):
         c1 = min(n_items, c0 + chunk)
         m = c1 - c0
