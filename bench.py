@@ -616,14 +616,30 @@ def run_ours(args, rank, world, local_rank):
 
 def run_case(args):
     """One stage of the 128D-5L path on stand-alone seeded inputs, a few launches, no JSON:
-    the target of profiler captures (small, no tables)."""
+    the target of profiler captures (small inputs; the gather case builds 8 target tables of
+    --case-rows rows, 2 GB at the default 1M, larger than L2)."""
     import torch
 
     from transformer_candidate_scoring_b200 import api
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags
 
     w = datagen.WORKLOADS[WORKLOAD]
     dims = w.dims
     n = args.case_n
+    if args.case == "gather":
+        ws = datagen.scaled(w, n_cand_per_request=n, rows=args.case_rows)
+        tables = [torch.empty(r, dims.D, dtype=torch.bfloat16, device="cuda") for r in ws.target_rows]
+        for t, x in enumerate(tables):
+            datagen.fill_table_device(x, ws.seed, datagen.target_table_id(ws, t))
+        bags = DeviceBags.of(datagen.make_target_bags(np.random.default_rng(ws.seed), ws, n), "cuda")
+        X = torch.empty(n * dims.n_target_fields, dims.D, dtype=torch.bfloat16, device="cuda")
+        for _ in range(args.case_reps):
+            api.aggregate(tables, bags.bag_table, bags.offsets, bags.keys, bags.weights, X)
+        torch.cuda.synchronize()
+        if api.sync_status() != 0:
+            raise RuntimeError("device status word set")
+        print("case gather: ok")
+        return
     m = api.Model(dims, datagen.workload_params(w))
     U = torch.from_numpy(datagen.rand_matrix(1, (64, dims.D), 0.01, "f32")).cuda()
     kv = torch.zeros(api.kv_cache_bytes(m, 64), dtype=torch.uint8, device="cuda")
@@ -729,10 +745,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side-configs", action="store_true", help="skip the 64D-3L, packed and large workloads")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--case", choices=["score", "compress", "prefill", "all", "bulk", "uncompressed"], default=None,
+    ap.add_argument("--case", choices=["score", "compress", "prefill", "all", "gather", "bulk", "uncompressed"],
+                    default=None,
                     help="run one stage on stand-alone inputs for a profiler (no timing, no JSON)")
     ap.add_argument("--case-n", type=int, default=40000)
     ap.add_argument("--case-reps", type=int, default=2)
+    ap.add_argument("--case-rows", type=int, default=1_000_000, help="table rows of the gather case")
     args = ap.parse_args()
     if args.case == "bulk":
         run_bulk(args)

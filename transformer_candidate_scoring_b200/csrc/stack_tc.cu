@@ -105,8 +105,12 @@ struct Cfg<64> {
   __host__ __device__ static constexpr int item_bytes(int j) { return j == 0 ? 40960 : 38912; }
 };
 
+// The LayerNorm gains and shifts are folded into the weights and biases of the products
+// that follow them (K, V, Q after LN1; W1 after LN2): LN(y) W + b = z (g o W) + (beta W + b),
+// z the standardized row.  The epilogue only standardizes; the one vector it still reads is
+// the head's (w o g_f and the folded bias).
 template <int D>
-constexpr int vec_per_layer() { return 4 * D; }   // LN1 gain, LN1 shift, LN2 gain, LN2 shift
+constexpr int vec_floats() { return D + 4; }
 
 // Head groups of one launch: a head's scores take SW work-area columns (SW = 32, 64 or 128,
 // at least the launch's longest padded user sequence), a group is the HG heads that fit.
@@ -125,7 +129,7 @@ struct ReqInfo {
   int unit_off;
   int L_u;
   int domain;
-  int pad;
+  int n_pair;                 // the request's first n_pair units hold two tiles, the rest one
 };
 
 struct StackParams {
@@ -137,6 +141,10 @@ struct StackParams {
   int* status;
   int n_layer, n_units, R, pair;
   int off_kv, off_ring, off_ones, off_vec, off_bar, stages;
+  // where slot 0 lets slot 1 start a unit of two tiles (layer 0): 0 after its own-V phase,
+  // 1 after the attention of its second head group.  Slot 0 alone may run at most `stages`
+  // weight items ahead, so with a two-item ring the gate must open before it needs Q.
+  int gate_phase;
   ReqInfo req[TR_MAX_REQUESTS];
 };
 
@@ -152,10 +160,12 @@ __device__ __forceinline__ Tile tile_of(const StackParams& p, int u, int slot) {
   while (r + 1 < p.R && u >= p.req[r + 1].unit_off) ++r;
   Tile t;
   t.r = r;
-  const long long local = (long long)(u - p.req[r].unit_off) * (p.pair ? 2 : 1) + slot;
+  const int k = u - p.req[r].unit_off, np = p.req[r].n_pair;
+  const bool two = p.pair && k < np;
+  const long long local = two ? 2ll * k + slot : (long long)np + k;   // np pair units, then singles
   t.row0 = p.req[r].cand_off + local * kM;
   const long long end = p.req[r].cand_off + p.req[r].n;
-  t.active = (slot == 0 || p.pair) && t.row0 < end;
+  t.active = (slot == 0 || two) && t.row0 < end;
   t.rows = t.active ? (int)min((long long)kM, end - t.row0) : 0;
   t.L_u = p.req[r].L_u;
   t.Lp = (t.L_u + 15) & ~15;
@@ -175,8 +185,10 @@ struct Bars {
   __device__ __forceinline__ uint32_t m2e(int slot) const { return at(2 * kMaxStages + 5 + slot); }
   __device__ __forceinline__ uint32_t mm(int slot) const { return at(2 * kMaxStages + 7 + slot); }
   __device__ __forceinline__ uint32_t drain(int slot) const { return at(2 * kMaxStages + 9 + slot); }
+  // epilogue turn of slot s (passed between the two slots of a unit)
+  __device__ __forceinline__ uint32_t tok(int slot) const { return at(2 * kMaxStages + 11 + slot); }
 };
-constexpr int kNumBars = 2 * kMaxStages + 11;
+constexpr int kNumBars = 2 * kMaxStages + 13;
 constexpr int kBarArea = 8 * kNumBars + 32;   // + TMEM address and abort flag
 
 // ------------------------------------------------------------------ small helpers
@@ -211,8 +223,46 @@ __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* r) {
       "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
-// Compiler-only barrier: keeps later loads from being hoisted above it.
-__device__ __forceinline__ void step_barrier() { asm volatile("" ::: "memory"); }
+
+// 2^x on the FMA pipe, for the share of the softmax exponentials that the MUFU pipe would
+// otherwise queue: x = n + f with n = round(x) (the 1.5 * 2^23 addition rounds x into t's low
+// bits), 2^f from a cubic fitted to minimise the relative error on [-1/2, 1/2] (7.6e-5, below
+// half an fp16 unit, the precision the numerators are kept in), 2^n added into the exponent
+// field.  Below -125 (masked keys are -inf) the result is 0, so that the exponent field
+// never wraps.
+__device__ __forceinline__ float exp2_fma(float x) {
+  const float xc = fmaxf(x, -125.f);
+  const float t = xc + 12582912.f;
+  const float f = xc - (t - 12582912.f);
+  const float p = fmaf(fmaf(fmaf(0.0551727042f, f, 0.242614001f), f, 0.693261027f), f, 0.999927819f);
+  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x >= -125.f ? r : 0.f;
+}
+
+// The numerator of key chunk c (16 keys): every path and slot width computes the same key
+// with the same function, so that a candidate's score does not depend on the other requests
+// of its launch.
+__device__ __forceinline__ float softmax_exp(float x, int c) { return c == 3 ? exp2_fma(x) : ex2(x); }
+
+// Bounded wait that polls without suspending the thread first (the MMA-issuing threads wait
+// for one event at a time and react faster this way).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+#pragma unroll 1
+  for (int i = 0; i < 4096; ++i)
+    if (mbar_test(bar, parity)) return true;
+  return mbar_wait(bar, parity, abort_flag);
+}
 
 // Bounded wait of one thread for its own bulk copies in flight, used while unwinding.
 __device__ __forceinline__ void settle(uint32_t bar, uint32_t parity) {
@@ -291,7 +341,7 @@ __device__ void mma_issuer(const StackParams& p, int slot, uint32_t tmem, uint32
   uint32_t phase = 0, ph_e = 0, ph_kv = 0, ph_mm = 0;
   bool ok = true, store_pending = false;
   auto wait_e = [&]() {
-    ok = ok && mbar_wait(e2m, ph_e, abort_flag);
+    ok = ok && mbar_wait_spin(e2m, ph_e, abort_flag);
     ph_e ^= 1;
     tc_fence_after();
     return ok;
@@ -310,7 +360,7 @@ __device__ void mma_issuer(const StackParams& p, int slot, uint32_t tmem, uint32
     const bool last = pi == C::kPieces - 1 || C::piece(pi + 1).item != pc.item;
     if (!ok) return;
     if (first) {
-      if (!(ok = mbar_wait(b.full(stage), phase, abort_flag))) return;
+      if (!(ok = mbar_wait_spin(b.full(stage), phase, abort_flag))) return;
       tc_fence_after();
     }
     const uint32_t item = ring + stage * C::kItemBytes;
@@ -433,9 +483,26 @@ struct Epi {
   uint32_t sA, rowoff, sKV;
   int m;
   uint32_t e2m, m2e, ph;
+  uint32_t gate, gph;         // the start gate of slot 1 in a unit of two tiles
+  int slot;
+  bool paired;                 // both slots of the unit hold a tile
   const float* vec;
   volatile int* abort_flag;
   bool ok;
+  // Slot 1 starts a unit of two tiles once slot 0 is well into it (through the attention of
+  // its second head group, or through its own-V phase when the weight ring is two items
+  // deep), so that the two slots' phases interleave: one slot's softmax runs while the
+  // tensor core serves the other slot's projections.
+  __device__ __forceinline__ bool acquire() {
+    if (paired && slot == 1) {
+      ok = ok && mbar_wait(gate, gph, abort_flag);
+      gph ^= 1;
+    }
+    return ok;
+  }
+  __device__ __forceinline__ void open_gate() {
+    if (paired && slot == 0) mbar_arrive(gate);
+  }
   __device__ __forceinline__ bool wait() {
     ok = ok && mbar_wait(m2e, ph, abort_flag);
     ph ^= 1;
@@ -475,19 +542,18 @@ __device__ __forceinline__ float2 row_stats(const float* y) {
   return make_float2(mean, rsqrtf(((a[0] + a[1]) + (a[2] + a[3])) * (1.f / D) + kLnEps));
 }
 
-// LayerNorm of the row -> fp16 A operand row.
+// The row standardized (LayerNorm without its gain and shift, which the next product's
+// weights carry) -> fp16 A operand row.
 template <int D>
-__device__ __forceinline__ void ln_to_A(const Epi& e, const float* y, const float* g, const float* b) {
+__device__ __forceinline__ void ln_to_A(const Epi& e, const float* y) {
   const float2 st = row_stats<D>(y);
+  const float nmr = -st.x * st.y;
 #pragma unroll
   for (int kc = 0; kc < D / 8; ++kc) {
-    float gg[8], bb[8], v[8];
-    ld8(g + 8 * kc, gg);
-    ld8(b + 8 * kc, bb);
+    float v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = fmaf((y[8 * kc + i] - st.x) * st.y, gg[i], bb[i]);
+    for (int i = 0; i < 8; ++i) v[i] = fmaf(y[8 * kc + i], st.y, nmr);
     st_row8h(e.sA + kc * 2048 + e.rowoff, v);
-    step_barrier();
   }
 }
 
@@ -521,9 +587,11 @@ __device__ __forceinline__ float2 softmax_head(uint32_t base, int Lp, int L_u, f
       if (c < nb) tmem_ld16(base + 16 * c, sv + 16 * c);
     tmem_wait_ld();
     reg_fence<SW>(sv);
+    if (L_u < SW) {   // keys past L_u (and unloaded chunks) out of the maximum and the sums
 #pragma unroll
-    for (int i = 0; i < SW; ++i)
-      if (i >= L_u) sv[i] = -INFINITY;
+      for (int i = 0; i < SW; ++i)
+        if (i >= L_u) sv[i] = -INFINITY;
+    }
     float m4[4] = {sself, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
     for (int i = 0; i < SW; i += 8) {
@@ -540,7 +608,8 @@ __device__ __forceinline__ float2 softmax_head(uint32_t base, int Lp, int L_u, f
         uint32_t r[8];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          sv[16 * c + i] = ex2(fmaf(sv[16 * c + i], kL2E, nm));
+          // a quarter of the exponentials (the fourth chunk of 16 keys) on the FMA pipe
+          sv[16 * c + i] = softmax_exp(fmaf(sv[16 * c + i], kL2E, nm), c);
           s4[i & 3] += sv[16 * c + i];
         }
 #pragma unroll
@@ -574,7 +643,7 @@ __device__ __forceinline__ float2 softmax_head(uint32_t base, int Lp, int L_u, f
       uint32_t r[8];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        v[i] = 16 * c + i < L_u ? ex2(fmaf(v[i], kL2E, nm)) : 0.f;
+        v[i] = 16 * c + i < L_u ? softmax_exp(fmaf(v[i], kL2E, nm), c) : 0.f;
         s4[i & 3] += v[i];
       }
 #pragma unroll
@@ -591,6 +660,7 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
   constexpr int NH = Cfg<D>::kNH;
   const int m = e.m;
   const bool live = m < t.rows;
+  if (!e.acquire()) return;
   // ---- Y = token + s_d (rows past the tile's end are zero and never stored)
   {
     float y[D];
@@ -613,12 +683,11 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
   // (Y is re-read from tensor memory at the top of every layer, so that no register copy of
   // it stays live through the layer)
   for (int l = 0; l < p.n_layer; ++l) {
-    const float* vl = e.vec + (size_t)l * vec_per_layer<D>();
-    if (l > 0 && !e.wait()) return;                // the previous layer's FFN product is in Y
+    if (l > 0 && !e.wait()) return;   // the previous layer's FFN product is in Y
     {
       float y[D];
       load_row<D>(e.tY, y);
-      ln_to_A<D>(e, y, vl, vl + D);
+      ln_to_A<D>(e, y);
     }
     e.signal();
     // ---- own K and V (user mode: this row of the layer's K and V^T images), read in two
@@ -669,6 +738,7 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
         }
       }
       e.signal();
+      if (l == 0 && pass == 1 && p.gate_phase == 0) e.open_gate();
     }
     // ---- Q (pre-scaled by 1/sqrt(d_h) through its weights) -> A; own score per head
     float sself[NH];
@@ -709,21 +779,21 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
       }
     }
     e.signal();
-    // ---- attention, one head group at a time
+    if (l == 0 && t.Lp == 0 && p.gate_phase == 1) e.open_gate();
+    // ---- attention, one head group at a time (loops kept rolled: the heads of a group are
+    // picked out of the per-head registers by comparison, which keeps the code small)
     constexpr int HG = Groups<D, SW>::HG;
     if (t.Lp > 0) {
-#pragma unroll
+#pragma unroll 1
       for (int g = 0; g < Groups<D, SW>::NG; ++g) {
         float ps[HG], li[HG];
-        if (!e.wait()) return;                     // scores of group g
-        // one head after the other (not interleaved by the compiler: that would hold several
-        // heads' scores in registers at once)
+        if (!e.wait()) return;   // scores of group g
 #pragma unroll 1
         for (int i = 0; i < HG; ++i) {
-          float ss = sself[g * HG];
+          const int h = g * HG + i;
+          float ss = sself[0];
 #pragma unroll
-          for (int k = 1; k < HG; ++k)
-            if (i == k) ss = sself[g * HG + k];
+          for (int k = 1; k < NH; ++k) ss = h == k ? sself[k] : ss;
           const float2 r = softmax_head<SW>(e.tW + i * SW, t.Lp, t.L_u, ss);
 #pragma unroll
           for (int k = 0; k < HG; ++k)
@@ -733,7 +803,7 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
             }
         }
         e.signal();
-        if (!e.wait()) return;                     // P V of group g
+        if (!e.wait()) return;   // P V of group g
 #pragma unroll
         for (int i = 0; i < HG; ++i) {
           const int h = g * HG + i;
@@ -741,28 +811,36 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
           tmem_ld16(e.tW + i * SW + SW / 2, o);
           tmem_wait_ld();
           reg_fence<16>(o);
+          if constexpr (UM) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if constexpr (UM) {
-              o[2 * j] *= li[i];
-              o[2 * j + 1] *= li[i];
-            } else {
-              o[2 * j] = fmaf(ps[i], h_lo(vreg[8 * h + j]), o[2 * j]) * li[i];
-              o[2 * j + 1] = fmaf(ps[i], h_hi(vreg[8 * h + j]), o[2 * j + 1]) * li[i];
+            for (int j = 0; j < 16; ++j) o[j] *= li[i];
+          } else {
+            uint32_t vv[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              vv[j] = vreg[j];
+#pragma unroll
+              for (int k = 1; k < NH; ++k) vv[j] = h == k ? vreg[8 * k + j] : vv[j];
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              o[2 * j] = fmaf(ps[i], h_lo(vv[j]), o[2 * j]) * li[i];
+              o[2 * j + 1] = fmaf(ps[i], h_hi(vv[j]), o[2 * j + 1]) * li[i];
             }
           }
           st_row8h(e.sA + (2 * h) * 2048 + e.rowoff, o);
           st_row8h(e.sA + (2 * h + 1) * 2048 + e.rowoff, o + 8);
         }
         e.signal();
+        if (l == 0 && g == (Groups<D, SW>::NG > 1 ? 1 : 0) && p.gate_phase == 1) e.open_gate();
       }
     }
     // ---- LN2 -> A
-    if (!e.wait()) return;                         // Y += attn Wo + bo
+    if (!e.wait()) return;        // Y += attn Wo + bo
     {
       float y[D];
       load_row<D>(e.tY, y);
-      ln_to_A<D>(e, y, vl + 2 * D, vl + 3 * D);
+      ln_to_A<D>(e, y);
     }
     e.signal();
     // ---- ReLU(hidden) -> fp16 A operand in the work area, a 128-unit half at a time
@@ -779,7 +857,7 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
   float y[D];
   load_row<D>(e.tY, y);
   const float2 st = row_stats<D>(y);
-  const float* vf = e.vec + (size_t)p.n_layer * vec_per_layer<D>();
+  const float* vf = e.vec;
   float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int c = 0; c < D / 8; ++c) {
@@ -805,11 +883,15 @@ __device__ void epilogue(const StackParams& p, int slot, uint32_t tmem, uint32_t
   e.e2m = b.e2m(slot);
   e.m2e = b.m2e(slot);
   e.ph = 0;
+  e.gate = b.tok(0);
+  e.gph = 0;
+  e.slot = slot;
   e.vec = vec;
   e.abort_flag = abort_flag;
   e.ok = true;
   for (int u = blockIdx.x; u < p.n_units && e.ok; u += gridDim.x) {
     const Tile t = tile_of<D>(p, u, slot);
+    e.paired = p.pair && tile_of<D>(p, u, 1).active;
     if (t.active) epi_tile<D, SW, UM>(p, t, e);
   }
 }
@@ -837,6 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       mbar_init(b.m2e(s), 1);
       mbar_init(b.mm(s), 1);
       mbar_init(b.drain(s), 1);
+      mbar_init(b.tok(s), kSlotThreads);
     }
     *abort_flag = 0;
     mbar_fence_init();
@@ -855,7 +938,7 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       st_row8h(sOnes + 2048 + ro, zero);
     }
     if (p.off_vec >= 0) {
-      const int nvec = p.n_layer * vec_per_layer<D>() + D + 4;
+      const int nvec = vec_floats<D>();
       float* sv = reinterpret_cast<float*>(smem + p.off_vec);
       for (int i = t; i < nvec; i += 2 * kSlotThreads) sv[i] = __ldg(p.vec + i);
     }
@@ -922,37 +1005,62 @@ void put_bias(uint16_t* dst, const float* bias, int n0, int N, float scale) {
   }
 }
 
+// W' = diag(g) W scale and b' = (beta W + b) scale for a product that follows a LayerNorm with
+// gain g and shift beta (fp64 on the host; W [K][ld] row-major, columns n0 .. n0 + N - 1).
+void fold_ln(const float* W, int ld, int n0, int K, int N, const float* g, const float* beta, const float* bias,
+             float scale, std::vector<float>& Wf, std::vector<float>& bf) {
+  Wf.assign((size_t)K * N, 0.f);
+  bf.assign(N, 0.f);
+  for (int n = 0; n < N; ++n) {
+    double acc = bias[n0 + n];
+    for (int k = 0; k < K; ++k) {
+      const double w = W[(size_t)k * ld + n0 + n];
+      Wf[(size_t)k * N + n] = (float)(w * g[k] * scale);
+      acc += (double)beta[k] * w;
+    }
+    bf[n] = (float)(acc * scale);
+  }
+}
+
 template <int D>
 void build_layer_items(uint8_t* li, const tr_layer_weights& L) {
   using C = Cfg<D>;
   const int H = 2 * D;
-  // Q's weights and bias carry 1/sqrt(d_h) = 1/4 (exact in floating point)
-  const float* Wn[4] = {L.Wk, L.Wv, L.Wq, L.Wo};
-  const float* bn[4] = {L.bk, L.bv, L.bq, L.bo};
-  const float sc[4] = {1.f, 1.f, 0.25f, 1.f};
   auto at = [&](int pi, int off) {
     const Piece pc = C::piece(pi);
     return reinterpret_cast<uint16_t*>(li + (size_t)pc.item * C::kItemBytes + off);
   };
-  for (int j = 0; j < 4; ++j) {
+  std::vector<float> Wf, bf;
+  // K, V, Q follow LN1; Q's weights and bias also carry 1/sqrt(d_h) = 1/4
+  const float* Wn[3] = {L.Wk, L.Wv, L.Wq};
+  const float* bn[3] = {L.bk, L.bv, L.bq};
+  const float sc[3] = {1.f, 1.f, 0.25f};
+  for (int j = 0; j < 3; ++j) {
     const Piece pc = C::piece(j);
-    put_B(at(j, pc.off), Wn[j], D, 0, 0, D, D, sc[j]);
-    put_bias(at(j, pc.bias), bn[j], 0, D, sc[j]);
+    fold_ln(Wn[j], D, 0, D, D, L.ln1_g, L.ln1_b, bn[j], sc[j], Wf, bf);
+    put_B(at(j, pc.off), Wf.data(), D, 0, 0, D, D, 1.f);
+    put_bias(at(j, pc.bias), bf.data(), 0, D, 1.f);
+  }
+  {
+    const Piece pc = C::piece(P_O);
+    put_B(at(P_O, pc.off), L.Wo, D, 0, 0, D, D, 1.f);
+    put_bias(at(P_O, pc.bias), L.bo, 0, D, 1.f);
   }
   for (int hf = 0; hf < C::kFfnHalves; ++hf) {
     const int p1 = hf == 0 ? P_W1A : P_W1B, p2 = hf == 0 ? P_W2A : P_W2B;
     const Piece a = C::piece(p1), b = C::piece(p2);
-    put_B(at(p1, a.off), L.W1, H, 128 * hf, 0, 128, D, 1.f);            // hidden units 128 hf ..
-    put_bias(at(p1, a.bias), L.b1, 128 * hf, 128, 1.f);
+    fold_ln(L.W1, H, 128 * hf, D, 128, L.ln2_g, L.ln2_b, L.b1, 1.f, Wf, bf);   // hidden units 128 hf ..
+    put_B(at(p1, a.off), Wf.data(), 128, 0, 0, 128, D, 1.f);
+    put_bias(at(p1, a.bias), bf.data(), 0, 128, 1.f);
     put_B(at(p2, b.off), L.W2, D, 0, 128 * hf, D, 128, 1.f);            // rows 128 hf .. of W2
     if (b.bias >= 0) put_bias(at(p2, b.bias), L.b2, 0, D, 1.f);
   }
 }
 
-// Whether every fp16 operand of the stack stays far inside fp16's range: LayerNorm outputs
-// are bounded by max|gain| sqrt(D) + max|shift|, a product's outputs by that bound times the
-// largest column sum of |W| plus max|bias|, the attention output by the bound of V, ReLU by
-// the bound of its input.
+// Whether every fp16 operand of the stack stays far inside fp16's range: the standardized
+// rows are bounded by sqrt(D); a product's outputs by that bound times the largest column
+// sum of |g o W| plus the largest |folded bias|; the attention output by the bound of V;
+// ReLU by the bound of its input; the folded weights by max |g| max |W|.
 bool fp16_operands_safe(const tr_model_desc& d, const tr_model_weights* w) {
   const int D = d.D, H = d.ffn_hidden;
   auto amax = [](const float* p, size_t n) {
@@ -960,28 +1068,31 @@ bool fp16_operands_safe(const tr_model_desc& d, const tr_model_weights* w) {
     for (size_t i = 0; i < n; ++i) m = std::max(m, (double)fabsf(p[i]));
     return m;
   };
-  auto colsum = [](const float* W, int K, int N) {
+  // bound of z W' + b' with W' = diag(g) W, b' = beta W + b, |z_k| <= sqrt(D)
+  auto out_bound = [&](const float* W, int K, int N, const float* g, const float* beta, const float* b) {
     double m = 0;
     for (int n = 0; n < N; ++n) {
-      double s = 0;
-      for (int k = 0; k < K; ++k) s += fabs((double)W[(size_t)k * N + n]);
-      m = std::max(m, s);
+      double s = 0, c = b ? fabs((double)b[n]) : 0.0;
+      for (int k = 0; k < K; ++k) {
+        s += fabs((double)W[(size_t)k * N + n] * g[k]);
+        c += fabs((double)W[(size_t)k * N + n] * beta[k]);
+      }
+      m = std::max(m, s * sqrt((double)K) + c);
     }
     return m;
   };
   const double limit = 16384.0;
   for (int l = 0; l < d.n_layer; ++l) {
     const tr_layer_weights& L = w->layers[l];
-    const double b1 = amax(L.ln1_g, D) * sqrt((double)D) + amax(L.ln1_b, D);
-    const double b2 = amax(L.ln2_g, D) * sqrt((double)D) + amax(L.ln2_b, D);
-    const double q = b1 * colsum(L.Wq, D, D) + amax(L.bq, D);
-    const double k = b1 * colsum(L.Wk, D, D) + amax(L.bk, D);
-    const double v = b1 * colsum(L.Wv, D, D) + amax(L.bv, D);
-    const double h = b2 * colsum(L.W1, D, H) + amax(L.b1, H);
-    if (!(b1 < limit && b2 < limit && q < limit && k < limit && v < limit && h < limit)) return false;
+    const double q = out_bound(L.Wq, D, D, L.ln1_g, L.ln1_b, L.bq);
+    const double k = out_bound(L.Wk, D, D, L.ln1_g, L.ln1_b, L.bk);
+    const double v = out_bound(L.Wv, D, D, L.ln1_g, L.ln1_b, L.bv);
+    const double h = out_bound(L.W1, D, H, L.ln2_g, L.ln2_b, L.b1);
+    if (!(q < limit && k < limit && v < limit && h < limit)) return false;
+    const double gmax = std::max(amax(L.ln1_g, D), amax(L.ln2_g, D));
     const double wmax = std::max({amax(L.Wq, (size_t)D * D), amax(L.Wk, (size_t)D * D), amax(L.Wv, (size_t)D * D),
                                   amax(L.Wo, (size_t)D * D), amax(L.W1, (size_t)D * H), amax(L.W2, (size_t)H * D)});
-    if (!(wmax < limit)) return false;
+    if (!(wmax * std::max(gmax, 1.0) < limit)) return false;
   }
   return true;
 }
@@ -998,19 +1109,9 @@ tr_status build_stack_images(tr_model* m, const tr_model_weights* w) {
   const tr_model_desc& d = m->desc;
   const int N = d.n_layer;
   std::vector<uint8_t> img((size_t)N * C::kItems * C::kItemBytes, 0);
-  std::vector<float> vec((size_t)N * vec_per_layer<D>() + D + 4, 0.f);
-  for (int l = 0; l < N; ++l) {
-    build_layer_items<D>(img.data() + (size_t)l * C::kItems * C::kItemBytes, w->layers[l]);
-    const tr_layer_weights& L = w->layers[l];
-    float* v = vec.data() + (size_t)l * vec_per_layer<D>();
-    for (int j = 0; j < D; ++j) {
-      v[j] = L.ln1_g[j];
-      v[D + j] = L.ln1_b[j];
-      v[2 * D + j] = L.ln2_g[j];
-      v[3 * D + j] = L.ln2_b[j];
-    }
-  }
-  float* vf = vec.data() + (size_t)N * vec_per_layer<D>();
+  std::vector<float> vec(vec_floats<D>(), 0.f);
+  for (int l = 0; l < N; ++l) build_layer_items<D>(img.data() + (size_t)l * C::kItems * C::kItemBytes, w->layers[l]);
+  float* vf = vec.data();
   double bh = w->b_head;
   for (int j = 0; j < D; ++j) {
     vf[j] = (float)((double)w->w_head[j] * w->lnf_g[j]);
@@ -1029,7 +1130,7 @@ tr_status build_stack_images(tr_model* m, const tr_model_weights* w) {
   m->tc_stack = m->tc_blob;
   m->tc_stack_layer_bytes = (size_t)C::kItems * C::kItemBytes;
   m->tc_vec = reinterpret_cast<const float*>((uint8_t*)m->tc_blob + img_bytes);
-  m->tc_vec_layer_floats = vec_per_layer<D>();
+  m->tc_vec_layer_floats = 0;
   return TR_OK;
 }
 
@@ -1052,7 +1153,7 @@ bool plan_smem(StackParams& p, int n_layer, int lp_max, bool pair, int& smem_byt
   const int kv_bytes = 2 * lp_max * D * 2;
   p.off_ones = p.off_kv + ((kv_bytes + 1023) & ~1023);
   p.off_ring = p.off_ones + kM * 16 * 2;
-  const int vec_bytes = (n_layer * vec_per_layer<D>() + D + 4) * 4;
+  const int vec_bytes = vec_floats<D>() * 4;
   const int fixed = p.off_ring + kBarArea;
   int stages = std::min(kMaxStages, (kSmemLimit - fixed - vec_bytes) / Cfg<D>::kItemBytes);
   bool vec_in_smem = true;
@@ -1062,6 +1163,9 @@ bool plan_smem(StackParams& p, int n_layer, int lp_max, bool pair, int& smem_byt
   }
   if (stages < 2) return false;
   p.stages = stages;
+  // slot 0 runs items K, V (and Q) of the unit's first layer before slot 1 starts: it needs
+  // a third stage to reach the attention alone (D = 64 keeps all four projections in one item)
+  p.gate_phase = (D == 128 && stages < 3) ? 0 : 1;
   int off = p.off_ring + stages * Cfg<D>::kItemBytes;
   if (vec_in_smem) {
     p.off_vec = off;
@@ -1097,19 +1201,48 @@ tr_status score_launch(const tr_model* m, const void* tokens, const int64_t* req
   p.status = ds->status;
   p.n_layer = m->desc.n_layer;
   p.pair = 1;
-  int units = 0, k = 0, lp_max = 0;
+  int sms = 148, dev = 0;
+  TR_CUDA_TRY(cudaGetDevice(&dev));
+  TR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  // Units: pairs of consecutive tiles of one request (the request's last unit is a single
+  // tile when its tile count is odd).  Units go to the CTAs round robin; when the last round
+  // is partial, its pairs are split into single tiles (as many as there are idle CTAs in that
+  // round), which spreads the round over more SMs.
+  int k = 0, lp_max = 0;
+  int tiles_of[TR_MAX_REQUESTS], pairs_of[TR_MAX_REQUESTS];
+  int units = 0;
   for (int r = 0; r < R; ++r) {
     const int64_t nr = req_offsets[r + 1] - req_offsets[r];
     if (nr == 0) continue;
     p.req[k].kv = static_cast<const uint8_t*>(kv[r]);
     p.req[k].cand_off = req_offsets[r];
     p.req[k].n = nr;
-    p.req[k].unit_off = units;
     p.req[k].L_u = L_u[r];
     p.req[k].domain = domain[r];
     lp_max = std::max(lp_max, round_up16(L_u[r]));
-    units += (int)((nr + 2 * kM - 1) / (2 * kM));
+    tiles_of[k] = (int)((nr + kM - 1) / kM);
+    pairs_of[k] = tiles_of[k] / 2;
+    units += tiles_of[k] - pairs_of[k];
     ++k;
+  }
+  if (units > 0) {
+    const int rem = units % sms;                 // units of the partial last round (0: none)
+    int window = rem, room = rem ? sms - rem : 0;
+    for (int q = k - 1; q >= 0 && window > 0 && room > 0; --q) {
+      const int singles = tiles_of[q] - 2 * pairs_of[q];
+      int in_window = std::min(window, singles + pairs_of[q]);
+      const int pairs_in_window = std::max(0, in_window - singles);
+      const int split = std::min(pairs_in_window, room);
+      pairs_of[q] -= split;
+      room -= split;
+      window -= in_window;
+    }
+    units = 0;
+    for (int q = 0; q < k; ++q) {
+      p.req[q].unit_off = units;
+      p.req[q].n_pair = pairs_of[q];
+      units += tiles_of[q] - pairs_of[q];
+    }
   }
   if (units == 0) return TR_OK;
   p.R = k;
@@ -1118,9 +1251,6 @@ tr_status score_launch(const tr_model* m, const void* tokens, const int64_t* req
   const int sw = lp_max <= 32 ? 32 : lp_max <= 64 ? 64 : kMaxLp;   // head slot width of this launch
   if (!plan_smem<D>(p, p.n_layer, sw, true, smem))
     return fail(TR_ERR_UNSUPPORTED, "stack kernel: %d layers do not fit shared memory", p.n_layer);
-  int sms = 148, dev = 0;
-  TR_CUDA_TRY(cudaGetDevice(&dev));
-  TR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   const int grid = std::min(units, sms);
   return sw == 32 ? launch<D, 32, false>(grid, p, smem, st)
        : sw == 64 ? launch<D, 64, false>(grid, p, smem, st)
@@ -1162,7 +1292,7 @@ tr_status tc_prefill_batch(const tr_model* m, const float* const* user_tokens, c
   p.status = ds->status;
   p.n_layer = m->desc.n_layer;
   p.pair = 0;
-  int k = 0;
+  int k = 0, lp_max = 0;
   for (int r = 0; r < R; ++r) {
     if (L_u[r] == 0) continue;
     if ((uintptr_t)kv[r] % 16 || (uintptr_t)user_tokens[r] % 16)
@@ -1174,16 +1304,23 @@ tr_status tc_prefill_batch(const tr_model* m, const float* const* user_tokens, c
     p.req[k].unit_off = k;
     p.req[k].L_u = L_u[r];
     p.req[k].domain = domain[r];
+    p.req[k].n_pair = 0;
+    lp_max = std::max(lp_max, round_up16(L_u[r]));
     ++k;
   }
   if (k == 0) return TR_OK;
   p.R = k;
   p.n_units = k;
   int smem = 0;
-  const bool fit = m->desc.D == 128 ? plan_smem<128>(p, p.n_layer, kMaxLp, false, smem)
-                                    : plan_smem<64>(p, p.n_layer, kMaxLp, false, smem);
+  const int sw = lp_max <= 32 ? 32 : lp_max <= 64 ? 64 : kMaxLp;   // head slot width of this launch
+  const bool fit = m->desc.D == 128 ? plan_smem<128>(p, p.n_layer, sw, false, smem)
+                                    : plan_smem<64>(p, p.n_layer, sw, false, smem);
   if (!fit) return fail(TR_ERR_UNSUPPORTED, "stack kernel: %d layers do not fit shared memory", p.n_layer);
-  return m->desc.D == 128 ? launch<128, kMaxLp, true>(k, p, smem, st) : launch<64, kMaxLp, true>(k, p, smem, st);
+  if (m->desc.D == 128)
+    return sw == 32 ? launch<128, 32, true>(k, p, smem, st)
+         : sw == 64 ? launch<128, 64, true>(k, p, smem, st) : launch<128, kMaxLp, true>(k, p, smem, st);
+  return sw == 32 ? launch<64, 32, true>(k, p, smem, st)
+       : sw == 64 ? launch<64, 64, true>(k, p, smem, st) : launch<64, kMaxLp, true>(k, p, smem, st);
 }
 
 // User side of one request (one CTA).
