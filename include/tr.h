@@ -29,7 +29,11 @@
  *    different streams never share scratch; calls on one stream are ordered by it.  A call
  *    that needs more scratch than its stream's buffer holds synchronises that stream and
  *    reallocates it, so the first such call on a stream must not be made while the stream
- *    is being captured into a CUDA graph.  The tensor-core paths use no scratch.
+ *    is being captured into a CUDA graph.  The tensor-core paths use no scratch; the
+ *    tensor-core compressor of a TR_BF16 model takes its tiles from a work counter, a few
+ *    device ints per (device, stream) that the library allocates (zeroed) on the first
+ *    such call on a stream, kept until process exit, and zeroes on the stream before every
+ *    launch; the same capture rule applies to that first call.
  *  - Row-major layouts unless stated; "[a][b]" means a rows of b contiguous elements.
  *  - dtype TR_F32 models compute in fp32 throughout.  TR_BF16 models store tables,
  *    weights and target-field tokens in bf16; the compressed candidate tokens are fp32 for

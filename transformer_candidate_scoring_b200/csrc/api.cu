@@ -96,6 +96,35 @@ tr_status workspace(size_t bytes, cudaStream_t st, void** out) {
   return TR_OK;
 }
 
+namespace {
+struct StreamInts {
+  int dev;
+  cudaStream_t stream;
+  int* ptr;
+};
+std::vector<StreamInts> g_counters;   // guarded by g_dev_mu
+}  // namespace
+
+tr_status stream_counters(cudaStream_t st, int** out) {
+  int dev = 0;
+  TR_CUDA_TRY(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  for (auto& e : g_counters)
+    if (e.dev == dev && e.stream == st) {
+      *out = e.ptr;
+      return TR_OK;
+    }
+  int* p = nullptr;
+  if (cudaMalloc(&p, 64 * sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(TR_ERR_NOMEM, "stream counters: allocation failed");
+  }
+  TR_CUDA_TRY(cudaMemset(p, 0, 64 * sizeof(int)));
+  g_counters.push_back({dev, st, p});
+  *out = p;
+  return TR_OK;
+}
+
 tr_status ensure_smem_attr(const void* kernel, int bytes) {
   int dev = 0;
   TR_CUDA_TRY(cudaGetDevice(&dev));

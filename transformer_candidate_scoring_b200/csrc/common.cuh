@@ -52,6 +52,9 @@ tr_status device_state(DeviceState** out);                 // of the current dev
 // so that calls on different streams never share scratch.  Growing it synchronises the
 // stream and reallocates.
 tr_status workspace(size_t bytes, cudaStream_t st, void** out);
+// A few zero-initialised device ints per (device, stream), for kernels that claim work at
+// run time (a launch zeroes what it uses on its stream first).  Allocated on first use.
+tr_status stream_counters(cudaStream_t st, int** out);
 // cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (device, kernel), under a lock.
 tr_status ensure_smem_attr(const void* kernel, int bytes);
 

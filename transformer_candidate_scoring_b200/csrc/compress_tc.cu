@@ -15,7 +15,10 @@
 // Warp 0 issues copies, warp 1 issues MMAs, warps 2-9 run the epilogues: two warps per TMEM
 // lane quadrant, each owning half of a row's columns; a row's LayerNorm statistics are merged
 // across the pair (Welford) through shared memory.  Waits are bounded as in the candidate
-// stack kernel.
+// stack kernel.  Every tile is claimed at run time from a per-launch counter: a CTA that
+// starts late, on an SM another kernel still holds, finds less work (or none) instead of
+// holding the launch back.  The producer passes each claimed tile index to the MMA and
+// epilogue threads through a two-entry ring in shared memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
@@ -54,13 +57,30 @@ struct CompParams {
   const float* vec;            // b1 a1 g1 be1 (c1 each), b2 a2 g2 be2 (c2 each), b3 (c3)
   float* out;                  // [n][c3]
   int* status;
+  int* claim;                  // next unclaimed tile (zero at launch)
   long long n;
   int n_tiles, c0, c1, c2, c3;
 };
 
 struct CBars {
   uint32_t full1[2], empty1[2], full2[2], empty2[2], r1_free, mma, epi, drain, qsync[4], vsync;
+  uint32_t tile_full[2], tile_empty[2], tile_slot[2];   // the claimed-tile ring
 };
+
+// Next tile index of this CTA from the two-entry ring (-1: no more); the reader releases
+// the entry at once.
+__device__ __forceinline__ int next_tile(const CBars& b, int& ts, uint32_t& tph, volatile int* abort_flag,
+                                         bool& ok) {
+  ok = ok && mbar_wait(b.tile_full[ts], tph, abort_flag);
+  int t = -1;
+  if (ok) asm volatile("ld.shared.b32 %0, [%1];" : "=r"(t) : "r"(b.tile_slot[ts]) : "memory");
+  mbar_arrive(b.tile_empty[ts]);
+  if (++ts == 2) {
+    ts = 0;
+    tph ^= 1;
+  }
+  return ok ? t : -1;
+}
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
   asm volatile(
@@ -93,7 +113,19 @@ __device__ void comp_producer(const CompParams& p, uint32_t r1, uint32_t r2, con
   bool ok = true;
   bool pend1[2] = {false, false}, pend2[2] = {false, false};
   uint32_t par1[2] = {0, 0}, par2[2] = {0, 0};
-  for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+  int ts = 0;
+  uint32_t tph = 0;
+  for (int tile = atomicAdd(p.claim, 1); ok;) {
+    // publish the tile (or the end) to the MMA and epilogue threads
+    if (!(ok = mbar_wait(b.tile_empty[ts], tph ^ 1, abort_flag))) break;
+    const int pub = tile < p.n_tiles ? tile : -1;
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(b.tile_slot[ts]), "r"(pub) : "memory");
+    mbar_arrive(b.tile_full[ts]);
+    if (++ts == 2) {
+      ts = 0;
+      tph ^= 1;
+    }
+    if (pub < 0) break;
     // the stage buffers hold the previous tile's activations until its last GEMM is done
     if (!(ok = mbar_wait(b.r1_free, free_phase ^ 1, abort_flag))) break;
     free_phase ^= 1;
@@ -118,6 +150,7 @@ __device__ void comp_producer(const CompParams& p, uint32_t r1, uint32_t r2, con
       par2[s2] = ph2;
       if (++s2 == 2) { s2 = 0; ph2 ^= 1; }
     }
+    tile = atomicAdd(p.claim, 1);
   }
   if (!ok) {
     for (int s = 0; s < 2; ++s) {
@@ -143,8 +176,12 @@ __device__ void comp_mma(const CompParams& p, uint32_t tmem, uint32_t r1, uint32
     tc_fence_after();
     return ok;
   };
-  for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-    if (tile != (int)blockIdx.x && !wait_epi()) break;   // previous tile's last epilogue has read TMEM
+  int ts = 0;
+  uint32_t tph = 0;
+  for (bool first = true; ok; first = false) {
+    const int tile = next_tile(b, ts, tph, abort_flag, ok);
+    if (tile < 0) break;
+    if (!first && !wait_epi()) break;   // previous tile's last epilogue has read TMEM
     // layer 1: [128 x c0] x [c0 x c1]
     for (int kc = 0; kc < p.c0 / 64 && ok; ++kc) {
       if (!(ok = mbar_wait(b.full1[s1], ph1, abort_flag))) break;
@@ -327,7 +364,11 @@ __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, c
     tc_fence_before();
     mbar_arrive(b.epi);
   };
-  for (int tile = blockIdx.x; tile < p.n_tiles && e.ok; tile += gridDim.x) {
+  int ts = 0;
+  uint32_t tph = 0;
+  for (;;) {
+    const int tile = next_tile(b, ts, tph, abort_flag, e.ok);
+    if (tile < 0) break;
     // layer 1's vectors (4 c1 floats) are read into registers while its GEMM runs and
     // stored once it is done
     float4 r1v[2];
@@ -392,6 +433,11 @@ __global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant_
   b.drain = bar0 + 88;
   for (int q = 0; q < 4; ++q) b.qsync[q] = bar0 + 96 + 8 * q;
   b.vsync = bar0 + 144;
+  for (int s = 0; s < 2; ++s) {
+    b.tile_full[s] = bar0 + 152 + 8 * s;
+    b.tile_empty[s] = bar0 + 168 + 8 * s;
+    b.tile_slot[s] = bar0 + 184 + 4 * s;
+  }
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_BAR + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_BAR + 136);
   if (threadIdx.x == 0) {
@@ -407,6 +453,10 @@ __global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant_
     mbar_init(b.drain, 1);
     for (int q = 0; q < 4; ++q) mbar_init(b.qsync[q], 64);
     mbar_init(b.vsync, 256);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(b.tile_full[s], 1);
+      mbar_init(b.tile_empty[s], 1 + 256);   // the MMA thread and every epilogue thread
+    }
     *abort_flag = 0;
     mbar_fence_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.xmap)) : "memory");
@@ -553,6 +603,8 @@ tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens,
   p.vec = m->tc_comp_vec;
   p.out = static_cast<float*>(tokens);
   p.status = ds->status;
+  TR_TRY(stream_counters(st, &p.claim));
+  TR_CUDA_TRY(cudaMemsetAsync(p.claim, 0, sizeof(int), st));
   p.n = n;
   p.n_tiles = (int)((n + kM - 1) / kM);
   p.c0 = c[0];
