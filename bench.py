@@ -9,10 +9,11 @@ A step is one pass of the whole scoring path over one request of the 128D-5L wor
 Stage times come from CUDA events on the stream each stage runs on; the user side
 overlaps the target side, so the stages do not add up to the step.
 ``value`` is candidates scored per second over all ranks, with inputs resident in HBM: the
-K timed steps are one stream of requests, captured into one CUDA graph, and consecutive
-requests overlap (request i + 1's aggregation starts when request i's score kernel reaches
-its last, partial wave of tiles; pipeline.Overlapped).  The same steps run one after the
-other are reported as ``serial_graph_ms_per_step``.  ``e2e`` repeats the K steps with each
+K timed steps are one stream of candidate tiles, captured into one CUDA graph, whose
+compress and score launches take fixed chunks across request boundaries (two compressor
+rounds, one score round each; pipeline.Streamed).  The same steps with each request's last
+partial rounds run beside the next request (pipeline.Overlapped) are reported as
+``overlapped_graph_ms_per_step``, and run one after the other as ``serial_graph_ms_per_step``.  ``e2e`` repeats the K steps with each
 request's bags copied from pinned host memory (during the previous request) and its scores
 copied back, all inside the timed region.  Requests rotate over several seeded request sets and the
 embedding tables (24.6 GB) are far larger than L2.
@@ -265,12 +266,13 @@ def stage_rooflines(dims, reqs, stage_ms, peaks, peak_kind):
 
 def measure_side(name, w, params, tables, reqs, dev, steps, warmup, peaks, peak_kind, cpu_seconds):
     """One of the other workloads on the same GPU (every stage through the C calls): stage
-    times from eager steps, the step from one CUDA graph per step replayed back to back, and
-    the overlapped stream of requests (one graph); the oracle's rate on the same request."""
+    times from eager steps, the step from one CUDA graph per step replayed back to back, the
+    overlapped requests and the stream of candidate tiles (one graph each; the value is the
+    stream's); the oracle's rate on the same request."""
     import torch
 
     from transformer_candidate_scoring_b200 import api
-    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload, Overlapped
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload, Overlapped, Streamed
 
     stream = torch.cuda.current_stream()
     dw = DeviceWorkload(w, device=dev, reqs=reqs, params=params, tables=tables)
@@ -308,19 +310,31 @@ def measure_side(name, w, params, tables, reqs, dev, steps, warmup, peaks, peak_
     torch.cuda.synchronize()
     ov_ms = e0.elapsed_time(e1) / steps
     del g
+    st = Streamed(dw)
+    st.run(0, warmup, stream)
+    torch.cuda.synchronize()
+    g = st.capture(warmup, steps)
+    g.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    st_ms = e0.elapsed_time(e1) / steps
+    del g
     if api.sync_status() != 0:
         raise RuntimeError(f"device status word set during the {name} measurement")
     n_cand = dw.n_cand
     out = {"workload": w.name, "candidates_per_step": n_cand, "requests": len(reqs),
            "L_u": [r.L_u for r in reqs] if len(reqs) > 1 else reqs[0].L_u,
-           "value": n_cand / (ov_ms / 1e3), "unit": "candidates/s", "ms_per_step": ov_ms,
-           "serial_graph_ms_per_step": serial_ms,
+           "value": n_cand / (st_ms / 1e3), "unit": "candidates/s", "ms_per_step": st_ms,
+           "overlapped_graph_ms_per_step": ov_ms, "serial_graph_ms_per_step": serial_ms,
            "stages": {k: {"ms": v} for k, v in stage_ms.items()}}
     for k, r in stage_rooflines(w.dims, reqs, stage_ms, peaks, peak_kind).items():
         out["stages"][k].update(r)
     if cpu_seconds > 0:
         out["cpu_baseline"] = oracle_rates(w, params, reqs[0], cpu_seconds, cpu_seconds / 2)
-    del dw, dw2, ov
+    del dw, dw2, ov, st
     torch.cuda.empty_cache()
     return out
 
@@ -366,7 +380,8 @@ def run_ours(args, rank, world, local_rank):
     import torch.distributed as dist
 
     from transformer_candidate_scoring_b200 import api
-    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload, HostFeed, Overlapped, score_split
+    from transformer_candidate_scoring_b200.pipeline import (DeviceBags, DeviceWorkload, HostFeed, Overlapped, Streamed,
+                                                             score_split)
     from transformer_candidate_scoring_b200.shard import max_over_ranks, rank_seed
 
     torch.cuda.set_device(local_rank)
@@ -452,34 +467,41 @@ def run_ours(args, rank, world, local_rank):
     serial_elapsed = max_over_ranks(g0.elapsed_time(g1) / 1e3)
     del graphs
 
-    # ---- the timed value: the K steps as one stream of requests, captured into one CUDA
-    # graph, consecutive requests overlapped (Overlapped: request i + 1's aggregation starts
-    # when request i's score kernel reaches its last partial wave) over two activation slots
-    dw2 = DeviceWorkload(w, device=dev, reqs=sets[0], params=dw.params,
-                         tables=(dw.user_tables, dw.target_tables))
-    ov = Overlapped([dw, dw2])
-
     def bind(i, slot, main):
         ub, tb, reqs = dsets[i % N_REQUEST_SETS]
         slot.use_bags(ub, tb, reqs)
 
-    ov.run(0, args.warmup, stream, bind=bind)             # eager warm-up of both slots
-    torch.cuda.synchronize()
-    g_ov = ov.capture(args.warmup, args.steps, bind=bind)
-    launches = ov.launches_per_step * args.steps
-    g_ov.replay()                                          # warm-up replay (K more steps)
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    g0.record(stream)
-    g_ov.replay()
-    g1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    if api.sync_status() != 0:
-        raise RuntimeError("device status word set during the overlapped replays")
-    graph_elapsed = max_over_ranks(g0.elapsed_time(g1) / 1e3)
-    del g_ov
+    def replay_time(runner, label):
+        runner.run(0, args.warmup, stream, bind=bind)          # eager warm-up of the slots
+        torch.cuda.synchronize()
+        g = runner.capture(args.warmup, args.steps, bind=bind)
+        g.replay()                                             # warm-up replay (K more steps)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        g0.record(stream)
+        g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        if api.sync_status() != 0:
+            raise RuntimeError(f"device status word set during the {label} replays")
+        del g
+        return max_over_ranks(g0.elapsed_time(g1) / 1e3)
+
+    # ---- consecutive requests overlapped over two activation slots (Overlapped: each
+    # request's last partial rounds of compression and scoring run beside the next request's
+    # aggregation), captured into one CUDA graph
+    dw2 = DeviceWorkload(w, device=dev, reqs=sets[0], params=dw.params,
+                         tables=(dw.user_tables, dw.target_tables))
+    ov = Overlapped([dw, dw2])
+    overlapped_elapsed = replay_time(ov, "overlapped")
+    # ---- the timed value: the K steps as one stream of candidate tiles (Streamed: every
+    # compress launch two rounds of tiles, every score launch one round of two-tile units,
+    # across request boundaries, over a ring of activation slots), one CUDA graph
+    st = Streamed(dw)
+    graph_elapsed = replay_time(st, "streamed")
+    launches = st.launches_per_step * args.steps
     use_graphs = True                     # the timed value is always graph-replayed
     elapsed = graph_elapsed
     clk = clocks.stop()
@@ -517,19 +539,19 @@ def run_ours(args, rank, world, local_rank):
     host_scores = [torch.empty(n_cand, dtype=torch.float32).pin_memory() for _ in range(2)]
     d2h = n_cand * 4
 
-    feed.run_overlapped(ov, 0, args.warmup, host_scores, stream)
+    feed.run_overlapped(st, 0, args.warmup, host_scores, stream)
     torch.cuda.synchronize()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    feed.run_overlapped(ov, args.warmup, args.steps, host_scores, stream)   # eager launches
+    feed.run_overlapped(st, args.warmup, args.steps, host_scores, stream)   # eager launches
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_eager_ms = max_over_ranks(e0.elapsed_time(e1) / 1e3) / args.steps * 1e3
     # the same launch mode as the timed value: one graph of the K steps, host copies inside
-    g_e2e = feed.capture_overlapped(ov, args.warmup, args.steps, host_scores)
+    g_e2e = feed.capture_overlapped(st, args.warmup, args.steps, host_scores)
     g_e2e.replay()
     torch.cuda.synchronize()
     barrier()
@@ -604,8 +626,11 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_gbs_copies_only": h2d / (copy_ms / 1e3) / 1e9},
         "gpu_launches": int(launches),
         "launch": {"graphs": bool(use_graphs), "e2e_graphs": bool(use_graphs),
-                   "overlap": "request i+1's aggregation runs beside request i's last partial wave of score tiles",
+                   "overlap": ("one stream of candidate tiles across requests: compress launches of two rounds "
+                               "of tiles, score launches of one round of two-tile units (pipeline.Streamed)"),
+                   "ring_slots": len(st.slots),
                    "graph_ms_per_step": graph_elapsed / args.steps * 1e3,
+                   "overlapped_graph_ms_per_step": overlapped_elapsed / args.steps * 1e3,
                    "serial_graph_ms_per_step": serial_elapsed / args.steps * 1e3,
                    "eager_ms_per_step": eager_ms},
         "clocks": clk,

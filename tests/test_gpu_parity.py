@@ -487,6 +487,67 @@ def test_overlapped_steps_match_serial_steps(name, n_sms):
         assert torch.equal(out[i], ref[i % 3]), ("graph", i)
 
 
+@pytest.mark.parametrize("name,n_cand,n_slots,comp_chunk,units", [
+    ("128d5l", 2000, 3, 640, 3),         # launches of 5 tiles / 3 units, across batches and ring wraps
+    ("128d5l", 40000, 4, None, None),    # the default launch sizes (two compressor rounds, one score round)
+    ("packed", 300, 2, 1000, 5),         # 16 requests of mixed L_u per batch (one request set:
+                                         # the slots' caches are sized by L_u); launches span many
+    ("64d3l", 2000, 3, 768, 4),
+    ("tiny", 500, 2, 256, 2),            # fp32: every stage on the CUDA-core kernels
+])
+def test_streamed_steps_match_serial_steps(name, n_cand, n_slots, comp_chunk, units):
+    """Batches scored as one stream of candidate tiles (compress and score launches of fixed
+    size across batch boundaries, over a ring of activation slots) give each batch the
+    scores of a serial step, bit for bit, eagerly and from one captured graph."""
+    from transformer_candidate_scoring_b200.pipeline import Streamed
+    w = datagen.scaled(datagen.WORKLOADS[name], n_cand_per_request=n_cand, rows=20000)
+    sets = [datagen.make_requests(w, seed=800 + k) for k in range(3)]
+    dw, ref = _serial_reference(w, sets)
+    one_set = name == "packed"
+    if one_set:
+        sets, ref = sets[:1], ref[:1]
+    st = Streamed(dw, n_slots=n_slots, comp_chunk=comp_chunk, score_units=units)
+    n_batch = 7
+    out = [torch.zeros(dw.n_cand, dtype=torch.float32, device="cuda") for _ in range(n_batch)]
+
+    def bind(i, slot, main):
+        slot.use_bags(*_set_bags(dw, sets, i))
+
+    def scored(i, slot, s):
+        with torch.cuda.stream(s):
+            out[i].copy_(slot.scores)
+
+    st.run(0, n_batch, bind=bind, scored=scored)
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    for i in range(n_batch):
+        assert torch.equal(out[i], ref[i % len(ref)]), ("eager", i)
+    g = st.capture(0, n_batch, bind=bind, scored=scored)
+    for o in out:
+        o.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    for i in range(n_batch):
+        assert torch.equal(out[i], ref[i % len(ref)]), ("graph", i)
+
+
+def test_full_request_scores_repeat_bit_identical():
+    """A 40,000-candidate request (148 two-tile units on every SM at once, then single tiles)
+    scored five times gives the same bits each time: no hand-off between the two tiles a CTA
+    holds depends on timing."""
+    from transformer_candidate_scoring_b200.pipeline import DeviceWorkload
+    w = datagen.scaled(datagen.WORKLOADS["128d5l"], n_cand_per_request=40000, rows=20000)
+    dw = DeviceWorkload(w)
+    dw.step()
+    first = dw.scores.clone()
+    for _ in range(4):
+        dw.score()
+        torch.cuda.synchronize()
+        assert torch.equal(dw.scores, first)
+    assert tr().sync_status() == 0
+
+
 _SET_BAGS = {}
 
 
@@ -495,7 +556,7 @@ def _set_bags(dw, sets, i):
     from transformer_candidate_scoring_b200.pipeline import DeviceBags, pack_target_bags, pack_user_bags
     reqs = sets[i % len(sets)]
     key = (id(dw), i % len(sets))
-    if key not in _SET_BAGS:
+    if key not in _SET_BAGS or _SET_BAGS[key][2] is not reqs:      # (ids of freed objects recur)
         _SET_BAGS[key] = (DeviceBags.of(pack_user_bags(reqs), dw.device),
                           DeviceBags.of(pack_target_bags(reqs), dw.device), reqs)
     return _SET_BAGS[key]

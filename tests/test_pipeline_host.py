@@ -373,3 +373,148 @@ def test_compress_range_passes_row_views(monkeypatch):
     (x0, t0), (x1, t1) = calls
     assert x0.shape[0] == 512 and x1.shape[0] == 288
     assert x1.data_ptr() == dw.X[512:].data_ptr() and t1.data_ptr() == dw.tokens[512:].data_ptr()
+
+
+# ---------------------------------------------------------------- the candidate stream (Streamed)
+
+def _check_plan(plan, n, count, first, n_slots, comp_chunk, bounds, score_units):
+    """Every candidate is gathered, compressed and scored once, in that order, each before
+    its ring slot is gathered over; launches have their full size except where a ring wrap,
+    a slot reuse or the end of the run cuts them; score launches end on unit ends."""
+    ring = n_slots * n
+    base = first * n
+    ends = {j * n + b for j in range(count) for b in bounds}      # unit ends of the stream
+    gathered, comp, score = -1, 0, 0
+    wraps = {w - base for w in range(ring, base + count * n + ring, ring)}
+    for step in plan:
+        if step[0] == "gather":
+            j = step[1]
+            assert j == gathered + 1
+            gathered = j
+            assert comp >= (j - n_slots + 1) * n and score >= (j - n_slots + 1) * n   # slot j - n_slots is done
+            continue
+        kind, a, b = step
+        assert b > a
+        assert not any(a < w < b for w in wraps)                 # never across the ring's end
+        cut = b in wraps or b == count * n or b % n == 0
+        if kind == "compress":
+            assert a == comp and b <= (gathered + 1) * n
+            assert b - a == comp_chunk or cut
+            comp = b
+        else:
+            assert a == score and b <= comp and b in ends
+            units = sum(1 for e in ends if a < e <= b)
+            assert units == score_units or (units < score_units and cut)
+            score = b
+    assert gathered == count - 1 and comp == score == count * n
+
+
+@pytest.mark.parametrize("n,count,first,n_slots,comp_chunk,units", [
+    (40000, 12, 3, 64, 294 * 128, 148),      # the 128D-5L batch: no wrap inside the run
+    (40000, 12, 3, 4, 294 * 128, 148),       # wraps every four batches
+    (300, 9, 0, 2, 1000, 3),                 # chunks longer than a batch: slot reuse forces flushes
+    (1000, 7, 5, 3, 384, 5),
+])
+def test_stream_plan_covers_every_candidate_once(n, count, first, n_slots, comp_chunk, units):
+    from transformer_candidate_scoring_b200.pipeline import stream_plan, unit_bounds
+    bounds = unit_bounds([0, n])
+    plan = stream_plan(n, count, first, n_slots, comp_chunk, bounds, units)
+    _check_plan(plan, n, count, first, n_slots, comp_chunk, bounds, units)
+
+
+def test_stream_plan_packed_batches_and_steady_state():
+    from transformer_candidate_scoring_b200.pipeline import stream_plan, unit_bounds
+    rng = np.random.default_rng(3)
+    for _ in range(30):
+        sizes = rng.integers(1, 700, size=rng.integers(1, 6))
+        off = np.concatenate([[0], np.cumsum(sizes)]).tolist()
+        n = off[-1]
+        bounds = unit_bounds(off)
+        assert bounds[-1] == n and sorted(bounds) == bounds
+        count, first, n_slots = int(rng.integers(1, 9)), int(rng.integers(0, 5)), int(rng.integers(2, 6))
+        comp_chunk, units = int(rng.integers(1, 2000)), int(rng.integers(1, 12))
+        plan = stream_plan(n, count, first, n_slots, comp_chunk, bounds, units)
+        _check_plan(plan, n, count, first, n_slots, comp_chunk, bounds, units)
+    # the 128D-5L batch in steady state: every launch between the first and the last two is
+    # full size (294 compressor tiles, 148 score units)
+    bounds = unit_bounds([0, 40000])
+    plan = stream_plan(40000, 20, 0, 64, 294 * 128, bounds, 148)
+    comp = [b - a for k, a, b in (s for s in plan if s[0] == "compress")]
+    assert all(c == 294 * 128 for c in comp[:-1])
+    score = [(a, b) for k, a, b in (s for s in plan if s[0] == "score")]
+    for a, b in score[:-1]:
+        assert sum(1 for j in range(20) for e in bounds if a < j * 40000 + e <= b) == 148
+
+
+def _stream_slot(cuda, name, n_cand):
+    s = _Slot(cuda, name, n_cand)
+    s.L_u, s.domain = [64], [1]
+    s.kv = [_Buf(cuda, f"{name}.kv")]
+    s.model = "model"
+    return s
+
+
+class _FakeApi:
+    def __init__(self, cuda):
+        self.cuda = cuda
+
+    def compress_targets(self, model, x, tokens, stream=None):
+        stream.launch([x.name], [tokens.name], f"compress {x.name}")
+
+    def score_candidates(self, model, tokens, off, kv, lu, dm, scores, stream=None):
+        stream.launch([tokens.name] + [k.name for k in kv], [scores.name], f"score {[k.name for k in kv]}")
+
+    def kernel_launches(self):
+        return 0
+
+
+@pytest.mark.parametrize("n_cand,count,n_slots", [(40000, 9, 4), (300, 8, 3)])
+def test_streamed_steps_have_no_stream_races(fake_cuda, monkeypatch, n_cand, count, n_slots):
+    from transformer_candidate_scoring_b200.pipeline import unit_bounds
+    pipeline, fake, log = fake_cuda
+    monkeypatch.setattr(pipeline, "api", _FakeApi(fake.cuda))
+    st = object.__new__(pipeline.Streamed)
+    st.slots = [_stream_slot(fake.cuda, f"slot{k}", n_cand) for k in range(n_slots)]
+    st.n = n_cand
+    st.X, st.tokens, st.scores = (_Buf(fake.cuda, "ring.X"), _Buf(fake.cuda, "ring.tokens"),
+                                  _Buf(fake.cuda, "ring.scores"))
+    st.comp_chunk, st.score_units, st.bounds = 294 * 128 if n_cand > 1000 else 500, 148 if n_cand > 1000 else 2, \
+        unit_bounds([0, n_cand])
+    st.user = fake.cuda.Stream()
+    resident = [(_Bags(fake.cuda, f"set{k}.user"), _Bags(fake.cuda, f"set{k}")) for k in range(3)]
+    done = []
+
+    def bind(i, dw, main):
+        dw.use_bags(*resident[i % 3], None)
+
+    def scored(i, dw, s):
+        done.append(i)
+        out = _Buf(fake.cuda, f"out{i}")
+        with fake.cuda.stream(s):
+            out.copy_(dw.scores)
+
+    st.run(2, count, fake.cuda.current_stream(), bind=bind, scored=scored)
+    assert done == list(range(2, 2 + count))
+    assert _races(log) == []
+
+
+@pytest.mark.parametrize("n_bag_slots", [2, 3])
+def test_host_feed_streamed_has_no_stream_races(fake_cuda, monkeypatch, n_bag_slots):
+    from transformer_candidate_scoring_b200.pipeline import unit_bounds
+    pipeline, fake, log = fake_cuda
+    monkeypatch.setattr(pipeline, "api", _FakeApi(fake.cuda))
+    st = object.__new__(pipeline.Streamed)
+    st.slots = [_stream_slot(fake.cuda, f"slot{k}", 40000) for k in range(4)]
+    st.n = 40000
+    st.X, st.tokens, st.scores = (_Buf(fake.cuda, "ring.X"), _Buf(fake.cuda, "ring.tokens"),
+                                  _Buf(fake.cuda, "ring.scores"))
+    st.comp_chunk, st.score_units, st.bounds = 294 * 128, 148, unit_bounds([0, 40000])
+    st.user = fake.cuda.Stream()
+    batches = [(_Bags(fake.cuda, f"host{k}.user"), _Bags(fake.cuda, f"host{k}.target"), None) for k in range(3)]
+    feed = pipeline.HostFeed(st.slots[0], batches, n_bag_slots=n_bag_slots)
+    host_scores = [_Buf(fake.cuda, f"host_scores{k}") for k in range(2)]
+    feed.run_overlapped(st, 0, 9, host_scores, fake.cuda.current_stream())
+    labels = [o[4] for o in log.ops]
+    assert sum(l.startswith("copy host") for l in labels) == 9 * 8
+    assert sum("-> host_scores" in l for l in labels) == 9
+    assert _races(log) == []

@@ -17,9 +17,10 @@
 //                   accumulate into it in place
 //     [D, D + 128)  work area W, in turn: own K, own V, Q (each read out by the epilogue),
 //                   the scores of one head group (numerators written back over them as
-//                   fp16, the A operand of P V, whose result lands beside them), the FFN
-//                   hidden units (a 128-wide half at a time; ReLU written back as fp16, the
-//                   A operand of W2)
+//                   fp16, the A operand of P V and of a product with ones, whose results,
+//                   the attention numerator sums and the row sum, land beside them), the
+//                   FFN hidden units (a 128-wide half at a time; ReLU written back as fp16,
+//                   the A operand of W2)
 //   shared memory
 //     A      per slot [128 x D] fp16: LN1 output -> Q -> attention output -> LN2 output
 //     KV     the unit's K and V^T images of the current layer (score mode: loaded by bulk
@@ -70,6 +71,10 @@ constexpr int kMaxStages = 4;
 constexpr int kMaxLp = 128;
 constexpr float kL2E = 1.44269504088896341f;
 constexpr int kSmemLimit = 232448;
+// The constant operands: the [128 x 16] A tile whose columns 0 and 1 are ones (bias
+// products), then at kOnesBOff a [16 x 16] B tile of ones (row sums of the numerators).
+constexpr int kOnesBOff = kM * 16 * 2;
+constexpr int kOnesBytes = kOnesBOff + 1024;
 
 // fp16 x fp16 -> fp32, both operands K-major
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
@@ -112,11 +117,15 @@ struct Cfg<64> {
 template <int D>
 constexpr int vec_floats() { return D + 4; }
 
-// Head groups of one launch: a head's scores take SW work-area columns (SW = 32, 64 or 128,
-// at least the launch's longest padded user sequence), a group is the HG heads that fit.
+// Head groups of one launch: SW (32, 64 or 128) is at least the launch's longest padded user
+// sequence.  A head owns HW = max(SW, 64) work-area columns: its scores (Lp columns), then,
+// written over them, its numerators as fp16 pairs (Lp / 2 columns), and from column HW / 2
+// the P V product (16 columns) and the numerators' row sum (16 equal columns).  A group is
+// the HG heads that fit.
 template <int D, int SW>
 struct Groups {
-  static constexpr int HG = kWork / SW;
+  static constexpr int HW = SW < 64 ? 64 : SW;
+  static constexpr int HG = kWork / HW;
   static constexpr int NG = Cfg<D>::kNH / HG;
   static_assert(SW == 32 || SW == 64 || SW == 128, "head slot width");
 };
@@ -210,6 +219,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   tmem_ld16(taddr, v);
   tmem_ld16(taddr + 16, v + 16);
 }
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+  return __uint_as_float(r);
+}
 __device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t* r) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
                "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
@@ -224,44 +238,20 @@ __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-// 2^x on the FMA pipe, for the share of the softmax exponentials that the MUFU pipe would
-// otherwise queue: x = n + f with n = round(x) (the 1.5 * 2^23 addition rounds x into t's low
-// bits), 2^f from a cubic fitted to minimise the relative error on [-1/2, 1/2] (7.6e-5, below
-// half an fp16 unit, the precision the numerators are kept in), 2^n added into the exponent
-// field.  Below -125 (masked keys are -inf) the result is 0, so that the exponent field
-// never wraps.
-__device__ __forceinline__ float exp2_fma(float x) {
-  const float xc = fmaxf(x, -125.f);
-  const float t = xc + 12582912.f;
-  const float f = xc - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(0.0551727042f, f, 0.242614001f), f, 0.693261027f), f, 0.999927819f);
-  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-  return x >= -125.f ? r : 0.f;
+// Softmax numerators two at a time: the exponents x (fp32, already shifted by the row
+// maximum, so x <= 0) are rounded to an fp16 pair and raised by one packed 2^x, giving the
+// fp16 numerators that the P V product consumes.  -inf (a masked key) gives 0.  Every path and slot width computes a key this way, so that a candidate's score
+// does not depend on the other requests of its launch.
+__device__ __forceinline__ uint32_t exp2_h2(float a, float b) {   // a -> low half
+  uint32_t h, r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(b), "f"(a));
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h));
+  return r;
 }
-
-// The numerator of key chunk c (16 keys): every path and slot width computes the same key
-// with the same function, so that a candidate's score does not depend on the other requests
-// of its launch.
-__device__ __forceinline__ float softmax_exp(float x, int c) { return c == 3 ? exp2_fma(x) : ex2(x); }
-
-// Bounded wait that polls without suspending the thread first (the MMA-issuing threads wait
-// for one event at a time and react faster this way).
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
-#pragma unroll 1
-  for (int i = 0; i < 4096; ++i)
-    if (mbar_test(bar, parity)) return true;
-  return mbar_wait(bar, parity, abort_flag);
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Bounded wait of one thread for its own bulk copies in flight, used while unwinding.
@@ -341,7 +331,7 @@ __device__ void mma_issuer(const StackParams& p, int slot, uint32_t tmem, uint32
   uint32_t phase = 0, ph_e = 0, ph_kv = 0, ph_mm = 0;
   bool ok = true, store_pending = false;
   auto wait_e = [&]() {
-    ok = ok && mbar_wait_spin(e2m, ph_e, abort_flag);
+    ok = ok && mbar_wait(e2m, ph_e, abort_flag);
     ph_e ^= 1;
     tc_fence_after();
     return ok;
@@ -360,7 +350,7 @@ __device__ void mma_issuer(const StackParams& p, int slot, uint32_t tmem, uint32
     const bool last = pi == C::kPieces - 1 || C::piece(pi + 1).item != pc.item;
     if (!ok) return;
     if (first) {
-      if (!(ok = mbar_wait_spin(b.full(stage), phase, abort_flag))) return;
+      if (!(ok = mbar_wait(b.full(stage), phase, abort_flag))) return;
       tc_fence_after();
     }
     const uint32_t item = ring + stage * C::kItemBytes;
@@ -426,22 +416,24 @@ __device__ void mma_issuer(const StackParams& p, int slot, uint32_t tmem, uint32
         ph_kv ^= 1;
         tc_fence_after();
       }
-      constexpr int HG = Groups<D, SW>::HG;
+      constexpr int HG = Groups<D, SW>::HG, HW = Groups<D, SW>::HW;
       const int ng = t.Lp > 0 ? Groups<D, SW>::NG : 0;
       for (int g = 0; g < ng && ok; ++g) {
         for (int i = 0; i < HG; ++i) {                 // scores of the group's heads
           const int h = g * HG + i;
-          mma_bf16(tW + i * SW, sdesc(sA + h * 4096, 2048, 128),
+          mma_bf16(tW + i * HW, sdesc(sA + h * 4096, 2048, 128),
                    sdesc(sKV + 2 * h * (t.Lp / 8) * 128, (t.Lp / 8) * 128, 128), idS, 0u);
         }
         mma_commit(m2e);
         if (!wait_e()) break;                          // numerators written
-        for (int i = 0; i < HG; ++i) {                 // P V beside each head's numerators
+        for (int i = 0; i < HG; ++i) {                 // P V and the row sum beside them
           const int h = g * HG + i;
-          const uint32_t pc = tW + i * SW;
-          for (int kk = 0; kk < t.Lp / 16; ++kk)
-            mma_bf16_ta(pc + SW / 2, pc + kk * 8, sdesc(vimg + (2 * kk * (D / 8) + 2 * h) * 128, (D / 8) * 128, 128),
+          const uint32_t pc = tW + i * HW;
+          for (int kk = 0; kk < t.Lp / 16; ++kk) {
+            mma_bf16_ta(pc + HW / 2, pc + kk * 8, sdesc(vimg + (2 * kk * (D / 8) + 2 * h) * 128, (D / 8) * 128, 128),
                         ID16, kk > 0 ? 1u : 0u);
+            mma_bf16_ta(pc + HW / 2 + 16, pc + kk * 8, sdesc(sOnes + kOnesBOff, 256, 128), ID16, kk > 0 ? 1u : 0u);
+          }
         }
         if (!UM && g == ng - 1) mma_commit(b.kv_empty(slot));
         mma_commit(m2e);
@@ -493,27 +485,34 @@ struct Epi {
   // its second head group, or through its own-V phase when the weight ring is two items
   // deep), so that the two slots' phases interleave: one slot's softmax runs while the
   // tensor core serves the other slot's projections.
+  // (A warp takes every wait's outcome together, so that its lanes leave together when a
+  // wait gives up and the single-lane arrivals below always see the whole warp.)
   __device__ __forceinline__ bool acquire() {
     if (paired && slot == 1) {
-      ok = ok && mbar_wait(gate, gph, abort_flag);
+      ok = __all_sync(0xffffffffu, ok && mbar_wait(gate, gph, abort_flag));
       gph ^= 1;
     }
     return ok;
   }
   __device__ __forceinline__ void open_gate() {
-    if (paired && slot == 0) mbar_arrive(gate);
+    __syncwarp();
+    if (paired && slot == 0 && (m & 31) == 0) mbar_arrive(gate);
   }
   __device__ __forceinline__ bool wait() {
-    ok = ok && mbar_wait(m2e, ph, abort_flag);
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(m2e, ph, abort_flag));
     ph ^= 1;
     tc_fence_after();
     return ok;
   }
+  // Each thread completes its tensor-memory stores and orders its shared-memory stores
+  // before the tensor core's reads; then one lane per warp arrives for the whole warp (128
+  // arrivals on one barrier queue behind each other, four do not).
   __device__ __forceinline__ void signal() {
     tmem_wait_st();
     fence_proxy_async_smem();
     tc_fence_before();
-    mbar_arrive(e2m);
+    __syncwarp();
+    if ((m & 31) == 0) mbar_arrive(e2m);
   }
 };
 
@@ -525,21 +524,40 @@ __device__ __forceinline__ void load_row(uint32_t taddr, float* y) {
   reg_fence<D>(y);
 }
 
-// Row mean and 1/sqrt(var + eps) (two passes over the registers).
+// Packed fp32 pairs (one instruction for two lanes' worth of values).
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ float lo32(uint64_t r) { return __uint_as_float((uint32_t)r); }
+__device__ __forceinline__ float hi32(uint64_t r) { return __uint_as_float((uint32_t)(r >> 32)); }
+
+// s_lo += lo(a) lo(b), s_hi += hi(a) hi(b) for two fp16 pairs: the products are exact in
+// fp32, the sums fp32.
+__device__ __forceinline__ void fma_h2(float& s_lo, float& s_hi, uint32_t a, uint32_t b) {
+  asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %2;\n\tmov.b32 {b0, b1}, %3;\n\t"
+      "fma.rn.f32.f16 %0, a0, b0, %0;\n\tfma.rn.f32.f16 %1, a1, b1, %1;\n\t}"
+      : "+f"(s_lo), "+f"(s_hi)
+      : "r"(a), "r"(b));
+}
+
+// Row mean and 1/sqrt(var + eps) (two passes over the registers, on packed pairs).
 template <int D>
 __device__ __forceinline__ float2 row_stats(const float* y) {
-  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  uint64_t a[2] = {0ull, 0ull};
 #pragma unroll
-  for (int i = 0; i < D; ++i) a[i & 3] += y[i];
-  const float mean = ((a[0] + a[1]) + (a[2] + a[3])) * (1.f / D);
+  for (int i = 0; i < D / 2; ++i) a[i & 1] = add_f32x2(a[i & 1], f32x2(y[2 * i], y[2 * i + 1]));
+  const float mean = ((lo32(a[0]) + lo32(a[1])) + (hi32(a[0]) + hi32(a[1]))) * (1.f / D);
+  const uint64_t nm = f32x2(-mean, -mean);
+  a[0] = a[1] = 0ull;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) a[i] = 0.f;
-#pragma unroll
-  for (int i = 0; i < D; ++i) {
-    const float d = y[i] - mean;
-    a[i & 3] = fmaf(d, d, a[i & 3]);
+  for (int i = 0; i < D / 2; ++i) {
+    const uint64_t d = add_f32x2(f32x2(y[2 * i], y[2 * i + 1]), nm);
+    a[i & 1] = fma2(d, d, a[i & 1]);
   }
-  return make_float2(mean, rsqrtf(((a[0] + a[1]) + (a[2] + a[3])) * (1.f / D) + kLnEps));
+  const float ss = (lo32(a[0]) + lo32(a[1])) + (hi32(a[0]) + hi32(a[1]));
+  return make_float2(mean, rsqrtf(ss * (1.f / D) + kLnEps));
 }
 
 // The row standardized (LayerNorm without its gain and shift, which the next product's
@@ -547,17 +565,21 @@ __device__ __forceinline__ float2 row_stats(const float* y) {
 template <int D>
 __device__ __forceinline__ void ln_to_A(const Epi& e, const float* y) {
   const float2 st = row_stats<D>(y);
-  const float nmr = -st.x * st.y;
+  const uint64_t r2 = f32x2(st.y, st.y), n2 = f32x2(-st.x * st.y, -st.x * st.y);
 #pragma unroll
   for (int kc = 0; kc < D / 8; ++kc) {
-    float v[8];
+    uint32_t h[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = fmaf(y[8 * kc + i], st.y, nmr);
-    st_row8h(e.sA + kc * 2048 + e.rowoff, v);
+    for (int i = 0; i < 4; ++i) {
+      const uint64_t v = fma2(f32x2(y[8 * kc + 2 * i], y[8 * kc + 2 * i + 1]), r2, n2);
+      h[i] = pack_h2(lo32(v), hi32(v));
+    }
+    st_shared_v4(e.sA + kc * 2048 + e.rowoff, h[0], h[1], h[2], h[3]);
   }
 }
 
-// 128 columns of the work area -> ReLU -> fp16 pairs in its first 64 columns (in place: every
+// 128 columns of the work area -> fp16 -> ReLU (max with 0 on the pairs; rounding keeps
+// the sign, so this equals rounding after the ReLU) -> its first 64 columns (in place: every
 // value is read before the first store).
 __device__ __forceinline__ void relu_in_place(uint32_t tW) {
   float h[128];
@@ -569,17 +591,23 @@ __device__ __forceinline__ void relu_in_place(uint32_t tW) {
   for (int c = 0; c < 4; ++c) {
     uint32_t r[16];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) r[i] = pack_h2(fmaxf(h[32 * c + 2 * i], 0.f), fmaxf(h[32 * c + 2 * i + 1], 0.f));
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t v = pack_h2(h[32 * c + 2 * i], h[32 * c + 2 * i + 1]);
+      asm("max.f16x2 %0, %1, %2;" : "=r"(r[i]) : "r"(v), "r"(0u));
+    }
     tmem_st16u(tW + 16 * c, r);
   }
 }
 
-// Softmax of one head's row over its Lp key columns at `base` (keys >= L_u masked) together
-// with the own key's score `sself` (-inf when there is none): numerators as fp16 pairs over
-// the first Lp/2 columns; returns (own numerator, 1 / sum).
+// Softmax numerators of one head's row over its Lp key columns at `base` (keys >= L_u
+// masked), with the own key's score `sself` (-inf when there is none) in the maximum: the
+// numerators go back as fp16 pairs over the first Lp / 2 columns; returns the own key's
+// numerator.  The row sum of the numerators comes from the tensor core (a product with a
+// tile of ones, beside P V), so it adds exactly the fp16 values that P V weighs.
 template <int SW>
-__device__ __forceinline__ float2 softmax_head(uint32_t base, int Lp, int L_u, float sself) {
+__device__ __forceinline__ float softmax_head(uint32_t base, int Lp, int L_u, float sself) {
   const int nb = Lp / 16;
+  float mx;
   if constexpr (SW <= 64) {
     float sv[SW];
 #pragma unroll
@@ -587,7 +615,7 @@ __device__ __forceinline__ float2 softmax_head(uint32_t base, int Lp, int L_u, f
       if (c < nb) tmem_ld16(base + 16 * c, sv + 16 * c);
     tmem_wait_ld();
     reg_fence<SW>(sv);
-    if (L_u < SW) {   // keys past L_u (and unloaded chunks) out of the maximum and the sums
+    if (L_u < SW) {   // keys past L_u (and unloaded chunks) out of the maximum
 #pragma unroll
       for (int i = 0; i < SW; ++i)
         if (i >= L_u) sv[i] = -INFINITY;
@@ -600,28 +628,23 @@ __device__ __forceinline__ float2 softmax_head(uint32_t base, int Lp, int L_u, f
       m4[2] = max3(m4[2], sv[i + 4], sv[i + 5]);
       m4[3] = max3(m4[3], sv[i + 6], sv[i + 7]);
     }
-    const float nm = -fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * kL2E;
-    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+    mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+    const uint64_t l2 = f32x2(kL2E, kL2E), n2 = f32x2(-mx * kL2E, -mx * kL2E);
 #pragma unroll
     for (int c = 0; c < SW / 16; ++c)
       if (c < nb) {
         uint32_t r[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          // a quarter of the exponentials (the fourth chunk of 16 keys) on the FMA pipe
-          sv[16 * c + i] = softmax_exp(fmaf(sv[16 * c + i], kL2E, nm), c);
-          s4[i & 3] += sv[16 * c + i];
+        for (int i = 0; i < 8; ++i) {
+          const uint64_t x = fma2(f32x2(sv[16 * c + 2 * i], sv[16 * c + 2 * i + 1]), l2, n2);
+          r[i] = exp2_h2(lo32(x), hi32(x));
         }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) r[i] = pack_h2(sv[16 * c + 2 * i], sv[16 * c + 2 * i + 1]);
         tmem_st8u(base + 8 * c, r);
       }
-    const float ps = ex2(fmaf(sself, kL2E, nm));
-    return make_float2(ps, 1.f / (((s4[0] + s4[1]) + (s4[2] + s4[3])) + ps));
   } else {
     // two passes over 16-key chunks: the maximum, then the numerators (chunk c's numerators
     // land in columns 8c .. 8c + 7, which only chunks up to c have occupied)
-    float mx = sself;
+    mx = sself;
 #pragma unroll 1
     for (int c = 0; c < nb; ++c) {
       float v[16];
@@ -632,27 +655,26 @@ __device__ __forceinline__ float2 softmax_head(uint32_t base, int Lp, int L_u, f
       for (int i = 0; i < 16; ++i)
         if (16 * c + i < L_u) mx = fmaxf(mx, v[i]);
     }
-    const float nm = -mx * kL2E;
-    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint64_t l2 = f32x2(kL2E, kL2E), n2 = f32x2(-mx * kL2E, -mx * kL2E);
 #pragma unroll 1
     for (int c = 0; c < nb; ++c) {
       float v[16];
       tmem_ld16(base + 16 * c, v);
       tmem_wait_ld();
       reg_fence<16>(v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (16 * c + i >= L_u) v[i] = -INFINITY;
       uint32_t r[8];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        v[i] = 16 * c + i < L_u ? softmax_exp(fmaf(v[i], kL2E, nm), c) : 0.f;
-        s4[i & 3] += v[i];
+      for (int i = 0; i < 8; ++i) {
+        const uint64_t x = fma2(f32x2(v[2 * i], v[2 * i + 1]), l2, n2);
+        r[i] = exp2_h2(lo32(x), hi32(x));
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) r[i] = pack_h2(v[2 * i], v[2 * i + 1]);
       tmem_st8u(base + 8 * c, r);
     }
-    const float ps = ex2(fmaf(sself, kL2E, nm));
-    return make_float2(ps, 1.f / (((s4[0] + s4[1]) + (s4[2] + s4[3])) + ps));
   }
+  return ex2(fmaf(sself, kL2E, -mx * kL2E));
 }
 
 template <int D, int SW, bool UM>
@@ -690,26 +712,25 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
       ln_to_A<D>(e, y);
     }
     e.signal();
-    // ---- own K and V (user mode: this row of the layer's K and V^T images), read in two
-    // halves of D/2 columns
+    // ---- own K and V (user mode: this row of the layer's K and V^T images), read 32
+    // columns at a time (the packed K stays live while V is read)
     uint32_t kreg[UM ? 1 : D / 2], vreg[UM ? 1 : D / 2];
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
       if (!e.wait()) return;
 #pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {
-        float x[D / 2];
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) tmem_ld32(e.tW + D / 2 * hb + 32 * c, x + 32 * c);
+      for (int hb = 0; hb < D / 32; ++hb) {
+        float x[32];
+        tmem_ld32(e.tW + 32 * hb, x);
         tmem_wait_ld();
-        reg_fence<D / 2>(x);
+        reg_fence<32>(x);
         if constexpr (UM) {
           if (m < t.Lp) {
             const bool real = m < t.L_u;
             if (pass == 0) {   // K image [Lp x D]: row m, eight columns per core-matrix row
 #pragma unroll
-              for (int j = 0; j < D / 16; ++j) {
-                const int cc = D / 16 * hb + j;
+              for (int j = 0; j < 4; ++j) {
+                const int cc = 4 * hb + j;
                 float v[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) v[i] = real ? x[8 * j + i] : 0.f;
@@ -718,8 +739,8 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
             } else {           // V^T image [D x Lp]: column m
               const uint32_t vb = e.sKV + t.Lp * D * 2 + (m >> 3) * (D / 8) * 128 + (m & 7) * 2;
 #pragma unroll
-              for (int i = 0; i < D / 2; ++i) {
-                const int d = D / 2 * hb + i;
+              for (int i = 0; i < 32; ++i) {
+                const int d = 32 * hb + i;
                 const __half hv = __float2half_rn(real ? x[i] : 0.f);
                 asm volatile("st.shared.b16 [%0], %1;" ::"r"(vb + (d >> 3) * 128 + (d & 7) * 16),
                              "h"(*reinterpret_cast<const unsigned short*>(&hv))
@@ -729,11 +750,11 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < D / 4; ++i) {
+          for (int i = 0; i < 16; ++i) {
             if (pass == 0)
-              kreg[D / 4 * hb + i] = pack_h2(x[2 * i], x[2 * i + 1]);
+              kreg[16 * hb + i] = pack_h2(x[2 * i], x[2 * i + 1]);
             else
-              vreg[D / 4 * hb + i] = pack_h2(x[2 * i], x[2 * i + 1]);
+              vreg[16 * hb + i] = pack_h2(x[2 * i], x[2 * i + 1]);
           }
         }
       }
@@ -752,20 +773,20 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int h = 2 * hc + j;
+        uint32_t qp[8];   // the head's query as the fp16 pairs the score product reads
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qp[i] = pack_h2(q[16 * j + 2 * i], q[16 * j + 2 * i + 1]);
         if constexpr (UM) {
           sself[h] = -INFINITY;
         } else {
           float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            s0 = fmaf(q[16 * j + 2 * i], h_lo(kreg[8 * h + i]), s0);
-            s1 = fmaf(q[16 * j + 2 * i + 1], h_hi(kreg[8 * h + i]), s1);
-          }
+          for (int i = 0; i < 8; ++i) fma_h2(s0, s1, qp[i], kreg[8 * h + i]);
           sself[h] = s0 + s1;
         }
         if (UM || t.Lp > 0) {
-          st_row8h(e.sA + (2 * h) * 2048 + e.rowoff, q + 16 * j);
-          st_row8h(e.sA + (2 * h + 1) * 2048 + e.rowoff, q + 16 * j + 8);
+          st_shared_v4(e.sA + (2 * h) * 2048 + e.rowoff, qp[0], qp[1], qp[2], qp[3]);
+          st_shared_v4(e.sA + (2 * h + 1) * 2048 + e.rowoff, qp[4], qp[5], qp[6], qp[7]);
         } else {             // no user keys: the attention output is the own value
           float o[16];
 #pragma unroll
@@ -782,11 +803,11 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
     if (l == 0 && t.Lp == 0 && p.gate_phase == 1) e.open_gate();
     // ---- attention, one head group at a time (loops kept rolled: the heads of a group are
     // picked out of the per-head registers by comparison, which keeps the code small)
-    constexpr int HG = Groups<D, SW>::HG;
+    constexpr int HG = Groups<D, SW>::HG, HW = Groups<D, SW>::HW;
     if (t.Lp > 0) {
 #pragma unroll 1
       for (int g = 0; g < Groups<D, SW>::NG; ++g) {
-        float ps[HG], li[HG];
+        float ps[HG];
         if (!e.wait()) return;   // scores of group g
 #pragma unroll 1
         for (int i = 0; i < HG; ++i) {
@@ -794,26 +815,26 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
           float ss = sself[0];
 #pragma unroll
           for (int k = 1; k < NH; ++k) ss = h == k ? sself[k] : ss;
-          const float2 r = softmax_head<SW>(e.tW + i * SW, t.Lp, t.L_u, ss);
+          const float r = softmax_head<SW>(e.tW + i * HW, t.Lp, t.L_u, ss);
 #pragma unroll
           for (int k = 0; k < HG; ++k)
-            if (i == k) {
-              ps[k] = r.x;
-              li[k] = r.y;
-            }
+            if (i == k) ps[k] = r;
         }
         e.signal();
-        if (!e.wait()) return;   // P V of group g
+        if (!e.wait()) return;   // P V and the row sums of group g
 #pragma unroll
         for (int i = 0; i < HG; ++i) {
           const int h = g * HG + i;
           float o[16];
-          tmem_ld16(e.tW + i * SW + SW / 2, o);
+          tmem_ld16(e.tW + i * HW + HW / 2, o);
+          float sum = tmem_ld1(e.tW + i * HW + HW / 2 + 16);
           tmem_wait_ld();
           reg_fence<16>(o);
+          asm volatile("" : "+f"(sum));
+          const float li = rcp_approx(sum + ps[i]);
           if constexpr (UM) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) o[j] *= li[i];
+            for (int j = 0; j < 16; ++j) o[j] *= li;
           } else {
             uint32_t vv[8];
 #pragma unroll
@@ -824,8 +845,8 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
             }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              o[2 * j] = fmaf(ps[i], h_lo(vv[j]), o[2 * j]) * li[i];
-              o[2 * j + 1] = fmaf(ps[i], h_hi(vv[j]), o[2 * j + 1]) * li[i];
+              o[2 * j] = fmaf(ps[i], h_lo(vv[j]), o[2 * j]) * li;
+              o[2 * j + 1] = fmaf(ps[i], h_hi(vv[j]), o[2 * j + 1]) * li;
             }
           }
           st_row8h(e.sA + (2 * h) * 2048 + e.rowoff, o);
@@ -915,11 +936,11 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
     mbar_init(b.kv_full(), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(b.kv_empty(s), 1);
-      mbar_init(b.e2m(s), kSlotThreads);
+      mbar_init(b.e2m(s), kSlotThreads / 32);
       mbar_init(b.m2e(s), 1);
       mbar_init(b.mm(s), 1);
       mbar_init(b.drain(s), 1);
-      mbar_init(b.tok(s), kSlotThreads);
+      mbar_init(b.tok(s), kSlotThreads / 32);
     }
     *abort_flag = 0;
     mbar_fence_init();
@@ -936,6 +957,7 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       const uint32_t ro = (t >> 3) * 128 + (t & 7) * 16;
       st_row8h(sOnes + ro, one2);
       st_row8h(sOnes + 2048 + ro, zero);
+      if (t < 32) st_shared_v4(sOnes + kOnesBOff + 16 * t, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u);
     }
     if (p.off_vec >= 0) {
       const int nvec = vec_floats<D>();
@@ -1152,7 +1174,7 @@ bool plan_smem(StackParams& p, int n_layer, int lp_max, bool pair, int& smem_byt
   p.off_kv = a_bytes;
   const int kv_bytes = 2 * lp_max * D * 2;
   p.off_ones = p.off_kv + ((kv_bytes + 1023) & ~1023);
-  p.off_ring = p.off_ones + kM * 16 * 2;
+  p.off_ring = p.off_ones + kOnesBytes;
   const int vec_bytes = vec_floats<D>() * 4;
   const int fixed = p.off_ring + kBarArea;
   int stages = std::min(kMaxStages, (kSmemLimit - fixed - vec_bytes) / Cfg<D>::kItemBytes);

@@ -8,6 +8,9 @@ device by datagen's counter-based generator.
 """
 from __future__ import annotations
 
+import bisect
+import copy
+import math
 from dataclasses import dataclass
 from typing import List
 
@@ -103,7 +106,15 @@ class DeviceWorkload:
         self.req_offsets = off
         n = off[-1]
         D, F = dims.D, dims.n_target_fields
-        # every request's user tokens in one buffer (one aggregation call fills them all)
+        self._user_buffers()
+        self.X = torch.empty(n, F * D, dtype=self.dt, device=dev)
+        self.tokens = torch.empty(n, D, dtype=torch.float32, device=dev)     # compressed tokens (fp32)
+        self.scores = torch.empty(n, dtype=torch.float32, device=dev)
+
+    def _user_buffers(self) -> None:
+        """Every request's user tokens in one buffer (one aggregation call fills them all)
+        and its K/V cache."""
+        D, dev = self.w.dims.D, self.device
         uoff = np.concatenate([[0], np.cumsum(self.L_u)]).astype(int)
         self.user_tokens_all = torch.empty(max(int(uoff[-1]), 1), D, dtype=torch.float32, device=dev)
         self.user_tokens = [self.user_tokens_all[uoff[r]:uoff[r] + max(l, 1)] if l else self.user_tokens_all[:1]
@@ -111,9 +122,17 @@ class DeviceWorkload:
         self.n_user = int(uoff[-1])
         self.kv = [torch.empty(max(api.kv_cache_bytes(self.model, l), 16), dtype=torch.uint8, device=dev)
                    for l in self.L_u]
-        self.X = torch.empty(n, F * D, dtype=self.dt, device=dev)
-        self.tokens = torch.empty(n, D, dtype=torch.float32, device=dev)     # compressed tokens (fp32)
-        self.scores = torch.empty(n, dtype=torch.float32, device=dev)
+
+    def clone_slot(self, activations: bool = True) -> "DeviceWorkload":
+        """Another slot of the same workload: shares the model, tables and current bags,
+        owns its user tokens and K/V caches (and, unless ``activations`` is False, its X,
+        tokens and scores)."""
+        c = copy.copy(self)
+        c._user_buffers()
+        if activations:
+            c.X, c.tokens, c.scores = (torch.empty_like(self.X), torch.empty_like(self.tokens),
+                                       torch.empty_like(self.scores))
+        return c
 
     @property
     def n_cand(self) -> int:
@@ -393,41 +412,256 @@ class Overlapped:
         return g
 
 
+def unit_bounds(req_offsets, tile: int = SCORE_TILE, unit: int = SCORE_UNIT) -> List[int]:
+    """End offsets (within a batch) of the score kernel's units: every request is cut into
+    runs of ``unit`` tiles of ``tile`` candidates from its own start, the last one shorter."""
+    out = []
+    per = tile * unit
+    for r in range(len(req_offsets) - 1):
+        s, e = req_offsets[r], req_offsets[r + 1]
+        out.extend(range(s + per, e, per))
+        if e > s:
+            out.append(e)
+    return out
+
+
+def stream_plan(n: int, count: int, first: int, n_slots: int, comp_chunk: int, bounds: List[int],
+                score_units: int):
+    """The launch order of Streamed.run over batches first .. first + count - 1 of n
+    candidates each: a list of ("gather", j), ("compress", a, b) and ("score", a, b) with
+    candidate positions a, b counted from the start of batch ``first`` (batch j covers
+    [j n, (j + 1) n)).  A compress launch takes ``comp_chunk`` candidates of the stream and a
+    score launch ``score_units`` of the score kernel's units (``bounds``: their end offsets
+    within a batch, unit_bounds), both across batch boundaries.  A launch is shorter only
+    where it meets the end of the activation ring (n_slots batches, batch i in slot
+    i mod n_slots), the end of the run, or a slot that the next batch is about to reuse
+    (everything of batch j - n_slots is compressed and scored before batch j is gathered)."""
+    if n <= 0 or count <= 0:
+        return []
+    ring = n_slots * n
+    base = first * n                          # absolute stream position of the run's start
+    K = len(bounds)
+
+    def wrap_end(a):
+        return ((base + a) // ring + 1) * ring - base
+
+    def unit_end(a, units):                   # the position `units` unit ends after a
+        j = a // n
+        t = j * K + bisect.bisect_right(bounds, a - j * n) + units
+        return (t // K) * n + (bounds[t % K - 1] if t % K else 0)
+
+    def step_end(kind, done):
+        return done + comp_chunk if kind == "compress" else unit_end(done, score_units)
+
+    def full(done, limit, kind, out):
+        while True:
+            e = min(step_end(kind, done), wrap_end(done))
+            if e > limit:
+                return done
+            out.append((kind, done, e))
+            done = e
+
+    def flush(done, target, kind, out):
+        while done < target:
+            e = min(step_end(kind, done), wrap_end(done), target)
+            out.append((kind, done, e))
+            done = e
+        return done
+
+    plan = []
+    comp = score = 0
+    for j in range(count):
+        need = (j - n_slots + 1) * n          # batch j - n_slots leaves its slot
+        if need > 0:
+            comp = flush(comp, need, "compress", plan)
+            score = flush(score, need, "score", plan)
+        plan.append(("gather", j))
+        comp = full(comp, (j + 1) * n, "compress", plan)
+        score = full(score, comp, "score", plan)
+    comp = flush(comp, count * n, "compress", plan)
+    flush(score, count * n, "score", plan)
+    return plan
+
+
+class Streamed:
+    """Request batches scored as one stream of candidate tiles.
+
+    Overlapped cuts every batch at the score kernel's last partial round and runs the tail
+    beside the next batch.  Here the compressor and the score kernel instead take
+    fixed-size chunks of one stream of candidates that runs across batch boundaries
+    (stream_plan): by default every compress launch is two rounds of 128-candidate tiles
+    on the SMs left beside one prefill CTA, every score launch one round of the score
+    kernel's two-tile units on all SMs, whichever batches the chunk falls in.  A launch that spans two batches scores
+    each candidate against its own request's cache (the kernels take a list of requests).
+      main stream  user aggregation, target aggregation of batch i, then every compress and
+                   score chunk that has become complete (a score chunk after the prefills of
+                   the batches it covers)
+      user stream  (high priority) the prefill of batch i, once batch i - n_slots (the same
+                   slot's previous batch) has been scored
+    The slots are clones of one DeviceWorkload (DeviceWorkload.clone_slot) whose X, tokens
+    and scores are views of ring buffers laid out slot after slot, so that a chunk spanning
+    consecutive batches is one contiguous range; by default the ring takes up to 64 batches
+    within ``ring_bytes``, so its wrap (where one compress and one score launch are cut
+    short) comes rarely.  Scores are identical to those of DeviceWorkload.step.
+    """
+
+    def __init__(self, dw: DeviceWorkload, n_slots: int = None, comp_chunk: int = None, score_units: int = None,
+                 ring_bytes: int = 8 << 30):
+        n = dw.n_cand
+        dims = dw.w.dims
+        F, D = dims.n_target_fields, dims.D
+        per_batch = n * (F * D * dw.X.element_size() + 4 * D + 4)
+        if n_slots is None:                   # a ring wrap costs one partial round of each kernel
+            n_slots = int(max(4, min(64, ring_bytes // max(per_batch, 1))))
+        if n_slots < 2:
+            raise ValueError("Streamed needs at least two slots")
+        m = n_slots
+        dev = dw.device
+        self.n = n
+        self.X = torch.empty(m * n, F * D, dtype=dw.dt, device=dev)
+        self.tokens = torch.empty(m * n, D, dtype=torch.float32, device=dev)
+        self.scores = torch.empty(m * n, dtype=torch.float32, device=dev)
+        self.slots = []
+        for k in range(m):
+            c = dw.clone_slot(activations=False)
+            c.X = self.X[k * n:(k + 1) * n]
+            c.tokens = self.tokens[k * n:(k + 1) * n]
+            c.scores = self.scores[k * n:(k + 1) * n]
+            self.slots.append(c)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        self.comp_chunk = comp_chunk if comp_chunk is not None else 2 * (sms - 1) * SCORE_TILE
+        self.score_units = score_units if score_units is not None else sms
+        self.bounds = unit_bounds(dw.req_offsets)
+        _, hi = torch.cuda.Stream.priority_range()
+        self.user = torch.cuda.Stream(dev, priority=hi)
+        self.cap = torch.cuda.Stream(dev)
+        self.launches_per_step = None
+
+    def _pos(self, first: int, a: int) -> int:
+        """Ring row of stream position a of a run that starts with batch ``first``."""
+        return (first * self.n + a) % (len(self.slots) * self.n)
+
+    def _score(self, first: int, a: int, b: int, stream) -> None:
+        n, m = self.n, len(self.slots)
+        off, kv, lu, dm = [0], [], [], []
+        for j in range(a // n, (b - 1) // n + 1):
+            dw = self.slots[(first + j) % m]
+            lo, hi = max(a, j * n) - j * n, min(b, (j + 1) * n) - j * n
+            for r in range(len(dw.L_u)):
+                r0, r1 = max(dw.req_offsets[r], lo), min(dw.req_offsets[r + 1], hi)
+                if r1 > r0:
+                    off.append(off[-1] + r1 - r0)
+                    kv.append(dw.kv[r])
+                    lu.append(dw.L_u[r])
+                    dm.append(dw.domain[r])
+        p = self._pos(first, a)
+        api.score_candidates(self.slots[0].model, self.tokens[p:p + b - a], off, kv, lu, dm,
+                             self.scores[p:p + b - a], stream=stream)
+
+    def run(self, first: int, count: int, stream=None, bind=None, fronted=None, scored=None) -> None:
+        """Batches first .. first + count - 1 on ``stream`` (the caller's), which waits for
+        all of them at the end.  Hooks as in Overlapped.run: bind(i, dw, main) before batch
+        i's first launch, fronted(i, dw, main) after its target aggregation, scored(i, dw, s)
+        after the launch that completes its scores (``dw.scores``)."""
+        n, m = self.n, len(self.slots)
+        main = stream if stream is not None else torch.cuda.current_stream(self.slots[0].device)
+        start = torch.cuda.Event()
+        start.record(main)
+        self.user.wait_event(start)
+        prefilled, done_ev = {}, {}
+        waited = set()
+        score_end = 0
+        for step in stream_plan(n, count, first, m, self.comp_chunk, self.bounds, self.score_units):
+            if step[0] == "gather":
+                j = step[1]
+                i, dw = first + j, self.slots[(first + j) % m]
+                if bind is not None:
+                    bind(i, dw, main)
+                dw.user_aggregate(main)
+                fork = torch.cuda.Event()
+                fork.record(main)
+                self.user.wait_event(fork)
+                if j - m in done_ev:                # the slot's previous batch is scored
+                    self.user.wait_event(done_ev.pop(j - m))
+                dw.user_prefill(self.user)
+                prefilled[j] = torch.cuda.Event()
+                prefilled[j].record(self.user)
+                dw.target_aggregate(main)
+                if fronted is not None:
+                    fronted(i, dw, main)
+            elif step[0] == "compress":
+                _, a, b = step
+                p = self._pos(first, a)
+                api.compress_targets(self.slots[0].model, self.X[p:p + b - a], self.tokens[p:p + b - a],
+                                     stream=main)
+            else:
+                _, a, b = step
+                for j in range(a // n, (b - 1) // n + 1):
+                    if j not in waited:
+                        main.wait_event(prefilled.pop(j))
+                        waited.add(j)
+                self._score(first, a, b, main)
+                for j in range(score_end // n, b // n):   # batches completed by this launch
+                    if scored is not None:
+                        scored(first + j, self.slots[(first + j) % m], main)
+                    done_ev[j] = torch.cuda.Event()
+                    done_ev[j].record(main)
+                score_end = b
+        end = torch.cuda.Event()
+        end.record(self.user)
+        main.wait_event(end)
+
+    def capture(self, first: int, count: int, **hooks) -> "torch.cuda.CUDAGraph":
+        """run(first, count, ...) captured into one CUDA graph (warmed as in
+        Overlapped.capture)."""
+        g = torch.cuda.CUDAGraph()
+        cap = self.cap
+        warm_up_stream(cap, lambda: self.run(first, count, cap, **hooks))
+        l0 = api.kernel_launches()
+        with torch.cuda.graph(g, stream=cap):
+            self.run(first, count, cap, **hooks)
+        self.launches_per_step = (api.kernel_launches() - l0) / max(count, 1)
+        return g
+
+
 def _bag_tensors(b: DeviceBags):
     return (b.offsets, b.keys, b.weights, b.bag_table)
 
 
 class HostFeed:
     """Request batches whose bags sit in pinned host memory, scored back to back (the
-    serving case).  The bags of batch i + 1 are copied to the device on a copy stream while
-    batch i computes (two device slots, guarded by events); each batch's scores are copied
-    back to a pinned host buffer on the compute stream.
+    serving case).  The bags of the next ``n_bag_slots - 1`` batches are copied to the device
+    on a copy stream while batch i computes (``n_bag_slots`` device slots, guarded by
+    events); each batch's scores are copied back to a pinned host buffer on the stream that
+    scored them.
 
     ``batches``: list of (user bags, target bags, requests) -- each the requests' bags packed
     as pack_user_bags / pack_target_bags do, every tensor in pinned host memory; all batches
     have the requests' L_u and candidate counts of ``dw``.
     """
 
-    def __init__(self, dw: DeviceWorkload, batches):
+    def __init__(self, dw: DeviceWorkload, batches, n_bag_slots: int = 3):
+        if n_bag_slots < 2:
+            raise ValueError("HostFeed needs at least two bag slots")
         self.dw = dw
         self.batches = batches
         dev = dw.device
         self.slots = []
-        for _ in range(2):   # device buffers with the largest size any batch needs
+        for _ in range(n_bag_slots):   # device buffers with the largest size any batch needs
             def alloc(pick):
                 return DeviceBags(*(torch.empty(max(int(getattr(pick(bt), f).numel()) for bt in batches),
                                                 dtype=getattr(pick(batches[0]), f).dtype, device=dev)
                                     for f in ("offsets", "keys", "weights", "bag_table")))
             self.slots.append((alloc(lambda bt: bt[0]), alloc(lambda bt: bt[1])))
         self.copy_stream = torch.cuda.Stream(dev)
-        self.ready = [torch.cuda.Event() for _ in range(2)]
-        self.free = [torch.cuda.Event() for _ in range(2)]
+        self.ready = [torch.cuda.Event() for _ in range(n_bag_slots)]
+        self.free = [torch.cuda.Event() for _ in range(n_bag_slots)]
         self.h2d_bytes = [sum(x.numel() * x.element_size() for b in (bt[0], bt[1]) for x in _bag_tensors(b))
                           for bt in batches]
 
     def _views(self, i):
-        """Device views of slot i % 2 sized for batch i."""
-        users, target = self.slots[i % 2]
+        """Device views of bag slot i mod n_bag_slots sized for batch i."""
+        users, target = self.slots[i % len(self.slots)]
         hu, ht, _ = self.batches[i % len(self.batches)]
 
         def fit(dst, src):
@@ -438,23 +672,24 @@ class HostFeed:
         hu, ht, _ = self.batches[i % len(self.batches)]
         du, dt = self._views(i)
         cs = self.copy_stream
-        cs.wait_event(self.free[i % 2])            # batch i - 2 is done with this slot
+        S = len(self.slots)
+        cs.wait_event(self.free[i % S])            # batch i - S is done with this slot
         with torch.cuda.stream(cs):
             for d, h in ((du, hu), (dt, ht)):
                 for dx, hx in zip(_bag_tensors(d), _bag_tensors(h)):
                     dx.copy_(hx, non_blocking=True)
-        self.ready[i % 2].record(cs)
+        self.ready[i % S].record(cs)
 
     def capture(self) -> None:
         """Capture one CUDA graph per (device slot, host batch) pair, so that run() replays
         the step instead of launching its kernels one by one (on the workload's capture
         stream; see DeviceWorkload.capture_step)."""
         self.graphs = {}
-        n = len(self.batches)
-        for i in range(2 * n if n % 2 else n):       # every (slot, batch) pair occurs
+        n, S = len(self.batches), len(self.slots)
+        for i in range(n * S // math.gcd(n, S)):       # every (slot, batch) pair occurs
             du, dt = self._views(i)
             self.dw.use_bags(du, dt, self.batches[i % n][2])
-            self.graphs[(i % 2, i % n)] = self.dw.capture_step()
+            self.graphs[(i % S, i % n)] = self.dw.capture_step()
 
     def run(self, first: int, count: int, host_scores, stream=None) -> None:
         """Score batches first .. first + count - 1 (batch i uses host batch i mod len);
@@ -464,45 +699,51 @@ class HostFeed:
         start = torch.cuda.Event()
         start.record(main)
         self.copy_stream.wait_event(start)         # copies begin after work already on main
-        self._copy_in(first)
-        for i in range(first, first + count):
-            if i + 1 < first + count:
-                self._copy_in(i + 1)
-            main.wait_event(self.ready[i % 2])
+        S = len(self.slots)
+        end = first + count
+        for i in range(first, min(first + S - 1, end)):
+            self._copy_in(i)
+        for i in range(first, end):
+            if i + S - 1 < end:
+                self._copy_in(i + S - 1)
+            main.wait_event(self.ready[i % S])
             if graphs is not None:
                 with torch.cuda.stream(main):
-                    graphs[(i % 2, i % len(self.batches))].replay()
+                    graphs[(i % S, i % len(self.batches))].replay()
             else:
                 du, dt = self._views(i)
                 self.dw.use_bags(du, dt, self.batches[i % len(self.batches)][2])
                 self.dw.step(main)
-            self.free[i % 2].record(main)
+            self.free[i % S].record(main)
             host_scores[i % len(host_scores)].copy_(self.dw.scores, non_blocking=True)
 
-    def run_overlapped(self, ov: "Overlapped", first: int, count: int, host_scores, stream=None) -> None:
-        """run() through an Overlapped pair of slots (``ov.slots[0]`` is ``self.dw`` or one
-        like it): batch i computes in slot i % 2 from bag slot i % 2, batch i + 1's bags are
-        copied while batch i computes, a bag slot is refilled once the batch before has
-        finished its target aggregation, and each batch's scores are copied to the host on
-        the stream that scored them, right after its last score launch."""
+    def run_overlapped(self, ov, first: int, count: int, host_scores, stream=None) -> None:
+        """run() through an Overlapped or a Streamed scheduler ``ov`` (its slots are
+        ``self.dw`` or clones of it): batch i reads bag slot i mod n_bag_slots, the bags of
+        the next n_bag_slots - 1 batches are copied while batch i computes, a bag slot is
+        refilled once its previous batch has finished its target aggregation, and each
+        batch's scores are copied to the host on the stream that scored them, right after
+        the launch that completes them."""
         main = stream if stream is not None else torch.cuda.current_stream(self.dw.device)
-        self.ready = [torch.cuda.Event() for _ in range(2)]   # fresh: no wait on an earlier run
-        self.free = [torch.cuda.Event() for _ in range(2)]
+        S = len(self.slots)
+        self.ready = [torch.cuda.Event() for _ in range(S)]   # fresh: no wait on an earlier run
+        self.free = [torch.cuda.Event() for _ in range(S)]
         start = torch.cuda.Event()
         start.record(main)
         self.copy_stream.wait_event(start)
-        self._copy_in(first)
         end = first + count
+        for i in range(first, min(first + S - 1, end)):
+            self._copy_in(i)
 
         def bind(i, dw, m):
-            if i + 1 < end:
-                self._copy_in(i + 1)
-            m.wait_event(self.ready[i % 2])
+            if i + S - 1 < end:
+                self._copy_in(i + S - 1)
+            m.wait_event(self.ready[i % S])
             du, dt = self._views(i)
             dw.use_bags(du, dt, self.batches[i % len(self.batches)][2])
 
         def fronted(i, dw, m):
-            self.free[i % 2].record(m)
+            self.free[i % S].record(m)
 
         def scored(i, dw, back):
             with torch.cuda.stream(back):
@@ -524,7 +765,7 @@ class HostFeed:
                         dx.copy_(hx, non_blocking=True)
                 host_scores[i % len(host_scores)].copy_(scores, non_blocking=True)
 
-    def capture_overlapped(self, ov: "Overlapped", first: int, count: int, host_scores) -> "torch.cuda.CUDAGraph":
+    def capture_overlapped(self, ov, first: int, count: int, host_scores) -> "torch.cuda.CUDAGraph":
         """run_overlapped(...) captured into one CUDA graph, host copies included (on
         ``ov``'s capture stream, warmed as in Overlapped.capture)."""
         g = torch.cuda.CUDAGraph()
