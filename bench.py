@@ -642,7 +642,8 @@ def run_ours(args, rank, world, local_rank):
 def run_case(args):
     """One stage of the 128D-5L path on stand-alone seeded inputs, a few launches, no JSON:
     the target of profiler captures (small inputs; the gather case builds 8 target tables of
-    --case-rows rows, 2 GB at the default 1M, larger than L2)."""
+    --case-rows rows, 2 GB at the default 1M, larger than L2; the stream case runs the timed
+    schedule itself on the full workload, eagerly, for a launch list)."""
     import torch
 
     from transformer_candidate_scoring_b200 import api
@@ -651,6 +652,20 @@ def run_case(args):
     w = datagen.WORKLOADS[WORKLOAD]
     dims = w.dims
     n = args.case_n
+    if args.case == "stream":
+        # the timed schedule itself, eagerly: --case-reps batches of the 128D-5L workload
+        # through pipeline.Streamed (after two warm-up batches), for a launch list
+        from transformer_candidate_scoring_b200.pipeline import DeviceWorkload, Streamed
+        dw = DeviceWorkload(w, device=torch.device("cuda"))
+        st = Streamed(dw)
+        st.run(0, 2)
+        torch.cuda.synchronize()
+        st.run(2, args.case_reps)
+        torch.cuda.synchronize()
+        if api.sync_status() != 0:
+            raise RuntimeError("device status word set")
+        print("case stream: ok")
+        return
     if args.case == "gather":
         ws = datagen.scaled(w, n_cand_per_request=n, rows=args.case_rows)
         tables = [torch.empty(r, dims.D, dtype=torch.bfloat16, device="cuda") for r in ws.target_rows]
@@ -770,7 +785,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-side-configs", action="store_true", help="skip the 64D-3L, packed and large workloads")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--case", choices=["score", "compress", "prefill", "all", "gather", "bulk", "uncompressed"],
+    ap.add_argument("--case", choices=["score", "compress", "prefill", "all", "gather", "stream", "bulk",
+                                       "uncompressed"],
                     default=None,
                     help="run one stage on stand-alone inputs for a profiler (no timing, no JSON)")
     ap.add_argument("--case-n", type=int, default=40000)

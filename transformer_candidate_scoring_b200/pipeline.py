@@ -349,7 +349,9 @@ class Overlapped:
         all of them at the end.  Hooks, each given (i, slot, stream):
           bind(i, dw, main)     before batch i's first launch (point ``dw`` at its bags);
           fronted(i, dw, main)  after its target aggregation (its bags are no longer read);
-          scored(i, dw, s)      after its last score launch, on that launch's stream.
+          scored(i, dw, s)      after its last score launch, on that launch's stream; it may
+                                return a CUDA event, and ``dw.scores`` is not written again
+                                before that event.
         ``first``/``count`` only name the batches for the hooks and pick slot i % 2."""
         main = stream if stream is not None else torch.cuda.current_stream(self.slots[0].device)
         start = torch.cuda.Event()
@@ -357,10 +359,13 @@ class Overlapped:
         self.back.wait_event(start)
         self.user.wait_event(start)
         tails = {}                                  # batch -> event: its tail launches are done
+        released = {}                               # batch -> event from the scored hook
         for i in range(first, first + count):
             dw = self.slots[i % 2]
             if i - 2 in tails:                      # the slot's previous batch has finished
                 main.wait_event(tails.pop(i - 2))
+            if released.get(i - 2) is not None:     # ... and its scores have been read
+                main.wait_event(released.pop(i - 2))
             if bind is not None:
                 bind(i, dw, main)
             dw.user_aggregate(main)
@@ -381,7 +386,7 @@ class Overlapped:
             if cut is None:
                 dw.score(main)
                 if scored is not None:
-                    scored(i, dw, main)
+                    released[i] = scored(i, dw, main)
                 continue
             dw.score_range(0, cut, main)
             full = torch.cuda.Event()
@@ -390,11 +395,14 @@ class Overlapped:
             dw.compress_range(cut, n, self.back)
             dw.score_range(cut, n, self.back)
             if scored is not None:
-                scored(i, dw, self.back)
+                released[i] = scored(i, dw, self.back)
             tails[i] = torch.cuda.Event()
             tails[i].record(self.back)
         for ev in tails.values():
             main.wait_event(ev)
+        for ev in released.values():
+            if ev is not None:
+                main.wait_event(ev)
 
     def capture(self, first: int, count: int, **hooks) -> "torch.cuda.CUDAGraph":
         """run(first, count, ...) captured into one CUDA graph (replay it to run the same
@@ -562,13 +570,14 @@ class Streamed:
         """Batches first .. first + count - 1 on ``stream`` (the caller's), which waits for
         all of them at the end.  Hooks as in Overlapped.run: bind(i, dw, main) before batch
         i's first launch, fronted(i, dw, main) after its target aggregation, scored(i, dw, s)
-        after the launch that completes its scores (``dw.scores``)."""
+        after the launch that completes its scores (``dw.scores``; an event it returns is
+        waited for before the slot's scores are written again)."""
         n, m = self.n, len(self.slots)
         main = stream if stream is not None else torch.cuda.current_stream(self.slots[0].device)
         start = torch.cuda.Event()
         start.record(main)
         self.user.wait_event(start)
-        prefilled, done_ev = {}, {}
+        prefilled, done_ev, released = {}, {}, {}
         waited = set()
         score_end = 0
         for step in stream_plan(n, count, first, m, self.comp_chunk, self.bounds, self.score_units):
@@ -599,17 +608,22 @@ class Streamed:
                 for j in range(a // n, (b - 1) // n + 1):
                     if j not in waited:
                         main.wait_event(prefilled.pop(j))
+                        if released.get(j - m) is not None:   # the slot's last scores were read
+                            main.wait_event(released.pop(j - m))
                         waited.add(j)
                 self._score(first, a, b, main)
                 for j in range(score_end // n, b // n):   # batches completed by this launch
                     if scored is not None:
-                        scored(first + j, self.slots[(first + j) % m], main)
+                        released[j] = scored(first + j, self.slots[(first + j) % m], main)
                     done_ev[j] = torch.cuda.Event()
                     done_ev[j].record(main)
                 score_end = b
         end = torch.cuda.Event()
         end.record(self.user)
         main.wait_event(end)
+        for ev in released.values():
+            if ev is not None:
+                main.wait_event(ev)
 
     def capture(self, first: int, count: int, **hooks) -> "torch.cuda.CUDAGraph":
         """run(first, count, ...) captured into one CUDA graph (warmed as in
@@ -654,6 +668,7 @@ class HostFeed:
                                     for f in ("offsets", "keys", "weights", "bag_table")))
             self.slots.append((alloc(lambda bt: bt[0]), alloc(lambda bt: bt[1])))
         self.copy_stream = torch.cuda.Stream(dev)
+        self.d2h_stream = torch.cuda.Stream(dev)
         self.ready = [torch.cuda.Event() for _ in range(n_bag_slots)]
         self.free = [torch.cuda.Event() for _ in range(n_bag_slots)]
         self.h2d_bytes = [sum(x.numel() * x.element_size() for b in (bt[0], bt[1]) for x in _bag_tensors(b))
@@ -722,8 +737,8 @@ class HostFeed:
         ``self.dw`` or clones of it): batch i reads bag slot i mod n_bag_slots, the bags of
         the next n_bag_slots - 1 batches are copied while batch i computes, a bag slot is
         refilled once its previous batch has finished its target aggregation, and each
-        batch's scores are copied to the host on the stream that scored them, right after
-        the launch that completes them."""
+        batch's scores are copied to the host right after the launch that completes them, on
+        a stream of their own (the caller's stream waits for the last copy)."""
         main = stream if stream is not None else torch.cuda.current_stream(self.dw.device)
         S = len(self.slots)
         self.ready = [torch.cuda.Event() for _ in range(S)]   # fresh: no wait on an earlier run
@@ -745,11 +760,22 @@ class HostFeed:
         def fronted(i, dw, m):
             self.free[i % S].record(m)
 
-        def scored(i, dw, back):
-            with torch.cuda.stream(back):
+        def scored(i, dw, s):
+            # on a stream of its own: a device-to-host copy queued behind the bag copies
+            # must not hold up the next launches of the stream that scored the batch
+            ev = torch.cuda.Event()
+            ev.record(s)
+            self.d2h_stream.wait_event(ev)
+            with torch.cuda.stream(self.d2h_stream):
                 host_scores[i % len(host_scores)].copy_(dw.scores, non_blocking=True)
+            read = torch.cuda.Event()
+            read.record(self.d2h_stream)
+            return read                   # the slot's scores may be overwritten after this
 
         ov.run(first, count, main, bind=bind, fronted=fronted, scored=scored)
+        done = torch.cuda.Event()
+        done.record(self.d2h_stream)
+        main.wait_event(done)
 
     def copies_only(self, first: int, count: int, host_scores, scores, stream=None) -> None:
         """The host traffic of run() alone, on ``stream``: each batch's bags in (the same
