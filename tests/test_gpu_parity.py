@@ -521,7 +521,17 @@ def test_streamed_steps_match_serial_steps(name, n_cand, n_slots, comp_chunk, un
     torch.cuda.synchronize()
     assert tr().sync_status() == 0
     for i in range(n_batch):
-        assert torch.equal(out[i], ref[i % len(ref)]), ("eager", i)
+        bad = torch.nonzero(out[i] != ref[i % len(ref)]).flatten()
+        if bad.numel():
+            # which side is off: score the batch serially once more
+            dw.use_bags(*_set_bags(dw, sets, i))
+            dw.step()
+            torch.cuda.synchronize()
+            again = dw.scores.clone()
+        assert bad.numel() == 0, ("eager", i, bad.numel(), sorted(set((bad // 128).tolist()))[:20],
+                                  float((out[i] - ref[i % len(ref)]).abs().max()),
+                                  "serial again == serial" if torch.equal(again, ref[i % len(ref)]) else
+                                  "serial again == streamed" if torch.equal(again, out[i]) else "three ways")
     g = st.capture(0, n_batch, bind=bind, scored=scored)
     for o in out:
         o.zero_()
@@ -533,18 +543,28 @@ def test_streamed_steps_match_serial_steps(name, n_cand, n_slots, comp_chunk, un
 
 
 def test_full_request_scores_repeat_bit_identical():
-    """A 40,000-candidate request (148 two-tile units on every SM at once, then single tiles)
-    scored five times gives the same bits each time: no hand-off between the two tiles a CTA
-    holds depends on timing."""
+    """A 40,000-candidate request: 148 two-tile units on every SM at once, then 17 single
+    tiles on 17 of the same CTAs.  Scored 20 times (every other time after the gather and the
+    compressor have cycled the caches), it gives the same bits each time, and the same bits
+    as two launches that hold no single tile behind a pair (one round of 148 units, then the
+    rest).  A CTA that moves from a pair to a single tile must not reload the K/V images
+    while the pair's second tile still reads them."""
     from transformer_candidate_scoring_b200.pipeline import DeviceWorkload
     w = datagen.scaled(datagen.WORKLOADS["128d5l"], n_cand_per_request=40000, rows=20000)
     dw = DeviceWorkload(w)
     dw.step()
-    first = dw.scores.clone()
-    for _ in range(4):
+    dw.score_range(0, 37888)
+    dw.score_range(37888, 40000)
+    torch.cuda.synchronize()
+    ref = dw.scores.clone()
+    for k in range(20):
+        if k % 2:
+            dw.target_aggregate()
+            dw.compress()
         dw.score()
         torch.cuda.synchronize()
-        assert torch.equal(dw.scores, first)
+        bad = torch.nonzero(dw.scores != ref).flatten()
+        assert bad.numel() == 0, (k, sorted(set((bad // 128).tolist()))[:20])
     assert tr().sync_status() == 0
 
 

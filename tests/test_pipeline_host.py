@@ -377,7 +377,7 @@ def test_compress_range_passes_row_views(monkeypatch):
 
 # ---------------------------------------------------------------- the candidate stream (Streamed)
 
-def _check_plan(plan, n, count, first, n_slots, comp_chunk, bounds, score_units):
+def _check_plan(plan, n, count, first, n_slots, comp_chunk, bounds, score_units, group=1):
     """Every candidate is gathered, compressed and scored once, in that order, each before
     its ring slot is gathered over; launches have their full size except where a ring wrap,
     a slot reuse or the end of the run cuts them; score launches end on unit ends."""
@@ -409,17 +409,26 @@ def _check_plan(plan, n, count, first, n_slots, comp_chunk, bounds, score_units)
     assert gathered == count - 1 and comp == score == count * n
 
 
+@pytest.mark.parametrize("group", [1, 2, 3])
 @pytest.mark.parametrize("n,count,first,n_slots,comp_chunk,units", [
     (40000, 12, 3, 64, 294 * 128, 148),      # the 128D-5L batch: no wrap inside the run
     (40000, 12, 3, 4, 294 * 128, 148),       # wraps every four batches
     (300, 9, 0, 2, 1000, 3),                 # chunks longer than a batch: slot reuse forces flushes
     (1000, 7, 5, 3, 384, 5),
 ])
-def test_stream_plan_covers_every_candidate_once(n, count, first, n_slots, comp_chunk, units):
+def test_stream_plan_covers_every_candidate_once(n, count, first, n_slots, comp_chunk, units, group):
     from transformer_candidate_scoring_b200.pipeline import stream_plan, unit_bounds
     bounds = unit_bounds([0, n])
-    plan = stream_plan(n, count, first, n_slots, comp_chunk, bounds, units)
+    plan = stream_plan(n, count, first, n_slots, comp_chunk, bounds, units, group)
     _check_plan(plan, n, count, first, n_slots, comp_chunk, bounds, units)
+    if group > 1:                             # compute launches only after every group-th gather
+        last_gather = -1
+        for step in plan:
+            if step[0] == "gather":
+                last_gather = step[1]
+            elif last_gather + 1 < count and (last_gather + 1) % group:
+                assert step[2] <= (last_gather + 1) * n and any(
+                    s[0] == "gather" and s[1] == last_gather + 1 for s in plan)   # a forced flush
 
 
 def test_stream_plan_packed_batches_and_steady_state():
@@ -433,7 +442,7 @@ def test_stream_plan_packed_batches_and_steady_state():
         assert bounds[-1] == n and sorted(bounds) == bounds
         count, first, n_slots = int(rng.integers(1, 9)), int(rng.integers(0, 5)), int(rng.integers(2, 6))
         comp_chunk, units = int(rng.integers(1, 2000)), int(rng.integers(1, 12))
-        plan = stream_plan(n, count, first, n_slots, comp_chunk, bounds, units)
+        plan = stream_plan(n, count, first, n_slots, comp_chunk, bounds, units, int(rng.integers(1, 4)))
         _check_plan(plan, n, count, first, n_slots, comp_chunk, bounds, units)
     # the 128D-5L batch in steady state: every launch between the first and the last two is
     # full size (294 compressor tiles, 148 score units)
@@ -468,8 +477,9 @@ class _FakeApi:
         return 0
 
 
-@pytest.mark.parametrize("n_cand,count,n_slots", [(40000, 9, 4), (300, 8, 3)])
-def test_streamed_steps_have_no_stream_races(fake_cuda, monkeypatch, n_cand, count, n_slots):
+@pytest.mark.parametrize("n_cand,count,n_slots,group", [(40000, 9, 4, 1), (300, 8, 3, 1), (40000, 9, 4, 2),
+                                                        (300, 8, 3, 3)])
+def test_streamed_steps_have_no_stream_races(fake_cuda, monkeypatch, n_cand, count, n_slots, group):
     from transformer_candidate_scoring_b200.pipeline import unit_bounds
     pipeline, fake, log = fake_cuda
     monkeypatch.setattr(pipeline, "api", _FakeApi(fake.cuda))
@@ -480,6 +490,7 @@ def test_streamed_steps_have_no_stream_races(fake_cuda, monkeypatch, n_cand, cou
                                   _Buf(fake.cuda, "ring.scores"))
     st.comp_chunk, st.score_units, st.bounds = 294 * 128 if n_cand > 1000 else 500, 148 if n_cand > 1000 else 2, \
         unit_bounds([0, n_cand])
+    st.group = group
     st.user = fake.cuda.Stream()
     resident = [(_Bags(fake.cuda, f"set{k}.user"), _Bags(fake.cuda, f"set{k}")) for k in range(3)]
     done = []
@@ -509,6 +520,7 @@ def test_host_feed_streamed_has_no_stream_races(fake_cuda, monkeypatch, n_bag_sl
     st.X, st.tokens, st.scores = (_Buf(fake.cuda, "ring.X"), _Buf(fake.cuda, "ring.tokens"),
                                   _Buf(fake.cuda, "ring.scores"))
     st.comp_chunk, st.score_units, st.bounds = 294 * 128, 148, unit_bounds([0, 40000])
+    st.group = 2
     st.user = fake.cuda.Stream()
     batches = [(_Bags(fake.cuda, f"host{k}.user"), _Bags(fake.cuda, f"host{k}.target"), None) for k in range(3)]
     feed = pipeline.HostFeed(st.slots[0], batches, n_bag_slots=n_bag_slots)

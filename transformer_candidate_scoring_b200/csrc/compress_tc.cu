@@ -460,6 +460,8 @@ __global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant_
     *abort_flag = 0;
     mbar_fence_init();
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.xmap)) : "memory");
+    // the grid's weight slices (one contiguous image) into L2 at once
+    prefetch_l2_share(p.w1, ((size_t)p.c0 * p.c1 + (size_t)p.c1 * p.c2 + (size_t)p.c2 * p.c3) * 2);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), 512);

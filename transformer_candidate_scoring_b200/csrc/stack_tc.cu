@@ -289,11 +289,13 @@ __device__ void weight_producer(const StackParams& p, uint32_t ring, const Bars&
 }
 
 // The unit's K/V images of each layer (score mode; warp 3, one thread).  A layer's images are
-// loaded once every active slot has finished the previous layer's attention.
+// loaded once every slot that used the images now in shared memory has finished its
+// attention on them: slot 1 releases them only in units where it holds a tile, and the unit
+// before a single-tile unit may still have slot 1 at work on its last layer.
 template <int D>
 __device__ void kv_producer(const StackParams& p, uint32_t sKV, const Bars& b, volatile int* abort_flag) {
   uint32_t ph0 = 0, ph1 = 0;
-  bool ok = true, pending = false;
+  bool ok = true, pending = false, slot1_reads = false;
   uint32_t pend_par = 0, kv_phase = 0;
   for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
     const Tile t0 = tile_of<D>(p, u, 0), t1 = tile_of<D>(p, u, 1);
@@ -301,10 +303,11 @@ __device__ void kv_producer(const StackParams& p, uint32_t sKV, const Bars& b, v
     for (int l = 0; l < p.n_layer && ok; ++l) {
       if (!(ok = mbar_wait(b.kv_empty(0), ph0 ^ 1, abort_flag))) break;
       ph0 ^= 1;
-      if (t1.active) {
-        if (!(ok = mbar_wait(b.kv_empty(1), ph1 ^ 1, abort_flag))) break;
+      if (slot1_reads) {   // slot 1's release of the previous images (its ph1-th release)
+        if (!(ok = mbar_wait(b.kv_empty(1), ph1, abort_flag))) break;
         ph1 ^= 1;
       }
+      slot1_reads = t1.active;
       if (bytes) {
         mbar_arrive_expect_tx(b.kv_full(), bytes);
         bulk_g2s(sKV, p.req[t0.r].kv + (size_t)l * bytes, bytes, b.kv_full());
@@ -944,6 +947,15 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
     }
     *abort_flag = 0;
     mbar_fence_init();
+    // The grid's weight images (and, in score mode, one layer's K/V images of this CTA's
+    // first unit) into L2 at once: otherwise every CTA misses on the same item at the same
+    // time when the launch follows kernels that have cycled L2.
+    prefetch_l2_share(p.wimg, (size_t)p.n_layer * Cfg<D>::kItems * Cfg<D>::kItemBytes);
+    if (!UM && (int)blockIdx.x < p.n_units) {
+      const Tile t0 = tile_of<D>(p, blockIdx.x, 0);
+      const uint32_t kvb = 2u * t0.Lp * D * 2u;
+      if (kvb) prefetch_l2(p.req[t0.r].kv + (size_t)(blockIdx.x % p.n_layer) * kvb, kvb);
+    }
   }
   if (warp == 3) {
     tmem_alloc(smem_u32(tmem_slot), 512);

@@ -80,6 +80,18 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                : "memory");
 }
 
+// Asks L2 to fetch [src, src + bytes) ahead of its first use (src 16-byte aligned, bytes a
+// multiple of 16); no completion to wait for.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+// This CTA's share of a buffer that the whole grid prefetches into L2 (bytes a multiple of 16).
+__device__ __forceinline__ void prefetch_l2_share(const void* buf, size_t bytes) {
+  const size_t share = ((bytes + gridDim.x - 1) / gridDim.x + 15) & ~(size_t)15;
+  const size_t off = (size_t)blockIdx.x * share;
+  if (off < bytes) prefetch_l2(static_cast<const uint8_t*>(buf) + off, (uint32_t)min(share, bytes - off));
+}
+
 // ------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

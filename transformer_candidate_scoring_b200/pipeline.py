@@ -434,7 +434,7 @@ def unit_bounds(req_offsets, tile: int = SCORE_TILE, unit: int = SCORE_UNIT) -> 
 
 
 def stream_plan(n: int, count: int, first: int, n_slots: int, comp_chunk: int, bounds: List[int],
-                score_units: int):
+                score_units: int, group: int = 1):
     """The launch order of Streamed.run over batches first .. first + count - 1 of n
     candidates each: a list of ("gather", j), ("compress", a, b) and ("score", a, b) with
     candidate positions a, b counted from the start of batch ``first`` (batch j covers
@@ -443,7 +443,10 @@ def stream_plan(n: int, count: int, first: int, n_slots: int, comp_chunk: int, b
     within a batch, unit_bounds), both across batch boundaries.  A launch is shorter only
     where it meets the end of the activation ring (n_slots batches, batch i in slot
     i mod n_slots), the end of the run, or a slot that the next batch is about to reuse
-    (everything of batch j - n_slots is compressed and scored before batch j is gathered)."""
+    (everything of batch j - n_slots is compressed and scored before batch j is gathered).
+    With ``group`` > 1, compress and score launches are issued only after every group-th
+    gather, so that launches of one kernel follow each other (a kernel that follows another
+    kind of kernel starts with cold instruction and data caches)."""
     if n <= 0 or count <= 0:
         return []
     ring = n_slots * n
@@ -484,6 +487,8 @@ def stream_plan(n: int, count: int, first: int, n_slots: int, comp_chunk: int, b
             comp = flush(comp, need, "compress", plan)
             score = flush(score, need, "score", plan)
         plan.append(("gather", j))
+        if (j + 1) % group and j + 1 < count:
+            continue
         comp = full(comp, (j + 1) * n, "compress", plan)
         score = full(score, comp, "score", plan)
     comp = flush(comp, count * n, "compress", plan)
@@ -514,7 +519,7 @@ class Streamed:
     """
 
     def __init__(self, dw: DeviceWorkload, n_slots: int = None, comp_chunk: int = None, score_units: int = None,
-                 ring_bytes: int = 8 << 30):
+                 ring_bytes: int = 8 << 30, group: int = 2):
         n = dw.n_cand
         dims = dw.w.dims
         F, D = dims.n_target_fields, dims.D
@@ -540,6 +545,7 @@ class Streamed:
         self.comp_chunk = comp_chunk if comp_chunk is not None else 2 * (sms - 1) * SCORE_TILE
         self.score_units = score_units if score_units is not None else sms
         self.bounds = unit_bounds(dw.req_offsets)
+        self.group = group
         _, hi = torch.cuda.Stream.priority_range()
         self.user = torch.cuda.Stream(dev, priority=hi)
         self.cap = torch.cuda.Stream(dev)
@@ -580,7 +586,7 @@ class Streamed:
         prefilled, done_ev, released = {}, {}, {}
         waited = set()
         score_end = 0
-        for step in stream_plan(n, count, first, m, self.comp_chunk, self.bounds, self.score_units):
+        for step in stream_plan(n, count, first, m, self.comp_chunk, self.bounds, self.score_units, self.group):
             if step[0] == "gather":
                 j = step[1]
                 i, dw = first + j, self.slots[(first + j) % m]
