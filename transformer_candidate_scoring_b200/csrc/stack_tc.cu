@@ -680,6 +680,53 @@ __device__ __forceinline__ float softmax_head(uint32_t base, int Lp, int L_u, fl
   return ex2(fmaf(sself, kL2E, -mx * kL2E));
 }
 
+// The two heads of a group (SW <= 64, two 64-column head regions from `base`): head 1's
+// scores are read chunk by chunk into the registers that head 0's numerators have just
+// left, so that their tensor-memory latency hides behind head 0's exponentials.
+template <int SW>
+__device__ __forceinline__ void softmax_two(uint32_t base, int Lp, int L_u, float ss0, float ss1, float* ps) {
+  const int nb = Lp / 16;
+  float sv[SW];
+#pragma unroll
+  for (int c = 0; c < SW / 16; ++c)
+    if (c < nb) tmem_ld16(base + 16 * c, sv + 16 * c);
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t hb = base + 64 * i;
+    const float sself = i == 0 ? ss0 : ss1;
+    tmem_wait_ld();
+    reg_fence<SW>(sv);
+    if (L_u < SW) {
+#pragma unroll
+      for (int k = 0; k < SW; ++k)
+        if (k >= L_u) sv[k] = -INFINITY;
+    }
+    float m4[4] = {sself, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int k = 0; k < SW; k += 8) {
+      m4[0] = max3(m4[0], sv[k], sv[k + 1]);
+      m4[1] = max3(m4[1], sv[k + 2], sv[k + 3]);
+      m4[2] = max3(m4[2], sv[k + 4], sv[k + 5]);
+      m4[3] = max3(m4[3], sv[k + 6], sv[k + 7]);
+    }
+    const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+    const uint64_t l2 = f32x2(kL2E, kL2E), n2 = f32x2(-mx * kL2E, -mx * kL2E);
+#pragma unroll
+    for (int c = 0; c < SW / 16; ++c)
+      if (c < nb) {
+        uint32_t r[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t x = fma2(f32x2(sv[16 * c + 2 * k], sv[16 * c + 2 * k + 1]), l2, n2);
+          r[k] = exp2_h2(lo32(x), hi32(x));
+        }
+        tmem_st8u(hb + 8 * c, r);
+        if (i == 0) tmem_ld16(base + 64 + 16 * c, sv + 16 * c);
+      }
+    ps[i] = ex2(fmaf(sself, kL2E, -mx * kL2E));
+  }
+}
+
 template <int D, int SW, bool UM>
 __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Epi& e) {
   constexpr int NH = Cfg<D>::kNH;
@@ -812,16 +859,26 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
       for (int g = 0; g < Groups<D, SW>::NG; ++g) {
         float ps[HG];
         if (!e.wait()) return;   // scores of group g
+        if constexpr (HG == 2) {
+          float s0 = sself[0], s1 = sself[1];
+#pragma unroll
+          for (int k = 2; k < NH; k += 2) {
+            s0 = 2 * g == k ? sself[k] : s0;
+            s1 = 2 * g == k ? sself[k + 1] : s1;
+          }
+          softmax_two<SW>(e.tW, t.Lp, t.L_u, s0, s1, ps);
+        } else {
 #pragma unroll 1
-        for (int i = 0; i < HG; ++i) {
-          const int h = g * HG + i;
-          float ss = sself[0];
+          for (int i = 0; i < HG; ++i) {
+            const int h = g * HG + i;
+            float ss = sself[0];
 #pragma unroll
-          for (int k = 1; k < NH; ++k) ss = h == k ? sself[k] : ss;
-          const float r = softmax_head<SW>(e.tW + i * HW, t.Lp, t.L_u, ss);
+            for (int k = 1; k < NH; ++k) ss = h == k ? sself[k] : ss;
+            const float r = softmax_head<SW>(e.tW + i * HW, t.Lp, t.L_u, ss);
 #pragma unroll
-          for (int k = 0; k < HG; ++k)
-            if (i == k) ps[k] = r;
+            for (int k = 0; k < HG; ++k)
+              if (i == k) ps[k] = r;
+          }
         }
         e.signal();
         if (!e.wait()) return;   // P V and the row sums of group g
