@@ -88,13 +88,18 @@ class _Stream:
 
     def __init__(self, log, *a, **k):
         self.log, self.n_ops = log, 0
+        self.deps = []                   # every (stream, count) this stream has waited for
         _Stream._n += 1
         self.id = _Stream._n
 
     def wait_event(self, ev):
         if ev.at is None:                # never recorded: no dependency (as in torch)
             return
-        self.log.waits.append((self, self.n_ops, ev.at[0], ev.at[1]))
+        # an event covers the recording stream's earlier operations and everything that
+        # stream had waited for before the record (as a CUDA event does)
+        for rs, count in [ev.at] + ev.deps:
+            self.log.waits.append((self, self.n_ops, rs, count))
+            self.deps.append((rs, count))
 
     def launch(self, reads, writes, label):
         self.log.ops.append((self, self.n_ops, tuple(reads), tuple(writes), label))
@@ -104,9 +109,11 @@ class _Stream:
 class _Event:
     def __init__(self, *a, **k):
         self.at = None
+        self.deps = []
 
     def record(self, stream):
         self.at = (stream, stream.n_ops)   # covers the stream's first n_ops operations
+        self.deps = list(stream.deps)
 
 
 class _Cuda:

@@ -506,11 +506,11 @@ class Streamed:
     on the SMs left beside one prefill CTA, every score launch one round of the score
     kernel's two-tile units on all SMs, whichever batches the chunk falls in.  A launch that spans two batches scores
     each candidate against its own request's cache (the kernels take a list of requests).
-      main stream  user aggregation, target aggregation of batch i, then every compress and
-                   score chunk that has become complete (a score chunk after the prefills of
-                   the batches it covers)
-      user stream  (high priority) the prefill of batch i, once batch i - n_slots (the same
-                   slot's previous batch) has been scored
+      main stream  target aggregation of batch i, then every compress and score chunk that
+                   has become complete (a score chunk after the prefills of the batches it
+                   covers)
+      user stream  (high priority) user aggregation and prefill of batch i, once batch
+                   i - n_slots (the same slot's previous batch) has been scored
     The slots are clones of one DeviceWorkload (DeviceWorkload.clone_slot) whose X, tokens
     and scores are views of ring buffers laid out slot after slot, so that a chunk spanning
     consecutive batches is one contiguous range; by default the ring takes up to 64 batches
@@ -592,16 +592,19 @@ class Streamed:
                 i, dw = first + j, self.slots[(first + j) % m]
                 if bind is not None:
                     bind(i, dw, main)
-                dw.user_aggregate(main)
                 fork = torch.cuda.Event()
                 fork.record(main)
                 self.user.wait_event(fork)
                 if j - m in done_ev:                # the slot's previous batch is scored
                     self.user.wait_event(done_ev.pop(j - m))
+                dw.user_aggregate(self.user)
+                user_read = torch.cuda.Event()      # the batch's user bags are read
+                user_read.record(self.user)
                 dw.user_prefill(self.user)
                 prefilled[j] = torch.cuda.Event()
                 prefilled[j].record(self.user)
                 dw.target_aggregate(main)
+                main.wait_event(user_read)
                 if fronted is not None:
                     fronted(i, dw, main)
             elif step[0] == "compress":
