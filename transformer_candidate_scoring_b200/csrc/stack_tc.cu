@@ -8,9 +8,10 @@
 //
 // Two 128-row tiles ("slots") are in flight per CTA, so that one slot's LayerNorm, softmax
 // and hand-offs run while the tensor core works on the other slot's products.  Each slot
-// owns 256 TMEM columns, four epilogue warps (one thread per tile row, the whole row) and an
-// MMA-issuing thread; the two slots of a CTA take two consecutive tiles of one request (a
-// "unit") and share its K/V images and every weight item of the stream.
+// owns 256 TMEM columns, 4 P epilogue warps (P threads per tile row: two at D = 128, each
+// with half of the row's columns and every other head, one at D = 64) and an MMA-issuing
+// thread; the two slots of a CTA take two consecutive tiles of one request (a "unit") and
+// share its K/V images and every weight item of the stream.
 //
 //   TMEM (per slot, 256 fp32 columns, lane = tile row)
 //     [0, D)        Y, the residual stream; the O and FFN2 products (and their biases)
@@ -37,8 +38,8 @@
 // is not built for this kernel (it runs on the CUDA-core path).
 //
 // Warp roles: warp 0 streams weight items, warp 3 streams K/V images (and owns the TMEM
-// allocation), warps 1 and 2 issue the MMAs of slot 0 and slot 1, warps 4-7 and 8-11 are the
-// epilogues of slot 0 and slot 1.  Every epilogue/MMA hand-off of a slot is a strict
+// allocation), warps 1 and 2 issue the MMAs of slot 0 and slot 1, the next 4 P warps are the
+// epilogue of slot 0 and the last 4 P that of slot 1.  Every epilogue/MMA hand-off of a slot is a strict
 // alternation on two mbarriers.  Every wait is bounded: a stalled barrier sets an error bit
 // and the kernel unwinds, releasing its tensor memory.
 #include <cuda_fp16.h>
@@ -63,10 +64,21 @@ using namespace tc;
 constexpr int kM = 128;
 constexpr int kSlotCols = 256;
 constexpr int kWork = 128;
-constexpr int kSlotThreads = 128;                    // epilogue threads per slot
-constexpr int kThreads = 128 + 2 * kSlotThreads;     // control warpgroup + two epilogue warpgroups
-constexpr int kCtlRegs = 56, kEpiRegs = 224;
-static_assert(4 * 32 * kCtlRegs + 8 * 32 * kEpiRegs <= kThreads * 168, "register split exceeds the launch");
+// Epilogue threads per tile row (P): two at D = 128, where a row's epilogue work is large
+// enough to split, one at D = 64.  The launch has a control warpgroup and 4 P epilogue
+// warps per slot; `setmaxnreg` moves registers from the control warps to the epilogues.
+template <int D>
+struct Par {
+  static constexpr int P = D == 128 ? 2 : 1;
+  static constexpr int kSlotThreads = 128 * P;
+  static constexpr int kThreads = 128 + 2 * kSlotThreads;
+  static constexpr int kLaunchRegs = P == 2 ? 96 : 168;   // 65,536 / kThreads, rounded down to 8
+  static constexpr int kCtlRegs = P == 2 ? 40 : 56, kEpiRegs = P == 2 ? 104 : 224;
+  static_assert(4 * 32 * kCtlRegs + 2 * kSlotThreads * kEpiRegs <= kThreads * kLaunchRegs,
+                "register split exceeds the launch");
+  static_assert(kThreads * kLaunchRegs <= 65536, "launch registers");
+};
+constexpr int kMaxParts = 2;
 constexpr int kMaxStages = 4;
 constexpr int kMaxLp = 128;
 constexpr float kL2E = 1.44269504088896341f;
@@ -149,7 +161,7 @@ struct StackParams {
   const float* domain_emb;    // fp32 [n_domains][D]
   int* status;
   int n_layer, n_units, R, pair;
-  int off_kv, off_ring, off_ones, off_vec, off_bar, stages;
+  int off_kv, off_ring, off_ones, off_xch, off_vec, off_bar, stages;
   // where slot 0 lets slot 1 start a unit of two tiles (layer 0): 0 after its own-V phase,
   // 1 after the attention of its second head group.  Slot 0 alone may run at most `stages`
   // weight items ahead, so with a two-item ring the gate must open before it needs Q.
@@ -196,8 +208,11 @@ struct Bars {
   __device__ __forceinline__ uint32_t drain(int slot) const { return at(2 * kMaxStages + 9 + slot); }
   // epilogue turn of slot s (passed between the two slots of a unit)
   __device__ __forceinline__ uint32_t tok(int slot) const { return at(2 * kMaxStages + 11 + slot); }
+  // the exchange between the two parts of the rows of lane quadrant q of slot s
+  __device__ __forceinline__ uint32_t xch(int slot, int q) const { return at(2 * kMaxStages + 13 + 4 * slot + q); }
 };
-constexpr int kNumBars = 2 * kMaxStages + 13;
+constexpr int kNumBars = 2 * kMaxStages + 21;
+constexpr int kXchBytes = 2 * kMaxParts * kM * 8;   // per slot: two alternating float2 buffers
 constexpr int kBarArea = 8 * kNumBars + 32;   // + TMEM address and abort flag
 
 // ------------------------------------------------------------------ small helpers
@@ -362,8 +377,8 @@ __device__ void mma_issuer(const StackParams& p, int slot, uint32_t tmem, uint32
     for (int kk = 0; kk < pc.K / 16; ++kk) {
       const uint64_t bd = sdesc(item + pc.off + kk * pc.N * 32, pc.N * 16, 128);
       const uint32_t accf = (kk > 0 || acc) ? 1u : 0u;
-      if (a_tmem)
-        mma_bf16_ta(dcol, a + kk * 8, bd, id, accf);
+      if (a_tmem)   // the epilogue parts' fp16 hidden units: [0, 64), or [0, 32) and [64, 96)
+        mma_bf16_ta(dcol, a + (Par<D>::P == 2 ? (kk & 3) * 8 + (kk >> 2) * 64 : kk * 8), bd, id, accf);
       else
         mma_bf16(dcol, sdesc(a + kk * 4096, 2048, 128), bd, id, accf);
     }
@@ -472,13 +487,18 @@ __device__ void mma_issuer(const StackParams& p, int slot, uint32_t tmem, uint32
   }
 }
 
-// ------------------------------------------------------------------ epilogue (one thread per row)
+// ------------------------------------------------------------------ epilogue (two threads per row)
+// The epilogue threads of a slot are P warps per TMEM lane quadrant: the thread of part p
+// owns row m's columns [p D/P, (p + 1) D/P) in every row-wise phase (Y, LayerNorm, ReLU) and
+// the heads h with h mod P = p in the attention; with two parts a row's LayerNorm statistics
+// and its score are merged across them through shared memory.
 struct Epi {
   uint32_t tY, tW;            // TMEM address of this row: residual, work area
   uint32_t sA, rowoff, sKV;
-  int m;
+  int m, part;
   uint32_t e2m, m2e, ph;
   uint32_t gate, gph;         // the start gate of slot 1 in a unit of two tiles
+  uint32_t xbar, xph, xbuf, xsel;   // the exchange with the row's other part
   int slot;
   bool paired;                 // both slots of the unit hold a tile
   const float* vec;
@@ -508,8 +528,7 @@ struct Epi {
     return ok;
   }
   // Each thread completes its tensor-memory stores and orders its shared-memory stores
-  // before the tensor core's reads; then one lane per warp arrives for the whole warp (128
-  // arrivals on one barrier queue behind each other, four do not).
+  // before the tensor core's reads; then one lane per warp arrives for the whole warp.
   __device__ __forceinline__ void signal() {
     tmem_wait_st();
     fence_proxy_async_smem();
@@ -517,15 +536,23 @@ struct Epi {
     __syncwarp();
     if ((m & 31) == 0) mbar_arrive(e2m);
   }
+  // Two floats to the row's other part and its two back (the two buffers alternate, so a
+  // buffer is rewritten only after the partner has passed the exchange that read it).
+  __device__ __forceinline__ float2 xchg(float2 mine) {
+    const uint32_t x = xbuf + xsel * (kMaxParts * kM * 8);
+    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(x + (part * kM + m) * 8), "f"(mine.x), "f"(mine.y)
+                 : "memory");
+    __syncwarp();
+    if ((m & 31) == 0) mbar_arrive(xbar);
+    ok = __all_sync(0xffffffffu, ok && mbar_wait(xbar, xph, abort_flag));
+    xph ^= 1;
+    float2 o;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(o.x), "=f"(o.y) : "r"(x + ((1 - part) * kM + m) * 8)
+                 : "memory");
+    xsel ^= 1;
+    return o;
+  }
 };
-
-template <int D>
-__device__ __forceinline__ void load_row(uint32_t taddr, float* y) {
-#pragma unroll
-  for (int c = 0; c < D / 32; ++c) tmem_ld32(taddr + 32 * c, y + 32 * c);
-  tmem_wait_ld();
-  reg_fence<D>(y);
-}
 
 // Packed fp32 pairs (one instruction for two lanes' worth of values).
 __device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
@@ -545,60 +572,85 @@ __device__ __forceinline__ void fma_h2(float& s_lo, float& s_hi, uint32_t a, uin
       : "r"(a), "r"(b));
 }
 
-// Row mean and 1/sqrt(var + eps) (two passes over the registers, on packed pairs).
+// This part's N columns of the row from tensor memory.
+template <int N>
+__device__ __forceinline__ void load_part(uint32_t taddr, float* y) {
+#pragma unroll
+  for (int c = 0; c < N / 16; ++c) tmem_ld16(taddr + 16 * c, y + 16 * c);
+  tmem_wait_ld();
+  reg_fence<N>(y);
+}
+
+// Row mean and 1/sqrt(var + eps) over D columns, of which this part holds y[0 .. D/P): each
+// part's mean and sum of squared deviations (on packed pairs), merged with the other part's
+// (Chan's update) when there are two.
 template <int D>
-__device__ __forceinline__ float2 row_stats(const float* y) {
+__device__ __forceinline__ float2 row_stats(Epi& e, const float* y) {
+  constexpr int P = Par<D>::P, N = D / P;
   uint64_t a[2] = {0ull, 0ull};
 #pragma unroll
-  for (int i = 0; i < D / 2; ++i) a[i & 1] = add_f32x2(a[i & 1], f32x2(y[2 * i], y[2 * i + 1]));
-  const float mean = ((lo32(a[0]) + lo32(a[1])) + (hi32(a[0]) + hi32(a[1]))) * (1.f / D);
+  for (int i = 0; i < N / 2; ++i) a[i & 1] = add_f32x2(a[i & 1], f32x2(y[2 * i], y[2 * i + 1]));
+  const float mean = ((lo32(a[0]) + lo32(a[1])) + (hi32(a[0]) + hi32(a[1]))) * (1.f / N);
   const uint64_t nm = f32x2(-mean, -mean);
   a[0] = a[1] = 0ull;
 #pragma unroll
-  for (int i = 0; i < D / 2; ++i) {
+  for (int i = 0; i < N / 2; ++i) {
     const uint64_t d = add_f32x2(f32x2(y[2 * i], y[2 * i + 1]), nm);
     a[i & 1] = fma2(d, d, a[i & 1]);
   }
-  const float ss = (lo32(a[0]) + lo32(a[1])) + (hi32(a[0]) + hi32(a[1]));
-  return make_float2(mean, rsqrtf(ss * (1.f / D) + kLnEps));
+  const float m2 = (lo32(a[0]) + lo32(a[1])) + (hi32(a[0]) + hi32(a[1]));
+  if constexpr (P == 1) {
+    return make_float2(mean, rsqrtf(m2 * (1.f / D) + kLnEps));
+  } else {
+    const float2 o = e.xchg(make_float2(mean, m2));
+    // the parts in a fixed order, so that both compute the same bits
+    const float ma = e.part == 0 ? mean : o.x, mb = e.part == 0 ? o.x : mean;
+    const float qa = e.part == 0 ? m2 : o.y, qb = e.part == 0 ? o.y : m2;
+    const float dm = ma - mb;
+    const float mu = 0.5f * (ma + mb);
+    const float var = ((qa + qb) + dm * dm * (0.25f * D)) * (1.f / D);
+    return make_float2(mu, rsqrtf(var + kLnEps));
+  }
 }
 
 // The row standardized (LayerNorm without its gain and shift, which the next product's
-// weights carry) -> fp16 A operand row.
+// weights carry) -> this part's columns of the fp16 A operand row.
 template <int D>
-__device__ __forceinline__ void ln_to_A(const Epi& e, const float* y) {
-  const float2 st = row_stats<D>(y);
+__device__ __forceinline__ void ln_to_A(Epi& e, const float* y) {
+  constexpr int P = Par<D>::P;
+  const float2 st = row_stats<D>(e, y);
   const uint64_t r2 = f32x2(st.y, st.y), n2 = f32x2(-st.x * st.y, -st.x * st.y);
 #pragma unroll
-  for (int kc = 0; kc < D / 8; ++kc) {
+  for (int kc = 0; kc < D / (8 * P); ++kc) {
     uint32_t h[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint64_t v = fma2(f32x2(y[8 * kc + 2 * i], y[8 * kc + 2 * i + 1]), r2, n2);
       h[i] = pack_h2(lo32(v), hi32(v));
     }
-    st_shared_v4(e.sA + kc * 2048 + e.rowoff, h[0], h[1], h[2], h[3]);
+    st_shared_v4(e.sA + (e.part * (D / (8 * P)) + kc) * 2048 + e.rowoff, h[0], h[1], h[2], h[3]);
   }
 }
 
-// 128 columns of the work area -> fp16 -> ReLU (max with 0 on the pairs; rounding keeps
-// the sign, so this equals rounding after the ReLU) -> its first 64 columns (in place: every
-// value is read before the first store).
-__device__ __forceinline__ void relu_in_place(uint32_t tW) {
-  float h[128];
+// This part's N hidden units of the work area -> fp16 -> ReLU (max with 0 on the pairs;
+// rounding keeps the sign, so this equals rounding after the ReLU) -> the first N/2 columns
+// of the same N (in place: every value is read before the first store).
+template <int N>
+__device__ __forceinline__ void relu_in_place(uint32_t tw) {
+  float h[N];
 #pragma unroll
-  for (int c = 0; c < 4; ++c) tmem_ld32(tW + 32 * c, h + 32 * c);
+  for (int c = 0; c < N / 32; ++c) tmem_ld32(tw + 32 * c, h + 32 * c);
   tmem_wait_ld();
-  reg_fence<128>(h);
+  reg_fence<N>(h);
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < N / 32; ++c) {
     uint32_t r[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       const uint32_t v = pack_h2(h[32 * c + 2 * i], h[32 * c + 2 * i + 1]);
       asm("max.f16x2 %0, %1, %2;" : "=r"(r[i]) : "r"(v), "r"(0u));
     }
-    tmem_st16u(tW + 16 * c, r);
+    tmem_st16u(tw + 16 * c, r);
   }
 }
 
@@ -607,11 +659,11 @@ __device__ __forceinline__ void relu_in_place(uint32_t tW) {
 // numerators go back as fp16 pairs over the first Lp / 2 columns; returns the own key's
 // numerator.  The row sum of the numerators comes from the tensor core (a product with a
 // tile of ones, beside P V), so it adds exactly the fp16 values that P V weighs.
-template <int SW>
+template <int SW, bool LEAN>
 __device__ __forceinline__ float softmax_head(uint32_t base, int Lp, int L_u, float sself) {
   const int nb = Lp / 16;
   float mx;
-  if constexpr (SW <= 64) {
+  if constexpr (SW <= 64 && !LEAN) {
     float sv[SW];
 #pragma unroll
     for (int c = 0; c < SW / 16; ++c)
@@ -680,9 +732,10 @@ __device__ __forceinline__ float softmax_head(uint32_t base, int Lp, int L_u, fl
   return ex2(fmaf(sself, kL2E, -mx * kL2E));
 }
 
-// The two heads of a group (SW <= 64, two 64-column head regions from `base`): head 1's
-// scores are read chunk by chunk into the registers that head 0's numerators have just
-// left, so that their tensor-memory latency hides behind head 0's exponentials.
+// The two heads of a group (SW <= 64, two 64-column head regions from `base`), both in one
+// thread: head 1's scores are read chunk by chunk into the registers that head 0's
+// numerators have just left, so that their tensor-memory latency hides behind head 0's
+// exponentials.
 template <int SW>
 __device__ __forceinline__ void softmax_two(uint32_t base, int Lp, int L_u, float ss0, float ss1, float* ps) {
   const int nb = Lp / 16;
@@ -727,20 +780,57 @@ __device__ __forceinline__ void softmax_two(uint32_t base, int Lp, int L_u, floa
   }
 }
 
+// Attention output of head h (own index k) from its P V product and row sum at `hb`:
+// o = (ps v_own + P V) / (sum + ps) -> the head's 16 columns of A.
+template <int D, bool UM>
+__device__ __forceinline__ void finish_head(const Epi& e, uint32_t hb, int hw, int h, int k, float ps,
+                                            const uint32_t* vreg) {
+  constexpr int NP = Cfg<D>::kNH / Par<D>::P;
+  float o[16];
+  tmem_ld16(hb + hw / 2, o);
+  float sum = tmem_ld1(hb + hw / 2 + 16);
+  tmem_wait_ld();
+  reg_fence<16>(o);
+  asm volatile("" : "+f"(sum));
+  const float li = rcp_approx(sum + ps);
+  if constexpr (UM) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) o[j] *= li;
+  } else {
+    uint32_t vv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      vv[j] = vreg[j];
+#pragma unroll
+      for (int kk = 1; kk < NP; ++kk) vv[j] = k == kk ? vreg[8 * kk + j] : vv[j];
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      o[2 * j] = fmaf(ps, h_lo(vv[j]), o[2 * j]) * li;
+      o[2 * j + 1] = fmaf(ps, h_hi(vv[j]), o[2 * j + 1]) * li;
+    }
+  }
+  st_row8h(e.sA + (2 * h) * 2048 + e.rowoff, o);
+  st_row8h(e.sA + (2 * h + 1) * 2048 + e.rowoff, o + 8);
+}
+
 template <int D, int SW, bool UM>
 __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Epi& e) {
+  constexpr int P = Par<D>::P;
   constexpr int NH = Cfg<D>::kNH;
-  const int m = e.m;
+  constexpr int NP = NH / P;                   // heads of this part: P k + part
+  constexpr int DP = D / P;                    // columns of this part
+  const int m = e.m, part = e.part;
   const bool live = m < t.rows;
   if (!e.acquire()) return;
-  // ---- Y = token + s_d (rows past the tile's end are zero and never stored)
+  // ---- Y = token + s_d, this part's columns (rows past the tile's end are zero, never stored)
   {
-    float y[D];
-    const float4* sd4 = reinterpret_cast<const float4*>(p.domain_emb + (size_t)t.dom * D);
+    float y[DP];
+    const float4* sd4 = reinterpret_cast<const float4*>(p.domain_emb + (size_t)t.dom * D + part * DP);
     const float4* src = reinterpret_cast<const float4*>(
-        UM ? p.req[t.r].utokens + (size_t)m * D : p.tokens + (size_t)(t.row0 + m) * D);
+        (UM ? p.req[t.r].utokens + (size_t)m * D : p.tokens + (size_t)(t.row0 + m) * D) + part * DP);
 #pragma unroll
-    for (int c = 0; c < D / 4; ++c) {
+    for (int c = 0; c < DP / 4; ++c) {
       const float4 u = live ? __ldg(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
       const float4 d = __ldg(sd4 + c);
       y[4 * c] = live ? u.x + d.x : 0.f;
@@ -749,7 +839,7 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
       y[4 * c + 3] = live ? u.w + d.w : 0.f;
     }
 #pragma unroll
-    for (int c = 0; c < D / 16; ++c) tmem_st16(e.tY + 16 * c, y + 16 * c);
+    for (int c = 0; c < DP / 16; ++c) tmem_st16(e.tY + part * DP + 16 * c, y + 16 * c);
     tmem_wait_st();
   }
   // (Y is re-read from tensor memory at the top of every layer, so that no register copy of
@@ -757,160 +847,134 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
   for (int l = 0; l < p.n_layer; ++l) {
     if (l > 0 && !e.wait()) return;   // the previous layer's FFN product is in Y
     {
-      float y[D];
-      load_row<D>(e.tY, y);
+      float y[DP];
+      load_part<DP>(e.tY + part * DP, y);
       ln_to_A<D>(e, y);
     }
     e.signal();
-    // ---- own K and V (user mode: this row of the layer's K and V^T images), read 32
-    // columns at a time (the packed K stays live while V is read)
-    uint32_t kreg[UM ? 1 : D / 2], vreg[UM ? 1 : D / 2];
+    // ---- own K and V of this part's heads (user mode: their columns of this row of the
+    // layer's K and V^T images), two heads at a time
+    uint32_t kreg[UM ? 1 : 8 * NP], vreg[UM ? 1 : 8 * NP];
 #pragma unroll
     for (int pass = 0; pass < 2; ++pass) {
       if (!e.wait()) return;
 #pragma unroll
-      for (int hb = 0; hb < D / 32; ++hb) {
+      for (int k2 = 0; k2 < NP; k2 += 2) {
         float x[32];
-        tmem_ld32(e.tW + 32 * hb, x);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) tmem_ld16(e.tW + 16 * (P * (k2 + j) + part), x + 16 * j);
         tmem_wait_ld();
         reg_fence<32>(x);
-        if constexpr (UM) {
-          if (m < t.Lp) {
-            const bool real = m < t.L_u;
-            if (pass == 0) {   // K image [Lp x D]: row m, eight columns per core-matrix row
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int cc = 4 * hb + j;
-                float v[8];
+        for (int j = 0; j < 2; ++j) {
+          const int k = k2 + j, h = P * k + part;
+          if constexpr (UM) {
+            if (m < t.Lp) {
+              const bool real = m < t.L_u;
+              if (pass == 0) {   // K image [Lp x D]: row m, eight columns per core-matrix row
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = real ? x[8 * j + i] : 0.f;
-                st_row8h(e.sKV + (cc * (t.Lp / 8) + (m >> 3)) * 128 + (m & 7) * 16, v);
-              }
-            } else {           // V^T image [D x Lp]: column m
-              const uint32_t vb = e.sKV + t.Lp * D * 2 + (m >> 3) * (D / 8) * 128 + (m & 7) * 2;
+                for (int c = 0; c < 2; ++c) {
+                  float v[8];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int d = 32 * hb + i;
-                const __half hv = __float2half_rn(real ? x[i] : 0.f);
-                asm volatile("st.shared.b16 [%0], %1;" ::"r"(vb + (d >> 3) * 128 + (d & 7) * 16),
-                             "h"(*reinterpret_cast<const unsigned short*>(&hv))
-                             : "memory");
+                  for (int i = 0; i < 8; ++i) v[i] = real ? x[16 * j + 8 * c + i] : 0.f;
+                  st_row8h(e.sKV + ((2 * h + c) * (t.Lp / 8) + (m >> 3)) * 128 + (m & 7) * 16, v);
+                }
+              } else {           // V^T image [D x Lp]: column m
+                const uint32_t vb = e.sKV + t.Lp * D * 2 + (m >> 3) * (D / 8) * 128 + (m & 7) * 2;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const int d = 16 * h + i;
+                  const __half hv = __float2half_rn(real ? x[16 * j + i] : 0.f);
+                  asm volatile("st.shared.b16 [%0], %1;" ::"r"(vb + (d >> 3) * 128 + (d & 7) * 16),
+                               "h"(*reinterpret_cast<const unsigned short*>(&hv))
+                               : "memory");
+                }
               }
             }
-          }
-        } else {
+          } else {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            if (pass == 0)
-              kreg[16 * hb + i] = pack_h2(x[2 * i], x[2 * i + 1]);
-            else
-              vreg[16 * hb + i] = pack_h2(x[2 * i], x[2 * i + 1]);
+            for (int i = 0; i < 8; ++i) {
+              if (pass == 0)
+                kreg[8 * k + i] = pack_h2(x[16 * j + 2 * i], x[16 * j + 2 * i + 1]);
+              else
+                vreg[8 * k + i] = pack_h2(x[16 * j + 2 * i], x[16 * j + 2 * i + 1]);
+            }
           }
         }
       }
       e.signal();
       if (l == 0 && pass == 1 && p.gate_phase == 0) e.open_gate();
     }
-    // ---- Q (pre-scaled by 1/sqrt(d_h) through its weights) -> A; own score per head
-    float sself[NH];
+    // ---- Q of this part's heads (pre-scaled by 1/sqrt(d_h) through its weights) -> A; own
+    // score per head
+    float sself[NP];
     if (!e.wait()) return;
 #pragma unroll
-    for (int hc = 0; hc < D / 32; ++hc) {
-      float q[32];
-      tmem_ld32(e.tW + 32 * hc, q);
+    for (int k = 0; k < NP; ++k) {
+      const int h = P * k + part;
+      float q[16];
+      tmem_ld16(e.tW + 16 * h, q);
       tmem_wait_ld();
-      reg_fence<32>(q);
+      reg_fence<16>(q);
+      uint32_t qp[8];   // the head's query as the fp16 pairs the score product reads
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int h = 2 * hc + j;
-        uint32_t qp[8];   // the head's query as the fp16 pairs the score product reads
+      for (int i = 0; i < 8; ++i) qp[i] = pack_h2(q[2 * i], q[2 * i + 1]);
+      if constexpr (UM) {
+        sself[k] = -INFINITY;
+      } else {
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) qp[i] = pack_h2(q[16 * j + 2 * i], q[16 * j + 2 * i + 1]);
-        if constexpr (UM) {
-          sself[h] = -INFINITY;
-        } else {
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) fma_h2(s0, s1, qp[i], kreg[8 * h + i]);
-          sself[h] = s0 + s1;
-        }
-        if (UM || t.Lp > 0) {
-          st_shared_v4(e.sA + (2 * h) * 2048 + e.rowoff, qp[0], qp[1], qp[2], qp[3]);
-          st_shared_v4(e.sA + (2 * h + 1) * 2048 + e.rowoff, qp[4], qp[5], qp[6], qp[7]);
-        } else {             // no user keys: the attention output is the own value
-          float o[16];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            o[2 * i] = h_lo(vreg[8 * h + i]);
-            o[2 * i + 1] = h_hi(vreg[8 * h + i]);
-          }
-          st_row8h(e.sA + (2 * h) * 2048 + e.rowoff, o);
-          st_row8h(e.sA + (2 * h + 1) * 2048 + e.rowoff, o + 8);
+        for (int i = 0; i < 8; ++i) fma_h2(s0, s1, qp[i], kreg[8 * k + i]);
+        sself[k] = s0 + s1;
+      }
+      if (UM || t.Lp > 0) {
+        st_shared_v4(e.sA + (2 * h) * 2048 + e.rowoff, qp[0], qp[1], qp[2], qp[3]);
+        st_shared_v4(e.sA + (2 * h + 1) * 2048 + e.rowoff, qp[4], qp[5], qp[6], qp[7]);
+      } else {             // no user keys: the attention output is the own value
+        if constexpr (!UM) {
+          st_shared_v4(e.sA + (2 * h) * 2048 + e.rowoff, vreg[8 * k], vreg[8 * k + 1], vreg[8 * k + 2],
+                       vreg[8 * k + 3]);
+          st_shared_v4(e.sA + (2 * h + 1) * 2048 + e.rowoff, vreg[8 * k + 4], vreg[8 * k + 5], vreg[8 * k + 6],
+                       vreg[8 * k + 7]);
         }
       }
     }
     e.signal();
     if (l == 0 && t.Lp == 0 && p.gate_phase == 1) e.open_gate();
-    // ---- attention, one head group at a time (loops kept rolled: the heads of a group are
-    // picked out of the per-head registers by comparison, which keeps the code small)
+    // ---- attention, one head group at a time.  Two heads per group: with two parts each
+    // takes one (head 2g + part), with one part the thread takes both; one head per group:
+    // the head's own part does it and the other waits.
     constexpr int HG = Groups<D, SW>::HG, HW = Groups<D, SW>::HW;
     if (t.Lp > 0) {
 #pragma unroll 1
       for (int g = 0; g < Groups<D, SW>::NG; ++g) {
-        float ps[HG];
         if (!e.wait()) return;   // scores of group g
-        if constexpr (HG == 2) {
+        if constexpr (HG == 2 && P == 1) {
+          float ps[2];
           float s0 = sself[0], s1 = sself[1];
 #pragma unroll
-          for (int k = 2; k < NH; k += 2) {
+          for (int k = 2; k < NP; k += 2) {
             s0 = 2 * g == k ? sself[k] : s0;
             s1 = 2 * g == k ? sself[k + 1] : s1;
           }
           softmax_two<SW>(e.tW, t.Lp, t.L_u, s0, s1, ps);
+          e.signal();
+          if (!e.wait()) return;   // P V and the row sums of group g
+#pragma unroll
+          for (int i = 0; i < 2; ++i) finish_head<D, UM>(e, e.tW + i * HW, HW, 2 * g + i, 2 * g + i, ps[i], vreg);
         } else {
-#pragma unroll 1
-          for (int i = 0; i < HG; ++i) {
-            const int h = g * HG + i;
-            float ss = sself[0];
+          const int h = HG == 2 ? 2 * g + part : g;
+          const bool mine = h % P == part;
+          const int k = h / P;                       // own index of head h
+          const uint32_t hb = e.tW + (HG == 2 ? part : 0) * HW;
+          float ss = sself[0];
 #pragma unroll
-            for (int k = 1; k < NH; ++k) ss = h == k ? sself[k] : ss;
-            const float r = softmax_head<SW>(e.tW + i * HW, t.Lp, t.L_u, ss);
-#pragma unroll
-            for (int k = 0; k < HG; ++k)
-              if (i == k) ps[k] = r;
-          }
-        }
-        e.signal();
-        if (!e.wait()) return;   // P V and the row sums of group g
-#pragma unroll
-        for (int i = 0; i < HG; ++i) {
-          const int h = g * HG + i;
-          float o[16];
-          tmem_ld16(e.tW + i * HW + HW / 2, o);
-          float sum = tmem_ld1(e.tW + i * HW + HW / 2 + 16);
-          tmem_wait_ld();
-          reg_fence<16>(o);
-          asm volatile("" : "+f"(sum));
-          const float li = rcp_approx(sum + ps[i]);
-          if constexpr (UM) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) o[j] *= li;
-          } else {
-            uint32_t vv[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              vv[j] = vreg[j];
-#pragma unroll
-              for (int k = 1; k < NH; ++k) vv[j] = h == k ? vreg[8 * k + j] : vv[j];
-            }
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              o[2 * j] = fmaf(ps[i], h_lo(vv[j]), o[2 * j]) * li;
-              o[2 * j + 1] = fmaf(ps[i], h_hi(vv[j]), o[2 * j + 1]) * li;
-            }
-          }
-          st_row8h(e.sA + (2 * h) * 2048 + e.rowoff, o);
-          st_row8h(e.sA + (2 * h + 1) * 2048 + e.rowoff, o + 8);
+          for (int j = 1; j < NP; ++j) ss = k == j ? sself[j] : ss;
+          float ps = 0.f;
+          if (mine) ps = softmax_head<SW, P == 2>(hb, t.Lp, t.L_u, ss);
+          e.signal();
+          if (!e.wait()) return;   // P V and the row sums of group g
+          if (mine) finish_head<D, UM>(e, hb, HW, h, k, ps, vreg);
         }
         e.signal();
         if (l == 0 && g == (Groups<D, SW>::NG > 1 ? 1 : 0) && p.gate_phase == 1) e.open_gate();
@@ -919,8 +983,8 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
     // ---- LN2 -> A
     if (!e.wait()) return;        // Y += attn Wo + bo
     {
-      float y[D];
-      load_row<D>(e.tY, y);
+      float y[DP];
+      load_part<DP>(e.tY + part * DP, y);
       ln_to_A<D>(e, y);
     }
     e.signal();
@@ -928,35 +992,44 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
 #pragma unroll
     for (int half = 0; half < Cfg<D>::kFfnHalves; ++half) {
       if (!e.wait()) return;
-      relu_in_place(e.tW);
+      relu_in_place<128 / P>(e.tW + (128 / P) * part);
       e.signal();
     }
   }
-  // ---- head: w . LN_f(y) + b (w folded with the final LayerNorm's gain)
+  // ---- head: w . LN_f(y) + b (w folded with the final LayerNorm's gain); with two parts
+  // their halves of the dot product are added in a fixed order
   if (!e.wait()) return;
   if (UM) return;
-  float y[D];
-  load_row<D>(e.tY, y);
-  const float2 st = row_stats<D>(y);
-  const float* vf = e.vec;
+  float y[DP];
+  load_part<DP>(e.tY + part * DP, y);
+  const float2 st = row_stats<D>(e, y);
+  const float* vf = e.vec + part * DP;
   float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int c = 0; c < D / 8; ++c) {
+  for (int c = 0; c < DP / 8; ++c) {
     float w[8];
     ld8(vf + 8 * c, w);
 #pragma unroll
     for (int i = 0; i < 8; ++i) a4[i & 3] = fmaf((y[8 * c + i] - st.x) * st.y, w[i], a4[i & 3]);
   }
-  if (live) p.scores[t.row0 + m] = ((a4[0] + a4[1]) + (a4[2] + a4[3])) + vf[D];
+  const float mine = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+  float dot = mine;
+  if constexpr (P == 2) {
+    const float other = e.xchg(make_float2(mine, 0.f)).x;
+    dot = part == 0 ? mine + other : other + mine;
+  }
+  if (live && part == 0) p.scores[t.row0 + m] = dot + e.vec[D];
 }
 
 template <int D, int SW, bool UM>
 __device__ void epilogue(const StackParams& p, int slot, uint32_t tmem, uint32_t sA, uint32_t sKV, uint32_t sOnes,
-                         const float* vec, const Bars& b, volatile int* abort_flag) {
+                         const float* vec, const Bars& b, uint32_t xbuf, volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Epi e;
-  e.m = (warp & 3) * 32 + lane;
-  e.tY = tmem + ((uint32_t)((warp & 3) * 32) << 16) + kSlotCols * slot;
+  const int q = warp & 3;
+  e.m = q * 32 + lane;
+  e.part = ((warp - 4) >> 2) % Par<D>::P;
+  e.tY = tmem + ((uint32_t)(q * 32) << 16) + kSlotCols * slot;
   e.tW = e.tY + D;
   e.sA = sA;
   e.rowoff = (e.m >> 3) * 128 + (e.m & 7) * 16;
@@ -966,6 +1039,10 @@ __device__ void epilogue(const StackParams& p, int slot, uint32_t tmem, uint32_t
   e.ph = 0;
   e.gate = b.tok(0);
   e.gph = 0;
+  e.xbar = b.xch(slot, q);
+  e.xph = 0;
+  e.xbuf = xbuf;
+  e.xsel = 0;
   e.slot = slot;
   e.vec = vec;
   e.abort_flag = abort_flag;
@@ -978,7 +1055,8 @@ __device__ void epilogue(const StackParams& p, int slot, uint32_t tmem, uint32_t
 }
 
 template <int D, int SW, bool UM>
-__global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
+__global__ void __launch_bounds__(Par<D>::kThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
+  constexpr int kSlotThreads = Par<D>::kSlotThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t base = smem_u32(smem);
@@ -1002,6 +1080,7 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       mbar_init(b.drain(s), 1);
       mbar_init(b.tok(s), kSlotThreads / 32);
     }
+    for (int i = 0; i < 8; ++i) mbar_init(b.xch(i >> 2, i & 3), Par<D>::P);
     *abort_flag = 0;
     mbar_fence_init();
     // The grid's weight images (and, in score mode, one layer's K/V images of this CTA's
@@ -1041,7 +1120,7 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtlRegs));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Par<D>::kCtlRegs));
     if (lane == 0) {
       if (warp == 0) weight_producer<D>(p, ring, b, abort_flag);
       if (warp == 1) mma_issuer<D, SW, UM>(p, 0, tmem, sA0, sKV, ring, sOnes, b, abort_flag);
@@ -1049,10 +1128,11 @@ __global__ void __launch_bounds__(kThreads, 1) stack_kernel(const __grid_constan
       if (warp == 3 && !UM) kv_producer<D>(p, sKV, b, abort_flag);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kEpiRegs));
-    const int slot = (warp - 4) >> 2;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Par<D>::kEpiRegs));
+    const int slot = (warp - 4) / (4 * Par<D>::P);
     if (slot == 0 || p.pair)
-      epilogue<D, SW, UM>(p, slot, tmem, sA0 + slot * kM * D * 2, sKV, sOnes, vec, b, abort_flag);
+      epilogue<D, SW, UM>(p, slot, tmem, sA0 + slot * kM * D * 2, sKV, sOnes, vec, b,
+                          base + p.off_xch + slot * kXchBytes, abort_flag);
   }
   tc_fence_before();
   __syncthreads();
@@ -1243,7 +1323,8 @@ bool plan_smem(StackParams& p, int n_layer, int lp_max, bool pair, int& smem_byt
   p.off_kv = a_bytes;
   const int kv_bytes = 2 * lp_max * D * 2;
   p.off_ones = p.off_kv + ((kv_bytes + 1023) & ~1023);
-  p.off_ring = p.off_ones + kOnesBytes;
+  p.off_xch = p.off_ones + kOnesBytes;
+  p.off_ring = p.off_xch + 2 * kXchBytes;
   const int vec_bytes = vec_floats<D>() * 4;
   const int fixed = p.off_ring + kBarArea;
   int stages = std::min(kMaxStages, (kSmemLimit - fixed - vec_bytes) / Cfg<D>::kItemBytes);
@@ -1273,7 +1354,7 @@ template <int D, int SW, bool UM>
 tr_status launch(int grid, const StackParams& p, int smem, cudaStream_t st) {
   auto k = stack_kernel<D, SW, UM>;
   TR_TRY(ensure_smem_attr((const void*)k, kSmemLimit));
-  k<<<grid, kThreads, smem, st>>>(p);
+  k<<<grid, Par<D>::kThreads, smem, st>>>(p);
   TR_LAUNCH_CHECK(UM ? "stack_kernel (user side)" : "stack_kernel");
   return TR_OK;
 }
