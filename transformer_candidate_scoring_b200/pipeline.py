@@ -572,12 +572,15 @@ class Streamed:
         api.score_candidates(self.slots[0].model, self.tokens[p:p + b - a], off, kv, lu, dm,
                              self.scores[p:p + b - a], stream=stream)
 
-    def run(self, first: int, count: int, stream=None, bind=None, fronted=None, scored=None) -> None:
+    def run(self, first: int, count: int, stream=None, bind=None, fronted=None, scored=None,
+            timing=None) -> None:
         """Batches first .. first + count - 1 on ``stream`` (the caller's), which waits for
         all of them at the end.  Hooks as in Overlapped.run: bind(i, dw, main) before batch
         i's first launch, fronted(i, dw, main) after its target aggregation, scored(i, dw, s)
         after the launch that completes its scores (``dw.scores``; an event it returns is
-        waited for before the slot's scores are written again)."""
+        waited for before the slot's scores are written again).  ``timing``: a list that
+        receives (kind, start event, end event, candidates) for every compress and score
+        launch (timing events around each; not for graph capture)."""
         n, m = self.n, len(self.slots)
         main = stream if stream is not None else torch.cuda.current_stream(self.slots[0].device)
         start = torch.cuda.Event()
@@ -610,8 +613,11 @@ class Streamed:
             elif step[0] == "compress":
                 _, a, b = step
                 p = self._pos(first, a)
+                t0 = self._mark(main, timing)
                 api.compress_targets(self.slots[0].model, self.X[p:p + b - a], self.tokens[p:p + b - a],
                                      stream=main)
+                if timing is not None:
+                    timing.append(("compress", t0, self._mark(main, timing), b - a))
             else:
                 _, a, b = step
                 for j in range(a // n, (b - 1) // n + 1):
@@ -620,7 +626,10 @@ class Streamed:
                         if released.get(j - m) is not None:   # the slot's last scores were read
                             main.wait_event(released.pop(j - m))
                         waited.add(j)
+                t0 = self._mark(main, timing)
                 self._score(first, a, b, main)
+                if timing is not None:
+                    timing.append(("score", t0, self._mark(main, timing), b - a))
                 for j in range(score_end // n, b // n):   # batches completed by this launch
                     if scored is not None:
                         released[j] = scored(first + j, self.slots[(first + j) % m], main)
@@ -633,6 +642,14 @@ class Streamed:
         for ev in released.values():
             if ev is not None:
                 main.wait_event(ev)
+
+    @staticmethod
+    def _mark(stream, timing):
+        if timing is None:
+            return None
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(stream)
+        return ev
 
     def capture(self, first: int, count: int, **hooks) -> "torch.cuda.CUDAGraph":
         """run(first, count, ...) captured into one CUDA graph (warmed as in
