@@ -18,8 +18,9 @@
 //                   accumulate into it in place
 //     [D, D + 128)  work area W, in turn: own K, own V, Q (each read out by the epilogue),
 //                   the scores of one head group (numerators written back over them as
-//                   fp16, the A operand of P V and of a product with ones, whose results,
-//                   the attention numerator sums and the row sum, land beside them), the
+//                   fp16, the A operand of P V, whose result lands beside them; with one
+//                   epilogue thread per row also of a product with ones that gives the
+//                   numerators' row sum, which two threads per row add up themselves), the
 //                   FFN hidden units (a 128-wide half at a time; ReLU written back as fp16,
 //                   the A operand of W2)
 //   shared memory
@@ -263,6 +264,13 @@ __device__ __forceinline__ uint32_t exp2_h2(float a, float b) {   // a -> low ha
   asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h));
   return r;
 }
+// s_lo += low half of w, s_hi += high half (fp16 -> fp32 adds)
+__device__ __forceinline__ void acc_h2(float& s_lo, float& s_hi, uint32_t w) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.f16 %0, l, %0;\n\tadd.rn.f32.f16 %1, h, %1;\n\t}"
+      : "+f"(s_lo), "+f"(s_hi)
+      : "r"(w));
+}
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -450,7 +458,8 @@ __device__ void mma_issuer(const StackParams& p, int slot, uint32_t tmem, uint32
           for (int kk = 0; kk < t.Lp / 16; ++kk) {
             mma_bf16_ta(pc + HW / 2, pc + kk * 8, sdesc(vimg + (2 * kk * (D / 8) + 2 * h) * 128, (D / 8) * 128, 128),
                         ID16, kk > 0 ? 1u : 0u);
-            mma_bf16_ta(pc + HW / 2 + 16, pc + kk * 8, sdesc(sOnes + kOnesBOff, 256, 128), ID16, kk > 0 ? 1u : 0u);
+            if (Par<D>::P == 1)   // with two epilogue parts the softmax adds the row sum itself
+              mma_bf16_ta(pc + HW / 2 + 16, pc + kk * 8, sdesc(sOnes + kOnesBOff, 256, 128), ID16, kk > 0 ? 1u : 0u);
           }
         }
         if (!UM && g == ng - 1) mma_commit(b.kv_empty(slot));
@@ -660,7 +669,7 @@ __device__ __forceinline__ void relu_in_place(uint32_t tw) {
 // numerator.  The row sum of the numerators comes from the tensor core (a product with a
 // tile of ones, beside P V), so it adds exactly the fp16 values that P V weighs.
 template <int SW, bool LEAN>
-__device__ __forceinline__ float softmax_head(uint32_t base, int Lp, int L_u, float sself) {
+__device__ __forceinline__ float softmax_head(uint32_t base, int Lp, int L_u, float sself, float* rowsum = nullptr) {
   const int nb = Lp / 16;
   float mx;
   if constexpr (SW <= 64 && !LEAN) {
@@ -711,6 +720,7 @@ __device__ __forceinline__ float softmax_head(uint32_t base, int Lp, int L_u, fl
         if (16 * c + i < L_u) mx = fmaxf(mx, v[i]);
     }
     const uint64_t l2 = f32x2(kL2E, kL2E), n2 = f32x2(-mx * kL2E, -mx * kL2E);
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
     for (int c = 0; c < nb; ++c) {
       float v[16];
@@ -725,9 +735,13 @@ __device__ __forceinline__ float softmax_head(uint32_t base, int Lp, int L_u, fl
       for (int i = 0; i < 8; ++i) {
         const uint64_t x = fma2(f32x2(v[2 * i], v[2 * i + 1]), l2, n2);
         r[i] = exp2_h2(lo32(x), hi32(x));
+        if constexpr (LEAN) acc_h2(s4[(2 * i) & 3], s4[(2 * i + 1) & 3], r[i]);
       }
       tmem_st8u(base + 8 * c, r);
     }
+    // LEAN: the numerators' row sum here (fp16 values added in fp32) instead of from the
+    // tensor core
+    if constexpr (LEAN) *rowsum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
   }
   return ex2(fmaf(sself, kL2E, -mx * kL2E));
 }
@@ -784,11 +798,12 @@ __device__ __forceinline__ void softmax_two(uint32_t base, int Lp, int L_u, floa
 // o = (ps v_own + P V) / (sum + ps) -> the head's 16 columns of A.
 template <int D, bool UM>
 __device__ __forceinline__ void finish_head(const Epi& e, uint32_t hb, int hw, int h, int k, float ps,
-                                            const uint32_t* vreg) {
+                                            const uint32_t* vreg, float rowsum) {
   constexpr int NP = Cfg<D>::kNH / Par<D>::P;
   float o[16];
   tmem_ld16(hb + hw / 2, o);
-  float sum = tmem_ld1(hb + hw / 2 + 16);
+  float sum = rowsum;
+  if constexpr (Par<D>::P == 1) sum = tmem_ld1(hb + hw / 2 + 16);
   tmem_wait_ld();
   reg_fence<16>(o);
   asm volatile("" : "+f"(sum));
@@ -961,7 +976,8 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
           e.signal();
           if (!e.wait()) return;   // P V and the row sums of group g
 #pragma unroll
-          for (int i = 0; i < 2; ++i) finish_head<D, UM>(e, e.tW + i * HW, HW, 2 * g + i, 2 * g + i, ps[i], vreg);
+          for (int i = 0; i < 2; ++i)
+            finish_head<D, UM>(e, e.tW + i * HW, HW, 2 * g + i, 2 * g + i, ps[i], vreg, 0.f);
         } else {
           const int h = HG == 2 ? 2 * g + part : g;
           const bool mine = h % P == part;
@@ -970,11 +986,11 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
           float ss = sself[0];
 #pragma unroll
           for (int j = 1; j < NP; ++j) ss = k == j ? sself[j] : ss;
-          float ps = 0.f;
-          if (mine) ps = softmax_head<SW, P == 2>(hb, t.Lp, t.L_u, ss);
+          float ps = 0.f, rowsum = 0.f;
+          if (mine) ps = softmax_head<SW, P == 2>(hb, t.Lp, t.L_u, ss, &rowsum);
           e.signal();
           if (!e.wait()) return;   // P V and the row sums of group g
-          if (mine) finish_head<D, UM>(e, hb, HW, h, k, ps, vreg);
+          if (mine) finish_head<D, UM>(e, hb, HW, h, k, ps, vreg, rowsum);
         }
         e.signal();
         if (l == 0 && g == (Groups<D, SW>::NG > 1 ? 1 : 0) && p.gate_phase == 1) e.open_gate();
