@@ -504,7 +504,8 @@ class Streamed:
     fixed-size chunks of one stream of candidates that runs across batch boundaries
     (stream_plan): by default every compress launch is two rounds of 128-candidate tiles
     on the SMs left beside one prefill CTA, every score launch one round of the score
-    kernel's two-tile units on all SMs, whichever batches the chunk falls in.  A launch that spans two batches scores
+    kernel's two-tile units on all SMs (or as many whole rounds as one batch fills),
+    whichever batches the chunk falls in.  A launch that spans two batches scores
     each candidate against its own request's cache (the kernels take a list of requests).
       main stream  target aggregation of batch i, then every compress and score chunk that
                    has become complete (a score chunk after the prefills of the batches it
@@ -542,9 +543,12 @@ class Streamed:
             c.scores = self.scores[k * n:(k + 1) * n]
             self.slots.append(c)
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
-        self.comp_chunk = comp_chunk if comp_chunk is not None else 2 * (sms - 1) * SCORE_TILE
-        self.score_units = score_units if score_units is not None else sms
         self.bounds = unit_bounds(dw.req_offsets)
+        # as many whole rounds per launch as one batch fills (a launch has a fixed cost, so a
+        # large batch takes a few large launches rather than many one-round ones)
+        comp_round = 2 * (sms - 1) * SCORE_TILE
+        self.comp_chunk = comp_chunk if comp_chunk is not None else comp_round * max(1, n // comp_round)
+        self.score_units = score_units if score_units is not None else sms * max(1, len(self.bounds) // sms)
         self.group = group
         _, hi = torch.cuda.Stream.priority_range()
         self.user = torch.cuda.Stream(dev, priority=hi)
