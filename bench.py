@@ -19,7 +19,7 @@ copied back, all inside the timed region.  Requests rotate over several seeded r
 embedding tables (24.6 GB) are far larger than L2.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-  python bench.py --case bulk|uncompressed [--case-n N]      side measurements (JSON line)
+  python bench.py --case bulk|uncompressed|fused [--case-n N]  side measurements (JSON line)
   python bench.py --case score|compress|prefill|all          one stage, for a profiler
 
 Multi-GPU: one process per GPU (torchrun); every rank scores its own requests (weak
@@ -694,7 +694,7 @@ def run_case(args):
         print("case stream: ok")
         return
     if args.case == "gather":
-        ws = datagen.scaled(w, n_cand_per_request=n, rows=args.case_rows)
+        ws = datagen.scaled(w, n_cand_per_request=n, rows=args.case_rows or 1_000_000)
         tables = [torch.empty(r, dims.D, dtype=torch.bfloat16, device="cuda") for r in ws.target_rows]
         for t, x in enumerate(tables):
             datagen.fill_table_device(x, ws.seed, datagen.target_table_id(ws, t))
@@ -803,6 +803,60 @@ def run_uncompressed(args):
                       "flops_per_candidate_L_t_1": f1, "flop_saving": 1 - f1 / f8}), flush=True)
 
 
+def run_fused(args):
+    """The target side of one 128D-5L request (--case-n candidates, 8 fields over the 4M-row
+    target tables) as two launches (tr_aggregate, then tr_compress_targets) and as one
+    (tr_compress_target_bags, the gather feeding the compressor on chip); prints one JSON
+    line with both device times (CUDA events, --case-reps launches each after a warm-up) and
+    whether the two results are bit-identical."""
+    import torch
+
+    from transformer_candidate_scoring_b200 import api
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags, DeviceWorkload
+
+    w = datagen.WORKLOADS[WORKLOAD]
+    if args.case_rows is not None and args.case_rows < min(w.target_rows):
+        w = datagen.scaled(w, rows=args.case_rows)
+    dims = w.dims
+    n, F, D = args.case_n, dims.n_target_fields, dims.D
+    tables = DeviceWorkload.make_tables(w.with_(user_tables=0), torch.device("cuda"))[1]
+    model = api.Model(dims, datagen.workload_params(w))
+    bags = DeviceBags.of(datagen.make_target_bags(np.random.default_rng(w.seed + 5), w, n), "cuda")
+    ba = (bags.bag_table, bags.offsets, bags.keys, bags.weights)
+    X = torch.empty(n * F, D, dtype=torch.bfloat16, device="cuda")
+    two = torch.empty(n, D, dtype=torch.float32, device="cuda")
+    fused = torch.empty_like(two)
+
+    def two_launch():
+        api.aggregate(tables, *ba, X)
+        api.compress_targets(model, X.view(n, F * D), two)
+
+    def one_launch():
+        api.compress_target_bags(model, tables, *ba, fused)
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+    reps = max(1, args.case_reps)
+    t_two = timed(two_launch, reps)
+    t_one = timed(one_launch, reps)
+    if api.sync_status() != 0:
+        raise RuntimeError("device status word set")
+    print(json.dumps({"case": "fused_target_side", "candidates": n, "ms_gather_then_compress": t_two,
+                      "ms_fused": t_one, "speedup": t_two / t_one, "bit_identical": bool(torch.equal(two, fused)),
+                      "workload": f"128D-5L target side, 8 fields of 1..8 keys over {min(w.target_rows)}-row "
+                                  "bf16 tables"}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -813,18 +867,22 @@ def main():
     ap.add_argument("--no-side-configs", action="store_true", help="skip the 64D-3L, packed and large workloads")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--case", choices=["score", "compress", "prefill", "all", "gather", "stream", "bulk",
-                                       "uncompressed"],
+                                       "uncompressed", "fused"],
                     default=None,
                     help="run one stage on stand-alone inputs for a profiler (no timing, no JSON)")
     ap.add_argument("--case-n", type=int, default=40000)
     ap.add_argument("--case-reps", type=int, default=2)
-    ap.add_argument("--case-rows", type=int, default=1_000_000, help="table rows of the gather case")
+    ap.add_argument("--case-rows", type=int, default=None,
+                    help="table rows of the gather case (default 1M) and of the fused case (default 4M)")
     args = ap.parse_args()
     if args.case == "bulk":
         run_bulk(args)
         return
     if args.case == "uncompressed":
         run_uncompressed(args)
+        return
+    if args.case == "fused":
+        run_fused(args)
         return
     if args.case:
         run_case(args)

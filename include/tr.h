@@ -7,6 +7,8 @@
  *   tr_prefill_user      user tokens + domain embedding through the N-layer Pre-LN
  *                        Transformer, writing the per-layer user K/V cache          (§3.1, §3.4)
  *   tr_compress_targets  3-layer MLP target compressor, F*D -> D                    (§3.3)
+ *   tr_compress_target_bags  the aggregation of the target fields feeding the compressor
+ *                        in one launch, the compressor's input built on chip (§3.2 + §3.3)
  *   tr_score_candidates  single-token candidates through the same layer stack over
  *                        the broadcast user K/V, then the linear head; candidates of
  *                        several requests packed in one call, each isolated to its
@@ -213,6 +215,29 @@ tr_status tr_prefill_users(const tr_model* m, const float* const* user_tokens, c
  */
 tr_status tr_compress_targets(const tr_model* m, const void* x, int64_t n, void* tokens,
                               tr_stream stream);
+
+/*
+ * The target side in one launch: the weighted-average aggregation of TransRetrieval §3.2
+ * feeding the compressor of §3.3, whose input row (the concatenation of a candidate's F
+ * field tokens) is built in shared memory and never written to device memory.  Candidate c's
+ * field f is bag c*F + f (F = n_target_fields), as tr_aggregate lays the rows of x out; its
+ * token is rounded to bf16 exactly as tr_aggregate(..., TR_BF16, ...) rounds it, so the
+ * result equals tr_aggregate followed by tr_compress_targets bit for bit, except where
+ * tr_aggregate takes its few-bags path (at most 4 bags per SM), which sums in another order.
+ *   tables     HOST array [n_tables] of bf16 tables of width D (DEVICE data, 16-byte aligned)
+ *   bag_table  DEVICE int32 [n*F]      table of each bag (outside 0..n_tables-1: token 0)
+ *   offsets    DEVICE int64 [n*F + 1]  CSR offsets into keys / weights
+ *   keys       DEVICE int32, weights DEVICE fp32 (a key outside its table is skipped and
+ *              sets the device status, as in tr_aggregate)
+ *   tokens     DEVICE fp32 [n][D], 16-byte aligned.
+ * Needs a TR_BF16 model served by the tensor-core compressor with D a multiple of 64 and
+ * comp_dims[0] == F*D; otherwise TR_ERR_UNSUPPORTED and nothing is launched.  Uses the same
+ * per-stream work counter as tr_compress_targets.
+ */
+tr_status tr_compress_target_bags(const tr_model* m, const tr_table* tables, int n_tables,
+                                  const int32_t* bag_table, const int64_t* offsets,
+                                  const int32_t* keys, const float* weights, int64_t n,
+                                  void* tokens, tr_stream stream);
 
 /*
  * Score packed candidates (TransRetrieval §3.3 and deployment "Hardware-aware inference

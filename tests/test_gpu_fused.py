@@ -1,0 +1,95 @@
+"""GPU parity of the fused target side, tr_compress_target_bags: the weighted-average
+aggregation of TransRetrieval §3.2 building the compressor's input rows (§3.3) on chip.
+
+Three checks on the same seeded tables and bags:
+  - against the fp64 oracle (weighted average, concatenation in field order, compressor),
+    at the intermediate bar of tests/common.py;
+  - bit for bit against the two launches it replaces (tr_aggregate to bf16, then
+    tr_compress_targets), whenever tr_aggregate takes its many-bags kernel, which sums in the
+    same order;
+  - empty bags, out-of-range keys and bad table ids behave as in tr_aggregate.
+"""
+import numpy as np
+import pytest
+import torch
+
+import datagen
+import oracle
+from common import check_close
+from test_gpu_parity import _bags, _oracle_agg, _tables, dev, dims_of, tr
+
+pytestmark = pytest.mark.gpu
+
+
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+def _both(m, dims, tables, bags, n):
+    """(fused tokens, two-launch tokens) for n candidates."""
+    F, D = dims.n_target_fields, dims.D
+    args = [dev(bags.bag_table), dev(bags.offsets), dev(bags.keys), dev(bags.weights)]
+    fused = torch.empty(n, D, dtype=torch.float32, device="cuda")
+    tr().compress_target_bags(m, tables, *args, fused)
+    X = torch.empty(n * F, D, dtype=torch.bfloat16, device="cuda")
+    tr().aggregate(tables, *args, X)
+    two = torch.empty(n, D, dtype=torch.float32, device="cuda")
+    tr().compress_targets(m, X.view(n, F * D), two)
+    torch.cuda.synchronize()
+    return fused, two
+
+
+@pytest.mark.parametrize("name,n,init,max_nf", [
+    ("128d5l", 300, "paper", 8),     # three tiles, a ragged one
+    ("128d5l", 1000, "wide", 8),     # eight tiles
+    ("128d5l", 130, "paper", 40),    # bags of several key chunks
+    ("64d3l", 777, "wide", 8),       # one 64-column slice per field
+    ("128d5l", 1, "wide", 8),        # one candidate
+])
+def test_fused_target_side_parity(name, n, init, max_nf):
+    dims = dims_of(name)
+    F, D = dims.n_target_fields, dims.D
+    P = datagen.make_params(dims, 4, init)
+    m = tr().Model(dims, P)
+    rows, n_tables = 5000, 3
+    tables = _tables(11, n_tables, rows, D, "bf16")
+    bags = _bags(np.random.default_rng(n + D), n * F, max_nf, rows, n_tables)
+    fused, two = _both(m, dims, tables, bags, n)
+    assert tr().sync_status() == 0
+    if n * F > 4 * _sms():
+        assert torch.equal(fused, two)
+    X = _oracle_agg(11, bags, rows, D, "bf16").reshape(n, F * D)
+    ref = oracle.compress_targets(P, X)
+    check_close(fused.double().cpu().numpy(), ref, "bf16", "tokens", kind="intermediate")
+
+
+def test_fused_target_side_bad_keys_and_tables():
+    """A key outside its table is skipped and reported; a bag naming no table gives a zero
+    token; both exactly as the two launches handle them."""
+    dims = dims_of("128d5l")
+    F = dims.n_target_fields
+    n = 200
+    m = tr().Model(dims, datagen.make_params(dims, 4, "paper"))
+    tables = _tables(11, 2, 3000, dims.D, "bf16")
+    bags = _bags(np.random.default_rng(3), n * F, 8, 3000, 2, empty_frac=0.2)
+    keys = bags.keys.copy()
+    keys[5] = 3000
+    keys[len(keys) // 2] = -1
+    tab = bags.bag_table.copy()
+    tab[17] = 2
+    tab[40] = -3
+    bad = datagen.Bags(bags.offsets, keys, bags.weights, tab)
+    fused, two = _both(m, dims, tables, bad, n)
+    assert tr().sync_status() == 4
+    assert tr().sync_status() == 0
+    assert torch.equal(fused, two)
+
+
+def test_fused_target_side_refuses_unsupported_models():
+    dims = dims_of("tiny")     # fp32 model: no tensor-core compressor
+    m = tr().Model(dims, datagen.make_params(dims, 4, "paper"))
+    tables = _tables(11, 1, 100, dims.D, "f32")
+    z = torch.zeros(2, dtype=torch.int64, device="cuda")
+    out = torch.empty(1, dims.D, dtype=torch.float32, device="cuda")
+    with pytest.raises(Exception):
+        tr().compress_target_bags(m, tables, z.int(), z, z.int(), z.float(), out)

@@ -5,8 +5,8 @@ include/tr.h); this package is its Python binding plus the device-resident workl
 driver.  There is no CPU fallback: every call raises if libtr.so is missing.
 """
 from . import api
-from .api import (Model, TrError, aggregate, compress_targets, kv_cache_bytes, prefill_user,
-                  prefill_user_noalloc, score_candidates, sync_status, topk)
+from .api import (Model, TrError, aggregate, compress_target_bags, compress_targets, kv_cache_bytes,
+                  prefill_user, prefill_user_noalloc, score_candidates, sync_status, topk)
 
-__all__ = ["api", "Model", "TrError", "aggregate", "compress_targets", "kv_cache_bytes",
+__all__ = ["api", "Model", "TrError", "aggregate", "compress_target_bags", "compress_targets", "kv_cache_bytes",
            "prefill_user", "prefill_user_noalloc", "score_candidates", "sync_status", "topk"]

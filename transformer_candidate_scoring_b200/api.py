@@ -185,6 +185,22 @@ def compress_targets(model: Model, x: torch.Tensor, tokens: torch.Tensor, stream
     return tokens
 
 
+def compress_target_bags(model: Model, tables: Sequence[torch.Tensor], bag_table: torch.Tensor,
+                         offsets: torch.Tensor, keys: torch.Tensor, weights: torch.Tensor, tokens: torch.Tensor,
+                         stream=None) -> torch.Tensor:
+    """tr_compress_target_bags: the target side in one launch, n = tokens.shape[0]
+    candidates whose F field bags are c*F .. c*F+F-1 -> tokens [n, D] fp32."""
+    if tokens.dtype != torch.float32:
+        raise ValueError("compressed tokens are fp32")
+    n = len(tables)
+    arr = (L.Table * max(n, 1))()
+    for i, t in enumerate(tables):
+        arr[i] = L.Table(t.data_ptr(), t.shape[0], dtype_code(t.dtype))
+    _check(L.load().tr_compress_target_bags(model.handle, arr, n, _ptr(bag_table), _ptr(offsets), _ptr(keys),
+                                            _ptr(weights), tokens.shape[0], _ptr(tokens), _stream(stream)))
+    return tokens
+
+
 def score_candidates(model: Model, tokens: torch.Tensor, req_offsets: Sequence[int], kv: Sequence[torch.Tensor],
                      L_u: Sequence[int], domain: Sequence[int], scores: torch.Tensor, stream=None) -> torch.Tensor:
     """tr_score_candidates over packed requests: tokens [n, D] fp32; scores [n] fp32."""

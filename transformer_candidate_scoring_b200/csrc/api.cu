@@ -144,6 +144,10 @@ tr_status tc_score(const tr_model* m, const void* tokens, int64_t n, const int64
                    cudaStream_t st);
 bool tc_comp_supported(const tr_model* m);
 tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens, cudaStream_t st);
+bool tc_comp_bags_supported(const tr_model* m);
+tr_status tc_compress_bags(const tr_model* m, const tr_table* tables, int n_tables, const int32_t* bag_table,
+                           const int64_t* offsets, const int32_t* keys, const float* weights, int64_t n,
+                           void* tokens, cudaStream_t st);
 bool tc_prefill_supported(const tr_model* m, int L_u);
 tr_status simt_prefill_noalloc(const tr_model* m, const float* user_tokens, int L_u, int domain, void* kv,
                                cudaStream_t st);
@@ -361,6 +365,27 @@ tr_status tr_compress_targets(const tr_model* m, const void* x, int64_t n, void*
   if (m->desc.dtype == TR_BF16 && tc_comp_supported(m))
     return tc_compress(m, x, n, tokens, (cudaStream_t)stream);
   return simt_compress(m, x, n, tokens, (cudaStream_t)stream);
+}
+
+tr_status tr_compress_target_bags(const tr_model* m, const tr_table* tables, int n_tables, const int32_t* bag_table,
+                                  const int64_t* offsets, const int32_t* keys, const float* weights, int64_t n,
+                                  void* tokens, tr_stream stream) {
+  TR_TRY(check_model_device(m));
+  if (n < 0) return fail(TR_ERR_INVALID_ARG, "n=%lld", (long long)n);
+  if (!tables || n_tables <= 0 || n_tables > TR_MAX_TABLES)
+    return fail(TR_ERR_INVALID_ARG, "n_tables=%d (need 1..%d) or tables null", n_tables, TR_MAX_TABLES);
+  for (int i = 0; i < n_tables; ++i) {
+    if (!tables[i].data || tables[i].n_rows <= 0) return fail(TR_ERR_INVALID_ARG, "table %d is empty or null", i);
+    if (tables[i].dtype != TR_BF16) return fail(TR_ERR_INVALID_ARG, "table %d is not bf16", i);
+    if ((uintptr_t)tables[i].data % 16) return fail(TR_ERR_INVALID_ARG, "table %d is not 16-byte aligned", i);
+  }
+  if (!(m->desc.dtype == TR_BF16 && tc_comp_bags_supported(m)))
+    return fail(TR_ERR_UNSUPPORTED,
+                "tr_compress_target_bags needs a bf16 model on the tensor-core compressor with D a multiple of 64");
+  if (n == 0) return TR_OK;
+  if (!bag_table || !offsets || !keys || !weights || !tokens) return fail(TR_ERR_INVALID_ARG, "null device pointer");
+  if ((n + 127) / 128 > INT32_MAX) return fail(TR_ERR_INVALID_ARG, "n=%lld is too large", (long long)n);
+  return tc_compress_bags(m, tables, n_tables, bag_table, offsets, keys, weights, n, tokens, (cudaStream_t)stream);
 }
 
 tr_status tr_score_candidates(const tr_model* m, const void* tokens, int64_t n, const int64_t* req_offsets,

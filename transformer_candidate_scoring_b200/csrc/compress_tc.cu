@@ -37,20 +37,62 @@ namespace {
 using namespace tc;
 
 constexpr int kM = 128;
-constexpr int STAGE1 = 80 * 1024;              // x slice (16 KB) + W1 slice (<= 64 KB)
-constexpr int OFF_R1 = 0;
-constexpr int OFF_R2 = 2 * STAGE1;             // 160 KB
-constexpr int STAGE2 = 32 * 1024;
-constexpr int OFF_BAR = OFF_R2 + 2 * STAGE2;   // 224 KB
-constexpr int OFF_B3 = OFF_BAR + 256;           // the last layer's bias (c3 <= 256 floats)
-constexpr int SMEM_BYTES = OFF_B3 + 1024 + 1024;
-// The per-column vectors of the layer whose epilogue runs are staged in shared memory at
-// R1 + 132 KB (8 KB): that part of the second x/W1 stage is idle from the end of a tile's
-// first GEMM until the next tile's loads, which wait for its last GEMM.
-constexpr int OFF_VEC = OFF_R1 + 132 * 1024;
+
+// Shared-memory plan of the two variants.
+//  - Plain (x from global memory): R1 holds two stages of [x slice (16 KB) | W1 slice (<= 64 KB)];
+//    R2 two stages of 64-wide W2 / W3 slices (32 KB).  The hidden activations of layers 1 and 2
+//    (fp16, <= 128 KB) are written over R1 once a tile's first GEMM is done; the LayerNorm
+//    exchange buffer (R1 + 128 KB) and the per-column vectors of the running epilogue
+//    (R1 + 132 KB, 8 KB) sit in the part of the second stage that is idle from the end of a
+//    tile's first GEMM until the next tile's loads, which wait for its last GEMM.
+//  - Gathering (x built on chip from the bags): R1 holds two W1 slices (64 KB each) and the
+//    hidden activations; x has a ring of its own (three 16 KB stages), so the gather warps run
+//    ahead of the tile in flight; W2 / W3 go in 32-wide slices (16 KB stages) to make room.
+template <bool G> struct CLayout;
+template <> struct CLayout<false> {
+  static constexpr int THREADS = 320, EPI0 = 2;   // warps 2-9 run the epilogues
+  static constexpr int STAGE1 = 80 * 1024, W1_OFF = 16384;
+  static constexpr int XR = 0, XSTAGE = 0;
+  static constexpr int R2 = 2 * STAGE1, STAGE2 = 32 * 1024, KW2 = 64;
+  static constexpr int XBUF = 128 * 1024, VEC = 132 * 1024;
+  static constexpr int BAR = R2 + 2 * STAGE2;
+};
+template <> struct CLayout<true> {
+  // five warpgroups: copy and MMA threads (warps 0-3), epilogues (4-11), gather (12-19);
+  // launched at 96 registers a thread, the control warpgroup gives registers to the others
+  static constexpr int THREADS = 640, EPI0 = 4, GW0 = 12;
+  static constexpr int LAUNCH_REGS = 96, CTL_REGS = 32, EPI_REGS = 104, GATHER_REGS = 120;
+  static constexpr int STAGE1 = 64 * 1024, W1_OFF = 0;
+  static constexpr int XR = 2 * STAGE1, XSTAGE = 16 * 1024, NX = 2;
+  static constexpr int R2 = XR + NX * XSTAGE, STAGE2 = 16 * 1024, KW2 = 32;
+  static constexpr int XBUF = R2 + 2 * STAGE2, VEC = XBUF + 4096;
+  // the tile's bag headers: kM * F + 1 offsets (int64), then kM * F table ids (F <= 8)
+  static constexpr int HDR = VEC + 8192, HDR_TAB = HDR + (kM * 8 + 2) * 8;
+  static constexpr int BAR = HDR_TAB + kM * 8 * 4;
+};
+template <bool G> constexpr int smem_bytes() { return CLayout<G>::BAR + 256 + 1024 + 1024; }
+static_assert(128 * CLayout<true>::CTL_REGS + 256 * (CLayout<true>::EPI_REGS + CLayout<true>::GATHER_REGS) <=
+                  CLayout<true>::THREADS * CLayout<true>::LAUNCH_REGS &&
+              CLayout<true>::THREADS * CLayout<true>::LAUNCH_REGS <= 65536,
+              "register split of the gathering variant");
+static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "shared memory plan");
+constexpr int kGatherWarps = 8;
+constexpr int kMaxGatherFields = 8;   // the header table holds kM * 8 bags
+
+// The bags of the gathering variant: candidate c's F field bags are c*F .. c*F + F - 1
+// (the layout tr_aggregate reads), each over one of the bf16 tables.
+struct GatherArgs {
+  const uint16_t* tab[TR_MAX_TABLES];
+  int rows[TR_MAX_TABLES];     // min(rows, INT32_MAX): every int32 key is below it past that
+  const int32_t* bag_table;
+  const int64_t* offsets;
+  const int32_t* keys;
+  const float* weights;
+  int n_tables, F, D;
+};
 
 struct CompParams {
-  CUtensorMap xmap;            // x [n][c0] bf16, box {64, 128}, 128-byte swizzle
+  CUtensorMap xmap;            // x [n][c0] bf16, box {64, 128}, 128-byte swizzle (plain variant)
   const uint8_t* w1;           // [c0/64] slices of W1^T [c1 x 64]
   const uint8_t* w2;           // [c1/64] slices of W2^T [c2 x 64]
   const uint8_t* w3;           // [c2/64] slices of W3^T [c3 x 64]
@@ -60,11 +102,14 @@ struct CompParams {
   int* claim;                  // next unclaimed tile (zero at launch)
   long long n;
   int n_tiles, c0, c1, c2, c3;
+  GatherArgs g;                // gathering variant only
 };
 
 struct CBars {
   uint32_t full1[2], empty1[2], full2[2], empty2[2], r1_free, mma, epi, drain, qsync[4], vsync;
   uint32_t tile_full[2], tile_empty[2], tile_slot[2];   // the claimed-tile ring
+  uint32_t xfull[3], xempty[3];                         // the x ring (gathering variant)
+  uint32_t gsync;                                       // rendezvous of the gather warps
 };
 
 // Next tile index of this CTA from the two-entry ring (-1: no more); the reader releases
@@ -80,6 +125,13 @@ __device__ __forceinline__ int next_tile(const CBars& b, int& ts, uint32_t& tph,
     tph ^= 1;
   }
   return ok ? t : -1;
+}
+
+// Long waits of the gathering variant suspend instead of spinning (its gather warps need the
+// issue slots); the plain variant keeps the spinning wait.
+template <bool G>
+__device__ __forceinline__ bool cwait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  return G ? mbar_wait_idle(bar, parity, abort_flag) : mbar_wait(bar, parity, abort_flag);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
@@ -106,51 +158,64 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
          (2ull << 61);
 }
 
+// Copy thread.  Plain variant: claims the tiles, publishes them to the other roles and
+// loads each x slice with its W1 slice.  Gathering variant: reads the tiles from the ring
+// (the gather warps claim them) and loads only weights.
+template <bool G>
 __device__ void comp_producer(const CompParams& p, uint32_t r1, uint32_t r2, const CBars& b, volatile int* abort_flag) {
+  using L = CLayout<G>;
   int s1 = 0, s2 = 0;
   uint32_t ph1 = 0, ph2 = 0, free_phase = 0;
-  const uint32_t w1_bytes = p.c1 * 128, w2_bytes = p.c2 * 128, w3_bytes = p.c3 * 128;
+  const uint32_t w1_bytes = p.c1 * 128, w2_bytes = p.c2 * L::KW2 * 2, w3_bytes = p.c3 * L::KW2 * 2;
   bool ok = true;
   bool pend1[2] = {false, false}, pend2[2] = {false, false};
   uint32_t par1[2] = {0, 0}, par2[2] = {0, 0};
   int ts = 0;
   uint32_t tph = 0;
-  for (int tile = atomicAdd(p.claim, 1); ok;) {
-    // publish the tile (or the end) to the MMA and epilogue threads
-    if (!(ok = mbar_wait(b.tile_empty[ts], tph ^ 1, abort_flag))) break;
-    const int pub = tile < p.n_tiles ? tile : -1;
-    asm volatile("st.shared.b32 [%0], %1;" ::"r"(b.tile_slot[ts]), "r"(pub) : "memory");
-    mbar_arrive(b.tile_full[ts]);
-    if (++ts == 2) {
-      ts = 0;
-      tph ^= 1;
+  for (int tile = G ? 0 : atomicAdd(p.claim, 1); ok;) {
+    int cur;
+    if constexpr (G) {
+      cur = next_tile(b, ts, tph, abort_flag, ok);
+    } else {
+      // publish the tile (or the end) to the MMA and epilogue threads
+      if (!(ok = mbar_wait(b.tile_empty[ts], tph ^ 1, abort_flag))) break;
+      cur = tile < p.n_tiles ? tile : -1;
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(b.tile_slot[ts]), "r"(cur) : "memory");
+      mbar_arrive(b.tile_full[ts]);
+      if (++ts == 2) {
+        ts = 0;
+        tph ^= 1;
+      }
     }
-    if (pub < 0) break;
+    if (cur < 0) break;
     // the stage buffers hold the previous tile's activations until its last GEMM is done
-    if (!(ok = mbar_wait(b.r1_free, free_phase ^ 1, abort_flag))) break;
+    if (!(ok = cwait<G>(b.r1_free, free_phase ^ 1, abort_flag))) break;
     free_phase ^= 1;
     for (int kc = 0; kc < p.c0 / 64 && ok; ++kc) {
-      if (!(ok = mbar_wait(b.empty1[s1], ph1 ^ 1, abort_flag))) break;
-      const uint32_t st = r1 + s1 * STAGE1;
-      mbar_arrive_expect_tx(b.full1[s1], kM * 64 * 2 + w1_bytes);
-      tma_load_2d(st, &p.xmap, kc * 64, tile * kM, b.full1[s1]);
-      bulk_g2s(st + 16384, p.w1 + (size_t)kc * w1_bytes, w1_bytes, b.full1[s1]);
+      if (!(ok = cwait<G>(b.empty1[s1], ph1 ^ 1, abort_flag))) break;
+      const uint32_t st = r1 + s1 * L::STAGE1;
+      mbar_arrive_expect_tx(b.full1[s1], (G ? 0 : kM * 64 * 2) + w1_bytes);
+      if constexpr (!G) tma_load_2d(st, &p.xmap, kc * 64, cur * kM, b.full1[s1]);
+      bulk_g2s(st + L::W1_OFF, p.w1 + (size_t)kc * w1_bytes, w1_bytes, b.full1[s1]);
       pend1[s1] = true;
       par1[s1] = ph1;
       if (++s1 == 2) { s1 = 0; ph1 ^= 1; }
     }
-    for (int j = 0; j < p.c1 / 64 + p.c2 / 64 && ok; ++j) {
-      if (!(ok = mbar_wait(b.empty2[s2], ph2 ^ 1, abort_flag))) break;
-      const bool is2 = j < p.c1 / 64;
+    // W2 / W3 in KW2-wide slices: the images hold 64-wide slices one after the other, and
+    // the first and second 32 columns of one are its two halves, so slice j of width KW2
+    // starts j slices in
+    for (int j = 0; j < p.c1 / L::KW2 + p.c2 / L::KW2 && ok; ++j) {
+      if (!(ok = cwait<G>(b.empty2[s2], ph2 ^ 1, abort_flag))) break;
+      const bool is2 = j < p.c1 / L::KW2;
       const uint32_t bytes = is2 ? w2_bytes : w3_bytes;
-      const uint8_t* src = is2 ? p.w2 + (size_t)j * w2_bytes : p.w3 + (size_t)(j - p.c1 / 64) * w3_bytes;
+      const uint8_t* src = is2 ? p.w2 + (size_t)j * w2_bytes : p.w3 + (size_t)(j - p.c1 / L::KW2) * w3_bytes;
       mbar_arrive_expect_tx(b.full2[s2], bytes);
-      bulk_g2s(r2 + s2 * STAGE2, src, bytes, b.full2[s2]);
+      bulk_g2s(r2 + s2 * L::STAGE2, src, bytes, b.full2[s2]);
       pend2[s2] = true;
       par2[s2] = ph2;
       if (++s2 == 2) { s2 = 0; ph2 ^= 1; }
     }
-    tile = atomicAdd(p.claim, 1);
+    if constexpr (!G) tile = atomicAdd(p.claim, 1);
   }
   if (!ok) {
     for (int s = 0; s < 2; ++s) {
@@ -162,16 +227,19 @@ __device__ void comp_producer(const CompParams& p, uint32_t r1, uint32_t r2, con
   }
 }
 
+template <bool G>
 __device__ void comp_mma(const CompParams& p, uint32_t tmem, uint32_t r1, uint32_t r2, const CBars& b,
                          volatile int* abort_flag) {
-  int s1 = 0, s2 = 0;
-  uint32_t ph1 = 0, ph2 = 0, epi_phase = 0;
+  using L = CLayout<G>;
+  constexpr int KS = L::KW2 / 16;   // MMAs per W2 / W3 slice
+  int s1 = 0, s2 = 0, sx = 0;
+  uint32_t ph1 = 0, ph2 = 0, phx = 0, epi_phase = 0;
   bool ok = true;
   const int n1 = std::min(p.c1, 256);
   // layer 1 multiplies bf16 x by bf16 W1; layers 2 and 3 fp16 activations by fp16 weights
   const uint32_t id1 = idesc_bf16(kM, n1), id2 = idesc_f16c(kM, p.c2), id3 = idesc_f16c(kM, p.c3);
   auto wait_epi = [&]() {
-    ok = ok && mbar_wait(b.epi, epi_phase, abort_flag);
+    ok = ok && cwait<G>(b.epi, epi_phase, abort_flag);
     epi_phase ^= 1;
     tc_fence_after();
     return ok;
@@ -184,9 +252,13 @@ __device__ void comp_mma(const CompParams& p, uint32_t tmem, uint32_t r1, uint32
     if (!first && !wait_epi()) break;   // previous tile's last epilogue has read TMEM
     // layer 1: [128 x c0] x [c0 x c1]
     for (int kc = 0; kc < p.c0 / 64 && ok; ++kc) {
-      if (!(ok = mbar_wait(b.full1[s1], ph1, abort_flag))) break;
+      if (!(ok = cwait<G>(b.full1[s1], ph1, abort_flag))) break;
+      if constexpr (G) {
+        if (!(ok = mbar_wait_idle(b.xfull[sx], phx, abort_flag))) break;
+      }
       tc_fence_after();
-      const uint32_t xa = r1 + s1 * STAGE1, wb = xa + 16384;
+      const uint32_t xa = G ? r1 + L::XR + sx * L::XSTAGE : r1 + s1 * L::STAGE1;
+      const uint32_t wb = r1 + s1 * L::STAGE1 + L::W1_OFF;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         for (int nh = 0; nh < p.c1 / n1; ++nh)
@@ -195,31 +267,35 @@ __device__ void comp_mma(const CompParams& p, uint32_t tmem, uint32_t r1, uint32
                    (kc > 0 || kk > 0) ? 1u : 0u);
       mma_commit(b.empty1[s1]);
       if (++s1 == 2) { s1 = 0; ph1 ^= 1; }
+      if constexpr (G) {
+        mma_commit(b.xempty[sx]);
+        if (++sx == L::NX) { sx = 0; phx ^= 1; }
+      }
     }
     if (!ok) break;
     mma_commit(b.mma);
-    if (!wait_epi()) break;                                // h1 (bf16) in R1
-    for (int kc = 0; kc < p.c1 / 64 && ok; ++kc) {
-      if (!(ok = mbar_wait(b.full2[s2], ph2, abort_flag))) break;
+    if (!wait_epi()) break;                                // h1 (fp16) in R1
+    for (int kc = 0; kc < p.c1 / L::KW2 && ok; ++kc) {
+      if (!(ok = cwait<G>(b.full2[s2], ph2, abort_flag))) break;
       tc_fence_after();
-      const uint32_t wb = r2 + s2 * STAGE2;
+      const uint32_t wb = r2 + s2 * L::STAGE2;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem, sdesc(r1 + (4 * kc + kk) * 2 * kM * 16, kM * 16, 128),
+      for (int kk = 0; kk < KS; ++kk)
+        mma_bf16(tmem, sdesc(r1 + (KS * kc + kk) * 2 * kM * 16, kM * 16, 128),
                  sdesc(wb + kk * 2 * p.c2 * 16, p.c2 * 16, 128), id2, (kc > 0 || kk > 0) ? 1u : 0u);
       mma_commit(b.empty2[s2]);
       if (++s2 == 2) { s2 = 0; ph2 ^= 1; }
     }
     if (!ok) break;
     mma_commit(b.mma);
-    if (!wait_epi()) break;                                // h2 (bf16) in R1
-    for (int kc = 0; kc < p.c2 / 64 && ok; ++kc) {
-      if (!(ok = mbar_wait(b.full2[s2], ph2, abort_flag))) break;
+    if (!wait_epi()) break;                                // h2 (fp16) in R1
+    for (int kc = 0; kc < p.c2 / L::KW2 && ok; ++kc) {
+      if (!(ok = cwait<G>(b.full2[s2], ph2, abort_flag))) break;
       tc_fence_after();
-      const uint32_t wb = r2 + s2 * STAGE2;
+      const uint32_t wb = r2 + s2 * L::STAGE2;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16(tmem + 256, sdesc(r1 + (4 * kc + kk) * 2 * kM * 16, kM * 16, 128),
+      for (int kk = 0; kk < KS; ++kk)
+        mma_bf16(tmem + 256, sdesc(r1 + (KS * kc + kk) * 2 * kM * 16, kM * 16, 128),
                  sdesc(wb + kk * 2 * p.c3 * 16, p.c3 * 16, 128), id3, (kc > 0 || kk > 0) ? 1u : 0u);
       mma_commit(b.empty2[s2]);
       if (++s2 == 2) { s2 = 0; ph2 ^= 1; }
@@ -325,16 +401,17 @@ __device__ __forceinline__ void prelu_ln_half(CEpi& e, int cols, const float* bi
   }
 }
 
+template <bool G>
 __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, const CBars& b, float* svec,
                               float* sb3, volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   CEpi e;
   e.q = warp & 3;
   e.m = e.q * 32 + lane;
-  e.hf = (warp - 2) >> 2;
+  e.hf = (warp - CLayout<G>::EPI0) >> 2;
   e.trow = tmem + ((uint32_t)(e.q * 32) << 16);
   e.rowoff = (e.m >> 3) * 128 + (e.m & 7) * 16;
-  e.xbuf = r1 + 128 * 1024;      // idle between the first layer's MMAs and the next tile's loads
+  e.xbuf = r1 + CLayout<G>::XBUF;
   e.qbar = b.qsync[e.q];
   e.ph_q = 0;
   e.abort_flag = abort_flag;
@@ -342,7 +419,7 @@ __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, c
   const float* v1 = p.vec;
   const float* v2 = p.vec + 4 * p.c1;
   const float* b3 = v2 + 4 * p.c2;
-  const int et = threadIdx.x - 64;                 // 0 .. 255
+  const int et = threadIdx.x - 32 * CLayout<G>::EPI0;   // 0 .. 255
   for (int i = et; i < p.c3; i += 256) sb3[i] = __ldg(b3 + i);   // visible after the first vsync
   uint32_t mma_phase = 0, vph = 0;
   // rendezvous of the 256 epilogue threads after a vector staging (bounded)
@@ -353,7 +430,7 @@ __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, c
     return e.ok;
   };
   auto wait_mma = [&]() {
-    e.ok = e.ok && mbar_wait(b.mma, mma_phase, abort_flag);
+    e.ok = e.ok && cwait<G>(b.mma, mma_phase, abort_flag);
     mma_phase ^= 1;
     tc_fence_after();
     return e.ok;
@@ -413,13 +490,238 @@ __device__ void comp_epilogue(const CompParams& p, uint32_t tmem, uint32_t r1, c
   }
 }
 
-__global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant__ CompParams p) {
+// a0 += w * x0, a1 += w * x1 as one packed fp32x2 FMA, each lane rounded as fmaf: the
+// accumulation of tr_aggregate, so that the x rows built on chip equal its tokens bit for bit
+__device__ __forceinline__ void fma2_acc(float& a0, float& a1, float w, float x0, float x1) {
+  asm("{\n\t.reg .b64 a, x, w;\n\t"
+      "mov.b64 a, {%0, %1};\n\tmov.b64 x, {%3, %4};\n\tmov.b64 w, {%2, %2};\n\t"
+      "fma.rn.f32x2 a, w, x, a;\n\tmov.b64 {%0, %1}, a;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(w), "f"(x0), "f"(x1));
+}
+
+__device__ __forceinline__ uint4 ld_row16(const uint16_t* q) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(q));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_bf2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Gather warps of the gathering variant (TransRetrieval §3.2 feeding §3.3): the x row of a
+// candidate is its F field tokens side by side, token f = sum_i v_i h(k_i) / sum_i v_i over
+// the bag c*F + f.  Every 64-column slice of the tile in flight (field f, columns d0 .. d0+63
+// of its token) is built in one stage of the x ring: eight lanes per bag, each owning 8
+// columns (one 16-byte vector of every row), two bags per lane group at a time (a work item),
+// so a group has up to 16 rows in flight.  Keys and weights are taken 8 at a time, one per
+// lane, and broadcast by shuffle; rows are summed in bag order with fp32 FMAs and the weight
+// sum is reduced across the 8 lanes, exactly as tr_aggregate does, then the token is rounded
+// to bf16 and stored in the 128-byte-swizzled K-major layout the MMA reads.
+// Latency: the tile's bag headers (offsets, table ids) are read into shared memory once per
+// tile, and the next work item's first keys and weights are requested while the current
+// item's rows are in flight, so an item costs about one row round trip.  Lane 0 of the first
+// gather warp claims the tiles and publishes them to the other roles.
+__device__ void comp_gather(const CompParams& p, uint32_t xr, uint8_t* hdr, const CBars& b, volatile int* abort_flag) {
+  using L = CLayout<true>;
+  const GatherArgs& g = p.g;
+  constexpr int NGRP = 4 * kGatherWarps;   // lane groups
+  constexpr int NPAIR = kM / NGRP / 2;     // work items of a group per slice
+  const int lane = threadIdx.x & 31, gw = (threadIdx.x >> 5) - L::GW0;
+  const int cl = lane & 7, grp = gw * 4 + (lane >> 3);
+  const int gt = threadIdx.x - 32 * L::GW0;   // 0 .. 255
+  const int F = g.F, per_field = g.D / 64, nkc = p.c0 / 64;
+  const int nb = kM * F;                      // bags per tile
+  const int64_t* s_off = reinterpret_cast<const int64_t*>(hdr);
+  const int* s_tab = reinterpret_cast<const int*>(hdr + (L::HDR_TAB - L::HDR));
+  const bool claimer = gw == 0 && lane == 0;
+  bool ok = true, bad = false;
+  int ts = 0, sx = 0;
+  uint32_t tph = 0, phx = 0, gph = 0;
+  // bounded rendezvous of the gather warps
+  auto gsync = [&]() {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(b.gsync);
+    ok = ok && mbar_wait(b.gsync, gph, abort_flag);
+    gph ^= 1;
+    ok = __all_sync(0xffffffffu, ok);
+    return ok;
+  };
+  for (;;) {
+    if (claimer) {
+      ok = ok && mbar_wait(b.tile_empty[ts], tph ^ 1, abort_flag);
+      const int t = ok ? atomicAdd(p.claim, 1) : -1;
+      const int pub = t >= 0 && t < p.n_tiles ? t : -1;
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(b.tile_slot[ts]), "r"(pub) : "memory");
+      mbar_arrive(b.tile_full[ts]);
+    }
+    const int tile = next_tile(b, ts, tph, abort_flag, ok);
+    if (__any_sync(0xffffffffu, tile < 0)) break;
+    // the tile's headers, once every gather warp is done with the previous tile's
+    if (!gsync()) break;
+    const long long bag0 = (long long)tile * nb;
+    const int nb_here = (int)min((long long)nb, p.n * F - bag0);
+    for (int i = gt; i <= nb_here; i += 32 * kGatherWarps)
+      const_cast<int64_t*>(s_off)[i] = __ldg(g.offsets + bag0 + i);
+    for (int i = gt; i < nb_here; i += 32 * kGatherWarps) const_cast<int*>(s_tab)[i] = __ldg(g.bag_table + bag0 + i);
+    if (!gsync()) break;
+    // header of bag slot j (0, 1) of work item (kc, pr): whether the candidate exists, its
+    // table, first key and key count
+    auto header = [&](int kc, int pr, int j, int& t, int64_t& s0, int& n) {
+      const int r = grp + NGRP * (2 * pr + j);
+      const int lb = r * F + kc / per_field;
+      t = 0;
+      s0 = 0;
+      n = 0;
+      if (lb >= nb_here) return false;
+      t = s_tab[lb];
+      s0 = s_off[lb];
+      n = (int)(s_off[lb + 1] - s0);
+      return true;
+    };
+    // first key chunk of work item (kc, pr), one key and weight per lane (k = -1: none)
+    auto first_keys = [&](int kc, int pr, int (&k)[2], float (&v)[2]) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        int t, n;
+        int64_t s0;
+        const bool live = header(kc, pr, j, t, s0, n);
+        k[j] = -1;
+        v[j] = 0.f;
+        if (live && t >= 0 && t < g.n_tables && cl < n) {
+          k[j] = __ldg(g.keys + s0 + cl);
+          v[j] = __ldg(g.weights + s0 + cl);
+        }
+      }
+    };
+    int kn[2];
+    float vn[2];
+    first_keys(0, 0, kn, vn);
+    for (int kc = 0; kc < nkc; ++kc) {
+      const int d0 = (kc % per_field) * 64;
+      ok = ok && mbar_wait_idle(b.xempty[sx], phx ^ 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const uint32_t xs = xr + sx * L::XSTAGE;
+#pragma unroll 1
+      for (int pr = 0; pr < NPAIR; ++pr) {
+        // a bag naming no table gets no rows: its weight sum stays 0 and its token 0
+        int n[2], tb[2];
+        const uint16_t* tp[2];
+        int k[2] = {kn[0], kn[1]};
+        float v[2] = {vn[0], vn[1]};
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          int64_t s0;
+          const bool live = header(kc, pr, j, tb[j], s0, n[j]);
+          const bool badt = live && (tb[j] < 0 || tb[j] >= g.n_tables);
+          bad |= badt;
+          if (badt) n[j] = 0;
+          if (n[j] == 0) tb[j] = 0;
+          tp[j] = g.tab[tb[j]] + d0 + cl * 8;
+        }
+        const int n_max = __reduce_max_sync(0xffffffffu, max(n[0], n[1]));
+        float acc[2][8], ws[2] = {0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[j][e] = 0.f;
+        for (int base = 0; base < n_max; base += 8) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int cnt = n[j] - base;
+            if (base > 0) {   // chunks after the first (bags of more than 8 keys)
+              k[j] = -1;
+              v[j] = 0.f;
+              if (cl < cnt) {
+                int t;
+                int64_t s0;
+                int nn;
+                header(kc, pr, j, t, s0, nn);
+                k[j] = __ldg(g.keys + s0 + base + cl);
+                v[j] = __ldg(g.weights + s0 + base + cl);
+              }
+            }
+            if (cl >= cnt) {
+              k[j] = -1;
+              v[j] = 0.f;
+            } else if (k[j] < 0 || k[j] >= g.rows[tb[j]]) {
+              bad = true;
+              k[j] = -1;
+              v[j] = 0.f;
+            }
+            ws[j] += v[j];
+          }
+          const int cnt_max = min(n_max - base, 8);   // warp-uniform
+          // a row past the bag's end or with a rejected key has k = -1 and weight 0
+          uint4 raw[2][8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int kk = __shfl_sync(0xffffffffu, k[j], u, 8);
+              raw[j][u] = u < cnt_max && kk >= 0 ? ld_row16(tp[j] + (int64_t)kk * g.D) : make_uint4(0, 0, 0, 0);
+            }
+          if (base == 0) {   // the next work item's first keys, while these rows are in flight
+            const int nkc2 = pr + 1 < NPAIR ? kc : kc + 1, npr = pr + 1 < NPAIR ? pr + 1 : 0;
+            if (nkc2 < nkc) first_keys(nkc2, npr, kn, vn);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            if (u >= cnt_max) break;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const float w = __shfl_sync(0xffffffffu, v[j], u, 8);
+              const uint32_t q[4] = {raw[j][u].x, raw[j][u].y, raw[j][u].z, raw[j][u].w};
+#pragma unroll
+              for (int h = 0; h < 4; ++h)
+                fma2_acc(acc[j][2 * h], acc[j][2 * h + 1], w, __uint_as_float(q[h] << 16),
+                         __uint_as_float(q[h] & 0xFFFF0000u));
+            }
+          }
+        }
+        if (n_max == 0) {   // no rows anywhere in the warp: the next keys are still needed
+          const int nkc2 = pr + 1 < NPAIR ? kc : kc + 1, npr = pr + 1 < NPAIR ? pr + 1 : 0;
+          if (nkc2 < nkc) first_keys(nkc2, npr, kn, vn);
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+#pragma unroll
+          for (int off = 4; off > 0; off >>= 1) ws[j] += __shfl_xor_sync(0xffffffffu, ws[j], off);
+          const float inv = ws[j] != 0.f ? 1.f / ws[j] : 0.f;
+          float o[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[e] = acc[j][e] * inv;
+          const int r = grp + NGRP * (2 * pr + j);
+          st_shared_v4(xs + (r >> 3) * 1024 + (r & 7) * 128 + ((cl ^ (r & 7)) << 4), pack_bf2(o[0], o[1]),
+                       pack_bf2(o[2], o[3]), pack_bf2(o[4], o[5]), pack_bf2(o[6], o[7]));
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b.xfull[sx]);
+      if (++sx == L::NX) {
+        sx = 0;
+        phx ^= 1;
+      }
+    }
+    if (!ok) break;
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.status, STATUS_KEY_RANGE);
+}
+
+template <bool G>
+__device__ __forceinline__ void compress_body(const CompParams& p) {
+  using L = CLayout<G>;
   extern __shared__ uint8_t smem_raw[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw);
-  const uint32_t r1 = base + OFF_R1, r2 = base + OFF_R2, bar0 = base + OFF_BAR;
+  const uint32_t r1 = base, r2 = base + L::R2, bar0 = base + L::BAR;
   CBars b;
   for (int s = 0; s < 2; ++s) {
     b.full1[s] = bar0 + 8 * s;
@@ -438,8 +740,13 @@ __global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant_
     b.tile_empty[s] = bar0 + 168 + 8 * s;
     b.tile_slot[s] = bar0 + 184 + 4 * s;
   }
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + OFF_BAR + 128);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + OFF_BAR + 136);
+  for (int s = 0; s < 3; ++s) {
+    b.xfull[s] = bar0 + 192 + 8 * s;
+    b.xempty[s] = bar0 + 216 + 8 * s;
+  }
+  b.gsync = bar0 + 240;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::BAR + 128);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::BAR + 136);
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(b.full1[s], 1);
@@ -455,11 +762,18 @@ __global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant_
     mbar_init(b.vsync, 256);
     for (int s = 0; s < 2; ++s) {
       mbar_init(b.tile_full[s], 1);
-      mbar_init(b.tile_empty[s], 1 + 256);   // the MMA thread and every epilogue thread
+      // readers: the MMA thread and every epilogue thread; with gathering also the copy
+      // thread and every gather thread
+      mbar_init(b.tile_empty[s], G ? 2 + 256 + 32 * kGatherWarps : 1 + 256);
     }
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(b.xfull[s], kGatherWarps);
+      mbar_init(b.xempty[s], 1);
+    }
+    mbar_init(b.gsync, kGatherWarps);
     *abort_flag = 0;
     mbar_fence_init();
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.xmap)) : "memory");
+    if constexpr (!G) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&p.xmap)) : "memory");
     // the grid's weight slices (one contiguous image) into L2 at once
     prefetch_l2_share(p.w1, ((size_t)p.c0 * p.c1 + (size_t)p.c1 * p.c2 + (size_t)p.c2 * p.c3) * 2);
   }
@@ -471,13 +785,29 @@ __global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (warp == 0) {
-    if (lane == 0) comp_producer(p, r1, r2, b, abort_flag);
-  } else if (warp == 1) {
-    if (lane == 0) comp_mma(p, tmem, r1, r2, b, abort_flag);
+  float* svec = reinterpret_cast<float*>(gbase + L::VEC);
+  float* sb3 = reinterpret_cast<float*>(gbase + L::BAR + 256);
+  if constexpr (G) {
+    // each role runs inside its own register budget
+    if (warp < 4) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(CLayout<true>::CTL_REGS));
+      if (warp == 0 && lane == 0) comp_producer<true>(p, r1, r2, b, abort_flag);
+      if (warp == 1 && lane == 0) comp_mma<true>(p, tmem, r1, r2, b, abort_flag);
+    } else if (warp < CLayout<true>::GW0) {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(CLayout<true>::EPI_REGS));
+      comp_epilogue<true>(p, tmem, r1, b, svec, sb3, abort_flag);
+    } else {
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(CLayout<true>::GATHER_REGS));
+      comp_gather(p, r1 + L::XR, gbase + L::HDR, b, abort_flag);
+    }
   } else {
-    comp_epilogue(p, tmem, r1, b, reinterpret_cast<float*>(gbase + OFF_VEC), reinterpret_cast<float*>(gbase + OFF_B3),
-                  abort_flag);
+    if (warp == 0) {
+      if (lane == 0) comp_producer<false>(p, r1, r2, b, abort_flag);
+    } else if (warp == 1) {
+      if (lane == 0) comp_mma<false>(p, tmem, r1, r2, b, abort_flag);
+    } else {
+      comp_epilogue<false>(p, tmem, r1, b, svec, sb3, abort_flag);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -486,6 +816,14 @@ __global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant_
     tmem_dealloc(tmem, 512);
   }
   if (threadIdx.x == 0 && *abort_flag) atomicOr(p.status, STATUS_KERNEL_TIMEOUT);
+}
+
+__global__ void __launch_bounds__(320, 1) compress_kernel(const __grid_constant__ CompParams p) {
+  compress_body<false>(p);
+}
+
+__global__ void __launch_bounds__(640, 1) compress_gather_kernel(const __grid_constant__ CompParams p) {
+  compress_body<true>(p);
 }
 
 // W^T slice rows [0, N) x cols [k0, k0 + 64) of W [K][N] in the core-matrix layout, as bf16
@@ -581,23 +919,13 @@ tr_status tc_build_comp(tr_model* m, const tr_model_weights* w) {
   return TR_OK;
 }
 
-tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens, cudaStream_t st) {
+namespace {
+
+// Weight images, vectors, work counter and sizes of one launch (the x source aside).
+tr_status comp_params(const tr_model* m, int64_t n, void* tokens, cudaStream_t st, CompParams& p, int& sms) {
   const int* c = m->desc.comp_dims;
-  if ((uintptr_t)x % 16 || (uintptr_t)tokens % 16) return fail(TR_ERR_INVALID_ARG, "x/tokens not 16-byte aligned");
-  auto encode = get_encode();
-  if (!encode) return fail(TR_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   DeviceState* ds = nullptr;
   TR_TRY(device_state(&ds));
-  CompParams p;
-  memset(&p, 0, sizeof p);
-  cuuint64_t gdim[2] = {(cuuint64_t)c[0], (cuuint64_t)n};
-  cuuint64_t gstride[1] = {(cuuint64_t)c[0] * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estride[2] = {1, 1};
-  CUresult r = encode(&p.xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box, estride,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(TR_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   const uint8_t* img = static_cast<const uint8_t*>(m->tc_comp);
   p.w1 = img;
   p.w2 = img + (size_t)c[0] * c[1] * 2;
@@ -613,13 +941,73 @@ tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens,
   p.c1 = c[1];
   p.c2 = c[2];
   p.c3 = c[3];
-  int dev = 0, sms = 148;
+  int dev = 0;
+  sms = 148;
   TR_CUDA_TRY(cudaGetDevice(&dev));
   TR_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  TR_TRY(ensure_smem_attr((const void*)compress_kernel, SMEM_BYTES));
-  compress_kernel<<<std::min(p.n_tiles, sms), 320, SMEM_BYTES, st>>>(p);
-  TR_LAUNCH_CHECK("compress_kernel");
   return TR_OK;
+}
+
+template <bool G>
+tr_status comp_launch(const CompParams& p, int sms, cudaStream_t st) {
+  const void* k = G ? (const void*)compress_gather_kernel : (const void*)compress_kernel;
+  TR_TRY(ensure_smem_attr(k, smem_bytes<G>()));
+  if (G)
+    compress_gather_kernel<<<std::min(p.n_tiles, sms), CLayout<G>::THREADS, smem_bytes<G>(), st>>>(p);
+  else
+    compress_kernel<<<std::min(p.n_tiles, sms), CLayout<G>::THREADS, smem_bytes<G>(), st>>>(p);
+  TR_LAUNCH_CHECK(G ? "compress_gather_kernel" : "compress_kernel");
+  return TR_OK;
+}
+
+}  // namespace
+
+tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens, cudaStream_t st) {
+  const int* c = m->desc.comp_dims;
+  if ((uintptr_t)x % 16 || (uintptr_t)tokens % 16) return fail(TR_ERR_INVALID_ARG, "x/tokens not 16-byte aligned");
+  auto encode = get_encode();
+  if (!encode) return fail(TR_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  CompParams p;
+  memset(&p, 0, sizeof p);
+  cuuint64_t gdim[2] = {(cuuint64_t)c[0], (cuuint64_t)n};
+  cuuint64_t gstride[1] = {(cuuint64_t)c[0] * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = encode(&p.xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), gdim, gstride, box, estride,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TR_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  int sms = 148;
+  TR_TRY(comp_params(m, n, tokens, st, p, sms));
+  return comp_launch<false>(p, sms, st);
+}
+
+bool tc_comp_bags_supported(const tr_model* m) {
+  const int D = m->desc.D;
+  return tc_comp_supported(m) && D % 64 == 0 && m->desc.n_target_fields <= kMaxGatherFields &&
+         m->desc.comp_dims[0] == m->desc.n_target_fields * D;
+}
+
+tr_status tc_compress_bags(const tr_model* m, const tr_table* tables, int n_tables, const int32_t* bag_table,
+                           const int64_t* offsets, const int32_t* keys, const float* weights, int64_t n,
+                           void* tokens, cudaStream_t st) {
+  if ((uintptr_t)tokens % 16) return fail(TR_ERR_INVALID_ARG, "tokens not 16-byte aligned");
+  CompParams p;
+  memset(&p, 0, sizeof p);
+  for (int i = 0; i < n_tables; ++i) {
+    p.g.tab[i] = static_cast<const uint16_t*>(tables[i].data);
+    p.g.rows[i] = (int)std::min<int64_t>(tables[i].n_rows, INT32_MAX);
+  }
+  p.g.bag_table = bag_table;
+  p.g.offsets = offsets;
+  p.g.keys = keys;
+  p.g.weights = weights;
+  p.g.n_tables = n_tables;
+  p.g.F = m->desc.n_target_fields;
+  p.g.D = m->desc.D;
+  int sms = 148;
+  TR_TRY(comp_params(m, n, tokens, st, p, sms));
+  return comp_launch<true>(p, sms, st);
 }
 
 }  // namespace tr
