@@ -763,9 +763,12 @@ def run_bulk(args):
 
 def run_uncompressed(args):
     """The cost target compression removes (§3.3): --case-n candidates of one 128D-5L request
-    scored as L_t = 8 uncompressed field tokens and as one compressed token, both on the
-    CUDA-core path (the only path that takes L_t > 1), plus the tensor-core single-token path
-    for reference; prints one JSON line with the times and the FLOP ratio."""
+    scored as L_t = 8 uncompressed field tokens and as one compressed token, on the
+    tensor-core stack kernel (the serving kernel) and, for reference, on the CUDA-core
+    kernels (a second model handle made with TR_FORCE_SIMT=1); prints one JSON line with the
+    device times (CUDA events) and the FLOP ratio."""
+    import os
+
     import torch
 
     from transformer_candidate_scoring_b200 import api
@@ -780,8 +783,13 @@ def run_uncompressed(args):
     X = dw.X.view(n, F, D)
     s = torch.empty(n, dtype=torch.float32, device="cuda")
     args_kv = (dw.req_offsets, dw.kv, dw.L_u, dw.domain, s)
+    os.environ["TR_FORCE_SIMT"] = "1"
+    try:
+        simt_model = api.Model(dims, dw.params)
+    finally:
+        del os.environ["TR_FORCE_SIMT"]
 
-    def timed(fn, reps=3):
+    def timed(fn, reps=5):
         fn()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -791,16 +799,23 @@ def run_uncompressed(args):
         e1.record()
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / reps
-    t8 = timed(lambda: api.score_candidates_uncompressed(dw.model, X, F, *args_kv))
-    t1 = timed(lambda: api.score_candidates_uncompressed(dw.model, dw.tokens, 1, *args_kv))
-    ttc = timed(lambda: api.score_candidates(dw.model, dw.tokens, *args_kv))
+    tc8 = timed(lambda: api.score_candidates_uncompressed(dw.model, X, F, *args_kv))
+    tc1 = timed(lambda: api.score_candidates(dw.model, dw.tokens, *args_kv))
+    cc8 = timed(lambda: api.score_candidates_uncompressed(simt_model, X, F, *args_kv), reps=2)
+    cc1 = timed(lambda: api.score_candidates_uncompressed(simt_model, dw.tokens, 1, *args_kv), reps=2)
+    if api.sync_status() != 0:
+        raise RuntimeError("device status word set")
     L_u = dw.L_u[0]
     f8 = dims.n_layer * (16 * F * D * D + 4 * F * (L_u + F) * D) + 2 * D * F
     f1 = stack_flops_per_candidate(dims, L_u)
     print(json.dumps({"case": "uncompressed_targets", "candidates": n, "L_t": F, "L_u": L_u,
-                      "ms_L_t_8_cuda_cores": t8, "ms_L_t_1_cuda_cores": t1, "ms_L_t_1_tensor_cores": ttc,
-                      "time_saving_cuda_cores": 1 - t1 / t8, "flops_per_candidate_L_t_8": f8,
-                      "flops_per_candidate_L_t_1": f1, "flop_saving": 1 - f1 / f8}), flush=True)
+                      "ms_L_t_8_tensor_cores": tc8, "ms_L_t_1_tensor_cores": tc1,
+                      "time_saving_tensor_cores": 1 - tc1 / tc8,
+                      "ms_L_t_8_cuda_cores": cc8, "ms_L_t_1_cuda_cores": cc1,
+                      "time_saving_cuda_cores": 1 - cc1 / cc8,
+                      "tflops_L_t_8_tensor_cores": f8 * n / tc8 / 1e9,
+                      "flops_per_candidate_L_t_8": f8, "flops_per_candidate_L_t_1": f1,
+                      "flop_saving": 1 - f1 / f8}), flush=True)
 
 
 def run_fused(args):

@@ -264,8 +264,12 @@ tr_status tr_score_candidates(const tr_model* m, const void* tokens, int64_t n,
  * layer stack, attending to its request's L_u cached user keys/values and to the keys/values
  * of its own candidate's L_t tokens (never another candidate's); the candidate's score is the
  * mean over its tokens of w_head . LayerNorm_f(y_t) + b_head.  With L_t = 1 this is
- * tr_score_candidates.  It runs on the CUDA-core path (fp32 arithmetic, any model dtype): it
- * exists to measure the per-candidate cost that target compression removes, not for serving.
+ * tr_score_candidates.  It exists to measure the per-candidate cost that target compression
+ * removes.  A TR_BF16 model on the tensor-core stack with L_t a power of two up to 16 (and
+ * every L_u <= 128) runs it in the same kernel as tr_score_candidates, a candidate's tokens
+ * being L_t consecutive rows of a tile whose own-candidate attention runs on CUDA cores
+ * (and with L_t = 1 its scores equal tr_score_candidates' on the same token values bit for
+ * bit); any other case runs the CUDA-core kernels (fp32 arithmetic).
  *   tokens      DEVICE [n][L_t][D] of the model dtype (candidate c's tokens are rows c*L_t ..)
  *   L_t         1 .. TR_MAX_LT
  *   req_offsets, kv, L_u, domain, R, scores: as tr_score_candidates (n counts candidates).

@@ -701,11 +701,19 @@ def test_captured_step_replays_bit_identical():
     ("tiny", "wide", 4, [8, 3], [37, 20]),
     ("tiny", "paper", 8, [8], [50]),
     ("64d3l", "wide", 8, [32, 0], [40, 9]),
+    ("64d3l", "paper", 4, [32, 5], [70, 9]),
     ("128d5l", "wide", 8, [64], [60]),
+    ("128d5l", "paper", 8, [64, 17], [60, 33]),     # two requests, ragged last tiles
+    ("128d5l", "wide", 8, [0, 64], [20, 30]),       # a request without user keys
+    ("128d5l", "wide", 2, [64], [100]),
+    ("128d5l", "paper", 16, [32], [20]),
+    ("128d5l", "wide", 3, [64], [30]),              # not a power of two: CUDA-core kernels
 ])
 def test_uncompressed_targets_parity(name, init, L_t, L_us, n_per):
     """Candidates of L_t target tokens (the variant target compression replaces) against the
-    oracle, packed requests included."""
+    oracle, packed requests included.  bf16 models with L_t a power of two up to 16 run the
+    tensor-core stack (own-candidate attention by warp shuffles), the rest the CUDA-core
+    kernels."""
     dims, P, m, users, _, doms, kvs = _score_setup(name, init, L_us, n_per)
     std = 0.5 if init == "wide" else 0.3
     toks = [datagen.rand_matrix(300 + r, (n, L_t, dims.D), std, dims.dtype) for r, n in enumerate(n_per)]
@@ -720,6 +728,20 @@ def test_uncompressed_targets_parity(name, init, L_t, L_us, n_per):
         K, V = oracle.prefill_user(P, dims.n_head, U, d)
         ref = oracle.score_candidates_uncompressed(P, dims.n_head, t, K, V, d)
         check_close(got[off[r]:off[r + 1]], ref, dims.dtype, f"request {r}")
+
+
+def test_uncompressed_with_one_token_equals_single_token_path_tensor_cores():
+    """L_t = 1 on the bf16 model: the tensor-core variant with bf16 tokens equals
+    tr_score_candidates on the same values in fp32 bit for bit (one own key, numerator sum 1,
+    the mean value is the own value)."""
+    dims, P, m, users, toks, doms, kvs = _score_setup("128d5l", "wide", [64, 20], [300, 45])
+    a, off = _gpu_scores(m, dims, toks, kvs, [64, 20], doms)
+    T = dev(np.concatenate(toks), torch.bfloat16)
+    assert torch.equal(T.float().cpu(), torch.from_numpy(np.concatenate(toks)).float())
+    s = torch.empty(int(off[-1]), dtype=torch.float32, device="cuda")
+    tr().api.score_candidates_uncompressed(m, T, 1, off.tolist(), kvs, [64, 20], doms, s)
+    torch.cuda.synchronize()
+    assert np.array_equal(s.cpu().numpy().astype(np.float64), a)
 
 
 def test_uncompressed_with_one_token_equals_single_token_path_fp32():

@@ -145,6 +145,10 @@ tr_status tc_score(const tr_model* m, const void* tokens, int64_t n, const int64
 bool tc_comp_supported(const tr_model* m);
 tr_status tc_compress(const tr_model* m, const void* x, int64_t n, void* tokens, cudaStream_t st);
 bool tc_comp_bags_supported(const tr_model* m);
+bool tc_score_lt_supported(const tr_model* m, int L_t, const int32_t* L_u, int R);
+tr_status tc_score_lt(const tr_model* m, const void* tokens, int L_t, const int64_t* req_offsets,
+                      const void* const* kv, const int32_t* L_u, const int32_t* domain, int R, float* scores,
+                      cudaStream_t st);
 tr_status tc_compress_bags(const tr_model* m, const tr_table* tables, int n_tables, const int32_t* bag_table,
                            const int64_t* offsets, const int32_t* keys, const float* weights, int64_t n,
                            void* tokens, cudaStream_t st);
@@ -432,6 +436,7 @@ tr_status tr_score_candidates_uncompressed(const tr_model* m, const void* tokens
   if (n == 0) return TR_OK;
   if (!tokens || !scores) return fail(TR_ERR_INVALID_ARG, "null device pointer");
   const cudaStream_t st = (cudaStream_t)stream;
+  if (tc_score_lt_supported(m, L_t, L_u, R)) return tc_score_lt(m, tokens, L_t, req_offsets, kv, L_u, domain, R, scores, st);
   for (int r = 0; r < R; ++r)
     TR_TRY(simt_score_lt(m, tokens, m->desc.dtype == TR_F32, req_offsets[r], req_offsets[r + 1], L_t, kv[r], L_u[r],
                          domain[r], scores, st));

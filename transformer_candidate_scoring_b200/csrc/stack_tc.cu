@@ -156,6 +156,8 @@ struct ReqInfo {
 
 struct StackParams {
   const float* tokens;        // score mode: fp32 candidate tokens [n][D]
+  const uint16_t* tokens_h;   // candidates of lt tokens: bf16 tokens [n * lt][D]
+  int lt;                     // tokens per candidate (1: one compressed token each)
   float* scores;
   const uint8_t* wimg;        // [n_layer][kItems][kItemBytes]
   const float* vec;           // [n_layer][4 D] + [D + 4]
@@ -829,7 +831,7 @@ __device__ __forceinline__ void finish_head(const Epi& e, uint32_t hb, int hw, i
   st_row8h(e.sA + (2 * h + 1) * 2048 + e.rowoff, o + 8);
 }
 
-template <int D, int SW, bool UM>
+template <int D, int SW, bool UM, bool OG>
 __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Epi& e) {
   constexpr int P = Par<D>::P;
   constexpr int NH = Cfg<D>::kNH;
@@ -842,16 +844,32 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
   {
     float y[DP];
     const float4* sd4 = reinterpret_cast<const float4*>(p.domain_emb + (size_t)t.dom * D + part * DP);
-    const float4* src = reinterpret_cast<const float4*>(
-        (UM ? p.req[t.r].utokens + (size_t)m * D : p.tokens + (size_t)(t.row0 + m) * D) + part * DP);
+    if constexpr (OG) {   // bf16 tokens, widened exactly
+      const uint4* src = reinterpret_cast<const uint4*>(p.tokens_h + (size_t)(t.row0 + m) * D + part * DP);
 #pragma unroll
-    for (int c = 0; c < DP / 4; ++c) {
-      const float4 u = live ? __ldg(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 d = __ldg(sd4 + c);
-      y[4 * c] = live ? u.x + d.x : 0.f;
-      y[4 * c + 1] = live ? u.y + d.y : 0.f;
-      y[4 * c + 2] = live ? u.z + d.z : 0.f;
-      y[4 * c + 3] = live ? u.w + d.w : 0.f;
+      for (int c = 0; c < DP / 8; ++c) {
+        const uint4 u = live ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        const float4 d0 = __ldg(sd4 + 2 * c), d1 = __ldg(sd4 + 2 * c + 1);
+        const float d[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          y[8 * c + 2 * i] = live ? __uint_as_float(w[i] << 16) + d[2 * i] : 0.f;
+          y[8 * c + 2 * i + 1] = live ? __uint_as_float(w[i] & 0xFFFF0000u) + d[2 * i + 1] : 0.f;
+        }
+      }
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(
+          (UM ? p.req[t.r].utokens + (size_t)m * D : p.tokens + (size_t)(t.row0 + m) * D) + part * DP);
+#pragma unroll
+      for (int c = 0; c < DP / 4; ++c) {
+        const float4 u = live ? __ldg(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 d = __ldg(sd4 + c);
+        y[4 * c] = live ? u.x + d.x : 0.f;
+        y[4 * c + 1] = live ? u.y + d.y : 0.f;
+        y[4 * c + 2] = live ? u.z + d.z : 0.f;
+        y[4 * c + 3] = live ? u.w + d.w : 0.f;
+      }
     }
 #pragma unroll
     for (int c = 0; c < DP / 16; ++c) tmem_st16(e.tY + part * DP + 16 * c, y + 16 * c);
@@ -923,6 +941,7 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
     // ---- Q of this part's heads (pre-scaled by 1/sqrt(d_h) through its weights) -> A; own
     // score per head
     float sself[NP];
+    float rsc[OG ? NP : 1];   // OG: the own tokens' numerator sum relative to their maximum
     if (!e.wait()) return;
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
@@ -936,6 +955,43 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
       for (int i = 0; i < 8; ++i) qp[i] = pack_h2(q[2 * i], q[2 * i + 1]);
       if constexpr (UM) {
         sself[k] = -INFINITY;
+      } else if constexpr (OG) {
+        // the own candidate's lt tokens sit in lanes g0 .. g0 + lt - 1: their keys and values
+        // come by shuffle; an online softmax over them leaves their largest score (which
+        // joins the user keys' maximum), the sum R of their numerators relative to it, and
+        // their numerator-weighted mean value, which replaces the own value: the attention
+        // output is then (ps R vmean + P V) / (sum + ps R), ps the numerator of the largest
+        const int g0 = (m & 31) & ~(p.lt - 1);
+        float mo = -INFINITY, R = 0.f, va[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) va[i] = 0.f;
+#pragma unroll 1
+        for (int j = 0; j < p.lt; ++j) {
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) fma_h2(s0, s1, qp[i], __shfl_sync(0xffffffffu, kreg[8 * k + i], g0 + j));
+          const float sj = s0 + s1;
+          if (sj > mo) {
+            const float c = ex2((mo - sj) * kL2E);
+            R *= c;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) va[i] *= c;
+            mo = sj;
+          }
+          const float rj = ex2((sj - mo) * kL2E);
+          R += rj;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t vv = __shfl_sync(0xffffffffu, vreg[8 * k + i], g0 + j);
+            va[2 * i] = fmaf(rj, h_lo(vv), va[2 * i]);
+            va[2 * i + 1] = fmaf(rj, h_hi(vv), va[2 * i + 1]);
+          }
+        }
+        sself[k] = mo;
+        rsc[k] = R;
+        const float ri = 1.f / R;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) vreg[8 * k + i] = pack_h2(va[2 * i] * ri, va[2 * i + 1] * ri);
       } else {
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
@@ -973,6 +1029,13 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
             s1 = 2 * g == k ? sself[k + 1] : s1;
           }
           softmax_two<SW>(e.tW, t.Lp, t.L_u, s0, s1, ps);
+          if constexpr (OG) {
+#pragma unroll
+            for (int k = 0; k < NP; k += 2) {
+              ps[0] = 2 * g == k ? ps[0] * rsc[k] : ps[0];
+              ps[1] = 2 * g == k ? ps[1] * rsc[k + 1] : ps[1];
+            }
+          }
           e.signal();
           if (!e.wait()) return;   // P V and the row sums of group g
 #pragma unroll
@@ -988,6 +1051,12 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
           for (int j = 1; j < NP; ++j) ss = k == j ? sself[j] : ss;
           float ps = 0.f, rowsum = 0.f;
           if (mine) ps = softmax_head<SW, P == 2>(hb, t.Lp, t.L_u, ss, &rowsum);
+          if constexpr (OG) {
+            float rs = rsc[0];
+#pragma unroll
+            for (int j = 1; j < NP; ++j) rs = k == j ? rsc[j] : rs;
+            ps *= rs;
+          }
           e.signal();
           if (!e.wait()) return;   // P V and the row sums of group g
           if (mine) finish_head<D, UM>(e, hb, HW, h, k, ps, vreg, rowsum);
@@ -1034,10 +1103,18 @@ __device__ __forceinline__ void epi_tile(const StackParams& p, const Tile& t, Ep
     const float other = e.xchg(make_float2(mine, 0.f)).x;
     dot = part == 0 ? mine + other : other + mine;
   }
-  if (live && part == 0) p.scores[t.row0 + m] = dot + e.vec[D];
+  if constexpr (OG) {
+    // the candidate's score: the mean of its lt tokens' scores, summed over its lanes in a
+    // fixed butterfly order (lt is a power of two)
+    float sc = dot + e.vec[D];
+    for (int off = 1; off < p.lt; off <<= 1) sc += __shfl_xor_sync(0xffffffffu, sc, off);
+    if (live && part == 0 && (m & (p.lt - 1)) == 0) p.scores[(t.row0 + m) / p.lt] = sc * (1.f / p.lt);
+  } else {
+    if (live && part == 0) p.scores[t.row0 + m] = dot + e.vec[D];
+  }
 }
 
-template <int D, int SW, bool UM>
+template <int D, int SW, bool UM, bool OG>
 __device__ void epilogue(const StackParams& p, int slot, uint32_t tmem, uint32_t sA, uint32_t sKV, uint32_t sOnes,
                          const float* vec, const Bars& b, uint32_t xbuf, volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1066,11 +1143,13 @@ __device__ void epilogue(const StackParams& p, int slot, uint32_t tmem, uint32_t
   for (int u = blockIdx.x; u < p.n_units && e.ok; u += gridDim.x) {
     const Tile t = tile_of<D>(p, u, slot);
     e.paired = p.pair && tile_of<D>(p, u, 1).active;
-    if (t.active) epi_tile<D, SW, UM>(p, t, e);
+    if (t.active) epi_tile<D, SW, UM, OG>(p, t, e);
   }
 }
 
-template <int D, int SW, bool UM>
+// OG: candidates of p.lt tokens each (lt consecutive rows of a tile, adjacent lanes of one
+// warp), every token attending to its own candidate's tokens as well as to the user.
+template <int D, int SW, bool UM, bool OG>
 __global__ void __launch_bounds__(Par<D>::kThreads, 1) stack_kernel(const __grid_constant__ StackParams p) {
   constexpr int kSlotThreads = Par<D>::kSlotThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -1147,7 +1226,7 @@ __global__ void __launch_bounds__(Par<D>::kThreads, 1) stack_kernel(const __grid
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Par<D>::kEpiRegs));
     const int slot = (warp - 4) / (4 * Par<D>::P);
     if (slot == 0 || p.pair)
-      epilogue<D, SW, UM>(p, slot, tmem, sA0 + slot * kM * D * 2, sKV, sOnes, vec, b,
+      epilogue<D, SW, UM, OG>(p, slot, tmem, sA0 + slot * kM * D * 2, sKV, sOnes, vec, b,
                           base + p.off_xch + slot * kXchBytes, abort_flag);
   }
   tc_fence_before();
@@ -1366,22 +1445,33 @@ bool plan_smem(StackParams& p, int n_layer, int lp_max, bool pair, int& smem_byt
   return smem_bytes <= kSmemLimit;
 }
 
-template <int D, int SW, bool UM>
+template <int D, int SW, bool UM, bool OG = false>
 tr_status launch(int grid, const StackParams& p, int smem, cudaStream_t st) {
-  auto k = stack_kernel<D, SW, UM>;
+  auto k = stack_kernel<D, SW, UM, OG>;
   TR_TRY(ensure_smem_attr((const void*)k, kSmemLimit));
   k<<<grid, Par<D>::kThreads, smem, st>>>(p);
   TR_LAUNCH_CHECK(UM ? "stack_kernel (user side)" : "stack_kernel");
   return TR_OK;
 }
 
+// lt = 0: one fp32 token per candidate; lt >= 1: lt bf16 tokens per candidate (the tile
+// rows are then tokens, lt to a candidate).
 template <int D>
 tr_status score_launch(const tr_model* m, const void* tokens, const int64_t* req_offsets, const void* const* kv,
-                       const int32_t* L_u, const int32_t* domain, int R, float* scores, cudaStream_t st) {
+                       const int32_t* L_u, const int32_t* domain, int R, float* scores, cudaStream_t st,
+                       int lt = 0) {
   DeviceState* ds = nullptr;
   TR_TRY(device_state(&ds));
   StackParams p{};
-  p.tokens = static_cast<const float*>(tokens);
+  const bool og = lt > 0;
+  const int rows_per = og ? lt : 1;
+  if (og) {
+    p.tokens_h = static_cast<const uint16_t*>(tokens);
+    p.lt = lt;
+  } else {
+    p.tokens = static_cast<const float*>(tokens);
+    p.lt = 1;
+  }
   p.scores = scores;
   p.wimg = static_cast<const uint8_t*>(m->tc_stack);
   p.vec = m->tc_vec;
@@ -1403,12 +1493,12 @@ tr_status score_launch(const tr_model* m, const void* tokens, const int64_t* req
     const int64_t nr = req_offsets[r + 1] - req_offsets[r];
     if (nr == 0) continue;
     p.req[k].kv = static_cast<const uint8_t*>(kv[r]);
-    p.req[k].cand_off = req_offsets[r];
-    p.req[k].n = nr;
+    p.req[k].cand_off = req_offsets[r] * rows_per;
+    p.req[k].n = nr * rows_per;
     p.req[k].L_u = L_u[r];
     p.req[k].domain = domain[r];
     lp_max = std::max(lp_max, round_up16(L_u[r]));
-    tiles_of[k] = (int)((nr + kM - 1) / kM);
+    tiles_of[k] = (int)((nr * rows_per + kM - 1) / kM);
     pairs_of[k] = tiles_of[k] / 2;
     units += tiles_of[k] - pairs_of[k];
     ++k;
@@ -1440,6 +1530,10 @@ tr_status score_launch(const tr_model* m, const void* tokens, const int64_t* req
   if (!plan_smem<D>(p, p.n_layer, sw, true, smem))
     return fail(TR_ERR_UNSUPPORTED, "stack kernel: %d layers do not fit shared memory", p.n_layer);
   const int grid = std::min(units, sms);
+  if (og)
+    return sw == 32 ? launch<D, 32, false, true>(grid, p, smem, st)
+         : sw == 64 ? launch<D, 64, false, true>(grid, p, smem, st)
+                    : launch<D, kMaxLp, false, true>(grid, p, smem, st);
   return sw == 32 ? launch<D, 32, false>(grid, p, smem, st)
        : sw == 64 ? launch<D, 64, false>(grid, p, smem, st)
                   : launch<D, kMaxLp, false>(grid, p, smem, st);
@@ -1463,6 +1557,28 @@ tr_status tc_score(const tr_model* m, const void* tokens, int64_t n, const int64
       return fail(TR_ERR_INVALID_ARG, "kv[%d] is not 16-byte aligned", r);
   return m->desc.D == 128 ? score_launch<128>(m, tokens, req_offsets, kv, L_u, domain, R, scores, st)
                           : score_launch<64>(m, tokens, req_offsets, kv, L_u, domain, R, scores, st);
+}
+
+// Candidates of L_t bf16 tokens (the uncompressed-target variant): whether the tensor-core
+// stack takes them (L_t a power of two up to 16, so that a candidate's tokens are adjacent
+// lanes of one warp, and every request's L_u within the kernel's reach).
+bool tc_score_lt_supported(const tr_model* m, int L_t, const int32_t* L_u, int R) {
+  if (!(m->desc.dtype == TR_BF16 && tc_stack_supported(m) && L_t >= 1 && L_t <= 16 && (L_t & (L_t - 1)) == 0))
+    return false;
+  for (int r = 0; r < R; ++r)
+    if (L_u[r] > kMaxLp) return false;
+  return true;
+}
+
+tr_status tc_score_lt(const tr_model* m, const void* tokens, int L_t, const int64_t* req_offsets,
+                      const void* const* kv, const int32_t* L_u, const int32_t* domain, int R, float* scores,
+                      cudaStream_t st) {
+  if ((uintptr_t)tokens % 16) return fail(TR_ERR_INVALID_ARG, "tokens not 16-byte aligned");
+  for (int r = 0; r < R; ++r)
+    if ((uintptr_t)kv[r] % 16 && L_u[r] > 0 && req_offsets[r + 1] > req_offsets[r])
+      return fail(TR_ERR_INVALID_ARG, "kv[%d] is not 16-byte aligned", r);
+  return m->desc.D == 128 ? score_launch<128>(m, tokens, req_offsets, kv, L_u, domain, R, scores, st, L_t)
+                          : score_launch<64>(m, tokens, req_offsets, kv, L_u, domain, R, scores, st, L_t);
 }
 
 bool tc_prefill_supported(const tr_model* m, int L_u) { return tc_stack_supported(m) && L_u <= kMaxLp; }
