@@ -204,7 +204,7 @@ class _Slot:
         s.launch([f"{self.name}.user_tokens"], [f"{self.name}.kv"], f"{self.name} prefill")
 
     def target_aggregate(self, s):
-        s.launch(self._bags([self.tb]), [f"{self.name}.X"], f"{self.name} target_aggregate")
+        s.launch(self._bags([self.tb]), [getattr(self, "xname", f"{self.name}.X")], f"{self.name} target_aggregate")
 
     def compress(self, s):
         s.launch([f"{self.name}.X"], [f"{self.name}.tokens"], f"{self.name} compress")
@@ -462,12 +462,51 @@ def test_stream_plan_packed_batches_and_steady_state():
         assert sum(1 for j in range(20) for e in bounds if a < j * 40000 + e <= b) == 148
 
 
-def _stream_slot(cuda, name, n_cand):
+class _RingView:
+    def __init__(self, names):
+        self.names = names
+        self.name = "+".join(names)
+
+
+class _Ring(_Buf):
+    """A ring of m slots of n rows: a row range names the slots it touches (ring.X#k), so
+    that the race check sees which batches a launch reads or writes."""
+
+    def __init__(self, cuda, name, n, m):
+        super().__init__(cuda, name)
+        self.rows, self.m = n, m
+
+    def slot(self, k):
+        return _Buf(self.cuda, f"{self.name}#{k % self.m}")
+
+    def __getitem__(self, sl):
+        a, b = sl.start, sl.stop
+        return _RingView([f"{self.name}#{k % self.m}" for k in range(a // self.rows, (b - 1) // self.rows + 1)])
+
+
+def _names(x):
+    return list(getattr(x, "names", [x.name]))
+
+
+def _stream_slot(cuda, name, n_cand, k=None, ring=None):
     s = _Slot(cuda, name, n_cand)
     s.L_u, s.domain = [64], [1]
     s.kv = [_Buf(cuda, f"{name}.kv")]
     s.model = "model"
+    if ring is not None:   # a Streamed slot: its X, tokens and scores are rows of the rings
+        s.xname = ring[0].slot(k).name
+        s.scores = ring[2].slot(k)
     return s
+
+
+def _streamed(pipeline, cuda, n_cand, n_slots):
+    st = object.__new__(pipeline.Streamed)
+    st.n = n_cand
+    st.X, st.tokens, st.scores = (_Ring(cuda, "ring.X", n_cand, n_slots), _Ring(cuda, "ring.tokens", n_cand, n_slots),
+                                  _Ring(cuda, "ring.scores", n_cand, n_slots))
+    st.slots = [_stream_slot(cuda, f"slot{k}", n_cand, k, (st.X, st.tokens, st.scores)) for k in range(n_slots)]
+    st.user = cuda.Stream()
+    return st
 
 
 class _FakeApi:
@@ -475,10 +514,10 @@ class _FakeApi:
         self.cuda = cuda
 
     def compress_targets(self, model, x, tokens, stream=None):
-        stream.launch([x.name], [tokens.name], f"compress {x.name}")
+        stream.launch(_names(x), _names(tokens), f"compress {_names(x)}")
 
     def score_candidates(self, model, tokens, off, kv, lu, dm, scores, stream=None):
-        stream.launch([tokens.name] + [k.name for k in kv], [scores.name], f"score {[k.name for k in kv]}")
+        stream.launch(_names(tokens) + [k.name for k in kv], _names(scores), f"score {[k.name for k in kv]}")
 
     def kernel_launches(self):
         return 0
@@ -490,15 +529,10 @@ def test_streamed_steps_have_no_stream_races(fake_cuda, monkeypatch, n_cand, cou
     from transformer_candidate_scoring_b200.pipeline import unit_bounds
     pipeline, fake, log = fake_cuda
     monkeypatch.setattr(pipeline, "api", _FakeApi(fake.cuda))
-    st = object.__new__(pipeline.Streamed)
-    st.slots = [_stream_slot(fake.cuda, f"slot{k}", n_cand) for k in range(n_slots)]
-    st.n = n_cand
-    st.X, st.tokens, st.scores = (_Buf(fake.cuda, "ring.X"), _Buf(fake.cuda, "ring.tokens"),
-                                  _Buf(fake.cuda, "ring.scores"))
+    st = _streamed(pipeline, fake.cuda, n_cand, n_slots)
     st.comp_chunk, st.score_units, st.bounds = 294 * 128 if n_cand > 1000 else 500, 148 if n_cand > 1000 else 2, \
         unit_bounds([0, n_cand])
     st.group = group
-    st.user = fake.cuda.Stream()
     resident = [(_Bags(fake.cuda, f"set{k}.user"), _Bags(fake.cuda, f"set{k}")) for k in range(3)]
     done = []
 
@@ -521,14 +555,9 @@ def test_host_feed_streamed_has_no_stream_races(fake_cuda, monkeypatch, n_bag_sl
     from transformer_candidate_scoring_b200.pipeline import unit_bounds
     pipeline, fake, log = fake_cuda
     monkeypatch.setattr(pipeline, "api", _FakeApi(fake.cuda))
-    st = object.__new__(pipeline.Streamed)
-    st.slots = [_stream_slot(fake.cuda, f"slot{k}", 40000) for k in range(4)]
-    st.n = 40000
-    st.X, st.tokens, st.scores = (_Buf(fake.cuda, "ring.X"), _Buf(fake.cuda, "ring.tokens"),
-                                  _Buf(fake.cuda, "ring.scores"))
+    st = _streamed(pipeline, fake.cuda, 40000, 4)
     st.comp_chunk, st.score_units, st.bounds = 294 * 128, 148, unit_bounds([0, 40000])
     st.group = 2
-    st.user = fake.cuda.Stream()
     batches = [(_Bags(fake.cuda, f"host{k}.user"), _Bags(fake.cuda, f"host{k}.target"), None) for k in range(3)]
     feed = pipeline.HostFeed(st.slots[0], batches, n_bag_slots=n_bag_slots)
     host_scores = [_Buf(fake.cuda, f"host_scores{k}") for k in range(2)]
