@@ -93,3 +93,42 @@ def test_fused_target_side_refuses_unsupported_models():
     out = torch.empty(1, dims.D, dtype=torch.float32, device="cuda")
     with pytest.raises(Exception):
         tr().compress_target_bags(m, tables, z.int(), z, z.int(), z.float(), out)
+
+
+@pytest.mark.parametrize("name,n_sample", [("128d5l", 64), ("large", 48)])
+def test_fused_target_side_full_size(name, n_sample):
+    """The full target sides of the 128D-5L request (40,000 candidates over eight 4M-row
+    tables) and of the large one (520,000 candidates, one 52M-row table): bit-identical to
+    the two launches, and the oracle on sampled candidates (the first and last included)."""
+    from oracle.pipeline import _select_candidates, aggregate_bags
+    from transformer_candidate_scoring_b200.pipeline import DeviceBags
+    w = datagen.WORKLOADS[name]
+    dims = w.dims
+    F, D = dims.n_target_fields, dims.D
+    P = datagen.workload_params(w)
+    m = tr().Model(dims, P)
+    tables = []
+    for t, rows in enumerate(w.target_rows):   # the workload's target tables (the ids the oracle reads)
+        x = torch.empty(rows, D, dtype=torch.bfloat16, device="cuda")
+        datagen.fill_table_device(x, w.seed, datagen.target_table_id(w, t))
+        tables.append(x)
+    req = datagen.make_requests(w)[0]
+    bags = DeviceBags.of(req.target, "cuda")
+    n = req.n_cand
+    args = [bags.bag_table, bags.offsets, bags.keys, bags.weights]
+    fused = torch.empty(n, D, dtype=torch.float32, device="cuda")
+    tr().compress_target_bags(m, tables, *args, fused)
+    X = torch.empty(n * F, D, dtype=torch.bfloat16, device="cuda")
+    tr().aggregate(tables, *args, X)
+    two = torch.empty_like(fused)
+    tr().compress_targets(m, X.view(n, F * D), two)
+    torch.cuda.synchronize()
+    assert tr().sync_status() == 0
+    assert torch.equal(fused, two)
+    rng = np.random.default_rng(1)
+    cand = np.unique(np.concatenate([rng.choice(n, size=n_sample, replace=False), [0, n - 1]]))
+    ref = oracle.compress_targets(P, aggregate_bags(w, _select_candidates(req, cand, F), "target").reshape(-1, F * D))
+    check_close(fused[torch.from_numpy(cand).cuda()].double().cpu().numpy(), ref, "bf16", "tokens",
+                kind="intermediate")
+    del tables, X, fused, two
+    torch.cuda.empty_cache()
