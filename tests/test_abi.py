@@ -85,3 +85,13 @@ def test_uncompressed_host_validation_without_gpu(lib):
     # a null model handle is refused before anything else
     assert lib.tr_score_candidates_uncompressed(None, None, 0, 8, None, None, None, None, 1, None,
                                                 None) == L.TR_ERR_INVALID_ARG
+
+
+def test_fused_target_side_host_validation_without_gpu(lib):
+    from transformer_candidate_scoring_b200 import _lib as L
+    t = (L.Table * 1)(L.Table(16, 10, 1))
+    # a null model is refused before any device call; the model check comes first
+    assert lib.tr_compress_target_bags(None, t, 1, None, None, None, None, 5, None, None) == L.TR_ERR_INVALID_ARG
+    assert b"model is null" in lib.tr_last_error()
+    assert lib.tr_compress_target_bags(None, None, 0, None, None, None, None, 0, None, None) == L.TR_ERR_INVALID_ARG
+    assert "tr_compress_target_bags" in declared_functions()
