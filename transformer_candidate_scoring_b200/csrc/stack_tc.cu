@@ -532,8 +532,9 @@ struct Epi {
     __syncwarp();
     if (paired && slot == 0 && (m & 31) == 0) mbar_arrive(gate);
   }
+  // (the wait suspends between polls, leaving the issue slots to the other slot's warps)
   __device__ __forceinline__ bool wait() {
-    ok = __all_sync(0xffffffffu, ok && mbar_wait(m2e, ph, abort_flag));
+    ok = __all_sync(0xffffffffu, ok && mbar_wait_idle(m2e, ph, abort_flag));
     ph ^= 1;
     tc_fence_after();
     return ok;
