@@ -497,8 +497,9 @@ def run_ours(args, rank, world, local_rank):
     ov = Overlapped([dw, dw2])
     overlapped_elapsed = replay_time(ov, "overlapped")
     # ---- the timed value: the K steps as one stream of candidate tiles (Streamed: every
-    # compress launch two rounds of tiles, every score launch one round of two-tile units,
-    # across request boundaries, over a ring of activation slots), one CUDA graph
+    # compress launch four rounds of tiles, every score launch two rounds of two-tile units
+    # at 40,000 candidates a request, across request boundaries, over a ring of activation
+    # slots), one CUDA graph
     st = Streamed(dw)
     graph_elapsed = replay_time(st, "streamed")
     launches = st.launches_per_step * args.steps
@@ -653,8 +654,9 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_gbs_copies_only": h2d / (copy_ms / 1e3) / 1e9},
         "gpu_launches": int(launches),
         "launch": {"graphs": bool(use_graphs), "e2e_graphs": bool(use_graphs),
-                   "overlap": ("one stream of candidate tiles across requests: compress launches of two rounds "
-                               "of tiles, score launches of one round of two-tile units (pipeline.Streamed)"),
+                   "overlap": ("one stream of candidate tiles across requests: compress launches of whole rounds "
+                               "of tiles, score launches of whole rounds of two-tile units, as many as two "
+                               "requests fill (pipeline.Streamed)"),
                    "ring_slots": len(st.slots),
                    "graph_ms_per_step": graph_elapsed / args.steps * 1e3,
                    "overlapped_graph_ms_per_step": overlapped_elapsed / args.steps * 1e3,

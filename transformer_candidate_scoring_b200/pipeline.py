@@ -502,9 +502,10 @@ class Streamed:
     Overlapped cuts every batch at the score kernel's last partial round and runs the tail
     beside the next batch.  Here the compressor and the score kernel instead take
     fixed-size chunks of one stream of candidates that runs across batch boundaries
-    (stream_plan): by default every compress launch is two rounds of 128-candidate tiles
-    on the SMs left beside one prefill CTA, every score launch one round of the score
-    kernel's two-tile units on all SMs (or as many whole rounds as one batch fills),
+    (stream_plan): by default every compress launch is a whole number of rounds (two
+    128-candidate tiles per SM on the SMs left beside one prefill CTA) and every score
+    launch a whole number of rounds of the score kernel's two-tile units on all SMs, as many
+    as the batches between two launch points fill,
     whichever batches the chunk falls in.  A launch that spans two batches scores
     each candidate against its own request's cache (the kernels take a list of requests).
       main stream  target aggregation of batch i, then every compress and score chunk that
@@ -544,11 +545,15 @@ class Streamed:
             self.slots.append(c)
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
         self.bounds = unit_bounds(dw.req_offsets)
-        # as many whole rounds per launch as one batch fills (a launch has a fixed cost, so a
-        # large batch takes a few large launches rather than many one-round ones)
+        # as many whole rounds per launch as the ``group`` batches between two launch points
+        # fill (a launch has a fixed cost, ~7 us of ramp for the score kernel, so the stream
+        # takes a few large launches rather than many one-round ones: at 40,000 candidates a
+        # batch, group 2, four rounds of compressor tiles and two of score units)
         comp_round = 2 * (sms - 1) * SCORE_TILE
-        self.comp_chunk = comp_chunk if comp_chunk is not None else comp_round * max(1, n // comp_round)
-        self.score_units = score_units if score_units is not None else sms * max(1, len(self.bounds) // sms)
+        self.comp_chunk = (comp_chunk if comp_chunk is not None
+                           else comp_round * max(1, group * n // comp_round))
+        self.score_units = (score_units if score_units is not None
+                            else sms * max(1, group * len(self.bounds) // sms))
         self.group = group
         _, hi = torch.cuda.Stream.priority_range()
         self.user = torch.cuda.Stream(dev, priority=hi)
