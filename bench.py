@@ -496,10 +496,10 @@ def run_ours(args, rank, world, local_rank):
                          tables=(dw.user_tables, dw.target_tables))
     ov = Overlapped([dw, dw2])
     overlapped_elapsed = replay_time(ov, "overlapped")
-    # ---- the timed value: the K steps as one stream of candidate tiles (Streamed: every
-    # compress launch four rounds of tiles, every score launch two rounds of two-tile units
-    # at 40,000 candidates a request, across request boundaries, over a ring of activation
-    # slots), one CUDA graph
+    # ---- the timed value: the K steps as one stream of candidate tiles (Streamed: after
+    # every fourth request's gather, one compress launch of eight rounds of tiles and one score
+    # launch of four rounds of two-tile units at 40,000 candidates a request, across request
+    # boundaries, over a ring of activation slots), one CUDA graph
     st = Streamed(dw)
     graph_elapsed = replay_time(st, "streamed")
     launches = st.launches_per_step * args.steps
@@ -655,7 +655,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": int(launches),
         "launch": {"graphs": bool(use_graphs), "e2e_graphs": bool(use_graphs),
                    "overlap": ("one stream of candidate tiles across requests: compress launches of whole rounds "
-                               "of tiles, score launches of whole rounds of two-tile units, as many as two "
+                               "of tiles, score launches of whole rounds of two-tile units, as many as four "
                                "requests fill (pipeline.Streamed)"),
                    "ring_slots": len(st.slots),
                    "graph_ms_per_step": graph_elapsed / args.steps * 1e3,

@@ -521,7 +521,7 @@ class Streamed:
     """
 
     def __init__(self, dw: DeviceWorkload, n_slots: int = None, comp_chunk: int = None, score_units: int = None,
-                 ring_bytes: int = 8 << 30, group: int = 2):
+                 ring_bytes: int = 8 << 30, group: int = 4):
         n = dw.n_cand
         dims = dw.w.dims
         F, D = dims.n_target_fields, dims.D
@@ -548,7 +548,8 @@ class Streamed:
         # as many whole rounds per launch as the ``group`` batches between two launch points
         # fill (a launch has a fixed cost, ~7 us of ramp for the score kernel, so the stream
         # takes a few large launches rather than many one-round ones: at 40,000 candidates a
-        # batch, group 2, four rounds of compressor tiles and two of score units)
+        # batch and group 4, eight rounds of compressor tiles and four of score units; a
+        # batch's scores then complete up to four batches after its gather)
         comp_round = 2 * (sms - 1) * SCORE_TILE
         self.comp_chunk = (comp_chunk if comp_chunk is not None
                            else comp_round * max(1, group * n // comp_round))
