@@ -548,23 +548,27 @@ def run_ours(args, rank, world, local_rank):
         ht = DeviceBags(*(x.cpu().pin_memory() for x in (tb.offsets, tb.keys, tb.weights, tb.bag_table)))
         host_batches.append((hu, ht, reqs))
     feed = HostFeed(dw, host_batches)
+    # the host-fed stream runs its launches after every second request: with the bag copies
+    # beside it, evenly spaced launches overlap them better than the resident stream's
+    # groups of four (measured: 0.382 against 0.411 ms per step)
+    st_feed = Streamed(dw, group=2)
     h2d = float(np.mean(feed.h2d_bytes))
     host_scores = [torch.empty(n_cand, dtype=torch.float32).pin_memory() for _ in range(2)]
     d2h = n_cand * 4
 
-    feed.run_overlapped(st, 0, args.warmup, host_scores, stream)
+    feed.run_overlapped(st_feed, 0, args.warmup, host_scores, stream)
     torch.cuda.synchronize()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    feed.run_overlapped(st, args.warmup, args.steps, host_scores, stream)   # eager launches
+    feed.run_overlapped(st_feed, args.warmup, args.steps, host_scores, stream)   # eager launches
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_eager_ms = max_over_ranks(e0.elapsed_time(e1) / 1e3) / args.steps * 1e3
     # the same launch mode as the timed value: one graph of the K steps, host copies inside
-    g_e2e = feed.capture_overlapped(st, args.warmup, args.steps, host_scores)
+    g_e2e = feed.capture_overlapped(st_feed, args.warmup, args.steps, host_scores)
     g_e2e.replay()
     torch.cuda.synchronize()
     barrier()
@@ -653,7 +657,8 @@ def run_ours(args, rank, world, local_rank):
                 "copies_only_ms_per_step": copy_ms,
                 "h2d_gbs_copies_only": h2d / (copy_ms / 1e3) / 1e9},
         "gpu_launches": int(launches),
-        "launch": {"graphs": bool(use_graphs), "e2e_graphs": bool(use_graphs),
+        "launch": {"graphs": bool(use_graphs), "e2e_graphs": bool(use_graphs), "group": st.group,
+                   "e2e_group": st_feed.group,
                    "overlap": ("one stream of candidate tiles across requests: compress launches of whole rounds "
                                "of tiles, score launches of whole rounds of two-tile units, as many as four "
                                "requests fill (pipeline.Streamed)"),

@@ -687,10 +687,13 @@ class HostFeed:
 
     ``batches``: list of (user bags, target bags, requests) -- each the requests' bags packed
     as pack_user_bags / pack_target_bags do, every tensor in pinned host memory; all batches
-    have the requests' L_u and candidate counts of ``dw``.
+    have the requests' L_u and candidate counts of ``dw``.  With a Streamed scheduler, whose
+    gathers come ``group`` at a time, ``n_bag_slots`` should exceed its group (the default 5
+    covers the default group of 4): otherwise a batch's bag copy waits for the gather of the
+    batch before it in the same slot and lands on the critical path.
     """
 
-    def __init__(self, dw: DeviceWorkload, batches, n_bag_slots: int = 3):
+    def __init__(self, dw: DeviceWorkload, batches, n_bag_slots: int = 5):
         if n_bag_slots < 2:
             raise ValueError("HostFeed needs at least two bag slots")
         self.dw = dw
