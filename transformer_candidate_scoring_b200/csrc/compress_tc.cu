@@ -19,6 +19,11 @@
 // starts late, on an SM another kernel still holds, finds less work (or none) instead of
 // holding the launch back.  The producer passes each claimed tile index to the MMA and
 // epilogue threads through a two-entry ring in shared memory.
+//
+// A second variant (compress_gather_kernel, tr_compress_target_bags) takes the candidates'
+// field bags instead of x: eight more warps compute each 64-column slice of x on chip (the
+// weighted averages of TransRetrieval §3.2) into a ring of their own, claim the tiles, and
+// leave W1 and W2 / W3 to the copy thread; the MMA and epilogue roles are the same code.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
