@@ -566,3 +566,21 @@ def test_host_feed_streamed_has_no_stream_races(fake_cuda, monkeypatch, n_bag_sl
     assert sum(l.startswith("copy host") for l in labels) == 9 * 8
     assert sum("-> host_scores" in l for l in labels) == 9
     assert _races(log) == []
+
+
+def test_launch_sizes_are_whole_rounds():
+    from transformer_candidate_scoring_b200.pipeline import SCORE_TILE, launch_sizes, unit_bounds
+    units = len(unit_bounds([0, 40000]))          # 313 tiles: 156 pairs and one single
+    assert units == 157
+    # the 128D-5L batch on 148 SMs: groups of four give eight compressor rounds (one tile per
+    # SM on 147 SMs each), four score rounds
+    assert launch_sizes(40000, units, 148, 4) == (8 * 147 * SCORE_TILE, 4 * 148)
+    assert launch_sizes(40000, units, 148, 2) == (4 * 147 * SCORE_TILE, 2 * 148)
+    assert launch_sizes(40000, units, 148, 1) == (2 * 147 * SCORE_TILE, 1 * 148)
+    # small batches still take one whole round
+    assert launch_sizes(300, 2, 148, 4) == (2 * 147 * SCORE_TILE, 148)
+    for n, u, sms, g in [(65536, 256, 148, 4), (520000, 2032, 148, 4), (1000, 4, 8, 3)]:
+        c, s = launch_sizes(n, u, sms, g)
+        assert c % (2 * (sms - 1) * SCORE_TILE) == 0 and c >= 2 * (sms - 1) * SCORE_TILE
+        assert s % sms == 0 and s >= sms
+        assert c <= max(g * n, 2 * (sms - 1) * SCORE_TILE) and s <= max(g * u, sms)

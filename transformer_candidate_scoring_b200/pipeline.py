@@ -433,6 +433,20 @@ def unit_bounds(req_offsets, tile: int = SCORE_TILE, unit: int = SCORE_UNIT) -> 
     return out
 
 
+def launch_sizes(n: int, units_per_batch: int, sms: int, group: int):
+    """Default launch sizes of Streamed: (candidates per compress launch, score-kernel units
+    per score launch), each as many whole rounds as the ``group`` batches between two launch
+    points fill, at least one.  The compressor's unit is two rounds, two 128-candidate tiles
+    on each SM but one (the prefill CTA's); the score kernel's is one round, one unit on
+    every SM.  A launch has a fixed
+    cost (~7 us of ramp for the score kernel), so the stream takes a few large launches
+    rather than many one-round ones: at 40,000 candidates a batch and group 4, eight rounds
+    of compressor tiles and four of score units; a batch's scores then complete up to four
+    batches after its gather."""
+    comp_round = 2 * (sms - 1) * SCORE_TILE
+    return comp_round * max(1, group * n // comp_round), sms * max(1, group * units_per_batch // sms)
+
+
 def stream_plan(n: int, count: int, first: int, n_slots: int, comp_chunk: int, bounds: List[int],
                 score_units: int, group: int = 1):
     """The launch order of Streamed.run over batches first .. first + count - 1 of n
@@ -545,16 +559,9 @@ class Streamed:
             self.slots.append(c)
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
         self.bounds = unit_bounds(dw.req_offsets)
-        # as many whole rounds per launch as the ``group`` batches between two launch points
-        # fill (a launch has a fixed cost, ~7 us of ramp for the score kernel, so the stream
-        # takes a few large launches rather than many one-round ones: at 40,000 candidates a
-        # batch and group 4, eight rounds of compressor tiles and four of score units; a
-        # batch's scores then complete up to four batches after its gather)
-        comp_round = 2 * (sms - 1) * SCORE_TILE
-        self.comp_chunk = (comp_chunk if comp_chunk is not None
-                           else comp_round * max(1, group * n // comp_round))
-        self.score_units = (score_units if score_units is not None
-                            else sms * max(1, group * len(self.bounds) // sms))
+        dc, du = launch_sizes(n, len(self.bounds), sms, group)
+        self.comp_chunk = comp_chunk if comp_chunk is not None else dc
+        self.score_units = score_units if score_units is not None else du
         self.group = group
         _, hi = torch.cuda.Stream.priority_range()
         self.user = torch.cuda.Stream(dev, priority=hi)
