@@ -489,7 +489,9 @@ def test_overlapped_steps_match_serial_steps(name, n_sms):
 
 @pytest.mark.parametrize("name,n_cand,n_slots,comp_chunk,units", [
     ("128d5l", 2000, 3, 640, 3),         # launches of 5 tiles / 3 units, across batches and ring wraps
-    ("128d5l", 40000, 4, None, None),    # the default launch sizes (two compressor rounds, one score round)
+    ("128d5l", 40000, 4, None, None),    # the default launch sizes (launches every fourth batch: eight
+                                         # compressor rounds, four score rounds) on a four-slot ring
+    ("128d5l", 40000, None, None, None), # the configuration bench.py times (a 64-slot ring)
     ("packed", 300, 2, 1000, 5),         # 16 requests of mixed L_u per batch (one request set:
                                          # the slots' caches are sized by L_u); launches span many
     ("64d3l", 2000, 3, 768, 4),
