@@ -44,6 +44,7 @@ def _both(m, dims, tables, bags, n):
     ("128d5l", 1000, "wide", 8),     # eight tiles
     ("128d5l", 130, "paper", 40),    # bags of several key chunks
     ("64d3l", 777, "wide", 8),       # one 64-column slice per field
+    ("64d3l", 200, "paper", 30),     # ... with bags of several key chunks
     ("128d5l", 1, "wide", 8),        # one candidate
 ])
 def test_fused_target_side_parity(name, n, init, max_nf):
