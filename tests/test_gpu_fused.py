@@ -133,3 +133,17 @@ def test_fused_target_side_full_size(name, n_sample):
                 kind="intermediate")
     del tables, X, fused, two
     torch.cuda.empty_cache()
+
+
+def test_fused_target_side_empty_call():
+    """n = 0 launches nothing and leaves the output alone."""
+    dims = dims_of("128d5l")
+    m = tr().Model(dims, datagen.make_params(dims, 4, "paper"))
+    tables = _tables(11, 1, 100, dims.D, "bf16")
+    z = torch.zeros(1, dtype=torch.int64, device="cuda")
+    out = torch.full((1, dims.D), 7.0, dtype=torch.float32, device="cuda")
+    before = tr().api.kernel_launches()
+    tr().compress_target_bags(m, tables, z.int(), z, z.int(), z.float(), out[:0])
+    torch.cuda.synchronize()
+    assert tr().api.kernel_launches() == before
+    assert torch.all(out == 7.0)
